@@ -1,0 +1,230 @@
+"""ctypes front end of the float64 CPU oracle (test infrastructure only).
+
+Only the tests, `__graft_entry__.smoke()` and the CPU-baseline leg of
+`bench.py` may import this package. It never imports the CUDA package and the
+CUDA package never imports it; both take their inputs from the seeded scene
+generator.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+
+class OrCamera(ctypes.Structure):
+    _fields_ = [
+        ("width", ctypes.c_int32), ("height", ctypes.c_int32),
+        ("fx", ctypes.c_double), ("fy", ctypes.c_double),
+        ("cx", ctypes.c_double), ("cy", ctypes.c_double),
+        ("R", ctypes.c_double * 9), ("t", ctypes.c_double * 3),
+        ("campos", ctypes.c_double * 3), ("bg", ctypes.c_double * 3),
+        ("near_z", ctypes.c_double),
+    ]
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = ctypes.CDLL(path)
+        P = ctypes.c_void_p
+        L.or_create.restype = P
+        L.or_destroy.argtypes = [P]
+        L.or_set_scene.argtypes = [P, ctypes.c_int64, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
+                                   P, P, P, P, P, ctypes.POINTER(OrCamera)]
+        L.or_set_scene.restype = ctypes.c_int
+        L.or_set_scene_f64.argtypes = L.or_set_scene.argtypes
+        L.or_set_scene_f64.restype = ctypes.c_int
+        L.or_get_preprocess.argtypes = [P] * 9
+        L.or_num_entries.argtypes = [P]
+        L.or_num_entries.restype = ctypes.c_int64
+        L.or_get_sorted.argtypes = [P] * 4
+        L.or_render.argtypes = [P] * 6
+        L.or_render_pixels.argtypes = [P, ctypes.c_int64] + [P] * 6
+        L.or_backward.argtypes = [P] * 8
+        L.or_loss.argtypes = [ctypes.c_int32, ctypes.c_int32, P, P, ctypes.c_double, P, P]
+        L.or_loss.restype = ctypes.c_int
+        L.or_loss_f64.argtypes = [ctypes.c_int32, ctypes.c_int32, P, P, ctypes.c_double, P, P]
+        L.or_loss_f64.restype = ctypes.c_int
+        L.or_adam.argtypes = [ctypes.c_int64, P, P, P, P, ctypes.c_double, ctypes.c_double,
+                              ctypes.c_double, ctypes.c_double, ctypes.c_int32]
+        L.or_blend_screen.argtypes = [ctypes.c_int32, P, ctypes.c_int32, P, ctypes.c_double,
+                                      ctypes.c_double, P, P, P, P, P]
+        L.or_sh_basis.argtypes = [ctypes.c_int32, ctypes.c_int64, P, P]
+        L.or_rotation_cov.argtypes = [P, P, P, P]
+        _lib = L
+    return _lib
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def camera(cam) -> OrCamera:
+    c = OrCamera()
+    c.width, c.height = int(cam.width), int(cam.height)
+    c.fx, c.fy, c.cx, c.cy = (float(np.float32(v)) for v in (cam.fx, cam.fy, cam.cx, cam.cy))
+    for i, v in enumerate(np.asarray(cam.R, np.float32).reshape(-1)):
+        c.R[i] = float(v)
+    for name in ("t", "campos", "bg"):
+        arr = getattr(c, name)
+        for i, v in enumerate(np.asarray(getattr(cam, name), np.float32).reshape(-1)):
+            arr[i] = float(v)
+    c.near_z = float(np.float32(cam.near_z))
+    return c
+
+
+class Oracle:
+    """One scene seen by one camera: preprocess and tile lists are built on
+    construction; render/backward walk the lists per pixel."""
+
+    def __init__(self, scene, cam, active_degree=None):
+        self.L = lib()
+        self.scene = scene
+        self.cam = cam
+        self.h = self.L.or_create()
+        self.active_degree = scene.sh_degree if active_degree is None else active_degree
+        f64 = np.asarray(scene.means).dtype == np.float64
+        dt = np.float64 if f64 else np.float32
+        arrs = [np.ascontiguousarray(a, dtype=dt) for a in
+                (scene.means, scene.log_scales, scene.quats, scene.opacity_logits, scene.sh)]
+        self._keep = arrs
+        self._cam = camera(cam)
+        fn = self.L.or_set_scene_f64 if f64 else self.L.or_set_scene
+        rc = fn(self.h, scene.n, scene.n_pad, scene.sh_degree, self.active_degree,
+                *[_p(a) for a in arrs], ctypes.byref(self._cam))
+        if rc != 0:
+            raise ValueError("oracle rejected the scene")
+
+    def __del__(self):
+        h = getattr(self, "h", None)
+        if h:
+            self.L.or_destroy(h)
+            self.h = None
+
+    @property
+    def tiles(self):
+        return ((self.cam.width + 15) // 16, (self.cam.height + 15) // 16)
+
+    def preprocess(self) -> dict:
+        n = self.scene.n
+        out = dict(screen=np.zeros((n, 9)), cov2d=np.zeros((n, 3)), depth=np.zeros(n),
+                   depth_key=np.zeros(n, np.float32), radius=np.zeros(n),
+                   rect=np.zeros((n, 4), np.int32), touched=np.zeros(n, np.int32),
+                   clamped=np.zeros((n, 3), np.uint8))
+        self.L.or_get_preprocess(self.h, *[_p(out[k]) for k in
+                                           ("screen", "cov2d", "depth", "depth_key", "radius",
+                                            "rect", "touched", "clamped")])
+        return out
+
+    def sorted(self) -> dict:
+        k = self.L.or_num_entries(self.h)
+        tx, ty = self.tiles
+        ids = np.zeros(k, np.int32)
+        tiles = np.zeros(k, np.int32)
+        ranges = np.zeros((tx * ty, 2), np.int64)
+        self.L.or_get_sorted(self.h, _p(ids), _p(tiles), _p(ranges))
+        return dict(ids=ids, tiles=tiles, ranges=ranges)
+
+    def render(self) -> dict:
+        H, W = self.cam.height, self.cam.width
+        out = dict(image=np.zeros((3, H, W)), final_T=np.zeros((H, W)),
+                   n_contrib=np.zeros((H, W), np.int32), ambiguous=np.zeros((H, W), np.uint8),
+                   stats=np.zeros(2, np.int64))
+        self.L.or_render(self.h, *[_p(out[k]) for k in
+                                   ("image", "final_T", "n_contrib", "ambiguous", "stats")])
+        return out
+
+    def render_pixels(self, px, py) -> dict:
+        px = np.ascontiguousarray(px, np.int32)
+        py = np.ascontiguousarray(py, np.int32)
+        n = px.size
+        out = dict(rgb=np.zeros((n, 3)), T=np.zeros(n), n_contrib=np.zeros(n, np.int32),
+                   ambiguous=np.zeros(n, np.uint8))
+        self.L.or_render_pixels(self.h, n, _p(px), _p(py), _p(out["rgb"]), _p(out["T"]),
+                                _p(out["n_contrib"]), _p(out["ambiguous"]))
+        return out
+
+    def backward(self, dimage) -> dict:
+        s = self.scene
+        dimage = np.ascontiguousarray(dimage, np.float64)
+        K = s.sh_k
+        out = dict(screen=np.zeros((s.n, 9)), means=np.zeros((3, s.n_pad)),
+                   log_scales=np.zeros((3, s.n_pad)), quats=np.zeros((4, s.n_pad)),
+                   opacity_logits=np.zeros(s.n_pad), sh=np.zeros((3, K, s.n_pad)))
+        self.L.or_backward(self.h, _p(dimage), *[_p(out[k]) for k in
+                                                  ("screen", "means", "log_scales", "quats",
+                                                   "opacity_logits", "sh")])
+        return out
+
+
+def loss(image, target, lam=0.2, with_grad=True):
+    """(1 - lam) L1 + lam (1 - SSIM). Returns (loss, l1, ssim, dL/dimage or None).
+    float32 inputs are read as float32 (as the CUDA path receives them); float64
+    inputs keep full precision."""
+    f64 = np.asarray(image).dtype == np.float64
+    dt = np.float64 if f64 else np.float32
+    image = np.ascontiguousarray(image, dt)
+    target = np.ascontiguousarray(target, dt)
+    _, H, W = image.shape
+    out3 = np.zeros(3)
+    d = np.zeros((3, H, W)) if with_grad else None
+    fn = lib().or_loss_f64 if f64 else lib().or_loss
+    rc = fn(H, W, _p(image), _p(target), float(lam), _p(out3), _p(d))
+    if rc != 0:
+        raise ValueError("oracle rejected the loss inputs")
+    return out3[0], out3[1], out3[2], d
+
+
+def adam(p, g, m, v, lr, step, beta1=0.9, beta2=0.999, eps=1e-8):
+    """One Adam step in float64 on copies; returns (p, g, m, v)."""
+    p, g, m, v = (np.array(a, dtype=np.float64, copy=True).reshape(-1) for a in (p, g, m, v))
+    lib().or_adam(p.size, _p(p), _p(g), _p(m), _p(v), lr, beta1, beta2, eps, int(step))
+    return p, g, m, v
+
+
+def blend_screen(screen, order, px, py, bg=(0.0, 0.0, 0.0), dldI=None):
+    """Blend one pixel over explicit screen-space Gaussians (n x 9) in `order`."""
+    screen = np.ascontiguousarray(screen, np.float64)
+    order = np.ascontiguousarray(order, np.int32)
+    bg = np.ascontiguousarray(bg, np.float64)
+    rgb = np.zeros(3)
+    T = np.zeros(1)
+    n = screen.shape[0]
+    sgrad = np.zeros((n, 9)) if dldI is not None else None
+    dl = None if dldI is None else np.ascontiguousarray(dldI, np.float64)
+    lib().or_blend_screen(n, _p(screen), order.size, _p(order), float(px), float(py), _p(bg),
+                          _p(dl), _p(rgb), _p(T), _p(sgrad))
+    return rgb, T[0], sgrad
+
+
+def sh_basis(degree, dirs):
+    dirs = np.ascontiguousarray(dirs, np.float64).reshape(-1, 3)
+    out = np.zeros((dirs.shape[0], 16))
+    lib().or_sh_basis(degree, dirs.shape[0], _p(dirs), _p(out))
+    return out
+
+
+def rotation_cov(q, ls):
+    q = np.ascontiguousarray(q, np.float64)
+    ls = np.ascontiguousarray(ls, np.float64)
+    R = np.zeros(9)
+    S = np.zeros(9)
+    lib().or_rotation_cov(_p(q), _p(ls), _p(R), _p(S))
+    return R.reshape(3, 3), S.reshape(3, 3)
+
+
+def full_loss(scene, cam, target, lam=0.2):
+    """Scalar training loss of `scene` seen by `cam` against `target` (render + loss)."""
+    o = Oracle(scene, cam)
+    r = o.render()
+    L, _, _, _ = loss(r["image"], np.asarray(target, np.float64), lam, with_grad=False)
+    return L
+
+
+__all__ = ["Oracle", "loss", "adam", "blend_screen", "sh_basis", "rotation_cov", "camera", "lib"]
