@@ -1,0 +1,553 @@
+#!/usr/bin/env python
+"""Training-step throughput of the B200 Gaussian-splat rasteriser.
+
+One step = one iteration of the hot path on one camera: preprocess -> tile
+sort + forward blend -> L1 + D-SSIM loss -> blend + projection backward ->
+Adam on every parameter group, all through the C ABI (include/gs_api.h).
+
+Default workload: the Dense scene (3,000,000 Gaussians from 64 clusters, SH
+degree 3, 32 ring cameras at 1920x1080, targets = renders of a perturbed copy
+made before timing), cameras drawn from a seeded permutation.
+
+Prints ONE JSON line on rank 0. `--impl reference` times the float64 CPU
+oracle on a bounded sample of the same workload instead.
+Multi-GPU (torchrun): replicas only - each rank trains its own copy, no
+collective on the data path; value = all ranks' iterations / max rank time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "train iters/s (fwd+loss+bwd+Adam), 3M Gaussians @1080p; Mpix/s; % roofline"
+UNIT = "iters/s"
+PKG_CSRC = os.path.join(ROOT, "gaussian_splatting_differentiable_rasteriser_b200", "csrc")
+
+WORKLOADS = {
+    "dense": "dense: 3,000,000 Gaussians (64 clusters, sigma 0.3), SH degree 3, 32 ring cameras "
+             "(r = 10) at 1920x1080, f = 1600, targets = renders of a N(0, 0.05^2)-perturbed copy, "
+             "seed 0",
+    "mid": "mid: 500,000 Gaussians in [-5,5]^3, SH degree 3, 16 ring cameras (r = 15) at 1280x720, "
+           "f = 1100, targets = renders of a perturbed copy, seed 0",
+    "heavy_tail": "heavy_tail: 6,000,000 Gaussians in 40x10x40, mixture log-scales, SH degree 3, "
+                  "32 ring cameras (r = 35) at 1920x1080, targets = renders of a perturbed copy, seed 0",
+    "small": "small: 10,000 Gaussians on a unit shell, SH degree 3, one 256x256 camera, "
+             "target = renders of a perturbed copy, seed 0",
+}
+
+# ncu DRAM traffic (read + write bytes per launch) of kernels on the dense workload,
+# with the sha256 (first 12 hex digits) of the source file each figure was taken from.
+# A figure whose source has changed since is reported as null.
+NCU_TRAFFIC = {}
+
+
+def sha12(path):
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:12]
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p.get("sm_max_mhz", 1965.0)), "measured"
+    except Exception:
+        return 6650.0, 1965.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        out = {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        if self.proc is None:
+            return out
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return out
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({names[k] for r in rows for k in range(4) if r[5 + k].lower() == "active"})
+        out.update(sm_mhz=statistics.median(sm) if sm else None, sm_max_mhz=max(mx) if mx else None,
+                   reasons=reasons, samples=len(rows))
+        return out
+
+
+def dist_setup():
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ workload
+def build_workload(config, device):
+    import numpy as np
+    import torch
+
+    from gaussian_splatting_differentiable_rasteriser_b200 import model, native, scenes
+
+    scene = scenes.CONFIGS[config]()
+    pert = scenes.perturbed(scene, 0.05, seed=1)
+    cams = scene.cameras
+    W = max(c.width for c in cams)
+    H = max(c.height for c in cams)
+    m = model.GaussianModel(pert, device=device)
+    cap = max(1 << 20, 8 * scene.n)
+    step = model.TrainStep(m, cap, W, H, device=device)
+    # targets: renders of the perturbed copy (forward only, before any timing)
+    targets = torch.empty((len(cams), 3, H, W), dtype=torch.float32, device=device)
+    kmax = 0
+    for i, cam in enumerate(cams):
+        img, _, _ = step.forward(native.camera_struct(cam), cam.height, cam.width)
+        targets[i].copy_(img)
+        kmax = max(kmax, step.last_entries)
+    torch.cuda.synchronize()
+    m.load(scene)
+    return scene, m, step, targets, kmax
+
+
+def run_steps(step, cams, targets, sched, start, count):
+    for i in range(start, start + count):
+        c = int(sched[i % len(sched)])
+        step(cams[c], targets[c])
+
+
+def time_device(step, cams, targets, sched, start, count, world):
+    import torch
+    barrier(world)
+    torch.cuda.synchronize()
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    ev0.record()
+    run_steps(step, cams, targets, sched, start, count)
+    ev1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    return ev0.elapsed_time(ev1)
+
+
+def profile_stages(step, cams, targets, sched, start, count):
+    """Per-stage kernel times (library events) plus Adam (torch events: the
+    Adam launches are the only work between them on the current stream)."""
+    import torch
+
+    from gaussian_splatting_differentiable_rasteriser_b200 import native
+    from gaussian_splatting_differentiable_rasteriser_b200.scenes import GROUP_NAMES
+
+    ctx = step.ctx
+    ctx.profile_enable(True)
+    ctx.profile_read()
+    adam_ms = 0.0
+    adam_launches = 0
+    m = step.model
+    ks = []
+    for i in range(start, start + count):
+        c = int(sched[i % len(sched)])
+        cam = cams[c]
+        cs = native.camera_struct(cam)
+        img, T, nc = step.forward(cs, cam.height, cam.width)
+        ks.append(step.last_entries)
+        ctx.loss_l1_dssim(img, targets[c], step.lam, step.loss, step.dimage)
+        ctx.render_backward(m.params_struct(), cs, T, nc, step.dimage, m.grads_struct())
+        m.step_count += 1
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for k in GROUP_NAMES:
+            native.adam_step(m.params[k], m.grads[k], m.m[k], m.v[k], step.lrs[k], m.step_count,
+                             step.betas[0], step.betas[1], step.eps)
+        e1.record()
+        torch.cuda.synchronize()
+        adam_ms += e0.elapsed_time(e1)
+        adam_launches += len(GROUP_NAMES)
+    prof = ctx.profile_read()
+    ctx.profile_enable(False)
+    prof["adam"] = {"ms": adam_ms, "launches": adam_launches, "work": count * m.flat.numel()}
+    return prof, ks
+
+
+def stage_models(scene, sh_k):
+    """Algorithmic bytes (HBM stages) or FP32-pipe instructions (blend stages) per unit of work."""
+    n_par = 11 + 3 * sh_k
+    return {
+        # params in (all groups) + 48 B screen + depth + rect + touched + clamp out, per Gaussian
+        "preprocess": ("hbm", 4 * n_par + 48 + 4 + 8 + 4 + 1),
+        # per entry and pass: key + value read and written
+        "sort": ("hbm", 24),
+        # keys + values written per entry
+        "duplicate": ("hbm", 12),
+        "ranges": ("hbm", 8),
+        # x, y read, dL/dx written, per pixel (3 channels)
+        "loss": ("hbm", 36),
+        # params + grads read, grads written, raw sums + screen record read, per Gaussian
+        "preprocess_backward": ("hbm", 4 * n_par * 3 + 48 + 48 + 5),
+        # p, g, m, v read; p, m, v, g = 0 written, per scalar
+        "adam": ("hbm", 32),
+        # per evaluated (pixel, Gaussian) pair: 2 subtractions + 5 for the quadratic form
+        "blend_forward": ("alu", 7),
+        # per pair up to the last contributor: the same 7 to recompute alpha
+        "blend_backward": ("alu", 7),
+    }
+
+
+def roofline(prof, scene, hbm_gbs, sm_mhz):
+    models = stage_models(scene, scene.sh_k)
+    per = {}
+    for name, d in prof.items():
+        if d["launches"] == 0 or name not in models:
+            continue
+        kind, per_unit = models[name]
+        t = d["ms"] / d["launches"] * 1e-3
+        units = d["work"] / d["launches"]
+        if kind == "hbm":
+            achieved = units * per_unit / t / 1e9
+            per[name] = {"bound": "hbm", "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s",
+                         "frac": achieved / hbm_gbs, "ms_per_launch": t * 1e3}
+        else:
+            # FP32 lanes: 148 SMs x 128 lanes x clock (one instruction per lane per cycle)
+            peak = 148 * 128 * sm_mhz * 1e6 / 1e12
+            achieved = units * per_unit / t / 1e12
+            per[name] = {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "Tinst/s",
+                         "frac": achieved / peak, "ms_per_launch": t * 1e3}
+    return per
+
+
+# ------------------------------------------------------------- oracle (CPU)
+def oracle_sample_step(scene, cam, target, rows=8, adam_frac=1 / 64):
+    """One training step of the float64 oracle on a bounded sample of the workload:
+    the full preprocess + tile sort of every Gaussian, then render, loss and
+    backward restricted to a band of `rows` pixel rows (scaled by height/rows),
+    and Adam on a 1/64 slice of the parameters (scaled by 64). Returns the
+    estimated seconds of one full step and the measured seconds spent."""
+    import numpy as np
+
+    import oracle
+
+    H, W = cam.height, cam.width
+    y0 = (H - rows) // 2
+    t0 = time.perf_counter()
+    o = oracle.Oracle(scene, cam)
+    t1 = time.perf_counter()
+    r = o.render_rows(y0, y0 + rows)
+    band = r["image"][:, y0:y0 + rows, :]
+    _, _, _, d = oracle.loss(band, np.asarray(target[:, y0:y0 + rows, :], np.float64), 0.2)
+    dfull = np.zeros((3, H, W))
+    dfull[:, y0:y0 + rows, :] = d
+    o.backward(dfull, rows=(y0, y0 + rows))
+    t2 = time.perf_counter()
+    total = scene.means.size + scene.log_scales.size + scene.quats.size + scene.opacity_logits.size + \
+        scene.sh.size
+    cnt = max(1, int(total * adam_frac))
+    rng = np.random.default_rng(0)
+    p = rng.normal(size=cnt)
+    g = rng.normal(size=cnt) * 1e-3
+    oracle.adam(p, g, np.zeros(cnt), np.zeros(cnt), 1e-3, 1)
+    t3 = time.perf_counter()
+    est = (t1 - t0) + (t2 - t1) * H / rows + (t3 - t2) / adam_frac
+    return est, t3 - t0
+
+
+def cpu_baseline(scene, cams, targets_host, sched, steps):
+    est, spent = [], 0.0
+    for i in range(steps):
+        c = int(sched[i % len(sched)])
+        e, s = oracle_sample_step(scene, cams[c], targets_host[c])
+        est.append(e)
+        spent += s
+    value = len(est) / sum(est)
+    return {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{len(est)} step(s): full float64 preprocess + tile sort of all Gaussians, "
+                      "render + loss + backward on an 8-row band scaled by height/8, Adam on a "
+                      "1/64 parameter slice scaled by 64; single-threaded",
+            "seconds_spent": spent}
+
+
+# ------------------------------------------------------------------- arms
+def main_ours(args):
+    import numpy as np
+    import torch
+
+    import __graft_entry__
+
+    world, rank, local = dist_setup()
+    if rank == 0:
+        __graft_entry__.build()
+    barrier(world)
+    from gaussian_splatting_differentiable_rasteriser_b200 import native, scenes
+    from gaussian_splatting_differentiable_rasteriser_b200.scenes import GROUP_NAMES
+
+    native.load()
+    device = f"cuda:{local}"
+    scene, m, step, targets, kmax = build_workload(args.config, device)
+    cams = scene.cameras
+    sched = scenes.camera_schedule(len(cams), args.warmup + args.steps, seed=rank)
+    # warm-up (also compiles nothing: the library is ahead-of-time built)
+    run_steps(step, cams, targets, sched, 0, args.warmup)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    ms = time_device(step, cams, targets, sched, args.warmup, args.steps, world)
+    clk = clocks.stop()
+    ms = max_over_ranks(ms, world)
+    ms_per_step = ms / args.steps
+    value = world * args.steps / (ms / 1e3)
+    H, W = cams[0].height, cams[0].width
+
+    # per-stage kernel times for the roofline (separate, profiled pass over the same steps)
+    prof, ks = profile_stages(step, cams, targets, sched, args.warmup, args.steps)
+    hbm_gbs, sm_max, peak_kind = peaks()
+    per = roofline(prof, scene, hbm_gbs, clk["sm_mhz"] or sm_max)
+    dominant = max((k for k in prof if prof[k]["launches"]), key=lambda k: prof[k]["ms"])
+    rf = dict(per.get(dominant, {}))
+    rf.pop("ms_per_launch", None)
+    rf["kernel"] = dominant
+    rf["peak_source"] = peak_kind
+    src = {"blend_forward": "blend.cu", "blend_backward": "blend.cu", "adam": "adam.cu",
+           "preprocess": "preprocess.cu", "sort": "sort.cu", "loss": "loss.cu",
+           "preprocess_backward": "preprocess_backward.cu"}.get(dominant)
+    tr = NCU_TRAFFIC.get(dominant)
+    rf["traffic"] = tr[0] if (tr and src and sha12(os.path.join(PKG_CSRC, src)) == tr[1]) else None
+
+    # launches of our kernels per step (sort = histogram + offsets + one per pass)
+    steps_p = max(1, args.steps)
+    sort_w = prof["sort"]["work"]
+    passes = (sort_w / max(1, sum(ks))) if sort_w else 0
+    per_step = (sum(prof[k]["launches"] for k in prof if k not in ("sort", "adam")) / steps_p +
+                (prof["sort"]["launches"] / steps_p) * (2 + passes) + len(GROUP_NAMES))
+    gpu_launches = int(round(per_step * args.steps))
+
+    # end to end: target streamed from pinned host memory each step, loss read back
+    e2e = None
+    if not args.no_e2e:
+        e2e = e2e_run(step, cams, targets, sched, args, world)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(scene, cams, targets.cpu().numpy(), sched, 1)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": WORKLOADS[args.config], "gaussians": scene.n,
+                       "width": W, "height": H, "cameras": len(cams),
+                       "parallelism": "replicas" if world > 1 else "single-gpu",
+                       "l2": "inputs larger than L2: 2.8 GB of parameter/gradient/moment state "
+                             "streamed every step" if args.config == "dense" else "see workload",
+                       "entries_per_step": int(statistics.mean(ks)) if ks else None},
+            "mpix_per_s": value * W * H / 1e6,
+            "roofline": rf,
+            "stages": {k: {"ms_per_step": prof[k]["ms"] / steps_p,
+                           "share": prof[k]["ms"] / max(1e-9, sum(v["ms"] for v in prof.values())),
+                           **({"frac": per[k]["frac"], "bound": per[k]["bound"],
+                               "achieved": per[k]["achieved"], "unit": per[k]["unit"]}
+                              if k in per else {})}
+                       for k in prof if prof[k]["launches"]},
+            "e2e": e2e, "gpu_launches": gpu_launches, "clocks": clk, "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def e2e_run(step, cams, targets, sched, args, world):
+    """Same steps through the public API with the target of every step copied
+    from pinned host memory (double-buffered on a copy stream, overlapped with the
+    previous step's work) and each step's loss read back to the host."""
+    import torch
+
+    from gaussian_splatting_differentiable_rasteriser_b200 import native
+    from gaussian_splatting_differentiable_rasteriser_b200.scenes import GROUP_NAMES
+
+    host_t = targets.cpu().pin_memory()
+    dev_t = [torch.empty_like(targets[0]) for _ in range(2)]
+    copy_stream = torch.cuda.Stream()
+    copied = [torch.cuda.Event() for _ in range(2)]
+    loss_host = torch.empty((2, 3), dtype=torch.float64).pin_memory()
+    m = step.model
+    n = args.steps
+    start = args.warmup
+    losses = []
+    barrier(world)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    c0 = int(sched[start % len(sched)])
+    with torch.cuda.stream(copy_stream):
+        dev_t[0].copy_(host_t[c0], non_blocking=True)
+        copied[0].record(copy_stream)
+    for j in range(n):
+        i = start + j
+        c = int(sched[i % len(sched)])
+        cam = cams[c]
+        cs = native.camera_struct(cam)
+        img, T, nc = step.forward(cs, cam.height, cam.width)  # waits for all earlier work
+        if j > 0:
+            losses.append(float(loss_host[(j - 1) % 2, 0]))
+        if j + 1 < n:
+            cn = int(sched[(i + 1) % len(sched)])
+            with torch.cuda.stream(copy_stream):
+                dev_t[(j + 1) % 2].copy_(host_t[cn], non_blocking=True)
+                copied[(j + 1) % 2].record(copy_stream)
+        torch.cuda.current_stream().wait_event(copied[j % 2])
+        step.ctx.loss_l1_dssim(img, dev_t[j % 2], step.lam, step.loss, step.dimage)
+        step.ctx.render_backward(m.params_struct(), cs, T, nc, step.dimage, m.grads_struct())
+        m.step_count += 1
+        for k in GROUP_NAMES:
+            native.adam_step(m.params[k], m.grads[k], m.m[k], m.v[k], step.lrs[k], m.step_count,
+                             step.betas[0], step.betas[1], step.eps)
+        loss_host[j % 2].copy_(step.loss, non_blocking=True)
+    torch.cuda.synchronize()
+    losses.append(float(loss_host[(n - 1) % 2, 0]))
+    dt = time.perf_counter() - t0
+    dt = max_over_ranks(dt, world)
+    barrier(world)
+    assert len(losses) == n
+    H, W = cams[0].height, cams[0].width
+    return {"value": world * n / dt, "unit": UNIT, "h2d_bytes_per_step": 3 * H * W * 4,
+            "d2h_bytes_per_step": 3 * 8 + 24, "last_loss": losses[-1]}
+
+
+def main_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import numpy as np
+
+    from gaussian_splatting_differentiable_rasteriser_b200 import scenes
+    import oracle
+
+    oracle.lib()
+    scene = scenes.CONFIGS[args.config]()
+    # targets: the oracle's own band renders of the perturbed copy are what the sample needs
+    pert = scenes.perturbed(scene, 0.05, seed=1)
+    cams = scene.cameras
+    sched = scenes.camera_schedule(len(cams), args.warmup + args.steps, seed=0)
+    H, W = cams[0].height, cams[0].width
+    rows = 8
+    targets = {}
+    for c in set(int(x) for x in sched):
+        o = oracle.Oracle(pert, cams[c])
+        y0 = (H - rows) // 2
+        targets[c] = o.render_rows(y0, y0 + rows)["image"]
+        del o
+    for i in range(args.warmup):
+        c = int(sched[i])
+        oracle_sample_step(scene, cams[c], targets[c], rows)
+    est = []
+    spent = 0.0
+    for i in range(args.warmup, args.warmup + args.steps):
+        c = int(sched[i])
+        e, s = oracle_sample_step(scene, cams[c], targets[c], rows)
+        est.append(e)
+        spent += s
+    value = len(est) / sum(est)
+    cpu = {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+           "sample": f"per step: full float64 preprocess + tile sort of all {scene.n} Gaussians, "
+                     f"render + loss + backward on a {rows}-row band scaled by height/{rows}, Adam on "
+                     "a 1/64 parameter slice scaled by 64; single-threaded",
+           "seconds_spent": spent}
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 / value,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": WORKLOADS[args.config], "gaussians": scene.n, "width": W,
+                       "height": H, "cameras": len(cams), "parallelism": "cpu"},
+            "cpu_baseline": cpu,
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--config", choices=tuple(WORKLOADS), default="dense")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        main_reference(args)
+    else:
+        main_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,610 @@
+// C ABI of the rasteriser (declared in include/gs_api.h): context management,
+// host-side argument checks and the order of kernel launches per call.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "gs_api.h"
+#include "gs_kernels.cuh"
+
+namespace gs {
+int64_t loss_num_blocks(int height, int width);
+}
+
+struct gs_ctx {
+  int64_t max_g = 0, max_k = 0, max_tiles = 0, max_blocks = 0, max_sort_tiles = 0,
+          max_loss_blocks = 0;
+  int32_t max_w = 0, max_h = 0;
+  // per Gaussian
+  gs::Screen* screen = nullptr;
+  float* depth = nullptr;
+  uint2* rect = nullptr;
+  uint32_t* touched = nullptr;
+  uint8_t* clamped = nullptr;
+  float* sgrad = nullptr;
+  uint32_t* block_sums = nullptr;
+  uint64_t* block_prefix = nullptr;
+  uint32_t* depth_range = nullptr;
+  // sort
+  uint64_t* keys[2] = {nullptr, nullptr};
+  uint32_t* vals[2] = {nullptr, nullptr};
+  uint32_t* hist = nullptr;
+  uint32_t* offsets = nullptr;
+  uint32_t* status = nullptr;
+  uint32_t* counters = nullptr;
+  uint2* ranges = nullptr;
+  // loss
+  double* loss_partials = nullptr;
+  uint32_t* loss_counter = nullptr;
+  // readback record (device + pinned host); the device error word lives in it
+  gs::ForwardInfo* info_dev = nullptr;
+  gs::ForwardInfo* info_host = nullptr;
+  // state of the camera in flight
+  bool have_pre = false, have_fwd = false;
+  int64_t n = 0, n_pad = 0;
+  gs::CamArgs cam{};
+  int64_t K = 0;
+  int depth_bits = 0;
+  uint32_t depth_min = 0;
+  int sorted_buf = 0;
+  // profiling (off by default)
+  struct Profiler {
+    static constexpr int kMaxRec = 128;
+    bool on = false, created = false;
+    cudaEvent_t ev[2 * kMaxRec];
+    int stage[kMaxRec];
+    int nrec = 0;
+    double ms[GS_NUM_STAGES] = {0};
+    int64_t launches[GS_NUM_STAGES] = {0};
+    int64_t work[GS_NUM_STAGES] = {0};
+  } prof;
+  unsigned long long* pairs = nullptr;  // [2] evaluated pairs of the two blends
+  char err[512] = {0};
+};
+
+namespace {
+
+gs_status fail(gs_ctx* c, gs_status s, const char* fmt, ...) {
+  if (c) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(c->err, sizeof(c->err), fmt, ap);
+    va_end(ap);
+  }
+  return s;
+}
+
+#define GS_CUDA(ctx, call)                                                              \
+  do {                                                                                  \
+    cudaError_t e_ = (call);                                                            \
+    if (e_ != cudaSuccess)                                                              \
+      return fail((ctx), GS_ERR_CUDA, "%s failed: %s", #call, cudaGetErrorString(e_)); \
+  } while (0)
+
+void free_all(gs_ctx* c) {
+  void* bufs[] = {c->screen, c->depth, c->rect, c->touched, c->clamped, c->sgrad, c->block_sums,
+                  c->block_prefix, c->depth_range, c->keys[0], c->keys[1], c->vals[0], c->vals[1],
+                  c->hist, c->offsets, c->status, c->counters, c->ranges, c->loss_partials,
+                  c->loss_counter, c->info_dev, c->pairs};
+  for (void* b : bufs)
+    if (b) cudaFree(b);
+  if (c->info_host) cudaFreeHost(c->info_host);
+  if (c->prof.created)
+    for (auto& e : c->prof.ev) cudaEventDestroy(e);
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+gs_status make_cam(gs_ctx* c, const gs_camera* cam, gs::CamArgs& out) {
+  if (!cam) return fail(c, GS_ERR_INVALID_ARG, "camera is NULL");
+  if (cam->width <= 0 || cam->height <= 0 || cam->width > c->max_w || cam->height > c->max_h)
+    return fail(c, GS_ERR_INVALID_ARG, "camera %dx%d outside the context's 1..%dx1..%d", cam->width,
+                cam->height, c->max_w, c->max_h);
+  if (!(std::isfinite(cam->fx) && std::isfinite(cam->fy) && cam->fx > 0.f && cam->fy > 0.f))
+    return fail(c, GS_ERR_INVALID_ARG, "focal lengths must be finite and positive");
+  out.width = cam->width;
+  out.height = cam->height;
+  out.tiles_x = (cam->width + gs::kTile - 1) / gs::kTile;
+  out.tiles_y = (cam->height + gs::kTile - 1) / gs::kTile;
+  out.fx = cam->fx;
+  out.fy = cam->fy;
+  out.cx = cam->cx;
+  out.cy = cam->cy;
+  std::memcpy(out.R, cam->R, sizeof(out.R));
+  std::memcpy(out.t, cam->t, sizeof(out.t));
+  std::memcpy(out.campos, cam->campos, sizeof(out.campos));
+  std::memcpy(out.bg, cam->bg, sizeof(out.bg));
+  out.near_z = cam->near_z;
+  return GS_OK;
+}
+
+gs_status check_params(gs_ctx* c, const gs_params* p) {
+  if (!p) return fail(c, GS_ERR_INVALID_ARG, "params is NULL");
+  if (p->n < 0 || p->n > c->max_g)
+    return fail(c, GS_ERR_INVALID_ARG, "n = %lld outside 0..%lld", (long long)p->n, (long long)c->max_g);
+  if (p->n_pad < p->n || p->n_pad % 4 != 0)
+    return fail(c, GS_ERR_INVALID_ARG, "n_pad = %lld must be >= n and a multiple of 4", (long long)p->n_pad);
+  if (p->sh_degree < 0 || p->sh_degree > 3 || p->active_degree < 0 || p->active_degree > p->sh_degree)
+    return fail(c, GS_ERR_INVALID_ARG, "sh_degree %d / active_degree %d out of range", p->sh_degree,
+                p->active_degree);
+  const void* ptrs[] = {p->means, p->log_scales, p->quats, p->opacity_logits, p->sh};
+  if (p->n > 0)
+    for (const void* q : ptrs)
+      if (!q || !aligned(q, 4)) return fail(c, GS_ERR_INVALID_ARG, "a parameter pointer is NULL or misaligned");
+  return GS_OK;
+}
+
+gs_status take_device_error(gs_ctx* c) {
+  const uint32_t e = c->info_host->device_error;
+  if (e == 0) return GS_OK;
+  c->info_host->device_error = 0;
+  cudaMemset(&c->info_dev->device_error, 0, sizeof(uint32_t));
+  return fail(c, GS_ERR_DEVICE, "a kernel recorded a device fault (code 0x%x: %s)", e,
+              (e & gs::kErrLookbackTimeout) ? "sort look-back wait gave up" : "index out of range");
+}
+
+void prof_harvest(gs_ctx* c) {
+  auto& P = c->prof;
+  for (int r = 0; r < P.nrec; ++r) {
+    float ms = 0.f;
+    if (cudaEventSynchronize(P.ev[2 * r + 1]) == cudaSuccess &&
+        cudaEventElapsedTime(&ms, P.ev[2 * r], P.ev[2 * r + 1]) == cudaSuccess)
+      P.ms[P.stage[r]] += ms;
+  }
+  P.nrec = 0;
+}
+
+void prof_begin(gs_ctx* c, cudaStream_t st) {
+  auto& P = c->prof;
+  if (!P.on) return;
+  if (P.nrec == gs_ctx::Profiler::kMaxRec) prof_harvest(c);
+  cudaEventRecord(P.ev[2 * P.nrec], st);
+}
+
+void prof_end(gs_ctx* c, int stage, int64_t work, cudaStream_t st) {
+  auto& P = c->prof;
+  if (!P.on) return;
+  cudaEventRecord(P.ev[2 * P.nrec + 1], st);
+  P.stage[P.nrec++] = stage;
+  P.launches[stage] += 1;
+  P.work[stage] += work;
+}
+
+__global__ void unpack_preprocess_kernel(const gs::Screen* screen, const float* depth,
+                                         const uint2* rect, const uint32_t* touched,
+                                         const uint8_t* clamped, int64_t n, float* mean2d,
+                                         float* conic, float* opacity, float* rgb, float* dep,
+                                         int32_t* rc, int32_t* tt, uint8_t* cl) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const gs::Screen s = screen[i];
+  if (mean2d) {
+    mean2d[2 * i] = s.a.x;
+    mean2d[2 * i + 1] = s.a.y;
+  }
+  if (conic) {
+    conic[3 * i] = s.a.z;
+    conic[3 * i + 1] = s.a.w;
+    conic[3 * i + 2] = s.b.x;
+  }
+  if (opacity) opacity[i] = s.b.y;
+  if (rgb) {
+    rgb[3 * i] = s.b.z;
+    rgb[3 * i + 1] = s.b.w;
+    rgb[3 * i + 2] = s.c.x;
+  }
+  if (dep) dep[i] = depth[i];
+  if (rc) {
+    const uint2 r = rect[i];
+    rc[4 * i] = static_cast<int32_t>(r.x & 0xffffu);
+    rc[4 * i + 1] = static_cast<int32_t>(r.y & 0xffffu);
+    rc[4 * i + 2] = static_cast<int32_t>(r.x >> 16);
+    rc[4 * i + 3] = static_cast<int32_t>(r.y >> 16);
+  }
+  if (tt) tt[i] = static_cast<int32_t>(touched[i]);
+  if (cl) cl[i] = clamped[i];
+}
+
+__global__ void key_tiles_kernel(const uint64_t* keys, int64_t n, int depth_bits, int32_t* tiles) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i < n) tiles[i] = static_cast<int32_t>(keys[i] >> depth_bits);
+}
+
+int bit_length(uint64_t v) { return v == 0 ? 0 : 64 - __builtin_clzll(v); }
+
+}  // namespace
+
+extern "C" {
+
+gs_status gs_create(gs_ctx** out, int64_t max_gaussians, int64_t max_entries, int32_t max_width,
+                    int32_t max_height) {
+  if (!out) return GS_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (max_gaussians <= 0 || max_entries <= 0 || max_width <= 0 || max_height <= 0 ||
+      max_gaussians > (int64_t(1) << 31) - 1 || max_entries >= (int64_t(1) << 30) ||
+      max_width > 16 * 65535 || max_height > 16 * 65535)
+    return GS_ERR_INVALID_ARG;
+  gs_ctx* c = new gs_ctx();
+  c->max_g = max_gaussians;
+  c->max_k = max_entries;
+  c->max_w = max_width;
+  c->max_h = max_height;
+  c->max_tiles = static_cast<int64_t>((max_width + 15) / 16) * ((max_height + 15) / 16);
+  c->max_blocks = (max_gaussians + 255) / 256;
+  c->max_sort_tiles = (max_entries + gs::kSortTileKeys - 1) / gs::kSortTileKeys;
+  c->max_loss_blocks = gs::loss_num_blocks(max_height, max_width);
+  const int64_t G = max_gaussians, K = max_entries;
+  cudaError_t e = cudaSuccess;
+#define GS_ALLOC(ptr, bytes) \
+  if (e == cudaSuccess) e = cudaMalloc(reinterpret_cast<void**>(&(ptr)), (bytes))
+  GS_ALLOC(c->screen, sizeof(gs::Screen) * G);
+  GS_ALLOC(c->depth, sizeof(float) * G);
+  GS_ALLOC(c->rect, sizeof(uint2) * G);
+  GS_ALLOC(c->touched, sizeof(uint32_t) * G);
+  GS_ALLOC(c->clamped, sizeof(uint8_t) * G);
+  GS_ALLOC(c->sgrad, sizeof(float) * gs::kGradStride * G);
+  GS_ALLOC(c->block_sums, sizeof(uint32_t) * c->max_blocks);
+  GS_ALLOC(c->block_prefix, sizeof(uint64_t) * c->max_blocks);
+  GS_ALLOC(c->depth_range, sizeof(uint32_t) * 2);
+  GS_ALLOC(c->keys[0], sizeof(uint64_t) * K);
+  GS_ALLOC(c->keys[1], sizeof(uint64_t) * K);
+  GS_ALLOC(c->vals[0], sizeof(uint32_t) * K);
+  GS_ALLOC(c->vals[1], sizeof(uint32_t) * K);
+  GS_ALLOC(c->hist, sizeof(uint32_t) * gs::kMaxPasses * gs::kRadix);
+  GS_ALLOC(c->offsets, sizeof(uint32_t) * gs::kMaxPasses * gs::kRadix);
+  GS_ALLOC(c->status, sizeof(uint32_t) * gs::kMaxPasses * gs::kRadix * c->max_sort_tiles);
+  GS_ALLOC(c->counters, sizeof(uint32_t) * gs::kMaxPasses);
+  GS_ALLOC(c->ranges, sizeof(uint2) * c->max_tiles);
+  GS_ALLOC(c->loss_partials, sizeof(double) * 2 * c->max_loss_blocks);
+  GS_ALLOC(c->loss_counter, sizeof(uint32_t));
+  GS_ALLOC(c->info_dev, sizeof(gs::ForwardInfo));
+  GS_ALLOC(c->pairs, sizeof(unsigned long long) * 2);
+#undef GS_ALLOC
+  if (e == cudaSuccess) e = cudaMallocHost(reinterpret_cast<void**>(&c->info_host), sizeof(gs::ForwardInfo));
+  if (e == cudaSuccess) e = cudaMemset(c->loss_counter, 0, sizeof(uint32_t));
+  if (e == cudaSuccess) e = cudaMemset(c->info_dev, 0, sizeof(gs::ForwardInfo));
+  if (e == cudaSuccess) e = cudaMemset(c->pairs, 0, sizeof(unsigned long long) * 2);
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) {
+    free_all(c);
+    delete c;
+    cudaGetLastError();
+    return GS_ERR_CUDA;
+  }
+  std::memset(c->info_host, 0, sizeof(gs::ForwardInfo));
+  *out = c;
+  return GS_OK;
+}
+
+void gs_destroy(gs_ctx* ctx) {
+  if (!ctx) return;
+  cudaDeviceSynchronize();
+  free_all(ctx);
+  delete ctx;
+}
+
+const char* gs_last_error(const gs_ctx* ctx) { return ctx ? ctx->err : "no context"; }
+
+gs_status gs_preprocess(gs_ctx* c, const gs_params* p, const gs_camera* cam, void* stream) {
+  if (!c) return GS_ERR_INVALID_ARG;
+  gs_status s = check_params(c, p);
+  if (s != GS_OK) return s;
+  gs::CamArgs ca;
+  if ((s = make_cam(c, cam, ca)) != GS_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  c->have_pre = c->have_fwd = false;
+  GS_CUDA(c, cudaMemsetAsync(c->depth_range, 0xff, sizeof(uint32_t), st));
+  GS_CUDA(c, cudaMemsetAsync(c->depth_range + 1, 0, sizeof(uint32_t), st));
+  gs::PreprocessArgs a;
+  a.means = p->means;
+  a.log_scales = p->log_scales;
+  a.quats = p->quats;
+  a.opacity_logits = p->opacity_logits;
+  a.sh = p->sh;
+  a.n = p->n;
+  a.n_pad = p->n_pad;
+  a.sh_k = (p->sh_degree + 1) * (p->sh_degree + 1);
+  a.active_degree = p->active_degree;
+  a.cam = ca;
+  a.screen = c->screen;
+  a.depth = c->depth;
+  a.rect = c->rect;
+  a.touched = c->touched;
+  a.clamped = c->clamped;
+  a.block_sums = c->block_sums;
+  a.depth_range = c->depth_range;
+  const int64_t nb = (p->n + 255) / 256;
+  prof_begin(c, st);
+  GS_CUDA(c, gs::launch_preprocess(a, nb, st));
+  prof_end(c, GS_STAGE_PREPROCESS, p->n, st);
+  prof_begin(c, st);
+  GS_CUDA(c, gs::launch_scan_blocks(c->block_sums, nb, c->block_prefix, c->depth_range, c->info_dev, st));
+  prof_end(c, GS_STAGE_SCAN, nb, st);
+  c->n = p->n;
+  c->n_pad = p->n_pad;
+  c->cam = ca;
+  c->have_pre = true;
+  return GS_OK;
+}
+
+gs_status gs_render_forward(gs_ctx* c, const gs_camera* cam, float* image, float* final_T,
+                            int32_t* n_contrib, int64_t* num_entries_out, void* stream) {
+  if (!c) return GS_ERR_INVALID_ARG;
+  if (!c->have_pre) return fail(c, GS_ERR_INVALID_ARG, "gs_preprocess has not run");
+  gs::CamArgs ca;
+  gs_status s = make_cam(c, cam, ca);
+  if (s != GS_OK) return s;
+  if (ca.width != c->cam.width || ca.height != c->cam.height)
+    return fail(c, GS_ERR_INVALID_ARG, "camera size differs from the one preprocessed");
+  if (!image || !final_T || !n_contrib || !aligned(image, 4) || !aligned(final_T, 4) ||
+      !aligned(n_contrib, 4))
+    return fail(c, GS_ERR_INVALID_ARG, "output pointers must be non-NULL and 4-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  c->have_fwd = false;
+  // The one host/device crossing of the step: entry count and depth-key range.
+  GS_CUDA(c, cudaMemcpyAsync(c->info_host, c->info_dev, sizeof(gs::ForwardInfo),
+                             cudaMemcpyDeviceToHost, st));
+  GS_CUDA(c, cudaStreamSynchronize(st));
+  if ((s = take_device_error(c)) != GS_OK) return s;
+  const uint64_t K = c->info_host->num_entries;
+  if (num_entries_out) *num_entries_out = static_cast<int64_t>(K);
+  if (K > static_cast<uint64_t>(c->max_k))
+    return fail(c, GS_ERR_CAPACITY, "%llu (Gaussian, tile) entries exceed the context's %lld",
+                (unsigned long long)K, (long long)c->max_k);
+  const int64_t tiles = static_cast<int64_t>(ca.tiles_x) * ca.tiles_y;
+  int depth_bits = 0;
+  uint32_t dmin = 0;
+  if (K > 0) {
+    dmin = c->info_host->depth_min;
+    depth_bits = bit_length(c->info_host->depth_max - dmin);
+  }
+  const int key_bits = bit_length(static_cast<uint64_t>(tiles - 1)) + depth_bits;
+  int sorted = 0;
+  if (K > 0) {
+    gs::DuplicateArgs d;
+    d.n = c->n;
+    d.touched = c->touched;
+    d.rect = c->rect;
+    d.depth = c->depth;
+    d.block_prefix = c->block_prefix;
+    d.depth_min = dmin;
+    d.depth_bits = depth_bits;
+    d.tiles_x = ca.tiles_x;
+    d.max_entries = c->max_k;
+    d.keys = c->keys[0];
+    d.vals = c->vals[0];
+    d.err = &c->info_dev->device_error;
+    prof_begin(c, st);
+    GS_CUDA(c, gs::launch_duplicate(d, (c->n + 255) / 256, st));
+    prof_end(c, GS_STAGE_DUPLICATE, static_cast<int64_t>(K), st);
+    gs::SortPlan plan;
+    plan.n = static_cast<int64_t>(K);
+    plan.depth_bits = depth_bits;
+    plan.key_bits = key_bits;
+    plan.passes = (key_bits + 7) / 8;
+    plan.tiles = (plan.n + gs::kSortTileKeys - 1) / gs::kSortTileKeys;
+    gs::SortBuffers b;
+    b.keys[0] = c->keys[0];
+    b.keys[1] = c->keys[1];
+    b.vals[0] = c->vals[0];
+    b.vals[1] = c->vals[1];
+    b.hist = c->hist;
+    b.offsets = c->offsets;
+    b.status = c->status;
+    b.counters = c->counters;
+    b.err = &c->info_dev->device_error;
+    prof_begin(c, st);
+    GS_CUDA(c, gs::launch_sort(plan, b, &sorted, st));
+    prof_end(c, GS_STAGE_SORT, plan.n > 1 ? plan.n * plan.passes : 0, st);
+  }
+  prof_begin(c, st);
+  GS_CUDA(c, gs::launch_ranges(c->keys[sorted], static_cast<int64_t>(K), depth_bits, c->ranges, tiles, st));
+  prof_end(c, GS_STAGE_RANGES, static_cast<int64_t>(K), st);
+  gs::BlendArgs ba{};
+  ba.ranges = c->ranges;
+  ba.order = c->vals[sorted];
+  ba.screen = c->screen;
+  ba.cam = c->cam;
+  std::memcpy(ba.cam.bg, ca.bg, sizeof(ba.cam.bg));
+  ba.image = image;
+  ba.final_T = final_T;
+  ba.n_contrib = n_contrib;
+  ba.pairs = c->prof.on ? c->pairs : nullptr;
+  prof_begin(c, st);
+  GS_CUDA(c, gs::launch_blend_forward(ba, st));
+  prof_end(c, GS_STAGE_BLEND_FORWARD, 0, st);
+  c->K = static_cast<int64_t>(K);
+  c->depth_bits = depth_bits;
+  c->depth_min = dmin;
+  c->sorted_buf = sorted;
+  c->cam.bg[0] = ca.bg[0];
+  c->cam.bg[1] = ca.bg[1];
+  c->cam.bg[2] = ca.bg[2];
+  c->have_fwd = true;
+  return GS_OK;
+}
+
+gs_status gs_loss_l1_dssim(gs_ctx* c, const float* image, const float* target, int32_t height,
+                           int32_t width, float lambda, double* loss_out, float* dloss_dimage,
+                           void* stream) {
+  if (!c) return GS_ERR_INVALID_ARG;
+  if (height <= 0 || width <= 0 || height > c->max_h || width > c->max_w)
+    return fail(c, GS_ERR_INVALID_ARG, "image %dx%d outside the context's maximum", width, height);
+  if (!image || !target || !loss_out || !aligned(image, 4) || !aligned(target, 4) ||
+      !aligned(loss_out, 8) || (dloss_dimage && !aligned(dloss_dimage, 4)))
+    return fail(c, GS_ERR_INVALID_ARG, "loss pointers must be non-NULL and aligned");
+  if (!std::isfinite(lambda)) return fail(c, GS_ERR_INVALID_ARG, "lambda must be finite");
+  gs::LossArgs a;
+  a.x = image;
+  a.y = target;
+  a.height = height;
+  a.width = width;
+  a.lambda = lambda;
+  double g[11], sum = 0.0;
+  for (int i = 0; i < 11; ++i) sum += (g[i] = std::exp(-((i - 5) * (i - 5)) / (2.0 * 1.5 * 1.5)));
+  for (int i = 0; i < 11; ++i) a.window[i] = static_cast<float>(g[i] / sum);
+  a.dx = dloss_dimage;
+  a.partials = c->loss_partials;
+  a.counter = c->loss_counter;
+  a.out = loss_out;
+  prof_begin(c, static_cast<cudaStream_t>(stream));
+  GS_CUDA(c, gs::launch_loss(a, static_cast<cudaStream_t>(stream)));
+  prof_end(c, GS_STAGE_LOSS, static_cast<int64_t>(height) * width, static_cast<cudaStream_t>(stream));
+  return GS_OK;
+}
+
+gs_status gs_render_backward(gs_ctx* c, const gs_params* p, const gs_camera* cam, const float* final_T,
+                             const int32_t* n_contrib, const float* dloss_dimage, gs_grads* g,
+                             void* stream) {
+  if (!c) return GS_ERR_INVALID_ARG;
+  if (!c->have_fwd) return fail(c, GS_ERR_INVALID_ARG, "gs_render_forward has not run");
+  gs_status s = check_params(c, p);
+  if (s != GS_OK) return s;
+  if (p->n != c->n || p->n_pad != c->n_pad)
+    return fail(c, GS_ERR_INVALID_ARG, "params differ from the ones preprocessed");
+  gs::CamArgs ca;
+  if ((s = make_cam(c, cam, ca)) != GS_OK) return s;
+  if (ca.width != c->cam.width || ca.height != c->cam.height)
+    return fail(c, GS_ERR_INVALID_ARG, "camera size differs from the one rendered");
+  if (!final_T || !n_contrib || !dloss_dimage || !g)
+    return fail(c, GS_ERR_INVALID_ARG, "backward inputs must be non-NULL");
+  float* gp[] = {g->means, g->log_scales, g->quats, g->opacity_logits, g->sh};
+  if (p->n > 0)
+    for (float* q : gp)
+      if (!q || !aligned(q, 4)) return fail(c, GS_ERR_INVALID_ARG, "a gradient pointer is NULL or misaligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (p->n > 0)
+    GS_CUDA(c, cudaMemsetAsync(c->sgrad, 0, sizeof(float) * gs::kGradStride * p->n, st));
+  gs::BlendArgs ba{};
+  ba.ranges = c->ranges;
+  ba.order = c->vals[c->sorted_buf];
+  ba.screen = c->screen;
+  ba.cam = c->cam;
+  ba.final_T = const_cast<float*>(final_T);
+  ba.n_contrib = const_cast<int32_t*>(n_contrib);
+  ba.dimage = dloss_dimage;
+  ba.sgrad = c->sgrad;
+  ba.pairs = c->prof.on ? c->pairs + 1 : nullptr;
+  prof_begin(c, st);
+  GS_CUDA(c, gs::launch_blend_backward(ba, st));
+  prof_end(c, GS_STAGE_BLEND_BACKWARD, 0, st);
+  gs::PreprocessBwdArgs a;
+  a.means = p->means;
+  a.log_scales = p->log_scales;
+  a.quats = p->quats;
+  a.opacity_logits = p->opacity_logits;
+  a.sh = p->sh;
+  a.n = p->n;
+  a.n_pad = p->n_pad;
+  a.sh_k = (p->sh_degree + 1) * (p->sh_degree + 1);
+  a.active_degree = p->active_degree;
+  a.cam = c->cam;
+  a.screen = c->screen;
+  a.touched = c->touched;
+  a.clamped = c->clamped;
+  a.sgrad = c->sgrad;
+  a.g_means = g->means;
+  a.g_log_scales = g->log_scales;
+  a.g_quats = g->quats;
+  a.g_opacity_logits = g->opacity_logits;
+  a.g_sh = g->sh;
+  prof_begin(c, st);
+  GS_CUDA(c, gs::launch_preprocess_backward(a, st));
+  prof_end(c, GS_STAGE_PREPROCESS_BACKWARD, p->n, st);
+  return GS_OK;
+}
+
+gs_status gs_adam_step(float* param, float* grad, float* m, float* v, int64_t count, float lr,
+                       float beta1, float beta2, float eps, int32_t step, void* stream) {
+  if (count < 0 || step < 1) return GS_ERR_INVALID_ARG;
+  if (count > 0 && (!param || !grad || !m || !v || !aligned(param, 4) || !aligned(grad, 4) ||
+                    !aligned(m, 4) || !aligned(v, 4)))
+    return GS_ERR_INVALID_ARG;
+  if (!(beta1 >= 0.f && beta1 < 1.f && beta2 >= 0.f && beta2 < 1.f && eps > 0.f && std::isfinite(lr)))
+    return GS_ERR_INVALID_ARG;
+  cudaError_t e = gs::launch_adam(param, grad, m, v, count, lr, beta1, beta2, eps, step,
+                                  static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? GS_OK : GS_ERR_CUDA;
+}
+
+gs_status gs_profile_enable(gs_ctx* c, int32_t enabled) {
+  if (!c) return GS_ERR_INVALID_ARG;
+  auto& P = c->prof;
+  if (enabled && !P.created) {
+    for (auto& e : P.ev) GS_CUDA(c, cudaEventCreate(&e));
+    P.created = true;
+  }
+  if (P.on && !enabled) prof_harvest(c);
+  P.on = enabled != 0;
+  return GS_OK;
+}
+
+gs_status gs_profile_read(gs_ctx* c, double* ms, int64_t* launches, int64_t* work) {
+  if (!c) return GS_ERR_INVALID_ARG;
+  auto& P = c->prof;
+  prof_harvest(c);
+  unsigned long long pairs[2] = {0ull, 0ull};
+  GS_CUDA(c, cudaMemcpy(pairs, c->pairs, sizeof(pairs), cudaMemcpyDeviceToHost));
+  GS_CUDA(c, cudaMemset(c->pairs, 0, sizeof(pairs)));
+  P.work[GS_STAGE_BLEND_FORWARD] += static_cast<int64_t>(pairs[0]);
+  P.work[GS_STAGE_BLEND_BACKWARD] += static_cast<int64_t>(pairs[1]);
+  for (int k = 0; k < GS_NUM_STAGES; ++k) {
+    if (ms) ms[k] = P.ms[k];
+    if (launches) launches[k] = P.launches[k];
+    if (work) work[k] = P.work[k];
+    P.ms[k] = 0.0;
+    P.launches[k] = 0;
+    P.work[k] = 0;
+  }
+  return GS_OK;
+}
+
+const char* gs_stage_name(int32_t stage) {
+  static const char* names[GS_NUM_STAGES] = {"preprocess", "scan", "duplicate", "sort", "ranges",
+                                             "blend_forward", "loss", "blend_backward",
+                                             "preprocess_backward"};
+  return (stage >= 0 && stage < GS_NUM_STAGES) ? names[stage] : "";
+}
+
+gs_status gs_debug_preprocess(gs_ctx* c, float* mean2d, float* conic, float* opacity, float* rgb,
+                              float* depth, int32_t* rect, int32_t* tiles_touched, uint8_t* clamped,
+                              void* stream) {
+  if (!c) return GS_ERR_INVALID_ARG;
+  if (!c->have_pre) return fail(c, GS_ERR_INVALID_ARG, "gs_preprocess has not run");
+  if (c->n == 0) return GS_OK;
+  unpack_preprocess_kernel<<<static_cast<unsigned>((c->n + 255) / 256), 256, 0,
+                             static_cast<cudaStream_t>(stream)>>>(
+      c->screen, c->depth, c->rect, c->touched, c->clamped, c->n, mean2d, conic, opacity, rgb, depth,
+      rect, tiles_touched, clamped);
+  GS_CUDA(c, cudaGetLastError());
+  return GS_OK;
+}
+
+gs_status gs_debug_sorted(gs_ctx* c, int32_t* ids, int32_t* tiles, int32_t* ranges, void* stream) {
+  if (!c) return GS_ERR_INVALID_ARG;
+  if (!c->have_fwd) return fail(c, GS_ERR_INVALID_ARG, "gs_render_forward has not run");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (ids && c->K > 0)
+    GS_CUDA(c, cudaMemcpyAsync(ids, c->vals[c->sorted_buf], sizeof(uint32_t) * c->K,
+                               cudaMemcpyDeviceToDevice, st));
+  if (tiles && c->K > 0) {
+    key_tiles_kernel<<<static_cast<unsigned>((c->K + 255) / 256), 256, 0, st>>>(
+        c->keys[c->sorted_buf], c->K, c->depth_bits, tiles);
+    GS_CUDA(c, cudaGetLastError());
+  }
+  if (ranges)
+    GS_CUDA(c, cudaMemcpyAsync(ranges, c->ranges,
+                               sizeof(uint2) * static_cast<int64_t>(c->cam.tiles_x) * c->cam.tiles_y,
+                               cudaMemcpyDeviceToDevice, st));
+  return GS_OK;
+}
+
+gs_status gs_debug_screen_grads(gs_ctx* c, float* out, void* stream) {
+  if (!c || !out) return GS_ERR_INVALID_ARG;
+  if (!c->have_fwd) return fail(c, GS_ERR_INVALID_ARG, "gs_render_forward has not run");
+  GS_CUDA(c, gs::launch_screen_grads(c->screen, c->sgrad, c->n, out, static_cast<cudaStream_t>(stream)));
+  return GS_OK;
+}
+
+}  // extern "C"

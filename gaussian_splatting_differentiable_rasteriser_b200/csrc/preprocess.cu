@@ -1,0 +1,231 @@
+// Preprocess: one thread per Gaussian projects it to the screen.
+//
+// Method: "Gaussian splatting training" study notes (bailiping.com), slides on
+// the parametrisation and "J is the 2 x 3 Jacobian of perspective projection";
+// "How a computer rebuilds a real place ... Gaussian Splats" (taosengine.com),
+// sections "Flattening a 3D blob into a 2D oval (EWA projection)" (T = J W,
+// Sigma' = T Sigma T^T, conic, radius from the largest eigenvalue, tile rect)
+// and "Spherical harmonics: color that changes with viewing angle".
+//
+// B200 notes: the kernel is HBM-bound (236 B of parameters in, 48 + 17 B out
+// per Gaussian at SH degree 3); all parameter loads are coalesced planar
+// reads. The geometry runs in float64 - free next to the memory time - so that
+// the integer decisions taken from it (culling, tile rect, depth key) are
+// stable to ~1e-15 and do not depend on float32 rounding order.
+#include "gs_kernels.cuh"
+#include "sh.cuh"
+
+namespace gs {
+
+namespace {
+
+__device__ __forceinline__ double dot3(const double* a, const double* b) {
+  return a[0] * b[0] + a[1] * b[1] + a[2] * b[2];
+}
+
+__global__ void __launch_bounds__(256) preprocess_kernel(PreprocessArgs a) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  uint32_t touched = 0;
+  uint32_t dkey = 0;
+  bool visible = false;
+  if (i < a.n) {
+    const int64_t np = a.n_pad;
+    const CamArgs& cam = a.cam;
+    const double p[3] = {a.means[i], a.means[np + i], a.means[2 * np + i]};
+    // p_c = R p + t, each row summed left to right without fused multiply-add:
+    // the depth key float32(Z) is then the same on every implementation.
+    double pc[3];
+#pragma unroll
+    for (int r = 0; r < 3; ++r)
+      pc[r] = __dadd_rn(__dadd_rn(__dadd_rn(__dmul_rn(cam.R[3 * r], p[0]),
+                                            __dmul_rn(cam.R[3 * r + 1], p[1])),
+                                  __dmul_rn(cam.R[3 * r + 2], p[2])),
+                        static_cast<double>(cam.t[r]));
+    const double X = pc[0], Y = pc[1], Z = pc[2];
+    const float depth = __double2float_rn(Z);
+    Screen s;
+    s.a = make_float4(0.f, 0.f, 0.f, 0.f);
+    s.b = s.a;
+    s.c = s.a;
+    uint2 rect = make_uint2(1u, 1u);  // x0 = 1 > x1 = 0: empty
+    uint8_t clamped = 0;
+    if (Z > static_cast<double>(cam.near_z)) {
+      // Sigma = M M^T, M = R(q/|q|) diag(exp(ls))
+      const double qw = a.quats[i], qx = a.quats[np + i], qy = a.quats[2 * np + i],
+                   qz = a.quats[3 * np + i];
+      const double qn = sqrt(qw * qw + qx * qx + qy * qy + qz * qz);
+      const double w = qw / qn, x = qx / qn, y = qy / qn, z = qz / qn;
+      const double Rq[9] = {1.0 - 2.0 * (y * y + z * z), 2.0 * (x * y - w * z), 2.0 * (x * z + w * y),
+                            2.0 * (x * y + w * z), 1.0 - 2.0 * (x * x + z * z), 2.0 * (y * z - w * x),
+                            2.0 * (x * z - w * y), 2.0 * (y * z + w * x), 1.0 - 2.0 * (x * x + y * y)};
+      const double sc[3] = {exp(static_cast<double>(a.log_scales[i])),
+                            exp(static_cast<double>(a.log_scales[np + i])),
+                            exp(static_cast<double>(a.log_scales[2 * np + i]))};
+      double M[9];
+#pragma unroll
+      for (int r = 0; r < 3; ++r)
+#pragma unroll
+        for (int c = 0; c < 3; ++c) M[3 * r + c] = Rq[3 * r + c] * sc[c];
+      const double S00 = dot3(M, M), S01 = dot3(M, M + 3), S02 = dot3(M, M + 6);
+      const double S11 = dot3(M + 3, M + 3), S12 = dot3(M + 3, M + 6), S22 = dot3(M + 6, M + 6);
+      // T = J W (rows t0, t1)
+      const double iz = 1.0 / Z;
+      const double jx = cam.fx * iz, jy = cam.fy * iz;
+      const double jxz = -cam.fx * X * iz * iz, jyz = -cam.fy * Y * iz * iz;
+      double t0[3], t1[3];
+#pragma unroll
+      for (int c = 0; c < 3; ++c) {
+        t0[c] = jx * cam.R[c] + jxz * cam.R[6 + c];
+        t1[c] = jy * cam.R[3 + c] + jyz * cam.R[6 + c];
+      }
+      // Sigma' = T Sigma T^T + 0.3 I
+      const double u0[3] = {S00 * t0[0] + S01 * t0[1] + S02 * t0[2],
+                            S01 * t0[0] + S11 * t0[1] + S12 * t0[2],
+                            S02 * t0[0] + S12 * t0[1] + S22 * t0[2]};
+      const double u1[3] = {S00 * t1[0] + S01 * t1[1] + S02 * t1[2],
+                            S01 * t1[0] + S11 * t1[1] + S12 * t1[2],
+                            S02 * t1[0] + S12 * t1[1] + S22 * t1[2]};
+      const double ca = dot3(t0, u0) + kDilation;
+      const double cb = dot3(t0, u1);
+      const double cc = dot3(t1, u1) + kDilation;
+      const double det = ca * cc - cb * cb;
+      if (det > 0.0) {
+        const double u = cam.fx * X * iz + cam.cx;
+        const double v = cam.fy * Y * iz + cam.cy;
+        const double mid = 0.5 * (ca + cc);
+        const double lmax = mid + sqrt(fmax(mid * mid - det, 0.0));
+        const double rad = kRadiusSigmas * sqrt(lmax);
+        // tiles whose pixels [16 t, 16 t + 15] meet [u - r, u + r] (same for y)
+        double fx0 = fmax(ceil((u - rad - (kTile - 1)) / kTile), 0.0);
+        double fx1 = fmin(floor((u + rad) / kTile), static_cast<double>(cam.tiles_x - 1));
+        double fy0 = fmax(ceil((v - rad - (kTile - 1)) / kTile), 0.0);
+        double fy1 = fmin(floor((v + rad) / kTile), static_cast<double>(cam.tiles_y - 1));
+        if (fx0 <= fx1 && fy0 <= fy1) {  // false for NaN too
+          const uint32_t x0 = static_cast<uint32_t>(fx0), x1 = static_cast<uint32_t>(fx1);
+          const uint32_t y0 = static_cast<uint32_t>(fy0), y1 = static_cast<uint32_t>(fy1);
+          rect = make_uint2(x0 | (x1 << 16), y0 | (y1 << 16));
+          touched = (x1 - x0 + 1) * (y1 - y0 + 1);
+          visible = true;
+          dkey = __float_as_uint(depth);
+          const float opacity = 1.0f / (1.0f + expf(-a.opacity_logits[i]));
+          // view-dependent colour at v = normalize(p - campos)
+          double d[3] = {p[0] - cam.campos[0], p[1] - cam.campos[1], p[2] - cam.campos[2]};
+          const double dn = sqrt(dot3(d, d));
+          const float dx = static_cast<float>(d[0] / dn), dy = static_cast<float>(d[1] / dn),
+                      dz = static_cast<float>(d[2] / dn);
+          float Yk[16];
+          sh_basis(a.active_degree, dx, dy, dz, Yk);
+          const int nk = (a.active_degree + 1) * (a.active_degree + 1);
+          float rgb[3];
+#pragma unroll
+          for (int ch = 0; ch < 3; ++ch) {
+            const float* shc = a.sh + static_cast<int64_t>(ch) * a.sh_k * np + i;
+            float col = 0.0f;
+            for (int k = 0; k < nk; ++k) col = fmaf(shc[static_cast<int64_t>(k) * np], Yk[k], col);
+            if (col < 0.0f) {
+              col = 0.0f;
+              clamped |= static_cast<uint8_t>(1u << ch);
+            }
+            rgb[ch] = col;
+          }
+          s.a = make_float4(static_cast<float>(u), static_cast<float>(v),
+                            static_cast<float>(cc / det), static_cast<float>(-cb / det));
+          s.b = make_float4(static_cast<float>(ca / det), opacity, rgb[0], rgb[1]);
+          s.c = make_float4(rgb[2], depth, 0.0f, 0.0f);
+        }
+      }
+    }
+    a.screen[i] = s;
+    a.depth[i] = depth;
+    a.rect[i] = rect;
+    a.touched[i] = touched;
+    a.clamped[i] = clamped;
+  }
+
+  // Block total of tiles_touched (for the prefix sum) and the depth-key range
+  // of visible Gaussians (to size the sort key).
+  __shared__ uint32_t s_sum[8];
+  uint32_t t = touched;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+  uint32_t kmin = visible ? dkey : 0xffffffffu, kmax = visible ? dkey : 0u;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+    kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+  }
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (lane == 0) {
+    s_sum[warp] = t;
+    if (kmin <= kmax) {
+      atomicMin(&a.depth_range[0], kmin);
+      atomicMax(&a.depth_range[1], kmax);
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t b = 0;
+    for (int k = 0; k < (blockDim.x >> 5); ++k) b += s_sum[k];
+    a.block_sums[blockIdx.x] = b;
+  }
+}
+
+// Exclusive prefix of the per-block totals (one CTA of 1024 threads), plus the
+// grand total and the depth-key range copied into the readback record.
+__global__ void __launch_bounds__(1024) scan_blocks_kernel(const uint32_t* block_sums, int64_t nb,
+                                                           uint64_t* block_prefix,
+                                                           const uint32_t* depth_range,
+                                                           ForwardInfo* info) {
+  __shared__ uint64_t s_warp[32];
+  const int tid = threadIdx.x;
+  const int64_t per = (nb + blockDim.x - 1) / blockDim.x;
+  const int64_t lo = tid * per, hi = min(nb, lo + per);
+  uint64_t local = 0;
+  for (int64_t k = lo; k < hi; ++k) local += block_sums[k];
+  // inclusive scan of `local` across the CTA
+  uint64_t v = local;
+  const int lane = tid & 31, warp = tid >> 5;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    uint64_t n = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += n;
+  }
+  if (lane == 31) s_warp[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    uint64_t w = s_warp[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      uint64_t n = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += n;
+    }
+    s_warp[lane] = w;
+  }
+  __syncthreads();
+  uint64_t run = v - local + (warp > 0 ? s_warp[warp - 1] : 0);
+  for (int64_t k = lo; k < hi; ++k) {
+    block_prefix[k] = run;
+    run += block_sums[k];
+  }
+  if (tid == blockDim.x - 1) {
+    info->num_entries = s_warp[31];
+    info->depth_min = depth_range[0];
+    info->depth_max = depth_range[1];
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_preprocess(const PreprocessArgs& a, int64_t num_blocks, cudaStream_t st) {
+  if (a.n == 0) return cudaSuccess;
+  preprocess_kernel<<<static_cast<unsigned>(num_blocks), 256, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_scan_blocks(const uint32_t* block_sums, int64_t num_blocks, uint64_t* block_prefix,
+                               const uint32_t* depth_range, ForwardInfo* info, cudaStream_t st) {
+  scan_blocks_kernel<<<1, 1024, 0, st>>>(block_sums, num_blocks, block_prefix, depth_range, info);
+  return cudaGetLastError();
+}
+
+}  // namespace gs

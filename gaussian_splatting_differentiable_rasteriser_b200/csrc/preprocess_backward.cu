@@ -1,0 +1,233 @@
+// Projection backward: per-Gaussian screen-space gradient -> stored parameters.
+//
+// Method: "How a computer rebuilds a real place ... Gaussian Splats"
+// (taosengine.com), sections "From a pixel's blame to the oval's shape and
+// place", "The covariance chain: oval -> 3D ellipsoid -> size & tilt" and
+// "Where the position gradient comes from", and the spherical-harmonics
+// backward (dL/dsh_k = dL/dcolour * Y_k, plus the view-direction term into the
+// position); "Gaussian splatting training" study notes (bailiping.com), slide
+// "J is the 2 x 3 Jacobian of perspective projection" (the position derivative
+// includes the path through J, not only the projected mean).
+//
+// Chain, per Gaussian (float32):
+//   raw blend sums -> dL/d(mean2d, A, B, C, opacity)
+//   conic K = V'^-1:        dL/dV' = -K G_K K   (G_K with the B gradient halved)
+//   V' = T Sigma T^T + 0.3I: dL/dSigma = T^T G_V T,   dL/dT = 2 G_V T Sigma
+//   T = J W:                dL/dJ = dL/dT W^T -> dL/d(X, Y, Z) (1/Z, 1/Z^2 terms)
+//   mean2d(X, Y, Z)         -> dL/d(X, Y, Z);   dL/dp = W^T dL/dp_c
+//   Sigma = M M^T:          dL/dM = 2 dL/dSigma M,  M = R(q^) diag(s)
+//   dL/ds_j = sum_i dL/dM_ij R_ij (times s for the log-scale), dL/dR = dL/dM diag(s)
+//   R(q^) -> dL/dq^, then dL/dq = (dL/dq^ - q^ <q^, dL/dq^>) / |q|
+//   colour: dL/dsh_k = dL/dc Y_k, dL/dv = sum dL/dc sh_k grad Y_k,
+//           dL/dp += (dL/dv - v <v, dL/dv>) / |p - campos|
+// The result is ADDED to the caller's gradient buffers (coalesced planar RMW).
+#include "gs_kernels.cuh"
+#include "sh.cuh"
+
+namespace gs {
+
+namespace {
+
+__global__ void __launch_bounds__(256) preprocess_backward_kernel(PreprocessBwdArgs a) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= a.n || a.touched[i] == 0) return;
+  const int64_t np = a.n_pad;
+  const CamArgs& cam = a.cam;
+  const float4* sg4 = reinterpret_cast<const float4*>(a.sgrad + i * kGradStride);
+  const float4 r0 = sg4[0], r1 = sg4[1], r2 = sg4[2];
+  const Screen scr = a.screen[i];
+  const float A = scr.a.z, B = scr.a.w, C = scr.b.x, o = scr.b.y;
+  const uint8_t clamped = a.clamped[i];
+
+  // Screen-space gradient from the raw sums (w = dL/dalpha * o exp(-e)).
+  const float d_u = A * r0.y + B * r0.z;
+  const float d_v = B * r0.y + C * r0.z;
+  const float dA = -0.5f * r0.w, dB = -r1.x, dC = -0.5f * r1.y;
+  const float d_o = r0.x / o;
+  const float drgb[3] = {(clamped & 1) ? 0.f : r1.z, (clamped & 2) ? 0.f : r1.w,
+                         (clamped & 4) ? 0.f : r2.x};
+
+  // Recompute the forward quantities.
+  const float p[3] = {a.means[i], a.means[np + i], a.means[2 * np + i]};
+  float pc[3];
+#pragma unroll
+  for (int r = 0; r < 3; ++r)
+    pc[r] = cam.R[3 * r] * p[0] + cam.R[3 * r + 1] * p[1] + cam.R[3 * r + 2] * p[2] + cam.t[r];
+  const float X = pc[0], Y = pc[1], Z = pc[2];
+  const float qr[4] = {a.quats[i], a.quats[np + i], a.quats[2 * np + i], a.quats[3 * np + i]};
+  const float qn = sqrtf(qr[0] * qr[0] + qr[1] * qr[1] + qr[2] * qr[2] + qr[3] * qr[3]);
+  const float iqn = 1.0f / qn;
+  const float w = qr[0] * iqn, x = qr[1] * iqn, y = qr[2] * iqn, z = qr[3] * iqn;
+  const float Rq[9] = {1.f - 2.f * (y * y + z * z), 2.f * (x * y - w * z), 2.f * (x * z + w * y),
+                       2.f * (x * y + w * z), 1.f - 2.f * (x * x + z * z), 2.f * (y * z - w * x),
+                       2.f * (x * z - w * y), 2.f * (y * z + w * x), 1.f - 2.f * (x * x + y * y)};
+  const float s[3] = {expf(a.log_scales[i]), expf(a.log_scales[np + i]),
+                      expf(a.log_scales[2 * np + i])};
+  float M[9];
+#pragma unroll
+  for (int r = 0; r < 3; ++r)
+#pragma unroll
+    for (int c = 0; c < 3; ++c) M[3 * r + c] = Rq[3 * r + c] * s[c];
+  float Sig[9];
+#pragma unroll
+  for (int r = 0; r < 3; ++r)
+#pragma unroll
+    for (int c = 0; c < 3; ++c)
+      Sig[3 * r + c] = M[3 * r] * M[3 * c] + M[3 * r + 1] * M[3 * c + 1] + M[3 * r + 2] * M[3 * c + 2];
+  const float iz = 1.0f / Z, iz2 = iz * iz;
+  const float jx = cam.fx * iz, jy = cam.fy * iz;
+  const float jxz = -cam.fx * X * iz2, jyz = -cam.fy * Y * iz2;
+  float T[6];
+#pragma unroll
+  for (int c = 0; c < 3; ++c) {
+    T[c] = jx * cam.R[c] + jxz * cam.R[6 + c];
+    T[3 + c] = jy * cam.R[3 + c] + jyz * cam.R[6 + c];
+  }
+
+  // conic -> V': G_V = -K G_K K, G_K = [[dA, dB/2], [dB/2, dC]]
+  const float hb = 0.5f * dB;
+  const float KG00 = A * dA + B * hb, KG01 = A * hb + B * dC;
+  const float KG10 = B * dA + C * hb, KG11 = B * hb + C * dC;
+  const float GV00 = -(KG00 * A + KG01 * B);
+  const float GV01 = -(KG00 * B + KG01 * C);
+  const float GV11 = -(KG10 * B + KG11 * C);
+  const float GV[4] = {GV00, GV01, GV01, GV11};
+
+  // V' = T Sigma T^T: dSigma = T^T G_V T; dT = 2 G_V T Sigma
+  float GVT[6];  // G_V T (2x3)
+#pragma unroll
+  for (int c = 0; c < 3; ++c) {
+    GVT[c] = GV[0] * T[c] + GV[1] * T[3 + c];
+    GVT[3 + c] = GV[2] * T[c] + GV[3] * T[3 + c];
+  }
+  float dSig[9];
+#pragma unroll
+  for (int r = 0; r < 3; ++r)
+#pragma unroll
+    for (int c = 0; c < 3; ++c) dSig[3 * r + c] = T[r] * GVT[c] + T[3 + r] * GVT[3 + c];
+  float dT[6];
+#pragma unroll
+  for (int r = 0; r < 2; ++r)
+#pragma unroll
+    for (int c = 0; c < 3; ++c)
+      dT[3 * r + c] = 2.f * (GVT[3 * r] * Sig[c] + GVT[3 * r + 1] * Sig[3 + c] + GVT[3 * r + 2] * Sig[6 + c]);
+  // T = J W -> dJ = dT W^T; only J00, J02, J11, J12 depend on p_c
+  float dJ[6];
+#pragma unroll
+  for (int r = 0; r < 2; ++r)
+#pragma unroll
+    for (int c = 0; c < 3; ++c)
+      dJ[3 * r + c] = dT[3 * r] * cam.R[3 * c] + dT[3 * r + 1] * cam.R[3 * c + 1] + dT[3 * r + 2] * cam.R[3 * c + 2];
+  float dX = dJ[2] * (-cam.fx * iz2);
+  float dY = dJ[5] * (-cam.fy * iz2);
+  float dZ = dJ[0] * (-cam.fx * iz2) + dJ[2] * (2.f * cam.fx * X * iz2 * iz) +
+             dJ[4] * (-cam.fy * iz2) + dJ[5] * (2.f * cam.fy * Y * iz2 * iz);
+  // projected mean
+  dX += d_u * jx;
+  dY += d_v * jy;
+  dZ += d_u * jxz + d_v * jyz;
+  float dp[3];
+#pragma unroll
+  for (int c = 0; c < 3; ++c) dp[c] = cam.R[c] * dX + cam.R[3 + c] * dY + cam.R[6 + c] * dZ;
+
+  // Sigma = M M^T -> dM = 2 dSigma M (dSigma symmetric)
+  float dM[9];
+#pragma unroll
+  for (int r = 0; r < 3; ++r)
+#pragma unroll
+    for (int c = 0; c < 3; ++c)
+      dM[3 * r + c] = 2.f * (dSig[3 * r] * M[c] + dSig[3 * r + 1] * M[3 + c] + dSig[3 * r + 2] * M[6 + c]);
+  float dls[3];
+#pragma unroll
+  for (int c = 0; c < 3; ++c)
+    dls[c] = (dM[c] * Rq[c] + dM[3 + c] * Rq[3 + c] + dM[6 + c] * Rq[6 + c]) * s[c];
+  float G[9];  // dL/dR = dM diag(s)
+#pragma unroll
+  for (int r = 0; r < 3; ++r)
+#pragma unroll
+    for (int c = 0; c < 3; ++c) G[3 * r + c] = dM[3 * r + c] * s[c];
+  const float gw = 2.f * (-z * G[1] + y * G[2] + z * G[3] - x * G[5] - y * G[6] + x * G[7]);
+  const float gx = 2.f * (y * G[1] + z * G[2] + y * G[3] - 2.f * x * G[4] - w * G[5] + z * G[6] +
+                          w * G[7] - 2.f * x * G[8]);
+  const float gy = 2.f * (-2.f * y * G[0] + x * G[1] + w * G[2] + x * G[3] + z * G[5] - w * G[6] +
+                          z * G[7] - 2.f * y * G[8]);
+  const float gz = 2.f * (-2.f * z * G[0] - w * G[1] + x * G[2] + w * G[3] - 2.f * z * G[4] +
+                          y * G[5] + x * G[6] + y * G[7]);
+  const float qdot = w * gw + x * gx + y * gy + z * gz;
+  const float dq[4] = {(gw - w * qdot) * iqn, (gx - x * qdot) * iqn, (gy - y * qdot) * iqn,
+                       (gz - z * qdot) * iqn};
+
+  // Colour: SH coefficients and the view-direction path into the position.
+  float dv[3] = {p[0] - cam.campos[0], p[1] - cam.campos[1], p[2] - cam.campos[2]};
+  const float dlen = sqrtf(dv[0] * dv[0] + dv[1] * dv[1] + dv[2] * dv[2]);
+  const float idl = 1.0f / dlen;
+  const float vx = dv[0] * idl, vy = dv[1] * idl, vz = dv[2] * idl;
+  float Yk[16];
+  sh_basis(a.active_degree, vx, vy, vz, Yk);
+  const int nk = (a.active_degree + 1) * (a.active_degree + 1);
+  float wsum[16];
+#pragma unroll
+  for (int k = 0; k < 16; ++k) wsum[k] = 0.f;
+#pragma unroll
+  for (int ch = 0; ch < 3; ++ch) {
+    if (drgb[ch] == 0.f) continue;
+    const float* shc = a.sh + static_cast<int64_t>(ch) * a.sh_k * np + i;
+    float* gsh = a.g_sh + static_cast<int64_t>(ch) * a.sh_k * np + i;
+    for (int k = 0; k < nk; ++k) {
+      gsh[static_cast<int64_t>(k) * np] += drgb[ch] * Yk[k];
+      wsum[k] += drgb[ch] * shc[static_cast<int64_t>(k) * np];
+    }
+  }
+  float gvx, gvy, gvz;
+  sh_grad_dir(a.active_degree, vx, vy, vz, wsum, gvx, gvy, gvz);
+  const float vdot = vx * gvx + vy * gvy + vz * gvz;
+  dp[0] += (gvx - vx * vdot) * idl;
+  dp[1] += (gvy - vy * vdot) * idl;
+  dp[2] += (gvz - vz * vdot) * idl;
+
+  a.g_means[i] += dp[0];
+  a.g_means[np + i] += dp[1];
+  a.g_means[2 * np + i] += dp[2];
+  a.g_log_scales[i] += dls[0];
+  a.g_log_scales[np + i] += dls[1];
+  a.g_log_scales[2 * np + i] += dls[2];
+#pragma unroll
+  for (int c = 0; c < 4; ++c) a.g_quats[c * np + i] += dq[c];
+  a.g_opacity_logits[i] += d_o * o * (1.f - o);
+}
+
+// Natural screen-space gradient from the raw sums (for stage checks).
+__global__ void screen_grads_kernel(const Screen* screen, const float* sgrad, int64_t n, float* out) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const float* r = sgrad + i * kGradStride;
+  const Screen s = screen[i];
+  const float A = s.a.z, B = s.a.w, C = s.b.x, o = s.b.y;
+  float* d = out + i * 9;
+  d[0] = A * r[1] + B * r[2];
+  d[1] = B * r[1] + C * r[2];
+  d[2] = -0.5f * r[3];
+  d[3] = -r[4];
+  d[4] = -0.5f * r[5];
+  d[5] = o > 0.f ? r[0] / o : 0.f;
+  d[6] = r[6];
+  d[7] = r[7];
+  d[8] = r[8];
+}
+
+}  // namespace
+
+cudaError_t launch_preprocess_backward(const PreprocessBwdArgs& a, cudaStream_t st) {
+  if (a.n == 0) return cudaSuccess;
+  preprocess_backward_kernel<<<static_cast<unsigned>((a.n + 255) / 256), 256, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_screen_grads(const Screen* screen, const float* sgrad, int64_t n, float* out,
+                                cudaStream_t st) {
+  if (n == 0) return cudaSuccess;
+  screen_grads_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(screen, sgrad, n, out);
+  return cudaGetLastError();
+}
+
+}  // namespace gs

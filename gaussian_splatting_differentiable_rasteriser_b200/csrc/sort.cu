@@ -1,0 +1,340 @@
+// Tile lists: duplicate one (tile | depth) key per touched tile, sort the keys
+// with a stable LSD onesweep radix sort, extract per-tile ranges.
+//
+// Method: "How a computer rebuilds a real place ... Gaussian Splats"
+// (taosengine.com), section "Why tiling, and the five stages": count -> scan
+// -> scatter -> sort by depth within each tile, equal keys broken by the
+// smaller id; each tile's range closes where the next tile begins.
+//
+// Design (B200): instead of a per-tile bitonic network, all entries are sorted
+// at once by a single 64-bit key
+//     key = tile << depth_bits | (float_bits(depth) - depth_min)
+// where depth_bits is the bit length of the visible depth-key range. Positive
+// float32 bit patterns order like the floats, and subtracting the minimum
+// keeps that order, so the key orders entries by (tile, depth) exactly while
+// needing only ceil((tile_bits + depth_bits) / 8) passes (typically 5 at
+// 1080p, not 8). Entries are emitted in Gaussian-index order and every pass
+// is stable, so equal keys stay in index order: the tie-break needs no bits.
+//
+// Each onesweep pass reads and writes every entry once (12 B in, 12 B out):
+// a CTA ranks 4096 keys in shared memory (warp match + per-warp digit
+// counters), publishes its digit counts, obtains the exclusive prefix of all
+// earlier CTAs by a decoupled look-back whose every wait is bounded, and
+// scatters through shared memory so the global writes are runs of consecutive
+// addresses.
+#include <algorithm>
+
+#include "gs_kernels.cuh"
+
+namespace gs {
+
+namespace {
+
+constexpr uint32_t kFlagAggregate = 1u << 30;
+constexpr uint32_t kFlagPrefix = 2u << 30;
+constexpr uint32_t kValueMask = (1u << 30) - 1u;
+constexpr int kLookbackSpinLimit = 1 << 22;
+
+__device__ __forceinline__ uint32_t ld_relaxed(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_relaxed(uint32_t* p, uint32_t v) {
+  asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// ------------------------------------------------------------- duplicate --
+__global__ void __launch_bounds__(256) duplicate_kernel(DuplicateArgs a) {
+  __shared__ uint32_t s_warp[8];
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const uint32_t t = i < a.n ? a.touched[i] : 0u;
+  // exclusive scan of t inside the CTA
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t v = t;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    uint32_t n = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += n;
+  }
+  if (lane == 31) s_warp[warp] = v;
+  __syncthreads();
+  uint32_t before = 0;
+  for (int k = 0; k < warp; ++k) before += s_warp[k];
+  if (t == 0) return;
+  uint64_t off = a.block_prefix[blockIdx.x] + before + (v - t);
+  if (off + t > static_cast<uint64_t>(a.max_entries)) {
+    record_error(a.err, kErrIndexRange);
+    return;
+  }
+  const uint2 rc = a.rect[i];
+  const uint32_t x0 = rc.x & 0xffffu, x1 = rc.x >> 16, y0 = rc.y & 0xffffu, y1 = rc.y >> 16;
+  const uint64_t dk = static_cast<uint64_t>(__float_as_uint(a.depth[i]) - a.depth_min);
+  for (uint32_t y = y0; y <= y1; ++y)
+    for (uint32_t x = x0; x <= x1; ++x) {
+      const uint64_t tile = static_cast<uint64_t>(y) * a.tiles_x + x;
+      a.keys[off] = (tile << a.depth_bits) | dk;
+      a.vals[off] = static_cast<uint32_t>(i);
+      ++off;
+    }
+}
+
+// ------------------------------------------------------------- histogram --
+__global__ void __launch_bounds__(256) histogram_kernel(const uint64_t* keys, int64_t n,
+                                                        int passes, uint32_t* hist) {
+  __shared__ uint32_t s_hist[kMaxPasses][kRadix];
+  for (int k = threadIdx.x; k < kMaxPasses * kRadix; k += blockDim.x) (&s_hist[0][0])[k] = 0;
+  __syncthreads();
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += stride) {
+    const uint64_t key = keys[i];
+    for (int p = 0; p < passes; ++p) atomicAdd(&s_hist[p][(key >> (8 * p)) & 0xffu], 1u);
+  }
+  __syncthreads();
+  for (int p = 0; p < passes; ++p) {
+    const uint32_t c = s_hist[p][threadIdx.x];
+    if (c) atomicAdd(&hist[p * kRadix + threadIdx.x], c);
+  }
+}
+
+// Exclusive scan of each pass's digit histogram: one CTA of 256 per pass.
+__global__ void __launch_bounds__(256) digit_offsets_kernel(const uint32_t* hist, uint32_t* offsets) {
+  __shared__ uint32_t s_warp[8];
+  const int p = blockIdx.x, d = threadIdx.x, lane = d & 31, warp = d >> 5;
+  const uint32_t c = hist[p * kRadix + d];
+  uint32_t v = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    uint32_t n = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += n;
+  }
+  if (lane == 31) s_warp[warp] = v;
+  __syncthreads();
+  uint32_t before = 0;
+  for (int k = 0; k < warp; ++k) before += s_warp[k];
+  offsets[p * kRadix + d] = before + v - c;
+}
+
+// --------------------------------------------------------------- onesweep --
+struct OnesweepArgs {
+  const uint64_t* keys_in;
+  const uint32_t* vals_in;
+  uint64_t* keys_out;
+  uint32_t* vals_out;
+  int64_t n;
+  int shift;
+  const uint32_t* digit_offsets;  // [256] for this pass
+  uint32_t* status;               // [tiles][256] for this pass, zeroed
+  uint32_t* ticket;               // zeroed
+  uint32_t* err;
+};
+
+// Shared memory of one onesweep CTA (dynamic: above the 48 KB static limit).
+struct OnesweepSmem {
+  uint64_t keys[kSortTileKeys];
+  uint32_t vals[kSortTileKeys];
+  uint32_t whist[kSortThreads / 32][kRadix];  // per-warp digit counts, then offsets
+  uint32_t start[kRadix];  // first slot of each digit inside this CTA
+  uint32_t base[kRadix];   // first global slot of each digit for this CTA
+  uint32_t wsum[kSortThreads / 32];
+  uint32_t tile;
+};
+
+__global__ void __launch_bounds__(kSortThreads) onesweep_kernel(OnesweepArgs a) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  OnesweepSmem& sm = *reinterpret_cast<OnesweepSmem*>(smem_raw);
+  uint64_t* s_keys = sm.keys;
+  uint32_t* s_vals = sm.vals;
+  auto& s_whist = sm.whist;
+  uint32_t* s_start = sm.start;
+  uint32_t* s_base = sm.base;
+  uint32_t* s_wsum = sm.wsum;
+  uint32_t& s_tile = sm.tile;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) s_tile = atomicAdd(a.ticket, 1u);
+  for (int k = tid; k < (kSortThreads / 32) * kRadix; k += kSortThreads) (&s_whist[0][0])[k] = 0;
+  __syncthreads();
+  const uint32_t tile = s_tile;
+  const int64_t base = static_cast<int64_t>(tile) * kSortTileKeys;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+
+  // Load: warp w owns the 512 consecutive entries [base + 512 w, base + 512 (w + 1)),
+  // item j of lane l is entry 32 j + l of that run (coalesced).
+  uint64_t key[kSortItems];
+  uint32_t val[kSortItems];
+  uint32_t rank[kSortItems];
+#pragma unroll
+  for (int j = 0; j < kSortItems; ++j) {
+    const int64_t idx = base + warp * (kSortItems * 32) + j * 32 + lane;
+    if (idx < a.n) {
+      key[j] = a.keys_in[idx];
+      val[j] = a.vals_in[idx];
+    } else {
+      key[j] = ~0ull;
+      val[j] = 0u;
+    }
+  }
+  // Stable rank inside the warp: items in entry order, lanes in lane order.
+#pragma unroll
+  for (int j = 0; j < kSortItems; ++j) {
+    const int64_t idx = base + warp * (kSortItems * 32) + j * 32 + lane;
+    const bool valid = idx < a.n;
+    const uint32_t d = static_cast<uint32_t>(key[j] >> a.shift) & 0xffu;
+    const uint32_t peers = __match_any_sync(0xffffffffu, valid ? d : (0x100u | lane));
+    const uint32_t b = valid ? s_whist[warp][d] : 0u;
+    __syncwarp();
+    if (valid && lane == __ffs(peers) - 1) s_whist[warp][d] = b + __popc(peers);
+    __syncwarp();
+    rank[j] = b + __popc(peers & lt_mask);
+  }
+  __syncthreads();
+
+  // Per digit: exclusive offsets of each warp, and the CTA total.
+  const uint32_t d = tid;  // kSortThreads == kRadix
+  uint32_t count = 0;
+#pragma unroll
+  for (int w = 0; w < kSortThreads / 32; ++w) {
+    const uint32_t c = s_whist[w][d];
+    s_whist[w][d] = count;
+    count += c;
+  }
+  // Publish this CTA's count before anything else, so later CTAs can proceed.
+  uint32_t* st = a.status + static_cast<int64_t>(tile) * kRadix;
+  st_relaxed(&st[d], (tile == 0 ? kFlagPrefix : kFlagAggregate) | count);
+
+  // CTA-wide exclusive scan of the digit counts.
+  uint32_t v = count;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    uint32_t n = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += n;
+  }
+  if (lane == 31) s_wsum[warp] = v;
+  __syncthreads();
+  uint32_t before = 0;
+  for (int k = 0; k < warp; ++k) before += s_wsum[k];
+  s_start[d] = before + v - count;
+
+  // Decoupled look-back over earlier CTAs for this digit; every wait is bounded.
+  uint32_t excl = 0;
+  if (tile > 0) {
+    int64_t t = static_cast<int64_t>(tile) - 1;
+    int spins = 0;
+    while (t >= 0) {
+      const uint32_t s = ld_relaxed(&a.status[t * kRadix + d]);
+      const uint32_t flag = s & ~kValueMask;
+      if (flag == 0u) {
+        if (++spins > kLookbackSpinLimit) {
+          record_error(a.err, kErrLookbackTimeout);
+          break;
+        }
+        __nanosleep(64);
+        continue;
+      }
+      excl += s & kValueMask;
+      if (flag == kFlagPrefix) break;
+      --t;
+    }
+    st_relaxed(&st[d], kFlagPrefix | (excl + count));
+  }
+  s_base[d] = a.digit_offsets[d] + excl;
+  __syncthreads();
+
+  // Scatter into shared memory in digit order, then out in runs.
+#pragma unroll
+  for (int j = 0; j < kSortItems; ++j) {
+    const int64_t idx = base + warp * (kSortItems * 32) + j * 32 + lane;
+    if (idx < a.n) {
+      const uint32_t dj = static_cast<uint32_t>(key[j] >> a.shift) & 0xffu;
+      const uint32_t pos = s_start[dj] + s_whist[warp][dj] + rank[j];
+      if (pos >= static_cast<uint32_t>(kSortTileKeys)) {
+        record_error(a.err, kErrIndexRange);
+        continue;
+      }
+      s_keys[pos] = key[j];
+      s_vals[pos] = val[j];
+    }
+  }
+  __syncthreads();
+  const int64_t rem = a.n - base;
+  const int tile_n = rem < kSortTileKeys ? static_cast<int>(rem) : kSortTileKeys;
+  for (int k = tid; k < tile_n; k += kSortThreads) {
+    const uint64_t kk = s_keys[k];
+    const uint32_t dk = static_cast<uint32_t>(kk >> a.shift) & 0xffu;
+    const int64_t dst = static_cast<int64_t>(s_base[dk]) + (k - static_cast<int64_t>(s_start[dk]));
+    if (dst < 0 || dst >= a.n) {
+      record_error(a.err, kErrIndexRange);
+      continue;
+    }
+    a.keys_out[dst] = kk;
+    a.vals_out[dst] = s_vals[k];
+  }
+}
+
+// ------------------------------------------------------------------ ranges --
+__global__ void __launch_bounds__(256) ranges_kernel(const uint64_t* keys, int64_t n, int depth_bits,
+                                                     uint2* ranges, int64_t num_tiles) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const uint64_t tile = keys[i] >> depth_bits;
+  if (tile >= static_cast<uint64_t>(num_tiles)) return;
+  if (i == 0 || (keys[i - 1] >> depth_bits) != tile) ranges[tile].x = static_cast<uint32_t>(i);
+  if (i == n - 1 || (keys[i + 1] >> depth_bits) != tile) ranges[tile].y = static_cast<uint32_t>(i + 1);
+}
+
+}  // namespace
+
+cudaError_t launch_duplicate(const DuplicateArgs& a, int64_t num_blocks, cudaStream_t st) {
+  if (num_blocks == 0) return cudaSuccess;
+  duplicate_kernel<<<static_cast<unsigned>(num_blocks), 256, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_sort(const SortPlan& plan, const SortBuffers& b, int* out_buf, cudaStream_t st) {
+  *out_buf = 0;
+  if (plan.n <= 1 || plan.passes == 0) return cudaSuccess;
+  cudaError_t e;
+  if ((e = cudaMemsetAsync(b.hist, 0, sizeof(uint32_t) * kMaxPasses * kRadix, st)) != cudaSuccess) return e;
+  if ((e = cudaMemsetAsync(b.counters, 0, sizeof(uint32_t) * kMaxPasses, st)) != cudaSuccess) return e;
+  if ((e = cudaMemsetAsync(b.status, 0, sizeof(uint32_t) * kRadix * plan.tiles * plan.passes, st)) !=
+      cudaSuccess)
+    return e;
+  if ((e = cudaFuncSetAttribute(onesweep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(sizeof(OnesweepSmem)))) != cudaSuccess)
+    return e;
+  int hist_blocks = static_cast<int>(std::min<int64_t>((plan.n + 4095) / 4096, 148 * 4));
+  histogram_kernel<<<hist_blocks, 256, 0, st>>>(b.keys[0], plan.n, plan.passes, b.hist);
+  digit_offsets_kernel<<<plan.passes, 256, 0, st>>>(b.hist, b.offsets);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  int cur = 0;
+  for (int p = 0; p < plan.passes; ++p) {
+    OnesweepArgs o;
+    o.keys_in = b.keys[cur];
+    o.vals_in = b.vals[cur];
+    o.keys_out = b.keys[cur ^ 1];
+    o.vals_out = b.vals[cur ^ 1];
+    o.n = plan.n;
+    o.shift = 8 * p;
+    o.digit_offsets = b.offsets + p * kRadix;
+    o.status = b.status + static_cast<int64_t>(p) * plan.tiles * kRadix;
+    o.ticket = b.counters + p;
+    o.err = b.err;
+    onesweep_kernel<<<static_cast<unsigned>(plan.tiles), kSortThreads, sizeof(OnesweepSmem), st>>>(o);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    cur ^= 1;
+  }
+  *out_buf = cur;
+  return cudaSuccess;
+}
+
+cudaError_t launch_ranges(const uint64_t* keys, int64_t n, int depth_bits, uint2* ranges,
+                          int64_t num_tiles, cudaStream_t st) {
+  cudaError_t e = cudaMemsetAsync(ranges, 0, sizeof(uint2) * num_tiles, st);
+  if (e != cudaSuccess || n == 0) return e;
+  ranges_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(keys, n, depth_bits, ranges,
+                                                                        num_tiles);
+  return cudaGetLastError();
+}
+
+}  // namespace gs

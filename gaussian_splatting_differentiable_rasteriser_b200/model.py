@@ -1,0 +1,110 @@
+"""Device-resident Gaussian parameters and one training step through the C ABI.
+
+Holds the parameters, their gradients and the two Adam moments as four flat
+float32 buffers with one planar view per group (so each group's start is
+16-byte aligned and Adam streams it with float4 accesses), and sequences the
+five entry points of one iteration: preprocess -> render_forward ->
+loss_l1_dssim -> render_backward -> adam_step (once per group, each with its
+own learning rate, as "Differentiable rasterisation" (splat-report), section
+"From a pixel error back to a quaternion", describes).
+"""
+from __future__ import annotations
+
+import torch
+
+from . import native
+from .scenes import GROUP_NAMES
+
+
+def group_shapes(n_pad: int, sh_degree: int) -> dict:
+    K = (sh_degree + 1) ** 2
+    return {"means": (3, n_pad), "log_scales": (3, n_pad), "quats": (4, n_pad),
+            "opacity_logits": (n_pad,), "sh": (3, K, n_pad)}
+
+
+class GaussianModel:
+    def __init__(self, scene, device="cuda", active_degree=None):
+        self.n, self.n_pad, self.sh_degree = scene.n, scene.n_pad, scene.sh_degree
+        self.active_degree = scene.sh_degree if active_degree is None else active_degree
+        shapes = group_shapes(self.n_pad, self.sh_degree)
+        sizes = {k: int(torch.Size(s).numel()) for k, s in shapes.items()}
+        total = sum(sizes.values())
+        self.flat = torch.empty(total, dtype=torch.float32, device=device)
+        self.grad_flat = torch.zeros(total, dtype=torch.float32, device=device)
+        self.m_flat = torch.zeros(total, dtype=torch.float32, device=device)
+        self.v_flat = torch.zeros(total, dtype=torch.float32, device=device)
+        self.params, self.grads, self.m, self.v, self.slices = {}, {}, {}, {}, {}
+        off = 0
+        for k in GROUP_NAMES:
+            sl = slice(off, off + sizes[k])
+            self.slices[k] = sl
+            self.params[k] = self.flat[sl].view(shapes[k])
+            self.grads[k] = self.grad_flat[sl].view(shapes[k])
+            self.m[k] = self.m_flat[sl].view(shapes[k])
+            self.v[k] = self.v_flat[sl].view(shapes[k])
+            off += sizes[k]
+        self.load(scene)
+        self.step_count = 0
+
+    def load(self, scene):
+        for k in GROUP_NAMES:
+            self.params[k].copy_(torch.from_numpy(getattr(scene, k)).to(torch.float32))
+
+    def params_struct(self) -> native.GsParams:
+        p = native.GsParams()
+        for k in GROUP_NAMES:
+            setattr(p, k, self.params[k].data_ptr())
+        p.n, p.n_pad = self.n, self.n_pad
+        p.sh_degree, p.active_degree = self.sh_degree, self.active_degree
+        return p
+
+    def grads_struct(self) -> native.GsGrads:
+        g = native.GsGrads()
+        for k in GROUP_NAMES:
+            setattr(g, k, self.grads[k].data_ptr())
+        return g
+
+
+DEFAULT_LR = {k: 1e-3 for k in GROUP_NAMES}
+
+
+class TrainStep:
+    """Buffers and the call sequence of one iteration for images up to width x height."""
+
+    def __init__(self, model: GaussianModel, max_entries: int, width: int, height: int, lrs=None,
+                 lam=0.2, betas=(0.9, 0.999), eps=1e-8, device="cuda"):
+        self.model = model
+        self.ctx = native.Context(model.n_pad, max_entries, width, height)
+        self.lrs = dict(DEFAULT_LR if lrs is None else lrs)
+        self.lam, self.betas, self.eps = lam, betas, eps
+        self.image = torch.empty((3, height, width), dtype=torch.float32, device=device)
+        self.final_T = torch.empty((height, width), dtype=torch.float32, device=device)
+        self.n_contrib = torch.empty((height, width), dtype=torch.int32, device=device)
+        self.dimage = torch.empty((3, height, width), dtype=torch.float32, device=device)
+        self.loss = torch.zeros(3, dtype=torch.float64, device=device)
+        self.last_entries = 0
+
+    def forward(self, cam_struct, H, W):
+        p = self.model.params_struct()
+        self.ctx.preprocess(p, cam_struct)
+        img, T, nc = self.image[:, :H, :W], self.final_T[:H, :W], self.n_contrib[:H, :W]
+        if H != self.image.shape[1] or W != self.image.shape[2]:
+            img = torch.empty((3, H, W), dtype=torch.float32, device=self.image.device)
+            T = torch.empty((H, W), dtype=torch.float32, device=self.image.device)
+            nc = torch.empty((H, W), dtype=torch.int32, device=self.image.device)
+        self.last_entries = self.ctx.render_forward(cam_struct, img, T, nc)
+        return img, T, nc
+
+    def __call__(self, cam, target):
+        """One iteration against `target` ([3, H, W] float32 on the device)."""
+        cs = native.camera_struct(cam)
+        H, W = cam.height, cam.width
+        img, T, nc = self.forward(cs, H, W)
+        dimg = self.dimage if img.shape == self.dimage.shape else torch.empty_like(img)
+        self.ctx.loss_l1_dssim(img, target, self.lam, self.loss, dimg)
+        self.ctx.render_backward(self.model.params_struct(), cs, T, nc, dimg, self.model.grads_struct())
+        self.model.step_count += 1
+        for k in GROUP_NAMES:
+            native.adam_step(self.model.params[k], self.model.grads[k], self.model.m[k], self.model.v[k],
+                             self.lrs[k], self.model.step_count, self.betas[0], self.betas[1], self.eps)
+        return self.loss

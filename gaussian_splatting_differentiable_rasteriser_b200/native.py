@@ -1,0 +1,196 @@
+"""ctypes binding of the C ABI in include/gs_api.h.
+
+Argument marshalling only: tensors become device pointers, the current torch
+stream becomes the `stream` argument, and a non-OK status becomes an
+exception carrying gs_last_error(). Every step of the path runs in the CUDA
+library; there is no fallback of any kind, so a missing or unloadable library
+raises immediately.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libgsb200.so")
+
+GS_OK, GS_ERR_INVALID_ARG, GS_ERR_CAPACITY, GS_ERR_CUDA, GS_ERR_DEVICE = range(5)
+_STATUS = {0: "GS_OK", 1: "GS_ERR_INVALID_ARG", 2: "GS_ERR_CAPACITY", 3: "GS_ERR_CUDA",
+           4: "GS_ERR_DEVICE"}
+
+EXPORTED = ("gs_create", "gs_destroy", "gs_last_error", "gs_preprocess", "gs_render_forward",
+            "gs_loss_l1_dssim", "gs_render_backward", "gs_adam_step", "gs_profile_enable",
+            "gs_profile_read", "gs_stage_name", "gs_debug_preprocess", "gs_debug_sorted",
+            "gs_debug_screen_grads")
+STAGES = ("preprocess", "scan", "duplicate", "sort", "ranges", "blend_forward", "loss",
+          "blend_backward", "preprocess_backward")
+
+
+class GsError(RuntimeError):
+    def __init__(self, status, msg):
+        super().__init__(f"{_STATUS.get(status, status)}: {msg}")
+        self.status = status
+
+
+class GsCamera(ctypes.Structure):
+    _fields_ = [("width", ctypes.c_int32), ("height", ctypes.c_int32),
+                ("fx", ctypes.c_float), ("fy", ctypes.c_float),
+                ("cx", ctypes.c_float), ("cy", ctypes.c_float),
+                ("R", ctypes.c_float * 9), ("t", ctypes.c_float * 3),
+                ("campos", ctypes.c_float * 3), ("bg", ctypes.c_float * 3),
+                ("near_z", ctypes.c_float)]
+
+
+class GsParams(ctypes.Structure):
+    _fields_ = [("means", ctypes.c_void_p), ("log_scales", ctypes.c_void_p),
+                ("quats", ctypes.c_void_p), ("opacity_logits", ctypes.c_void_p),
+                ("sh", ctypes.c_void_p), ("n", ctypes.c_int64), ("n_pad", ctypes.c_int64),
+                ("sh_degree", ctypes.c_int32), ("active_degree", ctypes.c_int32)]
+
+
+class GsGrads(ctypes.Structure):
+    _fields_ = [("means", ctypes.c_void_p), ("log_scales", ctypes.c_void_p),
+                ("quats", ctypes.c_void_p), ("opacity_logits", ctypes.c_void_p),
+                ("sh", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH):
+    """Loads the CUDA library (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"CUDA library not built: {path} is missing (run __graft_entry__.build())")
+    L = ctypes.CDLL(path)
+    P, I32, I64, F = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float
+    L.gs_create.argtypes = [ctypes.POINTER(P), I64, I64, I32, I32]
+    L.gs_destroy.argtypes = [P]
+    L.gs_destroy.restype = None
+    L.gs_last_error.argtypes = [P]
+    L.gs_last_error.restype = ctypes.c_char_p
+    L.gs_preprocess.argtypes = [P, ctypes.POINTER(GsParams), ctypes.POINTER(GsCamera), P]
+    L.gs_render_forward.argtypes = [P, ctypes.POINTER(GsCamera), P, P, P, ctypes.POINTER(I64), P]
+    L.gs_loss_l1_dssim.argtypes = [P, P, P, I32, I32, F, P, P, P]
+    L.gs_render_backward.argtypes = [P, ctypes.POINTER(GsParams), ctypes.POINTER(GsCamera), P, P, P,
+                                     ctypes.POINTER(GsGrads), P]
+    L.gs_adam_step.argtypes = [P, P, P, P, I64, F, F, F, F, I32, P]
+    L.gs_profile_enable.argtypes = [P, I32]
+    L.gs_profile_read.argtypes = [P, P, P, P]
+    L.gs_stage_name.argtypes = [I32]
+    L.gs_stage_name.restype = ctypes.c_char_p
+    L.gs_debug_preprocess.argtypes = [P] * 10
+    L.gs_debug_sorted.argtypes = [P] * 5
+    L.gs_debug_screen_grads.argtypes = [P] * 3
+    for name in EXPORTED:
+        if name not in ("gs_destroy", "gs_last_error", "gs_stage_name"):
+            getattr(L, name).restype = ctypes.c_int
+    _lib = L
+    return L
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def camera_struct(cam) -> GsCamera:
+    c = GsCamera()
+    c.width, c.height = int(cam.width), int(cam.height)
+    c.fx, c.fy, c.cx, c.cy = float(cam.fx), float(cam.fy), float(cam.cx), float(cam.cy)
+    for i, v in enumerate(np.asarray(cam.R, np.float32).reshape(-1)):
+        c.R[i] = float(v)
+    for name in ("t", "campos", "bg"):
+        arr = getattr(c, name)
+        for i, v in enumerate(np.asarray(getattr(cam, name), np.float32).reshape(-1)):
+            arr[i] = float(v)
+    c.near_z = float(cam.near_z)
+    return c
+
+
+class Context:
+    """Owns one gs_ctx; methods mirror the C entry points one to one."""
+
+    def __init__(self, max_gaussians, max_entries, max_width, max_height):
+        self.L = load()
+        h = ctypes.c_void_p()
+        st = self.L.gs_create(ctypes.byref(h), int(max_gaussians), int(max_entries), int(max_width),
+                              int(max_height))
+        if st != GS_OK:
+            raise GsError(st, "gs_create failed")
+        self.h = h
+
+    def close(self):
+        if getattr(self, "h", None):
+            self.L.gs_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def _check(self, st):
+        if st != GS_OK:
+            raise GsError(st, self.L.gs_last_error(self.h).decode())
+
+    def preprocess(self, params: GsParams, cam: GsCamera, stream=None):
+        self._check(self.L.gs_preprocess(self.h, ctypes.byref(params), ctypes.byref(cam), _stream(stream)))
+
+    def render_forward(self, cam: GsCamera, image, final_T, n_contrib, stream=None) -> int:
+        k = ctypes.c_int64(0)
+        self._check(self.L.gs_render_forward(self.h, ctypes.byref(cam), _ptr(image), _ptr(final_T),
+                                             _ptr(n_contrib), ctypes.byref(k), _stream(stream)))
+        return k.value
+
+    def loss_l1_dssim(self, image, target, lam, loss_out, dloss_dimage=None, stream=None):
+        _, H, W = image.shape
+        self._check(self.L.gs_loss_l1_dssim(self.h, _ptr(image), _ptr(target), H, W, float(lam),
+                                            _ptr(loss_out), _ptr(dloss_dimage), _stream(stream)))
+
+    def render_backward(self, params: GsParams, cam: GsCamera, final_T, n_contrib, dloss_dimage,
+                        grads: GsGrads, stream=None):
+        self._check(self.L.gs_render_backward(self.h, ctypes.byref(params), ctypes.byref(cam),
+                                              _ptr(final_T), _ptr(n_contrib), _ptr(dloss_dimage),
+                                              ctypes.byref(grads), _stream(stream)))
+
+    def profile_enable(self, on=True):
+        self._check(self.L.gs_profile_enable(self.h, 1 if on else 0))
+
+    def profile_read(self) -> dict:
+        n = len(STAGES)
+        ms = (ctypes.c_double * n)()
+        launches = (ctypes.c_int64 * n)()
+        work = (ctypes.c_int64 * n)()
+        self._check(self.L.gs_profile_read(self.h, ms, launches, work))
+        return {STAGES[k]: {"ms": ms[k], "launches": launches[k], "work": work[k]} for k in range(n)}
+
+    def debug_preprocess(self, mean2d=None, conic=None, opacity=None, rgb=None, depth=None, rect=None,
+                         touched=None, clamped=None, stream=None):
+        self._check(self.L.gs_debug_preprocess(self.h, _ptr(mean2d), _ptr(conic), _ptr(opacity),
+                                               _ptr(rgb), _ptr(depth), _ptr(rect), _ptr(touched),
+                                               _ptr(clamped), _stream(stream)))
+
+    def debug_sorted(self, ids=None, tiles=None, ranges=None, stream=None):
+        self._check(self.L.gs_debug_sorted(self.h, _ptr(ids), _ptr(tiles), _ptr(ranges), _stream(stream)))
+
+    def debug_screen_grads(self, out, stream=None):
+        self._check(self.L.gs_debug_screen_grads(self.h, _ptr(out), _stream(stream)))
+
+
+def adam_step(param, grad, m, v, lr, step, beta1=0.9, beta2=0.999, eps=1e-8, stream=None):
+    L = load()
+    st = L.gs_adam_step(_ptr(param), _ptr(grad), _ptr(m), _ptr(v), param.numel(), float(lr),
+                        float(beta1), float(beta2), float(eps), int(step), _stream(stream))
+    if st != GS_OK:
+        raise GsError(st, "gs_adam_step rejected its arguments")

@@ -1,0 +1,230 @@
+/*
+ * gs_api.h - C ABI of the B200 (sm_100a) differentiable tile-based
+ * Gaussian-splat rasteriser: preprocess, tile sort + forward blend, fused
+ * L1 + D-SSIM loss, blend + projection backward, and a fused Adam step.
+ *
+ * Conventions shared by every call
+ *   - Every data pointer is a DEVICE pointer owned by the caller, unless the
+ *     argument says "host". Buffers are never freed or retained by the library
+ *     beyond the call, except the scratch a gs_ctx owns.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Work is enqueued asynchronously on it. gs_render_forward is the one call
+ *     that waits on the stream (it reads the entry count back to the host).
+ *   - Parameters are structure-of-arrays, planar float32, with n <= n_pad and
+ *     n_pad a multiple of 4, so every plane starts 16-byte aligned:
+ *         means           [3][n_pad]
+ *         log_scales      [3][n_pad]
+ *         quats           [4][n_pad]      (w, x, y, z), any non-zero length
+ *         opacity_logits  [n_pad]
+ *         sh              [3][(sh_degree+1)^2][n_pad]   k = 0 is the base RGB
+ *     Entries n .. n_pad-1 are ignored by the rasteriser (Adam still updates
+ *     them as ordinary scalars; with zero gradient they do not move).
+ *   - Images are [3][height][width] float32 (channel-major, row-major);
+ *     per-pixel maps are [height][width].
+ *   - Pixel (i, j) sits at continuous coordinate (i, j). Camera axes: x right,
+ *     y down, z forward; p_cam = R p_world + t.
+ *   - Every call returns a gs_status. Argument and size errors are detected on
+ *     the host before anything is enqueued (GS_ERR_INVALID_ARG). A failed CUDA
+ *     launch returns GS_ERR_CUDA. A fault recorded by a kernel's own bounded
+ *     checks returns GS_ERR_DEVICE. No kernel traps or waits without bound.
+ *     gs_last_error() gives a one-line description of the last failure.
+ *
+ * Citations name the web pages this method is described on:
+ *   [DR]  "Differentiable rasterisation" (splat-report.pages.dev).
+ *   [TBR] "Tile-based differentiable rasterization in 3DGS"
+ *         (learn-ml-visualized-interactive).
+ *   [SN]  Gaussian splatting training study notes (bailiping.com).
+ *   [GS]  "How a computer rebuilds a real place out of soft colored dots
+ *         called Gaussian Splats" (taosengine.com).
+ */
+#ifndef GS_API_H
+#define GS_API_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  GS_OK = 0,
+  GS_ERR_INVALID_ARG = 1, /* bad pointer, size, order of calls or capacity request */
+  GS_ERR_CAPACITY = 2,    /* more (Gaussian, tile) entries than the context holds */
+  GS_ERR_CUDA = 3,        /* a CUDA API call or kernel launch failed */
+  GS_ERR_DEVICE = 4       /* a kernel's bounded self-check recorded a fault */
+} gs_status;
+
+/* Pinhole camera (host struct, passed by pointer, copied by value). */
+typedef struct {
+  int32_t width, height;
+  float fx, fy, cx, cy;
+  float R[9];      /* world -> camera rotation, row-major */
+  float t[3];      /* p_cam = R p_world + t */
+  float campos[3]; /* camera centre in world space; origin of the view direction */
+  float bg[3];     /* background colour */
+  float near_z;    /* Gaussians with camera depth <= near_z are culled */
+} gs_camera;
+
+/* Read-only parameters (host struct holding device pointers). */
+typedef struct {
+  const float *means, *log_scales, *quats, *opacity_logits, *sh;
+  int64_t n, n_pad;
+  int32_t sh_degree;     /* storage degree, 0..3 */
+  int32_t active_degree; /* bands used for colour, 0..sh_degree */
+} gs_params;
+
+/* Parameter gradients, same layout as gs_params. gs_render_backward ADDS
+ * into them (several views may be accumulated); gs_adam_step zeroes them. */
+typedef struct {
+  float *means, *log_scales, *quats, *opacity_logits, *sh;
+} gs_grads;
+
+/* Opaque context. It owns the scratch of one camera in flight: per-Gaussian
+ * screen state, sort keys and values (double-buffered), per-tile ranges,
+ * per-Gaussian screen-space gradients and the loss partial sums. */
+typedef struct gs_ctx gs_ctx;
+
+/* Allocates a context for up to max_gaussians Gaussians, max_entries
+ * (Gaussian, tile) entries and images up to max_width x max_height.
+ * The entry budget mirrors the global (blob, tile) budget of [GS] section
+ * "Why tiling, and the five stages". The caller owns *ctx and frees it with
+ * gs_destroy. Returns GS_ERR_INVALID_ARG for non-positive sizes and
+ * GS_ERR_CUDA if device memory cannot be allocated (nothing is leaked). */
+gs_status gs_create(gs_ctx **ctx, int64_t max_gaussians, int64_t max_entries,
+                    int32_t max_width, int32_t max_height);
+void gs_destroy(gs_ctx *ctx);
+/* Human-readable description of the last failure on this context ("" if none).
+ * The string is owned by the context. */
+const char *gs_last_error(const gs_ctx *ctx);
+
+/* Step 1 - preprocess, one thread per Gaussian ([SN] slides on the
+ * parametrisation and "J is the 2 x 3 Jacobian of perspective projection";
+ * [GS] sections "Flattening a 3D blob into a 2D oval (EWA projection)" and
+ * "Spherical harmonics: color that changes with viewing angle"):
+ * p_c = R p + t; cull if Z <= near_z; Sigma = R(q/|q|) S S^T R^T with
+ * S = diag(exp(log_scales)); Sigma' = J W Sigma W^T J^T + 0.3 I with
+ * J = [fx/Z, 0, -fx X/Z^2; 0, fy/Z, -fy Y/Z^2]; conic = Sigma'^-1; mean2d;
+ * radius 3 sqrt(lambda_max(Sigma')); rect of the 16x16 tiles meeting
+ * mean2d +- radius; opacity = sigmoid(logit); colour = max(0, sum_k sh_k Y_k(v))
+ * at v = normalize(p - campos) using bands up to active_degree.
+ * The geometry is evaluated in float64 (depth key = float32(Z)), the colour in
+ * float32. Results stay in the context for gs_render_forward/backward.
+ * Errors: GS_ERR_INVALID_ARG if n > max_gaussians, n_pad < n, n_pad % 4 != 0,
+ * a degree is out of range, a pointer is NULL or misaligned, or the camera is
+ * larger than the context's maximum image. */
+gs_status gs_preprocess(gs_ctx *ctx, const gs_params *params, const gs_camera *cam, void *stream);
+
+/* Step 2 - tile lists and forward blend ([GS] sections "Why tiling, and the
+ * five stages" and "The painting itself: front-to-back alpha compositing";
+ * [DR] section "The trick: recompute the blend state instead of storing it";
+ * [SN] slide on alpha and the background term).
+ * Duplicates one 64-bit key (tile | depth) with the Gaussian index as value
+ * per touched tile (prefix sum over tiles_touched), sorts them with a stable
+ * LSD onesweep radix sort (order = tile, depth, index), extracts per-tile
+ * ranges, then blends each 16x16 tile front to back:
+ * alpha = min(0.99, o exp(-e)), e = 1/2 (A dx^2 + C dy^2) + B dx dy, entries
+ * with alpha < 1/255 skipped, C += T alpha c, T *= 1 - alpha, and the walk
+ * stops after the entry that takes T below 1e-4. Writes
+ * image_chw = C + T bg, final_T = T, and n_contrib = 1 + list position of the
+ * last blended entry (0 if none). *num_entries_out (HOST pointer, may be
+ * NULL) receives the entry count. This call synchronises `stream` once to
+ * read the entry count. Errors: GS_ERR_INVALID_ARG if gs_preprocess has not
+ * run for this camera size; GS_ERR_CAPACITY (nothing written) if the entry
+ * count exceeds max_entries. */
+gs_status gs_render_forward(gs_ctx *ctx, const gs_camera *cam, float *image_chw, float *final_T,
+                            int32_t *n_contrib, int64_t *num_entries_out, void *stream);
+
+/* Step 3 - fused photometric loss ([SN] slides "An iteration samples a camera
+ * and differentiates its image loss", L1, and "11 x 11 Gaussian window,
+ * standard deviation 1.5 pixels"): L = (1 - lambda) L1 + lambda (1 - SSIM),
+ * L1 = mean |x - y| over 3HW, SSIM = mean over 3HW of the SSIM map with an
+ * 11x11 Gaussian window (sigma 1.5), C1 = 0.01^2, C2 = 0.03^2 and zero padding.
+ * Writes loss_out[0..2] = {L, L1, SSIM} (DEVICE pointer to 3 doubles; the
+ * reduction is deterministic) and, if dloss_dimage is not NULL, dL/dx with the
+ * L1 subgradient 0 at a zero residual. Works on any image up to the context's
+ * maximum size. Errors: GS_ERR_INVALID_ARG for bad sizes or pointers. */
+gs_status gs_loss_l1_dssim(gs_ctx *ctx, const float *image_chw, const float *target_chw,
+                           int32_t height, int32_t width, float lambda, double *loss_out,
+                           float *dloss_dimage, void *stream);
+
+/* Step 4 - backward ([DR] sections "The trick" and "From a pixel error back to
+ * a quaternion"; [GS] sections "The clever bit: a single backward sweep through
+ * the blend", "From a pixel's blame to the oval's shape and place", "The
+ * covariance chain", "Where the position gradient comes from"; [SN] slide
+ * "r is the RGB loss gradient"). Re-walks each tile back to front from each
+ * pixel's last contributor, recovering T by division by (1 - alpha), reduces
+ * the per-Gaussian screen gradients within each warp before the global
+ * atomics, then chains them through conic, Sigma', J, W, quaternion/scale,
+ * opacity and SH (including the view-direction path into the means).
+ * ADDS the result into *grads. `params` and `cam` must be the ones given to
+ * the last gs_preprocess, and final_T / n_contrib the outputs of the last
+ * gs_render_forward. Errors: GS_ERR_INVALID_ARG if the forward has not run
+ * or the inputs do not match it. Gradients are not bitwise reproducible
+ * (float32 atomics). */
+gs_status gs_render_backward(gs_ctx *ctx, const gs_params *params, const gs_camera *cam,
+                             const float *final_T, const int32_t *n_contrib,
+                             const float *dloss_dimage, gs_grads *grads, void *stream);
+
+/* Step 5 - fused Adam over one flat float32 buffer of `count` scalars
+ * ([GS] Adam paragraph after "Proving the blame is right"; [DR] per-group
+ * learning rates): m = b1 m + (1-b1) g; v = b2 v + (1-b2) g^2;
+ * p -= lr (m / (1 - b1^step)) / (sqrt(v / (1 - b2^step)) + eps); g = 0.
+ * step >= 1. Call once per parameter group to give each its own lr.
+ * Errors: GS_ERR_INVALID_ARG for NULL pointers, count < 0 or step < 1. */
+gs_status gs_adam_step(float *param, float *grad, float *m, float *v, int64_t count, float lr,
+                       float beta1, float beta2, float eps, int32_t step, void *stream);
+
+/* ------------------------------------------------------------ profiling --
+ * When enabled, every kernel launch a context makes is bracketed by CUDA
+ * events on the call's stream (a few microseconds of host time per launch;
+ * leave it off for throughput runs). gs_profile_read waits for the recorded
+ * events, returns per-stage totals accumulated since the previous read and
+ * resets them. Each output is a HOST array of GS_NUM_STAGES entries (any may
+ * be NULL): ms = summed kernel time, launches = launches, work = the units
+ * processed (Gaussians for the per-Gaussian stages, entries for the sort
+ * stages, evaluated (pixel, Gaussian) pairs for the blends, pixels for the
+ * loss). Adam takes no context and is not profiled here. */
+typedef enum {
+  GS_STAGE_PREPROCESS = 0,
+  GS_STAGE_SCAN = 1,
+  GS_STAGE_DUPLICATE = 2,
+  GS_STAGE_SORT = 3,
+  GS_STAGE_RANGES = 4,
+  GS_STAGE_BLEND_FORWARD = 5,
+  GS_STAGE_LOSS = 6,
+  GS_STAGE_BLEND_BACKWARD = 7,
+  GS_STAGE_PREPROCESS_BACKWARD = 8,
+  GS_NUM_STAGES = 9
+} gs_stage;
+
+gs_status gs_profile_enable(gs_ctx *ctx, int32_t enabled);
+gs_status gs_profile_read(gs_ctx *ctx, double *ms, int64_t *launches, int64_t *work);
+/* Static name of a stage ("preprocess", "sort", ...), or "" if out of range. */
+const char *gs_stage_name(int32_t stage);
+
+/* ---------------------------------------------------------------- debug --
+ * Copies of the context's internal state for stage-by-stage checks. Each
+ * output is a DEVICE pointer and may be NULL. Copies are asynchronous on
+ * `stream`. */
+
+/* After gs_preprocess, for the n Gaussians: mean2d [n][2], conic [n][3]
+ * (A, B, C), opacity [n], rgb [n][3], depth [n] (float32 camera Z),
+ * rect [n][4] (x0, y0, x1, y1 inclusive tile indices; x0 > x1 when culled),
+ * tiles_touched [n], clamped [n] (bit c set when colour channel c was
+ * clamped at 0). */
+gs_status gs_debug_preprocess(gs_ctx *ctx, float *mean2d, float *conic, float *opacity,
+                              float *rgb, float *depth, int32_t *rect, int32_t *tiles_touched,
+                              uint8_t *clamped, void *stream);
+/* After gs_render_forward: the sorted Gaussian index per entry [K], the tile
+ * per entry [K], and per-tile [lo, hi) ranges [tiles_y * tiles_x][2]. */
+gs_status gs_debug_sorted(gs_ctx *ctx, int32_t *ids, int32_t *tiles, int32_t *ranges,
+                          void *stream);
+/* After gs_render_backward: per-Gaussian screen-space gradient [n][9] =
+ * dL/d(mean2d x, mean2d y, A, B, C, opacity, r, g, b). */
+gs_status gs_debug_screen_grads(gs_ctx *ctx, float *out, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GS_API_H */

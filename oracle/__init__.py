@@ -46,6 +46,8 @@ def lib():
         L.or_get_sorted.argtypes = [P] * 4
         L.or_render.argtypes = [P] * 6
         L.or_render_pixels.argtypes = [P, ctypes.c_int64] + [P] * 6
+        L.or_render_rows.argtypes = [P, ctypes.c_int32, ctypes.c_int32] + [P] * 5
+        L.or_backward_rows.argtypes = [P, ctypes.c_int32, ctypes.c_int32] + [P] * 7
         L.or_backward.argtypes = [P] * 8
         L.or_loss.argtypes = [ctypes.c_int32, ctypes.c_int32, P, P, ctypes.c_double, P, P]
         L.or_loss.restype = ctypes.c_int
@@ -150,16 +152,29 @@ class Oracle:
                                 _p(out["n_contrib"]), _p(out["ambiguous"]))
         return out
 
-    def backward(self, dimage) -> dict:
+    def render_rows(self, y0, y1) -> dict:
+        H, W = self.cam.height, self.cam.width
+        out = dict(image=np.zeros((3, H, W)), final_T=np.zeros((H, W)),
+                   n_contrib=np.zeros((H, W), np.int32), ambiguous=np.zeros((H, W), np.uint8),
+                   stats=np.zeros(2, np.int64))
+        self.L.or_render_rows(self.h, int(y0), int(y1), *[_p(out[k]) for k in
+                                                           ("image", "final_T", "n_contrib",
+                                                            "ambiguous", "stats")])
+        return out
+
+    def backward(self, dimage, rows=None) -> dict:
+        """Parameter and screen gradients from dL/dimage; `rows` = (y0, y1)
+        restricts the walk to those pixel rows."""
         s = self.scene
         dimage = np.ascontiguousarray(dimage, np.float64)
         K = s.sh_k
         out = dict(screen=np.zeros((s.n, 9)), means=np.zeros((3, s.n_pad)),
                    log_scales=np.zeros((3, s.n_pad)), quats=np.zeros((4, s.n_pad)),
                    opacity_logits=np.zeros(s.n_pad), sh=np.zeros((3, K, s.n_pad)))
-        self.L.or_backward(self.h, _p(dimage), *[_p(out[k]) for k in
-                                                  ("screen", "means", "log_scales", "quats",
-                                                   "opacity_logits", "sh")])
+        y0, y1 = (0, self.cam.height) if rows is None else rows
+        self.L.or_backward_rows(self.h, int(y0), int(y1), _p(dimage),
+                                *[_p(out[k]) for k in ("screen", "means", "log_scales", "quats",
+                                                       "opacity_logits", "sh")])
         return out
 
 

@@ -664,15 +664,17 @@ void or_get_sorted(void* h, int32_t* ids, int32_t* tiles, int64_t* ranges) {
     }
 }
 
-// Full-image forward: image [3][H][W], final T [H][W], n_contrib [H][W],
-// ambiguity flags [H][W]; stats[0] = entries evaluated, stats[1] = contributions.
-void or_render(void* h, double* image, double* final_T, int32_t* n_contrib, uint8_t* ambiguous,
-               int64_t* stats) {
+// Forward over the pixel rows [y0, y1) (full-size outputs, other rows untouched):
+// image [3][H][W], final T [H][W], n_contrib [H][W], ambiguity flags [H][W];
+// stats[0] = entries evaluated, stats[1] = contributions.
+void or_render_rows(void* h, int32_t y0, int32_t y1, double* image, double* final_T,
+                    int32_t* n_contrib, uint8_t* ambiguous, int64_t* stats) {
   const Ctx& c = *static_cast<Ctx*>(h);
   const int W = c.cam.width, H = c.cam.height;
   int64_t evaluated = 0, contributions = 0;
-  std::vector<Contribution> list;
-  for (int py = 0; py < H; ++py)
+  y0 = std::max(y0, 0);
+  y1 = std::min(y1, H);
+  for (int py = y0; py < y1; ++py)
     for (int px = 0; px < W; ++px) {
       PixelResult r;
       walk_pixel(c, px, py, r, nullptr);
@@ -688,6 +690,12 @@ void or_render(void* h, double* image, double* final_T, int32_t* n_contrib, uint
     stats[0] = evaluated;
     stats[1] = contributions;
   }
+}
+
+// Full-image forward (all rows).
+void or_render(void* h, double* image, double* final_T, int32_t* n_contrib, uint8_t* ambiguous,
+               int64_t* stats) {
+  or_render_rows(h, 0, static_cast<Ctx*>(h)->cam.height, image, final_T, n_contrib, ambiguous, stats);
 }
 
 // Forward at a list of pixels only (for sampled checks at full size).
@@ -709,14 +717,19 @@ void or_render_pixels(void* h, int64_t npix, const int32_t* px, const int32_t* p
 // the planar layout of the parameters (means [3][n_pad], log_scales [3][n_pad],
 // quats [4][n_pad], opacity_logits [n_pad], sh [3][K][n_pad]). Any output
 // pointer may be null.
-void or_backward(void* h, const double* dimage, double* screen_grad, double* g_means,
-                 double* g_ls, double* g_quats, double* g_logits, double* g_sh) {
+// The same from the pixel rows [y0, y1) only (dL/dimage is full size; other
+// rows contribute nothing).
+void or_backward_rows(void* h, int32_t y0, int32_t y1, const double* dimage, double* screen_grad,
+                      double* g_means, double* g_ls, double* g_quats, double* g_logits,
+                      double* g_sh) {
   const Ctx& c = *static_cast<Ctx*>(h);
   const int W = c.cam.width, H = c.cam.height;
   const int64_t n = c.n, np = c.n_pad;
   std::vector<double> sg(static_cast<size_t>(n) * kScreen, 0.0);
   std::vector<Contribution> list;
-  for (int py = 0; py < H; ++py)
+  y0 = std::max(y0, 0);
+  y1 = std::min(y1, H);
+  for (int py = y0; py < y1; ++py)
     for (int px = 0; px < W; ++px) {
       PixelResult r;
       walk_pixel(c, px, py, r, &list);
@@ -737,6 +750,9 @@ void or_backward(void* h, const double* dimage, double* screen_grad, double* g_m
   for (int64_t i = 0; i < n; ++i) {
     if (c.aux[i].touched == 0) continue;
     const double* gs = &sg[static_cast<size_t>(i) * kScreen];
+    bool any = false;
+    for (int o = 0; o < kScreen; ++o) any = any || gs[o] != 0.0;
+    if (!any) continue;  // a zero screen gradient has a zero parameter gradient
     // Jacobian of the screen state w.r.t. (mean 3, log-scale 3, quat 4, logit).
     using D = Dual<11>;
     D p[3] = {seed<11>(c.means[i], 0), seed<11>(c.means[np + i], 1),
@@ -767,6 +783,12 @@ void or_backward(void* h, const double* dimage, double* screen_grad, double* g_m
           g_sh[(static_cast<size_t>(ch) * K + k) * np + i] = gs[6 + ch] * X.Y[k];
       }
   }
+}
+
+void or_backward(void* h, const double* dimage, double* screen_grad, double* g_means,
+                 double* g_ls, double* g_quats, double* g_logits, double* g_sh) {
+  or_backward_rows(h, 0, static_cast<Ctx*>(h)->cam.height, dimage, screen_grad, g_means, g_ls,
+                   g_quats, g_logits, g_sh);
 }
 
 // ------------------------------------------------------------------- loss --
