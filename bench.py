@@ -219,6 +219,9 @@ def profile_stages(step, cams, targets, sched, start, count):
         img, T, nc = step.forward(cs, cam.height, cam.width)
         ks.append(step.last_entries)
         ctx.loss_l1_dssim(img, targets[c], step.lam, step.loss, step.dimage)
+        if step.fused_adam:
+            step.backward_and_update(cs, T, nc, step.dimage)
+            continue
         ctx.render_backward(m.params_struct(), cs, T, nc, step.dimage, m.grads_struct())
         m.step_count += 1
         e0 = torch.cuda.Event(enable_timing=True)
@@ -233,7 +236,7 @@ def profile_stages(step, cams, targets, sched, start, count):
         adam_launches += len(GROUP_NAMES)
     prof = ctx.profile_read()
     ctx.profile_enable(False)
-    prof["adam"] = {"ms": adam_ms, "launches": adam_launches, "work": count * m.flat.numel()}
+    prof["adam"] = {"ms": adam_ms, "launches": adam_launches, "work": adam_launches and count * m.flat.numel()}
     return prof, ks
 
 
@@ -254,6 +257,9 @@ def stage_models(scene, sh_k):
         "preprocess_backward": ("hbm", 4 * n_par * 3 + 48 + 48 + 5),
         # p, g, m, v read; p, m, v, g = 0 written, per scalar
         "adam": ("hbm", 32),
+        # fused projection backward + Adam: 32 B per scalar of every group, plus the
+        # raw screen-gradient sums, the screen record and two flags, per Gaussian
+        "backward_adam": ("hbm", 32 * n_par + 48 + 48 + 5),
         # per evaluated (pixel, Gaussian) pair: 2 subtractions + 5 for the quadratic form
         "blend_forward": ("alu", 7),
         # per pair up to the last contributor: the same 7 to recompute alpha
@@ -375,7 +381,8 @@ def main_ours(args):
     rf["peak_source"] = peak_kind
     src = {"blend_forward": "blend.cu", "blend_backward": "blend.cu", "adam": "adam.cu",
            "preprocess": "preprocess.cu", "sort": "sort.cu", "loss": "loss.cu",
-           "preprocess_backward": "preprocess_backward.cu"}.get(dominant)
+           "preprocess_backward": "preprocess_backward.cu",
+           "backward_adam": "preprocess_backward.cu"}.get(dominant)
     tr = NCU_TRAFFIC.get(dominant)
     rf["traffic"] = tr[0] if (tr and src and sha12(os.path.join(PKG_CSRC, src)) == tr[1]) else None
 
@@ -384,7 +391,8 @@ def main_ours(args):
     sort_w = prof["sort"]["work"]
     passes = (sort_w / max(1, sum(ks))) if sort_w else 0
     per_step = (sum(prof[k]["launches"] for k in prof if k not in ("sort", "adam")) / steps_p +
-                (prof["sort"]["launches"] / steps_p) * (2 + passes) + len(GROUP_NAMES))
+                (prof["sort"]["launches"] / steps_p) * (2 + passes) +
+                (0 if step.fused_adam else len(GROUP_NAMES)))
     gpu_launches = int(round(per_step * args.steps))
 
     # end to end: target streamed from pinned host memory each step, loss read back
@@ -463,11 +471,7 @@ def e2e_run(step, cams, targets, sched, args, world):
                 copied[(j + 1) % 2].record(copy_stream)
         torch.cuda.current_stream().wait_event(copied[j % 2])
         step.ctx.loss_l1_dssim(img, dev_t[j % 2], step.lam, step.loss, step.dimage)
-        step.ctx.render_backward(m.params_struct(), cs, T, nc, step.dimage, m.grads_struct())
-        m.step_count += 1
-        for k in GROUP_NAMES:
-            native.adam_step(m.params[k], m.grads[k], m.m[k], m.v[k], step.lrs[k], m.step_count,
-                             step.betas[0], step.betas[1], step.eps)
+        step.backward_and_update(cs, T, nc, step.dimage)
         loss_host[j % 2].copy_(step.loss, non_blocking=True)
     torch.cuda.synchronize()
     losses.append(float(loss_host[(n - 1) % 2, 0]))

@@ -10,25 +10,12 @@
 // B200 design: purely HBM-bound, 32 B per scalar (p, g, m, v read; p, m, v and
 // the zeroed g written). float4 loads/stores, grid of 148 x 8 CTAs striding
 // over the buffer, bias corrections folded into two scalars on the host.
+#include "adam_math.cuh"
 #include "gs_kernels.cuh"
 
 namespace gs {
 
 namespace {
-
-struct AdamScalars {
-  float step_size;     // lr / (1 - b1^t)
-  float inv_sqrt_bc2;  // 1 / sqrt(1 - b2^t)
-  float beta1, beta2, eps;
-};
-
-__device__ __forceinline__ void adam_one(float& p, float& g, float& m, float& v, const AdamScalars& s) {
-  m = __fmaf_rn(s.beta1, m, (1.0f - s.beta1) * g);
-  v = __fmaf_rn(s.beta2, v, (1.0f - s.beta2) * g * g);
-  const float denom = __fmaf_rn(sqrtf(v), s.inv_sqrt_bc2, s.eps);
-  p = p - s.step_size * __fdiv_rn(m, denom);
-  g = 0.0f;
-}
 
 __global__ void __launch_bounds__(256) adam_vec_kernel(float4* __restrict__ p, float4* __restrict__ g,
                                                        float4* __restrict__ m, float4* __restrict__ v,
@@ -55,9 +42,7 @@ __global__ void adam_scalar_kernel(float* p, float* g, float* m, float* v, int64
 
 }  // namespace
 
-cudaError_t launch_adam(float* p, float* g, float* m, float* v, int64_t count, float lr, float beta1,
-                        float beta2, float eps, int step, cudaStream_t st) {
-  if (count == 0) return cudaSuccess;
+AdamScalars adam_scalars(float lr, float beta1, float beta2, float eps, int step) {
   AdamScalars s;
   const double bc1 = 1.0 - pow(static_cast<double>(beta1), step);
   const double bc2 = 1.0 - pow(static_cast<double>(beta2), step);
@@ -66,6 +51,13 @@ cudaError_t launch_adam(float* p, float* g, float* m, float* v, int64_t count, f
   s.beta1 = beta1;
   s.beta2 = beta2;
   s.eps = eps;
+  return s;
+}
+
+cudaError_t launch_adam(float* p, float* g, float* m, float* v, int64_t count, float lr, float beta1,
+                        float beta2, float eps, int step, cudaStream_t st) {
+  if (count == 0) return cudaSuccess;
+  const AdamScalars s = adam_scalars(lr, beta1, beta2, eps, step);
   const bool aligned = ((reinterpret_cast<uintptr_t>(p) | reinterpret_cast<uintptr_t>(g) |
                          reinterpret_cast<uintptr_t>(m) | reinterpret_cast<uintptr_t>(v)) & 15u) == 0;
   int64_t done = 0;

@@ -39,17 +39,40 @@ struct BlendSmem {
   float2 xy[kBatch];
   float4 q[kBatch];    // A', B', C', log2(o)
   float4 col[kBatch];  // r, g, b, o
+  float4 box[kBatch];  // x_lo, x_hi, y_lo, y_hi of the alpha >= 1/255 region
   uint32_t id[kBatch];
 };
 
 __device__ __forceinline__ void stage(BlendSmem& s, int slot, uint32_t gid, const Screen* screen) {
   const Screen g = screen[gid];
-  s.xy[slot] = make_float2(g.a.x, g.a.y);
-  const float o = g.b.y;
-  s.q[slot] = make_float4(__fmul_rn(-0.5f * kLog2e, g.a.z), __fmul_rn(-kLog2e, g.a.w),
-                          __fmul_rn(-0.5f * kLog2e, g.b.x), log2f(o));
+  const float u = g.a.x, v = g.a.y, A = g.a.z, B = g.a.w, C = g.b.x, o = g.b.y;
+  s.xy[slot] = make_float2(u, v);
+  s.q[slot] = make_float4(__fmul_rn(-0.5f * kLog2e, A), __fmul_rn(-kLog2e, B),
+                          __fmul_rn(-0.5f * kLog2e, C), log2f(o));
   s.col[slot] = make_float4(g.b.z, g.b.w, g.c.x, o);
+  // o exp(-e) >= 1/255 exactly when e <= E = ln(255 o); the ellipse e <= E has the
+  // axis-aligned half-widths sqrt(2 E Sigma'_xx), sqrt(2 E Sigma'_yy), with
+  // Sigma' = conic^-1. The box is widened by 0.1% + 0.02 px so that float32
+  // rounding of the per-pixel alpha can never pass the floor outside it: a warp
+  // whose pixels all lie outside skips the Gaussian with unchanged results.
+  const float E = logf(255.0f * o);
+  float4 box = make_float4(1.0f, -1.0f, 1.0f, -1.0f);  // empty
+  const float det = A * C - B * B;
+  if (E > 0.0f && det > 0.0f) {
+    const float hx = sqrtf(2.0f * E * C / det) * 1.001f + 0.02f;
+    const float hy = sqrtf(2.0f * E * A / det) * 1.001f + 0.02f;
+    box = make_float4(u - hx, u + hx, v - hy, v + hy);
+  }
+  s.box[slot] = box;
   s.id[slot] = gid;
+}
+
+// 2^x in one MUFU instruction (flushes results below 2^-126 to 0, far under
+// the 1/255 floor).
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 // Exponent in base 2 of o exp(-e) at offset (dx, dy); identical in both passes.
@@ -57,6 +80,12 @@ __device__ __forceinline__ float power2(const float4 q, float dx, float dy) {
   const float t = __fmaf_rn(__fmul_rn(q.z, dy), dy, q.w);
   const float s = __fmaf_rn(q.x, dx, __fmul_rn(q.y, dy));
   return __fmaf_rn(s, dx, t);
+}
+
+// True when the Gaussian's alpha >= 1/255 box misses the warp's 8x4 pixel block.
+__device__ __forceinline__ bool misses_block(const float4 box, float bx0, float bx1, float by0,
+                                             float by1) {
+  return box.y < bx0 || box.x > bx1 || box.w < by0 || box.z > by1;
 }
 
 // Adds this warp's count to *pairs (profiling builds of the kernels only).
@@ -80,6 +109,11 @@ __global__ void __launch_bounds__(256) blend_forward_kernel(BlendArgs a) {
   const int n = static_cast<int>(range.y - range.x);
   const float fx = static_cast<float>(px), fy = static_cast<float>(py);
 
+  // this warp's 8x4 pixel block
+  const float bx0 = static_cast<float>(tx * kTile + ((threadIdx.x >> 5) & 1) * 8);
+  const float by0 = static_cast<float>(ty * kTile + (threadIdx.x >> 6) * 4);
+  const float bx1 = bx0 + 7.0f, by1 = by0 + 3.0f;
+
   float T = 1.0f, C0 = 0.0f, C1 = 0.0f, C2 = 0.0f;
   int last = 0;
   bool done = !inside;
@@ -90,12 +124,15 @@ __global__ void __launch_bounds__(256) blend_forward_kernel(BlendArgs a) {
     if (k < n) stage(sm, threadIdx.x, a.order[range.x + k], a.screen);
     __syncthreads();
     const int cnt = min(kBatch, n - b);
-    for (int j = 0; j < cnt && !done; ++j) {
-      if (kCount) ++evals;
+    if (__all_sync(0xffffffffu, done)) continue;  // this warp is saturated
+    for (int j = 0; j < cnt; ++j) {
+      if ((j & 31) == 31 && __all_sync(0xffffffffu, done)) break;
+      if (misses_block(sm.box[j], bx0, bx1, by0, by1)) continue;
+      if (kCount) evals += !done;
       const float2 xy = sm.xy[j];
       const float p = power2(sm.q[j], fx - xy.x, fy - xy.y);
-      const float alpha = fminf(kAlphaMax, exp2f(p));
-      if (alpha >= kAlphaMin) {
+      const float alpha = fminf(kAlphaMax, fast_exp2(p));
+      if (!done && alpha >= kAlphaMin) {
         const float4 c = sm.col[j];
         const float w = alpha * T;
         C0 = __fmaf_rn(w, c.x, C0);
@@ -200,6 +237,11 @@ __global__ void __launch_bounds__(256) blend_backward_kernel(BlendArgs a) {
   // n_contrib comes from the caller: never walk past the tile's own list.
   const int max_last = min(s_max_last, static_cast<int>(range.y - range.x));
 
+  const float bx0 = static_cast<float>(tx * kTile + ((threadIdx.x >> 5) & 1) * 8);
+  const float by0 = static_cast<float>(ty * kTile + (threadIdx.x >> 6) * 4);
+  const float bx1 = bx0 + 7.0f, by1 = by0 + 3.0f;
+  const int warp_last = wmax;  // no lane of this warp blends anything at or after it
+
   // Which raw sum this lane holds after the reduce-scatter.
   const int red_idx = ((lane >> 1) & 1) * 8 + ((lane >> 2) & 1) * 4 + ((lane >> 3) & 1) * 2 +
                       ((lane >> 4) & 1);
@@ -212,11 +254,12 @@ __global__ void __launch_bounds__(256) blend_backward_kernel(BlendArgs a) {
     const int k = start + threadIdx.x;
     if (k < end) stage(sm, threadIdx.x, a.order[range.x + k], a.screen);
     __syncthreads();
-    for (int j = end - 1; j >= start; --j) {
+    for (int j = min(end, warp_last) - 1; j >= start; --j) {
       const int slot = j - start;
+      if (misses_block(sm.box[slot], bx0, bx1, by0, by1)) continue;
       const float2 xy = sm.xy[slot];
       const float dx = fx - xy.x, dy = fy - xy.y;
-      const float raw = exp2f(power2(sm.q[slot], dx, dy));
+      const float raw = fast_exp2(power2(sm.q[slot], dx, dy));
       const float alpha = fminf(kAlphaMax, raw);
       const bool contrib = j < last && alpha >= kAlphaMin;
       if (kCount && j < last) ++evals;

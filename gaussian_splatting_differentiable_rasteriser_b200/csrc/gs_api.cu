@@ -454,9 +454,15 @@ gs_status gs_loss_l1_dssim(gs_ctx* c, const float* image, const float* target, i
   return GS_OK;
 }
 
-gs_status gs_render_backward(gs_ctx* c, const gs_params* p, const gs_camera* cam, const float* final_T,
-                             const int32_t* n_contrib, const float* dloss_dimage, gs_grads* g,
-                             void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Shared front half of the two backward entry points: checks, the blend
+// backward, and the projection-backward argument record.
+gs_status backward_common(gs_ctx* c, const gs_params* p, const gs_camera* cam, const float* final_T,
+                          const int32_t* n_contrib, const float* dloss_dimage, gs_grads* g,
+                          cudaStream_t st, gs::PreprocessBwdArgs& a) {
   if (!c) return GS_ERR_INVALID_ARG;
   if (!c->have_fwd) return fail(c, GS_ERR_INVALID_ARG, "gs_render_forward has not run");
   gs_status s = check_params(c, p);
@@ -473,7 +479,6 @@ gs_status gs_render_backward(gs_ctx* c, const gs_params* p, const gs_camera* cam
   if (p->n > 0)
     for (float* q : gp)
       if (!q || !aligned(q, 4)) return fail(c, GS_ERR_INVALID_ARG, "a gradient pointer is NULL or misaligned");
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (p->n > 0)
     GS_CUDA(c, cudaMemsetAsync(c->sgrad, 0, sizeof(float) * gs::kGradStride * p->n, st));
   gs::BlendArgs ba{};
@@ -489,7 +494,6 @@ gs_status gs_render_backward(gs_ctx* c, const gs_params* p, const gs_camera* cam
   prof_begin(c, st);
   GS_CUDA(c, gs::launch_blend_backward(ba, st));
   prof_end(c, GS_STAGE_BLEND_BACKWARD, 0, st);
-  gs::PreprocessBwdArgs a;
   a.means = p->means;
   a.log_scales = p->log_scales;
   a.quats = p->quats;
@@ -509,9 +513,66 @@ gs_status gs_render_backward(gs_ctx* c, const gs_params* p, const gs_camera* cam
   a.g_quats = g->quats;
   a.g_opacity_logits = g->opacity_logits;
   a.g_sh = g->sh;
+  return GS_OK;
+}
+
+bool valid_betas(float beta1, float beta2, float eps) {
+  return beta1 >= 0.f && beta1 < 1.f && beta2 >= 0.f && beta2 < 1.f && eps > 0.f && std::isfinite(eps);
+}
+
+}  // namespace
+
+extern "C" {
+
+gs_status gs_render_backward(gs_ctx* c, const gs_params* p, const gs_camera* cam, const float* final_T,
+                             const int32_t* n_contrib, const float* dloss_dimage, gs_grads* g,
+                             void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  gs::PreprocessBwdArgs a;
+  gs_status s = backward_common(c, p, cam, final_T, n_contrib, dloss_dimage, g, st, a);
+  if (s != GS_OK) return s;
   prof_begin(c, st);
   GS_CUDA(c, gs::launch_preprocess_backward(a, st));
   prof_end(c, GS_STAGE_PREPROCESS_BACKWARD, p->n, st);
+  return GS_OK;
+}
+
+gs_status gs_render_backward_adam(gs_ctx* c, const gs_params* p, const gs_camera* cam,
+                                  const float* final_T, const int32_t* n_contrib,
+                                  const float* dloss_dimage, gs_grads* g, gs_grads* m, gs_grads* v,
+                                  const float* lr, float beta1, float beta2, float eps, int32_t step,
+                                  void* stream) {
+  if (!c) return GS_ERR_INVALID_ARG;
+  if (!m || !v || !lr) return fail(c, GS_ERR_INVALID_ARG, "moments and learning rates must be non-NULL");
+  if (step < 1 || !valid_betas(beta1, beta2, eps))
+    return fail(c, GS_ERR_INVALID_ARG, "step must be >= 1, betas in [0, 1), eps > 0");
+  for (int k = 0; k < 5; ++k)
+    if (!std::isfinite(lr[k])) return fail(c, GS_ERR_INVALID_ARG, "learning rates must be finite");
+  if (p && p->n_pad > 0) {
+    float* mp[] = {m->means, m->log_scales, m->quats, m->opacity_logits, m->sh,
+                   v->means, v->log_scales, v->quats, v->opacity_logits, v->sh};
+    for (float* q : mp)
+      if (!q || !aligned(q, 4)) return fail(c, GS_ERR_INVALID_ARG, "a moment pointer is NULL or misaligned");
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  gs::PreprocessBwdArgs a;
+  gs_status s = backward_common(c, p, cam, final_T, n_contrib, dloss_dimage, g, st, a);
+  if (s != GS_OK) return s;
+  gs::FusedAdamArgs f;
+  const float* pp[5] = {p->means, p->log_scales, p->quats, p->opacity_logits, p->sh};
+  float* gg[5] = {g->means, g->log_scales, g->quats, g->opacity_logits, g->sh};
+  float* mm[5] = {m->means, m->log_scales, m->quats, m->opacity_logits, m->sh};
+  float* vv[5] = {v->means, v->log_scales, v->quats, v->opacity_logits, v->sh};
+  for (int k = 0; k < 5; ++k) {
+    f.p[k] = const_cast<float*>(pp[k]);  // documented: updated in place
+    f.g[k] = gg[k];
+    f.m[k] = mm[k];
+    f.v[k] = vv[k];
+    f.s[k] = gs::adam_scalars(lr[k], beta1, beta2, eps, step);
+  }
+  prof_begin(c, st);
+  GS_CUDA(c, gs::launch_preprocess_backward_adam(a, f, st));
+  prof_end(c, GS_STAGE_BACKWARD_ADAM, p->n_pad, st);
   return GS_OK;
 }
 
@@ -521,8 +582,7 @@ gs_status gs_adam_step(float* param, float* grad, float* m, float* v, int64_t co
   if (count > 0 && (!param || !grad || !m || !v || !aligned(param, 4) || !aligned(grad, 4) ||
                     !aligned(m, 4) || !aligned(v, 4)))
     return GS_ERR_INVALID_ARG;
-  if (!(beta1 >= 0.f && beta1 < 1.f && beta2 >= 0.f && beta2 < 1.f && eps > 0.f && std::isfinite(lr)))
-    return GS_ERR_INVALID_ARG;
+  if (!valid_betas(beta1, beta2, eps) || !std::isfinite(lr)) return GS_ERR_INVALID_ARG;
   cudaError_t e = gs::launch_adam(param, grad, m, v, count, lr, beta1, beta2, eps, step,
                                   static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? GS_OK : GS_ERR_CUDA;
@@ -563,7 +623,7 @@ gs_status gs_profile_read(gs_ctx* c, double* ms, int64_t* launches, int64_t* wor
 const char* gs_stage_name(int32_t stage) {
   static const char* names[GS_NUM_STAGES] = {"preprocess", "scan", "duplicate", "sort", "ranges",
                                              "blend_forward", "loss", "blend_backward",
-                                             "preprocess_backward"};
+                                             "preprocess_backward", "backward_adam"};
   return (stage >= 0 && stage < GS_NUM_STAGES) ? names[stage] : "";
 }
 

@@ -2,6 +2,7 @@
 // Everything here is internal to the library; the public surface is gs_api.h.
 #pragma once
 
+#include "adam_math.cuh"
 #include "gs_common.cuh"
 
 namespace gs {
@@ -131,6 +132,21 @@ struct PreprocessBwdArgs {
 };
 
 cudaError_t launch_preprocess_backward(const PreprocessBwdArgs& a, cudaStream_t st);
+
+// Parameters (written in place), accumulated gradients (zeroed), Adam moments
+// and per-group scalars, in group order means, log_scales, quats,
+// opacity_logits, sh.
+struct FusedAdamArgs {
+  float* p[5];
+  float* g[5];
+  float* m[5];
+  float* v[5];
+  AdamScalars s[5];
+};
+
+cudaError_t launch_preprocess_backward_adam(const PreprocessBwdArgs& a, const FusedAdamArgs& f,
+                                           cudaStream_t st);
+AdamScalars adam_scalars(float lr, float beta1, float beta2, float eps, int step);
 cudaError_t launch_screen_grads(const Screen* screen, const float* sgrad, int64_t n, float* out,
                                 cudaStream_t st);
 

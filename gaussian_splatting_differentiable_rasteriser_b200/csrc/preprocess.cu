@@ -23,6 +23,7 @@ __device__ __forceinline__ double dot3(const double* a, const double* b) {
   return a[0] * b[0] + a[1] * b[1] + a[2] * b[2];
 }
 
+template <int kDeg>
 __global__ void __launch_bounds__(256) preprocess_kernel(PreprocessArgs a) {
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   uint32_t touched = 0;
@@ -113,14 +114,15 @@ __global__ void __launch_bounds__(256) preprocess_kernel(PreprocessArgs a) {
           const double dn = sqrt(dot3(d, d));
           const float dx = static_cast<float>(d[0] / dn), dy = static_cast<float>(d[1] / dn),
                       dz = static_cast<float>(d[2] / dn);
+          constexpr int nk = (kDeg + 1) * (kDeg + 1);
           float Yk[16];
-          sh_basis(a.active_degree, dx, dy, dz, Yk);
-          const int nk = (a.active_degree + 1) * (a.active_degree + 1);
+          sh_basis(kDeg, dx, dy, dz, Yk);
           float rgb[3];
 #pragma unroll
           for (int ch = 0; ch < 3; ++ch) {
             const float* shc = a.sh + static_cast<int64_t>(ch) * a.sh_k * np + i;
             float col = 0.0f;
+#pragma unroll
             for (int k = 0; k < nk; ++k) col = fmaf(shc[static_cast<int64_t>(k) * np], Yk[k], col);
             if (col < 0.0f) {
               col = 0.0f;
@@ -218,7 +220,13 @@ __global__ void __launch_bounds__(1024) scan_blocks_kernel(const uint32_t* block
 
 cudaError_t launch_preprocess(const PreprocessArgs& a, int64_t num_blocks, cudaStream_t st) {
   if (a.n == 0) return cudaSuccess;
-  preprocess_kernel<<<static_cast<unsigned>(num_blocks), 256, 0, st>>>(a);
+  const unsigned grid = static_cast<unsigned>(num_blocks);
+  switch (a.active_degree) {
+    case 0: preprocess_kernel<0><<<grid, 256, 0, st>>>(a); break;
+    case 1: preprocess_kernel<1><<<grid, 256, 0, st>>>(a); break;
+    case 2: preprocess_kernel<2><<<grid, 256, 0, st>>>(a); break;
+    default: preprocess_kernel<3><<<grid, 256, 0, st>>>(a); break;
+  }
   return cudaGetLastError();
 }
 

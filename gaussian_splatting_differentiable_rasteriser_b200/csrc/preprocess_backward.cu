@@ -20,7 +20,11 @@
 //   R(q^) -> dL/dq^, then dL/dq = (dL/dq^ - q^ <q^, dL/dq^>) / |q|
 //   colour: dL/dsh_k = dL/dc Y_k, dL/dv = sum dL/dc sh_k grad Y_k,
 //           dL/dp += (dL/dv - v <v, dL/dv>) / |p - campos|
-// The result is ADDED to the caller's gradient buffers (coalesced planar RMW).
+// The result is ADDED to the caller's gradient buffers (coalesced planar RMW),
+// or, in the fused variant, added to them and consumed by the Adam step of
+// every parameter group in the same pass (the gradient never makes a separate
+// round trip through HBM).
+#include "adam_math.cuh"
 #include "gs_kernels.cuh"
 #include "sh.cuh"
 
@@ -28,9 +32,17 @@ namespace gs {
 
 namespace {
 
-__global__ void __launch_bounds__(256) preprocess_backward_kernel(PreprocessBwdArgs a) {
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (i >= a.n || a.touched[i] == 0) return;
+// Gradient of one visible Gaussian with respect to everything but its SH
+// coefficients, plus what the SH part needs (masked colour gradient and the
+// view direction). The view-direction term of the position is added by
+// add_view_dir_term once the SH coefficients have been read.
+struct GaussGrad {
+  float dp[3], dls[3], dq[4], dlogit;
+  float drgb[3];
+  float vx, vy, vz, idl;
+};
+
+__device__ __forceinline__ void geometry_grad(const PreprocessBwdArgs& a, int64_t i, GaussGrad& out) {
   const int64_t np = a.n_pad;
   const CamArgs& cam = a.cam;
   const float4* sg4 = reinterpret_cast<const float4*>(a.sgrad + i * kGradStride);
@@ -44,8 +56,10 @@ __global__ void __launch_bounds__(256) preprocess_backward_kernel(PreprocessBwdA
   const float d_v = B * r0.y + C * r0.z;
   const float dA = -0.5f * r0.w, dB = -r1.x, dC = -0.5f * r1.y;
   const float d_o = r0.x / o;
-  const float drgb[3] = {(clamped & 1) ? 0.f : r1.z, (clamped & 2) ? 0.f : r1.w,
-                         (clamped & 4) ? 0.f : r2.x};
+  out.drgb[0] = (clamped & 1) ? 0.f : r1.z;
+  out.drgb[1] = (clamped & 2) ? 0.f : r1.w;
+  out.drgb[2] = (clamped & 4) ? 0.f : r2.x;
+  out.dlogit = d_o * o * (1.f - o);
 
   // Recompute the forward quantities.
   const float p[3] = {a.means[i], a.means[np + i], a.means[2 * np + i]};
@@ -126,9 +140,8 @@ __global__ void __launch_bounds__(256) preprocess_backward_kernel(PreprocessBwdA
   dX += d_u * jx;
   dY += d_v * jy;
   dZ += d_u * jxz + d_v * jyz;
-  float dp[3];
 #pragma unroll
-  for (int c = 0; c < 3; ++c) dp[c] = cam.R[c] * dX + cam.R[3 + c] * dY + cam.R[6 + c] * dZ;
+  for (int c = 0; c < 3; ++c) out.dp[c] = cam.R[c] * dX + cam.R[3 + c] * dY + cam.R[6 + c] * dZ;
 
   // Sigma = M M^T -> dM = 2 dSigma M (dSigma symmetric)
   float dM[9];
@@ -137,10 +150,9 @@ __global__ void __launch_bounds__(256) preprocess_backward_kernel(PreprocessBwdA
 #pragma unroll
     for (int c = 0; c < 3; ++c)
       dM[3 * r + c] = 2.f * (dSig[3 * r] * M[c] + dSig[3 * r + 1] * M[3 + c] + dSig[3 * r + 2] * M[6 + c]);
-  float dls[3];
 #pragma unroll
   for (int c = 0; c < 3; ++c)
-    dls[c] = (dM[c] * Rq[c] + dM[3 + c] * Rq[3 + c] + dM[6 + c] * Rq[6 + c]) * s[c];
+    out.dls[c] = (dM[c] * Rq[c] + dM[3 + c] * Rq[3 + c] + dM[6 + c] * Rq[6 + c]) * s[c];
   float G[9];  // dL/dR = dM diag(s)
 #pragma unroll
   for (int r = 0; r < 3; ++r)
@@ -154,46 +166,133 @@ __global__ void __launch_bounds__(256) preprocess_backward_kernel(PreprocessBwdA
   const float gz = 2.f * (-2.f * z * G[0] - w * G[1] + x * G[2] + w * G[3] - 2.f * z * G[4] +
                           y * G[5] + x * G[6] + y * G[7]);
   const float qdot = w * gw + x * gx + y * gy + z * gz;
-  const float dq[4] = {(gw - w * qdot) * iqn, (gx - x * qdot) * iqn, (gy - y * qdot) * iqn,
-                       (gz - z * qdot) * iqn};
+  out.dq[0] = (gw - w * qdot) * iqn;
+  out.dq[1] = (gx - x * qdot) * iqn;
+  out.dq[2] = (gy - y * qdot) * iqn;
+  out.dq[3] = (gz - z * qdot) * iqn;
 
-  // Colour: SH coefficients and the view-direction path into the position.
-  float dv[3] = {p[0] - cam.campos[0], p[1] - cam.campos[1], p[2] - cam.campos[2]};
+  // view direction v = normalize(p - campos)
+  const float dv[3] = {p[0] - cam.campos[0], p[1] - cam.campos[1], p[2] - cam.campos[2]};
   const float dlen = sqrtf(dv[0] * dv[0] + dv[1] * dv[1] + dv[2] * dv[2]);
-  const float idl = 1.0f / dlen;
-  const float vx = dv[0] * idl, vy = dv[1] * idl, vz = dv[2] * idl;
+  out.idl = 1.0f / dlen;
+  out.vx = dv[0] * out.idl;
+  out.vy = dv[1] * out.idl;
+  out.vz = dv[2] * out.idl;
+}
+
+// dp += (dL/dv - v <v, dL/dv>) / |p - campos| with dL/dv = sum_c dL/dc sum_k sh_ck grad Y_k.
+template <int kDeg>
+__device__ __forceinline__ void add_view_dir_term(GaussGrad& g, const float (&wsum)[16]) {
+  float gvx, gvy, gvz;
+  sh_grad_dir(kDeg, g.vx, g.vy, g.vz, wsum, gvx, gvy, gvz);
+  const float vdot = g.vx * gvx + g.vy * gvy + g.vz * gvz;
+  g.dp[0] += (gvx - g.vx * vdot) * g.idl;
+  g.dp[1] += (gvy - g.vy * vdot) * g.idl;
+  g.dp[2] += (gvz - g.vz * vdot) * g.idl;
+}
+
+// Backward that ADDS the gradient into the caller's buffers.
+template <int kDeg>
+__global__ void __launch_bounds__(256) preprocess_backward_kernel(PreprocessBwdArgs a) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= a.n || a.touched[i] == 0) return;
+  const int64_t np = a.n_pad;
+  GaussGrad g;
+  geometry_grad(a, i, g);
+  constexpr int nk = (kDeg + 1) * (kDeg + 1);
   float Yk[16];
-  sh_basis(a.active_degree, vx, vy, vz, Yk);
-  const int nk = (a.active_degree + 1) * (a.active_degree + 1);
+  sh_basis(kDeg, g.vx, g.vy, g.vz, Yk);
   float wsum[16];
 #pragma unroll
   for (int k = 0; k < 16; ++k) wsum[k] = 0.f;
 #pragma unroll
   for (int ch = 0; ch < 3; ++ch) {
-    if (drgb[ch] == 0.f) continue;
+    if (g.drgb[ch] == 0.f) continue;
     const float* shc = a.sh + static_cast<int64_t>(ch) * a.sh_k * np + i;
     float* gsh = a.g_sh + static_cast<int64_t>(ch) * a.sh_k * np + i;
+#pragma unroll
     for (int k = 0; k < nk; ++k) {
-      gsh[static_cast<int64_t>(k) * np] += drgb[ch] * Yk[k];
-      wsum[k] += drgb[ch] * shc[static_cast<int64_t>(k) * np];
+      const int64_t o = static_cast<int64_t>(k) * np;
+      gsh[o] = __fmaf_rn(g.drgb[ch], Yk[k], gsh[o]);
+      wsum[k] = __fmaf_rn(g.drgb[ch], shc[o], wsum[k]);
     }
   }
-  float gvx, gvy, gvz;
-  sh_grad_dir(a.active_degree, vx, vy, vz, wsum, gvx, gvy, gvz);
-  const float vdot = vx * gvx + vy * gvy + vz * gvz;
-  dp[0] += (gvx - vx * vdot) * idl;
-  dp[1] += (gvy - vy * vdot) * idl;
-  dp[2] += (gvz - vz * vdot) * idl;
-
-  a.g_means[i] += dp[0];
-  a.g_means[np + i] += dp[1];
-  a.g_means[2 * np + i] += dp[2];
-  a.g_log_scales[i] += dls[0];
-  a.g_log_scales[np + i] += dls[1];
-  a.g_log_scales[2 * np + i] += dls[2];
+  add_view_dir_term<kDeg>(g, wsum);
 #pragma unroll
-  for (int c = 0; c < 4; ++c) a.g_quats[c * np + i] += dq[c];
-  a.g_opacity_logits[i] += d_o * o * (1.f - o);
+  for (int c = 0; c < 3; ++c) a.g_means[c * np + i] += g.dp[c];
+#pragma unroll
+  for (int c = 0; c < 3; ++c) a.g_log_scales[c * np + i] += g.dls[c];
+#pragma unroll
+  for (int c = 0; c < 4; ++c) a.g_quats[c * np + i] += g.dq[c];
+  a.g_opacity_logits[i] += g.dlogit;
+}
+
+// The same backward fused with the Adam step of every group, over all n_pad
+// Gaussians (Adam is dense: invisible Gaussians still move by their moments).
+// Per scalar: g = accumulated gradient + this view's gradient, then the update
+// of adam_one; the gradient buffer is left zeroed. Bit-identical to the
+// accumulate kernel followed by the standalone Adam kernel.
+template <int kDeg>
+__global__ void __launch_bounds__(256) preprocess_backward_adam_kernel(PreprocessBwdArgs a, FusedAdamArgs f) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= a.n_pad) return;
+  const int64_t np = a.n_pad;
+  const bool visible = i < a.n && a.touched[i] != 0;
+  GaussGrad g;
+  if (visible) {
+    geometry_grad(a, i, g);
+  } else {
+#pragma unroll
+    for (int c = 0; c < 3; ++c) g.dp[c] = g.dls[c] = g.drgb[c] = 0.f;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) g.dq[c] = 0.f;
+    g.dlogit = 0.f;
+    g.vx = g.vy = g.vz = 0.f;
+    g.idl = 0.f;
+  }
+  constexpr int nk = (kDeg + 1) * (kDeg + 1);
+  float Yk[16];
+  sh_basis(kDeg, g.vx, g.vy, g.vz, Yk);
+  float wsum[16];
+#pragma unroll
+  for (int k = 0; k < 16; ++k) wsum[k] = 0.f;
+  // SH first: the view-direction term of the position needs their old values.
+#pragma unroll
+  for (int ch = 0; ch < 3; ++ch) {
+    const int64_t base = static_cast<int64_t>(ch) * a.sh_k * np + i;
+    const float dc = g.drgb[ch];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      if (k >= a.sh_k) break;
+      const int64_t o = base + static_cast<int64_t>(k) * np;
+      float p = f.p[4][o], gr = f.g[4][o], m = f.m[4][o], v = f.v[4][o];
+      if (k < nk && dc != 0.f) {
+        wsum[k] = __fmaf_rn(dc, p, wsum[k]);
+        gr = __fmaf_rn(dc, Yk[k], gr);
+      }
+      adam_one(p, gr, m, v, f.s[4]);
+      f.p[4][o] = p;
+      f.g[4][o] = gr;
+      f.m[4][o] = m;
+      f.v[4][o] = v;
+    }
+  }
+  if (visible) add_view_dir_term<kDeg>(g, wsum);
+  const float view[11] = {g.dp[0],  g.dp[1],  g.dp[2],  g.dls[0], g.dls[1], g.dls[2],
+                          g.dq[0],  g.dq[1],  g.dq[2],  g.dq[3],  g.dlogit};
+#pragma unroll
+  for (int j = 0; j < 11; ++j) {
+    const int grp = j < 3 ? 0 : (j < 6 ? 1 : (j < 10 ? 2 : 3));
+    const int c = j < 3 ? j : (j < 6 ? j - 3 : (j < 10 ? j - 6 : 0));
+    const int64_t o = c * np + i;
+    float p = f.p[grp][o], gr = f.g[grp][o], m = f.m[grp][o], v = f.v[grp][o];
+    gr += view[j];
+    adam_one(p, gr, m, v, f.s[grp]);
+    f.p[grp][o] = p;
+    f.g[grp][o] = gr;
+    f.m[grp][o] = m;
+    f.v[grp][o] = v;
+  }
 }
 
 // Natural screen-space gradient from the raw sums (for stage checks).
@@ -219,7 +318,26 @@ __global__ void screen_grads_kernel(const Screen* screen, const float* sgrad, in
 
 cudaError_t launch_preprocess_backward(const PreprocessBwdArgs& a, cudaStream_t st) {
   if (a.n == 0) return cudaSuccess;
-  preprocess_backward_kernel<<<static_cast<unsigned>((a.n + 255) / 256), 256, 0, st>>>(a);
+  const unsigned grid = static_cast<unsigned>((a.n + 255) / 256);
+  switch (a.active_degree) {
+    case 0: preprocess_backward_kernel<0><<<grid, 256, 0, st>>>(a); break;
+    case 1: preprocess_backward_kernel<1><<<grid, 256, 0, st>>>(a); break;
+    case 2: preprocess_backward_kernel<2><<<grid, 256, 0, st>>>(a); break;
+    default: preprocess_backward_kernel<3><<<grid, 256, 0, st>>>(a); break;
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_preprocess_backward_adam(const PreprocessBwdArgs& a, const FusedAdamArgs& f,
+                                           cudaStream_t st) {
+  if (a.n_pad == 0) return cudaSuccess;
+  const unsigned grid = static_cast<unsigned>((a.n_pad + 255) / 256);
+  switch (a.active_degree) {
+    case 0: preprocess_backward_adam_kernel<0><<<grid, 256, 0, st>>>(a, f); break;
+    case 1: preprocess_backward_adam_kernel<1><<<grid, 256, 0, st>>>(a, f); break;
+    case 2: preprocess_backward_adam_kernel<2><<<grid, 256, 0, st>>>(a, f); break;
+    default: preprocess_backward_adam_kernel<3><<<grid, 256, 0, st>>>(a, f); break;
+  }
   return cudaGetLastError();
 }
 

@@ -58,11 +58,17 @@ class GaussianModel:
         p.sh_degree, p.active_degree = self.sh_degree, self.active_degree
         return p
 
-    def grads_struct(self) -> native.GsGrads:
+    def _struct(self, tensors) -> native.GsGrads:
         g = native.GsGrads()
         for k in GROUP_NAMES:
-            setattr(g, k, self.grads[k].data_ptr())
+            setattr(g, k, tensors[k].data_ptr())
         return g
+
+    def grads_struct(self) -> native.GsGrads:
+        return self._struct(self.grads)
+
+    def moments_structs(self):
+        return self._struct(self.m), self._struct(self.v)
 
 
 DEFAULT_LR = {k: 1e-3 for k in GROUP_NAMES}
@@ -72,8 +78,9 @@ class TrainStep:
     """Buffers and the call sequence of one iteration for images up to width x height."""
 
     def __init__(self, model: GaussianModel, max_entries: int, width: int, height: int, lrs=None,
-                 lam=0.2, betas=(0.9, 0.999), eps=1e-8, device="cuda"):
+                 lam=0.2, betas=(0.9, 0.999), eps=1e-8, device="cuda", fused_adam=True):
         self.model = model
+        self.fused_adam = fused_adam
         self.ctx = native.Context(model.n_pad, max_entries, width, height)
         self.lrs = dict(DEFAULT_LR if lrs is None else lrs)
         self.lam, self.betas, self.eps = lam, betas, eps
@@ -102,9 +109,21 @@ class TrainStep:
         img, T, nc = self.forward(cs, H, W)
         dimg = self.dimage if img.shape == self.dimage.shape else torch.empty_like(img)
         self.ctx.loss_l1_dssim(img, target, self.lam, self.loss, dimg)
-        self.ctx.render_backward(self.model.params_struct(), cs, T, nc, dimg, self.model.grads_struct())
-        self.model.step_count += 1
-        for k in GROUP_NAMES:
-            native.adam_step(self.model.params[k], self.model.grads[k], self.model.m[k], self.model.v[k],
-                             self.lrs[k], self.model.step_count, self.betas[0], self.betas[1], self.eps)
+        self.backward_and_update(cs, T, nc, dimg)
         return self.loss
+
+    def backward_and_update(self, cs, T, nc, dimg):
+        """Backward of the last forward plus the Adam step of every group: one fused
+        pass over the parameters, or gs_render_backward then gs_adam_step per group."""
+        m = self.model
+        m.step_count += 1
+        if self.fused_adam:
+            em, ev = m.moments_structs()
+            self.ctx.render_backward_adam(m.params_struct(), cs, T, nc, dimg, m.grads_struct(), em, ev,
+                                          [self.lrs[k] for k in GROUP_NAMES], m.step_count,
+                                          self.betas[0], self.betas[1], self.eps)
+            return
+        self.ctx.render_backward(m.params_struct(), cs, T, nc, dimg, m.grads_struct())
+        for k in GROUP_NAMES:
+            native.adam_step(m.params[k], m.grads[k], m.m[k], m.v[k], self.lrs[k], m.step_count,
+                             self.betas[0], self.betas[1], self.eps)

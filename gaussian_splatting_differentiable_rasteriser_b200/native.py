@@ -21,11 +21,13 @@ _STATUS = {0: "GS_OK", 1: "GS_ERR_INVALID_ARG", 2: "GS_ERR_CAPACITY", 3: "GS_ERR
            4: "GS_ERR_DEVICE"}
 
 EXPORTED = ("gs_create", "gs_destroy", "gs_last_error", "gs_preprocess", "gs_render_forward",
-            "gs_loss_l1_dssim", "gs_render_backward", "gs_adam_step", "gs_profile_enable",
+            "gs_loss_l1_dssim", "gs_render_backward", "gs_render_backward_adam", "gs_adam_step",
+            "gs_profile_enable",
             "gs_profile_read", "gs_stage_name", "gs_debug_preprocess", "gs_debug_sorted",
             "gs_debug_screen_grads")
 STAGES = ("preprocess", "scan", "duplicate", "sort", "ranges", "blend_forward", "loss",
-          "blend_backward", "preprocess_backward")
+          "blend_backward", "preprocess_backward", "backward_adam")
+GROUPS = ("means", "log_scales", "quats", "opacity_logits", "sh")
 
 
 class GsError(RuntimeError):
@@ -78,6 +80,9 @@ def load(path: str = LIB_PATH):
     L.gs_loss_l1_dssim.argtypes = [P, P, P, I32, I32, F, P, P, P]
     L.gs_render_backward.argtypes = [P, ctypes.POINTER(GsParams), ctypes.POINTER(GsCamera), P, P, P,
                                      ctypes.POINTER(GsGrads), P]
+    L.gs_render_backward_adam.argtypes = [P, ctypes.POINTER(GsParams), ctypes.POINTER(GsCamera), P, P, P,
+                                          ctypes.POINTER(GsGrads), ctypes.POINTER(GsGrads),
+                                          ctypes.POINTER(GsGrads), ctypes.POINTER(F), F, F, F, I32, P]
     L.gs_adam_step.argtypes = [P, P, P, P, I64, F, F, F, F, I32, P]
     L.gs_profile_enable.argtypes = [P, I32]
     L.gs_profile_read.argtypes = [P, P, P, P]
@@ -163,6 +168,15 @@ class Context:
         self._check(self.L.gs_render_backward(self.h, ctypes.byref(params), ctypes.byref(cam),
                                               _ptr(final_T), _ptr(n_contrib), _ptr(dloss_dimage),
                                               ctypes.byref(grads), _stream(stream)))
+
+    def render_backward_adam(self, params: GsParams, cam: GsCamera, final_T, n_contrib, dloss_dimage,
+                             grads: GsGrads, exp_avg: GsGrads, exp_avg_sq: GsGrads, lrs, step,
+                             beta1=0.9, beta2=0.999, eps=1e-8, stream=None):
+        lr = (ctypes.c_float * 5)(*[float(x) for x in lrs])
+        self._check(self.L.gs_render_backward_adam(
+            self.h, ctypes.byref(params), ctypes.byref(cam), _ptr(final_T), _ptr(n_contrib),
+            _ptr(dloss_dimage), ctypes.byref(grads), ctypes.byref(exp_avg), ctypes.byref(exp_avg_sq),
+            lr, float(beta1), float(beta2), float(eps), int(step), _stream(stream)))
 
     def profile_enable(self, on=True):
         self._check(self.L.gs_profile_enable(self.h, 1 if on else 0))

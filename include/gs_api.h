@@ -165,6 +165,25 @@ gs_status gs_render_backward(gs_ctx *ctx, const gs_params *params, const gs_came
                              const float *final_T, const int32_t *n_contrib,
                              const float *dloss_dimage, gs_grads *grads, void *stream);
 
+/* Steps 4 + 5 in one pass - the backward of gs_render_backward followed, in the
+ * same pass over the parameters, by the Adam step of gs_adam_step on every
+ * group: for each scalar g = grads + this view's gradient, then the Adam update
+ * with that group's learning rate; params are updated IN PLACE (the pointers in
+ * *params must be writable), m and v are updated, and grads are left zeroed.
+ * The result is bit-identical to gs_render_backward(..., grads) followed by
+ * gs_adam_step on each group, but the gradient makes no separate round trip
+ * through memory ([DR] section "From a pixel error back to a quaternion":
+ * every group updated by Adam with its own learning rate). lr is a HOST array
+ * of 5 learning rates in the order means, log_scales, quats, opacity_logits,
+ * sh; exp_avg and exp_avg_sq hold the first and second moments in the
+ * parameter layout. Errors as gs_render_backward, plus GS_ERR_INVALID_ARG for
+ * a NULL moment pointer, step < 1 or betas outside [0, 1). */
+gs_status gs_render_backward_adam(gs_ctx *ctx, const gs_params *params, const gs_camera *cam,
+                                  const float *final_T, const int32_t *n_contrib,
+                                  const float *dloss_dimage, gs_grads *grads, gs_grads *exp_avg,
+                                  gs_grads *exp_avg_sq, const float *lr, float beta1, float beta2,
+                                  float eps, int32_t step, void *stream);
+
 /* Step 5 - fused Adam over one flat float32 buffer of `count` scalars
  * ([GS] Adam paragraph after "Proving the blame is right"; [DR] per-group
  * learning rates): m = b1 m + (1-b1) g; v = b2 v + (1-b2) g^2;
@@ -181,9 +200,11 @@ gs_status gs_adam_step(float *param, float *grad, float *m, float *v, int64_t co
  * events, returns per-stage totals accumulated since the previous read and
  * resets them. Each output is a HOST array of GS_NUM_STAGES entries (any may
  * be NULL): ms = summed kernel time, launches = launches, work = the units
- * processed (Gaussians for the per-Gaussian stages, entries for the sort
- * stages, evaluated (pixel, Gaussian) pairs for the blends, pixels for the
- * loss). Adam takes no context and is not profiled here. */
+ * processed (Gaussians for the per-Gaussian stages - n_pad for the fused
+ * backward + Adam pass -, entries x passes for the sort, entries for the
+ * duplication and ranges, evaluated (pixel, Gaussian) pairs for the blends,
+ * pixels for the loss). gs_adam_step takes no context and is not profiled
+ * here. */
 typedef enum {
   GS_STAGE_PREPROCESS = 0,
   GS_STAGE_SCAN = 1,
@@ -194,7 +215,8 @@ typedef enum {
   GS_STAGE_LOSS = 6,
   GS_STAGE_BLEND_BACKWARD = 7,
   GS_STAGE_PREPROCESS_BACKWARD = 8,
-  GS_NUM_STAGES = 9
+  GS_STAGE_BACKWARD_ADAM = 9, /* the fused projection backward + Adam pass */
+  GS_NUM_STAGES = 10
 } gs_stage;
 
 gs_status gs_profile_enable(gs_ctx *ctx, int32_t enabled);
