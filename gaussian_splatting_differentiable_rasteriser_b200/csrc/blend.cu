@@ -8,63 +8,84 @@
 // training" study notes (bailiping.com), slide on alpha (cap 0.99, skip below
 // 1/255, stop when nearly opaque) and slide "r is the RGB loss gradient".
 //
-// B200 design. One CTA of 256 threads per 16x16 tile, one pixel per thread,
-// each warp an 8x4 pixel block (compact blocks let the backward skip whole
-// warps a small Gaussian does not reach). The tile's sorted Gaussians are
-// gathered from the 48-byte screen records in batches of 256 into shared
-// memory, already rescaled for the exponent: alpha = min(0.99, 2^p) with
-//     p = A' dx^2 + B' dx dy + C' dy^2 + log2(o),
-//     A' = -A log2(e) / 2, B' = -B log2(e), C' = -C log2(e) / 2,
-// so each (pixel, Gaussian) pair costs 7 FP32 ops, one MUFU.EX2 and a min.
-// The forward stops a CTA when every pixel is saturated (syncthreads_count).
+// B200 design. One CTA of 256 threads per 16x16 tile, one pixel per thread;
+// each warp owns an 8x4 pixel block and walks the tile's list on its own (no
+// CTA-wide barrier: a warp whose pixels are saturated stops while its
+// neighbours go on). The list is consumed 32 entries at a time: lane l gathers
+// entry base + l (its 48-byte screen record, prefetched one chunk ahead into
+// registers), tests the record's alpha >= 1/255 box against the warp's block,
+// and a ballot compacts the survivors into the warp's slice of shared memory.
+// The pixel loop then visits only survivors, so a Gaussian that cannot reach
+// the block costs 1/32 of a warp instruction slot instead of a full
+// evaluation; the box is conservative, so results do not change.
+// Per evaluated pair: alpha = min(0.99, 2^p) with the exponent-ready conic of
+// the screen record (7 FP32 ops and one MUFU.EX2).
 // The forward stores only the final T and n_contrib per pixel; the backward
 // re-walks back to front from each pixel's last contributor, recovers T by
-// dividing by (1 - alpha), and keeps a single running scalar g . S (S = colour
-// already composited behind) instead of the three channels. Per pair it
-// produces 9 raw sums (w, w dx, w dy, w dx^2, w dx dy, w dy^2, dL/dc) with
+// dividing by (1 - alpha), and keeps one running scalar g . S (S = colour
+// already composited behind) instead of three channels. Per pair it forms 9
+// raw sums (w, w dx, w dy, w dx^2, w dx dy, w dy^2, dL/dc) with
 // w = dL/dalpha * o exp(-e); a warp reduce-scatter (12 shuffles instead of 45)
 // leaves the 9 warp totals in 9 lanes, which issue one coalesced group of 9
-// float32 atomics. The conic/opacity/mean2d chain of those sums is applied once
-// per Gaussian in the projection backward.
+// float32 atomics. The conic/opacity/mean2d chain of those sums is applied
+// once per Gaussian in the projection backward.
 #include "gs_kernels.cuh"
 
 namespace gs {
 
 namespace {
 
-constexpr int kBatch = 256;
+constexpr int kWarps = 8;
 
-// Shared-memory copy of one batch of Gaussians.
-struct BlendSmem {
-  float2 xy[kBatch];
-  float4 q[kBatch];    // A', B', C', log2(o)
-  float4 col[kBatch];  // r, g, b, o
-  float4 box[kBatch];  // x_lo, x_hi, y_lo, y_hi of the alpha >= 1/255 region
-  uint32_t id[kBatch];
+// Warp-private slots of the surviving Gaussians of the current chunk.
+struct WarpSlots {
+  float2 xy[32];
+  float4 q[32];    // A', B', C', log2(o)
+  float4 col[32];  // r, g, b, o
+  int pos[32];     // list position relative to the tile start
+  uint32_t id[32];
 };
 
-__device__ __forceinline__ void stage(BlendSmem& s, int slot, uint32_t gid, const Screen* screen) {
-  const Screen g = screen[gid];
-  const float u = g.a.x, v = g.a.y, A = g.a.z, B = g.a.w, C = g.b.x, o = g.b.y;
-  s.xy[slot] = make_float2(u, v);
-  s.q[slot] = make_float4(__fmul_rn(-0.5f * kLog2e, A), __fmul_rn(-kLog2e, B),
-                          __fmul_rn(-0.5f * kLog2e, C), log2f(o));
-  s.col[slot] = make_float4(g.b.z, g.b.w, g.c.x, o);
-  // o exp(-e) >= 1/255 exactly when e <= E = ln(255 o); the ellipse e <= E has the
-  // axis-aligned half-widths sqrt(2 E Sigma'_xx), sqrt(2 E Sigma'_yy), with
-  // Sigma' = conic^-1. The box is widened by 0.1% + 0.02 px so that float32
-  // rounding of the per-pixel alpha can never pass the floor outside it: a warp
-  // whose pixels all lie outside skips the Gaussian with unchanged results.
-  const float E = logf(255.0f * o);
-  float4 box = make_float4(1.0f, -1.0f, 1.0f, -1.0f);  // empty
-  const float det = A * C - B * B;
-  if (E > 0.0f && det > 0.0f) {
-    const float hx = sqrtf(2.0f * E * C / det) * 1.001f + 0.02f;
-    const float hy = sqrtf(2.0f * E * A / det) * 1.001f + 0.02f;
-    box = make_float4(u - hx, u + hx, v - hy, v + hy);
+// One gathered list entry: the screen record of its Gaussian.
+struct Entry {
+  Screen s;
+  uint32_t gid;
+  bool valid;
+};
+
+__device__ __forceinline__ uint32_t load_gid(const uint32_t* order, int j, int lo, int hi) {
+  return (j >= lo && j < hi) ? __ldg(order + j) : 0u;
+}
+
+__device__ __forceinline__ Entry load_entry(const Screen* screen, uint32_t gid, bool valid) {
+  Entry e;
+  e.valid = valid;
+  e.gid = gid;
+  if (valid) {
+    const float4* r = reinterpret_cast<const float4*>(screen + gid);
+    e.s.a = __ldg(r);
+    e.s.b = __ldg(r + 1);
+    e.s.c = __ldg(r + 2);
+  } else {
+    e.s.a = e.s.b = e.s.c = make_float4(0.f, 0.f, 0.f, 0.f);
   }
-  s.box[slot] = box;
-  s.id[slot] = gid;
+  return e;
+}
+
+// The entry's alpha >= 1/255 box meets the pixel block [bx0, bx0+7] x [by0, by0+3].
+__device__ __forceinline__ bool hits_block(const Entry& e, float bx0, float by0) {
+  const float u = e.s.a.x, v = e.s.a.y, hx = e.s.c.z, hy = e.s.c.w;
+  const float cx = fminf(fmaxf(u, bx0), bx0 + 7.0f);
+  const float cy = fminf(fmaxf(v, by0), by0 + 3.0f);
+  return e.valid && fabsf(u - cx) <= hx && fabsf(v - cy) <= hy;
+}
+
+__device__ __forceinline__ void put_slot(WarpSlots& w, int slot, const Entry& e, int pos) {
+  w.xy[slot] = make_float2(e.s.a.x, e.s.a.y);
+  w.q[slot] = make_float4(e.s.a.z, e.s.a.w, e.s.b.x, e.s.b.y);
+  w.col[slot] = make_float4(e.s.b.z, e.s.b.w, e.s.c.x, e.s.c.y);
+  w.pos[slot] = pos;
+  w.id[slot] = e.gid;
 }
 
 // 2^x in one MUFU instruction (flushes results below 2^-126 to 0, far under
@@ -82,12 +103,6 @@ __device__ __forceinline__ float power2(const float4 q, float dx, float dy) {
   return __fmaf_rn(s, dx, t);
 }
 
-// True when the Gaussian's alpha >= 1/255 box misses the warp's 8x4 pixel block.
-__device__ __forceinline__ bool misses_block(const float4 box, float bx0, float bx1, float by0,
-                                             float by1) {
-  return box.y < bx0 || box.x > bx1 || box.w < by0 || box.z > by1;
-}
-
 // Adds this warp's count to *pairs (profiling builds of the kernels only).
 __device__ __forceinline__ void count_pairs(unsigned long long* pairs, unsigned c) {
   unsigned long long v = c;
@@ -98,51 +113,58 @@ __device__ __forceinline__ void count_pairs(unsigned long long* pairs, unsigned 
 
 template <bool kCount>
 __global__ void __launch_bounds__(256) blend_forward_kernel(BlendArgs a) {
-  __shared__ BlendSmem sm;
+  __shared__ WarpSlots slots[kWarps];
   const int tile = blockIdx.x;
   const int tx = tile % a.cam.tiles_x, ty = tile / a.cam.tiles_x;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  WarpSlots& ws = slots[warp];
   int lx, ly;
   tile_pixel(threadIdx.x, lx, ly);
   const int px = tx * kTile + lx, py = ty * kTile + ly;
   const bool inside = px < a.cam.width && py < a.cam.height;
-  const uint2 range = a.ranges[tile];
-  const int n = static_cast<int>(range.y - range.x);
   const float fx = static_cast<float>(px), fy = static_cast<float>(py);
-
-  // this warp's 8x4 pixel block
-  const float bx0 = static_cast<float>(tx * kTile + ((threadIdx.x >> 5) & 1) * 8);
-  const float by0 = static_cast<float>(ty * kTile + (threadIdx.x >> 6) * 4);
-  const float bx1 = bx0 + 7.0f, by1 = by0 + 3.0f;
+  const float bx0 = static_cast<float>(tx * kTile + (warp & 1) * 8);
+  const float by0 = static_cast<float>(ty * kTile + (warp >> 1) * 4);
+  const uint2 range = a.ranges[tile];
+  const int beg = static_cast<int>(range.x), end = static_cast<int>(range.y);
+  const unsigned lt = (1u << lane) - 1u;
 
   float T = 1.0f, C0 = 0.0f, C1 = 0.0f, C2 = 0.0f;
   int last = 0;
   bool done = !inside;
   unsigned evals = 0;
-  for (int b = 0; b < n; b += kBatch) {
-    if (__syncthreads_count(!done) == 0) break;
-    const int k = b + threadIdx.x;
-    if (k < n) stage(sm, threadIdx.x, a.order[range.x + k], a.screen);
-    __syncthreads();
-    const int cnt = min(kBatch, n - b);
-    if (__all_sync(0xffffffffu, done)) continue;  // this warp is saturated
-    for (int j = 0; j < cnt; ++j) {
-      if ((j & 31) == 31 && __all_sync(0xffffffffu, done)) break;
-      if (misses_block(sm.box[j], bx0, bx1, by0, by1)) continue;
-      if (kCount) evals += !done;
-      const float2 xy = sm.xy[j];
-      const float p = power2(sm.q[j], fx - xy.x, fy - xy.y);
+
+  // two-stage prefetch: the order entries of chunk i+2, the records of chunk i+1
+  uint32_t gid_next = load_gid(a.order, beg + lane, beg, end);
+  Entry nxt = load_entry(a.screen, gid_next, beg + lane < end);
+  gid_next = load_gid(a.order, beg + 32 + lane, beg, end);
+  for (int base = beg; base < end; base += 32) {
+    if (__all_sync(0xffffffffu, done)) break;
+    const Entry cur = nxt;
+    nxt = load_entry(a.screen, gid_next, base + 32 + lane < end);
+    gid_next = load_gid(a.order, base + 64 + lane, beg, end);
+    const bool keep = hits_block(cur, bx0, by0);
+    const unsigned mask = __ballot_sync(0xffffffffu, keep);
+    if (keep) put_slot(ws, __popc(mask & lt), cur, base + lane - beg);
+    __syncwarp();
+    const int cnt = __popc(mask);
+    for (int k = 0; k < cnt; ++k) {
+      const float2 xy = ws.xy[k];
+      const float p = power2(ws.q[k], fx - xy.x, fy - xy.y);
       const float alpha = fminf(kAlphaMax, fast_exp2(p));
+      if (kCount) evals += !done;
       if (!done && alpha >= kAlphaMin) {
-        const float4 c = sm.col[j];
+        const float4 c = ws.col[k];
         const float w = alpha * T;
         C0 = __fmaf_rn(w, c.x, C0);
         C1 = __fmaf_rn(w, c.y, C1);
         C2 = __fmaf_rn(w, c.z, C2);
         T = T * (1.0f - alpha);
-        last = b + j + 1;
+        last = ws.pos[k] + 1;
         done = T < kTMin;
       }
     }
+    __syncwarp();  // the slots are rewritten by the next chunk
   }
   if (inside) {
     const int64_t hw = static_cast<int64_t>(a.cam.width) * a.cam.height;
@@ -201,17 +223,21 @@ __device__ __forceinline__ float warp_reduce_scatter9(const float (&v)[9], int l
 
 template <bool kCount>
 __global__ void __launch_bounds__(256) blend_backward_kernel(BlendArgs a) {
-  __shared__ BlendSmem sm;
-  __shared__ int s_max_last;
+  __shared__ WarpSlots slots[kWarps];
   const int tile = blockIdx.x;
   const int tx = tile % a.cam.tiles_x, ty = tile / a.cam.tiles_x;
-  const int lane = threadIdx.x & 31;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  WarpSlots& ws = slots[warp];
   int lx, ly;
   tile_pixel(threadIdx.x, lx, ly);
   const int px = tx * kTile + lx, py = ty * kTile + ly;
   const bool inside = px < a.cam.width && py < a.cam.height;
-  const uint2 range = a.ranges[tile];
   const float fx = static_cast<float>(px), fy = static_cast<float>(py);
+  const float bx0 = static_cast<float>(tx * kTile + (warp & 1) * 8);
+  const float by0 = static_cast<float>(ty * kTile + (warp >> 1) * 4);
+  const uint2 range = a.ranges[tile];
+  const int beg = static_cast<int>(range.x);
+  const unsigned lt = (1u << lane) - 1u;
 
   const int64_t hw = static_cast<int64_t>(a.cam.width) * a.cam.height;
   const int64_t pix = static_cast<int64_t>(py) * a.cam.width + px;
@@ -226,21 +252,11 @@ __global__ void __launch_bounds__(256) blend_backward_kernel(BlendArgs a) {
   }
   // g . S with S the colour composited behind the current Gaussian; starts at T_final bg.
   float gS = T * (g0 * a.cam.bg[0] + g1 * a.cam.bg[1] + g2 * a.cam.bg[2]);
-
-  if (threadIdx.x == 0) s_max_last = 0;
-  __syncthreads();
-  int wmax = last;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) wmax = max(wmax, __shfl_xor_sync(0xffffffffu, wmax, o));
-  if (lane == 0) atomicMax(&s_max_last, wmax);
-  __syncthreads();
   // n_contrib comes from the caller: never walk past the tile's own list.
-  const int max_last = min(s_max_last, static_cast<int>(range.y - range.x));
-
-  const float bx0 = static_cast<float>(tx * kTile + ((threadIdx.x >> 5) & 1) * 8);
-  const float by0 = static_cast<float>(ty * kTile + (threadIdx.x >> 6) * 4);
-  const float bx1 = bx0 + 7.0f, by1 = by0 + 3.0f;
-  const int warp_last = wmax;  // no lane of this warp blends anything at or after it
+  int wlast = last;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) wlast = max(wlast, __shfl_xor_sync(0xffffffffu, wlast, o));
+  const int top = beg + max(0, min(wlast, static_cast<int>(range.y - range.x)));  // exclusive
 
   // Which raw sum this lane holds after the reduce-scatter.
   const int red_idx = ((lane >> 1) & 1) * 8 + ((lane >> 2) & 1) * 4 + ((lane >> 3) & 1) * 2 +
@@ -248,21 +264,29 @@ __global__ void __launch_bounds__(256) blend_backward_kernel(BlendArgs a) {
   const bool red_writer = !(lane & 1) && red_idx < 9;
   unsigned evals = 0;
 
-  for (int end = max_last; end > 0; end -= kBatch) {
-    const int start = max(0, end - kBatch);
-    __syncthreads();  // the previous batch is no longer read
-    const int k = start + threadIdx.x;
-    if (k < end) stage(sm, threadIdx.x, a.order[range.x + k], a.screen);
-    __syncthreads();
-    for (int j = min(end, warp_last) - 1; j >= start; --j) {
-      const int slot = j - start;
-      if (misses_block(sm.box[slot], bx0, bx1, by0, by1)) continue;
-      const float2 xy = sm.xy[slot];
+  // Chunks walk down from the top; lane l takes entry hi - 1 - l, so ballot
+  // order (lane order) is descending list order.
+  uint32_t gid_next = load_gid(a.order, top - 1 - lane, beg, top);
+  Entry nxt = load_entry(a.screen, gid_next, top - 1 - lane >= beg);
+  gid_next = load_gid(a.order, top - 33 - lane, beg, top);
+  for (int hi = top; hi > beg; hi -= 32) {
+    const Entry cur = nxt;
+    const int j_cur = hi - 1 - lane;
+    nxt = load_entry(a.screen, gid_next, j_cur - 32 >= beg);
+    gid_next = load_gid(a.order, j_cur - 64, beg, top);
+    const bool keep = j_cur >= beg && hits_block(cur, bx0, by0);
+    const unsigned mask = __ballot_sync(0xffffffffu, keep);
+    if (keep) put_slot(ws, __popc(mask & lt), cur, j_cur - beg);
+    __syncwarp();
+    const int cnt = __popc(mask);
+    for (int k = 0; k < cnt; ++k) {
+      const int pos = ws.pos[k];
+      const float2 xy = ws.xy[k];
       const float dx = fx - xy.x, dy = fy - xy.y;
-      const float raw = fast_exp2(power2(sm.q[slot], dx, dy));
+      const float raw = fast_exp2(power2(ws.q[k], dx, dy));
       const float alpha = fminf(kAlphaMax, raw);
-      const bool contrib = j < last && alpha >= kAlphaMin;
-      if (kCount && j < last) ++evals;
+      const bool contrib = pos < last && alpha >= kAlphaMin;
+      if (kCount && pos < last) ++evals;
       if (!__any_sync(0xffffffffu, contrib)) continue;
       float v[9];
 #pragma unroll
@@ -270,7 +294,7 @@ __global__ void __launch_bounds__(256) blend_backward_kernel(BlendArgs a) {
       if (contrib) {
         const float rcp = __fdividef(1.0f, 1.0f - alpha);
         T = T * rcp;  // transmittance in front of this Gaussian
-        const float4 c = sm.col[slot];
+        const float4 c = ws.col[k];
         const float gc = __fmaf_rn(g2, c.z, __fmaf_rn(g1, c.y, g0 * c.x));
         const float dalpha = __fmaf_rn(T, gc, -gS * rcp);  // dI/dalpha = T c - S / (1 - alpha)
         const float aT = alpha * T;
@@ -288,8 +312,9 @@ __global__ void __launch_bounds__(256) blend_backward_kernel(BlendArgs a) {
         v[5] = wdy * dy;
       }
       const float tot = warp_reduce_scatter9(v, lane);
-      if (red_writer) atomicAdd(a.sgrad + static_cast<int64_t>(sm.id[slot]) * kGradStride + red_idx, tot);
+      if (red_writer) atomicAdd(a.sgrad + static_cast<int64_t>(ws.id[k]) * kGradStride + red_idx, tot);
     }
+    __syncwarp();
   }
   if (kCount) count_pairs(a.pairs, evals);
 }

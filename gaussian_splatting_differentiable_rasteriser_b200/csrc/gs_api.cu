@@ -184,11 +184,11 @@ __global__ void unpack_preprocess_kernel(const gs::Screen* screen, const float* 
     mean2d[2 * i + 1] = s.a.y;
   }
   if (conic) {
-    conic[3 * i] = s.a.z;
-    conic[3 * i + 1] = s.a.w;
-    conic[3 * i + 2] = s.b.x;
+    conic[3 * i] = gs::conic_A(s);
+    conic[3 * i + 1] = gs::conic_B(s);
+    conic[3 * i + 2] = gs::conic_C(s);
   }
-  if (opacity) opacity[i] = s.b.y;
+  if (opacity) opacity[i] = gs::screen_opacity(s);
   if (rgb) {
     rgb[3 * i] = s.b.z;
     rgb[3 * i + 1] = s.b.w;

@@ -16,13 +16,26 @@ constexpr double kRadiusSigmas = 3.0;   // sqrt(2 * 4.5): the falloff cut E_CUT 
 constexpr float kLog2e = 1.4426950408889634f;
 
 // Per-Gaussian screen state written by the preprocess and gathered by the
-// blend kernels: 48 bytes, three 16-byte vectors.
-//   a = (u, v, A, B)   mean2d and the first two conic entries
-//   b = (C, o, r, g)   last conic entry, opacity, red, green
-//   c = (blue, depth, 0, 0)
+// blend kernels: 48 bytes, three 16-byte vectors, with the conic and opacity
+// already in the form the exponent needs: alpha = min(0.99, 2^p),
+//   p = A' dx^2 + B' dx dy + C' dy^2 + log2(o),
+//   A' = -A log2(e) / 2, B' = -B log2(e), C' = -C log2(e) / 2
+// for the conic (A, B, C) (e = A dx^2 / 2 + B dx dy + C dy^2 / 2).
+//   a = (u, v, A', B')
+//   b = (C', log2(o), r, g)
+//   c = (blue, o, hx, hy)   hx, hy: conservative half-widths of the box holding
+//                           every pixel where o exp(-e) >= 1/255 (negative if none)
 struct alignas(16) Screen {
   float4 a, b, c;
 };
+
+// Scale between the natural conic entries and the stored exponent form.
+constexpr float kConicToExpAC = -0.5f * 1.4426950408889634f;  // A' = A * this (also C)
+constexpr float kConicToExpB = -1.4426950408889634f;          // B' = B * this
+__device__ __forceinline__ float conic_A(const Screen& s) { return s.a.z / kConicToExpAC; }
+__device__ __forceinline__ float conic_B(const Screen& s) { return s.a.w / kConicToExpB; }
+__device__ __forceinline__ float conic_C(const Screen& s) { return s.b.x / kConicToExpAC; }
+__device__ __forceinline__ float screen_opacity(const Screen& s) { return s.c.y; }
 
 // Raw per-Gaussian screen-gradient sums accumulated by the blend backward
 // (12 floats, 9 used). With w = dL/dalpha * o exp(-e) summed over pixels:

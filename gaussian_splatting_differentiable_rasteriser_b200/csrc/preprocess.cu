@@ -130,10 +130,23 @@ __global__ void __launch_bounds__(256) preprocess_kernel(PreprocessArgs a) {
             }
             rgb[ch] = col;
           }
+          // conic (cc, -cb, ca) / det in the exponent form, and the box of the
+          // alpha >= 1/255 region: o exp(-e) >= 1/255 exactly when e <= E =
+          // ln(255 o), an ellipse with axis-aligned half-widths sqrt(2 E a),
+          // sqrt(2 E c) (a, c the diagonal of Sigma'), widened by 0.1% + 0.02 px so
+          // float32 rounding of the per-pixel alpha never passes the floor outside.
+          const double l2e = 1.4426950408889634;
+          const double E = log(255.0 * static_cast<double>(opacity));
+          float hx = -1.0f, hy = -1.0f;
+          if (E > 0.0) {
+            hx = static_cast<float>(sqrt(2.0 * E * ca) * 1.001 + 0.02);
+            hy = static_cast<float>(sqrt(2.0 * E * cc) * 1.001 + 0.02);
+          }
           s.a = make_float4(static_cast<float>(u), static_cast<float>(v),
-                            static_cast<float>(cc / det), static_cast<float>(-cb / det));
-          s.b = make_float4(static_cast<float>(ca / det), opacity, rgb[0], rgb[1]);
-          s.c = make_float4(rgb[2], depth, 0.0f, 0.0f);
+                            static_cast<float>(-0.5 * l2e * cc / det), static_cast<float>(l2e * cb / det));
+          s.b = make_float4(static_cast<float>(-0.5 * l2e * ca / det),
+                            static_cast<float>(log2(static_cast<double>(opacity))), rgb[0], rgb[1]);
+          s.c = make_float4(rgb[2], opacity, hx, hy);
         }
       }
     }

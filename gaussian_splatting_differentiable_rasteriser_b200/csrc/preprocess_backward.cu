@@ -48,7 +48,7 @@ __device__ __forceinline__ void geometry_grad(const PreprocessBwdArgs& a, int64_
   const float4* sg4 = reinterpret_cast<const float4*>(a.sgrad + i * kGradStride);
   const float4 r0 = sg4[0], r1 = sg4[1], r2 = sg4[2];
   const Screen scr = a.screen[i];
-  const float A = scr.a.z, B = scr.a.w, C = scr.b.x, o = scr.b.y;
+  const float A = conic_A(scr), B = conic_B(scr), C = conic_C(scr), o = screen_opacity(scr);
   const uint8_t clamped = a.clamped[i];
 
   // Screen-space gradient from the raw sums (w = dL/dalpha * o exp(-e)).
@@ -301,7 +301,7 @@ __global__ void screen_grads_kernel(const Screen* screen, const float* sgrad, in
   if (i >= n) return;
   const float* r = sgrad + i * kGradStride;
   const Screen s = screen[i];
-  const float A = s.a.z, B = s.a.w, C = s.b.x, o = s.b.y;
+  const float A = conic_A(s), B = conic_B(s), C = conic_C(s), o = screen_opacity(s);
   float* d = out + i * 9;
   d[0] = A * r[1] + B * r[2];
   d[1] = B * r[1] + C * r[2];
