@@ -232,66 +232,129 @@ __global__ void __launch_bounds__(256) preprocess_backward_kernel(PreprocessBwdA
 // Per scalar: g = accumulated gradient + this view's gradient, then the update
 // of adam_one; the gradient buffer is left zeroed. Bit-identical to the
 // accumulate kernel followed by the standalone Adam kernel.
+//
+// Compute, then stream: a CTA owns 128 consecutive Gaussians. Phase 1 (one
+// thread per Gaussian) computes the view gradient of the 11 geometric scalars
+// and what the 48 SH gradients need (masked dL/dcolour and Y_k) into shared
+// memory. Phase 2 streams Adam over the CTA's 59 planes x 128 Gaussians: each
+// plane segment is 512 contiguous bytes, handled as 32 float4 units, four units
+// per thread per round with all 16 loads issued before any store, so many
+// loads are in flight per thread (the kernel is bound by HBM, not by math).
+constexpr int kFusedBlock = 128;
+constexpr int kGeomPlanes = 11;  // means 3, log-scales 3, quats 4, opacity logit 1
+
+struct FusedSmem {
+  float geom[kGeomPlanes][kFusedBlock];  // view gradient of the geometric scalars
+  float drgb[3][kFusedBlock];            // masked dL/dcolour (0 when invisible)
+  float Y[16][kFusedBlock];              // SH basis at the view direction
+};
+
 template <int kDeg>
-__global__ void __launch_bounds__(256) preprocess_backward_adam_kernel(PreprocessBwdArgs a, FusedAdamArgs f) {
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (i >= a.n_pad) return;
+__global__ void __launch_bounds__(kFusedBlock) preprocess_backward_adam_kernel(PreprocessBwdArgs a,
+                                                                              FusedAdamArgs f) {
+  __shared__ __align__(16) FusedSmem sm;
+  const int t = threadIdx.x;
+  const int64_t i0 = static_cast<int64_t>(blockIdx.x) * kFusedBlock;
   const int64_t np = a.n_pad;
-  const bool visible = i < a.n && a.touched[i] != 0;
-  GaussGrad g;
-  if (visible) {
-    geometry_grad(a, i, g);
-  } else {
-#pragma unroll
-    for (int c = 0; c < 3; ++c) g.dp[c] = g.dls[c] = g.drgb[c] = 0.f;
-#pragma unroll
-    for (int c = 0; c < 4; ++c) g.dq[c] = 0.f;
-    g.dlogit = 0.f;
-    g.vx = g.vy = g.vz = 0.f;
-    g.idl = 0.f;
-  }
   constexpr int nk = (kDeg + 1) * (kDeg + 1);
-  float Yk[16];
-  sh_basis(kDeg, g.vx, g.vy, g.vz, Yk);
-  float wsum[16];
+
+  // Phase 1: this view's gradient of Gaussian i0 + t.
+  {
+    const int64_t i = i0 + t;
+    const bool visible = i < a.n && a.touched[i] != 0;
+    if (visible) {
+      GaussGrad g;
+      geometry_grad(a, i, g);
+      float Yk[16];
+      sh_basis(kDeg, g.vx, g.vy, g.vz, Yk);
+      float wsum[16];
 #pragma unroll
-  for (int k = 0; k < 16; ++k) wsum[k] = 0.f;
-  // SH first: the view-direction term of the position needs their old values.
+      for (int k = 0; k < 16; ++k) wsum[k] = 0.f;
 #pragma unroll
-  for (int ch = 0; ch < 3; ++ch) {
-    const int64_t base = static_cast<int64_t>(ch) * a.sh_k * np + i;
-    const float dc = g.drgb[ch];
+      for (int ch = 0; ch < 3; ++ch) {
+        if (g.drgb[ch] == 0.f) continue;
+        const float* shc = a.sh + static_cast<int64_t>(ch) * a.sh_k * np + i;
 #pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      if (k >= a.sh_k) break;
-      const int64_t o = base + static_cast<int64_t>(k) * np;
-      float p = f.p[4][o], gr = f.g[4][o], m = f.m[4][o], v = f.v[4][o];
-      if (k < nk && dc != 0.f) {
-        wsum[k] = __fmaf_rn(dc, p, wsum[k]);
-        gr = __fmaf_rn(dc, Yk[k], gr);
+        for (int k = 0; k < nk; ++k)
+          wsum[k] = __fmaf_rn(g.drgb[ch], shc[static_cast<int64_t>(k) * np], wsum[k]);
       }
-      adam_one(p, gr, m, v, f.s[4]);
-      f.p[4][o] = p;
-      f.g[4][o] = gr;
-      f.m[4][o] = m;
-      f.v[4][o] = v;
+      add_view_dir_term<kDeg>(g, wsum);
+      const float geom[kGeomPlanes] = {g.dp[0], g.dp[1], g.dp[2], g.dls[0], g.dls[1], g.dls[2],
+                                       g.dq[0], g.dq[1], g.dq[2], g.dq[3], g.dlogit};
+#pragma unroll
+      for (int j = 0; j < kGeomPlanes; ++j) sm.geom[j][t] = geom[j];
+#pragma unroll
+      for (int ch = 0; ch < 3; ++ch) sm.drgb[ch][t] = g.drgb[ch];
+#pragma unroll
+      for (int k = 0; k < 16; ++k) sm.Y[k][t] = k < nk ? Yk[k] : 0.f;
+    } else {
+#pragma unroll
+      for (int j = 0; j < kGeomPlanes; ++j) sm.geom[j][t] = 0.f;
+#pragma unroll
+      for (int ch = 0; ch < 3; ++ch) sm.drgb[ch][t] = 0.f;
+#pragma unroll
+      for (int k = 0; k < 16; ++k) sm.Y[k][t] = 0.f;
     }
   }
-  if (visible) add_view_dir_term<kDeg>(g, wsum);
-  const float view[11] = {g.dp[0],  g.dp[1],  g.dp[2],  g.dls[0], g.dls[1], g.dls[2],
-                          g.dq[0],  g.dq[1],  g.dq[2],  g.dq[3],  g.dlogit};
+  __syncthreads();
+
+  // Phase 2: Adam over planes x float4 columns of this CTA's Gaussians.
+  const int64_t rem = np - i0;
+  const int cols = static_cast<int>((rem < kFusedBlock ? rem : kFusedBlock) / 4);  // n_pad % 4 == 0
+  const int planes = kGeomPlanes + 3 * a.sh_k;
+  const int units = planes * (kFusedBlock / 4);
+  for (int u0 = t; u0 < units; u0 += 4 * kFusedBlock) {
+    float4 P[4], G[4], M[4], V[4];
+    int64_t off[4];
+    int plane[4], col[4], grp[4];
+    bool ok[4];
 #pragma unroll
-  for (int j = 0; j < 11; ++j) {
-    const int grp = j < 3 ? 0 : (j < 6 ? 1 : (j < 10 ? 2 : 3));
-    const int c = j < 3 ? j : (j < 6 ? j - 3 : (j < 10 ? j - 6 : 0));
-    const int64_t o = c * np + i;
-    float p = f.p[grp][o], gr = f.g[grp][o], m = f.m[grp][o], v = f.v[grp][o];
-    gr += view[j];
-    adam_one(p, gr, m, v, f.s[grp]);
-    f.p[grp][o] = p;
-    f.g[grp][o] = gr;
-    f.m[grp][o] = m;
-    f.v[grp][o] = v;
+    for (int r = 0; r < 4; ++r) {
+      const int u = u0 + r * kFusedBlock;
+      const int pl = u / (kFusedBlock / 4);
+      plane[r] = pl;
+      col[r] = u % (kFusedBlock / 4);
+      ok[r] = u < units && col[r] < cols;
+      int c;
+      if (pl < 3) { grp[r] = 0; c = pl; }
+      else if (pl < 6) { grp[r] = 1; c = pl - 3; }
+      else if (pl < 10) { grp[r] = 2; c = pl - 6; }
+      else if (pl < 11) { grp[r] = 3; c = 0; }
+      else { grp[r] = 4; c = pl - kGeomPlanes; }
+      off[r] = static_cast<int64_t>(c) * np + i0 + 4 * col[r];
+      if (ok[r]) {
+        P[r] = *reinterpret_cast<const float4*>(f.p[grp[r]] + off[r]);
+        G[r] = *reinterpret_cast<const float4*>(f.g[grp[r]] + off[r]);
+        M[r] = *reinterpret_cast<const float4*>(f.m[grp[r]] + off[r]);
+        V[r] = *reinterpret_cast<const float4*>(f.v[grp[r]] + off[r]);
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      if (!ok[r]) continue;
+      const int pl = plane[r];
+      float* p4 = &P[r].x;
+      float* g4 = &G[r].x;
+      float* m4 = &M[r].x;
+      float* v4 = &V[r].x;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int j = 4 * col[r] + e;
+        if (pl < kGeomPlanes) {
+          g4[e] += sm.geom[pl][j];
+        } else {
+          const int sp = pl - kGeomPlanes;
+          const int ch = sp / a.sh_k, k = sp % a.sh_k;
+          const float dc = sm.drgb[ch][j];
+          if (k < nk && dc != 0.f) g4[e] = __fmaf_rn(dc, sm.Y[k][j], g4[e]);
+        }
+        adam_one(p4[e], g4[e], m4[e], v4[e], f.s[grp[r]]);
+      }
+      *reinterpret_cast<float4*>(f.p[grp[r]] + off[r]) = P[r];
+      *reinterpret_cast<float4*>(f.g[grp[r]] + off[r]) = G[r];
+      *reinterpret_cast<float4*>(f.m[grp[r]] + off[r]) = M[r];
+      *reinterpret_cast<float4*>(f.v[grp[r]] + off[r]) = V[r];
+    }
   }
 }
 
@@ -331,12 +394,12 @@ cudaError_t launch_preprocess_backward(const PreprocessBwdArgs& a, cudaStream_t 
 cudaError_t launch_preprocess_backward_adam(const PreprocessBwdArgs& a, const FusedAdamArgs& f,
                                            cudaStream_t st) {
   if (a.n_pad == 0) return cudaSuccess;
-  const unsigned grid = static_cast<unsigned>((a.n_pad + 255) / 256);
+  const unsigned grid = static_cast<unsigned>((a.n_pad + kFusedBlock - 1) / kFusedBlock);
   switch (a.active_degree) {
-    case 0: preprocess_backward_adam_kernel<0><<<grid, 256, 0, st>>>(a, f); break;
-    case 1: preprocess_backward_adam_kernel<1><<<grid, 256, 0, st>>>(a, f); break;
-    case 2: preprocess_backward_adam_kernel<2><<<grid, 256, 0, st>>>(a, f); break;
-    default: preprocess_backward_adam_kernel<3><<<grid, 256, 0, st>>>(a, f); break;
+    case 0: preprocess_backward_adam_kernel<0><<<grid, kFusedBlock, 0, st>>>(a, f); break;
+    case 1: preprocess_backward_adam_kernel<1><<<grid, kFusedBlock, 0, st>>>(a, f); break;
+    case 2: preprocess_backward_adam_kernel<2><<<grid, kFusedBlock, 0, st>>>(a, f); break;
+    default: preprocess_backward_adam_kernel<3><<<grid, kFusedBlock, 0, st>>>(a, f); break;
   }
   return cudaGetLastError();
 }

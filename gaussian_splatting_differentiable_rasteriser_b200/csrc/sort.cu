@@ -123,6 +123,7 @@ struct OnesweepArgs {
   uint32_t* vals_out;
   int64_t n;
   int shift;
+  int digit_bits;                 // significant bits of this pass's digit (1..8)
   const uint32_t* digit_offsets;  // [256] for this pass
   uint32_t* status;               // [tiles][256] for this pass, zeroed
   uint32_t* ticket;               // zeroed
@@ -176,12 +177,20 @@ __global__ void __launch_bounds__(kSortThreads) onesweep_kernel(OnesweepArgs a) 
     }
   }
   // Stable rank inside the warp: items in entry order, lanes in lane order.
+  // Lanes holding the same digit are found with one ballot per digit bit.
 #pragma unroll
   for (int j = 0; j < kSortItems; ++j) {
     const int64_t idx = base + warp * (kSortItems * 32) + j * 32 + lane;
     const bool valid = idx < a.n;
     const uint32_t d = static_cast<uint32_t>(key[j] >> a.shift) & 0xffu;
-    const uint32_t peers = __match_any_sync(0xffffffffu, valid ? d : (0x100u | lane));
+    uint32_t peers = __ballot_sync(0xffffffffu, valid);
+#pragma unroll
+    for (int bit = 0; bit < 8; ++bit) {
+      if (bit >= a.digit_bits) break;
+      const bool on = (d >> bit) & 1u;
+      const uint32_t vote = __ballot_sync(0xffffffffu, on);
+      peers &= on ? vote : ~vote;
+    }
     const uint32_t b = valid ? s_whist[warp][d] : 0u;
     __syncwarp();
     if (valid && lane == __ffs(peers) - 1) s_whist[warp][d] = b + __popc(peers);
@@ -216,25 +225,42 @@ __global__ void __launch_bounds__(kSortThreads) onesweep_kernel(OnesweepArgs a) 
   for (int k = 0; k < warp; ++k) before += s_wsum[k];
   s_start[d] = before + v - count;
 
-  // Decoupled look-back over earlier CTAs for this digit; every wait is bounded.
+  // Decoupled look-back over earlier CTAs for this digit, 8 predecessors per
+  // round (their status words are loaded together, so a long run of
+  // aggregate-only predecessors costs one memory latency per 8, not per CTA).
+  // Every wait is bounded.
   uint32_t excl = 0;
   if (tile > 0) {
     int64_t t = static_cast<int64_t>(tile) - 1;
     int spins = 0;
     while (t >= 0) {
-      const uint32_t s = ld_relaxed(&a.status[t * kRadix + d]);
-      const uint32_t flag = s & ~kValueMask;
-      if (flag == 0u) {
+      uint32_t w[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        w[k] = (t - k >= 0) ? ld_relaxed(&a.status[(t - k) * kRadix + d]) : kFlagPrefix;
+      int used = 0;
+      bool stop = false, blocked = false;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        if (stop || blocked) continue;
+        const uint32_t flag = w[k] & ~kValueMask;
+        if (flag == 0u) {
+          blocked = true;
+          continue;
+        }
+        excl += w[k] & kValueMask;
+        ++used;
+        if (flag == kFlagPrefix) stop = true;
+      }
+      if (stop) break;
+      t -= used;
+      if (blocked) {
         if (++spins > kLookbackSpinLimit) {
           record_error(a.err, kErrLookbackTimeout);
           break;
         }
-        __nanosleep(64);
-        continue;
+        __nanosleep(32);
       }
-      excl += s & kValueMask;
-      if (flag == kFlagPrefix) break;
-      --t;
     }
     st_relaxed(&st[d], kFlagPrefix | (excl + count));
   }
@@ -316,6 +342,7 @@ cudaError_t launch_sort(const SortPlan& plan, const SortBuffers& b, int* out_buf
     o.vals_out = b.vals[cur ^ 1];
     o.n = plan.n;
     o.shift = 8 * p;
+    o.digit_bits = std::min(8, plan.key_bits - 8 * p);
     o.digit_offsets = b.offsets + p * kRadix;
     o.status = b.status + static_cast<int64_t>(p) * plan.tiles * kRadix;
     o.ticket = b.counters + p;
