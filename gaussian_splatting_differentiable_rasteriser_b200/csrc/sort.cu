@@ -225,23 +225,25 @@ __global__ void __launch_bounds__(kSortThreads) onesweep_kernel(OnesweepArgs a) 
   for (int k = 0; k < warp; ++k) before += s_wsum[k];
   s_start[d] = before + v - count;
 
-  // Decoupled look-back over earlier CTAs for this digit, 8 predecessors per
-  // round (their status words are loaded together, so a long run of
-  // aggregate-only predecessors costs one memory latency per 8, not per CTA).
-  // Every wait is bounded.
+  // Decoupled look-back over earlier CTAs for this digit, kWindow predecessors
+  // per round: their status words are loaded together, so a run of
+  // aggregate-only predecessors costs one memory latency per kWindow CTAs.
+  // (When a whole wave of CTAs starts at once, none has its inclusive prefix
+  // yet and CTA k of the wave must sum back k aggregates.) Every wait is bounded.
+  constexpr int kWindow = 32;
   uint32_t excl = 0;
   if (tile > 0) {
     int64_t t = static_cast<int64_t>(tile) - 1;
     int spins = 0;
     while (t >= 0) {
-      uint32_t w[8];
+      uint32_t w[kWindow];
 #pragma unroll
-      for (int k = 0; k < 8; ++k)
+      for (int k = 0; k < kWindow; ++k)
         w[k] = (t - k >= 0) ? ld_relaxed(&a.status[(t - k) * kRadix + d]) : kFlagPrefix;
       int used = 0;
       bool stop = false, blocked = false;
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
+      for (int k = 0; k < kWindow; ++k) {
         if (stop || blocked) continue;
         const uint32_t flag = w[k] & ~kValueMask;
         if (flag == 0u) {
