@@ -230,7 +230,7 @@ __global__ void __launch_bounds__(kSortThreads) onesweep_kernel(OnesweepArgs a) 
   // aggregate-only predecessors costs one memory latency per kWindow CTAs.
   // (When a whole wave of CTAs starts at once, none has its inclusive prefix
   // yet and CTA k of the wave must sum back k aggregates.) Every wait is bounded.
-  constexpr int kWindow = 32;
+  constexpr int kWindow = 8;
   uint32_t excl = 0;
   if (tile > 0) {
     int64_t t = static_cast<int64_t>(tile) - 1;
