@@ -260,10 +260,13 @@ def stage_models(scene, sh_k):
         # fused projection backward + Adam: 32 B per scalar of every group, plus the
         # raw screen-gradient sums, the screen record and two flags, per Gaussian
         "backward_adam": ("hbm", 32 * n_par + 48 + 48 + 5),
-        # per evaluated (pixel, Gaussian) pair: 2 subtractions + 5 for the quadratic form
-        "blend_forward": ("alu", 7),
-        # per pair up to the last contributor: the same 7 to recompute alpha
-        "blend_backward": ("alu", 7),
+        # FP32 instructions: 7 per pair the method's walk visits (2 subtractions + 5 for the
+        # exponent's quadratic form), plus per blended pair 6 in the forward (weight, 3
+        # colour FMAs, transmittance update) and 19 in the backward (T recovery 2,
+        # colour dot 3, dL/dalpha 2, weight 1, tail update 1, 3 colour grads, 7 for the
+        # six raw sums)
+        "blend_forward": ("alu", (7, 6)),
+        "blend_backward": ("alu", (7, 19)),
     }
 
 
@@ -283,7 +286,9 @@ def roofline(prof, scene, hbm_gbs, sm_mhz):
         else:
             # FP32 lanes: 148 SMs x 128 lanes x clock (one instruction per lane per cycle)
             peak = 148 * 128 * sm_mhz * 1e6 / 1e12
-            achieved = units * per_unit / t / 1e12
+            per_visit, per_blend = per_unit
+            blended = d.get("blended", 0) / d["launches"]
+            achieved = (units * per_visit + blended * per_blend) / t / 1e12
             per[name] = {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "Tinst/s",
                          "frac": achieved / peak, "ms_per_launch": t * 1e3}
     return per

@@ -132,7 +132,7 @@ __global__ void __launch_bounds__(256) blend_forward_kernel(BlendArgs a) {
   float T = 1.0f, C0 = 0.0f, C1 = 0.0f, C2 = 0.0f;
   int last = 0;
   bool done = !inside;
-  unsigned evals = 0;
+  unsigned blended = 0;
 
   // two-stage prefetch: the order entries of chunk i+2, the records of chunk i+1
   uint32_t gid_next = load_gid(a.order, beg + lane, beg, end);
@@ -152,8 +152,8 @@ __global__ void __launch_bounds__(256) blend_forward_kernel(BlendArgs a) {
       const float2 xy = ws.xy[k];
       const float p = power2(ws.q[k], fx - xy.x, fy - xy.y);
       const float alpha = fminf(kAlphaMax, fast_exp2(p));
-      if (kCount) evals += !done;
       if (!done && alpha >= kAlphaMin) {
+        if (kCount) ++blended;
         const float4 c = ws.col[k];
         const float w = alpha * T;
         C0 = __fmaf_rn(w, c.x, C0);
@@ -175,7 +175,13 @@ __global__ void __launch_bounds__(256) blend_forward_kernel(BlendArgs a) {
     a.final_T[pix] = T;
     a.n_contrib[pix] = last;
   }
-  if (kCount) count_pairs(a.pairs, evals);
+  if (kCount) {
+    // the method's walk evaluates every list entry up to the one that saturates
+    // the pixel (all of them if it never saturates); culling skips most of them
+    const unsigned walked = !inside ? 0u : (done ? static_cast<unsigned>(last) : static_cast<unsigned>(end - beg));
+    count_pairs(a.pairs, walked);
+    count_pairs(a.pairs + 2, blended);
+  }
 }
 
 // Reduces v[0..8] over the warp; on return lane l (l even) holds the warp total
@@ -262,7 +268,7 @@ __global__ void __launch_bounds__(256) blend_backward_kernel(BlendArgs a) {
   const int red_idx = ((lane >> 1) & 1) * 8 + ((lane >> 2) & 1) * 4 + ((lane >> 3) & 1) * 2 +
                       ((lane >> 4) & 1);
   const bool red_writer = !(lane & 1) && red_idx < 9;
-  unsigned evals = 0;
+  unsigned blended = 0;
 
   // Chunks walk down from the top; lane l takes entry hi - 1 - l, so ballot
   // order (lane order) is descending list order.
@@ -286,7 +292,7 @@ __global__ void __launch_bounds__(256) blend_backward_kernel(BlendArgs a) {
       const float raw = fast_exp2(power2(ws.q[k], dx, dy));
       const float alpha = fminf(kAlphaMax, raw);
       const bool contrib = pos < last && alpha >= kAlphaMin;
-      if (kCount && pos < last) ++evals;
+      if (kCount && contrib) ++blended;
       if (!__any_sync(0xffffffffu, contrib)) continue;
       float v[9];
 #pragma unroll
@@ -316,7 +322,11 @@ __global__ void __launch_bounds__(256) blend_backward_kernel(BlendArgs a) {
     }
     __syncwarp();
   }
-  if (kCount) count_pairs(a.pairs, evals);
+  if (kCount) {
+    // the method's backward walk visits every entry before the pixel's last contributor
+    count_pairs(a.pairs, static_cast<unsigned>(min(last, static_cast<int>(range.y - range.x))));
+    count_pairs(a.pairs + 2, blended);
+  }
 }
 
 }  // namespace

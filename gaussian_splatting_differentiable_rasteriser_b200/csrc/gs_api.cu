@@ -59,7 +59,7 @@ struct gs_ctx {
     int64_t launches[GS_NUM_STAGES] = {0};
     int64_t work[GS_NUM_STAGES] = {0};
   } prof;
-  unsigned long long* pairs = nullptr;  // [2] evaluated pairs of the two blends
+  unsigned long long* pairs = nullptr;  // [8]: forward at [0], [2]; backward at [4], [6]
   char err[512] = {0};
 };
 
@@ -259,12 +259,12 @@ gs_status gs_create(gs_ctx** out, int64_t max_gaussians, int64_t max_entries, in
   GS_ALLOC(c->loss_partials, sizeof(double) * 2 * c->max_loss_blocks);
   GS_ALLOC(c->loss_counter, sizeof(uint32_t));
   GS_ALLOC(c->info_dev, sizeof(gs::ForwardInfo));
-  GS_ALLOC(c->pairs, sizeof(unsigned long long) * 2);
+  GS_ALLOC(c->pairs, sizeof(unsigned long long) * 8);
 #undef GS_ALLOC
   if (e == cudaSuccess) e = cudaMallocHost(reinterpret_cast<void**>(&c->info_host), sizeof(gs::ForwardInfo));
   if (e == cudaSuccess) e = cudaMemset(c->loss_counter, 0, sizeof(uint32_t));
   if (e == cudaSuccess) e = cudaMemset(c->info_dev, 0, sizeof(gs::ForwardInfo));
-  if (e == cudaSuccess) e = cudaMemset(c->pairs, 0, sizeof(unsigned long long) * 2);
+  if (e == cudaSuccess) e = cudaMemset(c->pairs, 0, sizeof(unsigned long long) * 8);
   if (e == cudaSuccess) e = cudaDeviceSynchronize();
   if (e != cudaSuccess) {
     free_all(c);
@@ -490,7 +490,7 @@ gs_status backward_common(gs_ctx* c, const gs_params* p, const gs_camera* cam, c
   ba.n_contrib = const_cast<int32_t*>(n_contrib);
   ba.dimage = dloss_dimage;
   ba.sgrad = c->sgrad;
-  ba.pairs = c->prof.on ? c->pairs + 1 : nullptr;
+  ba.pairs = c->prof.on ? c->pairs + 4 : nullptr;
   prof_begin(c, st);
   GS_CUDA(c, gs::launch_blend_backward(ba, st));
   prof_end(c, GS_STAGE_BLEND_BACKWARD, 0, st);
@@ -600,19 +600,23 @@ gs_status gs_profile_enable(gs_ctx* c, int32_t enabled) {
   return GS_OK;
 }
 
-gs_status gs_profile_read(gs_ctx* c, double* ms, int64_t* launches, int64_t* work) {
+gs_status gs_profile_read(gs_ctx* c, double* ms, int64_t* launches, int64_t* work,
+                          int64_t* blended) {
   if (!c) return GS_ERR_INVALID_ARG;
   auto& P = c->prof;
   prof_harvest(c);
-  unsigned long long pairs[2] = {0ull, 0ull};
+  unsigned long long pairs[8] = {0ull};
   GS_CUDA(c, cudaMemcpy(pairs, c->pairs, sizeof(pairs), cudaMemcpyDeviceToHost));
   GS_CUDA(c, cudaMemset(c->pairs, 0, sizeof(pairs)));
   P.work[GS_STAGE_BLEND_FORWARD] += static_cast<int64_t>(pairs[0]);
-  P.work[GS_STAGE_BLEND_BACKWARD] += static_cast<int64_t>(pairs[1]);
+  P.work[GS_STAGE_BLEND_BACKWARD] += static_cast<int64_t>(pairs[4]);
   for (int k = 0; k < GS_NUM_STAGES; ++k) {
     if (ms) ms[k] = P.ms[k];
     if (launches) launches[k] = P.launches[k];
     if (work) work[k] = P.work[k];
+    if (blended)
+      blended[k] = k == GS_STAGE_BLEND_FORWARD ? static_cast<int64_t>(pairs[2])
+                   : k == GS_STAGE_BLEND_BACKWARD ? static_cast<int64_t>(pairs[6]) : 0;
     P.ms[k] = 0.0;
     P.launches[k] = 0;
     P.work[k] = 0;

@@ -96,7 +96,8 @@ struct BlendArgs {
   // backward only
   const float* dimage;
   float* sgrad;  // [n][kGradStride]
-  // when not null, the number of evaluated (pixel, Gaussian) pairs is added here
+  // when not null: pairs[0] += (pixel, Gaussian) pairs the method's walk visits,
+  // pairs[2] += pairs that blend (alpha >= 1/255 before the walk stops)
   unsigned long long* pairs;
 };
 

@@ -85,7 +85,7 @@ def load(path: str = LIB_PATH):
                                           ctypes.POINTER(GsGrads), ctypes.POINTER(F), F, F, F, I32, P]
     L.gs_adam_step.argtypes = [P, P, P, P, I64, F, F, F, F, I32, P]
     L.gs_profile_enable.argtypes = [P, I32]
-    L.gs_profile_read.argtypes = [P, P, P, P]
+    L.gs_profile_read.argtypes = [P, P, P, P, P]
     L.gs_stage_name.argtypes = [I32]
     L.gs_stage_name.restype = ctypes.c_char_p
     L.gs_debug_preprocess.argtypes = [P] * 10
@@ -186,8 +186,10 @@ class Context:
         ms = (ctypes.c_double * n)()
         launches = (ctypes.c_int64 * n)()
         work = (ctypes.c_int64 * n)()
-        self._check(self.L.gs_profile_read(self.h, ms, launches, work))
-        return {STAGES[k]: {"ms": ms[k], "launches": launches[k], "work": work[k]} for k in range(n)}
+        blended = (ctypes.c_int64 * n)()
+        self._check(self.L.gs_profile_read(self.h, ms, launches, work, blended))
+        return {STAGES[k]: {"ms": ms[k], "launches": launches[k], "work": work[k], "blended": blended[k]}
+                for k in range(n)}
 
     def debug_preprocess(self, mean2d=None, conic=None, opacity=None, rgb=None, depth=None, rect=None,
                          touched=None, clamped=None, stream=None):

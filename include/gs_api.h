@@ -202,8 +202,11 @@ gs_status gs_adam_step(float *param, float *grad, float *m, float *v, int64_t co
  * be NULL): ms = summed kernel time, launches = launches, work = the units
  * processed (Gaussians for the per-Gaussian stages - n_pad for the fused
  * backward + Adam pass -, entries x passes for the sort, entries for the
- * duplication and ranges, evaluated (pixel, Gaussian) pairs for the blends,
- * pixels for the loss). gs_adam_step takes no context and is not profiled
+ * duplication and ranges, pixels for the loss; for the two blends the
+ * (pixel, Gaussian) pairs the method's walk visits: every list entry up to
+ * the pixel's stopping point in the forward, every entry before its last
+ * contributor in the backward), blended = for the two blends the pairs that
+ * actually blend (alpha >= 1/255 before the walk stops), 0 elsewhere. gs_adam_step takes no context and is not profiled
  * here. */
 typedef enum {
   GS_STAGE_PREPROCESS = 0,
@@ -220,7 +223,8 @@ typedef enum {
 } gs_stage;
 
 gs_status gs_profile_enable(gs_ctx *ctx, int32_t enabled);
-gs_status gs_profile_read(gs_ctx *ctx, double *ms, int64_t *launches, int64_t *work);
+gs_status gs_profile_read(gs_ctx *ctx, double *ms, int64_t *launches, int64_t *work,
+                          int64_t *blended);
 /* Static name of a stage ("preprocess", "sort", ...), or "" if out of range. */
 const char *gs_stage_name(int32_t stage);
 
