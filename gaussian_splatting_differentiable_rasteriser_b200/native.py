@@ -84,6 +84,8 @@ def load(path: str = LIB_PATH):
                                           ctypes.POINTER(GsGrads), ctypes.POINTER(GsGrads),
                                           ctypes.POINTER(GsGrads), ctypes.POINTER(F), F, F, F, I32, P]
     L.gs_adam_step.argtypes = [P, P, P, P, I64, F, F, F, F, I32, P]
+    L.gs_loss_l1_dssim_noalloc.argtypes = [P, P, I32, I32, F, P, P, P]
+    L.gs_loss_l1_dssim_noalloc.restype = ctypes.c_int
     L.gs_profile_enable.argtypes = [P, I32]
     L.gs_profile_read.argtypes = [P, P, P, P, P]
     L.gs_stage_name.argtypes = [I32]

@@ -165,6 +165,27 @@ gs_status gs_render_backward(gs_ctx *ctx, const gs_params *params, const gs_came
                              const float *final_T, const int32_t *n_contrib,
                              const float *dloss_dimage, gs_grads *grads, void *stream);
 
+/* Step 3 without allocation - the same fused loss as gs_loss_l1_dssim, for
+ * callers that cannot allocate device memory where they need the loss (code
+ * being captured into a CUDA graph, loops whose memory is fixed after
+ * start-up, hosts that hand over only input and output pointers). The pages
+ * describe no counterpart; this is an interface convenience of this library.
+ * It needs no context: the kernel's scratch (per-CTA partial sums and a
+ * completion counter, about 0.8 MB) is a file-scope __device__ array that
+ * every GPU loading the library holds until the process exits. The first call
+ * on each device looks up the array's device address (cudaGetSymbolAddress,
+ * with that device current), so make that first call before any stream
+ * capture. All calls on a device share the one array: calls that overlap on
+ * the GPU (other streams, other threads) race and must be serialised by the
+ * caller. Arguments and outputs as gs_loss_l1_dssim. Returns
+ * GS_ERR_CAPACITY, with nothing enqueued, for an image wider or taller than
+ * 4096 pixels; GS_ERR_INVALID_ARG for bad pointers or sizes; GS_ERR_CUDA if
+ * the symbol lookup, the counter reset or the launch fails. Allocates
+ * nothing and frees nothing. */
+gs_status gs_loss_l1_dssim_noalloc(const float *image_chw, const float *target_chw, int32_t height,
+                                   int32_t width, float lambda, double *loss_out,
+                                   float *dloss_dimage, void *stream);
+
 /* Steps 4 + 5 in one pass - the backward of gs_render_backward followed, in the
  * same pass over the parameters, by the Adam step of gs_adam_step on every
  * group: for each scalar g = grads + this view's gradient, then the Adam update
