@@ -49,6 +49,8 @@ def lib():
         L.or_render_rows.argtypes = [P, ctypes.c_int32, ctypes.c_int32] + [P] * 5
         L.or_backward_rows.argtypes = [P, ctypes.c_int32, ctypes.c_int32] + [P] * 7
         L.or_backward.argtypes = [P] * 8
+        L.or_blend_backward_rows.argtypes = [P, ctypes.c_int32, ctypes.c_int32, P, P]
+        L.or_project_backward.argtypes = [P, P, ctypes.c_int64, ctypes.c_int64] + [P] * 5
         L.or_loss.argtypes = [ctypes.c_int32, ctypes.c_int32, P, P, ctypes.c_double, P, P]
         L.or_loss.restype = ctypes.c_int
         L.or_loss_f64.argtypes = [ctypes.c_int32, ctypes.c_int32, P, P, ctypes.c_double, P, P]
@@ -152,11 +154,14 @@ class Oracle:
                                 _p(out["n_contrib"]), _p(out["ambiguous"]))
         return out
 
-    def render_rows(self, y0, y1) -> dict:
+    def render_rows(self, y0, y1, out=None) -> dict:
+        """Forward over the pixel rows [y0, y1) into full-size outputs (`out`, as
+        returned by an earlier call, is reused when given)."""
         H, W = self.cam.height, self.cam.width
-        out = dict(image=np.zeros((3, H, W)), final_T=np.zeros((H, W)),
-                   n_contrib=np.zeros((H, W), np.int32), ambiguous=np.zeros((H, W), np.uint8),
-                   stats=np.zeros(2, np.int64))
+        if out is None:
+            out = dict(image=np.zeros((3, H, W)), final_T=np.zeros((H, W)),
+                       n_contrib=np.zeros((H, W), np.int32), ambiguous=np.zeros((H, W), np.uint8),
+                       stats=np.zeros(2, np.int64))
         self.L.or_render_rows(self.h, int(y0), int(y1), *[_p(out[k]) for k in
                                                            ("image", "final_T", "n_contrib",
                                                             "ambiguous", "stats")])
@@ -175,6 +180,21 @@ class Oracle:
         self.L.or_backward_rows(self.h, int(y0), int(y1), _p(dimage),
                                 *[_p(out[k]) for k in ("screen", "means", "log_scales", "quats",
                                                        "opacity_logits", "sh")])
+        return out
+
+    def blend_backward_rows(self, y0, y1, dimage, screen_grad):
+        """Adds the blend backward of the pixel rows [y0, y1) to screen_grad (n x 9)."""
+        assert screen_grad.dtype == np.float64 and screen_grad.shape == (self.scene.n, 9)
+        dimage = np.ascontiguousarray(dimage, np.float64)
+        self.L.or_blend_backward_rows(self.h, int(y0), int(y1), _p(dimage), _p(screen_grad))
+
+    def project_backward(self, screen_grad, i0, i1, out) -> dict:
+        """Parameter gradients of the Gaussians [i0, i1) from their screen
+        gradient, written into `out` (the dict `backward` returns)."""
+        assert screen_grad.dtype == np.float64 and screen_grad.shape == (self.scene.n, 9)
+        self.L.or_project_backward(self.h, _p(screen_grad), int(i0), int(i1),
+                                   *[_p(out[k]) for k in ("means", "log_scales", "quats",
+                                                          "opacity_logits", "sh")])
         return out
 
 

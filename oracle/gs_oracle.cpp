@@ -712,20 +712,13 @@ void or_render_pixels(void* h, int64_t npix, const int32_t* px, const int32_t* p
   }
 }
 
-// Backward from dL/dimage [3][H][W]. Writes the screen gradient n x 9
-// (dL/du, dv, dA, dB, dC, d opacity, dr, dg, db) and the parameter gradients in
-// the planar layout of the parameters (means [3][n_pad], log_scales [3][n_pad],
-// quats [4][n_pad], opacity_logits [n_pad], sh [3][K][n_pad]). Any output
-// pointer may be null.
-// The same from the pixel rows [y0, y1) only (dL/dimage is full size; other
-// rows contribute nothing).
-void or_backward_rows(void* h, int32_t y0, int32_t y1, const double* dimage, double* screen_grad,
-                      double* g_means, double* g_ls, double* g_quats, double* g_logits,
-                      double* g_sh) {
+// Blend backward over the pixel rows [y0, y1): ADDS each pixel's contribution to
+// the screen gradient n x 9 (dL/du, dv, dA, dB, dC, d opacity, dr, dg, db);
+// dL/dimage is [3][H][W], full size.
+void or_blend_backward_rows(void* h, int32_t y0, int32_t y1, const double* dimage,
+                            double* screen_grad) {
   const Ctx& c = *static_cast<Ctx*>(h);
   const int W = c.cam.width, H = c.cam.height;
-  const int64_t n = c.n, np = c.n_pad;
-  std::vector<double> sg(static_cast<size_t>(n) * kScreen, 0.0);
   std::vector<Contribution> list;
   y0 = std::max(y0, 0);
   y1 = std::min(y1, H);
@@ -736,20 +729,36 @@ void or_backward_rows(void* h, int32_t y0, int32_t y1, const double* dimage, dou
       size_t p = static_cast<size_t>(py) * W + px;
       double g[3] = {dimage[p], dimage[static_cast<size_t>(H) * W + p],
                      dimage[2 * static_cast<size_t>(H) * W + p]};
-      backward_pixel(c, list, g, sg.data());
+      backward_pixel(c, list, g, screen_grad);
     }
-  if (screen_grad) std::memcpy(screen_grad, sg.data(), sg.size() * sizeof(double));
+}
 
+// Projection backward of the Gaussians [i0, i1): from their screen gradient
+// (n x 9) to the parameter gradients in the planar layout of the parameters
+// (means [3][n_pad], log_scales [3][n_pad], quats [4][n_pad], opacity_logits
+// [n_pad], sh [3][K][n_pad]); writes those Gaussians' entries only (a culled
+// Gaussian or one with a zero screen gradient gets zeros). Any output may be null.
+void or_project_backward(void* h, const double* screen_grad, int64_t i0, int64_t i1,
+                         double* g_means, double* g_ls, double* g_quats, double* g_logits,
+                         double* g_sh) {
+  const Ctx& c = *static_cast<Ctx*>(h);
+  const int64_t n = c.n, np = c.n_pad;
   const int K = (c.sh_degree + 1) * (c.sh_degree + 1);
   const int nk = (c.active_degree + 1) * (c.active_degree + 1);
-  if (g_means) std::memset(g_means, 0, sizeof(double) * 3 * np);
-  if (g_ls) std::memset(g_ls, 0, sizeof(double) * 3 * np);
-  if (g_quats) std::memset(g_quats, 0, sizeof(double) * 4 * np);
-  if (g_logits) std::memset(g_logits, 0, sizeof(double) * np);
-  if (g_sh) std::memset(g_sh, 0, sizeof(double) * 3 * K * np);
-  for (int64_t i = 0; i < n; ++i) {
+  i0 = std::max<int64_t>(i0, 0);
+  i1 = std::min<int64_t>(i1, n);
+  for (int64_t i = i0; i < i1; ++i) {
+    if (g_means)
+      for (int j = 0; j < 3; ++j) g_means[j * np + i] = 0.0;
+    if (g_ls)
+      for (int j = 0; j < 3; ++j) g_ls[j * np + i] = 0.0;
+    if (g_quats)
+      for (int j = 0; j < 4; ++j) g_quats[j * np + i] = 0.0;
+    if (g_logits) g_logits[i] = 0.0;
+    if (g_sh)
+      for (int k = 0; k < 3 * K; ++k) g_sh[static_cast<size_t>(k) * np + i] = 0.0;
     if (c.aux[i].touched == 0) continue;
-    const double* gs = &sg[static_cast<size_t>(i) * kScreen];
+    const double* gs = &screen_grad[static_cast<size_t>(i) * kScreen];
     bool any = false;
     for (int o = 0; o < kScreen; ++o) any = any || gs[o] != 0.0;
     if (!any) continue;  // a zero screen gradient has a zero parameter gradient
@@ -783,6 +792,27 @@ void or_backward_rows(void* h, int32_t y0, int32_t y1, const double* dimage, dou
           g_sh[(static_cast<size_t>(ch) * K + k) * np + i] = gs[6 + ch] * X.Y[k];
       }
   }
+}
+
+// Backward from dL/dimage [3][H][W] over the pixel rows [y0, y1) (other rows
+// contribute nothing): the screen gradient n x 9 and the parameter gradients of
+// all Gaussians (padding entries of the planar outputs are zeroed). Any output
+// pointer may be null.
+void or_backward_rows(void* h, int32_t y0, int32_t y1, const double* dimage, double* screen_grad,
+                      double* g_means, double* g_ls, double* g_quats, double* g_logits,
+                      double* g_sh) {
+  const Ctx& c = *static_cast<Ctx*>(h);
+  const int64_t n = c.n, np = c.n_pad;
+  std::vector<double> sg(static_cast<size_t>(n) * kScreen, 0.0);
+  or_blend_backward_rows(h, y0, y1, dimage, sg.data());
+  if (screen_grad) std::memcpy(screen_grad, sg.data(), sg.size() * sizeof(double));
+  const int K = (c.sh_degree + 1) * (c.sh_degree + 1);
+  if (g_means) std::memset(g_means, 0, sizeof(double) * 3 * np);
+  if (g_ls) std::memset(g_ls, 0, sizeof(double) * 3 * np);
+  if (g_quats) std::memset(g_quats, 0, sizeof(double) * 4 * np);
+  if (g_logits) std::memset(g_logits, 0, sizeof(double) * np);
+  if (g_sh) std::memset(g_sh, 0, sizeof(double) * 3 * K * np);
+  or_project_backward(h, sg.data(), 0, n, g_means, g_ls, g_quats, g_logits, g_sh);
 }
 
 void or_backward(void* h, const double* dimage, double* screen_grad, double* g_means,

@@ -141,3 +141,26 @@ def test_view_direction_path_is_included():
     _, _, _, dimg0 = oracle.loss(o0.render()["image"], target, 0.2)
     g0 = o0.backward(dimg0)["means"]
     assert np.abs(g_full - g0).max() > 1e-4
+
+
+def test_split_backward_equals_whole_backward():
+    """The blend backward over two row bands plus the projection backward over
+    two Gaussian slices reproduce the one-call backward exactly (the parts are
+    sums over disjoint pixels and maps over disjoint Gaussians)."""
+    s = scenes.tiny()
+    cam = s.cameras[0]
+    o = oracle.Oracle(s, cam)
+    rng = np.random.default_rng(3)
+    dimage = rng.normal(size=(3, cam.height, cam.width))
+    whole = o.backward(dimage)
+    sg = np.zeros((s.n, 9))
+    mid = cam.height // 2
+    o.blend_backward_rows(0, mid, dimage, sg)
+    o.blend_backward_rows(mid, cam.height, dimage, sg)
+    np.testing.assert_allclose(sg, whole["screen"], rtol=1e-12, atol=1e-15)
+    parts = {k: np.full_like(v, np.nan) for k, v in whole.items() if k != "screen"}
+    o.project_backward(sg, 0, s.n // 3, parts)
+    o.project_backward(sg, s.n // 3, s.n, parts)
+    for k, v in parts.items():
+        idx = (Ellipsis, slice(0, s.n))
+        np.testing.assert_allclose(v[idx], whole[k][idx], rtol=1e-12, atol=1e-15, err_msg=k)
