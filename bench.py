@@ -47,8 +47,15 @@ WORKLOADS = {
 
 # ncu DRAM traffic (read + write bytes per launch) of kernels on the dense workload,
 # with the sha256 (first 12 hex digits) of the source file each figure was taken from.
-# A figure whose source has changed since is reported as null.
-NCU_TRAFFIC = {}
+# A figure whose source has changed since is reported as null. Both were captured on
+# the Mid workload (500k Gaussians, 1.06M entries; profiles/kernels_mid_720p.md) and
+# scaled to Dense by the units a launch processes (n_pad 3,000,000 / 500,000 for the
+# per-Gaussian pass, entries 6.32M / 1.06M for the blend), in which traffic grows in
+# proportion.
+NCU_TRAFFIC = {
+    "backward_adam": ((537.409536e6 + 412.686848e6) * 6.0, "acabd81e2d44"),
+    "blend_backward": ((70.30784e6 + 2.051584e6) * 6.32 / 1.064, "1386ae1844b4"),
+}
 
 
 def sha12(path):
@@ -84,7 +91,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
@@ -295,53 +302,102 @@ def roofline(prof, scene, hbm_gbs, sm_mhz):
 
 
 # ------------------------------------------------------------- oracle (CPU)
-def oracle_sample_step(scene, cam, target, rows=8, adam_frac=1 / 64):
-    """One training step of the float64 oracle on a bounded sample of the workload:
-    the full preprocess + tile sort of every Gaussian, then render, loss and
-    backward restricted to a band of `rows` pixel rows (scaled by height/rows),
-    and Adam on a 1/64 slice of the parameters (scaled by 64). Returns the
-    estimated seconds of one full step and the measured seconds spent."""
-    import numpy as np
+def subset_scene(scene, stride):
+    """Every stride-th Gaussian of the scene (input preparation for a bounded sample)."""
+    from gaussian_splatting_differentiable_rasteriser_b200 import scenes
+    sl = slice(0, scene.n, stride)
+    return scenes.make_scene(scene.name + f"/{stride}", scene.means[:, sl], scene.log_scales[:, sl],
+                             scene.quats[:, sl], scene.opacity_logits[sl], scene.sh_degree,
+                             scene.sh[:, :, sl], scene.cameras)
 
-    import oracle
 
-    H, W = cam.height, cam.width
-    y0 = (H - rows) // 2
+class OracleSampler:
+    """Estimates the host time of one full training step of the float64 oracle
+    from a bounded sample, part by part, each part scaled by the share of the
+    step it covers:
+      preprocess + tile sort of every `stride`-th Gaussian        x stride
+      render + loss + blend backward of a band of `rows` rows      x height / rows
+      projection backward of a 1/stride slice of the Gaussians     x stride
+      Adam over a slice of the parameters                          x 1 / adam_frac
+    The band and the projection slice use the full scene seen by one camera,
+    prepared once outside the timed parts (its preprocess is the one timed on
+    the subset); every output buffer is allocated once."""
+
+    def __init__(self, scene, cam, target, rows, stride, adam_frac):
+        import numpy as np
+
+        import oracle
+
+        self.np, self.oracle = np, oracle
+        self.scene, self.rows, self.stride, self.adam_frac = scene, rows, stride, adam_frac
+        self.sub = subset_scene(scene, stride) if stride > 1 else scene
+        self.full = oracle.Oracle(scene, cam)
+        H, W = cam.height, cam.width
+        self.H = H
+        self.y0 = (H - rows) // 2
+        self.target = np.asarray(target[:, self.y0:self.y0 + rows, :], np.float64)
+        self.out = None
+        self.dimage = np.zeros((3, H, W))
+        self.sg = np.zeros((scene.n, 9))
+        n = scene.n
+        self.grads = dict(means=np.zeros((3, scene.n_pad)), log_scales=np.zeros((3, scene.n_pad)),
+                          quats=np.zeros((4, scene.n_pad)), opacity_logits=np.zeros(scene.n_pad),
+                          sh=np.zeros((3, scene.sh_k, scene.n_pad)))
+        # screen gradients for the projection slice: every touched Gaussian gets a
+        # non-zero one, as in a full step where every visible Gaussian is reached
+        touched = self.full.preprocess()["touched"] > 0
+        self.i0 = n // 2 - n // (2 * stride)
+        self.i1 = self.i0 + max(1, n // stride)
+        self.sg_slice = np.zeros((n, 9))
+        self.sg_slice[self.i0:self.i1][touched[self.i0:self.i1]] = 1e-3
+        total = scene.means.size + scene.log_scales.size + scene.quats.size + \
+            scene.opacity_logits.size + scene.sh.size
+        cnt = max(1, int(total * adam_frac))
+        rng = np.random.default_rng(0)
+        self.adam_arrays = (rng.normal(size=cnt), rng.normal(size=cnt) * 1e-3, np.zeros(cnt),
+                            np.zeros(cnt))
+
+    def step(self, cam):
+        """One sampled step with camera `cam` for the preprocess part; returns
+        (estimated seconds of a full step, seconds spent)."""
+        np, oracle = self.np, self.oracle
+        rows, y0 = self.rows, self.y0
+        t0 = time.perf_counter()
+        oracle.Oracle(self.sub, cam)  # preprocess + duplicate + sort + ranges
+        t1 = time.perf_counter()
+        self.out = self.full.render_rows(y0, y0 + rows, out=self.out)
+        img = self.out["image"][:, y0:y0 + rows, :]
+        _, _, _, d = oracle.loss(img, self.target, 0.2)
+        self.dimage[:, y0:y0 + rows, :] = d
+        self.sg.fill(0.0)
+        self.full.blend_backward_rows(y0, y0 + rows, self.dimage, self.sg)
+        t2 = time.perf_counter()
+        self.full.project_backward(self.sg_slice, self.i0, self.i1, self.grads)
+        t3 = time.perf_counter()
+        oracle.adam(*self.adam_arrays, 1e-3, 1)
+        t4 = time.perf_counter()
+        est = ((t1 - t0) * self.stride + (t2 - t1) * self.H / rows + (t3 - t2) * self.stride +
+               (t4 - t3) / self.adam_frac)
+        return est, t4 - t0
+
+    def describe(self):
+        return (f"float64 preprocess + tile sort of every {self.stride}th of {self.scene.n} "
+                f"Gaussians x {self.stride}; render + loss + blend backward of a {self.rows}-row "
+                f"band x height/{self.rows}; projection backward of a 1/{self.stride} slice "
+                f"x {self.stride}; Adam on a 1/{round(1 / self.adam_frac)} parameter slice "
+                f"x {round(1 / self.adam_frac)}; single-threaded")
+
+
+def cpu_baseline(scene, cams, targets_host, sched):
+    """One sampled step of the oracle on the host (our arm's reported baseline)."""
+    c = int(sched[0])
     t0 = time.perf_counter()
-    o = oracle.Oracle(scene, cam)
-    t1 = time.perf_counter()
-    r = o.render_rows(y0, y0 + rows)
-    band = r["image"][:, y0:y0 + rows, :]
-    _, _, _, d = oracle.loss(band, np.asarray(target[:, y0:y0 + rows, :], np.float64), 0.2)
-    dfull = np.zeros((3, H, W))
-    dfull[:, y0:y0 + rows, :] = d
-    o.backward(dfull, rows=(y0, y0 + rows))
-    t2 = time.perf_counter()
-    total = scene.means.size + scene.log_scales.size + scene.quats.size + scene.opacity_logits.size + \
-        scene.sh.size
-    cnt = max(1, int(total * adam_frac))
-    rng = np.random.default_rng(0)
-    p = rng.normal(size=cnt)
-    g = rng.normal(size=cnt) * 1e-3
-    oracle.adam(p, g, np.zeros(cnt), np.zeros(cnt), 1e-3, 1)
-    t3 = time.perf_counter()
-    est = (t1 - t0) + (t2 - t1) * H / rows + (t3 - t2) / adam_frac
-    return est, t3 - t0
-
-
-def cpu_baseline(scene, cams, targets_host, sched, steps):
-    est, spent = [], 0.0
-    for i in range(steps):
-        c = int(sched[i % len(sched)])
-        e, s = oracle_sample_step(scene, cams[c], targets_host[c])
-        est.append(e)
-        spent += s
-    value = len(est) / sum(est)
-    return {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"{len(est)} step(s): full float64 preprocess + tile sort of all Gaussians, "
-                      "render + loss + backward on an 8-row band scaled by height/8, Adam on a "
-                      "1/64 parameter slice scaled by 64; single-threaded",
-            "seconds_spent": spent}
+    s = OracleSampler(scene, cams[c], targets_host[c], rows=48, stride=8, adam_frac=1 / 64)
+    prep = time.perf_counter() - t0
+    est, spent = s.step(cams[c])
+    return {"value": 1.0 / est, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": "1 step: " + s.describe(), "seconds_spent": spent,
+            "seconds_setup": prep}
 
 
 # ------------------------------------------------------------------- arms
@@ -363,11 +419,11 @@ def main_ours(args):
     scene, m, step, targets, kmax = build_workload(args.config, device)
     cams = scene.cameras
     sched = scenes.camera_schedule(len(cams), args.warmup + args.steps, seed=rank)
-    # warm-up (also compiles nothing: the library is ahead-of-time built)
-    run_steps(step, cams, targets, sched, 0, args.warmup)
-    torch.cuda.synchronize()
+    # clocks are sampled from the start of the warm-up to the end of the timed region
     clocks = ClockSampler(torch.cuda.current_device())
     clocks.start()
+    run_steps(step, cams, targets, sched, 0, args.warmup)
+    torch.cuda.synchronize()
     ms = time_device(step, cams, targets, sched, args.warmup, args.steps, world)
     clk = clocks.stop()
     ms = max_over_ranks(ms, world)
@@ -407,7 +463,7 @@ def main_ours(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(scene, cams, targets.cpu().numpy(), sched, 1)
+        cpu = cpu_baseline(scene, cams, targets.cpu().numpy(), sched)
 
     if rank == 0:
         line = {
@@ -490,45 +546,36 @@ def e2e_run(step, cams, targets, sched, args, world):
 
 
 def main_reference(args):
+    """The float64 CPU oracle on the same workload, each step a bounded sample
+    (OracleSampler with a 2-row band and 1/256 subsets) so that the whole run
+    stays within minutes. Rank 0 alone runs; other ranks exit without work."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    import numpy as np
-
-    from gaussian_splatting_differentiable_rasteriser_b200 import scenes
     import oracle
+    from gaussian_splatting_differentiable_rasteriser_b200 import scenes
 
     oracle.lib()
     scene = scenes.CONFIGS[args.config]()
-    # targets: the oracle's own band renders of the perturbed copy are what the sample needs
     pert = scenes.perturbed(scene, 0.05, seed=1)
     cams = scene.cameras
     sched = scenes.camera_schedule(len(cams), args.warmup + args.steps, seed=0)
     H, W = cams[0].height, cams[0].width
-    rows = 8
-    targets = {}
-    for c in set(int(x) for x in sched):
-        o = oracle.Oracle(pert, cams[c])
-        y0 = (H - rows) // 2
-        targets[c] = o.render_rows(y0, y0 + rows)["image"]
-        del o
-    for i in range(args.warmup):
-        c = int(sched[i])
-        oracle_sample_step(scene, cams[c], targets[c], rows)
-    est = []
-    spent = 0.0
-    for i in range(args.warmup, args.warmup + args.steps):
-        c = int(sched[i])
-        e, s = oracle_sample_step(scene, cams[c], targets[c], rows)
-        est.append(e)
-        spent += s
+    rows = 2
+    c0 = int(sched[0])
+    y0 = (H - rows) // 2
+    target = oracle.Oracle(pert, cams[c0]).render_rows(y0, y0 + rows)["image"]
+    sampler = OracleSampler(scene, cams[c0], target, rows=rows, stride=256, adam_frac=1 / 4096)
+    est, spent = [], 0.0
+    for i in range(args.warmup + args.steps):
+        e, s = sampler.step(cams[int(sched[i])])
+        if i >= args.warmup:
+            est.append(e)
+            spent += s
     value = len(est) / sum(est)
     cpu = {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
-           "sample": f"per step: full float64 preprocess + tile sort of all {scene.n} Gaussians, "
-                     f"render + loss + backward on a {rows}-row band scaled by height/{rows}, Adam on "
-                     "a 1/64 parameter slice scaled by 64; single-threaded",
-           "seconds_spent": spent}
+           "sample": "per step: " + sampler.describe(), "seconds_spent": spent}
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 / value,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
@@ -543,8 +590,8 @@ def main_reference(args):
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--config", choices=tuple(WORKLOADS), default="dense")
     ap.add_argument("--no-e2e", action="store_true")
