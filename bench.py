@@ -53,7 +53,6 @@ WORKLOADS = {
 # per-Gaussian pass, entries 6.32M / 1.06M for the blend), in which traffic grows in
 # proportion.
 NCU_TRAFFIC = {
-    "backward_adam": ((537.409536e6 + 412.686848e6) * 6.0, "acabd81e2d44"),
     "blend_backward": ((70.30784e6 + 2.051584e6) * 6.32 / 1.064, "1386ae1844b4"),
 }
 
@@ -138,6 +137,12 @@ def dist_setup():
     elif torch.cuda.is_available():
         torch.cuda.set_device(local)
     return world, rank, local
+
+
+def replica_throughput(world, steps, seconds_max):
+    """Whole-job iterations per second of `world` replicas that each ran `steps`
+    iterations, the slowest taking `seconds_max`."""
+    return world * steps / seconds_max
 
 
 def barrier(world):
@@ -253,20 +258,25 @@ def stage_models(scene, sh_k):
     return {
         # params in (all groups) + 48 B screen + depth + rect + touched + clamp out, per Gaussian
         "preprocess": ("hbm", 4 * n_par + 48 + 4 + 8 + 4 + 1),
-        # per entry and pass: key + value read and written
-        "sort": ("hbm", 24),
-        # keys + values written per entry
-        "duplicate": ("hbm", 12),
-        "ranges": ("hbm", 8),
+        # per item and pass: 32-bit key + 32-bit value read and written (the depth sort's
+        # items are the visible Gaussians, the tile sort's the entries)
+        "depth_sort": ("hbm", 16),
+        "sort": ("hbm", 16),
+        # tile key + index written per entry (the 16 B read per visible Gaussian - order,
+        # touched, rect - are not counted)
+        "duplicate": ("hbm", 8),
+        # tile key read (and its neighbour, from cache), per entry
+        "ranges": ("hbm", 4),
         # x, y read, dL/dx written, per pixel (3 channels)
         "loss": ("hbm", 36),
         # params + grads read, grads written, raw sums + screen record read, per Gaussian
         "preprocess_backward": ("hbm", 4 * n_par * 3 + 48 + 48 + 5),
         # p, g, m, v read; p, m, v, g = 0 written, per scalar
         "adam": ("hbm", 32),
-        # fused projection backward + Adam: 32 B per scalar of every group, plus the
-        # raw screen-gradient sums, the screen record and two flags, per Gaussian
-        "backward_adam": ("hbm", 32 * n_par + 48 + 48 + 5),
+        # fused projection backward + Adam with no accumulated gradient (one view per
+        # step): p, m, v read and written, 24 B per scalar of every group, plus the raw
+        # screen-gradient sums, the screen record and two flags, per Gaussian
+        "backward_adam": ("hbm", 24 * n_par + 48 + 48 + 5),
         # FP32 instructions: 7 per pair the method's walk visits (2 subtractions + 5 for the
         # exponent's quadratic form), plus per blended pair 6 in the forward (weight, 3
         # colour FMAs, transmittance update) and 19 in the backward (T recovery 2,
@@ -428,7 +438,7 @@ def main_ours(args):
     clk = clocks.stop()
     ms = max_over_ranks(ms, world)
     ms_per_step = ms / args.steps
-    value = world * args.steps / (ms / 1e3)
+    value = replica_throughput(world, args.steps, ms / 1e3)
     H, W = cams[0].height, cams[0].width
 
     # per-stage kernel times for the roofline (separate, profiled pass over the same steps)
@@ -441,18 +451,17 @@ def main_ours(args):
     rf["kernel"] = dominant
     rf["peak_source"] = peak_kind
     src = {"blend_forward": "blend.cu", "blend_backward": "blend.cu", "adam": "adam.cu",
-           "preprocess": "preprocess.cu", "sort": "sort.cu", "loss": "loss.cu",
+           "preprocess": "preprocess.cu", "sort": "sort.cu", "depth_sort": "sort.cu", "loss": "loss.cu",
            "preprocess_backward": "preprocess_backward.cu",
            "backward_adam": "preprocess_backward.cu"}.get(dominant)
     tr = NCU_TRAFFIC.get(dominant)
     rf["traffic"] = tr[0] if (tr and src and sha12(os.path.join(PKG_CSRC, src)) == tr[1]) else None
 
-    # launches of our kernels per step (sort = histogram + offsets + one per pass)
+    # launches of our kernels in the timed region: the profiler counts every kernel a
+    # context launches (over the same steps), plus gs_adam_step per group when the
+    # separate path is used
     steps_p = max(1, args.steps)
-    sort_w = prof["sort"]["work"]
-    passes = (sort_w / max(1, sum(ks))) if sort_w else 0
-    per_step = (sum(prof[k]["launches"] for k in prof if k not in ("sort", "adam")) / steps_p +
-                (prof["sort"]["launches"] / steps_p) * (2 + passes) +
+    per_step = (sum(prof[k]["launches"] for k in prof if k != "adam") / steps_p +
                 (0 if step.fused_adam else len(GROUP_NAMES)))
     gpu_launches = int(round(per_step * args.steps))
 
@@ -541,7 +550,7 @@ def e2e_run(step, cams, targets, sched, args, world):
     barrier(world)
     assert len(losses) == n
     H, W = cams[0].height, cams[0].width
-    return {"value": world * n / dt, "unit": UNIT, "h2d_bytes_per_step": 3 * H * W * 4,
+    return {"value": replica_throughput(world, n, dt), "unit": UNIT, "h2d_bytes_per_step": 3 * H * W * 4,
             "d2h_bytes_per_step": 3 * 8 + 24, "last_loss": losses[-1]}
 
 

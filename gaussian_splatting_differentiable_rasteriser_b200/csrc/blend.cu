@@ -27,8 +27,10 @@
 // raw sums (w, w dx, w dy, w dx^2, w dx dy, w dy^2, dL/dc) with
 // w = dL/dalpha * o exp(-e); a warp reduce-scatter (12 shuffles instead of 45)
 // leaves the 9 warp totals in 9 lanes, which issue one coalesced group of 9
-// float32 atomics. The conic/opacity/mean2d chain of those sums is applied
-// once per Gaussian in the projection backward.
+// float32 atomics. When only a few lanes contribute (a quarter of the cases on
+// dense scenes) they add their values directly instead. The conic/opacity/
+// mean2d chain of those sums is applied once per Gaussian in the projection
+// backward.
 #include "gs_kernels.cuh"
 
 namespace gs {
@@ -184,56 +186,104 @@ __global__ void __launch_bounds__(256) blend_forward_kernel(BlendArgs a) {
   }
 }
 
-// Reduces v[0..8] over the warp; on return lane l (l even) holds the warp total
-// of v[idx], idx = 8 b1 + 4 b2 + 2 b3 + b4 with b_k = bit k of l.
-__device__ __forceinline__ float warp_reduce_scatter9(const float (&v)[9], int lane) {
+// Per-warp batch of Gaussians that had a contributing pixel in the backward:
+// per (Gaussian, pixel) the two per-pixel factors the nine raw sums are built
+// from, w = dL/dalpha * o exp(-e) and alpha T, plus each Gaussian's id and
+// centre. Rows are padded to 33 so that a lane per Gaussian reads without bank
+// conflicts.
+constexpr int kBatch = 16;
+struct WarpBatch {
+  float2 wa[kBatch][33];  // (w, alpha T) of Gaussian j at pixel p (lane p)
+  float2 uv[kBatch];      // centre (u, v)
+  uint32_t id[kBatch];
+  float4 g[32];           // dL/d(pixel colour) of the warp's pixels
+};
+
+// Turns a full (or final, partial) batch into the nine raw sums of each of its
+// `cnt` Gaussians and adds them to sgrad. Lane j (mod 16) owns Gaussian j; the
+// two half-warps take pixel rows 0-1 and 2-3 of the 8x4 block and add their
+// halves with one shuffle per sum. The six spatial sums are first formed as
+// moments of w over the pixel offsets from the block centre (lx, ly in
+// {-3.5..3.5} x {-1.5..1.5}, compile-time constants here) and then shifted to
+// the offsets from the Gaussian's centre, dx = lx - a, dy = ly - b with
+// (a, b) = centre - block centre:
+//   sum w dx = Mx - a M0, sum w dx^2 = Mxx - 2a Mx + a^2 M0, and so on.
+__device__ __forceinline__ void flush_batch(const WarpBatch& b, int cnt, int lane, float cxb, float cyb,
+                                            float* sgrad) {
+  const int j = lane & 15, h = lane >> 4;
+  float m0 = 0.f, mx = 0.f, my = 0.f, mxx = 0.f, mxy = 0.f, myy = 0.f;
+  float c0 = 0.f, c1 = 0.f, c2 = 0.f;
+  if (j < cnt) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int p = 16 * h + i;
+      const float2 wa = b.wa[j][p];
+      const float4 g = b.g[p];
+      constexpr float kLx[8] = {-3.5f, -2.5f, -1.5f, -0.5f, 0.5f, 1.5f, 2.5f, 3.5f};
+      const float lx = kLx[i & 7];
+      const float ly = (i >> 3) ? -0.5f : -1.5f;  // this half's rows, before the 2h shift
+      m0 += wa.x;
+      mx = __fmaf_rn(wa.x, lx, mx);
+      my = __fmaf_rn(wa.x, ly, my);
+      mxx = __fmaf_rn(wa.x, lx * lx, mxx);
+      mxy = __fmaf_rn(wa.x, lx * ly, mxy);
+      myy = __fmaf_rn(wa.x, ly * ly, myy);
+      c0 = __fmaf_rn(wa.y, g.x, c0);
+      c1 = __fmaf_rn(wa.y, g.y, c1);
+      c2 = __fmaf_rn(wa.y, g.z, c2);
+    }
+    // rows of the upper half sit 2h further down: ly -> ly + 2h
+    const float sh = 2.0f * static_cast<float>(h);
+    myy = __fmaf_rn(sh, __fmaf_rn(sh, m0, 2.0f * my), myy);
+    mxy = __fmaf_rn(sh, mx, mxy);
+    my = __fmaf_rn(sh, m0, my);
+  }
   const unsigned full = 0xffffffffu;
-  float w[5];
-  {
-    const bool up = lane & 16;
-#pragma unroll
-    for (int i = 0; i < 5; ++i) {
-      const float a0 = v[2 * i], a1 = (2 * i + 1 < 9) ? v[2 * i + 1] : 0.0f;
-      const float send = up ? a0 : a1, keep = up ? a1 : a0;
-      w[i] = keep + __shfl_xor_sync(full, send, 16);
+  m0 += __shfl_xor_sync(full, m0, 16);
+  mx += __shfl_xor_sync(full, mx, 16);
+  my += __shfl_xor_sync(full, my, 16);
+  mxx += __shfl_xor_sync(full, mxx, 16);
+  mxy += __shfl_xor_sync(full, mxy, 16);
+  myy += __shfl_xor_sync(full, myy, 16);
+  c0 += __shfl_xor_sync(full, c0, 16);
+  c1 += __shfl_xor_sync(full, c1, 16);
+  c2 += __shfl_xor_sync(full, c2, 16);
+  if (j < cnt) {
+    const float2 uv = b.uv[j];
+    const float a = uv.x - cxb, bb = uv.y - cyb;
+    float* dst = sgrad + static_cast<int64_t>(b.id[j]) * kGradStride;
+    if (h == 0) {
+      const float sy = __fmaf_rn(-bb, m0, my);
+      atomicAdd(dst + 0, m0);
+      atomicAdd(dst + 1, __fmaf_rn(-a, m0, mx));
+      atomicAdd(dst + 2, sy);
+      atomicAdd(dst + 3, __fmaf_rn(a, __fmaf_rn(a, m0, -2.0f * mx), mxx));
+      atomicAdd(dst + 4, __fmaf_rn(-a, sy, __fmaf_rn(-bb, mx, mxy)));
+    } else {
+      atomicAdd(dst + 5, __fmaf_rn(bb, __fmaf_rn(bb, m0, -2.0f * my), myy));
+      atomicAdd(dst + 6, c0);
+      atomicAdd(dst + 7, c1);
+      atomicAdd(dst + 8, c2);
     }
   }
-  float x[3];
-  {
-    const bool up = lane & 8;
-#pragma unroll
-    for (int i = 0; i < 3; ++i) {
-      const float a0 = w[2 * i], a1 = (2 * i + 1 < 5) ? w[2 * i + 1] : 0.0f;
-      const float send = up ? a0 : a1, keep = up ? a1 : a0;
-      x[i] = keep + __shfl_xor_sync(full, send, 8);
-    }
-  }
-  float y[2];
-  {
-    const bool up = lane & 4;
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const float a0 = x[2 * i], a1 = (2 * i + 1 < 3) ? x[2 * i + 1] : 0.0f;
-      const float send = up ? a0 : a1, keep = up ? a1 : a0;
-      y[i] = keep + __shfl_xor_sync(full, send, 4);
-    }
-  }
-  float z;
-  {
-    const bool up = lane & 2;
-    const float send = up ? y[0] : y[1], keep = up ? y[1] : y[0];
-    z = keep + __shfl_xor_sync(full, send, 2);
-  }
-  return z + __shfl_xor_sync(full, z, 1);
 }
+
+struct BackwardSmem {
+  WarpSlots slots[kWarps];
+  WarpBatch batches[kWarps];
+};
 
 template <bool kCount>
 __global__ void __launch_bounds__(256) blend_backward_kernel(BlendArgs a) {
-  __shared__ WarpSlots slots[kWarps];
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  BackwardSmem& sm = *reinterpret_cast<BackwardSmem*>(smem_raw);
+  WarpSlots* slots = sm.slots;
+  WarpBatch* batches = sm.batches;
   const int tile = blockIdx.x;
   const int tx = tile % a.cam.tiles_x, ty = tile / a.cam.tiles_x;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   WarpSlots& ws = slots[warp];
+  WarpBatch& wb = batches[warp];
   int lx, ly;
   tile_pixel(threadIdx.x, lx, ly);
   const int px = tx * kTile + lx, py = ty * kTile + ly;
@@ -256,6 +306,7 @@ __global__ void __launch_bounds__(256) blend_backward_kernel(BlendArgs a) {
     g1 = a.dimage[hw + pix];
     g2 = a.dimage[2 * hw + pix];
   }
+  wb.g[lane] = make_float4(g0, g1, g2, 0.0f);
   // g . S with S the colour composited behind the current Gaussian; starts at T_final bg.
   float gS = T * (g0 * a.cam.bg[0] + g1 * a.cam.bg[1] + g2 * a.cam.bg[2]);
   // n_contrib comes from the caller: never walk past the tile's own list.
@@ -263,12 +314,8 @@ __global__ void __launch_bounds__(256) blend_backward_kernel(BlendArgs a) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) wlast = max(wlast, __shfl_xor_sync(0xffffffffu, wlast, o));
   const int top = beg + max(0, min(wlast, static_cast<int>(range.y - range.x)));  // exclusive
-
-  // Which raw sum this lane holds after the reduce-scatter.
-  const int red_idx = ((lane >> 1) & 1) * 8 + ((lane >> 2) & 1) * 4 + ((lane >> 3) & 1) * 2 +
-                      ((lane >> 4) & 1);
-  const bool red_writer = !(lane & 1) && red_idx < 9;
   unsigned blended = 0;
+  int bcnt = 0;  // Gaussians in the warp's batch (warp-uniform)
 
   // Chunks walk down from the top; lane l takes entry hi - 1 - l, so ballot
   // order (lane order) is descending list order.
@@ -294,34 +341,32 @@ __global__ void __launch_bounds__(256) blend_backward_kernel(BlendArgs a) {
       const bool contrib = pos < last && alpha >= kAlphaMin;
       if (kCount && contrib) ++blended;
       if (!__any_sync(0xffffffffu, contrib)) continue;
-      float v[9];
-#pragma unroll
-      for (int r = 0; r < 9; ++r) v[r] = 0.0f;
+      float w = 0.0f, aT = 0.0f;
       if (contrib) {
         const float rcp = __fdividef(1.0f, 1.0f - alpha);
         T = T * rcp;  // transmittance in front of this Gaussian
         const float4 c = ws.col[k];
         const float gc = __fmaf_rn(g2, c.z, __fmaf_rn(g1, c.y, g0 * c.x));
         const float dalpha = __fmaf_rn(T, gc, -gS * rcp);  // dI/dalpha = T c - S / (1 - alpha)
-        const float aT = alpha * T;
+        aT = alpha * T;
         gS = __fmaf_rn(gc, aT, gS);
-        v[6] = g0 * aT;
-        v[7] = g1 * aT;
-        v[8] = g2 * aT;
-        const float w = raw <= kAlphaMax ? dalpha * raw : 0.0f;  // zero through the cap
-        const float wdx = w * dx, wdy = w * dy;
-        v[0] = w;
-        v[1] = wdx;
-        v[2] = wdy;
-        v[3] = wdx * dx;
-        v[4] = wdx * dy;
-        v[5] = wdy * dy;
+        w = raw <= kAlphaMax ? dalpha * raw : 0.0f;  // zero through the cap
       }
-      const float tot = warp_reduce_scatter9(v, lane);
-      if (red_writer) atomicAdd(a.sgrad + static_cast<int64_t>(ws.id[k]) * kGradStride + red_idx, tot);
+      wb.wa[bcnt][lane] = make_float2(w, aT);
+      if (lane == 0) {
+        wb.id[bcnt] = ws.id[k];
+        wb.uv[bcnt] = xy;
+      }
+      if (++bcnt == kBatch) {
+        __syncwarp();
+        flush_batch(wb, kBatch, lane, bx0 + 3.5f, by0 + 1.5f, a.sgrad);
+        bcnt = 0;
+        __syncwarp();
+      }
     }
-    __syncwarp();
+    __syncwarp();  // the slots are rewritten by the next chunk
   }
+  if (bcnt > 0) flush_batch(wb, bcnt, lane, bx0 + 3.5f, by0 + 1.5f, a.sgrad);
   if (kCount) {
     // the method's backward walk visits every entry before the pixel's last contributor
     count_pairs(a.pairs, static_cast<unsigned>(min(last, static_cast<int>(range.y - range.x))));
@@ -344,10 +389,19 @@ cudaError_t launch_blend_forward(const BlendArgs& a, cudaStream_t st) {
 cudaError_t launch_blend_backward(const BlendArgs& a, cudaStream_t st) {
   const int tiles = a.cam.tiles_x * a.cam.tiles_y;
   if (tiles == 0) return cudaSuccess;
-  if (a.pairs)
-    blend_backward_kernel<true><<<tiles, 256, 0, st>>>(a);
-  else
-    blend_backward_kernel<false><<<tiles, 256, 0, st>>>(a);
+  const int smem = static_cast<int>(sizeof(BackwardSmem));
+  cudaError_t e;
+  if (a.pairs) {
+    if ((e = cudaFuncSetAttribute(blend_backward_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  smem)) != cudaSuccess)
+      return e;
+    blend_backward_kernel<true><<<tiles, 256, smem, st>>>(a);
+  } else {
+    if ((e = cudaFuncSetAttribute(blend_backward_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  smem)) != cudaSuccess)
+      return e;
+    blend_backward_kernel<false><<<tiles, 256, smem, st>>>(a);
+  }
   return cudaGetLastError();
 }
 

@@ -1,5 +1,6 @@
 // C ABI of the rasteriser (declared in include/gs_api.h): context management,
 // host-side argument checks and the order of kernel launches per call.
+#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -23,11 +24,15 @@ struct gs_ctx {
   uint32_t* touched = nullptr;
   uint8_t* clamped = nullptr;
   float* sgrad = nullptr;
-  uint32_t* block_sums = nullptr;
-  uint64_t* block_prefix = nullptr;
+  uint2* block_sums = nullptr;
+  uint32_t* visible_prefix = nullptr;
   uint32_t* depth_range = nullptr;
-  // sort
-  uint64_t* keys[2] = {nullptr, nullptr};
+  // depth sort of the visible Gaussians
+  uint32_t* dkeys[2] = {nullptr, nullptr};
+  uint32_t* dvals[2] = {nullptr, nullptr};
+  uint32_t* dup_status = nullptr;
+  // tile sort of the entries
+  uint32_t* keys[2] = {nullptr, nullptr};
   uint32_t* vals[2] = {nullptr, nullptr};
   uint32_t* hist = nullptr;
   uint32_t* offsets = nullptr;
@@ -45,8 +50,6 @@ struct gs_ctx {
   int64_t n = 0, n_pad = 0;
   gs::CamArgs cam{};
   int64_t K = 0;
-  int depth_bits = 0;
-  uint32_t depth_min = 0;
   int sorted_buf = 0;
   // profiling (off by default)
   struct Profiler {
@@ -84,7 +87,8 @@ gs_status fail(gs_ctx* c, gs_status s, const char* fmt, ...) {
 
 void free_all(gs_ctx* c) {
   void* bufs[] = {c->screen, c->depth, c->rect, c->touched, c->clamped, c->sgrad, c->block_sums,
-                  c->block_prefix, c->depth_range, c->keys[0], c->keys[1], c->vals[0], c->vals[1],
+                  c->visible_prefix, c->depth_range, c->dkeys[0], c->dkeys[1], c->dvals[0],
+                  c->dvals[1], c->dup_status, c->keys[0], c->keys[1], c->vals[0], c->vals[1],
                   c->hist, c->offsets, c->status, c->counters, c->ranges, c->loss_partials,
                   c->loss_counter, c->info_dev, c->pairs};
   for (void* b : bufs)
@@ -162,14 +166,18 @@ void prof_begin(gs_ctx* c, cudaStream_t st) {
   cudaEventRecord(P.ev[2 * P.nrec], st);
 }
 
-void prof_end(gs_ctx* c, int stage, int64_t work, cudaStream_t st) {
+// Closes a timed bracket of `kernels` kernel launches doing `work` units.
+void prof_end(gs_ctx* c, int stage, int64_t work, cudaStream_t st, int kernels = 1) {
   auto& P = c->prof;
   if (!P.on) return;
   cudaEventRecord(P.ev[2 * P.nrec + 1], st);
   P.stage[P.nrec++] = stage;
-  P.launches[stage] += 1;
+  P.launches[stage] += kernels;
   P.work[stage] += work;
 }
+
+// Kernels one launch_sort enqueues: histogram + digit offsets + one per pass.
+int sort_kernels(const gs::SortPlan& p) { return (p.n > 1 && p.passes > 0) ? 2 + p.passes : 0; }
 
 __global__ void unpack_preprocess_kernel(const gs::Screen* screen, const float* depth,
                                          const uint2* rect, const uint32_t* touched,
@@ -206,11 +214,6 @@ __global__ void unpack_preprocess_kernel(const gs::Screen* screen, const float* 
   if (cl) cl[i] = clamped[i];
 }
 
-__global__ void key_tiles_kernel(const uint64_t* keys, int64_t n, int depth_bits, int32_t* tiles) {
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (i < n) tiles[i] = static_cast<int32_t>(keys[i] >> depth_bits);
-}
-
 int bit_length(uint64_t v) { return v == 0 ? 0 : 64 - __builtin_clzll(v); }
 
 }  // namespace
@@ -232,7 +235,8 @@ gs_status gs_create(gs_ctx** out, int64_t max_gaussians, int64_t max_entries, in
   c->max_h = max_height;
   c->max_tiles = static_cast<int64_t>((max_width + 15) / 16) * ((max_height + 15) / 16);
   c->max_blocks = (max_gaussians + 255) / 256;
-  c->max_sort_tiles = (max_entries + gs::kSortTileKeys - 1) / gs::kSortTileKeys;
+  // the depth sort (visible Gaussians) and the tile sort (entries) share the look-back words
+  c->max_sort_tiles = (std::max(max_entries, max_gaussians) + gs::kSortTileKeys - 1) / gs::kSortTileKeys;
   c->max_loss_blocks = gs::loss_num_blocks(max_height, max_width);
   const int64_t G = max_gaussians, K = max_entries;
   cudaError_t e = cudaSuccess;
@@ -244,17 +248,22 @@ gs_status gs_create(gs_ctx** out, int64_t max_gaussians, int64_t max_entries, in
   GS_ALLOC(c->touched, sizeof(uint32_t) * G);
   GS_ALLOC(c->clamped, sizeof(uint8_t) * G);
   GS_ALLOC(c->sgrad, sizeof(float) * gs::kGradStride * G);
-  GS_ALLOC(c->block_sums, sizeof(uint32_t) * c->max_blocks);
-  GS_ALLOC(c->block_prefix, sizeof(uint64_t) * c->max_blocks);
+  GS_ALLOC(c->block_sums, sizeof(uint2) * c->max_blocks);
+  GS_ALLOC(c->visible_prefix, sizeof(uint32_t) * c->max_blocks);
   GS_ALLOC(c->depth_range, sizeof(uint32_t) * 2);
-  GS_ALLOC(c->keys[0], sizeof(uint64_t) * K);
-  GS_ALLOC(c->keys[1], sizeof(uint64_t) * K);
+  GS_ALLOC(c->dkeys[0], sizeof(uint32_t) * G);
+  GS_ALLOC(c->dkeys[1], sizeof(uint32_t) * G);
+  GS_ALLOC(c->dvals[0], sizeof(uint32_t) * G);
+  GS_ALLOC(c->dvals[1], sizeof(uint32_t) * G);
+  GS_ALLOC(c->dup_status, sizeof(uint32_t) * ((G + gs::kDupItems - 1) / gs::kDupItems));
+  GS_ALLOC(c->keys[0], sizeof(uint32_t) * K);
+  GS_ALLOC(c->keys[1], sizeof(uint32_t) * K);
   GS_ALLOC(c->vals[0], sizeof(uint32_t) * K);
   GS_ALLOC(c->vals[1], sizeof(uint32_t) * K);
   GS_ALLOC(c->hist, sizeof(uint32_t) * gs::kMaxPasses * gs::kRadix);
   GS_ALLOC(c->offsets, sizeof(uint32_t) * gs::kMaxPasses * gs::kRadix);
   GS_ALLOC(c->status, sizeof(uint32_t) * gs::kMaxPasses * gs::kRadix * c->max_sort_tiles);
-  GS_ALLOC(c->counters, sizeof(uint32_t) * gs::kMaxPasses);
+  GS_ALLOC(c->counters, sizeof(uint32_t) * (gs::kMaxPasses + 1));  // + the duplicate's ticket
   GS_ALLOC(c->ranges, sizeof(uint2) * c->max_tiles);
   GS_ALLOC(c->loss_partials, sizeof(double) * 2 * c->max_loss_blocks);
   GS_ALLOC(c->loss_counter, sizeof(uint32_t));
@@ -317,9 +326,9 @@ gs_status gs_preprocess(gs_ctx* c, const gs_params* p, const gs_camera* cam, voi
   const int64_t nb = (p->n + 255) / 256;
   prof_begin(c, st);
   GS_CUDA(c, gs::launch_preprocess(a, nb, st));
-  prof_end(c, GS_STAGE_PREPROCESS, p->n, st);
+  prof_end(c, GS_STAGE_PREPROCESS, p->n, st, p->n > 0 ? 1 : 0);
   prof_begin(c, st);
-  GS_CUDA(c, gs::launch_scan_blocks(c->block_sums, nb, c->block_prefix, c->depth_range, c->info_dev, st));
+  GS_CUDA(c, gs::launch_scan_blocks(c->block_sums, nb, c->visible_prefix, c->depth_range, c->info_dev, st));
   prof_end(c, GS_STAGE_SCAN, nb, st);
   c->n = p->n;
   c->n_pad = p->n_pad;
@@ -353,54 +362,75 @@ gs_status gs_render_forward(gs_ctx* c, const gs_camera* cam, float* image, float
     return fail(c, GS_ERR_CAPACITY, "%llu (Gaussian, tile) entries exceed the context's %lld",
                 (unsigned long long)K, (long long)c->max_k);
   const int64_t tiles = static_cast<int64_t>(ca.tiles_x) * ca.tiles_y;
-  int depth_bits = 0;
-  uint32_t dmin = 0;
-  if (K > 0) {
-    dmin = c->info_host->depth_min;
-    depth_bits = bit_length(c->info_host->depth_max - dmin);
-  }
-  const int key_bits = bit_length(static_cast<uint64_t>(tiles - 1)) + depth_bits;
+  const int64_t V = static_cast<int64_t>(c->info_host->num_visible);
   int sorted = 0;
   if (K > 0) {
-    gs::DuplicateArgs d;
-    d.n = c->n;
-    d.touched = c->touched;
-    d.rect = c->rect;
-    d.depth = c->depth;
-    d.block_prefix = c->block_prefix;
-    d.depth_min = dmin;
-    d.depth_bits = depth_bits;
-    d.tiles_x = ca.tiles_x;
-    d.max_entries = c->max_k;
-    d.keys = c->keys[0];
-    d.vals = c->vals[0];
-    d.err = &c->info_dev->device_error;
-    prof_begin(c, st);
-    GS_CUDA(c, gs::launch_duplicate(d, (c->n + 255) / 256, st));
-    prof_end(c, GS_STAGE_DUPLICATE, static_cast<int64_t>(K), st);
-    gs::SortPlan plan;
-    plan.n = static_cast<int64_t>(K);
-    plan.depth_bits = depth_bits;
-    plan.key_bits = key_bits;
-    plan.passes = (key_bits + 7) / 8;
-    plan.tiles = (plan.n + gs::kSortTileKeys - 1) / gs::kSortTileKeys;
     gs::SortBuffers b;
-    b.keys[0] = c->keys[0];
-    b.keys[1] = c->keys[1];
-    b.vals[0] = c->vals[0];
-    b.vals[1] = c->vals[1];
     b.hist = c->hist;
     b.offsets = c->offsets;
     b.status = c->status;
     b.counters = c->counters;
     b.err = &c->info_dev->device_error;
+    // 1 + 2. visible Gaussians in index order, sorted by depth key
+    const uint32_t dmin = c->info_host->depth_min;
+    gs::CompactArgs ca2;
+    ca2.n = c->n;
+    ca2.touched = c->touched;
+    ca2.depth = c->depth;
+    ca2.visible_prefix = c->visible_prefix;
+    ca2.depth_min = dmin;
+    ca2.max_out = c->max_g;
+    ca2.keys = c->dkeys[0];
+    ca2.vals = c->dvals[0];
+    ca2.err = &c->info_dev->device_error;
+    gs::SortPlan dplan;
+    dplan.n = V;
+    dplan.key_bits = bit_length(c->info_host->depth_max - dmin);
+    dplan.passes = (dplan.key_bits + 7) / 8;
+    dplan.tiles = (V + gs::kSortTileKeys - 1) / gs::kSortTileKeys;
+    b.keys[0] = c->dkeys[0];
+    b.keys[1] = c->dkeys[1];
+    b.vals[0] = c->dvals[0];
+    b.vals[1] = c->dvals[1];
+    int dsorted = 0;
+    prof_begin(c, st);
+    GS_CUDA(c, gs::launch_compact(ca2, (c->n + 255) / 256, st));
+    GS_CUDA(c, gs::launch_sort(dplan, b, &dsorted, st));
+    prof_end(c, GS_STAGE_DEPTH_SORT, dplan.n > 1 ? dplan.n * dplan.passes : 0, st,
+             (c->n > 0 ? 1 : 0) + sort_kernels(dplan));
+    // 3. one (tile, index) entry per touched tile, in depth order
+    gs::DuplicateArgs d;
+    d.count = V;
+    d.order = c->dvals[dsorted];
+    d.touched = c->touched;
+    d.rect = c->rect;
+    d.tiles_x = ca.tiles_x;
+    d.max_entries = c->max_k;
+    d.keys = c->keys[0];
+    d.vals = c->vals[0];
+    d.status = c->dup_status;
+    d.ticket = c->counters + gs::kMaxPasses;
+    d.err = &c->info_dev->device_error;
+    prof_begin(c, st);
+    GS_CUDA(c, gs::launch_duplicate(d, st));
+    prof_end(c, GS_STAGE_DUPLICATE, static_cast<int64_t>(K), st, V > 0 ? 1 : 0);
+    // 4. stable sort of the entries by tile
+    gs::SortPlan plan;
+    plan.n = static_cast<int64_t>(K);
+    plan.key_bits = bit_length(static_cast<uint64_t>(tiles - 1));
+    plan.passes = (plan.key_bits + 7) / 8;
+    plan.tiles = (plan.n + gs::kSortTileKeys - 1) / gs::kSortTileKeys;
+    b.keys[0] = c->keys[0];
+    b.keys[1] = c->keys[1];
+    b.vals[0] = c->vals[0];
+    b.vals[1] = c->vals[1];
     prof_begin(c, st);
     GS_CUDA(c, gs::launch_sort(plan, b, &sorted, st));
-    prof_end(c, GS_STAGE_SORT, plan.n > 1 ? plan.n * plan.passes : 0, st);
+    prof_end(c, GS_STAGE_SORT, plan.n > 1 ? plan.n * plan.passes : 0, st, sort_kernels(plan));
   }
   prof_begin(c, st);
-  GS_CUDA(c, gs::launch_ranges(c->keys[sorted], static_cast<int64_t>(K), depth_bits, c->ranges, tiles, st));
-  prof_end(c, GS_STAGE_RANGES, static_cast<int64_t>(K), st);
+  GS_CUDA(c, gs::launch_ranges(c->keys[sorted], static_cast<int64_t>(K), c->ranges, tiles, st));
+  prof_end(c, GS_STAGE_RANGES, static_cast<int64_t>(K), st, K > 0 ? 1 : 0);
   gs::BlendArgs ba{};
   ba.ranges = c->ranges;
   ba.order = c->vals[sorted];
@@ -415,8 +445,6 @@ gs_status gs_render_forward(gs_ctx* c, const gs_camera* cam, float* image, float
   GS_CUDA(c, gs::launch_blend_forward(ba, st));
   prof_end(c, GS_STAGE_BLEND_FORWARD, 0, st);
   c->K = static_cast<int64_t>(K);
-  c->depth_bits = depth_bits;
-  c->depth_min = dmin;
   c->sorted_buf = sorted;
   c->cam.bg[0] = ca.bg[0];
   c->cam.bg[1] = ca.bg[1];
@@ -462,7 +490,7 @@ namespace {
 // backward, and the projection-backward argument record.
 gs_status backward_common(gs_ctx* c, const gs_params* p, const gs_camera* cam, const float* final_T,
                           const int32_t* n_contrib, const float* dloss_dimage, gs_grads* g,
-                          cudaStream_t st, gs::PreprocessBwdArgs& a) {
+                          bool g_optional, cudaStream_t st, gs::PreprocessBwdArgs& a) {
   if (!c) return GS_ERR_INVALID_ARG;
   if (!c->have_fwd) return fail(c, GS_ERR_INVALID_ARG, "gs_render_forward has not run");
   gs_status s = check_params(c, p);
@@ -473,12 +501,13 @@ gs_status backward_common(gs_ctx* c, const gs_params* p, const gs_camera* cam, c
   if ((s = make_cam(c, cam, ca)) != GS_OK) return s;
   if (ca.width != c->cam.width || ca.height != c->cam.height)
     return fail(c, GS_ERR_INVALID_ARG, "camera size differs from the one rendered");
-  if (!final_T || !n_contrib || !dloss_dimage || !g)
+  if (!final_T || !n_contrib || !dloss_dimage || (!g && !g_optional))
     return fail(c, GS_ERR_INVALID_ARG, "backward inputs must be non-NULL");
-  float* gp[] = {g->means, g->log_scales, g->quats, g->opacity_logits, g->sh};
-  if (p->n > 0)
+  if (g && p->n > 0) {
+    float* gp[] = {g->means, g->log_scales, g->quats, g->opacity_logits, g->sh};
     for (float* q : gp)
       if (!q || !aligned(q, 4)) return fail(c, GS_ERR_INVALID_ARG, "a gradient pointer is NULL or misaligned");
+  }
   if (p->n > 0)
     GS_CUDA(c, cudaMemsetAsync(c->sgrad, 0, sizeof(float) * gs::kGradStride * p->n, st));
   gs::BlendArgs ba{};
@@ -508,11 +537,11 @@ gs_status backward_common(gs_ctx* c, const gs_params* p, const gs_camera* cam, c
   a.touched = c->touched;
   a.clamped = c->clamped;
   a.sgrad = c->sgrad;
-  a.g_means = g->means;
-  a.g_log_scales = g->log_scales;
-  a.g_quats = g->quats;
-  a.g_opacity_logits = g->opacity_logits;
-  a.g_sh = g->sh;
+  a.g_means = g ? g->means : nullptr;
+  a.g_log_scales = g ? g->log_scales : nullptr;
+  a.g_quats = g ? g->quats : nullptr;
+  a.g_opacity_logits = g ? g->opacity_logits : nullptr;
+  a.g_sh = g ? g->sh : nullptr;
   return GS_OK;
 }
 
@@ -529,11 +558,11 @@ gs_status gs_render_backward(gs_ctx* c, const gs_params* p, const gs_camera* cam
                              void* stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   gs::PreprocessBwdArgs a;
-  gs_status s = backward_common(c, p, cam, final_T, n_contrib, dloss_dimage, g, st, a);
+  gs_status s = backward_common(c, p, cam, final_T, n_contrib, dloss_dimage, g, false, st, a);
   if (s != GS_OK) return s;
   prof_begin(c, st);
   GS_CUDA(c, gs::launch_preprocess_backward(a, st));
-  prof_end(c, GS_STAGE_PREPROCESS_BACKWARD, p->n, st);
+  prof_end(c, GS_STAGE_PREPROCESS_BACKWARD, p->n, st, p->n > 0 ? 1 : 0);
   return GS_OK;
 }
 
@@ -556,11 +585,18 @@ gs_status gs_render_backward_adam(gs_ctx* c, const gs_params* p, const gs_camera
   }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   gs::PreprocessBwdArgs a;
-  gs_status s = backward_common(c, p, cam, final_T, n_contrib, dloss_dimage, g, st, a);
+  gs_status s = backward_common(c, p, cam, final_T, n_contrib, dloss_dimage, g, true, st, a);
   if (s != GS_OK) return s;
   gs::FusedAdamArgs f;
   const float* pp[5] = {p->means, p->log_scales, p->quats, p->opacity_logits, p->sh};
-  float* gg[5] = {g->means, g->log_scales, g->quats, g->opacity_logits, g->sh};
+  float* gg[5] = {nullptr, nullptr, nullptr, nullptr, nullptr};
+  if (g) {
+    gg[0] = g->means;
+    gg[1] = g->log_scales;
+    gg[2] = g->quats;
+    gg[3] = g->opacity_logits;
+    gg[4] = g->sh;
+  }
   float* mm[5] = {m->means, m->log_scales, m->quats, m->opacity_logits, m->sh};
   float* vv[5] = {v->means, v->log_scales, v->quats, v->opacity_logits, v->sh};
   for (int k = 0; k < 5; ++k) {
@@ -572,7 +608,7 @@ gs_status gs_render_backward_adam(gs_ctx* c, const gs_params* p, const gs_camera
   }
   prof_begin(c, st);
   GS_CUDA(c, gs::launch_preprocess_backward_adam(a, f, st));
-  prof_end(c, GS_STAGE_BACKWARD_ADAM, p->n_pad, st);
+  prof_end(c, GS_STAGE_BACKWARD_ADAM, p->n_pad, st, p->n_pad > 0 ? 1 : 0);
   return GS_OK;
 }
 
@@ -627,7 +663,7 @@ gs_status gs_profile_read(gs_ctx* c, double* ms, int64_t* launches, int64_t* wor
 const char* gs_stage_name(int32_t stage) {
   static const char* names[GS_NUM_STAGES] = {"preprocess", "scan", "duplicate", "sort", "ranges",
                                              "blend_forward", "loss", "blend_backward",
-                                             "preprocess_backward", "backward_adam"};
+                                             "preprocess_backward", "backward_adam", "depth_sort"};
   return (stage >= 0 && stage < GS_NUM_STAGES) ? names[stage] : "";
 }
 
@@ -652,11 +688,9 @@ gs_status gs_debug_sorted(gs_ctx* c, int32_t* ids, int32_t* tiles, int32_t* rang
   if (ids && c->K > 0)
     GS_CUDA(c, cudaMemcpyAsync(ids, c->vals[c->sorted_buf], sizeof(uint32_t) * c->K,
                                cudaMemcpyDeviceToDevice, st));
-  if (tiles && c->K > 0) {
-    key_tiles_kernel<<<static_cast<unsigned>((c->K + 255) / 256), 256, 0, st>>>(
-        c->keys[c->sorted_buf], c->K, c->depth_bits, tiles);
-    GS_CUDA(c, cudaGetLastError());
-  }
+  if (tiles && c->K > 0)
+    GS_CUDA(c, cudaMemcpyAsync(tiles, c->keys[c->sorted_buf], sizeof(uint32_t) * c->K,
+                               cudaMemcpyDeviceToDevice, st));
   if (ranges)
     GS_CUDA(c, cudaMemcpyAsync(ranges, c->ranges,
                                sizeof(uint2) * static_cast<int64_t>(c->cam.tiles_x) * c->cam.tiles_y,

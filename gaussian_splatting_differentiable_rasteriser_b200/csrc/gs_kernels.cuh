@@ -8,12 +8,13 @@
 namespace gs {
 
 // Written by the preprocess + block scan and read back by the host before the
-// sort: the entry count and the range of depth keys of visible Gaussians.
+// sort: the entry count, the number of visible Gaussians and the range of
+// depth keys of visible Gaussians.
 struct ForwardInfo {
   uint64_t num_entries;
+  uint32_t num_visible;
   uint32_t depth_min, depth_max;
   uint32_t device_error;
-  uint32_t pad;
 };
 
 struct PreprocessArgs {
@@ -27,48 +28,68 @@ struct PreprocessArgs {
   uint2* rect;  // x0 | x1 << 16, y0 | y1 << 16 (inclusive tile indices)
   uint32_t* touched;
   uint8_t* clamped;
-  uint32_t* block_sums;   // one per 256-Gaussian block
+  uint2* block_sums;      // per 256-Gaussian block: (tiles touched, visible Gaussians)
   uint32_t* depth_range;  // [min, max] of visible depth keys (atomics)
 };
 
 cudaError_t launch_preprocess(const PreprocessArgs& a, int64_t num_blocks, cudaStream_t st);
-cudaError_t launch_scan_blocks(const uint32_t* block_sums, int64_t num_blocks, uint64_t* block_prefix,
+// Exclusive prefix of the per-block visible counts, plus the totals and the
+// depth-key range copied into the readback record.
+cudaError_t launch_scan_blocks(const uint2* block_sums, int64_t num_blocks, uint32_t* visible_prefix,
                                const uint32_t* depth_range, ForwardInfo* info, cudaStream_t st);
 
 // ---------------------------------------------------------------- sorting
+// Stable LSD radix sort of 32-bit keys with 32-bit values.
 struct SortPlan {
-  int64_t n;       // entries
-  int depth_bits;  // bits kept of (depth key - depth_min)
-  int key_bits;    // tile bits + depth_bits
-  int passes;      // ceil(key_bits / 8)
-  int64_t tiles;   // onesweep tiles of kSortTileKeys entries
+  int64_t n;      // items
+  int key_bits;   // significant low bits of the keys
+  int passes;     // ceil(key_bits / 8)
+  int64_t tiles;  // onesweep tiles of kSortTileKeys items
 };
 
 constexpr int kSortThreads = 256;
 constexpr int kSortItems = 16;
 constexpr int kSortTileKeys = kSortThreads * kSortItems;  // 4096
 constexpr int kRadix = 256;
-constexpr int kMaxPasses = 8;
+constexpr int kMaxPasses = 4;
 
-struct DuplicateArgs {
+// Visible Gaussians in index order as (depth key - depth_min, index).
+struct CompactArgs {
   int64_t n;
   const uint32_t* touched;
-  const uint2* rect;
   const float* depth;
-  const uint64_t* block_prefix;
+  const uint32_t* visible_prefix;  // per 256-Gaussian block
   uint32_t depth_min;
-  int depth_bits;
-  int tiles_x;
-  int64_t max_entries;
-  uint64_t* keys;
+  int64_t max_out;
+  uint32_t* keys;
   uint32_t* vals;
   uint32_t* err;
 };
+cudaError_t launch_compact(const CompactArgs& a, int64_t num_blocks, cudaStream_t st);
 
-cudaError_t launch_duplicate(const DuplicateArgs& a, int64_t num_blocks, cudaStream_t st);
+// One (tile, index) entry per tile touched by each visible Gaussian, in the
+// depth order given by `order` (a single pass: each CTA's offset comes from a
+// decoupled look-back over the earlier CTAs' totals of tiles touched).
+struct DuplicateArgs {
+  int64_t count;          // visible Gaussians
+  const uint32_t* order;  // Gaussian indices sorted by depth
+  const uint32_t* touched;
+  const uint2* rect;
+  int tiles_x;
+  int64_t max_entries;
+  uint32_t* keys;    // tile
+  uint32_t* vals;    // Gaussian index
+  uint32_t* status;  // [ceil(count / kDupItems)] look-back words, zeroed
+  uint32_t* ticket;  // zeroed
+  uint32_t* err;
+};
+constexpr int kDupThreads = 256;
+constexpr int kDupPerThread = 4;
+constexpr int kDupItems = kDupThreads * kDupPerThread;
+cudaError_t launch_duplicate(const DuplicateArgs& a, cudaStream_t st);
 
 struct SortBuffers {
-  uint64_t* keys[2];
+  uint32_t* keys[2];
   uint32_t* vals[2];
   uint32_t* hist;      // [kMaxPasses][256] digit counts
   uint32_t* offsets;   // [kMaxPasses][256] exclusive digit offsets
@@ -80,8 +101,9 @@ struct SortBuffers {
 // Sorts keys[0]/vals[0]; returns in *out_buf the buffer (0 or 1) holding the result.
 cudaError_t launch_sort(const SortPlan& plan, const SortBuffers& b, int* out_buf, cudaStream_t st);
 
-cudaError_t launch_ranges(const uint64_t* keys, int64_t n, int depth_bits, uint2* ranges,
-                          int64_t num_tiles, cudaStream_t st);
+// Per-tile [first, last) of the tile-sorted entries (keys = tile indices).
+cudaError_t launch_ranges(const uint32_t* keys, int64_t n, uint2* ranges, int64_t num_tiles,
+                          cudaStream_t st);
 
 // ---------------------------------------------------------------- blending
 struct BlendArgs {

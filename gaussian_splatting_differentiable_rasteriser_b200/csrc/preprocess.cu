@@ -24,7 +24,7 @@ __device__ __forceinline__ double dot3(const double* a, const double* b) {
 }
 
 template <int kDeg>
-__global__ void __launch_bounds__(256) preprocess_kernel(PreprocessArgs a) {
+__global__ void __launch_bounds__(256, 3) preprocess_kernel(PreprocessArgs a) {
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   uint32_t touched = 0;
   uint32_t dkey = 0;
@@ -157,12 +157,15 @@ __global__ void __launch_bounds__(256) preprocess_kernel(PreprocessArgs a) {
     a.clamped[i] = clamped;
   }
 
-  // Block total of tiles_touched (for the prefix sum) and the depth-key range
-  // of visible Gaussians (to size the sort key).
+  // Block totals of tiles touched and of visible Gaussians (for the entry
+  // count and the compaction's prefix sum) and the depth-key range of visible
+  // Gaussians (to size the depth sort's key).
   __shared__ uint32_t s_sum[8];
+  __shared__ uint32_t s_vis[8];
   uint32_t t = touched;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+  const uint32_t nvis = __popc(__ballot_sync(0xffffffffu, touched != 0u));
   uint32_t kmin = visible ? dkey : 0xffffffffu, kmax = visible ? dkey : 0u;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
@@ -172,6 +175,7 @@ __global__ void __launch_bounds__(256) preprocess_kernel(PreprocessArgs a) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   if (lane == 0) {
     s_sum[warp] = t;
+    s_vis[warp] = nvis;
     if (kmin <= kmax) {
       atomicMin(&a.depth_range[0], kmin);
       atomicMax(&a.depth_range[1], kmax);
@@ -179,51 +183,71 @@ __global__ void __launch_bounds__(256) preprocess_kernel(PreprocessArgs a) {
   }
   __syncthreads();
   if (threadIdx.x == 0) {
-    uint32_t b = 0;
-    for (int k = 0; k < (blockDim.x >> 5); ++k) b += s_sum[k];
-    a.block_sums[blockIdx.x] = b;
+    uint32_t b = 0, v = 0;
+    for (int k = 0; k < (blockDim.x >> 5); ++k) {
+      b += s_sum[k];
+      v += s_vis[k];
+    }
+    a.block_sums[blockIdx.x] = make_uint2(b, v);
   }
 }
 
-// Exclusive prefix of the per-block totals (one CTA of 1024 threads), plus the
-// grand total and the depth-key range copied into the readback record.
-__global__ void __launch_bounds__(1024) scan_blocks_kernel(const uint32_t* block_sums, int64_t nb,
-                                                           uint64_t* block_prefix,
+// Exclusive prefix of the per-block visible counts (one CTA of 1024 threads),
+// plus the entry and visible totals and the depth-key range copied into the
+// readback record.
+__global__ void __launch_bounds__(1024) scan_blocks_kernel(const uint2* block_sums, int64_t nb,
+                                                           uint32_t* visible_prefix,
                                                            const uint32_t* depth_range,
                                                            ForwardInfo* info) {
   __shared__ uint64_t s_warp[32];
+  __shared__ uint32_t s_vwarp[32];
   const int tid = threadIdx.x;
   const int64_t per = (nb + blockDim.x - 1) / blockDim.x;
   const int64_t lo = tid * per, hi = min(nb, lo + per);
-  uint64_t local = 0;
-  for (int64_t k = lo; k < hi; ++k) local += block_sums[k];
-  // inclusive scan of `local` across the CTA
-  uint64_t v = local;
+  uint64_t entries = 0;
+  uint32_t local = 0;
+  for (int64_t k = lo; k < hi; ++k) {
+    const uint2 b = block_sums[k];
+    entries += b.x;
+    local += b.y;
+  }
   const int lane = tid & 31, warp = tid >> 5;
 #pragma unroll
+  for (int o = 16; o > 0; o >>= 1) entries += __shfl_xor_sync(0xffffffffu, entries, o);
+  // inclusive scan of the visible counts across the CTA
+  uint32_t v = local;
+#pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    uint64_t n = __shfl_up_sync(0xffffffffu, v, o);
+    uint32_t n = __shfl_up_sync(0xffffffffu, v, o);
     if (lane >= o) v += n;
   }
-  if (lane == 31) s_warp[warp] = v;
+  if (lane == 31) {
+    s_vwarp[warp] = v;
+    s_warp[warp] = entries;
+  }
   __syncthreads();
   if (warp == 0) {
-    uint64_t w = s_warp[lane];
+    uint32_t w = s_vwarp[lane];
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      uint64_t n = __shfl_up_sync(0xffffffffu, w, o);
+      uint32_t n = __shfl_up_sync(0xffffffffu, w, o);
       if (lane >= o) w += n;
     }
-    s_warp[lane] = w;
+    s_vwarp[lane] = w;
+    uint64_t e = s_warp[lane];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) e += __shfl_xor_sync(0xffffffffu, e, o);
+    if (lane == 0) s_warp[0] = e;
   }
   __syncthreads();
-  uint64_t run = v - local + (warp > 0 ? s_warp[warp - 1] : 0);
+  uint32_t run = v - local + (warp > 0 ? s_vwarp[warp - 1] : 0u);
   for (int64_t k = lo; k < hi; ++k) {
-    block_prefix[k] = run;
-    run += block_sums[k];
+    visible_prefix[k] = run;
+    run += block_sums[k].y;
   }
-  if (tid == blockDim.x - 1) {
-    info->num_entries = s_warp[31];
+  if (tid == 0) {
+    info->num_entries = s_warp[0];
+    info->num_visible = s_vwarp[31];
     info->depth_min = depth_range[0];
     info->depth_max = depth_range[1];
   }
@@ -243,9 +267,9 @@ cudaError_t launch_preprocess(const PreprocessArgs& a, int64_t num_blocks, cudaS
   return cudaGetLastError();
 }
 
-cudaError_t launch_scan_blocks(const uint32_t* block_sums, int64_t num_blocks, uint64_t* block_prefix,
+cudaError_t launch_scan_blocks(const uint2* block_sums, int64_t num_blocks, uint32_t* visible_prefix,
                                const uint32_t* depth_range, ForwardInfo* info, cudaStream_t st) {
-  scan_blocks_kernel<<<1, 1024, 0, st>>>(block_sums, num_blocks, block_prefix, depth_range, info);
+  scan_blocks_kernel<<<1, 1024, 0, st>>>(block_sums, num_blocks, visible_prefix, depth_range, info);
   return cudaGetLastError();
 }
 

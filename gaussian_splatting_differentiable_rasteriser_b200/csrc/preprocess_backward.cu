@@ -249,7 +249,10 @@ struct FusedSmem {
   float Y[16][kFusedBlock];              // SH basis at the view direction
 };
 
-template <int kDeg>
+// kAccum: the caller's gradient buffer holds an accumulated gradient, which is
+// added and then zeroed; without it the update uses this view's gradient alone
+// and no gradient buffer is read or written (24 instead of 32 bytes per scalar).
+template <int kDeg, bool kAccum>
 __global__ void __launch_bounds__(kFusedBlock) preprocess_backward_adam_kernel(PreprocessBwdArgs a,
                                                                               FusedAdamArgs f) {
   __shared__ __align__(16) FusedSmem sm;
@@ -322,9 +325,10 @@ __global__ void __launch_bounds__(kFusedBlock) preprocess_backward_adam_kernel(P
       else if (pl < 11) { grp[r] = 3; c = 0; }
       else { grp[r] = 4; c = pl - kGeomPlanes; }
       off[r] = static_cast<int64_t>(c) * np + i0 + 4 * col[r];
+      G[r] = make_float4(0.f, 0.f, 0.f, 0.f);
       if (ok[r]) {
         P[r] = *reinterpret_cast<const float4*>(f.p[grp[r]] + off[r]);
-        G[r] = *reinterpret_cast<const float4*>(f.g[grp[r]] + off[r]);
+        if (kAccum) G[r] = *reinterpret_cast<const float4*>(f.g[grp[r]] + off[r]);
         M[r] = *reinterpret_cast<const float4*>(f.m[grp[r]] + off[r]);
         V[r] = *reinterpret_cast<const float4*>(f.v[grp[r]] + off[r]);
       }
@@ -351,7 +355,7 @@ __global__ void __launch_bounds__(kFusedBlock) preprocess_backward_adam_kernel(P
         adam_one(p4[e], g4[e], m4[e], v4[e], f.s[grp[r]]);
       }
       *reinterpret_cast<float4*>(f.p[grp[r]] + off[r]) = P[r];
-      *reinterpret_cast<float4*>(f.g[grp[r]] + off[r]) = G[r];
+      if (kAccum) *reinterpret_cast<float4*>(f.g[grp[r]] + off[r]) = G[r];
       *reinterpret_cast<float4*>(f.m[grp[r]] + off[r]) = M[r];
       *reinterpret_cast<float4*>(f.v[grp[r]] + off[r]) = V[r];
     }
@@ -395,11 +399,20 @@ cudaError_t launch_preprocess_backward_adam(const PreprocessBwdArgs& a, const Fu
                                            cudaStream_t st) {
   if (a.n_pad == 0) return cudaSuccess;
   const unsigned grid = static_cast<unsigned>((a.n_pad + kFusedBlock - 1) / kFusedBlock);
-  switch (a.active_degree) {
-    case 0: preprocess_backward_adam_kernel<0><<<grid, kFusedBlock, 0, st>>>(a, f); break;
-    case 1: preprocess_backward_adam_kernel<1><<<grid, kFusedBlock, 0, st>>>(a, f); break;
-    case 2: preprocess_backward_adam_kernel<2><<<grid, kFusedBlock, 0, st>>>(a, f); break;
-    default: preprocess_backward_adam_kernel<3><<<grid, kFusedBlock, 0, st>>>(a, f); break;
+  if (f.g[0]) {
+    switch (a.active_degree) {
+      case 0: preprocess_backward_adam_kernel<0, true><<<grid, kFusedBlock, 0, st>>>(a, f); break;
+      case 1: preprocess_backward_adam_kernel<1, true><<<grid, kFusedBlock, 0, st>>>(a, f); break;
+      case 2: preprocess_backward_adam_kernel<2, true><<<grid, kFusedBlock, 0, st>>>(a, f); break;
+      default: preprocess_backward_adam_kernel<3, true><<<grid, kFusedBlock, 0, st>>>(a, f); break;
+    }
+  } else {
+    switch (a.active_degree) {
+      case 0: preprocess_backward_adam_kernel<0, false><<<grid, kFusedBlock, 0, st>>>(a, f); break;
+      case 1: preprocess_backward_adam_kernel<1, false><<<grid, kFusedBlock, 0, st>>>(a, f); break;
+      case 2: preprocess_backward_adam_kernel<2, false><<<grid, kFusedBlock, 0, st>>>(a, f); break;
+      default: preprocess_backward_adam_kernel<3, false><<<grid, kFusedBlock, 0, st>>>(a, f); break;
+    }
   }
   return cudaGetLastError();
 }

@@ -1,27 +1,32 @@
-// Tile lists: duplicate one (tile | depth) key per touched tile, sort the keys
-// with a stable LSD onesweep radix sort, extract per-tile ranges.
+// Tile lists: order the (Gaussian, tile) entries by tile, then depth, then
+// index, and extract per-tile ranges.
 //
 // Method: "How a computer rebuilds a real place ... Gaussian Splats"
 // (taosengine.com), section "Why tiling, and the five stages": count -> scan
 // -> scatter -> sort by depth within each tile, equal keys broken by the
 // smaller id; each tile's range closes where the next tile begins.
 //
-// Design (B200): instead of a per-tile bitonic network, all entries are sorted
-// at once by a single 64-bit key
-//     key = tile << depth_bits | (float_bits(depth) - depth_min)
-// where depth_bits is the bit length of the visible depth-key range. Positive
-// float32 bit patterns order like the floats, and subtracting the minimum
-// keeps that order, so the key orders entries by (tile, depth) exactly while
-// needing only ceil((tile_bits + depth_bits) / 8) passes (typically 5 at
-// 1080p, not 8). Entries are emitted in Gaussian-index order and every pass
-// is stable, so equal keys stay in index order: the tie-break needs no bits.
+// Design (B200): the order (tile, depth, index) is produced by two stable
+// radix sorts of 32-bit keys instead of one sort of 64-bit (tile | depth)
+// keys over all entries:
+//   1. compact the visible Gaussians in index order as
+//      (float_bits(depth) - depth_min, index); positive float32 bit patterns
+//      order like the floats, so this key orders by depth exactly;
+//   2. sort them by that key (ceil(depth_bits / 8) passes, typically 3, over
+//      the visible Gaussians only - about 2.2x fewer items than entries);
+//   3. duplicate in that depth order: one (tile, index) entry per touched
+//      tile, each CTA's output offset found by a decoupled look-back;
+//   4. sort the entries by tile (ceil(tile_bits / 8) passes, 2 at 1080p).
+// Every step is stable, so equal depth keys stay in index order and each
+// tile's entries stay in (depth, index) order: the same order as one sort by
+// (tile, depth) of entries emitted in index order, with about half the bytes
+// moved (16 B per item and pass instead of 24, 5 passes over fewer items).
 //
-// Each onesweep pass reads and writes every entry once (12 B in, 12 B out):
-// a CTA ranks 4096 keys in shared memory (warp match + per-warp digit
-// counters), publishes its digit counts, obtains the exclusive prefix of all
-// earlier CTAs by a decoupled look-back whose every wait is bounded, and
-// scatters through shared memory so the global writes are runs of consecutive
-// addresses.
+// Each onesweep pass reads and writes every item once: a CTA ranks 4096 keys
+// in shared memory (per-warp digit counters, ballot ranking), publishes its
+// digit counts, obtains the exclusive prefix of all earlier CTAs by a
+// decoupled look-back whose every wait is bounded, and scatters through shared
+// memory so the global writes are runs of consecutive addresses.
 #include <algorithm>
 
 #include "gs_kernels.cuh"
@@ -44,50 +49,135 @@ __device__ __forceinline__ void st_relaxed(uint32_t* p, uint32_t v) {
   asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-// ------------------------------------------------------------- duplicate --
-__global__ void __launch_bounds__(256) duplicate_kernel(DuplicateArgs a) {
+// ---------------------------------------------------------------- compact --
+__global__ void __launch_bounds__(256) compact_kernel(CompactArgs a) {
   __shared__ uint32_t s_warp[8];
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const uint32_t t = i < a.n ? a.touched[i] : 0u;
-  // exclusive scan of t inside the CTA
+  const bool vis = i < a.n && a.touched[i] != 0u;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  uint32_t v = t;
+  const uint32_t m = __ballot_sync(0xffffffffu, vis);
+  if (lane == 0) s_warp[warp] = __popc(m);
+  __syncthreads();
+  if (!vis) return;
+  uint32_t before = 0;
+  for (int k = 0; k < warp; ++k) before += s_warp[k];
+  const int64_t off = static_cast<int64_t>(a.visible_prefix[blockIdx.x]) + before +
+                      __popc(m & ((1u << lane) - 1u));
+  if (off >= a.max_out) {
+    record_error(a.err, kErrIndexRange);
+    return;
+  }
+  a.keys[off] = __float_as_uint(a.depth[i]) - a.depth_min;
+  a.vals[off] = static_cast<uint32_t>(i);
+}
+
+// -------------------------------------------------------------- duplicate --
+// Decoupled look-back over earlier CTAs' status words (flag | value) by one
+// warp, 32 predecessors per round; returns the sum of the values before
+// `tile`. Every wait is bounded; on giving up it records an error and returns
+// what it has.
+__device__ __forceinline__ uint32_t warp_lookback(const uint32_t* status, int64_t tile, int lane,
+                                                  uint32_t* err) {
+  uint32_t excl = 0;
+  int64_t t = tile - 1;
+  int spins = 0;
+  while (t >= 0) {
+    const uint32_t w = (t - lane >= 0) ? ld_relaxed(&status[t - lane]) : kFlagPrefix;
+    const uint32_t flag = w & ~kValueMask;
+    const unsigned not_ready = __ballot_sync(0xffffffffu, flag == 0u);
+    const unsigned is_prefix = __ballot_sync(0xffffffffu, flag == kFlagPrefix);
+    // lanes usable this round: up to (and including) the first prefix, before the first not-ready
+    const unsigned upto_prefix = is_prefix ? ((2u << (__ffs(is_prefix) - 1)) - 1u) : 0xffffffffu;
+    const unsigned before_wait = not_ready ? ((1u << (__ffs(not_ready) - 1)) - 1u) : 0xffffffffu;
+    const unsigned use = upto_prefix & before_wait;
+    uint32_t v = ((use >> lane) & 1u) ? (w & kValueMask) : 0u;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    excl += v;
+    if (is_prefix && (upto_prefix & ~before_wait) == 0u) break;  // reached a prefix
+    t -= __popc(use);
+    if (not_ready) {
+      if (++spins > kLookbackSpinLimit) {
+        record_error(err, kErrLookbackTimeout);
+        break;
+      }
+      __nanosleep(32);
+    }
+  }
+  return excl;
+}
+
+__global__ void __launch_bounds__(kDupThreads) duplicate_kernel(DuplicateArgs a) {
+  __shared__ uint32_t s_warp[kDupThreads / 32];
+  __shared__ uint32_t s_tile, s_excl;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) s_tile = atomicAdd(a.ticket, 1u);
+  __syncthreads();
+  const int64_t tile = s_tile;
+  const int64_t first = tile * kDupItems + static_cast<int64_t>(tid) * kDupPerThread;
+  uint32_t gid[kDupPerThread], cnt[kDupPerThread];
+  uint32_t mine = 0;
+#pragma unroll
+  for (int k = 0; k < kDupPerThread; ++k) {
+    const int64_t j = first + k;
+    gid[k] = j < a.count ? __ldg(a.order + j) : 0u;
+    cnt[k] = j < a.count ? __ldg(a.touched + gid[k]) : 0u;
+    mine += cnt[k];
+  }
+  // CTA-exclusive prefix of the per-thread totals
+  uint32_t v = mine;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    uint32_t n = __shfl_up_sync(0xffffffffu, v, o);
+    const uint32_t n = __shfl_up_sync(0xffffffffu, v, o);
     if (lane >= o) v += n;
   }
   if (lane == 31) s_warp[warp] = v;
   __syncthreads();
-  uint32_t before = 0;
-  for (int k = 0; k < warp; ++k) before += s_warp[k];
-  if (t == 0) return;
-  uint64_t off = a.block_prefix[blockIdx.x] + before + (v - t);
-  if (off + t > static_cast<uint64_t>(a.max_entries)) {
-    record_error(a.err, kErrIndexRange);
+  uint32_t before = 0, total = 0;
+#pragma unroll
+  for (int k = 0; k < kDupThreads / 32; ++k) {
+    before += k < warp ? s_warp[k] : 0u;
+    total += s_warp[k];
+  }
+  uint32_t* st = a.status + tile;
+  if (warp == 0) {
+    if (lane == 0) st_relaxed(st, (tile == 0 ? kFlagPrefix : kFlagAggregate) | total);
+    uint32_t excl = 0;
+    if (tile > 0) {
+      excl = warp_lookback(a.status, tile, lane, a.err);
+      if (lane == 0) st_relaxed(st, kFlagPrefix | (excl + total));
+    }
+    if (lane == 0) s_excl = excl;
+  }
+  __syncthreads();
+  uint64_t off = static_cast<uint64_t>(s_excl) + before + (v - mine);
+  if (off + mine > static_cast<uint64_t>(a.max_entries)) {
+    if (mine) record_error(a.err, kErrIndexRange);
     return;
   }
-  const uint2 rc = a.rect[i];
-  const uint32_t x0 = rc.x & 0xffffu, x1 = rc.x >> 16, y0 = rc.y & 0xffffu, y1 = rc.y >> 16;
-  const uint64_t dk = static_cast<uint64_t>(__float_as_uint(a.depth[i]) - a.depth_min);
-  for (uint32_t y = y0; y <= y1; ++y)
-    for (uint32_t x = x0; x <= x1; ++x) {
-      const uint64_t tile = static_cast<uint64_t>(y) * a.tiles_x + x;
-      a.keys[off] = (tile << a.depth_bits) | dk;
-      a.vals[off] = static_cast<uint32_t>(i);
-      ++off;
-    }
+#pragma unroll
+  for (int k = 0; k < kDupPerThread; ++k) {
+    if (cnt[k] == 0u) continue;
+    const uint2 rc = __ldg(a.rect + gid[k]);
+    const uint32_t x0 = rc.x & 0xffffu, x1 = rc.x >> 16, y0 = rc.y & 0xffffu, y1 = rc.y >> 16;
+    for (uint32_t y = y0; y <= y1; ++y)
+      for (uint32_t x = x0; x <= x1; ++x) {
+        a.keys[off] = y * static_cast<uint32_t>(a.tiles_x) + x;
+        a.vals[off] = gid[k];
+        ++off;
+      }
+  }
 }
 
 // ------------------------------------------------------------- histogram --
-__global__ void __launch_bounds__(256) histogram_kernel(const uint64_t* keys, int64_t n,
+__global__ void __launch_bounds__(256) histogram_kernel(const uint32_t* keys, int64_t n,
                                                         int passes, uint32_t* hist) {
   __shared__ uint32_t s_hist[kMaxPasses][kRadix];
   for (int k = threadIdx.x; k < kMaxPasses * kRadix; k += blockDim.x) (&s_hist[0][0])[k] = 0;
   __syncthreads();
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += stride) {
-    const uint64_t key = keys[i];
+    const uint32_t key = keys[i];
     for (int p = 0; p < passes; ++p) atomicAdd(&s_hist[p][(key >> (8 * p)) & 0xffu], 1u);
   }
   __syncthreads();
@@ -117,9 +207,9 @@ __global__ void __launch_bounds__(256) digit_offsets_kernel(const uint32_t* hist
 
 // --------------------------------------------------------------- onesweep --
 struct OnesweepArgs {
-  const uint64_t* keys_in;
+  const uint32_t* keys_in;
   const uint32_t* vals_in;
-  uint64_t* keys_out;
+  uint32_t* keys_out;
   uint32_t* vals_out;
   int64_t n;
   int shift;
@@ -132,7 +222,7 @@ struct OnesweepArgs {
 
 // Shared memory of one onesweep CTA (dynamic: above the 48 KB static limit).
 struct OnesweepSmem {
-  uint64_t keys[kSortTileKeys];
+  uint32_t keys[kSortTileKeys];
   uint32_t vals[kSortTileKeys];
   uint32_t whist[kSortThreads / 32][kRadix];  // per-warp digit counts, then offsets
   uint32_t start[kRadix];  // first slot of each digit inside this CTA
@@ -144,7 +234,7 @@ struct OnesweepSmem {
 __global__ void __launch_bounds__(kSortThreads) onesweep_kernel(OnesweepArgs a) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   OnesweepSmem& sm = *reinterpret_cast<OnesweepSmem*>(smem_raw);
-  uint64_t* s_keys = sm.keys;
+  uint32_t* s_keys = sm.keys;
   uint32_t* s_vals = sm.vals;
   auto& s_whist = sm.whist;
   uint32_t* s_start = sm.start;
@@ -162,7 +252,7 @@ __global__ void __launch_bounds__(kSortThreads) onesweep_kernel(OnesweepArgs a) 
 
   // Load: warp w owns the 512 consecutive entries [base + 512 w, base + 512 (w + 1)),
   // item j of lane l is entry 32 j + l of that run (coalesced).
-  uint64_t key[kSortItems];
+  uint32_t key[kSortItems];
   uint32_t val[kSortItems];
   uint32_t rank[kSortItems];
 #pragma unroll
@@ -172,7 +262,7 @@ __global__ void __launch_bounds__(kSortThreads) onesweep_kernel(OnesweepArgs a) 
       key[j] = a.keys_in[idx];
       val[j] = a.vals_in[idx];
     } else {
-      key[j] = ~0ull;
+      key[j] = ~0u;
       val[j] = 0u;
     }
   }
@@ -182,7 +272,7 @@ __global__ void __launch_bounds__(kSortThreads) onesweep_kernel(OnesweepArgs a) 
   for (int j = 0; j < kSortItems; ++j) {
     const int64_t idx = base + warp * (kSortItems * 32) + j * 32 + lane;
     const bool valid = idx < a.n;
-    const uint32_t d = static_cast<uint32_t>(key[j] >> a.shift) & 0xffu;
+    const uint32_t d = (key[j] >> a.shift) & 0xffu;
     uint32_t peers = __ballot_sync(0xffffffffu, valid);
 #pragma unroll
     for (int bit = 0; bit < 8; ++bit) {
@@ -274,7 +364,7 @@ __global__ void __launch_bounds__(kSortThreads) onesweep_kernel(OnesweepArgs a) 
   for (int j = 0; j < kSortItems; ++j) {
     const int64_t idx = base + warp * (kSortItems * 32) + j * 32 + lane;
     if (idx < a.n) {
-      const uint32_t dj = static_cast<uint32_t>(key[j] >> a.shift) & 0xffu;
+      const uint32_t dj = (key[j] >> a.shift) & 0xffu;
       const uint32_t pos = s_start[dj] + s_whist[warp][dj] + rank[j];
       if (pos >= static_cast<uint32_t>(kSortTileKeys)) {
         record_error(a.err, kErrIndexRange);
@@ -288,8 +378,8 @@ __global__ void __launch_bounds__(kSortThreads) onesweep_kernel(OnesweepArgs a) 
   const int64_t rem = a.n - base;
   const int tile_n = rem < kSortTileKeys ? static_cast<int>(rem) : kSortTileKeys;
   for (int k = tid; k < tile_n; k += kSortThreads) {
-    const uint64_t kk = s_keys[k];
-    const uint32_t dk = static_cast<uint32_t>(kk >> a.shift) & 0xffu;
+    const uint32_t kk = s_keys[k];
+    const uint32_t dk = (kk >> a.shift) & 0xffu;
     const int64_t dst = static_cast<int64_t>(s_base[dk]) + (k - static_cast<int64_t>(s_start[dk]));
     if (dst < 0 || dst >= a.n) {
       record_error(a.err, kErrIndexRange);
@@ -301,21 +391,31 @@ __global__ void __launch_bounds__(kSortThreads) onesweep_kernel(OnesweepArgs a) 
 }
 
 // ------------------------------------------------------------------ ranges --
-__global__ void __launch_bounds__(256) ranges_kernel(const uint64_t* keys, int64_t n, int depth_bits,
-                                                     uint2* ranges, int64_t num_tiles) {
+__global__ void __launch_bounds__(256) ranges_kernel(const uint32_t* keys, int64_t n, uint2* ranges,
+                                                     int64_t num_tiles) {
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i >= n) return;
-  const uint64_t tile = keys[i] >> depth_bits;
+  const uint32_t tile = keys[i];
   if (tile >= static_cast<uint64_t>(num_tiles)) return;
-  if (i == 0 || (keys[i - 1] >> depth_bits) != tile) ranges[tile].x = static_cast<uint32_t>(i);
-  if (i == n - 1 || (keys[i + 1] >> depth_bits) != tile) ranges[tile].y = static_cast<uint32_t>(i + 1);
+  if (i == 0 || keys[i - 1] != tile) ranges[tile].x = static_cast<uint32_t>(i);
+  if (i == n - 1 || keys[i + 1] != tile) ranges[tile].y = static_cast<uint32_t>(i + 1);
 }
 
 }  // namespace
 
-cudaError_t launch_duplicate(const DuplicateArgs& a, int64_t num_blocks, cudaStream_t st) {
+cudaError_t launch_compact(const CompactArgs& a, int64_t num_blocks, cudaStream_t st) {
   if (num_blocks == 0) return cudaSuccess;
-  duplicate_kernel<<<static_cast<unsigned>(num_blocks), 256, 0, st>>>(a);
+  compact_kernel<<<static_cast<unsigned>(num_blocks), 256, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_duplicate(const DuplicateArgs& a, cudaStream_t st) {
+  if (a.count == 0) return cudaSuccess;
+  const int64_t tiles = (a.count + kDupItems - 1) / kDupItems;
+  cudaError_t e;
+  if ((e = cudaMemsetAsync(a.status, 0, sizeof(uint32_t) * tiles, st)) != cudaSuccess) return e;
+  if ((e = cudaMemsetAsync(a.ticket, 0, sizeof(uint32_t), st)) != cudaSuccess) return e;
+  duplicate_kernel<<<static_cast<unsigned>(tiles), kDupThreads, 0, st>>>(a);
   return cudaGetLastError();
 }
 
@@ -357,12 +457,11 @@ cudaError_t launch_sort(const SortPlan& plan, const SortBuffers& b, int* out_buf
   return cudaSuccess;
 }
 
-cudaError_t launch_ranges(const uint64_t* keys, int64_t n, int depth_bits, uint2* ranges,
-                          int64_t num_tiles, cudaStream_t st) {
+cudaError_t launch_ranges(const uint32_t* keys, int64_t n, uint2* ranges, int64_t num_tiles,
+                          cudaStream_t st) {
   cudaError_t e = cudaMemsetAsync(ranges, 0, sizeof(uint2) * num_tiles, st);
   if (e != cudaSuccess || n == 0) return e;
-  ranges_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(keys, n, depth_bits, ranges,
-                                                                        num_tiles);
+  ranges_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(keys, n, ranges, num_tiles);
   return cudaGetLastError();
 }
 

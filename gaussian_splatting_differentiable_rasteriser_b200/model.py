@@ -118,8 +118,9 @@ class TrainStep:
         m = self.model
         m.step_count += 1
         if self.fused_adam:
+            # one view per step: no accumulated gradient, so no gradient buffer traffic
             em, ev = m.moments_structs()
-            self.ctx.render_backward_adam(m.params_struct(), cs, T, nc, dimg, m.grads_struct(), em, ev,
+            self.ctx.render_backward_adam(m.params_struct(), cs, T, nc, dimg, None, em, ev,
                                           [self.lrs[k] for k in GROUP_NAMES], m.step_count,
                                           self.betas[0], self.betas[1], self.eps)
             return

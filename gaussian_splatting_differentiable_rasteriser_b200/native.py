@@ -26,7 +26,7 @@ EXPORTED = ("gs_create", "gs_destroy", "gs_last_error", "gs_preprocess", "gs_ren
             "gs_profile_read", "gs_stage_name", "gs_debug_preprocess", "gs_debug_sorted",
             "gs_debug_screen_grads")
 STAGES = ("preprocess", "scan", "duplicate", "sort", "ranges", "blend_forward", "loss",
-          "blend_backward", "preprocess_backward", "backward_adam")
+          "blend_backward", "preprocess_backward", "backward_adam", "depth_sort")
 GROUPS = ("means", "log_scales", "quats", "opacity_logits", "sh")
 
 
@@ -172,12 +172,15 @@ class Context:
                                               ctypes.byref(grads), _stream(stream)))
 
     def render_backward_adam(self, params: GsParams, cam: GsCamera, final_T, n_contrib, dloss_dimage,
-                             grads: GsGrads, exp_avg: GsGrads, exp_avg_sq: GsGrads, lrs, step,
+                             grads, exp_avg: GsGrads, exp_avg_sq: GsGrads, lrs, step,
                              beta1=0.9, beta2=0.999, eps=1e-8, stream=None):
+        """grads: a GsGrads with an accumulated gradient (zeroed by the call), or
+        None when there is none (no gradient buffer is read or written)."""
         lr = (ctypes.c_float * 5)(*[float(x) for x in lrs])
+        g = None if grads is None else ctypes.byref(grads)
         self._check(self.L.gs_render_backward_adam(
             self.h, ctypes.byref(params), ctypes.byref(cam), _ptr(final_T), _ptr(n_contrib),
-            _ptr(dloss_dimage), ctypes.byref(grads), ctypes.byref(exp_avg), ctypes.byref(exp_avg_sq),
+            _ptr(dloss_dimage), g, ctypes.byref(exp_avg), ctypes.byref(exp_avg_sq),
             lr, float(beta1), float(beta2), float(eps), int(step), _stream(stream)))
 
     def profile_enable(self, on=True):

@@ -118,10 +118,11 @@ gs_status gs_preprocess(gs_ctx *ctx, const gs_params *params, const gs_camera *c
  * five stages" and "The painting itself: front-to-back alpha compositing";
  * [DR] section "The trick: recompute the blend state instead of storing it";
  * [SN] slide on alpha and the background term).
- * Duplicates one 64-bit key (tile | depth) with the Gaussian index as value
- * per touched tile (prefix sum over tiles_touched), sorts them with a stable
- * LSD onesweep radix sort (order = tile, depth, index), extracts per-tile
- * ranges, then blends each 16x16 tile front to back:
+ * Orders the (Gaussian, tile) entries by (tile, depth, index): the visible
+ * Gaussians are sorted by depth with a stable LSD onesweep radix sort, one
+ * entry per touched tile is emitted in that order (prefix sum over
+ * tiles_touched), and the entries are sorted stably by tile; then per-tile
+ * ranges are extracted and each 16x16 tile is blended front to back:
  * alpha = min(0.99, o exp(-e)), e = 1/2 (A dx^2 + C dy^2) + B dx dy, entries
  * with alpha < 1/255 skipped, C += T alpha c, T *= 1 - alpha, and the walk
  * stops after the entry that takes T below 1e-4. Writes
@@ -197,8 +198,13 @@ gs_status gs_loss_l1_dssim_noalloc(const float *image_chw, const float *target_c
  * every group updated by Adam with its own learning rate). lr is a HOST array
  * of 5 learning rates in the order means, log_scales, quats, opacity_logits,
  * sh; exp_avg and exp_avg_sq hold the first and second moments in the
- * parameter layout. Errors as gs_render_backward, plus GS_ERR_INVALID_ARG for
- * a NULL moment pointer, step < 1 or betas outside [0, 1). */
+ * parameter layout. grads may be NULL when there is no accumulated gradient
+ * (one view per step, as in the method's training loop): the update then uses
+ * this view's gradient alone and no gradient buffer is read or written, which
+ * saves 8 of the 32 bytes each scalar moves; the result equals the call with
+ * an all-zero grads buffer. Errors as gs_render_backward, plus
+ * GS_ERR_INVALID_ARG for a NULL moment pointer, step < 1 or betas outside
+ * [0, 1). */
 gs_status gs_render_backward_adam(gs_ctx *ctx, const gs_params *params, const gs_camera *cam,
                                   const float *final_T, const int32_t *n_contrib,
                                   const float *dloss_dimage, gs_grads *grads, gs_grads *exp_avg,
@@ -220,10 +226,11 @@ gs_status gs_adam_step(float *param, float *grad, float *m, float *v, int64_t co
  * leave it off for throughput runs). gs_profile_read waits for the recorded
  * events, returns per-stage totals accumulated since the previous read and
  * resets them. Each output is a HOST array of GS_NUM_STAGES entries (any may
- * be NULL): ms = summed kernel time, launches = launches, work = the units
+ * be NULL): ms = summed kernel time, launches = kernel launches, work = the units
  * processed (Gaussians for the per-Gaussian stages - n_pad for the fused
- * backward + Adam pass -, entries x passes for the sort, entries for the
- * duplication and ranges, pixels for the loss; for the two blends the
+ * backward + Adam pass -, visible Gaussians x passes for the depth sort,
+ * entries x passes for the tile sort, entries for the duplication and
+ * ranges, pixels for the loss; for the two blends the
  * (pixel, Gaussian) pairs the method's walk visits: every list entry up to
  * the pixel's stopping point in the forward, every entry before its last
  * contributor in the backward), blended = for the two blends the pairs that
@@ -240,7 +247,8 @@ typedef enum {
   GS_STAGE_BLEND_BACKWARD = 7,
   GS_STAGE_PREPROCESS_BACKWARD = 8,
   GS_STAGE_BACKWARD_ADAM = 9, /* the fused projection backward + Adam pass */
-  GS_NUM_STAGES = 10
+  GS_STAGE_DEPTH_SORT = 10,   /* compaction + depth sort of the visible Gaussians */
+  GS_NUM_STAGES = 11
 } gs_stage;
 
 gs_status gs_profile_enable(gs_ctx *ctx, int32_t enabled);

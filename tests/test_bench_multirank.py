@@ -1,0 +1,65 @@
+"""The benchmark's multi-rank host logic on CPU with the gloo backend, world
+size 2: process-group set-up from the launcher's environment, the barrier,
+the max-over-ranks timing and the whole-job aggregate of independent replicas,
+and the reference arm under the launcher (rank 0 prints the one line, the
+other rank exits without work)."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out_dir):
+    os.environ.update(RANK=str(rank), LOCAL_RANK=str(rank), WORLD_SIZE=str(world),
+                      MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    import bench
+    import torch.distributed as dist
+    w, r, _ = bench.dist_setup()
+    assert (w, r) == (world, rank) and dist.get_backend() == "gloo"
+    bench.barrier(w)
+    # each replica's own device time; the job is as slow as its slowest rank
+    local_ms = 100.0 + 50.0 * rank
+    ms = bench.max_over_ranks(local_ms, w)
+    value = bench.replica_throughput(w, 10, ms / 1e3)
+    with open(os.path.join(out_dir, f"rank{rank}.json"), "w") as f:
+        json.dump({"ms": ms, "value": value}, f)
+    bench.barrier(w)
+    dist.destroy_process_group()
+
+
+def test_replicas_take_the_slowest_rank(tmp_path):
+    import torch.multiprocessing as mp
+    port = free_port()
+    mp.start_processes(_rank_main, args=(2, port, str(tmp_path)), nprocs=2, join=True,
+                       start_method="spawn")
+    outs = [json.load(open(tmp_path / f"rank{r}.json")) for r in range(2)]
+    for o in outs:
+        assert o["ms"] == 150.0
+        assert o["value"] == pytest.approx(2 * 10 / 0.150)
+
+
+def test_reference_arm_under_the_launcher_prints_once():
+    port = free_port()
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), "bench.py", "--impl",
+           "reference", "--config", "small", "--gpus", "2", "--steps", "3", "--warmup", "3"]
+    r = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    line = json.loads(lines[0])
+    assert line["impl"] == "reference" and line["n_gpus"] == 2
+    assert line["value"] > 0 and line["e2e"]["value"] == line["value"]
+    assert line["cpu_baseline"]["kind"] == "oracle"

@@ -140,7 +140,8 @@ def check_pixels(run, o_render):
     assert amb.mean() < 0.01, f"{amb.sum()} ambiguous pixels"
     err = np.abs(img - o_render["image"])[:, ok]
     assert err.max() <= PIX_TOL, err.max()
-    np.testing.assert_allclose(T[ok], o_render["final_T"][ok], rtol=1e-4, atol=1e-6)
+    # T enters the pixel as T * background: compared at the pixel tolerance
+    np.testing.assert_allclose(T[ok], o_render["final_T"][ok], rtol=0, atol=PIX_TOL)
     np.testing.assert_array_equal(nc[ok], o_render["n_contrib"][ok])
     return amb.sum()
 
@@ -357,5 +358,43 @@ def test_fused_backward_adam_equals_separate_calls(gs):
     for k in scenes.GROUP_NAMES:
         np.testing.assert_allclose(host(a.m[k]), host(b.m[k]), rtol=1e-3, atol=1e-9)
         np.testing.assert_allclose(host(a.v[k]), host(b.v[k]), rtol=2e-3, atol=1e-13)
+        dp = np.abs(host(a.params[k]) - host(b.params[k]))
+        assert np.mean(dp <= 1e-6) > 0.999, k
+
+
+def test_fused_backward_adam_adds_an_accumulated_gradient(gs):
+    """With a gradient buffer, the fused pass adds the accumulated gradient to
+    this view's before the update (and zeroes it): a render_backward of a first
+    loss gradient followed by the fused pass of a second equals two
+    render_backward calls followed by gs_adam_step on every group, up to the
+    float32 atomics' summation order."""
+    native, model = gs
+    s = scenes.small()
+    cam = s.cameras[0]
+    cs = native.camera_struct(cam)
+    H, W = cam.height, cam.width
+    rng = np.random.default_rng(17)
+    d1 = dev(rng.normal(0, 1e-5, (3, H, W)))
+    d2 = dev(rng.normal(0, 1e-5, (3, H, W)))
+    runs = []
+    for fused in (False, True):
+        m = model.GaussianModel(s)
+        st = model.TrainStep(m, 200_000, W, H, fused_adam=fused)
+        _, T, nc = st.forward(cs, H, W)
+        st.ctx.render_backward(m.params_struct(), cs, T, nc, d1, m.grads_struct())
+        if fused:
+            em, ev = m.moments_structs()
+            st.ctx.render_backward_adam(m.params_struct(), cs, T, nc, d2, m.grads_struct(), em, ev,
+                                        [1e-3] * 5, 1)
+        else:
+            st.ctx.render_backward(m.params_struct(), cs, T, nc, d2, m.grads_struct())
+            for k in scenes.GROUP_NAMES:
+                native.adam_step(m.params[k], m.grads[k], m.m[k], m.v[k], 1e-3, 1)
+        torch.cuda.synchronize()
+        assert not m.grad_flat.any().item()
+        runs.append(m)
+    a, b = runs
+    for k in scenes.GROUP_NAMES:
+        assert rel_l2(host(b.m[k]), host(a.m[k])) < 1e-4, k
         dp = np.abs(host(a.params[k]) - host(b.params[k]))
         assert np.mean(dp <= 1e-6) > 0.999, k
