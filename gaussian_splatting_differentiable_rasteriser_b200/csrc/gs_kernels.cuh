@@ -84,7 +84,7 @@ struct DuplicateArgs {
   uint32_t* err;
 };
 constexpr int kDupThreads = 256;
-constexpr int kDupPerThread = 4;
+constexpr int kDupPerThread = 16;
 constexpr int kDupItems = kDupThreads * kDupPerThread;
 cudaError_t launch_duplicate(const DuplicateArgs& a, cudaStream_t st);
 

@@ -107,6 +107,9 @@ __device__ __forceinline__ uint32_t warp_lookback(const uint32_t* status, int64_
   return excl;
 }
 
+// Items are warp-striped: item j of lane l of warp w is the CTA's item
+// 32 (kDupPerThread w + j) + l, so the order reads are coalesced and, for a
+// given j, the lanes' output runs are adjacent in memory.
 __global__ void __launch_bounds__(kDupThreads) duplicate_kernel(DuplicateArgs a) {
   __shared__ uint32_t s_warp[kDupThreads / 32];
   __shared__ uint32_t s_tile, s_excl;
@@ -114,24 +117,38 @@ __global__ void __launch_bounds__(kDupThreads) duplicate_kernel(DuplicateArgs a)
   if (tid == 0) s_tile = atomicAdd(a.ticket, 1u);
   __syncthreads();
   const int64_t tile = s_tile;
-  const int64_t first = tile * kDupItems + static_cast<int64_t>(tid) * kDupPerThread;
-  uint32_t gid[kDupPerThread], cnt[kDupPerThread];
-  uint32_t mine = 0;
+  const int64_t wbase = tile * kDupItems + static_cast<int64_t>(warp) * (32 * kDupPerThread);
+  uint32_t gid[kDupPerThread];
+  uint2 rc[kDupPerThread];
 #pragma unroll
-  for (int k = 0; k < kDupPerThread; ++k) {
-    const int64_t j = first + k;
-    gid[k] = j < a.count ? __ldg(a.order + j) : 0u;
-    cnt[k] = j < a.count ? __ldg(a.touched + gid[k]) : 0u;
-    mine += cnt[k];
+  for (int j = 0; j < kDupPerThread; ++j) {
+    const int64_t idx = wbase + 32 * j + lane;
+    gid[j] = idx < a.count ? __ldg(a.order + idx) : 0u;
   }
-  // CTA-exclusive prefix of the per-thread totals
-  uint32_t v = mine;
 #pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t n = __shfl_up_sync(0xffffffffu, v, o);
-    if (lane >= o) v += n;
+  for (int j = 0; j < kDupPerThread; ++j) {
+    const int64_t idx = wbase + 32 * j + lane;
+    // x0 | x1 << 16, y0 | y1 << 16; an empty rect (x1 < x0) for padding items
+    rc[j] = idx < a.count ? __ldg(a.rect + gid[j]) : make_uint2(1u, 1u);
   }
-  if (lane == 31) s_warp[warp] = v;
+  // exclusive prefix of the tiles touched in (j, lane) order inside the warp
+  uint32_t pre[kDupPerThread];
+  uint32_t run = 0;
+#pragma unroll
+  for (int j = 0; j < kDupPerThread; ++j) {
+    const uint32_t w = (rc[j].x >> 16) + 1u - (rc[j].x & 0xffffu);
+    const uint32_t h = (rc[j].y >> 16) + 1u - (rc[j].y & 0xffffu);
+    const uint32_t c = w * h;
+    uint32_t v = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t n = __shfl_up_sync(0xffffffffu, v, o);
+      if (lane >= o) v += n;
+    }
+    pre[j] = run + v - c;
+    run += __shfl_sync(0xffffffffu, v, 31);
+  }
+  if (lane == 0) s_warp[warp] = run;
   __syncthreads();
   uint32_t before = 0, total = 0;
 #pragma unroll
@@ -150,20 +167,19 @@ __global__ void __launch_bounds__(kDupThreads) duplicate_kernel(DuplicateArgs a)
     if (lane == 0) s_excl = excl;
   }
   __syncthreads();
-  uint64_t off = static_cast<uint64_t>(s_excl) + before + (v - mine);
-  if (off + mine > static_cast<uint64_t>(a.max_entries)) {
-    if (mine) record_error(a.err, kErrIndexRange);
+  const uint64_t off0 = static_cast<uint64_t>(s_excl) + before;
+  if (off0 + run > static_cast<uint64_t>(a.max_entries)) {
+    if (lane == 0 && run) record_error(a.err, kErrIndexRange);
     return;
   }
 #pragma unroll
-  for (int k = 0; k < kDupPerThread; ++k) {
-    if (cnt[k] == 0u) continue;
-    const uint2 rc = __ldg(a.rect + gid[k]);
-    const uint32_t x0 = rc.x & 0xffffu, x1 = rc.x >> 16, y0 = rc.y & 0xffffu, y1 = rc.y >> 16;
+  for (int j = 0; j < kDupPerThread; ++j) {
+    const uint32_t x0 = rc[j].x & 0xffffu, x1 = rc[j].x >> 16, y0 = rc[j].y & 0xffffu, y1 = rc[j].y >> 16;
+    uint64_t off = off0 + pre[j];
     for (uint32_t y = y0; y <= y1; ++y)
       for (uint32_t x = x0; x <= x1; ++x) {
         a.keys[off] = y * static_cast<uint32_t>(a.tiles_x) + x;
-        a.vals[off] = gid[k];
+        a.vals[off] = gid[j];
         ++off;
       }
   }
