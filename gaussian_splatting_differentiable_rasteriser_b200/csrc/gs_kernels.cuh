@@ -139,6 +139,15 @@ struct LossArgs {
   double* out;           // {loss, l1, ssim}
 };
 
+// The loss runs one CTA per channel and strip of kLossCols columns x
+// kLossStrip rows.
+constexpr int kLossCols = 32;
+constexpr int kLossStrip = 128;
+constexpr int64_t loss_blocks(int height, int width) {
+  return 3 * static_cast<int64_t>((width + kLossCols - 1) / kLossCols) *
+         ((height + kLossStrip - 1) / kLossStrip);
+}
+
 cudaError_t launch_loss(const LossArgs& a, cudaStream_t st);
 
 // ------------------------------------------------------- projection backward

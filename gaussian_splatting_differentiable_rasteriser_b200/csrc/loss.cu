@@ -8,44 +8,51 @@
 // The SSIM gradient couples neighbours through the window moments:
 //   dSSIM/dx_p = 1/(3HW) sum_q w(q - p) [dS_q/dmu_x + 2 x_p dS_q/dE[x^2] + y_p dS_q/dE[xy]].
 //
-// B200 design: one CTA per 32x32 output tile and channel does everything in
-// shared memory with halo recompute - no intermediate maps in HBM, so the
-// kernel reads the two images once and writes the gradient once (36 B per
-// pixel over the three channels). Every filter pass is register-tiled: a
-// thread produces 4 (or 4 x 2) consecutive outputs from a window it loads once
-// with vector loads, so shared memory serves several times fewer loads than
-// one per tap; the squared and cross products are formed once per window
-// element. The adjoint buffer reuses the horizontal-moment buffer once that is
-// dead (about 90 KB per CTA). Steps: load the 52x52 input region (zero outside
-// the image), separable 11-tap horizontal then vertical filtering of the 5
-// moments over the 42x42 region of SSIM-map positions the tile's gradient
-// depends on, the map and its three partial derivatives there (zero outside
-// the image), then the separable adjoint filter back onto the 32x32 tile.
-// Block partial sums of |x - y| and of the map go to a small array that the
-// last CTA to finish reduces in a fixed order in float64, so the loss is
-// deterministic.
+// B200 design: one CTA per channel and 32-column x kStrip-row strip walks down
+// the strip in steps of 16 rows, with the separable filters pipelined through
+// ring buffers in shared memory, so every input row is filtered horizontally
+// once, every SSIM-map row is formed once, and every intermediate stays on
+// chip (the kernel reads the two images once and writes the gradient once, 36
+// B per pixel over the three channels). A step:
+//   1. loads 16 input rows x 52 columns of both images (zero outside);
+//   2. filters them horizontally into the 5 moments at the 42 map columns
+//      the strip's gradient depends on (ring of 28 rows);
+//   3. filters 16 map rows vertically from the ring, forms the SSIM map and
+//      its partial derivatives there (zero outside the image);
+//   4. filters those partials horizontally onto the 32 output columns (ring);
+//   5. filters the output rows whose 11 rows of partials are complete
+//      vertically and writes dL/dx with the L1 term.
+// Each stage lags the previous one by the window radius, so the outputs of a
+// step are 20 rows behind its inputs. Block partial sums of |x - y| and of the
+// map go to a small array that the last CTA to finish reduces in a fixed
+// order in float64, so the loss is deterministic.
 #include "gs_kernels.cuh"
 
 namespace gs {
 
 namespace {
 
-constexpr int kOut = 32;                 // output tile side
-constexpr int kR = 5;                    // window radius
-constexpr int kQ = kOut + 2 * kR;        // 42: SSIM-map positions needed
-constexpr int kIn = kOut + 4 * kR;       // 52: input pixels needed
-constexpr int kQs = 44;                  // padded row stride of the 42-wide maps (16 B rows)
+constexpr int kCols = kLossCols;          // output columns per CTA
+constexpr int kStrip = kLossStrip;        // output rows per CTA
+constexpr int kStep = 16;                 // rows per pipeline step
+constexpr int kR = 5;                     // window radius
+constexpr int kMapCols = kCols + 2 * kR;  // 42: SSIM-map columns needed
+constexpr int kInCols = kCols + 4 * kR;   // 52: input columns needed
+constexpr int kInS = 56;                  // padded input row stride (zeros beyond 52)
+constexpr int kHs = 44;                   // padded map row stride (16-byte rows)
+constexpr int kRing = 28;                 // ring rows (>= kStep + 2 kR = 26)
 constexpr int kLossThreads = 256;
-static_assert(kQs >= kQ && kQs % 4 == 0, "map rows must hold the 42 columns and stay 16-byte aligned");
+static_assert(kRing >= kStep + 2 * kR, "a ring must hold a step and its halo");
+
+// Ring slot of a row given its offset from the strip's first ring row
+// (offsets down to -2 kRing occur for rows above the strip, which are never read).
+__device__ __forceinline__ int ring_slot(int v) { return (v + 2 * kRing) % kRing; }
 
 struct LossSmem {
-  float x[kIn * kIn];
-  float y[kIn * kIn];
-  union {
-    float h[5][kIn * kQs];   // horizontal moments: input rows x map columns
-    float a[3][kQ * kOut];   // (after the vertical pass) horizontally filtered partials
-  };
-  float d[3][kQ * kQs];  // map partials dS/dmu_x, dS/dE[x^2], dS/dE[xy]
+  float in[2][kStep][kInS];       // x, y rows of this step
+  float h[5][kRing][kHs];         // horizontal moments mu_x, mu_y, E[x^2], E[y^2], E[xy]
+  float d[3][kStep][kHs];         // map partials dS/dmu_x, dS/dE[x^2], dS/dE[xy] of this step
+  float a[3][kRing][kCols];       // horizontally filtered partials
   double red[2][kLossThreads / 32];
   int last;
 };
@@ -62,8 +69,9 @@ __global__ void __launch_bounds__(kLossThreads) loss_kernel(LossArgs a) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   LossSmem& s = *reinterpret_cast<LossSmem*>(smem_raw);
   const int tid = threadIdx.x;
-  const int x0 = blockIdx.x * kOut, y0 = blockIdx.y * kOut;
+  const int x0 = blockIdx.x * kCols, Y0 = blockIdx.y * kStrip;
   const int H = a.height, W = a.width;
+  const int Yend = min(Y0 + kStrip, H);
   const int64_t HW = static_cast<int64_t>(H) * W;
   const float inv = static_cast<float>(1.0 / (3.0 * static_cast<double>(HW)));
   const float C1 = 0.01f * 0.01f, C2 = 0.03f * 0.03f;
@@ -71,106 +79,101 @@ __global__ void __launch_bounds__(kLossThreads) loss_kernel(LossArgs a) {
   float w[2 * kR + 1];
 #pragma unroll
   for (int t = 0; t <= 2 * kR; ++t) w[t] = a.window[t];
-
   const int ch = blockIdx.z;
   const float* X = a.x + ch * HW;
   const float* Yc = a.y + ch * HW;
-  // 1. input region [y0 - 10, y0 + 42) x [x0 - 10, x0 + 42), zero padded
-  for (int k = tid; k < kIn * kIn; k += kLossThreads) {
-    const int r = k / kIn, c = k % kIn;
-    const int gy = y0 - 2 * kR + r, gx = x0 - 2 * kR + c;
-    const bool in = gy >= 0 && gy < H && gx >= 0 && gx < W;
-    const int64_t g = static_cast<int64_t>(gy) * W + gx;
-    s.x[k] = in ? __ldg(X + g) : 0.0f;
-    s.y[k] = in ? __ldg(Yc + g) : 0.0f;
-  }
-  __syncthreads();
-  // 2. horizontal moments, 4 map columns per item from a 16-wide window in
-  //    registers; map column j <-> image x0 - 5 + j
-  for (int it = tid; it < kIn * 11; it += kLossThreads) {
-    const int r = it / 11, j0 = 4 * (it % 11);
-    float xv[16], yv[16];
+
+  // outputs trail the inputs by 4 kR rows: step st writes output rows
+  // [Y0 - 4 kR + kStep st, Y0 - 4 kR + kStep (st + 1)), so L rows need the
+  // smallest S with kStep (S - 1) >= L + 4 kR - kStep
+  const int steps = (Yend - Y0 + 4 * kR - 1) / kStep + 1;
+  for (int st = 0; st < steps; ++st) {
+    const int hb = Y0 - 2 * kR + kStep * st;  // first input row of this step
+    const int mb = hb - kR;                   // first map row of this step
+    const int ob = mb - kR;                   // first output row of this step
+    // 1. input rows [hb, hb + 16) x image columns [x0 - 10, x0 + 46) (zero outside)
+    for (int k = tid; k < 2 * kStep * kInS; k += kLossThreads) {
+      const int img = k / (kStep * kInS), rem = k % (kStep * kInS);
+      const int r = rem / kInS, c = rem % kInS;
+      const int gy = hb + r, gx = x0 - 2 * kR + c;
+      const bool in = c < kInCols && gy >= 0 && gy < H && gy < Yend + 2 * kR && gx >= 0 && gx < W;
+      s.in[img][r][c] = in ? __ldg((img ? Yc : X) + static_cast<int64_t>(gy) * W + gx) : 0.0f;
+    }
+    __syncthreads();
+    // 2. horizontal moments of the 16 rows at map columns j (image x0 - 5 + j),
+    //    4 columns per item from a 14-wide window held in registers
+    for (int it = tid; it < kStep * 11; it += kLossThreads) {
+      const int r = it / 11, j0 = 4 * (it % 11);
+      float xv[16], yv[16];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int c = j0 + 4 * q;
-      if (c < kIn) {
-        load4(s.x + r * kIn + c, xv + 4 * q);
-        load4(s.y + r * kIn + c, yv + 4 * q);
-      } else {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) xv[4 * q + e] = yv[4 * q + e] = 0.f;
+      for (int q = 0; q < 4; ++q) {
+        load4(&s.in[0][r][j0 + 4 * q], xv + 4 * q);  // j0 + 4 q + 3 <= 55 < kInS
+        load4(&s.in[1][r][j0 + 4 * q], yv + 4 * q);
       }
-    }
-    float pxx[14], pyy[14], pxy[14];  // products once per window element
+      float pxx[14], pyy[14], pxy[14];
 #pragma unroll
-    for (int e = 0; e < 14; ++e) {
-      pxx[e] = xv[e] * xv[e];
-      pyy[e] = yv[e] * yv[e];
-      pxy[e] = xv[e] * yv[e];
-    }
-    float m[5][4];
-#pragma unroll
-    for (int o = 0; o < 4; ++o) {
-      float mx = 0.f, my = 0.f, mxx = 0.f, myy = 0.f, mxy = 0.f;
-#pragma unroll
-      for (int t = 0; t <= 2 * kR; ++t) {
-        mx = __fmaf_rn(w[t], xv[o + t], mx);
-        my = __fmaf_rn(w[t], yv[o + t], my);
-        mxx = __fmaf_rn(w[t], pxx[o + t], mxx);
-        myy = __fmaf_rn(w[t], pyy[o + t], myy);
-        mxy = __fmaf_rn(w[t], pxy[o + t], mxy);
+      for (int e = 0; e < 14; ++e) {
+        pxx[e] = xv[e] * xv[e];
+        pyy[e] = yv[e] * yv[e];
+        pxy[e] = xv[e] * yv[e];
       }
-      m[0][o] = mx;
-      m[1][o] = my;
-      m[2][o] = mxx;
-      m[3][o] = myy;
-      m[4][o] = mxy;
+      const int ring = ring_slot(hb + r - Y0 + 2 * kR);
+      float m[5][4];
+#pragma unroll
+      for (int o = 0; o < 4; ++o) {
+        float mx = 0.f, my = 0.f, mxx = 0.f, myy = 0.f, mxy = 0.f;
+#pragma unroll
+        for (int t = 0; t <= 2 * kR; ++t) {
+          mx = __fmaf_rn(w[t], xv[o + t], mx);
+          my = __fmaf_rn(w[t], yv[o + t], my);
+          mxx = __fmaf_rn(w[t], pxx[o + t], mxx);
+          myy = __fmaf_rn(w[t], pyy[o + t], myy);
+          mxy = __fmaf_rn(w[t], pxy[o + t], mxy);
+        }
+        m[0][o] = mx;
+        m[1][o] = my;
+        m[2][o] = mxx;
+        m[3][o] = myy;
+        m[4][o] = mxy;
+      }
+#pragma unroll
+      for (int c = 0; c < 5; ++c)
+        *reinterpret_cast<float4*>(&s.h[c][ring][j0]) = make_float4(m[c][0], m[c][1], m[c][2], m[c][3]);
     }
+    __syncthreads();
+    // 3. vertical pass for map rows [mb, mb + 16) (1 column x 4 rows per item),
+    //    SSIM map and its partial derivatives
+    for (int it = tid; it < kMapCols * 4; it += kLossThreads) {
+      const int j = it % kMapCols, k0 = 4 * (it / kMapCols);
+      const int q0 = mb + k0;
+      float acc[5][4];
 #pragma unroll
-    for (int c = 0; c < 5; ++c)
-      *reinterpret_cast<float4*>(s.h[c] + r * kQs + j0) = make_float4(m[c][0], m[c][1], m[c][2], m[c][3]);
-  }
-  __syncthreads();
-  // 3. vertical pass (2 map columns x 4 map rows per item), SSIM map and its
-  //    partial derivatives at the 42x42 positions
-  for (int it = tid; it < 21 * 11; it += kLossThreads) {
-    const int qj = 2 * (it % 21), qi0 = 4 * (it / 21);
-    float acc[5][4][2];
+      for (int c = 0; c < 5; ++c)
 #pragma unroll
-    for (int c = 0; c < 5; ++c)
+        for (int o = 0; o < 4; ++o) acc[c][o] = 0.f;
+      if (q0 + 3 >= Y0 - kR) {  // rows above Y0 - 5 feed no output of this strip
 #pragma unroll
-      for (int o = 0; o < 4; ++o) acc[c][o][0] = acc[c][o][1] = 0.f;
+        for (int rr = 0; rr < 14; ++rr) {
+          const int ring = ring_slot(q0 - kR + rr - Y0 + 2 * kR);
 #pragma unroll
-    for (int rr = 0; rr < 14; ++rr) {
-      const int row = qi0 + rr;
-      if (row >= kIn) break;
+          for (int c = 0; c < 5; ++c) {
+            const float hv = s.h[c][ring][j];
 #pragma unroll
-      for (int c = 0; c < 5; ++c) {
-        const float2 hv = *reinterpret_cast<const float2*>(s.h[c] + row * kQs + qj);
-#pragma unroll
-        for (int o = 0; o < 4; ++o) {
-          const int t = rr - o;
-          if (t >= 0 && t <= 2 * kR) {
-            acc[c][o][0] = __fmaf_rn(w[t], hv.x, acc[c][o][0]);
-            acc[c][o][1] = __fmaf_rn(w[t], hv.y, acc[c][o][1]);
+            for (int o = 0; o < 4; ++o) {
+              const int t = rr - o;
+              if (t >= 0 && t <= 2 * kR) acc[c][o] = __fmaf_rn(w[t], hv, acc[c][o]);
+            }
           }
         }
       }
-    }
 #pragma unroll
-    for (int o = 0; o < 4; ++o) {
-      const int qi = qi0 + o;
-      if (qi >= kQ) break;
-      float dm2[2], dxx2[2], dxy2[2];
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int qje = qj + e;
-        const int gy = y0 - kR + qi, gx = x0 - kR + qje;
+      for (int o = 0; o < 4; ++o) {
+        const int q = q0 + o, gx = x0 - kR + j;
         float dm = 0.f, dxx = 0.f, dxy = 0.f;
-        if (gy >= 0 && gy < H && gx >= 0 && gx < W) {
-          const float mux = acc[0][o][e], muy = acc[1][o][e];
-          const float sxx = acc[2][o][e] - mux * mux, syy = acc[3][o][e] - muy * muy;
-          const float sxy = acc[4][o][e] - mux * muy;
+        if (q >= 0 && q < H && q >= Y0 - kR && gx >= 0 && gx < W) {
+          const float mux = acc[0][o], muy = acc[1][o];
+          const float sxx = acc[2][o] - mux * mux, syy = acc[3][o] - muy * muy;
+          const float sxy = acc[4][o] - mux * muy;
           const float A1 = 2.f * mux * muy + C1, A2 = 2.f * sxy + C2;
           const float B1 = mux * mux + muy * muy + C1, B2 = sxx + syy + C2;
           const float iB1 = 1.0f / B1, iB2 = 1.0f / B2;
@@ -180,91 +183,79 @@ __global__ void __launch_bounds__(kLossThreads) loss_kernel(LossArgs a) {
           dm = 2.f * muy * (A2 - A1) * iB - 2.f * mux * S * (iB1 - iB2);
           dxx = -S * iB2;
           dxy = 2.f * A1 * iB;
-          if (qi >= kR && qi < kR + kOut && qje >= kR && qje < kR + kOut) ssim_acc += S;
+          if (q >= Y0 && q < Yend && j >= kR && j < kR + kCols) ssim_acc += S;
         }
-        dm2[e] = dm;
-        dxx2[e] = dxx;
-        dxy2[e] = dxy;
-      }
-      *reinterpret_cast<float2*>(s.d[0] + qi * kQs + qj) = make_float2(dm2[0], dm2[1]);
-      *reinterpret_cast<float2*>(s.d[1] + qi * kQs + qj) = make_float2(dxx2[0], dxx2[1]);
-      *reinterpret_cast<float2*>(s.d[2] + qi * kQs + qj) = make_float2(dxy2[0], dxy2[1]);
-    }
-  }
-  __syncthreads();
-  // 4. horizontal adjoint onto the output columns (the window is symmetric):
-  //    4 output columns per item from a 16-wide window of each partial map
-  for (int it = tid; it < kQ * 8; it += kLossThreads) {
-    const int r = it / 8, j0 = 4 * (it % 8);
-    float out[3][4];
-#pragma unroll
-    for (int c = 0; c < 3; ++c) {
-      float dv[16];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int col = j0 + 4 * q;
-        if (col < kQs) {
-          load4(s.d[c] + r * kQs + col, dv + 4 * q);
-        } else {
-#pragma unroll
-          for (int e = 0; e < 4; ++e) dv[4 * q + e] = 0.f;
-        }
-      }
-#pragma unroll
-      for (int o = 0; o < 4; ++o) {
-        float acc = 0.f;
-#pragma unroll
-        for (int t = 0; t <= 2 * kR; ++t) acc = __fmaf_rn(w[t], dv[o + t], acc);
-        out[c][o] = acc;
+        s.d[0][k0 + o][j] = dm;
+        s.d[1][k0 + o][j] = dxx;
+        s.d[2][k0 + o][j] = dxy;
       }
     }
-#pragma unroll
-    for (int c = 0; c < 3; ++c)
-      *reinterpret_cast<float4*>(s.a[c] + r * kOut + j0) = make_float4(out[c][0], out[c][1], out[c][2], out[c][3]);
-  }
-  __syncthreads();
-  // 5. vertical adjoint (2 columns x 4 rows per item), L1 term, gradient out
-  for (int it = tid; it < 16 * 8; it += kLossThreads) {
-    const int j = 2 * (it % 16), i0 = 4 * (it / 16);
-    float acc[3][4][2];
-#pragma unroll
-    for (int c = 0; c < 3; ++c)
-#pragma unroll
-      for (int o = 0; o < 4; ++o) acc[c][o][0] = acc[c][o][1] = 0.f;
-#pragma unroll
-    for (int rr = 0; rr < 14; ++rr) {
-      const int row = i0 + rr;
+    __syncthreads();
+    // 4. horizontal adjoint of the map rows onto the 32 output columns
+    //    (the window is symmetric), 2 columns per item
+    for (int it = tid; it < kStep * (kCols / 2); it += kLossThreads) {
+      const int k = it / (kCols / 2), jj = 2 * (it % (kCols / 2));
+      const int ring = ring_slot(mb + k - Y0 + kR);
 #pragma unroll
       for (int c = 0; c < 3; ++c) {
-        const float2 av = *reinterpret_cast<const float2*>(s.a[c] + row * kOut + j);
+        float dv[12];
 #pragma unroll
-        for (int o = 0; o < 4; ++o) {
-          const int t = rr - o;
-          if (t >= 0 && t <= 2 * kR) {
-            acc[c][o][0] = __fmaf_rn(w[t], av.x, acc[c][o][0]);
-            acc[c][o][1] = __fmaf_rn(w[t], av.y, acc[c][o][1]);
+        for (int e = 0; e < 12; e += 2) {
+          const float2 t2 = *reinterpret_cast<const float2*>(&s.d[c][k][jj + e]);
+          dv[e] = t2.x;
+          dv[e + 1] = t2.y;
+        }
+        float o0 = 0.f, o1 = 0.f;
+#pragma unroll
+        for (int t = 0; t <= 2 * kR; ++t) {
+          o0 = __fmaf_rn(w[t], dv[t], o0);
+          o1 = __fmaf_rn(w[t], dv[t + 1], o1);
+        }
+        *reinterpret_cast<float2*>(&s.a[c][ring][jj]) = make_float2(o0, o1);
+      }
+    }
+    __syncthreads();
+    // 5. vertical adjoint for output rows [ob, ob + 16) (1 column x 2 rows per item),
+    //    L1 term and the gradient
+    for (int it = tid; it < kCols * (kStep / 2); it += kLossThreads) {
+      const int jj = it % kCols, k0 = 2 * (it / kCols);
+      const int r0 = ob + k0;
+      if (r0 + 1 < Y0 || r0 >= Yend) continue;
+      float acc[3][2];
+#pragma unroll
+      for (int c = 0; c < 3; ++c) acc[c][0] = acc[c][1] = 0.f;
+#pragma unroll
+      for (int rr = 0; rr < 12; ++rr) {
+        const int ring = ring_slot(r0 - kR + rr - Y0 + kR);
+#pragma unroll
+        for (int c = 0; c < 3; ++c) {
+          const float av = s.a[c][ring][jj];
+#pragma unroll
+          for (int o = 0; o < 2; ++o) {
+            const int t = rr - o;
+            if (t >= 0 && t <= 2 * kR) acc[c][o] = __fmaf_rn(w[t], av, acc[c][o]);
           }
         }
       }
-    }
+      const int gx = x0 + jj;
 #pragma unroll
-    for (int o = 0; o < 4; ++o)
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int i = i0 + o, jj = j + e;
-        const int gy = y0 + i, gx = x0 + jj;
-        if (gy >= H || gx >= W) continue;
-        const float xv = s.x[(i + 2 * kR) * kIn + jj + 2 * kR];
-        const float yv = s.y[(i + 2 * kR) * kIn + jj + 2 * kR];
+      for (int o = 0; o < 2; ++o) {
+        const int gy = r0 + o;
+        if (gy < Y0 || gy >= Yend || gx >= W) continue;
+        const int64_t g = static_cast<int64_t>(gy) * W + gx;
+        const float xv = __ldg(X + g), yv = __ldg(Yc + g);
         const float r = xv - yv;
         l1_acc += fabsf(r);
         if (a.dx) {
-          const float G = acc[0][o][e] + 2.f * xv * acc[1][o][e] + yv * acc[2][o][e];
+          const float G = acc[0][o] + 2.f * xv * acc[1][o] + yv * acc[2][o];
           const float sgn = r > 0.f ? 1.f : (r < 0.f ? -1.f : 0.f);
-          a.dx[ch * HW + static_cast<int64_t>(gy) * W + gx] = (1.f - a.lambda) * inv * sgn - a.lambda * inv * G;
+          a.dx[ch * HW + g] = (1.f - a.lambda) * inv * sgn - a.lambda * inv * G;
         }
       }
+    }
+    // the next step's stage 1 writes only the input rows; its stage 2 waits at a barrier
   }
+  __syncthreads();
 
   // Block partial sums in float64, then the last CTA reduces all in fixed order.
   double l1 = l1_acc, ss = ssim_acc;
@@ -333,13 +324,11 @@ cudaError_t launch_loss(const LossArgs& a, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(loss_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(sizeof(LossSmem)));
   if (e != cudaSuccess) return e;
-  dim3 grid((a.width + kOut - 1) / kOut, (a.height + kOut - 1) / kOut, 3);
+  dim3 grid((a.width + kCols - 1) / kCols, (a.height + kStrip - 1) / kStrip, 3);
   loss_kernel<<<grid, kLossThreads, sizeof(LossSmem), st>>>(a);
   return cudaGetLastError();
 }
 
-int64_t loss_num_blocks(int height, int width) {
-  return 3 * static_cast<int64_t>((width + kOut - 1) / kOut) * ((height + kOut - 1) / kOut);
-}
+int64_t loss_num_blocks(int height, int width) { return loss_blocks(height, width); }
 
 }  // namespace gs

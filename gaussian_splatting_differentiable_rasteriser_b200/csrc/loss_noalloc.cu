@@ -10,7 +10,7 @@
 // fixed size instead of in a context.
 //
 // The arrays are part of the library image: every GPU that loads the library
-// holds them (about 0.8 MB) until the process exits. In host code the array
+// holds them (about 0.2 MB) until the process exits. In host code the array
 // names are host-side stand-ins, not device addresses, so the device address
 // is taken once per device with cudaGetSymbolAddress while that device is
 // current, and that address is what the kernel receives.
@@ -26,10 +26,10 @@ int64_t loss_num_blocks(int height, int width);
 
 namespace {
 
-// Largest image the variant accepts: 4096 x 4096 (the loss runs one CTA per
-// 32x32 tile and channel, so 3 * 128 * 128 CTAs).
+// Largest image the variant accepts: 4096 x 4096 (one loss CTA per channel
+// and 32 x 128 strip, so 3 * 128 * 32 CTAs).
 constexpr int kNoAllocMaxSide = 4096;
-constexpr int64_t kNoAllocMaxBlocks = 3LL * (kNoAllocMaxSide / 32) * (kNoAllocMaxSide / 32);
+constexpr int64_t kNoAllocMaxBlocks = gs::loss_blocks(kNoAllocMaxSide, kNoAllocMaxSide);
 
 static __device__ __align__(256) double g_loss_partials[2 * kNoAllocMaxBlocks];
 static __device__ __align__(256) uint32_t g_loss_counter[1];

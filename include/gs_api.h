@@ -172,7 +172,7 @@ gs_status gs_render_backward(gs_ctx *ctx, const gs_params *params, const gs_came
  * start-up, hosts that hand over only input and output pointers). The pages
  * describe no counterpart; this is an interface convenience of this library.
  * It needs no context: the kernel's scratch (per-CTA partial sums and a
- * completion counter, about 0.8 MB) is a file-scope __device__ array that
+ * completion counter, about 0.2 MB) is a file-scope __device__ array that
  * every GPU loading the library holds until the process exits. The first call
  * on each device looks up the array's device address (cudaGetSymbolAddress,
  * with that device current), so make that first call before any stream

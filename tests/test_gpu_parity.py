@@ -229,7 +229,7 @@ def test_invalid_arguments_are_rejected_on_the_host(gs):
         native.Context(s.n_pad, 4096, 64, 64).render_forward(cs, img, img[0], img[0].int())
 
 
-@pytest.mark.parametrize("shape", [(256, 256), (37, 45), (70, 33)])
+@pytest.mark.parametrize("shape", [(256, 256), (37, 45), (70, 33), (300, 97), (1, 40), (7, 3), (129, 64)])
 def test_loss_matches_oracle(gs, shape):
     native, _ = gs
     H, W = shape
