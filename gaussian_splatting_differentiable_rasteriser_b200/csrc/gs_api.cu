@@ -135,7 +135,8 @@ gs_status check_params(gs_ctx* c, const gs_params* p) {
   const void* ptrs[] = {p->means, p->log_scales, p->quats, p->opacity_logits, p->sh};
   if (p->n > 0)
     for (const void* q : ptrs)
-      if (!q || !aligned(q, 4)) return fail(c, GS_ERR_INVALID_ARG, "a parameter pointer is NULL or misaligned");
+      if (!q || !aligned(q, 16))
+        return fail(c, GS_ERR_INVALID_ARG, "a parameter pointer is NULL or not 16-byte aligned");
   return GS_OK;
 }
 
@@ -145,7 +146,9 @@ gs_status take_device_error(gs_ctx* c) {
   c->info_host->device_error = 0;
   cudaMemset(&c->info_dev->device_error, 0, sizeof(uint32_t));
   return fail(c, GS_ERR_DEVICE, "a kernel recorded a device fault (code 0x%x: %s)", e,
-              (e & gs::kErrLookbackTimeout) ? "sort look-back wait gave up" : "index out of range");
+              (e & gs::kErrLookbackTimeout) ? "sort look-back wait gave up"
+              : (e & gs::kErrCopyTimeout)   ? "parameter copy wait gave up"
+                                            : "index out of range");
 }
 
 void prof_harvest(gs_ctx* c) {
@@ -323,6 +326,7 @@ gs_status gs_preprocess(gs_ctx* c, const gs_params* p, const gs_camera* cam, voi
   a.clamped = c->clamped;
   a.block_sums = c->block_sums;
   a.depth_range = c->depth_range;
+  a.err = &c->info_dev->device_error;
   const int64_t nb = (p->n + 255) / 256;
   prof_begin(c, st);
   GS_CUDA(c, gs::launch_preprocess(a, nb, st));

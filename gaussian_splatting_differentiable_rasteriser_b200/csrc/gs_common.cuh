@@ -61,6 +61,7 @@ struct CamArgs {
 enum DeviceError : uint32_t {
   kErrLookbackTimeout = 1u,
   kErrIndexRange = 2u,
+  kErrCopyTimeout = 4u,
 };
 
 __device__ __forceinline__ void record_error(uint32_t* err, uint32_t code) {

@@ -30,6 +30,7 @@ struct PreprocessArgs {
   uint8_t* clamped;
   uint2* block_sums;      // per 256-Gaussian block: (tiles touched, visible Gaussians)
   uint32_t* depth_range;  // [min, max] of visible depth keys (atomics)
+  uint32_t* err;          // device error word
 };
 
 cudaError_t launch_preprocess(const PreprocessArgs& a, int64_t num_blocks, cudaStream_t st);

@@ -8,10 +8,12 @@
 // and "Spherical harmonics: color that changes with viewing angle".
 //
 // B200 notes: the kernel is HBM-bound (236 B of parameters in, 48 + 17 B out
-// per Gaussian at SH degree 3); all parameter loads are coalesced planar
-// reads. The geometry runs in float64 - free next to the memory time - so that
+// per Gaussian at SH degree 3). Each CTA stages its Gaussians' parameter
+// planes in shared memory with bulk asynchronous copies (the untiled TMA
+// path) completed on an mbarrier, then computes from shared memory. The geometry runs in float64 - free next to the memory time - so that
 // the integer decisions taken from it (culling, tile rect, depth key) are
 // stable to ~1e-15 and do not depend on float32 rounding order.
+#include "bulk_copy.cuh"
 #include "gs_kernels.cuh"
 #include "sh.cuh"
 
@@ -23,16 +25,63 @@ __device__ __forceinline__ double dot3(const double* a, const double* b) {
   return a[0] * b[0] + a[1] * b[1] + a[2] * b[2];
 }
 
+constexpr int kPreThreads = 256;
+constexpr int kGeomPlanes = 11;  // means 3, log-scales 3, quats 4, opacity logit 1
+
+// The parameters of a CTA's 256 Gaussians, one 1 KB row per plane: the
+// geometric planes, then the 3 x (kDeg + 1)^2 active SH planes.
 template <int kDeg>
-__global__ void __launch_bounds__(256, 3) preprocess_kernel(PreprocessArgs a) {
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+struct PreprocessSmem {
+  float plane[kGeomPlanes + 3 * (kDeg + 1) * (kDeg + 1)][kPreThreads];
+  uint64_t bar;
+  int ok;
+};
+
+template <int kDeg>
+__global__ void __launch_bounds__(kPreThreads, 3) preprocess_kernel(PreprocessArgs a) {
+  constexpr int nk = (kDeg + 1) * (kDeg + 1);
+  constexpr int kPlanes = kGeomPlanes + 3 * nk;
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  PreprocessSmem<kDeg>& sm = *reinterpret_cast<PreprocessSmem<kDeg>*>(smem_raw);
+  const int tid = threadIdx.x;
+  const int64_t i0 = static_cast<int64_t>(blockIdx.x) * kPreThreads;
+  const int64_t i = i0 + tid;
+  const int64_t np = a.n_pad;
+  // Stage the CTA's slice of every parameter plane in shared memory with bulk
+  // asynchronous copies issued by one thread, so all of a Gaussian's loads
+  // (about 240 B at degree 3) are in flight at once instead of behind the
+  // geometry's dependency chain. Planes start 16-byte aligned (n_pad % 4 == 0,
+  // 16-byte aligned parameter pointers) and a slice is a multiple of 4 floats.
+  if (tid == 0) {
+    mbar_init(&sm.bar);
+    const int cnt = static_cast<int>(np - i0 < kPreThreads ? np - i0 : kPreThreads);
+    const uint32_t bytes = static_cast<uint32_t>(cnt) * 4u;
+    mbar_arrive_expect_tx(&sm.bar, bytes * kPlanes);
+#pragma unroll
+    for (int c = 0; c < 3; ++c) bulk_copy_g2s(sm.plane[c], a.means + c * np + i0, bytes, &sm.bar);
+#pragma unroll
+    for (int c = 0; c < 3; ++c) bulk_copy_g2s(sm.plane[3 + c], a.log_scales + c * np + i0, bytes, &sm.bar);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) bulk_copy_g2s(sm.plane[6 + c], a.quats + c * np + i0, bytes, &sm.bar);
+    bulk_copy_g2s(sm.plane[10], a.opacity_logits + i0, bytes, &sm.bar);
+    for (int ch = 0; ch < 3; ++ch)
+      for (int k = 0; k < nk; ++k)
+        bulk_copy_g2s(sm.plane[kGeomPlanes + ch * nk + k],
+                      a.sh + (static_cast<int64_t>(ch) * a.sh_k + k) * np + i0, bytes, &sm.bar);
+    bool ok = mbar_wait(&sm.bar, 0, 1 << 16);
+    if (!ok) {
+      record_error(a.err, kErrCopyTimeout);
+      mbar_wait(&sm.bar, 0, 1 << 16);  // let the copies land before the CTA can exit
+    }
+    sm.ok = ok ? 1 : 0;
+  }
+  __syncthreads();
   uint32_t touched = 0;
   uint32_t dkey = 0;
   bool visible = false;
-  if (i < a.n) {
-    const int64_t np = a.n_pad;
+  if (i < a.n && sm.ok) {
     const CamArgs& cam = a.cam;
-    const double p[3] = {a.means[i], a.means[np + i], a.means[2 * np + i]};
+    const double p[3] = {sm.plane[0][tid], sm.plane[1][tid], sm.plane[2][tid]};
     // p_c = R p + t, each row summed left to right without fused multiply-add:
     // the depth key float32(Z) is then the same on every implementation.
     double pc[3];
@@ -52,16 +101,16 @@ __global__ void __launch_bounds__(256, 3) preprocess_kernel(PreprocessArgs a) {
     uint8_t clamped = 0;
     if (Z > static_cast<double>(cam.near_z)) {
       // Sigma = M M^T, M = R(q/|q|) diag(exp(ls))
-      const double qw = a.quats[i], qx = a.quats[np + i], qy = a.quats[2 * np + i],
-                   qz = a.quats[3 * np + i];
+      const double qw = sm.plane[6][tid], qx = sm.plane[7][tid], qy = sm.plane[8][tid],
+                   qz = sm.plane[9][tid];
       const double qn = sqrt(qw * qw + qx * qx + qy * qy + qz * qz);
       const double w = qw / qn, x = qx / qn, y = qy / qn, z = qz / qn;
       const double Rq[9] = {1.0 - 2.0 * (y * y + z * z), 2.0 * (x * y - w * z), 2.0 * (x * z + w * y),
                             2.0 * (x * y + w * z), 1.0 - 2.0 * (x * x + z * z), 2.0 * (y * z - w * x),
                             2.0 * (x * z - w * y), 2.0 * (y * z + w * x), 1.0 - 2.0 * (x * x + y * y)};
-      const double sc[3] = {exp(static_cast<double>(a.log_scales[i])),
-                            exp(static_cast<double>(a.log_scales[np + i])),
-                            exp(static_cast<double>(a.log_scales[2 * np + i]))};
+      const double sc[3] = {exp(static_cast<double>(sm.plane[3][tid])),
+                            exp(static_cast<double>(sm.plane[4][tid])),
+                            exp(static_cast<double>(sm.plane[5][tid]))};
       double M[9];
 #pragma unroll
       for (int r = 0; r < 3; ++r)
@@ -108,22 +157,20 @@ __global__ void __launch_bounds__(256, 3) preprocess_kernel(PreprocessArgs a) {
           touched = (x1 - x0 + 1) * (y1 - y0 + 1);
           visible = true;
           dkey = __float_as_uint(depth);
-          const float opacity = 1.0f / (1.0f + expf(-a.opacity_logits[i]));
+          const float opacity = 1.0f / (1.0f + expf(-sm.plane[10][tid]));
           // view-dependent colour at v = normalize(p - campos)
           double d[3] = {p[0] - cam.campos[0], p[1] - cam.campos[1], p[2] - cam.campos[2]};
           const double dn = sqrt(dot3(d, d));
           const float dx = static_cast<float>(d[0] / dn), dy = static_cast<float>(d[1] / dn),
                       dz = static_cast<float>(d[2] / dn);
-          constexpr int nk = (kDeg + 1) * (kDeg + 1);
           float Yk[16];
           sh_basis(kDeg, dx, dy, dz, Yk);
           float rgb[3];
 #pragma unroll
           for (int ch = 0; ch < 3; ++ch) {
-            const float* shc = a.sh + static_cast<int64_t>(ch) * a.sh_k * np + i;
             float col = 0.0f;
 #pragma unroll
-            for (int k = 0; k < nk; ++k) col = fmaf(shc[static_cast<int64_t>(k) * np], Yk[k], col);
+            for (int k = 0; k < nk; ++k) col = fmaf(sm.plane[kGeomPlanes + ch * nk + k][tid], Yk[k], col);
             if (col < 0.0f) {
               col = 0.0f;
               clamped |= static_cast<uint8_t>(1u << ch);
@@ -155,6 +202,12 @@ __global__ void __launch_bounds__(256, 3) preprocess_kernel(PreprocessArgs a) {
     a.rect[i] = rect;
     a.touched[i] = touched;
     a.clamped[i] = clamped;
+  } else if (i < a.n) {  // parameters not staged (the copy wait gave up): treat as culled
+    a.screen[i] = Screen{};
+    a.depth[i] = 0.0f;
+    a.rect[i] = make_uint2(1u, 1u);
+    a.touched[i] = 0u;
+    a.clamped[i] = 0u;
   }
 
   // Block totals of tiles touched and of visible Gaussians (for the entry
@@ -253,18 +306,26 @@ __global__ void __launch_bounds__(1024) scan_blocks_kernel(const uint2* block_su
   }
 }
 
+template <int kDeg>
+cudaError_t launch_preprocess_deg(const PreprocessArgs& a, unsigned grid, cudaStream_t st) {
+  const int smem = static_cast<int>(sizeof(PreprocessSmem<kDeg>));
+  cudaError_t e = cudaFuncSetAttribute(preprocess_kernel<kDeg>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  preprocess_kernel<kDeg><<<grid, kPreThreads, smem, st>>>(a);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_preprocess(const PreprocessArgs& a, int64_t num_blocks, cudaStream_t st) {
   if (a.n == 0) return cudaSuccess;
   const unsigned grid = static_cast<unsigned>(num_blocks);
   switch (a.active_degree) {
-    case 0: preprocess_kernel<0><<<grid, 256, 0, st>>>(a); break;
-    case 1: preprocess_kernel<1><<<grid, 256, 0, st>>>(a); break;
-    case 2: preprocess_kernel<2><<<grid, 256, 0, st>>>(a); break;
-    default: preprocess_kernel<3><<<grid, 256, 0, st>>>(a); break;
+    case 0: return launch_preprocess_deg<0>(a, grid, st);
+    case 1: return launch_preprocess_deg<1>(a, grid, st);
+    case 2: return launch_preprocess_deg<2>(a, grid, st);
+    default: return launch_preprocess_deg<3>(a, grid, st);
   }
-  return cudaGetLastError();
 }
 
 cudaError_t launch_scan_blocks(const uint2* block_sums, int64_t num_blocks, uint32_t* visible_prefix,

@@ -10,8 +10,9 @@
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
  *     Work is enqueued asynchronously on it. gs_render_forward is the one call
  *     that waits on the stream (it reads the entry count back to the host).
- *   - Parameters are structure-of-arrays, planar float32, with n <= n_pad and
- *     n_pad a multiple of 4, so every plane starts 16-byte aligned:
+ *   - Parameters are structure-of-arrays, planar float32, with n <= n_pad,
+ *     n_pad a multiple of 4 and 16-byte aligned base pointers, so every plane
+ *     starts 16-byte aligned:
  *         means           [3][n_pad]
  *         log_scales      [3][n_pad]
  *         quats           [4][n_pad]      (w, x, y, z), any non-zero length
