@@ -243,10 +243,20 @@ __global__ void __launch_bounds__(256) preprocess_backward_kernel(PreprocessBwdA
 constexpr int kFusedBlock = 128;
 constexpr int kGeomPlanes = 11;  // means 3, log-scales 3, quats 4, opacity logit 1
 
+constexpr int kMaxPlanes = kGeomPlanes + 3 * 16;
+
+// Where plane pl of the CTA's slice lives: group grp, plane c of that group,
+// and for an SH plane its channel ch and coefficient k (k = -1 when the
+// coefficient is outside the active bands, so this view adds nothing).
+struct PlaneInfo {
+  int grp, c, ch, k;
+};
+
 struct FusedSmem {
   float geom[kGeomPlanes][kFusedBlock];  // view gradient of the geometric scalars
   float drgb[3][kFusedBlock];            // masked dL/dcolour (0 when invisible)
   float Y[16][kFusedBlock];              // SH basis at the view direction
+  PlaneInfo plane[kMaxPlanes];
 };
 
 // kAccum: the caller's gradient buffer holds an accumulated gradient, which is
@@ -299,65 +309,73 @@ __global__ void __launch_bounds__(kFusedBlock) preprocess_backward_adam_kernel(P
       for (int k = 0; k < 16; ++k) sm.Y[k][t] = 0.f;
     }
   }
+  if (t < kGeomPlanes + 3 * a.sh_k) {
+    PlaneInfo pi;
+    if (t < 3) pi = PlaneInfo{0, t, 0, -1};
+    else if (t < 6) pi = PlaneInfo{1, t - 3, 0, -1};
+    else if (t < 10) pi = PlaneInfo{2, t - 6, 0, -1};
+    else if (t < 11) pi = PlaneInfo{3, 0, 0, -1};
+    else {
+      const int sp = t - kGeomPlanes, ch = sp / a.sh_k, k = sp % a.sh_k;
+      pi = PlaneInfo{4, sp, ch, k < nk ? k : -1};
+    }
+    sm.plane[t] = pi;
+  }
   __syncthreads();
 
-  // Phase 2: Adam over planes x float4 columns of this CTA's Gaussians.
+  // Phase 2: Adam over planes x float4 columns of this CTA's Gaussians. Thread
+  // t takes float4 column t % 32 of planes t / 32, t / 32 + 4, ...; four planes
+  // per round with all their loads issued before any store. Plane bookkeeping
+  // comes from the table built in phase 1 (one broadcast load per plane).
   const int64_t rem = np - i0;
   const int cols = static_cast<int>((rem < kFusedBlock ? rem : kFusedBlock) / 4);  // n_pad % 4 == 0
   const int planes = kGeomPlanes + 3 * a.sh_k;
-  const int units = planes * (kFusedBlock / 4);
-  for (int u0 = t; u0 < units; u0 += 4 * kFusedBlock) {
+  constexpr int kColUnits = kFusedBlock / 4;            // float4 columns per plane
+  constexpr int kPlaneStep = kFusedBlock / kColUnits;   // planes per sweep of the CTA
+  const int col = t % kColUnits;
+  const bool col_ok = col < cols;
+  for (int pl0 = t / kColUnits; pl0 < planes; pl0 += 4 * kPlaneStep) {
     float4 P[4], G[4], M[4], V[4];
+    PlaneInfo info[4];
     int64_t off[4];
-    int plane[4], col[4], grp[4];
-    bool ok[4];
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
-      const int u = u0 + r * kFusedBlock;
-      const int pl = u / (kFusedBlock / 4);
-      plane[r] = pl;
-      col[r] = u % (kFusedBlock / 4);
-      ok[r] = u < units && col[r] < cols;
-      int c;
-      if (pl < 3) { grp[r] = 0; c = pl; }
-      else if (pl < 6) { grp[r] = 1; c = pl - 3; }
-      else if (pl < 10) { grp[r] = 2; c = pl - 6; }
-      else if (pl < 11) { grp[r] = 3; c = 0; }
-      else { grp[r] = 4; c = pl - kGeomPlanes; }
-      off[r] = static_cast<int64_t>(c) * np + i0 + 4 * col[r];
+      const int pl = pl0 + r * kPlaneStep;
+      const bool ok = col_ok && pl < planes;
+      info[r] = sm.plane[pl < planes ? pl : 0];
+      off[r] = static_cast<int64_t>(info[r].c) * np + i0 + 4 * col;
       G[r] = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (ok[r]) {
-        P[r] = *reinterpret_cast<const float4*>(f.p[grp[r]] + off[r]);
-        if (kAccum) G[r] = *reinterpret_cast<const float4*>(f.g[grp[r]] + off[r]);
-        M[r] = *reinterpret_cast<const float4*>(f.m[grp[r]] + off[r]);
-        V[r] = *reinterpret_cast<const float4*>(f.v[grp[r]] + off[r]);
+      if (ok) {
+        P[r] = *reinterpret_cast<const float4*>(f.p[info[r].grp] + off[r]);
+        if (kAccum) G[r] = *reinterpret_cast<const float4*>(f.g[info[r].grp] + off[r]);
+        M[r] = *reinterpret_cast<const float4*>(f.m[info[r].grp] + off[r]);
+        V[r] = *reinterpret_cast<const float4*>(f.v[info[r].grp] + off[r]);
       }
     }
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
-      if (!ok[r]) continue;
-      const int pl = plane[r];
+      const int pl = pl0 + r * kPlaneStep;
+      if (!col_ok || pl >= planes) continue;
       float* p4 = &P[r].x;
       float* g4 = &G[r].x;
       float* m4 = &M[r].x;
       float* v4 = &V[r].x;
+      const AdamScalars sc = f.s[info[r].grp];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const int j = 4 * col[r] + e;
+        const int j = 4 * col + e;
         if (pl < kGeomPlanes) {
           g4[e] += sm.geom[pl][j];
-        } else {
-          const int sp = pl - kGeomPlanes;
-          const int ch = sp / a.sh_k, k = sp % a.sh_k;
-          const float dc = sm.drgb[ch][j];
-          if (k < nk && dc != 0.f) g4[e] = __fmaf_rn(dc, sm.Y[k][j], g4[e]);
+        } else if (info[r].k >= 0) {
+          const float dc = sm.drgb[info[r].ch][j];
+          if (dc != 0.f) g4[e] = __fmaf_rn(dc, sm.Y[info[r].k][j], g4[e]);
         }
-        adam_one(p4[e], g4[e], m4[e], v4[e], f.s[grp[r]]);
+        adam_one(p4[e], g4[e], m4[e], v4[e], sc);
       }
-      *reinterpret_cast<float4*>(f.p[grp[r]] + off[r]) = P[r];
-      if (kAccum) *reinterpret_cast<float4*>(f.g[grp[r]] + off[r]) = G[r];
-      *reinterpret_cast<float4*>(f.m[grp[r]] + off[r]) = M[r];
-      *reinterpret_cast<float4*>(f.v[grp[r]] + off[r]) = V[r];
+      *reinterpret_cast<float4*>(f.p[info[r].grp] + off[r]) = P[r];
+      if (kAccum) *reinterpret_cast<float4*>(f.g[info[r].grp] + off[r]) = G[r];
+      *reinterpret_cast<float4*>(f.m[info[r].grp] + off[r]) = M[r];
+      *reinterpret_cast<float4*>(f.v[info[r].grp] + off[r]) = V[r];
     }
   }
 }
