@@ -135,6 +135,9 @@ __global__ void __launch_bounds__(256) blend_forward_kernel(BlendArgs a) {
   int last = 0;
   bool done = !inside;
   unsigned blended = 0;
+  // this warp's survivors of the box test, in list order, for the backward
+  uint2* surv = a.surv + 8LL * beg + static_cast<int64_t>(warp) * (end - beg);
+  int nsurv = 0;
 
   // two-stage prefetch: the order entries of chunk i+2, the records of chunk i+1
   uint32_t gid_next = load_gid(a.order, beg + lane, beg, end);
@@ -147,9 +150,14 @@ __global__ void __launch_bounds__(256) blend_forward_kernel(BlendArgs a) {
     gid_next = load_gid(a.order, base + 64 + lane, beg, end);
     const bool keep = hits_block(cur, bx0, by0);
     const unsigned mask = __ballot_sync(0xffffffffu, keep);
-    if (keep) put_slot(ws, __popc(mask & lt), cur, base + lane - beg);
+    if (keep) {
+      const int slot = __popc(mask & lt);
+      put_slot(ws, slot, cur, base + lane - beg);
+      surv[nsurv + slot] = make_uint2(static_cast<uint32_t>(base + lane - beg), cur.gid);
+    }
     __syncwarp();
     const int cnt = __popc(mask);
+    nsurv += cnt;
     for (int k = 0; k < cnt; ++k) {
       const float2 xy = ws.xy[k];
       const float p = power2(ws.q[k], fx - xy.x, fy - xy.y);
@@ -168,6 +176,7 @@ __global__ void __launch_bounds__(256) blend_forward_kernel(BlendArgs a) {
     }
     __syncwarp();  // the slots are rewritten by the next chunk
   }
+  if (lane == 0) a.surv_count[tile * kWarps + warp] = static_cast<uint32_t>(nsurv);
   if (inside) {
     const int64_t hw = static_cast<int64_t>(a.cam.width) * a.cam.height;
     const int64_t pix = static_cast<int64_t>(py) * a.cam.width + px;
@@ -317,19 +326,28 @@ __global__ void __launch_bounds__(256) blend_backward_kernel(BlendArgs a) {
   unsigned blended = 0;
   int bcnt = 0;  // Gaussians in the warp's batch (warp-uniform)
 
-  // Chunks walk down from the top; lane l takes entry hi - 1 - l, so ballot
-  // order (lane order) is descending list order.
-  uint32_t gid_next = load_gid(a.order, top - 1 - lane, beg, top);
-  Entry nxt = load_entry(a.screen, gid_next, top - 1 - lane >= beg);
-  gid_next = load_gid(a.order, top - 33 - lane, beg, top);
-  for (int hi = top; hi > beg; hi -= 32) {
+  // The forward stored this warp's survivors of the box test (list position,
+  // Gaussian) in list order; walk them from the last one down. Lane l takes
+  // survivor hi - 1 - l, so ballot order (lane order) is descending list order;
+  // survivors at or past the warp's last contributor are dropped.
+  const int end = static_cast<int>(range.y);
+  const uint2* surv = a.surv + 8LL * beg + static_cast<int64_t>(warp) * (end - beg);
+  const int nsurv = min(static_cast<int>(a.surv_count[tile * kWarps + warp]), end - beg);
+  const int toprel = top - beg;
+  uint2 sv_next = nsurv - 1 - lane >= 0 ? surv[nsurv - 1 - lane] : make_uint2(0u, 0u);
+  Entry nxt = load_entry(a.screen, sv_next.y, nsurv - 1 - lane >= 0);
+  int pos_next = static_cast<int>(sv_next.x);
+  sv_next = nsurv - 33 - lane >= 0 ? surv[nsurv - 33 - lane] : make_uint2(0u, 0u);
+  for (int hi = nsurv; hi > 0; hi -= 32) {
     const Entry cur = nxt;
+    const int pos_cur = pos_next;
     const int j_cur = hi - 1 - lane;
-    nxt = load_entry(a.screen, gid_next, j_cur - 32 >= beg);
-    gid_next = load_gid(a.order, j_cur - 64, beg, top);
-    const bool keep = j_cur >= beg && hits_block(cur, bx0, by0);
+    nxt = load_entry(a.screen, sv_next.y, j_cur - 32 >= 0);
+    pos_next = static_cast<int>(sv_next.x);
+    sv_next = j_cur - 64 >= 0 ? surv[j_cur - 64] : make_uint2(0u, 0u);
+    const bool keep = j_cur >= 0 && pos_cur < toprel;
     const unsigned mask = __ballot_sync(0xffffffffu, keep);
-    if (keep) put_slot(ws, __popc(mask & lt), cur, j_cur - beg);
+    if (keep) put_slot(ws, __popc(mask & lt), cur, pos_cur);
     __syncwarp();
     const int cnt = __popc(mask);
     for (int k = 0; k < cnt; ++k) {

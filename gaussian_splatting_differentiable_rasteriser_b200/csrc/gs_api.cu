@@ -39,6 +39,8 @@ struct gs_ctx {
   uint32_t* status = nullptr;
   uint32_t* counters = nullptr;
   uint2* ranges = nullptr;
+  uint2* surv = nullptr;           // [8][max_entries]: per-warp survivors of the blend's box test
+  uint32_t* surv_count = nullptr;  // [max_tiles][8]
   // loss
   double* loss_partials = nullptr;
   uint32_t* loss_counter = nullptr;
@@ -89,7 +91,8 @@ void free_all(gs_ctx* c) {
   void* bufs[] = {c->screen, c->depth, c->rect, c->touched, c->clamped, c->sgrad, c->block_sums,
                   c->visible_prefix, c->depth_range, c->dkeys[0], c->dkeys[1], c->dvals[0],
                   c->dvals[1], c->dup_status, c->keys[0], c->keys[1], c->vals[0], c->vals[1],
-                  c->hist, c->offsets, c->status, c->counters, c->ranges, c->loss_partials,
+                  c->hist, c->offsets, c->status, c->counters, c->ranges, c->surv, c->surv_count,
+                  c->loss_partials,
                   c->loss_counter, c->info_dev, c->pairs};
   for (void* b : bufs)
     if (b) cudaFree(b);
@@ -268,6 +271,8 @@ gs_status gs_create(gs_ctx** out, int64_t max_gaussians, int64_t max_entries, in
   GS_ALLOC(c->status, sizeof(uint32_t) * gs::kMaxPasses * gs::kRadix * c->max_sort_tiles);
   GS_ALLOC(c->counters, sizeof(uint32_t) * (gs::kMaxPasses + 1));  // + the duplicate's ticket
   GS_ALLOC(c->ranges, sizeof(uint2) * c->max_tiles);
+  GS_ALLOC(c->surv, sizeof(uint2) * 8 * K);
+  GS_ALLOC(c->surv_count, sizeof(uint32_t) * 8 * c->max_tiles);
   GS_ALLOC(c->loss_partials, sizeof(double) * 2 * c->max_loss_blocks);
   GS_ALLOC(c->loss_counter, sizeof(uint32_t));
   GS_ALLOC(c->info_dev, sizeof(gs::ForwardInfo));
@@ -445,6 +450,8 @@ gs_status gs_render_forward(gs_ctx* c, const gs_camera* cam, float* image, float
   ba.final_T = final_T;
   ba.n_contrib = n_contrib;
   ba.pairs = c->prof.on ? c->pairs : nullptr;
+  ba.surv = c->surv;
+  ba.surv_count = c->surv_count;
   prof_begin(c, st);
   GS_CUDA(c, gs::launch_blend_forward(ba, st));
   prof_end(c, GS_STAGE_BLEND_FORWARD, 0, st);
@@ -524,6 +531,8 @@ gs_status backward_common(gs_ctx* c, const gs_params* p, const gs_camera* cam, c
   ba.dimage = dloss_dimage;
   ba.sgrad = c->sgrad;
   ba.pairs = c->prof.on ? c->pairs + 4 : nullptr;
+  ba.surv = c->surv;
+  ba.surv_count = c->surv_count;
   prof_begin(c, st);
   GS_CUDA(c, gs::launch_blend_backward(ba, st));
   prof_end(c, GS_STAGE_BLEND_BACKWARD, 0, st);

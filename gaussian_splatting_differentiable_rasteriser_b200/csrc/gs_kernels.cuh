@@ -122,6 +122,11 @@ struct BlendArgs {
   // when not null: pairs[0] += (pixel, Gaussian) pairs the method's walk visits,
   // pairs[2] += pairs that blend (alpha >= 1/255 before the walk stops)
   unsigned long long* pairs;
+  // per warp (8 per tile) the entries that pass its box test, written by the
+  // forward and walked by the backward: (list position, Gaussian) in list
+  // order, warp w of a tile with list [beg, end) at surv[8 beg + w (end - beg)]
+  uint2* surv;
+  uint32_t* surv_count;  // [tiles][8]
 };
 
 cudaError_t launch_blend_forward(const BlendArgs& a, cudaStream_t st);
