@@ -65,7 +65,28 @@ __device__ __forceinline__ void load4(const float* p, float* v) {
   v[3] = t.w;
 }
 
-__global__ void __launch_bounds__(kLossThreads) loss_kernel(LossArgs a) {
+constexpr int kLoadsPerThread = (2 * kStep * kInS + kLossThreads - 1) / kLossThreads;  // 7
+
+// The input rows [hb, hb + kStep) x image columns [x0 - 2 kR, x0 - 2 kR + kInS)
+// of both images, as they lie in LossSmem::in, this thread's share (zero
+// outside the image, beyond the 52 needed columns and beyond the rows the
+// strip needs).
+__device__ __forceinline__ void load_rows(const LossArgs& a, const float* X, const float* Yc, int x0, int hb,
+                                          int Yend, int tid, float (&pre)[kLoadsPerThread]) {
+  const int H = a.height, W = a.width;
+#pragma unroll
+  for (int u = 0; u < kLoadsPerThread; ++u) {
+    const int k = tid + u * kLossThreads;
+    const int img = k / (kStep * kInS), rem = k % (kStep * kInS);
+    const int r = rem / kInS, c = rem % kInS;
+    const int gy = hb + r, gx = x0 - 2 * kR + c;
+    const bool in = k < 2 * kStep * kInS && c < kInCols && gy >= 0 && gy < H && gy < Yend + 2 * kR &&
+                    gx >= 0 && gx < W;
+    pre[u] = in ? __ldg((img ? Yc : X) + static_cast<int64_t>(gy) * W + gx) : 0.0f;
+  }
+}
+
+__global__ void __launch_bounds__(kLossThreads, 4) loss_kernel(LossArgs a) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   LossSmem& s = *reinterpret_cast<LossSmem*>(smem_raw);
   const int tid = threadIdx.x;
@@ -87,19 +108,22 @@ __global__ void __launch_bounds__(kLossThreads) loss_kernel(LossArgs a) {
   // [Y0 - 4 kR + kStep st, Y0 - 4 kR + kStep (st + 1)), so L rows need the
   // smallest S with kStep (S - 1) >= L + 4 kR - kStep
   const int steps = (Yend - Y0 + 4 * kR - 1) / kStep + 1;
+  float pre[kLoadsPerThread];
   for (int st = 0; st < steps; ++st) {
     const int hb = Y0 - 2 * kR + kStep * st;  // first input row of this step
     const int mb = hb - kR;                   // first map row of this step
     const int ob = mb - kR;                   // first output row of this step
-    // 1. input rows [hb, hb + 16) x image columns [x0 - 10, x0 + 46) (zero outside)
-    for (int k = tid; k < 2 * kStep * kInS; k += kLossThreads) {
-      const int img = k / (kStep * kInS), rem = k % (kStep * kInS);
-      const int r = rem / kInS, c = rem % kInS;
-      const int gy = hb + r, gx = x0 - 2 * kR + c;
-      const bool in = c < kInCols && gy >= 0 && gy < H && gy < Yend + 2 * kR && gx >= 0 && gx < W;
-      s.in[img][r][c] = in ? __ldg((img ? Yc : X) + static_cast<int64_t>(gy) * W + gx) : 0.0f;
+    // 1. input rows [hb, hb + 16) x image columns [x0 - 10, x0 + 46) (zero
+    //    outside), loaded into registers one step ahead so their latency
+    //    overlaps the previous step's filtering
+    if (st == 0) load_rows(a, X, Yc, x0, hb, Yend, tid, pre);
+#pragma unroll
+    for (int u = 0; u < kLoadsPerThread; ++u) {
+      const int k = tid + u * kLossThreads;
+      if (k < 2 * kStep * kInS) (&s.in[0][0][0])[k] = pre[u];
     }
     __syncthreads();
+    if (st + 1 < steps) load_rows(a, X, Yc, x0, hb + kStep, Yend, tid, pre);
     // 2. horizontal moments of the 16 rows at map columns j (image x0 - 5 + j),
     //    4 columns per item from a 14-wide window held in registers
     for (int it = tid; it < kStep * 11; it += kLossThreads) {
