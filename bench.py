@@ -47,13 +47,15 @@ WORKLOADS = {
 
 # ncu DRAM traffic (read + write bytes per launch) of kernels on the dense workload,
 # with the sha256 (first 12 hex digits) of the source file each figure was taken from.
-# A figure whose source has changed since is reported as null. Both were captured on
-# the Mid workload (500k Gaussians, 1.06M entries; profiles/kernels_mid_720p.md) and
-# scaled to Dense by the units a launch processes (n_pad 3,000,000 / 500,000 for the
+# A figure whose source has changed since is reported as null. Both were captured
+# with ncu on the Mid workload (500k Gaussians, about 1.06M entries) and scaled to
+# Dense by the units a launch processes (n_pad 3,000,000 / 500,000 for the
 # per-Gaussian pass, entries 6.32M / 1.06M for the blend), in which traffic grows in
-# proportion.
+# proportion. The fused pass's write counter undercounts: its last writes are still
+# in L2 when the kernel ends.
 NCU_TRAFFIC = {
-    "blend_backward": ((70.30784e6 + 2.051584e6) * 6.32 / 1.064, "1386ae1844b4"),
+    "backward_adam": ((408.017408e6 + 295.502080e6) * 6.0, "07567fb73e7b"),
+    "blend_backward": ((85.316096e6 + 4.134912e6) * 6.32 / 1.064, "9e7084e8dff0"),
 }
 
 
