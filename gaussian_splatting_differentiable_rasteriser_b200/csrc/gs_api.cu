@@ -53,6 +53,8 @@ struct gs_ctx {
   gs::CamArgs cam{};
   int64_t K = 0;
   int sorted_buf = 0;
+  // options (gs_set_option)
+  int opacity_rect = 0;
   // profiling (off by default)
   struct Profiler {
     static constexpr int kMaxRec = 128;
@@ -303,6 +305,19 @@ void gs_destroy(gs_ctx* ctx) {
 
 const char* gs_last_error(const gs_ctx* ctx) { return ctx ? ctx->err : "no context"; }
 
+gs_status gs_set_option(gs_ctx* c, int32_t option, int32_t value) {
+  if (!c) return GS_ERR_INVALID_ARG;
+  switch (option) {
+    case GS_OPTION_OPACITY_RECT:
+      if (value != 0 && value != 1) return fail(c, GS_ERR_INVALID_ARG, "option value must be 0 or 1");
+      c->opacity_rect = value;
+      c->have_pre = c->have_fwd = false;  // the tile lists depend on it
+      return GS_OK;
+    default:
+      return fail(c, GS_ERR_INVALID_ARG, "unknown option %d", option);
+  }
+}
+
 gs_status gs_preprocess(gs_ctx* c, const gs_params* p, const gs_camera* cam, void* stream) {
   if (!c) return GS_ERR_INVALID_ARG;
   gs_status s = check_params(c, p);
@@ -332,6 +347,7 @@ gs_status gs_preprocess(gs_ctx* c, const gs_params* p, const gs_camera* cam, voi
   a.block_sums = c->block_sums;
   a.depth_range = c->depth_range;
   a.err = &c->info_dev->device_error;
+  a.opacity_rect = c->opacity_rect;
   const int64_t nb = (p->n + 255) / 256;
   prof_begin(c, st);
   GS_CUDA(c, gs::launch_preprocess(a, nb, st));

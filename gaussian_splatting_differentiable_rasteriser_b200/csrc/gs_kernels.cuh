@@ -31,6 +31,7 @@ struct PreprocessArgs {
   uint2* block_sums;      // per 256-Gaussian block: (tiles touched, visible Gaussians)
   uint32_t* depth_range;  // [min, max] of visible depth keys (atomics)
   uint32_t* err;          // device error word
+  int opacity_rect;       // opacity-aware tile rect (GS_OPTION_OPACITY_RECT)
 };
 
 cudaError_t launch_preprocess(const PreprocessArgs& a, int64_t num_blocks, cudaStream_t st);

@@ -144,7 +144,13 @@ __global__ void __launch_bounds__(kPreThreads, 3) preprocess_kernel(PreprocessAr
         const double v = cam.fy * Y * iz + cam.cy;
         const double mid = 0.5 * (ca + cc);
         const double lmax = mid + sqrt(fmax(mid * mid - det, 0.0));
-        const double rad = kRadiusSigmas * sqrt(lmax);
+        double rad = kRadiusSigmas * sqrt(lmax);
+        if (a.opacity_rect) {
+          // opacity-aware cut: beyond sqrt(2 E) sigma along the long axis alpha < 1/255
+          const double od = 1.0 / (1.0 + exp(-static_cast<double>(sm.plane[10][tid])));
+          const double e_cut = fmin(4.5, log(fmax(od * 255.0, 1.0001)));
+          rad = sqrt(2.0 * e_cut) * sqrt(lmax);
+        }
         // tiles whose pixels [16 t, 16 t + 15] meet [u - r, u + r] (same for y)
         double fx0 = fmax(ceil((u - rad - (kTile - 1)) / kTile), 0.0);
         double fx1 = fmin(floor((u + rad) / kTile), static_cast<double>(cam.tiles_x - 1));

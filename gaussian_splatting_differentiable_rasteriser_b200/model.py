@@ -78,10 +78,13 @@ class TrainStep:
     """Buffers and the call sequence of one iteration for images up to width x height."""
 
     def __init__(self, model: GaussianModel, max_entries: int, width: int, height: int, lrs=None,
-                 lam=0.2, betas=(0.9, 0.999), eps=1e-8, device="cuda", fused_adam=True):
+                 lam=0.2, betas=(0.9, 0.999), eps=1e-8, device="cuda", fused_adam=True,
+                 opacity_rect=False):
         self.model = model
         self.fused_adam = fused_adam
         self.ctx = native.Context(model.n_pad, max_entries, width, height)
+        if opacity_rect:
+            self.ctx.set_option(native.GS_OPTION_OPACITY_RECT, 1)
         self.lrs = dict(DEFAULT_LR if lrs is None else lrs)
         self.lam, self.betas, self.eps = lam, betas, eps
         self.image = torch.empty((3, height, width), dtype=torch.float32, device=device)

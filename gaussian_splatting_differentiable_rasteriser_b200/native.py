@@ -24,7 +24,8 @@ EXPORTED = ("gs_create", "gs_destroy", "gs_last_error", "gs_preprocess", "gs_ren
             "gs_loss_l1_dssim", "gs_render_backward", "gs_render_backward_adam", "gs_adam_step",
             "gs_profile_enable",
             "gs_profile_read", "gs_stage_name", "gs_debug_preprocess", "gs_debug_sorted",
-            "gs_debug_screen_grads")
+            "gs_debug_screen_grads", "gs_set_option", "gs_loss_l1_dssim_noalloc")
+GS_OPTION_OPACITY_RECT = 1
 STAGES = ("preprocess", "scan", "duplicate", "sort", "ranges", "blend_forward", "loss",
           "blend_backward", "preprocess_backward", "backward_adam", "depth_sort")
 GROUPS = ("means", "log_scales", "quats", "opacity_logits", "sh")
@@ -84,6 +85,8 @@ def load(path: str = LIB_PATH):
                                           ctypes.POINTER(GsGrads), ctypes.POINTER(GsGrads),
                                           ctypes.POINTER(GsGrads), ctypes.POINTER(F), F, F, F, I32, P]
     L.gs_adam_step.argtypes = [P, P, P, P, I64, F, F, F, F, I32, P]
+    L.gs_set_option.argtypes = [P, I32, I32]
+    L.gs_set_option.restype = ctypes.c_int
     L.gs_loss_l1_dssim_noalloc.argtypes = [P, P, I32, I32, F, P, P, P]
     L.gs_loss_l1_dssim_noalloc.restype = ctypes.c_int
     L.gs_profile_enable.argtypes = [P, I32]
@@ -150,6 +153,9 @@ class Context:
     def _check(self, st):
         if st != GS_OK:
             raise GsError(st, self.L.gs_last_error(self.h).decode())
+
+    def set_option(self, option, value):
+        self._check(self.L.gs_set_option(self.h, int(option), int(value)))
 
     def preprocess(self, params: GsParams, cam: GsCamera, stream=None):
         self._check(self.L.gs_preprocess(self.h, ctypes.byref(params), ctypes.byref(cam), _stream(stream)))

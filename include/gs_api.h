@@ -100,6 +100,23 @@ void gs_destroy(gs_ctx *ctx);
  * The string is owned by the context. */
 const char *gs_last_error(const gs_ctx *ctx);
 
+/* Context options. */
+typedef enum {
+  /* Value 1: each Gaussian's tile rect uses the opacity-aware radius of [GS]
+   * section "Why tiling, and the five stages" (the code after the list):
+   * r = sqrt(2 E) sqrt(lambda_max) with E = min(4.5, ln(max(255 o, 1.0001))),
+   * alpha_min = 1/255 and no compensation factor, instead of 3 sqrt(lambda_max).
+   * Alpha stays below 1/255 in every tile it drops, so the image and
+   * gradients do not change; the (Gaussian, tile) lists get shorter. Value 0
+   * (the default): the 3-sigma rect. */
+  GS_OPTION_OPACITY_RECT = 1
+} gs_option;
+
+/* Sets a context option; it applies from the next gs_preprocess (the state
+ * of the camera in flight is discarded). Errors: GS_ERR_INVALID_ARG for an
+ * unknown option or value. */
+gs_status gs_set_option(gs_ctx *ctx, int32_t option, int32_t value);
+
 /* Step 1 - preprocess, one thread per Gaussian ([SN] slides on the
  * parametrisation and "J is the 2 x 3 Jacobian of perspective projection";
  * [GS] sections "Flattening a 3D blob into a 2D oval (EWA projection)" and

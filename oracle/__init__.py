@@ -50,6 +50,8 @@ def lib():
         L.or_backward_rows.argtypes = [P, ctypes.c_int32, ctypes.c_int32] + [P] * 7
         L.or_backward.argtypes = [P] * 8
         L.or_blend_backward_rows.argtypes = [P, ctypes.c_int32, ctypes.c_int32, P, P]
+        L.or_set_option.argtypes = [P, ctypes.c_int32, ctypes.c_int32]
+        L.or_set_option.restype = ctypes.c_int
         L.or_project_backward.argtypes = [P, P, ctypes.c_int64, ctypes.c_int64] + [P] * 5
         L.or_loss.argtypes = [ctypes.c_int32, ctypes.c_int32, P, P, ctypes.c_double, P, P]
         L.or_loss.restype = ctypes.c_int
@@ -87,11 +89,13 @@ class Oracle:
     """One scene seen by one camera: preprocess and tile lists are built on
     construction; render/backward walk the lists per pixel."""
 
-    def __init__(self, scene, cam, active_degree=None):
+    def __init__(self, scene, cam, active_degree=None, opacity_rect=False):
         self.L = lib()
         self.scene = scene
         self.cam = cam
         self.h = self.L.or_create()
+        if opacity_rect:
+            self.L.or_set_option(self.h, 1, 1)
         self.active_degree = scene.sh_degree if active_degree is None else active_degree
         f64 = np.asarray(scene.means).dtype == np.float64
         dt = np.float64 if f64 else np.float32

@@ -312,9 +312,17 @@ void covariance3d(const S ls[3], const S q[4], S Sigma[9]) {
 // One Gaussian through the preprocess. Returns false if it is culled (behind
 // the near plane, degenerate screen covariance, or a tile rect that misses the
 // image), in which case it touches no tile.
+//
+// With opacity_rect the tile rect uses the opacity-aware radius of "How a
+// computer rebuilds a real place ... Gaussian Splats", section "Why tiling,
+// and the five stages" (the code after the five stages): the falloff cut is
+// E = min(4.5, ln(max(o / alpha_min, 1.0001))) with alpha_min = 1/255 and no
+// compensation factor, and r = sqrt(2 E) sqrt(lambda_max). Beyond r along
+// the long axis o exp(-e) < 1/255, so the tiles it drops hold no contribution.
 template <class S>
 bool project(const or_camera& cam, const S p[3], const S ls[3], const S q[4], const S& logit,
-             const double* sh, int64_t sh_stride, int active_degree, Proj<S>& P, Aux& X) {
+             const double* sh, int64_t sh_stride, int active_degree, Proj<S>& P, Aux& X,
+             bool opacity_rect = false) {
   X = Aux();
   const double* R = cam.R;
   // p_c = R p + t, each row summed left to right.
@@ -365,6 +373,11 @@ bool project(const or_camera& cam, const S p[3], const S ls[3], const S q[4], co
   double dt = val(det);
   X.lmax = mid + std::sqrt(std::max(mid * mid - dt, 0.0));
   X.radius = kRadiusSigmas * std::sqrt(X.lmax);
+  if (opacity_rect) {
+    const double o = 1.0 / (1.0 + std::exp(-val(logit)));
+    const double e_cut = std::min(4.5, std::log(std::max(o * 255.0, 1.0001)));
+    X.radius = std::sqrt(2.0 * e_cut) * std::sqrt(X.lmax);
+  }
   // Tiles whose pixel square [16 tx, 16 tx + 15] meets [u - r, u + r].
   double u = val(P.u), v = val(P.v), r = X.radius;
   int tx0 = static_cast<int>(std::ceil((u - r - (kTile - 1)) / kTile));
@@ -447,6 +460,7 @@ struct Ctx {
   std::vector<Aux> aux;
   std::vector<Entry> entries;            // sorted
   std::vector<int64_t> range_lo, range_hi;  // per tile, [lo, hi)
+  bool opacity_rect = false;             // opacity-aware tile rect (see project)
 };
 
 // Margins used to flag float32/float64 threshold ambiguity.
@@ -530,7 +544,8 @@ void run_preprocess_and_sort(Ctx& c) {
     double q[4] = {c.quats[i], c.quats[np + i], c.quats[2 * np + i], c.quats[3 * np + i]};
     Proj<double> P;
     Aux& X = c.aux[i];
-    bool ok = project<double>(c.cam, p, ls, q, c.logits[i], &c.sh[i], np, c.active_degree, P, X);
+    bool ok = project<double>(c.cam, p, ls, q, c.logits[i], &c.sh[i], np, c.active_degree, P, X,
+                              c.opacity_rect);
     if (!ok) {
       X.touched = 0;
       continue;
@@ -583,6 +598,17 @@ extern "C" {
 
 void* or_create() { return new Ctx(); }
 void or_destroy(void* h) { delete static_cast<Ctx*>(h); }
+
+// Options, set before or_set_scene: 1 = opacity-aware tile rect (value 0/1).
+// Returns 0, or 1 for an unknown option.
+int or_set_option(void* h, int32_t option, int32_t value) {
+  Ctx& c = *static_cast<Ctx*>(h);
+  if (option == 1) {
+    c.opacity_rect = value != 0;
+    return 0;
+  }
+  return 1;
+}
 
 // Loads the parameters (planar float32, see the scene layout) and the camera,
 // then runs the preprocess and builds the sorted tile lists.
@@ -772,7 +798,7 @@ void or_project_backward(void* h, const double* screen_grad, int64_t i0, int64_t
     D logit = seed<11>(c.logits[i], 10);
     Proj<D> P;
     Aux X;
-    project<D>(c.cam, p, ls, q, logit, &c.sh[i], np, c.active_degree, P, X);
+    project<D>(c.cam, p, ls, q, logit, &c.sh[i], np, c.active_degree, P, X, c.opacity_rect);
     const D* outs[kScreen] = {&P.u, &P.v, &P.A, &P.B, &P.C, &P.o, &P.rgb[0], &P.rgb[1], &P.rgb[2]};
     double gp[11] = {0};
     for (int o = 0; o < kScreen; ++o)

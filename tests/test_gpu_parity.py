@@ -42,15 +42,17 @@ def host(t):
 class GpuRun:
     """Preprocess + forward of one scene/camera through the C ABI."""
 
-    def __init__(self, native, model, scene, cam, max_entries=None, active_degree=None):
+    def __init__(self, native, model, scene, cam, max_entries=None, active_degree=None, opacity_rect=False):
         self.native = native
         self.m = model.GaussianModel(scene, active_degree=active_degree)
         self.cam = cam
         self.cs = native.camera_struct(cam)
-        o = oracle.Oracle(scene, cam, active_degree)
+        o = oracle.Oracle(scene, cam, active_degree, opacity_rect=opacity_rect)
         self.oracle = o
         K_or = oracle.lib().or_num_entries(o.h)
         self.ctx = native.Context(scene.n_pad, max_entries or max(16, 2 * K_or + 16), cam.width, cam.height)
+        if opacity_rect:
+            self.ctx.set_option(native.GS_OPTION_OPACITY_RECT, 1)
         H, W = cam.height, cam.width
         self.image = torch.empty((3, H, W), device="cuda")
         self.T = torch.empty((H, W), device="cuda")
@@ -398,3 +400,45 @@ def test_fused_backward_adam_adds_an_accumulated_gradient(gs):
         assert rel_l2(host(b.m[k]), host(a.m[k])) < 1e-4, k
         dp = np.abs(host(a.params[k]) - host(b.params[k]))
         assert np.mean(dp <= 1e-6) > 0.999, k
+
+
+@pytest.mark.parametrize("name", ["tiny", "small"])
+def test_opacity_aware_rect_path_matches_oracle(gs, name):
+    """With the opacity-aware tile rect: rects and the sort bit-exact, pixels
+    and gradients within tolerance, against the oracle run with the same rect;
+    fewer entries than the 3-sigma rect."""
+    native, model = gs
+    s, ci = SCENES[name]()
+    cam = s.cameras[ci]
+    run = GpuRun(native, model, s, cam, opacity_rect=True)
+    g = run.preprocess_out()
+    o = run.oracle.preprocess()
+    np.testing.assert_array_equal(g["touched"], o["touched"])
+    vis = o["touched"] > 0
+    np.testing.assert_array_equal(g["rect"][vis], o["rect"][vis])
+    ids, tiles, ranges = run.sorted_out()
+    srt = run.oracle.sorted()
+    np.testing.assert_array_equal(ids, srt["ids"])
+    np.testing.assert_array_equal(tiles, srt["tiles"])
+    np.testing.assert_array_equal(ranges.astype(np.int64), srt["ranges"])
+    assert run.K < GpuRun(native, model, s, cam).K
+    r = run.oracle.render()
+    check_pixels(run, r)
+    target = scenes.uniform_image(cam.height, cam.width, seed=7)
+    _, _, _, dimg = oracle.loss(r["image"].astype(np.float32), target, 0.2)
+    dimg32 = dimg.astype(np.float32)
+    ref = run.oracle.backward(dimg32.astype(np.float64))
+    grads, sg = run.backward(dimg32)
+    assert rel_l2(sg[vis], ref["screen"][vis]) < GRAD_RL2
+    for k in scenes.GROUP_NAMES:
+        e = rel_l2(grads[k][..., :s.n], ref[k][..., :s.n])
+        assert e < GRAD_RL2, (k, e)
+
+
+def test_set_option_rejects_unknown_options(gs):
+    native, _ = gs
+    ctx = native.Context(16, 16, 16, 16)
+    with pytest.raises(native.GsError):
+        ctx.set_option(99, 1)
+    with pytest.raises(native.GsError):
+        ctx.set_option(native.GS_OPTION_OPACITY_RECT, 2)

@@ -164,3 +164,42 @@ def test_split_backward_equals_whole_backward():
     for k, v in parts.items():
         idx = (Ellipsis, slice(0, s.n))
         np.testing.assert_allclose(v[idx], whole[k][idx], rtol=1e-12, atol=1e-15, err_msg=k)
+
+
+def test_opacity_aware_rect_drops_only_tiles_without_contribution():
+    """The opacity-aware tile rect (falloff cut min(4.5, ln(255 o)) instead of
+    4.5) keeps a subset of the 3-sigma rect, drops only tiles in which the
+    Gaussian's alpha stays below 1/255 at every pixel (checked by brute force),
+    and leaves the rendered image and transmittance unchanged."""
+    s = scenes.small()
+    cam = s.cameras[0]
+    o3 = oracle.Oracle(s, cam)
+    oa = oracle.Oracle(s, cam, opacity_rect=True)
+    p3, pa = o3.preprocess(), oa.preprocess()
+    assert pa["touched"].sum() < p3["touched"].sum()
+    vis = pa["touched"] > 0
+    assert np.all(p3["touched"][vis] > 0)
+    r3, ra = p3["rect"], pa["rect"]  # x0, y0, x1, y1
+    assert np.all(ra[vis, 0] >= r3[vis, 0]) and np.all(ra[vis, 1] >= r3[vis, 1])
+    assert np.all(ra[vis, 2] <= r3[vis, 2]) and np.all(ra[vis, 3] <= r3[vis, 3])
+    # every pixel of a dropped tile is below the alpha floor
+    changed = np.nonzero(p3["touched"] != pa["touched"])[0]
+    assert changed.size > 100
+    tx_n, ty_n = o3.tiles
+    for i in changed[:400]:
+        u, v, A, B, C, o = p3["screen"][i, :6]
+        x0, y0, x1, y1 = r3[i]
+        keep = np.zeros((ty_n, tx_n), bool)
+        if pa["touched"][i] > 0:
+            keep[ra[i, 1]:ra[i, 3] + 1, ra[i, 0]:ra[i, 2] + 1] = True
+        for ty in range(y0, y1 + 1):
+            for tx in range(x0, x1 + 1):
+                if keep[ty, tx]:
+                    continue
+                ys, xs = np.mgrid[16 * ty:16 * ty + 16, 16 * tx:16 * tx + 16]
+                dx, dy = xs - u, ys - v
+                alpha = o * np.exp(-(0.5 * A * dx * dx + B * dx * dy + 0.5 * C * dy * dy))
+                assert alpha.max() < 1.0 / 255.0, (i, tx, ty, alpha.max())
+    i3, ia = o3.render(), oa.render()
+    np.testing.assert_allclose(ia["image"], i3["image"], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(ia["final_T"], i3["final_T"], rtol=0, atol=1e-12)
