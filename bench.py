@@ -165,7 +165,7 @@ def max_over_ranks(x, world):
 
 
 # ------------------------------------------------------------------ workload
-def build_workload(config, device, opacity_rect=False):
+def build_workload(config, device, opacity_rect=False, deterministic=False):
     import numpy as np
     import torch
 
@@ -178,7 +178,8 @@ def build_workload(config, device, opacity_rect=False):
     H = max(c.height for c in cams)
     m = model.GaussianModel(pert, device=device)
     cap = max(1 << 20, 8 * scene.n)
-    step = model.TrainStep(m, cap, W, H, device=device, opacity_rect=opacity_rect)
+    step = model.TrainStep(m, cap, W, H, device=device, opacity_rect=opacity_rect,
+                           deterministic=deterministic)
     # targets: renders of the perturbed copy (forward only, before any timing)
     targets = torch.empty((len(cams), 3, H, W), dtype=torch.float32, device=device)
     kmax = 0
@@ -428,7 +429,8 @@ def main_ours(args):
 
     native.load()
     device = f"cuda:{local}"
-    scene, m, step, targets, kmax = build_workload(args.config, device, args.rect == "opacity")
+    scene, m, step, targets, kmax = build_workload(args.config, device, args.rect == "opacity",
+                                                   args.deterministic)
     cams = scene.cameras
     sched = scenes.camera_schedule(len(cams), args.warmup + args.steps, seed=rank)
     # clocks are sampled from the start of the warm-up to the end of the timed region
@@ -485,6 +487,7 @@ def main_ours(args):
                        "width": W, "height": H, "cameras": len(cams),
                        "parallelism": "replicas" if world > 1 else "single-gpu",
                        "tile_rect": "3 sigma" if args.rect == "3sigma" else "opacity-aware",
+                       "gradient_sums": "fixed-point (deterministic)" if args.deterministic else "float32 atomics",
                        "l2": "inputs larger than L2: 2.8 GB of parameter/gradient/moment state "
                              "streamed every step" if args.config == "dense" else "see workload",
                        "entries_per_step": int(statistics.mean(ks)) if ks else None},
@@ -610,6 +613,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--rect", choices=("3sigma", "opacity"), default="3sigma",
                     help="tile rect: the 3-sigma radius, or the opacity-aware one (same image, fewer entries)")
+    ap.add_argument("--deterministic", action="store_true",
+                    help="fixed-point gradient atomics (bitwise-reproducible backward)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

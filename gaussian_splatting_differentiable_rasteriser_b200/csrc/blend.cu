@@ -217,8 +217,21 @@ struct WarpBatch {
 // the offsets from the Gaussian's centre, dx = lx - a, dy = ly - b with
 // (a, b) = centre - block centre:
 //   sum w dx = Mx - a M0, sum w dx^2 = Mxx - 2a Mx + a^2 M0, and so on.
+// Adds v to raw sum r of a Gaussian: a float32 atomic, or, in deterministic
+// mode, an integer atomic of v in 2^-40 fixed point (integer sums do not
+// depend on the order the warps arrive in, so the result is bitwise
+// reproducible; |v| is clamped to 2^22, far above any screen-gradient sum).
+__device__ __forceinline__ void add_sum(float* dst, unsigned long long* fdst, int r, float v) {
+  if (fdst) {
+    const double q = fmin(fmax(static_cast<double>(v) * kFixedScale, -kFixedClamp), kFixedClamp);
+    atomicAdd(fdst + r, static_cast<unsigned long long>(__double2ll_rn(q)));
+  } else {
+    atomicAdd(dst + r, v);
+  }
+}
+
 __device__ __forceinline__ void flush_batch(const WarpBatch& b, int cnt, int lane, float cxb, float cyb,
-                                            float* sgrad) {
+                                            float* sgrad, unsigned long long* sgrad_fixed) {
   const int j = lane & 15, h = lane >> 4;
   float m0 = 0.f, mx = 0.f, my = 0.f, mxx = 0.f, mxy = 0.f, myy = 0.f;
   float c0 = 0.f, c1 = 0.f, c2 = 0.f;
@@ -261,18 +274,19 @@ __device__ __forceinline__ void flush_batch(const WarpBatch& b, int cnt, int lan
     const float2 uv = b.uv[j];
     const float a = uv.x - cxb, bb = uv.y - cyb;
     float* dst = sgrad + static_cast<int64_t>(b.id[j]) * kGradStride;
+    unsigned long long* fdst = sgrad_fixed ? sgrad_fixed + static_cast<int64_t>(b.id[j]) * kFixedStride : nullptr;
     if (h == 0) {
       const float sy = __fmaf_rn(-bb, m0, my);
-      atomicAdd(dst + 0, m0);
-      atomicAdd(dst + 1, __fmaf_rn(-a, m0, mx));
-      atomicAdd(dst + 2, sy);
-      atomicAdd(dst + 3, __fmaf_rn(a, __fmaf_rn(a, m0, -2.0f * mx), mxx));
-      atomicAdd(dst + 4, __fmaf_rn(-a, sy, __fmaf_rn(-bb, mx, mxy)));
+      add_sum(dst, fdst, 0, m0);
+      add_sum(dst, fdst, 1, __fmaf_rn(-a, m0, mx));
+      add_sum(dst, fdst, 2, sy);
+      add_sum(dst, fdst, 3, __fmaf_rn(a, __fmaf_rn(a, m0, -2.0f * mx), mxx));
+      add_sum(dst, fdst, 4, __fmaf_rn(-a, sy, __fmaf_rn(-bb, mx, mxy)));
     } else {
-      atomicAdd(dst + 5, __fmaf_rn(bb, __fmaf_rn(bb, m0, -2.0f * my), myy));
-      atomicAdd(dst + 6, c0);
-      atomicAdd(dst + 7, c1);
-      atomicAdd(dst + 8, c2);
+      add_sum(dst, fdst, 5, __fmaf_rn(bb, __fmaf_rn(bb, m0, -2.0f * my), myy));
+      add_sum(dst, fdst, 6, c0);
+      add_sum(dst, fdst, 7, c1);
+      add_sum(dst, fdst, 8, c2);
     }
   }
 }
@@ -377,14 +391,14 @@ __global__ void __launch_bounds__(256) blend_backward_kernel(BlendArgs a) {
       }
       if (++bcnt == kBatch) {
         __syncwarp();
-        flush_batch(wb, kBatch, lane, bx0 + 3.5f, by0 + 1.5f, a.sgrad);
+        flush_batch(wb, kBatch, lane, bx0 + 3.5f, by0 + 1.5f, a.sgrad, a.sgrad_fixed);
         bcnt = 0;
         __syncwarp();
       }
     }
     __syncwarp();  // the slots are rewritten by the next chunk
   }
-  if (bcnt > 0) flush_batch(wb, bcnt, lane, bx0 + 3.5f, by0 + 1.5f, a.sgrad);
+  if (bcnt > 0) flush_batch(wb, bcnt, lane, bx0 + 3.5f, by0 + 1.5f, a.sgrad, a.sgrad_fixed);
   if (kCount) {
     // the method's backward walk visits every entry before the pixel's last contributor
     count_pairs(a.pairs, static_cast<unsigned>(min(last, static_cast<int>(range.y - range.x))));
@@ -392,7 +406,26 @@ __global__ void __launch_bounds__(256) blend_backward_kernel(BlendArgs a) {
   }
 }
 
+// Deterministic mode: the fixed-point sums back to float32 raw sums.
+__global__ void decode_fixed_kernel(const unsigned long long* fixed, int64_t n, float* sgrad) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const unsigned long long* f = fixed + i * kFixedStride;
+  float* o = sgrad + i * kGradStride;
+#pragma unroll
+  for (int r = 0; r < 9; ++r)
+    o[r] = static_cast<float>(static_cast<double>(static_cast<long long>(f[r])) / kFixedScale);
+#pragma unroll
+  for (int r = 9; r < kGradStride; ++r) o[r] = 0.0f;
+}
+
 }  // namespace
+
+cudaError_t launch_decode_fixed(const unsigned long long* fixed, int64_t n, float* sgrad, cudaStream_t st) {
+  if (n == 0) return cudaSuccess;
+  decode_fixed_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(fixed, n, sgrad);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_blend_forward(const BlendArgs& a, cudaStream_t st) {
   const int tiles = a.cam.tiles_x * a.cam.tiles_y;

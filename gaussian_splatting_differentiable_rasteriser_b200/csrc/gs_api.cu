@@ -55,6 +55,8 @@ struct gs_ctx {
   int sorted_buf = 0;
   // options (gs_set_option)
   int opacity_rect = 0;
+  unsigned long long* sgrad_fixed = nullptr;  // [max_g][9], allocated by GS_OPTION_DETERMINISTIC
+  int deterministic = 0;
   // profiling (off by default)
   struct Profiler {
     static constexpr int kMaxRec = 128;
@@ -94,7 +96,7 @@ void free_all(gs_ctx* c) {
                   c->visible_prefix, c->depth_range, c->dkeys[0], c->dkeys[1], c->dvals[0],
                   c->dvals[1], c->dup_status, c->keys[0], c->keys[1], c->vals[0], c->vals[1],
                   c->hist, c->offsets, c->status, c->counters, c->ranges, c->surv, c->surv_count,
-                  c->loss_partials,
+                  c->sgrad_fixed, c->loss_partials,
                   c->loss_counter, c->info_dev, c->pairs};
   for (void* b : bufs)
     if (b) cudaFree(b);
@@ -312,6 +314,13 @@ gs_status gs_set_option(gs_ctx* c, int32_t option, int32_t value) {
       if (value != 0 && value != 1) return fail(c, GS_ERR_INVALID_ARG, "option value must be 0 or 1");
       c->opacity_rect = value;
       c->have_pre = c->have_fwd = false;  // the tile lists depend on it
+      return GS_OK;
+    case GS_OPTION_DETERMINISTIC:
+      if (value != 0 && value != 1) return fail(c, GS_ERR_INVALID_ARG, "option value must be 0 or 1");
+      if (value && !c->sgrad_fixed)
+        GS_CUDA(c, cudaMalloc(reinterpret_cast<void**>(&c->sgrad_fixed),
+                              sizeof(unsigned long long) * gs::kFixedStride * c->max_g));
+      c->deterministic = value;
       return GS_OK;
     default:
       return fail(c, GS_ERR_INVALID_ARG, "unknown option %d", option);
@@ -535,8 +544,12 @@ gs_status backward_common(gs_ctx* c, const gs_params* p, const gs_camera* cam, c
     for (float* q : gp)
       if (!q || !aligned(q, 4)) return fail(c, GS_ERR_INVALID_ARG, "a gradient pointer is NULL or misaligned");
   }
-  if (p->n > 0)
-    GS_CUDA(c, cudaMemsetAsync(c->sgrad, 0, sizeof(float) * gs::kGradStride * p->n, st));
+  if (p->n > 0) {
+    if (c->deterministic)
+      GS_CUDA(c, cudaMemsetAsync(c->sgrad_fixed, 0, sizeof(unsigned long long) * gs::kFixedStride * p->n, st));
+    else
+      GS_CUDA(c, cudaMemsetAsync(c->sgrad, 0, sizeof(float) * gs::kGradStride * p->n, st));
+  }
   gs::BlendArgs ba{};
   ba.ranges = c->ranges;
   ba.order = c->vals[c->sorted_buf];
@@ -549,9 +562,11 @@ gs_status backward_common(gs_ctx* c, const gs_params* p, const gs_camera* cam, c
   ba.pairs = c->prof.on ? c->pairs + 4 : nullptr;
   ba.surv = c->surv;
   ba.surv_count = c->surv_count;
+  ba.sgrad_fixed = c->deterministic ? c->sgrad_fixed : nullptr;
   prof_begin(c, st);
   GS_CUDA(c, gs::launch_blend_backward(ba, st));
-  prof_end(c, GS_STAGE_BLEND_BACKWARD, 0, st);
+  if (c->deterministic) GS_CUDA(c, gs::launch_decode_fixed(c->sgrad_fixed, p->n, c->sgrad, st));
+  prof_end(c, GS_STAGE_BLEND_BACKWARD, 0, st, 1 + (c->deterministic && p->n > 0 ? 1 : 0));
   a.means = p->means;
   a.log_scales = p->log_scales;
   a.quats = p->quats;

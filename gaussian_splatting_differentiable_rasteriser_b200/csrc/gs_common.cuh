@@ -45,6 +45,12 @@ __device__ __forceinline__ float screen_opacity(const Screen& s) { return s.c.y;
 // The projection backward turns them into dL/d(mean2d, conic, opacity).
 constexpr int kGradStride = 12;
 
+// Deterministic mode keeps the 9 raw sums as 64-bit integers in 2^-40 fixed
+// point, kFixedStride per Gaussian.
+constexpr int kFixedStride = 9;
+constexpr double kFixedScale = 1099511627776.0;      // 2^40
+constexpr double kFixedClamp = 4611686018427387904.0;  // 2^62
+
 // Camera in the form the kernels take it (by value).
 struct CamArgs {
   int width, height, tiles_x, tiles_y;

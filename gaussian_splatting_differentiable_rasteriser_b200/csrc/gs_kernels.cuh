@@ -128,10 +128,13 @@ struct BlendArgs {
   // order, warp w of a tile with list [beg, end) at surv[8 beg + w (end - beg)]
   uint2* surv;
   uint32_t* surv_count;  // [tiles][8]
+  // backward in deterministic mode: the raw sums in fixed point ([n][9], zeroed)
+  unsigned long long* sgrad_fixed;
 };
 
 cudaError_t launch_blend_forward(const BlendArgs& a, cudaStream_t st);
 cudaError_t launch_blend_backward(const BlendArgs& a, cudaStream_t st);
+cudaError_t launch_decode_fixed(const unsigned long long* fixed, int64_t n, float* sgrad, cudaStream_t st);
 
 // ---------------------------------------------------------------- loss
 struct LossArgs {

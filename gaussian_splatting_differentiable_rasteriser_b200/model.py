@@ -79,12 +79,14 @@ class TrainStep:
 
     def __init__(self, model: GaussianModel, max_entries: int, width: int, height: int, lrs=None,
                  lam=0.2, betas=(0.9, 0.999), eps=1e-8, device="cuda", fused_adam=True,
-                 opacity_rect=False):
+                 opacity_rect=False, deterministic=False):
         self.model = model
         self.fused_adam = fused_adam
         self.ctx = native.Context(model.n_pad, max_entries, width, height)
         if opacity_rect:
             self.ctx.set_option(native.GS_OPTION_OPACITY_RECT, 1)
+        if deterministic:
+            self.ctx.set_option(native.GS_OPTION_DETERMINISTIC, 1)
         self.lrs = dict(DEFAULT_LR if lrs is None else lrs)
         self.lam, self.betas, self.eps = lam, betas, eps
         self.image = torch.empty((3, height, width), dtype=torch.float32, device=device)

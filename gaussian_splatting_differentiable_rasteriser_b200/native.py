@@ -26,6 +26,7 @@ EXPORTED = ("gs_create", "gs_destroy", "gs_last_error", "gs_preprocess", "gs_ren
             "gs_profile_read", "gs_stage_name", "gs_debug_preprocess", "gs_debug_sorted",
             "gs_debug_screen_grads", "gs_set_option", "gs_loss_l1_dssim_noalloc")
 GS_OPTION_OPACITY_RECT = 1
+GS_OPTION_DETERMINISTIC = 2
 STAGES = ("preprocess", "scan", "duplicate", "sort", "ranges", "blend_forward", "loss",
           "blend_backward", "preprocess_backward", "backward_adam", "depth_sort")
 GROUPS = ("means", "log_scales", "quats", "opacity_logits", "sh")

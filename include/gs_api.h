@@ -109,7 +109,18 @@ typedef enum {
    * Alpha stays below 1/255 in every tile it drops, so the image and
    * gradients do not change; the (Gaussian, tile) lists get shorter. Value 0
    * (the default): the 3-sigma rect. */
-  GS_OPTION_OPACITY_RECT = 1
+  GS_OPTION_OPACITY_RECT = 1,
+  /* Value 1: the backward accumulates each Gaussian's screen-space gradient
+   * sums as 64-bit integers in 2^-40 fixed point instead of float32 atomics
+   * (the integer-atomic idea of [GS] section "Making the parallel sums exact:
+   * fixed-point, and the conic trick", with a 64-bit word and a finer scale
+   * instead of 32 bits x 16384, because mean-reduced losses give per-pixel
+   * gradients near 1e-7). Integer sums do not depend on the order of the
+   * additions, so gs_render_backward and gs_render_backward_adam are then
+   * bitwise reproducible. Enabling it allocates 72 B per Gaussian of the
+   * context (GS_ERR_CUDA if that fails). Value 0 (the default): float32
+   * atomics. */
+  GS_OPTION_DETERMINISTIC = 2
 } gs_option;
 
 /* Sets a context option; it applies from the next gs_preprocess (the state
@@ -181,7 +192,7 @@ gs_status gs_loss_l1_dssim(gs_ctx *ctx, const float *image_chw, const float *tar
  * the last gs_preprocess, and final_T / n_contrib the outputs of the last
  * gs_render_forward. Errors: GS_ERR_INVALID_ARG if the forward has not run
  * or the inputs do not match it. Gradients are not bitwise reproducible
- * (float32 atomics). */
+ * (float32 atomics) unless GS_OPTION_DETERMINISTIC is set. */
 gs_status gs_render_backward(gs_ctx *ctx, const gs_params *params, const gs_camera *cam,
                              const float *final_T, const int32_t *n_contrib,
                              const float *dloss_dimage, gs_grads *grads, void *stream);

@@ -442,3 +442,44 @@ def test_set_option_rejects_unknown_options(gs):
         ctx.set_option(99, 1)
     with pytest.raises(native.GsError):
         ctx.set_option(native.GS_OPTION_OPACITY_RECT, 2)
+
+
+def test_deterministic_backward_is_bitwise_reproducible_and_matches_oracle(gs):
+    """With GS_OPTION_DETERMINISTIC the screen-gradient sums are integer
+    (fixed-point) atomics: two independent runs give the same bits, for the
+    backward and for two fused training steps, and the gradients still match
+    the oracle."""
+    native, model = gs
+    s = scenes.small()
+    cam = s.cameras[0]
+    target = scenes.uniform_image(cam.height, cam.width, seed=7)
+    outs = []
+    for _ in range(2):
+        run = GpuRun(native, model, s, cam)
+        run.ctx.set_option(native.GS_OPTION_DETERMINISTIC, 1)
+        run.ctx.preprocess(run.m.params_struct(), run.cs)
+        run.K = run.ctx.render_forward(run.cs, run.image, run.T, run.nc)
+        r = run.oracle.render()
+        _, _, _, dimg = oracle.loss(r["image"].astype(np.float32), target, 0.2)
+        grads, sg = run.backward(dimg.astype(np.float32))
+        outs.append((grads, sg, run))
+    (g1, sg1, run), (g2, sg2, _) = outs
+    np.testing.assert_array_equal(sg1.view(np.uint32), sg2.view(np.uint32))
+    for k in scenes.GROUP_NAMES:
+        np.testing.assert_array_equal(g1[k].view(np.uint32), g2[k].view(np.uint32))
+    ref = run.oracle.backward(dimg.astype(np.float32).astype(np.float64))
+    vis = run.oracle.preprocess()["touched"] > 0
+    assert rel_l2(sg1[vis], ref["screen"][vis]) < GRAD_RL2
+    for k in scenes.GROUP_NAMES:
+        assert rel_l2(g1[k][..., :s.n], ref[k][..., :s.n]) < GRAD_RL2, k
+    # two fused training steps, twice from the same start
+    tgt = dev(target)
+    params = []
+    for _ in range(2):
+        m = model.GaussianModel(s)
+        st = model.TrainStep(m, 200_000, cam.width, cam.height, deterministic=True)
+        for _ in range(2):
+            st(cam, tgt)
+        torch.cuda.synchronize()
+        params.append(host(m.flat).view(np.uint32).copy())
+    np.testing.assert_array_equal(params[0], params[1])
