@@ -309,6 +309,61 @@ gs_status gs_debug_sorted(gs_ctx *ctx, int32_t *ids, int32_t *tiles, int32_t *ra
  * dL/d(mean2d x, mean2d y, A, B, C, opacity, r, g, b). */
 gs_status gs_debug_screen_grads(gs_ctx *ctx, float *out, void *stream);
 
+/* ------------------------------------------------------ density control --
+ * Adaptive density control, run between training steps ([SN] slides "Where
+ * to add capacity" and "A separate heuristic": the screen-space centre
+ * gradient magnitude averaged over the views that saw a Gaussian flags
+ * regions to densify; small flagged Gaussians are cloned, large ones split;
+ * very low opacity prunes; opacity reset clamps opacity to at most 0.01;
+ * [GS] "Densification": split halves shrink by 1.6 and restart their Adam
+ * moments). The thresholds are the caller's settings, as the pages say. */
+
+/* Registers two DEVICE buffers of max_gaussians entries that every later
+ * gs_render_backward / gs_render_backward_adam on this context accumulates
+ * into: grad_accum[i] += |dL/dmean2d_i| (Euclidean norm, pixels) and
+ * view_count[i] += 1 for every Gaussian the view touched (tiles_touched > 0).
+ * The caller zeroes them when it starts a statistics window. Pass NULL for
+ * both to stop accumulating. Errors: GS_ERR_INVALID_ARG if exactly one is
+ * NULL. */
+gs_status gs_set_densify_stats(gs_ctx *ctx, float *grad_accum, uint32_t *view_count);
+
+/* One densification pass from the set `in` (n Gaussians, planar with
+ * in->n_pad) to the set `out` (planar with stride out_n_pad, written through
+ * the float pointers of a gs_grads), moments m/v alongside. For Gaussian i,
+ * with avg = grad_accum[i] / view_count[i] (float64), s_max = the largest
+ * log-scale and o = sigmoid(logit):
+ *   prune  if logit < logit(min_opacity)                 -> not written;
+ *   else if view_count[i] > 0 and avg >= grad_threshold:
+ *     clone if s_max <= log(scale_threshold)            -> i kept + one copy,
+ *     split otherwise                                   -> i replaced by two
+ *       children: mean + R(q/|q|) diag(exp(log-scales)) z_k with the caller's
+ *       N(0, 1) draws z_k = normals[i][k][0..2] (k = 0, 1), log-scales
+ *       - ln(1.6), the other parameters copied;
+ *   else kept.
+ * Output order: the kept Gaussians (cloned parents included) in index order,
+ * then the clones in parent order, then the split children (child 0, child 1)
+ * in parent order. Kept Gaussians keep their moments; clones and children
+ * start at zero. *n_out (HOST) receives the new count; entries beyond it are
+ * not written. The comparisons are taken in float64 against thresholds
+ * converted once on the host, so they are exact. This call synchronises
+ * `stream` once (to read the count). Errors: GS_ERR_INVALID_ARG for bad
+ * pointers, n > the context's max_gaussians, a non-positive threshold or
+ * min_opacity outside (0, 1); GS_ERR_CAPACITY (nothing written) if the new
+ * count exceeds out_n_pad. */
+gs_status gs_densify(gs_ctx *ctx, const gs_params *in, const gs_grads *m_in, const gs_grads *v_in,
+                     const float *grad_accum, const uint32_t *view_count, const float *normals,
+                     float grad_threshold, float scale_threshold, float min_opacity,
+                     const gs_grads *out, const gs_grads *m_out, const gs_grads *v_out,
+                     int64_t out_n_pad, int64_t *n_out, void *stream);
+
+/* Opacity reset over n Gaussians: logit = min(logit, logit(max_opacity)) and
+ * the Adam moments of the opacity logits set to zero ([SN] "A separate
+ * heuristic": reset clamps opacity down to at most 0.01, the usual
+ * max_opacity). All pointers DEVICE, [n] floats. Errors: GS_ERR_INVALID_ARG
+ * for NULL pointers, n < 0 or max_opacity outside (0, 1). */
+gs_status gs_opacity_reset(float *opacity_logits, float *m_logits, float *v_logits, int64_t n,
+                           float max_opacity, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

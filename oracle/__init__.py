@@ -8,6 +8,7 @@ generator.
 from __future__ import annotations
 
 import ctypes
+import math
 
 import numpy as np
 
@@ -267,3 +268,96 @@ def full_loss(scene, cam, target, lam=0.2):
 
 
 __all__ = ["Oracle", "loss", "adam", "blend_screen", "sh_basis", "rotation_cov", "camera", "lib"]
+
+
+# ------------------------------------------------------------ density control
+# Adaptive density control between training steps, after the study notes
+# (bailiping.com) slides "Where to add capacity" / "A separate heuristic" and
+# "How a computer rebuilds a real place ... Gaussian Splats" (taosengine.com),
+# section "Densification": plain float64 numpy, one Gaussian at a time in
+# index order.
+
+def densify_stats(screen_grad, touched):
+    """This view's contribution to the densification statistics: the norm of
+    dL/dmean2d (columns 0, 1 of the n x 9 screen gradient) and a count of 1 for
+    every Gaussian the view touched."""
+    sg = np.asarray(screen_grad, np.float64)
+    vis = np.asarray(touched) > 0
+    norm = np.where(vis, np.sqrt(sg[:, 0] ** 2 + sg[:, 1] ** 2), 0.0)
+    return norm, vis.astype(np.int64)
+
+
+def _rotation(q):
+    """Rotation matrix of the normalised quaternion (w, x, y, z)."""
+    w, x, y, z = np.asarray(q, np.float64) / np.linalg.norm(q)
+    return np.array([[1 - 2 * (y * y + z * z), 2 * (x * y - w * z), 2 * (x * z + w * y)],
+                     [2 * (x * y + w * z), 1 - 2 * (x * x + z * z), 2 * (y * z - w * x)],
+                     [2 * (x * z - w * y), 2 * (y * z + w * x), 1 - 2 * (x * x + y * y)]])
+
+
+def densify(params, m, v, n, grad_accum, view_count, normals, grad_threshold, scale_threshold,
+            min_opacity):
+    """One densification pass. params / m / v: dicts of planar arrays (groups as
+    in the scene layout, last axis >= n). Returns (params, m, v, n_out) with the
+    last axis exactly n_out: kept Gaussians in index order, then clones in
+    parent order, then split children (child 0, child 1) in parent order.
+
+    Per Gaussian: pruned if logit < logit(min_opacity); else, if it was seen
+    and its average screen-gradient norm reaches grad_threshold, cloned when
+    its largest log-scale is at most log(scale_threshold) and split otherwise:
+    two children at mean + R S z_k (z_k the given N(0,1) draws), log-scales
+    minus ln 1.6. Kept Gaussians keep their moments, new ones start at zero."""
+    groups = ("means", "log_scales", "quats", "opacity_logits", "sh")
+    logit_thr = math.log(min_opacity / (1.0 - min_opacity))
+    log_scale_thr = math.log(scale_threshold)
+    kept, clones, children = [], [], []
+    for i in range(n):
+        logit = float(params["opacity_logits"][..., i])
+        if logit < logit_thr:
+            continue
+        cnt = int(view_count[i])
+        dense = cnt > 0 and float(grad_accum[i]) / cnt >= grad_threshold
+        ls = np.asarray(params["log_scales"][:, i], np.float64)
+        if dense and ls.max() > log_scale_thr:
+            R = _rotation(params["quats"][:, i])
+            S = np.diag(np.exp(ls))
+            mu = np.asarray(params["means"][:, i], np.float64)
+            for k in range(2):
+                z = np.asarray(normals[i, k], np.float64)
+                children.append((i, mu + R @ S @ z, ls - math.log(1.6)))
+            continue
+        kept.append(i)
+        if dense:
+            clones.append(i)
+    n_out = len(kept) + len(clones) + len(children)
+    out_p, out_m, out_v = {}, {}, {}
+    for g in groups:
+        shape = params[g].shape[:-1] + (n_out,)
+        out_p[g] = np.zeros(shape)
+        out_m[g] = np.zeros(shape)
+        out_v[g] = np.zeros(shape)
+        col = 0
+        for i in kept:
+            out_p[g][..., col] = params[g][..., i]
+            out_m[g][..., col] = m[g][..., i]
+            out_v[g][..., col] = v[g][..., i]
+            col += 1
+        for i in clones:
+            out_p[g][..., col] = params[g][..., i]
+            col += 1
+        for (i, mean, ls) in children:
+            if g == "means":
+                out_p[g][..., col] = mean
+            elif g == "log_scales":
+                out_p[g][..., col] = ls
+            else:
+                out_p[g][..., col] = params[g][..., i]
+            col += 1
+    return out_p, out_m, out_v, n_out
+
+
+def opacity_reset(logits, m, v, max_opacity):
+    """logit = min(logit, logit(max_opacity)); the moments of the logits set to zero."""
+    cap = math.log(max_opacity / (1.0 - max_opacity))
+    logits = np.minimum(np.asarray(logits, np.float64), cap)
+    return logits, np.zeros_like(np.asarray(m, np.float64)), np.zeros_like(np.asarray(v, np.float64))
