@@ -602,6 +602,109 @@ def main_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def densify_inputs(scene, seed=0):
+    """Seeded synthetic density-control inputs for a scene: view counts 0..4,
+    accumulated gradient norms (exponential per view), N(0,1) split draws, and
+    thresholds placing about 10% of the Gaussians above the gradient cut and
+    half of those above the scale cut; opacity prune at 0.005."""
+    import numpy as np
+    rng = np.random.default_rng(seed)
+    n_pad = scene.n_pad
+    count = rng.integers(0, 5, n_pad).astype(np.int32)
+    accum = (rng.exponential(1.0, n_pad) * count).astype(np.float32)
+    normals = rng.normal(size=(n_pad, 2, 3)).astype(np.float32)
+    avg = np.where(count > 0, accum / np.maximum(count, 1), 0.0)[: scene.n]
+    grad_thr = float(np.quantile(avg[count[: scene.n] > 0], 0.9))
+    scale_thr = float(np.exp(np.median(scene.log_scales[:, : scene.n].max(axis=0))))
+    return accum, count, normals, grad_thr, scale_thr, 0.005
+
+
+def main_densify(args):
+    """Throughput of one densification pass (gs_densify) on the workload's
+    Gaussians with synthetic statistics, against the HBM roofline (parameters
+    and moments read, statistics read, new set written); the oracle timed on a
+    1/200 sample of the Gaussians beside it."""
+    import numpy as np
+    import torch
+
+    import __graft_entry__
+
+    world, rank, local = dist_setup()
+    if rank == 0:
+        __graft_entry__.build()
+    barrier(world)
+    from gaussian_splatting_differentiable_rasteriser_b200 import model, native, scenes
+    from gaussian_splatting_differentiable_rasteriser_b200.scenes import GROUP_NAMES
+
+    native.load()
+    device = f"cuda:{local}"
+    scene = scenes.CONFIGS[args.config]()
+    accum, count, normals, gthr, sthr, mop = densify_inputs(scene)
+    m = model.GaussianModel(scene, device=device)
+    m.m_flat.normal_(0, 1e-3)
+    m.v_flat.uniform_(0, 1e-6)
+    out = model.GaussianModel(scene, device=device)  # output storage, re-strided below
+    cap = (2 * scene.n + 3) // 4 * 4
+    out._alloc(cap)
+    ctx = native.Context(scene.n_pad, 16, 16, 16)
+    d_acc = torch.from_numpy(accum).to(device)
+    d_cnt = torch.from_numpy(count).to(device)
+    d_nrm = torch.from_numpy(normals).to(device)
+    p_in, (m_in, v_in) = m.params_struct(), m.moments_structs()
+    p_out, (m_out, v_out) = out._struct(out.params), out.moments_structs()
+
+    def one():
+        return ctx.densify(p_in, m_in, v_in, d_acc, d_cnt, d_nrm, gthr, sthr, mop, p_out, m_out, v_out, cap)
+
+    for _ in range(args.warmup):
+        n_out = one()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        n_out = one()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1), world)
+    value = replica_throughput(world, args.steps, ms / 1e3)
+    n = scene.n
+    planes = 11 + 3 * scene.sh_k
+    splits = n_out - n  # each split adds one net Gaussian, each clone one, each prune removes one
+    algo_bytes = n * (planes * 12 + 8) + n_out * planes * 12
+    hbm_gbs, _, peak_kind = peaks()
+    achieved = algo_bytes * value / world / 1e9
+    cpu = None
+    if rank == 0 and not args.no_cpu_baseline:
+        import oracle
+        sl = slice(0, n, 200)
+        sub = {k: getattr(scene, k)[..., sl].astype(np.float64) for k in GROUP_NAMES}
+        zeros = {k: np.zeros_like(x) for k, x in sub.items()}
+        k_n = sub["opacity_logits"].shape[-1]
+        t0 = time.perf_counter()
+        oracle.densify(sub, zeros, zeros, k_n, accum[sl][:k_n], count[sl][:k_n], normals[sl][:k_n], gthr, sthr,
+                       mop)
+        est = (time.perf_counter() - t0) * n / k_n
+        cpu = {"value": 1.0 / est, "unit": "passes/s", "cores": 1, "kind": "oracle",
+               "sample": f"float64 oracle densify of every 200th of {n} Gaussians, scaled by 200; single-threaded"}
+    if rank == 0:
+        line = {"metric": "densify passes/s (prune/clone/split with compaction)", "value": value,
+                "unit": "passes/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+                "config": {"workload": WORKLOADS[args.config] + "; synthetic densification statistics",
+                           "gaussians_in": n, "gaussians_out": int(n_out), "net_added": int(splits),
+                           "grad_threshold": gthr, "scale_threshold": sthr, "min_opacity": mop},
+                "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s",
+                             "frac": achieved / hbm_gbs, "traffic": None, "peak_source": peak_kind,
+                             "bytes_per_pass": algo_bytes},
+                "e2e": None, "gpu_launches": 3 * args.steps, "cpu_baseline": cpu}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -615,11 +718,15 @@ def main():
                     help="tile rect: the 3-sigma radius, or the opacity-aware one (same image, fewer entries)")
     ap.add_argument("--deterministic", action="store_true",
                     help="fixed-point gradient atomics (bitwise-reproducible backward)")
+    ap.add_argument("--op", choices=("step", "densify"), default="step",
+                    help="the training step (default) or one densification pass")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         main_reference(args)
+    elif args.op == "densify":
+        main_densify(args)
     else:
         main_ours(args)
 

@@ -57,6 +57,13 @@ struct gs_ctx {
   int opacity_rect = 0;
   unsigned long long* sgrad_fixed = nullptr;  // [max_g][9], allocated by GS_OPTION_DETERMINISTIC
   int deterministic = 0;
+  // density control: caller-owned statistics buffers, and the pass's scratch
+  float* stat_accum = nullptr;
+  uint32_t* stat_count = nullptr;
+  uint4* dens_counts = nullptr;  // [max_blocks]
+  uint4* dens_prefix = nullptr;  // [max_blocks]
+  uint4* dens_totals = nullptr;  // [1], device
+  uint4* dens_host = nullptr;    // [1], pinned host
   // profiling (off by default)
   struct Profiler {
     static constexpr int kMaxRec = 128;
@@ -96,11 +103,12 @@ void free_all(gs_ctx* c) {
                   c->visible_prefix, c->depth_range, c->dkeys[0], c->dkeys[1], c->dvals[0],
                   c->dvals[1], c->dup_status, c->keys[0], c->keys[1], c->vals[0], c->vals[1],
                   c->hist, c->offsets, c->status, c->counters, c->ranges, c->surv, c->surv_count,
-                  c->sgrad_fixed, c->loss_partials,
+                  c->sgrad_fixed, c->dens_counts, c->dens_prefix, c->dens_totals, c->loss_partials,
                   c->loss_counter, c->info_dev, c->pairs};
   for (void* b : bufs)
     if (b) cudaFree(b);
   if (c->info_host) cudaFreeHost(c->info_host);
+  if (c->dens_host) cudaFreeHost(c->dens_host);
   if (c->prof.created)
     for (auto& e : c->prof.ev) cudaEventDestroy(e);
 }
@@ -277,12 +285,16 @@ gs_status gs_create(gs_ctx** out, int64_t max_gaussians, int64_t max_entries, in
   GS_ALLOC(c->ranges, sizeof(uint2) * c->max_tiles);
   GS_ALLOC(c->surv, sizeof(uint2) * 8 * K);
   GS_ALLOC(c->surv_count, sizeof(uint32_t) * 8 * c->max_tiles);
+  GS_ALLOC(c->dens_counts, sizeof(uint4) * ((G + gs::kDensifyBlock - 1) / gs::kDensifyBlock));
+  GS_ALLOC(c->dens_prefix, sizeof(uint4) * ((G + gs::kDensifyBlock - 1) / gs::kDensifyBlock));
+  GS_ALLOC(c->dens_totals, sizeof(uint4));
   GS_ALLOC(c->loss_partials, sizeof(double) * 2 * c->max_loss_blocks);
   GS_ALLOC(c->loss_counter, sizeof(uint32_t));
   GS_ALLOC(c->info_dev, sizeof(gs::ForwardInfo));
   GS_ALLOC(c->pairs, sizeof(unsigned long long) * 8);
 #undef GS_ALLOC
   if (e == cudaSuccess) e = cudaMallocHost(reinterpret_cast<void**>(&c->info_host), sizeof(gs::ForwardInfo));
+  if (e == cudaSuccess) e = cudaMallocHost(reinterpret_cast<void**>(&c->dens_host), sizeof(uint4));
   if (e == cudaSuccess) e = cudaMemset(c->loss_counter, 0, sizeof(uint32_t));
   if (e == cudaSuccess) e = cudaMemset(c->info_dev, 0, sizeof(gs::ForwardInfo));
   if (e == cudaSuccess) e = cudaMemset(c->pairs, 0, sizeof(unsigned long long) * 8);
@@ -586,6 +598,8 @@ gs_status backward_common(gs_ctx* c, const gs_params* p, const gs_camera* cam, c
   a.g_quats = g ? g->quats : nullptr;
   a.g_opacity_logits = g ? g->opacity_logits : nullptr;
   a.g_sh = g ? g->sh : nullptr;
+  a.stat_accum = c->stat_accum;
+  a.stat_count = c->stat_count;
   return GS_OK;
 }
 
@@ -747,6 +761,95 @@ gs_status gs_debug_screen_grads(gs_ctx* c, float* out, void* stream) {
   if (!c->have_fwd) return fail(c, GS_ERR_INVALID_ARG, "gs_render_forward has not run");
   GS_CUDA(c, gs::launch_screen_grads(c->screen, c->sgrad, c->n, out, static_cast<cudaStream_t>(stream)));
   return GS_OK;
+}
+
+
+gs_status gs_set_densify_stats(gs_ctx* c, float* grad_accum, uint32_t* view_count) {
+  if (!c) return GS_ERR_INVALID_ARG;
+  if ((grad_accum == nullptr) != (view_count == nullptr))
+    return fail(c, GS_ERR_INVALID_ARG, "grad_accum and view_count must both be set or both be NULL");
+  if ((grad_accum && !aligned(grad_accum, 4)) || (view_count && !aligned(view_count, 4)))
+    return fail(c, GS_ERR_INVALID_ARG, "statistics buffers must be 4-byte aligned");
+  c->stat_accum = grad_accum;
+  c->stat_count = view_count;
+  return GS_OK;
+}
+
+gs_status gs_densify(gs_ctx* c, const gs_params* in, const gs_grads* m_in, const gs_grads* v_in,
+                     const float* grad_accum, const uint32_t* view_count, const float* normals,
+                     float grad_threshold, float scale_threshold, float min_opacity, const gs_grads* out,
+                     const gs_grads* m_out, const gs_grads* v_out, int64_t out_n_pad, int64_t* n_out,
+                     void* stream) {
+  if (!c) return GS_ERR_INVALID_ARG;
+  gs_status s = check_params(c, in);
+  if (s != GS_OK) return s;
+  if (!m_in || !v_in || !out || !m_out || !v_out || !n_out)
+    return fail(c, GS_ERR_INVALID_ARG, "moment, output and count pointers must be non-NULL");
+  if (!(grad_threshold > 0.f) || !(scale_threshold > 0.f) || !(min_opacity > 0.f && min_opacity < 1.f) ||
+      !std::isfinite(grad_threshold) || !std::isfinite(scale_threshold))
+    return fail(c, GS_ERR_INVALID_ARG, "thresholds must be positive and min_opacity in (0, 1)");
+  if (out_n_pad < 0) return fail(c, GS_ERR_INVALID_ARG, "out_n_pad must be >= 0");
+  const gs_grads* sets[5] = {m_in, v_in, out, m_out, v_out};
+  if (in->n > 0) {
+    if (!grad_accum || !view_count || !normals) return fail(c, GS_ERR_INVALID_ARG, "statistics/normals NULL");
+    for (const gs_grads* g : sets) {
+      const float* q[5] = {g->means, g->log_scales, g->quats, g->opacity_logits, g->sh};
+      for (const float* x : q)
+        if (!x || !aligned(x, 4)) return fail(c, GS_ERR_INVALID_ARG, "a buffer pointer is NULL or misaligned");
+    }
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  gs::DensifyArgs a;
+  a.means = in->means;
+  a.log_scales = in->log_scales;
+  a.quats = in->quats;
+  a.opacity_logits = in->opacity_logits;
+  a.sh = in->sh;
+  const float* mi[5] = {m_in->means, m_in->log_scales, m_in->quats, m_in->opacity_logits, m_in->sh};
+  const float* vi[5] = {v_in->means, v_in->log_scales, v_in->quats, v_in->opacity_logits, v_in->sh};
+  float* po[5] = {out->means, out->log_scales, out->quats, out->opacity_logits, out->sh};
+  float* mo[5] = {m_out->means, m_out->log_scales, m_out->quats, m_out->opacity_logits, m_out->sh};
+  float* vo[5] = {v_out->means, v_out->log_scales, v_out->quats, v_out->opacity_logits, v_out->sh};
+  for (int k = 0; k < 5; ++k) {
+    a.m[k] = mi[k];
+    a.v[k] = vi[k];
+    a.out_p[k] = po[k];
+    a.out_m[k] = mo[k];
+    a.out_v[k] = vo[k];
+  }
+  a.n = in->n;
+  a.np_in = in->n_pad;
+  a.sh_k = (in->sh_degree + 1) * (in->sh_degree + 1);
+  a.grad_accum = grad_accum;
+  a.view_count = view_count;
+  a.normals = normals;
+  a.grad_threshold = static_cast<double>(grad_threshold);
+  a.log_scale_threshold = std::log(static_cast<double>(scale_threshold));
+  a.logit_threshold = std::log(static_cast<double>(min_opacity) / (1.0 - static_cast<double>(min_opacity)));
+  a.np_out = out_n_pad;
+  a.block_counts = c->dens_counts;
+  a.block_prefix = c->dens_prefix;
+  a.totals = c->dens_totals;
+  GS_CUDA(c, gs::launch_densify_count(a, st));
+  GS_CUDA(c, cudaMemcpyAsync(c->dens_host, c->dens_totals, sizeof(uint4), cudaMemcpyDeviceToHost, st));
+  GS_CUDA(c, cudaStreamSynchronize(st));
+  const uint4 tot = *c->dens_host;
+  const int64_t count = static_cast<int64_t>(tot.x) + tot.y + 2 * static_cast<int64_t>(tot.z);
+  *n_out = count;
+  if (count > out_n_pad)
+    return fail(c, GS_ERR_CAPACITY, "densification gives %lld Gaussians; the output holds %lld",
+                (long long)count, (long long)out_n_pad);
+  GS_CUDA(c, gs::launch_densify_write(a, tot, st));
+  return GS_OK;
+}
+
+gs_status gs_opacity_reset(float* logits, float* m, float* v, int64_t n, float max_opacity, void* stream) {
+  if (n < 0 || !(max_opacity > 0.f && max_opacity < 1.f)) return GS_ERR_INVALID_ARG;
+  if (n > 0 && (!logits || !m || !v)) return GS_ERR_INVALID_ARG;
+  const double mo = static_cast<double>(max_opacity);
+  const float cap = static_cast<float>(std::log(mo / (1.0 - mo)));
+  cudaError_t e = gs::launch_opacity_reset(logits, m, v, n, cap, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? GS_OK : GS_ERR_CUDA;
 }
 
 }  // extern "C"

@@ -171,6 +171,9 @@ struct PreprocessBwdArgs {
   const uint8_t* clamped;
   const float* sgrad;
   float *g_means, *g_log_scales, *g_quats, *g_opacity_logits, *g_sh;
+  // density-control statistics (both null when not accumulating)
+  float* stat_accum;
+  uint32_t* stat_count;
 };
 
 cudaError_t launch_preprocess_backward(const PreprocessBwdArgs& a, cudaStream_t st);
@@ -191,6 +194,27 @@ cudaError_t launch_preprocess_backward_adam(const PreprocessBwdArgs& a, const Fu
 AdamScalars adam_scalars(float lr, float beta1, float beta2, float eps, int step);
 cudaError_t launch_screen_grads(const Screen* screen, const float* sgrad, int64_t n, float* out,
                                 cudaStream_t st);
+
+// ------------------------------------------------------- density control
+struct DensifyArgs {
+  const float *means, *log_scales, *quats, *opacity_logits, *sh;  // in, planar with stride np_in
+  const float *m[5], *v[5];                                       // moments in, same layout
+  int64_t n, np_in;
+  int sh_k;
+  const float* grad_accum;
+  const uint32_t* view_count;
+  const float* normals;  // [n][2][3]
+  double grad_threshold, log_scale_threshold, logit_threshold;
+  float *out_p[5], *out_m[5], *out_v[5];  // planar with stride np_out
+  int64_t np_out;
+  uint4* block_counts;   // [blocks]: kept, clones, splits
+  uint4* block_prefix;   // [blocks]: exclusive prefixes of the same
+  uint4* totals;         // [1]
+};
+constexpr int kDensifyBlock = 256;
+cudaError_t launch_densify_count(const DensifyArgs& a, cudaStream_t st);
+cudaError_t launch_densify_write(const DensifyArgs& a, uint4 totals, cudaStream_t st);
+cudaError_t launch_opacity_reset(float* logits, float* m, float* v, int64_t n, float cap, cudaStream_t st);
 
 // ---------------------------------------------------------------- Adam
 cudaError_t launch_adam(float* p, float* g, float* m, float* v, int64_t count, float lr,

@@ -40,7 +40,17 @@ struct GaussGrad {
   float dp[3], dls[3], dq[4], dlogit;
   float drgb[3];
   float vx, vy, vz, idl;
+  float du, dv;  // dL/dmean2d (pixels)
 };
+
+// Density-control statistics of a Gaussian this view touched: the norm of
+// dL/dmean2d and one more view (one thread per Gaussian: no atomics needed).
+__device__ __forceinline__ void add_densify_stats(const PreprocessBwdArgs& a, int64_t i, const GaussGrad& g) {
+  if (a.stat_accum) {
+    a.stat_accum[i] += sqrtf(g.du * g.du + g.dv * g.dv);
+    a.stat_count[i] += 1u;
+  }
+}
 
 __device__ __forceinline__ void geometry_grad(const PreprocessBwdArgs& a, int64_t i, GaussGrad& out) {
   const int64_t np = a.n_pad;
@@ -54,6 +64,8 @@ __device__ __forceinline__ void geometry_grad(const PreprocessBwdArgs& a, int64_
   // Screen-space gradient from the raw sums (w = dL/dalpha * o exp(-e)).
   const float d_u = A * r0.y + B * r0.z;
   const float d_v = B * r0.y + C * r0.z;
+  out.du = d_u;
+  out.dv = d_v;
   const float dA = -0.5f * r0.w, dB = -r1.x, dC = -0.5f * r1.y;
   const float d_o = r0.x / o;
   out.drgb[0] = (clamped & 1) ? 0.f : r1.z;
@@ -199,6 +211,7 @@ __global__ void __launch_bounds__(256) preprocess_backward_kernel(PreprocessBwdA
   const int64_t np = a.n_pad;
   GaussGrad g;
   geometry_grad(a, i, g);
+  add_densify_stats(a, i, g);
   constexpr int nk = (kDeg + 1) * (kDeg + 1);
   float Yk[16];
   sh_basis(kDeg, g.vx, g.vy, g.vz, Yk);
@@ -278,6 +291,7 @@ __global__ void __launch_bounds__(kFusedBlock) preprocess_backward_adam_kernel(P
     if (visible) {
       GaussGrad g;
       geometry_grad(a, i, g);
+      add_densify_stats(a, i, g);
       float Yk[16];
       sh_basis(kDeg, g.vx, g.vy, g.vz, Yk);
       float wsum[16];

@@ -24,15 +24,24 @@ def group_shapes(n_pad: int, sh_degree: int) -> dict:
 
 class GaussianModel:
     def __init__(self, scene, device="cuda", active_degree=None):
-        self.n, self.n_pad, self.sh_degree = scene.n, scene.n_pad, scene.sh_degree
+        self.n, self.sh_degree = scene.n, scene.sh_degree
         self.active_degree = scene.sh_degree if active_degree is None else active_degree
-        shapes = group_shapes(self.n_pad, self.sh_degree)
+        self.device = device
+        self._alloc(scene.n_pad)
+        self.load(scene)
+        self.step_count = 0
+
+    def _alloc(self, n_pad):
+        """Fresh flat buffers (parameters uninitialised, the rest zero) for n_pad slots."""
+        self.n_pad = n_pad
+        shapes = group_shapes(n_pad, self.sh_degree)
         sizes = {k: int(torch.Size(s).numel()) for k, s in shapes.items()}
         total = sum(sizes.values())
-        self.flat = torch.empty(total, dtype=torch.float32, device=device)
-        self.grad_flat = torch.zeros(total, dtype=torch.float32, device=device)
-        self.m_flat = torch.zeros(total, dtype=torch.float32, device=device)
-        self.v_flat = torch.zeros(total, dtype=torch.float32, device=device)
+        dev = self.device
+        self.flat = torch.empty(total, dtype=torch.float32, device=dev)
+        self.grad_flat = torch.zeros(total, dtype=torch.float32, device=dev)
+        self.m_flat = torch.zeros(total, dtype=torch.float32, device=dev)
+        self.v_flat = torch.zeros(total, dtype=torch.float32, device=dev)
         self.params, self.grads, self.m, self.v, self.slices = {}, {}, {}, {}, {}
         off = 0
         for k in GROUP_NAMES:
@@ -43,8 +52,24 @@ class GaussianModel:
             self.m[k] = self.m_flat[sl].view(shapes[k])
             self.v[k] = self.v_flat[sl].view(shapes[k])
             off += sizes[k]
-        self.load(scene)
-        self.step_count = 0
+
+    def densify(self, ctx, grad_accum, view_count, normals, grad_threshold, scale_threshold,
+                min_opacity, capacity=None):
+        """One gs_densify pass into new buffers of `capacity` slots (default: room
+        for every Gaussian to split); the model then holds the new set, its
+        moments and zeroed gradients. Returns the new count."""
+        p_in, (m_in, v_in) = self.params_struct(), self.moments_structs()
+        keep = (self.flat, self.m_flat, self.v_flat, self.grad_flat)  # alive until the call returns
+        cap = capacity if capacity is not None else max(4, (2 * self.n + 3) // 4 * 4)
+        old_params, old_m, old_v = self.params, self.m, self.v
+        self._alloc(cap)
+        self.flat.zero_()
+        out, (m_out, v_out) = self._struct(self.params), self.moments_structs()
+        n_out = ctx.densify(p_in, m_in, v_in, grad_accum, view_count, normals, grad_threshold,
+                            scale_threshold, min_opacity, out, m_out, v_out, cap)
+        del keep, old_params, old_m, old_v
+        self.n = n_out
+        return n_out
 
     def load(self, scene):
         for k in GROUP_NAMES:

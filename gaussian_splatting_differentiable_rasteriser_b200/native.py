@@ -24,7 +24,8 @@ EXPORTED = ("gs_create", "gs_destroy", "gs_last_error", "gs_preprocess", "gs_ren
             "gs_loss_l1_dssim", "gs_render_backward", "gs_render_backward_adam", "gs_adam_step",
             "gs_profile_enable",
             "gs_profile_read", "gs_stage_name", "gs_debug_preprocess", "gs_debug_sorted",
-            "gs_debug_screen_grads", "gs_set_option", "gs_loss_l1_dssim_noalloc")
+            "gs_debug_screen_grads", "gs_set_option", "gs_loss_l1_dssim_noalloc",
+            "gs_set_densify_stats", "gs_densify", "gs_opacity_reset")
 GS_OPTION_OPACITY_RECT = 1
 GS_OPTION_DETERMINISTIC = 2
 STAGES = ("preprocess", "scan", "duplicate", "sort", "ranges", "blend_forward", "loss",
@@ -86,6 +87,11 @@ def load(path: str = LIB_PATH):
                                           ctypes.POINTER(GsGrads), ctypes.POINTER(GsGrads),
                                           ctypes.POINTER(GsGrads), ctypes.POINTER(F), F, F, F, I32, P]
     L.gs_adam_step.argtypes = [P, P, P, P, I64, F, F, F, F, I32, P]
+    L.gs_set_densify_stats.argtypes = [P, P, P]
+    L.gs_densify.argtypes = [P, ctypes.POINTER(GsParams), ctypes.POINTER(GsGrads), ctypes.POINTER(GsGrads),
+                             P, P, P, F, F, F, ctypes.POINTER(GsGrads), ctypes.POINTER(GsGrads),
+                             ctypes.POINTER(GsGrads), I64, ctypes.POINTER(I64), P]
+    L.gs_opacity_reset.argtypes = [P, P, P, I64, F, P]
     L.gs_set_option.argtypes = [P, I32, I32]
     L.gs_set_option.restype = ctypes.c_int
     L.gs_loss_l1_dssim_noalloc.argtypes = [P, P, I32, I32, F, P, P, P]
@@ -158,6 +164,20 @@ class Context:
     def set_option(self, option, value):
         self._check(self.L.gs_set_option(self.h, int(option), int(value)))
 
+    def set_densify_stats(self, grad_accum, view_count):
+        self._check(self.L.gs_set_densify_stats(self.h, _ptr(grad_accum), _ptr(view_count)))
+
+    def densify(self, params: GsParams, m_in: GsGrads, v_in: GsGrads, grad_accum, view_count, normals,
+                grad_threshold, scale_threshold, min_opacity, out: GsGrads, m_out: GsGrads, v_out: GsGrads,
+                out_n_pad, stream=None) -> int:
+        n_out = ctypes.c_int64(0)
+        self._check(self.L.gs_densify(self.h, ctypes.byref(params), ctypes.byref(m_in), ctypes.byref(v_in),
+                                      _ptr(grad_accum), _ptr(view_count), _ptr(normals),
+                                      float(grad_threshold), float(scale_threshold), float(min_opacity),
+                                      ctypes.byref(out), ctypes.byref(m_out), ctypes.byref(v_out),
+                                      int(out_n_pad), ctypes.byref(n_out), _stream(stream)))
+        return n_out.value
+
     def preprocess(self, params: GsParams, cam: GsCamera, stream=None):
         self._check(self.L.gs_preprocess(self.h, ctypes.byref(params), ctypes.byref(cam), _stream(stream)))
 
@@ -222,3 +242,11 @@ def adam_step(param, grad, m, v, lr, step, beta1=0.9, beta2=0.999, eps=1e-8, str
                         float(beta1), float(beta2), float(eps), int(step), _stream(stream))
     if st != GS_OK:
         raise GsError(st, "gs_adam_step rejected its arguments")
+
+
+def opacity_reset(logits, m, v, max_opacity=0.01, stream=None):
+    L = load()
+    st = L.gs_opacity_reset(_ptr(logits), _ptr(m), _ptr(v), logits.numel(), float(max_opacity),
+                            _stream(stream))
+    if st != GS_OK:
+        raise GsError(st, "gs_opacity_reset rejected its arguments")
