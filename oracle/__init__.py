@@ -361,3 +361,27 @@ def opacity_reset(logits, m, v, max_opacity):
     cap = math.log(max_opacity / (1.0 - max_opacity))
     logits = np.minimum(np.asarray(logits, np.float64), cap)
     return logits, np.zeros_like(np.asarray(m, np.float64)), np.zeros_like(np.asarray(v, np.float64))
+
+
+# --------------------------------------------------- Charbonnier + exposure
+def charbonnier_loss(image, target, gain, bias, delta=0.03):
+    """Robust photometric loss with a per-photo exposure correction, after "How a
+    computer rebuilds a real place ... Gaussian Splats" (taosengine.com), the
+    loss paragraph before "The chain rule, in one breath": per pixel p and
+    channel c, err = gain_c C + bias_c - target, root = sqrt(err^2 + delta^2),
+    pixel loss = sum_c root - 3 delta; the image loss is the mean over the H W
+    pixels. Returns (loss, dL/dimage [3,H,W], dL/dgain [3], dL/dbias [3]) in
+    float64."""
+    x = np.asarray(image, np.float64)
+    y = np.asarray(target, np.float64)
+    g = np.asarray(gain, np.float64).reshape(3, 1, 1)
+    b = np.asarray(bias, np.float64).reshape(3, 1, 1)
+    P = x.shape[1] * x.shape[2]
+    err = g * x + b - y
+    root = np.sqrt(err * err + delta * delta)
+    loss = float((root.sum(axis=0) - 3.0 * delta).sum() / P)
+    slope = err / root
+    d_image = g * slope / P
+    d_gain = (slope * x).sum(axis=(1, 2)) / P
+    d_bias = slope.sum(axis=(1, 2)) / P
+    return loss, d_image, d_gain, d_bias
