@@ -54,8 +54,8 @@ WORKLOADS = {
 # proportion. The fused pass's write counter undercounts: its last writes are still
 # in L2 when the kernel ends.
 NCU_TRAFFIC = {
-    "backward_adam": ((408.017408e6 + 295.502080e6) * 6.0, "07567fb73e7b"),
-    "blend_backward": ((85.316096e6 + 4.134912e6) * 6.32 / 1.064, "9e7084e8dff0"),
+    "backward_adam": ((409.031424e6 + 290.892288e6) * 6.0, "2ade6b8bdb45"),
+    "blend_backward": ((85.229824e6 + 2.950144e6) * 6.32 / 1.064, "0758f6489db1"),
 }
 
 
@@ -165,7 +165,7 @@ def max_over_ranks(x, world):
 
 
 # ------------------------------------------------------------------ workload
-def build_workload(config, device, opacity_rect=False, deterministic=False):
+def build_workload(config, device, opacity_rect=False, deterministic=False, loss="l1_dssim"):
     import numpy as np
     import torch
 
@@ -179,7 +179,7 @@ def build_workload(config, device, opacity_rect=False, deterministic=False):
     m = model.GaussianModel(pert, device=device)
     cap = max(1 << 20, 8 * scene.n)
     step = model.TrainStep(m, cap, W, H, device=device, opacity_rect=opacity_rect,
-                           deterministic=deterministic)
+                           deterministic=deterministic, loss=loss)
     # targets: renders of the perturbed copy (forward only, before any timing)
     targets = torch.empty((len(cams), 3, H, W), dtype=torch.float32, device=device)
     kmax = 0
@@ -233,7 +233,7 @@ def profile_stages(step, cams, targets, sched, start, count):
         cs = native.camera_struct(cam)
         img, T, nc = step.forward(cs, cam.height, cam.width)
         ks.append(step.last_entries)
-        ctx.loss_l1_dssim(img, targets[c], step.lam, step.loss, step.dimage)
+        step.compute_loss(img, targets[c], step.dimage)
         if step.fused_adam:
             step.backward_and_update(cs, T, nc, step.dimage)
             continue
@@ -430,7 +430,7 @@ def main_ours(args):
     native.load()
     device = f"cuda:{local}"
     scene, m, step, targets, kmax = build_workload(args.config, device, args.rect == "opacity",
-                                                   args.deterministic)
+                                                   args.deterministic, args.loss)
     cams = scene.cameras
     sched = scenes.camera_schedule(len(cams), args.warmup + args.steps, seed=rank)
     # clocks are sampled from the start of the warm-up to the end of the timed region
@@ -488,6 +488,7 @@ def main_ours(args):
                        "parallelism": "replicas" if world > 1 else "single-gpu",
                        "tile_rect": "3 sigma" if args.rect == "3sigma" else "opacity-aware",
                        "gradient_sums": "fixed-point (deterministic)" if args.deterministic else "float32 atomics",
+                       "loss": "L1 + D-SSIM (lambda 0.2)" if args.loss == "l1_dssim" else "Charbonnier + exposure",
                        "l2": "inputs larger than L2: 2.8 GB of parameter/gradient/moment state "
                              "streamed every step" if args.config == "dense" else "see workload",
                        "entries_per_step": int(statistics.mean(ks)) if ks else None},
@@ -546,9 +547,9 @@ def e2e_run(step, cams, targets, sched, args, world):
                 dev_t[(j + 1) % 2].copy_(host_t[cn], non_blocking=True)
                 copied[(j + 1) % 2].record(copy_stream)
         torch.cuda.current_stream().wait_event(copied[j % 2])
-        step.ctx.loss_l1_dssim(img, dev_t[j % 2], step.lam, step.loss, step.dimage)
+        step.compute_loss(img, dev_t[j % 2], step.dimage)
         step.backward_and_update(cs, T, nc, step.dimage)
-        loss_host[j % 2].copy_(step.loss, non_blocking=True)
+        loss_host[j % 2].copy_(step.loss[:3], non_blocking=True)
     torch.cuda.synchronize()
     losses.append(float(loss_host[(n - 1) % 2, 0]))
     dt = time.perf_counter() - t0
@@ -718,6 +719,8 @@ def main():
                     help="tile rect: the 3-sigma radius, or the opacity-aware one (same image, fewer entries)")
     ap.add_argument("--deterministic", action="store_true",
                     help="fixed-point gradient atomics (bitwise-reproducible backward)")
+    ap.add_argument("--loss", choices=("l1_dssim", "charbonnier"), default="l1_dssim",
+                    help="photometric loss of the step")
     ap.add_argument("--op", choices=("step", "densify"), default="step",
                     help="the training step (default) or one densification pass")
     args = ap.parse_args()

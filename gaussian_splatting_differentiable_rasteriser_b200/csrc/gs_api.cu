@@ -44,6 +44,8 @@ struct gs_ctx {
   // loss
   double* loss_partials = nullptr;
   uint32_t* loss_counter = nullptr;
+  double* charb_partials = nullptr;  // [kCharbMaxBlocks][7]
+  uint32_t* charb_counter = nullptr;
   // readback record (device + pinned host); the device error word lives in it
   gs::ForwardInfo* info_dev = nullptr;
   gs::ForwardInfo* info_host = nullptr;
@@ -103,7 +105,8 @@ void free_all(gs_ctx* c) {
                   c->visible_prefix, c->depth_range, c->dkeys[0], c->dkeys[1], c->dvals[0],
                   c->dvals[1], c->dup_status, c->keys[0], c->keys[1], c->vals[0], c->vals[1],
                   c->hist, c->offsets, c->status, c->counters, c->ranges, c->surv, c->surv_count,
-                  c->sgrad_fixed, c->dens_counts, c->dens_prefix, c->dens_totals, c->loss_partials,
+                  c->sgrad_fixed, c->dens_counts, c->dens_prefix, c->dens_totals, c->charb_partials,
+                  c->charb_counter, c->loss_partials,
                   c->loss_counter, c->info_dev, c->pairs};
   for (void* b : bufs)
     if (b) cudaFree(b);
@@ -290,12 +293,15 @@ gs_status gs_create(gs_ctx** out, int64_t max_gaussians, int64_t max_entries, in
   GS_ALLOC(c->dens_totals, sizeof(uint4));
   GS_ALLOC(c->loss_partials, sizeof(double) * 2 * c->max_loss_blocks);
   GS_ALLOC(c->loss_counter, sizeof(uint32_t));
+  GS_ALLOC(c->charb_partials, sizeof(double) * 7 * gs::kCharbMaxBlocks);
+  GS_ALLOC(c->charb_counter, sizeof(uint32_t));
   GS_ALLOC(c->info_dev, sizeof(gs::ForwardInfo));
   GS_ALLOC(c->pairs, sizeof(unsigned long long) * 8);
 #undef GS_ALLOC
   if (e == cudaSuccess) e = cudaMallocHost(reinterpret_cast<void**>(&c->info_host), sizeof(gs::ForwardInfo));
   if (e == cudaSuccess) e = cudaMallocHost(reinterpret_cast<void**>(&c->dens_host), sizeof(uint4));
   if (e == cudaSuccess) e = cudaMemset(c->loss_counter, 0, sizeof(uint32_t));
+  if (e == cudaSuccess) e = cudaMemset(c->charb_counter, 0, sizeof(uint32_t));
   if (e == cudaSuccess) e = cudaMemset(c->info_dev, 0, sizeof(gs::ForwardInfo));
   if (e == cudaSuccess) e = cudaMemset(c->pairs, 0, sizeof(unsigned long long) * 8);
   if (e == cudaSuccess) e = cudaDeviceSynchronize();
@@ -850,6 +856,40 @@ gs_status gs_opacity_reset(float* logits, float* m, float* v, int64_t n, float m
   const float cap = static_cast<float>(std::log(mo / (1.0 - mo)));
   cudaError_t e = gs::launch_opacity_reset(logits, m, v, n, cap, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? GS_OK : GS_ERR_CUDA;
+}
+
+
+gs_status gs_loss_charbonnier(gs_ctx* c, const float* image, const float* target, int32_t height,
+                              int32_t width, const float* gain, const float* bias, float delta,
+                              double* out, float* dloss_dimage, void* stream) {
+  if (!c) return GS_ERR_INVALID_ARG;
+  if (height <= 0 || width <= 0 || height > c->max_h || width > c->max_w)
+    return fail(c, GS_ERR_INVALID_ARG, "image %dx%d outside the context's maximum", width, height);
+  if (!image || !target || !out || !gain || !bias || !aligned(image, 4) || !aligned(target, 4) ||
+      !aligned(out, 8) || (dloss_dimage && !aligned(dloss_dimage, 4)))
+    return fail(c, GS_ERR_INVALID_ARG, "loss pointers must be non-NULL and aligned");
+  if (!(delta > 0.f) || !std::isfinite(delta)) return fail(c, GS_ERR_INVALID_ARG, "delta must be positive");
+  for (int k = 0; k < 3; ++k)
+    if (!std::isfinite(gain[k]) || !std::isfinite(bias[k]))
+      return fail(c, GS_ERR_INVALID_ARG, "gain and bias must be finite");
+  gs::CharbonnierArgs a;
+  a.x = image;
+  a.y = target;
+  a.pixels = static_cast<int64_t>(height) * width;
+  for (int k = 0; k < 3; ++k) {
+    a.gain[k] = gain[k];
+    a.bias[k] = bias[k];
+  }
+  a.delta = delta;
+  a.dx = dloss_dimage;
+  a.partials = c->charb_partials;
+  a.counter = c->charb_counter;
+  a.out = out;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  prof_begin(c, st);
+  GS_CUDA(c, gs::launch_charbonnier(a, st));
+  prof_end(c, GS_STAGE_LOSS, a.pixels, st);
+  return GS_OK;
 }
 
 }  // extern "C"

@@ -160,6 +160,21 @@ constexpr int64_t loss_blocks(int height, int width) {
 
 cudaError_t launch_loss(const LossArgs& a, cudaStream_t st);
 
+// The Charbonnier + exposure loss: out = {loss, dL/dgain[3], dL/dbias[3]}.
+struct CharbonnierArgs {
+  const float* x;
+  const float* y;
+  int64_t pixels;  // H W
+  float gain[3], bias[3], delta;
+  float* dx;           // may be null
+  double* partials;    // [blocks][7]
+  uint32_t* counter;   // zero between calls
+  double* out;         // [7]
+};
+constexpr int kCharbMaxBlocks = 148 * 8;
+int charbonnier_blocks(int64_t pixels);
+cudaError_t launch_charbonnier(const CharbonnierArgs& a, cudaStream_t st);
+
 // ------------------------------------------------------- projection backward
 struct PreprocessBwdArgs {
   const float *means, *log_scales, *quats, *opacity_logits, *sh;

@@ -104,9 +104,14 @@ class TrainStep:
 
     def __init__(self, model: GaussianModel, max_entries: int, width: int, height: int, lrs=None,
                  lam=0.2, betas=(0.9, 0.999), eps=1e-8, device="cuda", fused_adam=True,
-                 opacity_rect=False, deterministic=False):
+                 opacity_rect=False, deterministic=False, loss="l1_dssim"):
         self.model = model
         self.fused_adam = fused_adam
+        if loss not in ("l1_dssim", "charbonnier"):
+            raise ValueError("loss must be 'l1_dssim' or 'charbonnier'")
+        self.loss_kind = loss
+        # per-photo exposure of the Charbonnier loss (identity by default)
+        self.gain, self.bias = [1.0, 1.0, 1.0], [0.0, 0.0, 0.0]
         self.ctx = native.Context(model.n_pad, max_entries, width, height)
         if opacity_rect:
             self.ctx.set_option(native.GS_OPTION_OPACITY_RECT, 1)
@@ -118,7 +123,8 @@ class TrainStep:
         self.final_T = torch.empty((height, width), dtype=torch.float32, device=device)
         self.n_contrib = torch.empty((height, width), dtype=torch.int32, device=device)
         self.dimage = torch.empty((3, height, width), dtype=torch.float32, device=device)
-        self.loss = torch.zeros(3, dtype=torch.float64, device=device)
+        # {loss, L1, SSIM}, or for the Charbonnier loss {loss, dL/dgain[3], dL/dbias[3]}
+        self.loss = torch.zeros(7, dtype=torch.float64, device=device)
         self.last_entries = 0
 
     def forward(self, cam_struct, H, W):
@@ -138,9 +144,16 @@ class TrainStep:
         H, W = cam.height, cam.width
         img, T, nc = self.forward(cs, H, W)
         dimg = self.dimage if img.shape == self.dimage.shape else torch.empty_like(img)
-        self.ctx.loss_l1_dssim(img, target, self.lam, self.loss, dimg)
+        self.compute_loss(img, target, dimg)
         self.backward_and_update(cs, T, nc, dimg)
         return self.loss
+
+    def compute_loss(self, img, target, dimg):
+        """The configured loss of `img` against `target`, its gradient into dimg."""
+        if self.loss_kind == "charbonnier":
+            self.ctx.loss_charbonnier(img, target, self.gain, self.bias, self.loss, dimg)
+        else:
+            self.ctx.loss_l1_dssim(img, target, self.lam, self.loss, dimg)
 
     def backward_and_update(self, cs, T, nc, dimg):
         """Backward of the last forward plus the Adam step of every group: one fused

@@ -25,7 +25,7 @@ EXPORTED = ("gs_create", "gs_destroy", "gs_last_error", "gs_preprocess", "gs_ren
             "gs_profile_enable",
             "gs_profile_read", "gs_stage_name", "gs_debug_preprocess", "gs_debug_sorted",
             "gs_debug_screen_grads", "gs_set_option", "gs_loss_l1_dssim_noalloc",
-            "gs_set_densify_stats", "gs_densify", "gs_opacity_reset")
+            "gs_set_densify_stats", "gs_densify", "gs_opacity_reset", "gs_loss_charbonnier")
 GS_OPTION_OPACITY_RECT = 1
 GS_OPTION_DETERMINISTIC = 2
 STAGES = ("preprocess", "scan", "duplicate", "sort", "ranges", "blend_forward", "loss",
@@ -92,6 +92,7 @@ def load(path: str = LIB_PATH):
                              P, P, P, F, F, F, ctypes.POINTER(GsGrads), ctypes.POINTER(GsGrads),
                              ctypes.POINTER(GsGrads), I64, ctypes.POINTER(I64), P]
     L.gs_opacity_reset.argtypes = [P, P, P, I64, F, P]
+    L.gs_loss_charbonnier.argtypes = [P, P, P, I32, I32, ctypes.POINTER(F), ctypes.POINTER(F), F, P, P, P]
     L.gs_set_option.argtypes = [P, I32, I32]
     L.gs_set_option.restype = ctypes.c_int
     L.gs_loss_l1_dssim_noalloc.argtypes = [P, P, I32, I32, F, P, P, P]
@@ -163,6 +164,13 @@ class Context:
 
     def set_option(self, option, value):
         self._check(self.L.gs_set_option(self.h, int(option), int(value)))
+
+    def loss_charbonnier(self, image, target, gain, bias, out, dloss_dimage=None, delta=0.03, stream=None):
+        _, H, W = image.shape
+        g = (ctypes.c_float * 3)(*[float(x) for x in gain])
+        b = (ctypes.c_float * 3)(*[float(x) for x in bias])
+        self._check(self.L.gs_loss_charbonnier(self.h, _ptr(image), _ptr(target), H, W, g, b, float(delta),
+                                               _ptr(out), _ptr(dloss_dimage), _stream(stream)))
 
     def set_densify_stats(self, grad_accum, view_count):
         self._check(self.L.gs_set_densify_stats(self.h, _ptr(grad_accum), _ptr(view_count)))

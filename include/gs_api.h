@@ -309,6 +309,21 @@ gs_status gs_debug_sorted(gs_ctx *ctx, int32_t *ids, int32_t *tiles, int32_t *ra
  * dL/d(mean2d x, mean2d y, A, B, C, opacity, r, g, b). */
 gs_status gs_debug_screen_grads(gs_ctx *ctx, float *out, void *stream);
 
+/* Step 3, second loss ([GS] the loss paragraph before "The chain rule, in one
+ * breath"): a Charbonnier loss with a per-photo exposure correction,
+ * err = gain_c C + bias_c - target per channel c, root = sqrt(err^2 +
+ * delta^2), pixel loss = sum_c root - 3 delta (the page uses delta = 0.03),
+ * image loss = the mean over the H W pixels. image_chw and target_chw are
+ * [3][H][W] DEVICE float32; gain and bias are HOST arrays of 3. out is a
+ * DEVICE array of 7 doubles: {loss, dL/dgain[3], dL/dbias[3]};
+ * dloss_dimage (DEVICE [3][H][W], may be NULL) receives gain_c err / root / (H W).
+ * The reductions are float64 in a fixed order (deterministic). Errors:
+ * GS_ERR_INVALID_ARG for bad pointers, an image larger than the context's
+ * maximum, delta <= 0 or non-finite gain / bias. */
+gs_status gs_loss_charbonnier(gs_ctx *ctx, const float *image_chw, const float *target_chw,
+                              int32_t height, int32_t width, const float *gain, const float *bias,
+                              float delta, double *out, float *dloss_dimage, void *stream);
+
 /* ------------------------------------------------------ density control --
  * Adaptive density control, run between training steps ([SN] slides "Where
  * to add capacity" and "A separate heuristic": the screen-space centre

@@ -483,3 +483,55 @@ def test_deterministic_backward_is_bitwise_reproducible_and_matches_oracle(gs):
         torch.cuda.synchronize()
         params.append(host(m.flat).view(np.uint32).copy())
     np.testing.assert_array_equal(params[0], params[1])
+
+
+@pytest.mark.parametrize("shape", [(256, 256), (37, 45), (1, 5)])
+def test_charbonnier_loss_matches_oracle(gs, shape):
+    native, _ = gs
+    H, W = shape
+    rng = np.random.default_rng(H + W)
+    x = rng.uniform(0, 1, (3, H, W)).astype(np.float32)
+    y = np.clip(x + rng.normal(0, 0.2, x.shape), 0, 1).astype(np.float32)
+    y[0, 0, 0] = 40.0  # an outlier
+    gain, bias = [1.1, 0.9, 1.02], [0.03, -0.02, 0.0]
+    ctx = native.Context(16, 16, max(W, 16), max(H, 16))
+    out = torch.zeros(7, dtype=torch.float64, device="cuda")
+    d = torch.empty((3, H, W), device="cuda")
+    f32 = [float(np.float32(v)) for v in gain], [float(np.float32(v)) for v in bias]
+    ctx.loss_charbonnier(dev(x), dev(y), gain, bias, out, d)
+    torch.cuda.synchronize()
+    L, dref, dg, db = oracle.charbonnier_loss(x, y, f32[0], f32[1])
+    got = host(out)
+    assert got[0] == pytest.approx(L, rel=LOSS_RTOL)
+    np.testing.assert_allclose(got[1:4], dg, rtol=1e-5, atol=1e-9)
+    np.testing.assert_allclose(got[4:7], db, rtol=1e-5, atol=1e-9)
+    assert rel_l2(host(d), dref) < 1e-5
+    ctx.loss_charbonnier(dev(x), dev(y), gain, bias, out, d)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(host(out), got)  # deterministic, counter reset
+
+
+def test_training_step_with_the_charbonnier_loss(gs):
+    """One TrainStep iteration with the Charbonnier loss: its loss value is the
+    oracle's for the same render, and the update moves parameters as the
+    oracle's backward + Adam of that loss does."""
+    native, model = gs
+    s = scenes.small()
+    cam = s.cameras[0]
+    target = scenes.uniform_image(cam.height, cam.width, seed=9)
+    m = model.GaussianModel(s)
+    step = model.TrainStep(m, 200_000, cam.width, cam.height, loss="charbonnier")
+    loss = step(cam, dev(target))
+    torch.cuda.synchronize()
+    o = oracle.Oracle(s, cam)
+    r = o.render()
+    L, dimg, _, _ = oracle.charbonnier_loss(r["image"].astype(np.float32), target, [1, 1, 1], [0, 0, 0])
+    assert host(loss)[0] == pytest.approx(L, rel=1e-4)
+    ref = o.backward(dimg)
+    for k in scenes.GROUP_NAMES:
+        p0 = getattr(s, k).astype(np.float64)
+        rp, _, _, _ = oracle.adam(p0, ref[k], np.zeros_like(p0), np.zeros_like(p0), 1e-3, 1)
+        upd_ref = (rp.reshape(p0.shape) - p0)[..., : s.n]
+        upd = (host(m.params[k]).astype(np.float64) - p0)[..., : s.n]
+        big = np.abs(ref[k][..., : s.n]) > 1e-3 * np.abs(ref[k][..., : s.n]).max()
+        assert np.mean(np.abs(upd[big] - upd_ref[big]) <= 1e-6) > 0.99, k
