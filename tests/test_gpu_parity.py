@@ -39,7 +39,7 @@ def host(t):
     return t.detach().cpu().numpy()
 
 
-class GpuRun:
+class DeviceRun:
     """Preprocess + forward of one scene/camera through the C ABI."""
 
     def __init__(self, native, model, scene, cam, max_entries=None, active_degree=None, opacity_rect=False):
@@ -105,7 +105,7 @@ SCENES = {"tiny": lambda: (scenes.tiny(), 0), "small": lambda: (scenes.small(), 
 def test_preprocess_matches_oracle(gs, name):
     native, model = gs
     s, ci = SCENES[name]()
-    run = GpuRun(native, model, s, s.cameras[ci])
+    run = DeviceRun(native, model, s, s.cameras[ci])
     g = run.preprocess_out()
     o = run.oracle.preprocess()
     np.testing.assert_array_equal(g["touched"], o["touched"])
@@ -126,7 +126,7 @@ def test_preprocess_matches_oracle(gs, name):
 def test_sort_and_ranges_bit_exact(gs, name):
     native, model = gs
     s, ci = SCENES[name]()
-    run = GpuRun(native, model, s, s.cameras[ci])
+    run = DeviceRun(native, model, s, s.cameras[ci])
     ids, tiles, ranges = run.sorted_out()
     o = run.oracle.sorted()
     assert run.K == o["ids"].size
@@ -152,7 +152,7 @@ def check_pixels(run, o_render):
 def test_forward_pixels_match_oracle(gs, name):
     native, model = gs
     s, ci = SCENES[name]()
-    run = GpuRun(native, model, s, s.cameras[ci])
+    run = DeviceRun(native, model, s, s.cameras[ci])
     check_pixels(run, run.oracle.render())
 
 
@@ -162,7 +162,7 @@ def test_forward_ragged_image_and_background(gs):
     native, model = gs
     s = scenes.small(seed=3)
     cam = scenes.look_at((0.4, 0.3, -3.2), (0.0, 0.0, 0.0), 150, 93, 140.0, bg=(0.2, 0.5, 0.9))
-    run = GpuRun(native, model, s, cam, active_degree=1)
+    run = DeviceRun(native, model, s, cam, active_degree=1)
     check_pixels(run, run.oracle.render())
     ids, _, ranges = run.sorted_out()
     o = run.oracle.sorted()
@@ -175,7 +175,7 @@ def test_empty_and_fully_culled_scenes(gs):
     cam = scenes.identity_camera(40, 24, 30.0, bg=(0.1, 0.2, 0.3))
     s = scenes.tiny()
     s.means[2, :] = -1.0  # every Gaussian behind the camera
-    run = GpuRun(native, model, s, cam)
+    run = DeviceRun(native, model, s, cam)
     assert run.K == 0
     img = host(run.image)
     for c in range(3):
@@ -261,7 +261,7 @@ def test_backward_matches_oracle(gs, name):
     native, model = gs
     s, ci = SCENES[name]()
     cam = s.cameras[ci]
-    run = GpuRun(native, model, s, cam)
+    run = DeviceRun(native, model, s, cam)
     r = run.oracle.render()
     target = scenes.uniform_image(cam.height, cam.width, seed=7)
     _, _, _, dimg = oracle.loss(r["image"].astype(np.float32), target, 0.2)
@@ -410,7 +410,7 @@ def test_opacity_aware_rect_path_matches_oracle(gs, name):
     native, model = gs
     s, ci = SCENES[name]()
     cam = s.cameras[ci]
-    run = GpuRun(native, model, s, cam, opacity_rect=True)
+    run = DeviceRun(native, model, s, cam, opacity_rect=True)
     g = run.preprocess_out()
     o = run.oracle.preprocess()
     np.testing.assert_array_equal(g["touched"], o["touched"])
@@ -421,7 +421,7 @@ def test_opacity_aware_rect_path_matches_oracle(gs, name):
     np.testing.assert_array_equal(ids, srt["ids"])
     np.testing.assert_array_equal(tiles, srt["tiles"])
     np.testing.assert_array_equal(ranges.astype(np.int64), srt["ranges"])
-    assert run.K < GpuRun(native, model, s, cam).K
+    assert run.K < DeviceRun(native, model, s, cam).K
     r = run.oracle.render()
     check_pixels(run, r)
     target = scenes.uniform_image(cam.height, cam.width, seed=7)
@@ -455,7 +455,7 @@ def test_deterministic_backward_is_bitwise_reproducible_and_matches_oracle(gs):
     target = scenes.uniform_image(cam.height, cam.width, seed=7)
     outs = []
     for _ in range(2):
-        run = GpuRun(native, model, s, cam)
+        run = DeviceRun(native, model, s, cam)
         run.ctx.set_option(native.GS_OPTION_DETERMINISTIC, 1)
         run.ctx.preprocess(run.m.params_struct(), run.cs)
         run.K = run.ctx.render_forward(run.cs, run.image, run.T, run.nc)
