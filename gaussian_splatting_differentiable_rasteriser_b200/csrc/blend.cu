@@ -221,8 +221,9 @@ struct WarpBatch {
 // mode, an integer atomic of v in 2^-40 fixed point (integer sums do not
 // depend on the order the warps arrive in, so the result is bitwise
 // reproducible; |v| is clamped to 2^22, far above any screen-gradient sum).
+template <bool kFixed>
 __device__ __forceinline__ void add_sum(float* dst, unsigned long long* fdst, int r, float v) {
-  if (fdst) {
+  if (kFixed) {
     const double q = fmin(fmax(static_cast<double>(v) * kFixedScale, -kFixedClamp), kFixedClamp);
     atomicAdd(fdst + r, static_cast<unsigned long long>(__double2ll_rn(q)));
   } else {
@@ -230,6 +231,7 @@ __device__ __forceinline__ void add_sum(float* dst, unsigned long long* fdst, in
   }
 }
 
+template <bool kFixed>
 __device__ __forceinline__ void flush_batch(const WarpBatch& b, int cnt, int lane, float cxb, float cyb,
                                             float* sgrad, unsigned long long* sgrad_fixed) {
   const int j = lane & 15, h = lane >> 4;
@@ -274,19 +276,19 @@ __device__ __forceinline__ void flush_batch(const WarpBatch& b, int cnt, int lan
     const float2 uv = b.uv[j];
     const float a = uv.x - cxb, bb = uv.y - cyb;
     float* dst = sgrad + static_cast<int64_t>(b.id[j]) * kGradStride;
-    unsigned long long* fdst = sgrad_fixed ? sgrad_fixed + static_cast<int64_t>(b.id[j]) * kFixedStride : nullptr;
+    unsigned long long* fdst = kFixed ? sgrad_fixed + static_cast<int64_t>(b.id[j]) * kFixedStride : nullptr;
     if (h == 0) {
       const float sy = __fmaf_rn(-bb, m0, my);
-      add_sum(dst, fdst, 0, m0);
-      add_sum(dst, fdst, 1, __fmaf_rn(-a, m0, mx));
-      add_sum(dst, fdst, 2, sy);
-      add_sum(dst, fdst, 3, __fmaf_rn(a, __fmaf_rn(a, m0, -2.0f * mx), mxx));
-      add_sum(dst, fdst, 4, __fmaf_rn(-a, sy, __fmaf_rn(-bb, mx, mxy)));
+      add_sum<kFixed>(dst, fdst, 0, m0);
+      add_sum<kFixed>(dst, fdst, 1, __fmaf_rn(-a, m0, mx));
+      add_sum<kFixed>(dst, fdst, 2, sy);
+      add_sum<kFixed>(dst, fdst, 3, __fmaf_rn(a, __fmaf_rn(a, m0, -2.0f * mx), mxx));
+      add_sum<kFixed>(dst, fdst, 4, __fmaf_rn(-a, sy, __fmaf_rn(-bb, mx, mxy)));
     } else {
-      add_sum(dst, fdst, 5, __fmaf_rn(bb, __fmaf_rn(bb, m0, -2.0f * my), myy));
-      add_sum(dst, fdst, 6, c0);
-      add_sum(dst, fdst, 7, c1);
-      add_sum(dst, fdst, 8, c2);
+      add_sum<kFixed>(dst, fdst, 5, __fmaf_rn(bb, __fmaf_rn(bb, m0, -2.0f * my), myy));
+      add_sum<kFixed>(dst, fdst, 6, c0);
+      add_sum<kFixed>(dst, fdst, 7, c1);
+      add_sum<kFixed>(dst, fdst, 8, c2);
     }
   }
 }
@@ -296,7 +298,7 @@ struct BackwardSmem {
   WarpBatch batches[kWarps];
 };
 
-template <bool kCount>
+template <bool kCount, bool kFixed>
 __global__ void __launch_bounds__(256) blend_backward_kernel(BlendArgs a) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   BackwardSmem& sm = *reinterpret_cast<BackwardSmem*>(smem_raw);
@@ -391,14 +393,14 @@ __global__ void __launch_bounds__(256) blend_backward_kernel(BlendArgs a) {
       }
       if (++bcnt == kBatch) {
         __syncwarp();
-        flush_batch(wb, kBatch, lane, bx0 + 3.5f, by0 + 1.5f, a.sgrad, a.sgrad_fixed);
+        flush_batch<kFixed>(wb, kBatch, lane, bx0 + 3.5f, by0 + 1.5f, a.sgrad, a.sgrad_fixed);
         bcnt = 0;
         __syncwarp();
       }
     }
     __syncwarp();  // the slots are rewritten by the next chunk
   }
-  if (bcnt > 0) flush_batch(wb, bcnt, lane, bx0 + 3.5f, by0 + 1.5f, a.sgrad, a.sgrad_fixed);
+  if (bcnt > 0) flush_batch<kFixed>(wb, bcnt, lane, bx0 + 3.5f, by0 + 1.5f, a.sgrad, a.sgrad_fixed);
   if (kCount) {
     // the method's backward walk visits every entry before the pixel's last contributor
     count_pairs(a.pairs, static_cast<unsigned>(min(last, static_cast<int>(range.y - range.x))));
@@ -437,23 +439,24 @@ cudaError_t launch_blend_forward(const BlendArgs& a, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+template <bool kCount, bool kFixed>
+cudaError_t launch_backward_variant(const BlendArgs& a, int tiles, cudaStream_t st) {
+  const int smem = static_cast<int>(sizeof(BackwardSmem));
+  cudaError_t e = cudaFuncSetAttribute(blend_backward_kernel<kCount, kFixed>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  blend_backward_kernel<kCount, kFixed><<<tiles, 256, smem, st>>>(a);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_blend_backward(const BlendArgs& a, cudaStream_t st) {
   const int tiles = a.cam.tiles_x * a.cam.tiles_y;
   if (tiles == 0) return cudaSuccess;
-  const int smem = static_cast<int>(sizeof(BackwardSmem));
-  cudaError_t e;
-  if (a.pairs) {
-    if ((e = cudaFuncSetAttribute(blend_backward_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  smem)) != cudaSuccess)
-      return e;
-    blend_backward_kernel<true><<<tiles, 256, smem, st>>>(a);
-  } else {
-    if ((e = cudaFuncSetAttribute(blend_backward_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  smem)) != cudaSuccess)
-      return e;
-    blend_backward_kernel<false><<<tiles, 256, smem, st>>>(a);
-  }
-  return cudaGetLastError();
+  if (a.pairs)
+    return a.sgrad_fixed ? launch_backward_variant<true, true>(a, tiles, st)
+                         : launch_backward_variant<true, false>(a, tiles, st);
+  return a.sgrad_fixed ? launch_backward_variant<false, true>(a, tiles, st)
+                       : launch_backward_variant<false, false>(a, tiles, st);
 }
 
 }  // namespace gs

@@ -45,8 +45,9 @@ struct GaussGrad {
 
 // Density-control statistics of a Gaussian this view touched: the norm of
 // dL/dmean2d and one more view (one thread per Gaussian: no atomics needed).
+template <bool kStats>
 __device__ __forceinline__ void add_densify_stats(const PreprocessBwdArgs& a, int64_t i, const GaussGrad& g) {
-  if (a.stat_accum) {
+  if (kStats) {
     a.stat_accum[i] += sqrtf(g.du * g.du + g.dv * g.dv);
     a.stat_count[i] += 1u;
   }
@@ -204,14 +205,14 @@ __device__ __forceinline__ void add_view_dir_term(GaussGrad& g, const float (&ws
 }
 
 // Backward that ADDS the gradient into the caller's buffers.
-template <int kDeg>
+template <int kDeg, bool kStats>
 __global__ void __launch_bounds__(256) preprocess_backward_kernel(PreprocessBwdArgs a) {
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i >= a.n || a.touched[i] == 0) return;
   const int64_t np = a.n_pad;
   GaussGrad g;
   geometry_grad(a, i, g);
-  add_densify_stats(a, i, g);
+  add_densify_stats<kStats>(a, i, g);
   constexpr int nk = (kDeg + 1) * (kDeg + 1);
   float Yk[16];
   sh_basis(kDeg, g.vx, g.vy, g.vz, Yk);
@@ -275,7 +276,7 @@ struct FusedSmem {
 // kAccum: the caller's gradient buffer holds an accumulated gradient, which is
 // added and then zeroed; without it the update uses this view's gradient alone
 // and no gradient buffer is read or written (24 instead of 32 bytes per scalar).
-template <int kDeg, bool kAccum>
+template <int kDeg, bool kAccum, bool kStats>
 __global__ void __launch_bounds__(kFusedBlock) preprocess_backward_adam_kernel(PreprocessBwdArgs a,
                                                                               FusedAdamArgs f) {
   __shared__ __align__(16) FusedSmem sm;
@@ -291,7 +292,7 @@ __global__ void __launch_bounds__(kFusedBlock) preprocess_backward_adam_kernel(P
     if (visible) {
       GaussGrad g;
       geometry_grad(a, i, g);
-      add_densify_stats(a, i, g);
+      add_densify_stats<kStats>(a, i, g);
       float Yk[16];
       sh_basis(kDeg, g.vx, g.vy, g.vz, Yk);
       float wsum[16];
@@ -415,38 +416,49 @@ __global__ void screen_grads_kernel(const Screen* screen, const float* sgrad, in
 
 }  // namespace
 
+// The kernels are instantiated per active SH degree and per option (an
+// accumulated gradient buffer, density statistics), so the default path
+// carries no runtime test of either.
+template <int kDeg>
+cudaError_t launch_bwd_deg(const PreprocessBwdArgs& a, unsigned grid, cudaStream_t st) {
+  if (a.stat_accum)
+    preprocess_backward_kernel<kDeg, true><<<grid, 256, 0, st>>>(a);
+  else
+    preprocess_backward_kernel<kDeg, false><<<grid, 256, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+template <int kDeg>
+cudaError_t launch_fused_deg(const PreprocessBwdArgs& a, const FusedAdamArgs& f, unsigned grid, cudaStream_t st) {
+  const bool accum = f.g[0] != nullptr, stats = a.stat_accum != nullptr;
+  if (accum && stats) preprocess_backward_adam_kernel<kDeg, true, true><<<grid, kFusedBlock, 0, st>>>(a, f);
+  else if (accum) preprocess_backward_adam_kernel<kDeg, true, false><<<grid, kFusedBlock, 0, st>>>(a, f);
+  else if (stats) preprocess_backward_adam_kernel<kDeg, false, true><<<grid, kFusedBlock, 0, st>>>(a, f);
+  else preprocess_backward_adam_kernel<kDeg, false, false><<<grid, kFusedBlock, 0, st>>>(a, f);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_preprocess_backward(const PreprocessBwdArgs& a, cudaStream_t st) {
   if (a.n == 0) return cudaSuccess;
   const unsigned grid = static_cast<unsigned>((a.n + 255) / 256);
   switch (a.active_degree) {
-    case 0: preprocess_backward_kernel<0><<<grid, 256, 0, st>>>(a); break;
-    case 1: preprocess_backward_kernel<1><<<grid, 256, 0, st>>>(a); break;
-    case 2: preprocess_backward_kernel<2><<<grid, 256, 0, st>>>(a); break;
-    default: preprocess_backward_kernel<3><<<grid, 256, 0, st>>>(a); break;
+    case 0: return launch_bwd_deg<0>(a, grid, st);
+    case 1: return launch_bwd_deg<1>(a, grid, st);
+    case 2: return launch_bwd_deg<2>(a, grid, st);
+    default: return launch_bwd_deg<3>(a, grid, st);
   }
-  return cudaGetLastError();
 }
 
 cudaError_t launch_preprocess_backward_adam(const PreprocessBwdArgs& a, const FusedAdamArgs& f,
                                            cudaStream_t st) {
   if (a.n_pad == 0) return cudaSuccess;
   const unsigned grid = static_cast<unsigned>((a.n_pad + kFusedBlock - 1) / kFusedBlock);
-  if (f.g[0]) {
-    switch (a.active_degree) {
-      case 0: preprocess_backward_adam_kernel<0, true><<<grid, kFusedBlock, 0, st>>>(a, f); break;
-      case 1: preprocess_backward_adam_kernel<1, true><<<grid, kFusedBlock, 0, st>>>(a, f); break;
-      case 2: preprocess_backward_adam_kernel<2, true><<<grid, kFusedBlock, 0, st>>>(a, f); break;
-      default: preprocess_backward_adam_kernel<3, true><<<grid, kFusedBlock, 0, st>>>(a, f); break;
-    }
-  } else {
-    switch (a.active_degree) {
-      case 0: preprocess_backward_adam_kernel<0, false><<<grid, kFusedBlock, 0, st>>>(a, f); break;
-      case 1: preprocess_backward_adam_kernel<1, false><<<grid, kFusedBlock, 0, st>>>(a, f); break;
-      case 2: preprocess_backward_adam_kernel<2, false><<<grid, kFusedBlock, 0, st>>>(a, f); break;
-      default: preprocess_backward_adam_kernel<3, false><<<grid, kFusedBlock, 0, st>>>(a, f); break;
-    }
+  switch (a.active_degree) {
+    case 0: return launch_fused_deg<0>(a, f, grid, st);
+    case 1: return launch_fused_deg<1>(a, f, grid, st);
+    case 2: return launch_fused_deg<2>(a, f, grid, st);
+    default: return launch_fused_deg<3>(a, f, grid, st);
   }
-  return cudaGetLastError();
 }
 
 cudaError_t launch_screen_grads(const Screen* screen, const float* sgrad, int64_t n, float* out,
