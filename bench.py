@@ -124,12 +124,20 @@ class ClockSampler:
         return out
 
 
-def dist_setup():
+def dist_setup(group_always=False):
+    """Rank, world size and device from the launcher's environment; a process group
+    when there is more than one rank (or always, for the data-parallel step, whose
+    collectives then run on one rank too)."""
     import torch
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
+    if world == 1 and group_always:
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        os.environ.setdefault("MASTER_PORT", str(free_port()))
+        os.environ.setdefault("RANK", "0")
+        os.environ.setdefault("WORLD_SIZE", "1")
+    if world > 1 or group_always:
         import datetime
         import torch.distributed as dist
         backend = "nccl" if torch.cuda.is_available() else "gloo"
@@ -141,6 +149,18 @@ def dist_setup():
     return world, rank, local
 
 
+def free_port():
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def dist_on():
+    import torch.distributed as dist
+    return dist.is_available() and dist.is_initialized()
+
+
 def replica_throughput(world, steps, seconds_max):
     """Whole-job iterations per second of `world` replicas that each ran `steps`
     iterations, the slowest taking `seconds_max`."""
@@ -148,7 +168,7 @@ def replica_throughput(world, steps, seconds_max):
 
 
 def barrier(world):
-    if world > 1:
+    if dist_on():
         import torch.distributed as dist
         dist.barrier()
 
@@ -165,7 +185,8 @@ def max_over_ranks(x, world):
 
 
 # ------------------------------------------------------------------ workload
-def build_workload(config, device, opacity_rect=False, deterministic=False, loss="l1_dssim"):
+def build_workload(config, device, opacity_rect=False, deterministic=False, loss="l1_dssim",
+                   data_parallel=False):
     import numpy as np
     import torch
 
@@ -178,8 +199,13 @@ def build_workload(config, device, opacity_rect=False, deterministic=False, loss
     H = max(c.height for c in cams)
     m = model.GaussianModel(pert, device=device)
     cap = max(1 << 20, 8 * scene.n)
-    step = model.TrainStep(m, cap, W, H, device=device, opacity_rect=opacity_rect,
-                           deterministic=deterministic, loss=loss)
+    if data_parallel:
+        from gaussian_splatting_differentiable_rasteriser_b200.data_parallel import DataParallelTrainStep
+        step = DataParallelTrainStep(m, cap, W, H, device=device, opacity_rect=opacity_rect,
+                                     deterministic=deterministic, loss=loss)
+    else:
+        step = model.TrainStep(m, cap, W, H, device=device, opacity_rect=opacity_rect,
+                               deterministic=deterministic, loss=loss)
     # targets: renders of the perturbed copy (forward only, before any timing)
     targets = torch.empty((len(cams), 3, H, W), dtype=torch.float32, device=device)
     kmax = 0
@@ -214,11 +240,12 @@ def time_device(step, cams, targets, sched, start, count, world):
 
 def profile_stages(step, cams, targets, sched, start, count):
     """Per-stage kernel times (library events) plus Adam (torch events: the
-    Adam launches are the only work between them on the current stream)."""
+    Adam launches are the only work between them on the current stream). For the
+    data-parallel step that stage is "exchange_adam": reduce-scatter, Adam on the
+    shard, all-gather."""
     import torch
 
     from gaussian_splatting_differentiable_rasteriser_b200 import native
-    from gaussian_splatting_differentiable_rasteriser_b200.scenes import GROUP_NAMES
 
     ctx = step.ctx
     ctx.profile_enable(True)
@@ -237,21 +264,20 @@ def profile_stages(step, cams, targets, sched, start, count):
         if step.fused_adam:
             step.backward_and_update(cs, T, nc, step.dimage)
             continue
-        ctx.render_backward(m.params_struct(), cs, T, nc, step.dimage, m.grads_struct())
         m.step_count += 1
+        ctx.render_backward(m.params_struct(), cs, T, nc, step.dimage, m.grads_struct())
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record()
-        for k in GROUP_NAMES:
-            native.adam_step(m.params[k], m.grads[k], m.m[k], m.v[k], step.lrs[k], m.step_count,
-                             step.betas[0], step.betas[1], step.eps)
+        step.update_from_grads()
         e1.record()
         torch.cuda.synchronize()
         adam_ms += e0.elapsed_time(e1)
-        adam_launches += len(GROUP_NAMES)
+        adam_launches += step.adam_launches
     prof = ctx.profile_read()
     ctx.profile_enable(False)
-    prof["adam"] = {"ms": adam_ms, "launches": adam_launches, "work": adam_launches and count * m.flat.numel()}
+    name = "exchange_adam" if hasattr(step, "param_pad") else "adam"
+    prof[name] = {"ms": adam_ms, "launches": adam_launches, "work": adam_launches and count * m.flat.numel()}
     return prof, ks
 
 
@@ -420,17 +446,16 @@ def main_ours(args):
 
     import __graft_entry__
 
-    world, rank, local = dist_setup()
+    world, rank, local = dist_setup(group_always=args.parallel == "dp")
     if rank == 0:
         __graft_entry__.build()
     barrier(world)
     from gaussian_splatting_differentiable_rasteriser_b200 import native, scenes
-    from gaussian_splatting_differentiable_rasteriser_b200.scenes import GROUP_NAMES
 
     native.load()
     device = f"cuda:{local}"
     scene, m, step, targets, kmax = build_workload(args.config, device, args.rect == "opacity",
-                                                   args.deterministic, args.loss)
+                                                   args.deterministic, args.loss, args.parallel == "dp")
     cams = scene.cameras
     sched = scenes.camera_schedule(len(cams), args.warmup + args.steps, seed=rank)
     # clocks are sampled from the start of the warm-up to the end of the timed region
@@ -465,8 +490,8 @@ def main_ours(args):
     # context launches (over the same steps), plus gs_adam_step per group when the
     # separate path is used
     steps_p = max(1, args.steps)
-    per_step = (sum(prof[k]["launches"] for k in prof if k != "adam") / steps_p +
-                (0 if step.fused_adam else len(GROUP_NAMES)))
+    per_step = (sum(prof[k]["launches"] for k in prof if k not in ("adam", "exchange_adam")) / steps_p +
+                (0 if step.fused_adam else step.adam_launches))
     gpu_launches = int(round(per_step * args.steps))
 
     # end to end: target streamed from pinned host memory each step, loss read back
@@ -485,7 +510,9 @@ def main_ours(args):
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": WORKLOADS[args.config], "gaussians": scene.n,
                        "width": W, "height": H, "cameras": len(cams),
-                       "parallelism": "replicas" if world > 1 else "single-gpu",
+                       "parallelism": ("data-parallel: one camera per rank, gradients reduce-scattered, "
+                                       "Adam sharded, parameters all-gathered" if args.parallel == "dp"
+                                       else "replicas" if world > 1 else "single-gpu"),
                        "tile_rect": "3 sigma" if args.rect == "3sigma" else "opacity-aware",
                        "gradient_sums": "fixed-point (deterministic)" if args.deterministic else "float32 atomics",
                        "loss": "L1 + D-SSIM (lambda 0.2)" if args.loss == "l1_dssim" else "Charbonnier + exposure",
@@ -503,7 +530,7 @@ def main_ours(args):
             "e2e": e2e, "gpu_launches": gpu_launches, "clocks": clk, "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
-    if world > 1:
+    if dist_on():
         import torch.distributed as dist
         dist.destroy_process_group()
 
@@ -515,7 +542,6 @@ def e2e_run(step, cams, targets, sched, args, world):
     import torch
 
     from gaussian_splatting_differentiable_rasteriser_b200 import native
-    from gaussian_splatting_differentiable_rasteriser_b200.scenes import GROUP_NAMES
 
     host_t = targets.cpu().pin_memory()
     dev_t = [torch.empty_like(targets[0]) for _ in range(2)]
@@ -721,6 +747,9 @@ def main():
                     help="fixed-point gradient atomics (bitwise-reproducible backward)")
     ap.add_argument("--loss", choices=("l1_dssim", "charbonnier"), default="l1_dssim",
                     help="photometric loss of the step")
+    ap.add_argument("--parallel", choices=("replicas", "dp"), default="replicas",
+                    help="N>1: independent replicas (default), or data-parallel training over cameras "
+                         "(one camera per rank per iteration; value counts camera-iterations)")
     ap.add_argument("--op", choices=("step", "densify"), default="step",
                     help="the training step (default) or one densification pass")
     args = ap.parse_args()

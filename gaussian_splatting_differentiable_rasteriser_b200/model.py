@@ -53,6 +53,17 @@ class GaussianModel:
             self.v[k] = self.v_flat[sl].view(shapes[k])
             off += sizes[k]
 
+    def attach_storage(self, flat, grad_flat):
+        """Moves the parameters and gradients into the given flat buffers (same size;
+        the current parameters must already be in `flat`) and rebuilds the group views."""
+        assert flat.numel() == self.flat.numel() and grad_flat.numel() == self.grad_flat.numel()
+        self.flat, self.grad_flat = flat, grad_flat
+        shapes = group_shapes(self.n_pad, self.sh_degree)
+        for k in GROUP_NAMES:
+            sl = self.slices[k]
+            self.params[k] = self.flat[sl].view(shapes[k])
+            self.grads[k] = self.grad_flat[sl].view(shapes[k])
+
     def densify(self, ctx, grad_accum, view_count, normals, grad_threshold, scale_threshold,
                 min_opacity, capacity=None):
         """One gs_densify pass into new buffers of `capacity` slots (default: room
@@ -168,6 +179,15 @@ class TrainStep:
                                           self.betas[0], self.betas[1], self.eps)
             return
         self.ctx.render_backward(m.params_struct(), cs, T, nc, dimg, m.grads_struct())
+        self.update_from_grads()
+
+    # gs_adam_step launches of one update_from_grads call
+    adam_launches = len(GROUP_NAMES)
+
+    def update_from_grads(self):
+        """Adam on every group from the gradient buffer (which it zeroes), at the
+        model's current step count."""
+        m = self.model
         for k in GROUP_NAMES:
             native.adam_step(m.params[k], m.grads[k], m.m[k], m.v[k], self.lrs[k], m.step_count,
                              self.betas[0], self.betas[1], self.eps)

@@ -1,0 +1,94 @@
+"""The data-parallel exchange step on the host with the gloo backend, world
+size 2: the reduce-scatter / sharded Adam / all-gather leaves both ranks with
+the parameters of one Adam step on the batch-mean gradient, as the float64
+oracle computes it on the whole buffer; plus the sharding arithmetic."""
+import os
+import socket
+import sys
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def test_shards_cover_the_buffer_once_and_stay_aligned():
+    sys.path.insert(0, ROOT)
+    from gaussian_splatting_differentiable_rasteriser_b200 import data_parallel as dp
+    for total in (1, 7, 4096, 10_003):
+        for world in (1, 2, 3, 8):
+            b = [dp.shard_bounds(total, world, r) for r in range(world)]
+            assert b[0][0] == 0 and b[-1][1] == dp.padded_size(total, world) >= total
+            assert all(b[r][1] == b[r + 1][0] for r in range(world - 1))
+            assert all(lo % dp.ALIGN == 0 and (hi - lo) == b[0][1] - b[0][0] for lo, hi in b)
+
+
+def _slices(sizes):
+    out, off = {}, 0
+    for k, n in sizes.items():
+        out[k] = slice(off, off + n)
+        off += n
+    return out, off
+
+
+def _rank(rank, world, port, out_dir):
+    os.environ.update(RANK=str(rank), WORLD_SIZE=str(world), MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    import oracle
+    from gaussian_splatting_differentiable_rasteriser_b200 import data_parallel as dp
+    from gaussian_splatting_differentiable_rasteriser_b200.scenes import GROUP_NAMES
+    dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+    sizes = dict(zip(GROUP_NAMES, (30, 30, 40, 10, 130)))
+    slices, total = _slices(sizes)
+    lrs = dict(zip(GROUP_NAMES, (1e-3, 2e-3, 5e-4, 1e-2, 1e-3)))
+    rng = np.random.default_rng(0)
+    p0 = rng.normal(size=total).astype(np.float32)
+    grads = [rng.normal(0, 1e-2, total).astype(np.float32) for _ in range(world)]
+    pad = dp.padded_size(total, world)
+    param_pad = torch.zeros(pad)
+    param_pad[:total] = torch.from_numpy(p0)
+    grad_pad = torch.zeros(pad)
+    grad_pad[:total] = torch.from_numpy(grads[rank])
+    m = torch.zeros(total)
+    v = torch.zeros(total)
+
+    def adam(p, g, mm, vv, k):  # the float64 oracle as the update, on the host
+        rp, _, rm, rv = oracle.adam(p.numpy(), g.numpy(), mm.numpy(), vv.numpy(), lrs[k], 1)
+        p.copy_(torch.from_numpy(rp.astype(np.float32)))
+        mm.copy_(torch.from_numpy(rm.astype(np.float32)))
+        vv.copy_(torch.from_numpy(rv.astype(np.float32)))
+        g.zero_()
+
+    dp.exchange_and_update(grad_pad, param_pad, m, v, slices, total, world, rank, adam)
+    assert not grad_pad.any()
+    np.save(os.path.join(out_dir, f"p{rank}.npy"), param_pad[:total].numpy())
+    if rank == 0:
+        gmean = (grads[0].astype(np.float64) + grads[1].astype(np.float64)) / 2
+        ref = np.empty(total)
+        for k in GROUP_NAMES:
+            s = slices[k]
+            ref[s] = oracle.adam(p0[s], gmean[s].astype(np.float32), np.zeros(sizes[k]), np.zeros(sizes[k]),
+                                 lrs[k], 1)[0]
+        np.save(os.path.join(out_dir, "ref.npy"), ref)
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_exchange_matches_adam_on_the_batch_mean_gradient(tmp_path):
+    import torch.multiprocessing as mp
+    mp.start_processes(_rank, args=(2, free_port(), str(tmp_path)), nprocs=2, join=True, start_method="spawn")
+    p0, p1, ref = (np.load(tmp_path / f) for f in ("p0.npy", "p1.npy", "ref.npy"))
+    np.testing.assert_array_equal(p0, p1)
+    # the shard's mean gradient is float32 (g0 + g1) / 2: within a few float32 ulps of lr-sized steps
+    np.testing.assert_allclose(p0, ref, rtol=0, atol=1e-6)
