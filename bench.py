@@ -54,8 +54,8 @@ WORKLOADS = {
 # proportion. The fused pass's write counter undercounts: its last writes are still
 # in L2 when the kernel ends.
 NCU_TRAFFIC = {
-    "backward_adam": ((409.031424e6 + 290.892288e6) * 6.0, "2ade6b8bdb45"),
-    "blend_backward": ((85.229824e6 + 2.950144e6) * 6.32 / 1.064, "0758f6489db1"),
+    "backward_adam": ((408.091648e6 + 292.852480e6) * 6.0, "f1df474a7794"),
+    "blend_backward": ((85.319936e6 + 3.207936e6) * 6.32 / 1.064, "2dcc3feaade8"),
 }
 
 
@@ -186,7 +186,7 @@ def max_over_ranks(x, world):
 
 # ------------------------------------------------------------------ workload
 def build_workload(config, device, opacity_rect=False, deterministic=False, loss="l1_dssim",
-                   data_parallel=False):
+                   data_parallel=False, exchange="p2p"):
     import numpy as np
     import torch
 
@@ -202,7 +202,7 @@ def build_workload(config, device, opacity_rect=False, deterministic=False, loss
     if data_parallel:
         from gaussian_splatting_differentiable_rasteriser_b200.data_parallel import DataParallelTrainStep
         step = DataParallelTrainStep(m, cap, W, H, device=device, opacity_rect=opacity_rect,
-                                     deterministic=deterministic, loss=loss)
+                                     deterministic=deterministic, loss=loss, exchange=exchange)
     else:
         step = model.TrainStep(m, cap, W, H, device=device, opacity_rect=opacity_rect,
                                deterministic=deterministic, loss=loss)
@@ -302,6 +302,10 @@ def stage_models(scene, sh_k):
         "preprocess_backward": ("hbm", 4 * n_par * 3 + 48 + 48 + 5),
         # p, g, m, v read; p, m, v, g = 0 written, per scalar
         "adam": ("hbm", 32),
+        # the data-parallel exchange + Adam on one rank (gs_adam_step_reduce with one
+        # source, zeroing it): the same 32 B per scalar; with several ranks the stage
+        # also holds the two barriers and the NVLink transfers
+        "exchange_adam": ("hbm", 32),
         # fused projection backward + Adam with no accumulated gradient (one view per
         # step): p, m, v read and written, 24 B per scalar of every group, plus the raw
         # screen-gradient sums, the screen record and two flags, per Gaussian
@@ -455,7 +459,8 @@ def main_ours(args):
     native.load()
     device = f"cuda:{local}"
     scene, m, step, targets, kmax = build_workload(args.config, device, args.rect == "opacity",
-                                                   args.deterministic, args.loss, args.parallel == "dp")
+                                                   args.deterministic, args.loss, args.parallel == "dp",
+                                                   args.exchange)
     cams = scene.cameras
     sched = scenes.camera_schedule(len(cams), args.warmup + args.steps, seed=rank)
     # clocks are sampled from the start of the warm-up to the end of the timed region
@@ -482,7 +487,7 @@ def main_ours(args):
     src = {"blend_forward": "blend.cu", "blend_backward": "blend.cu", "adam": "adam.cu",
            "preprocess": "preprocess.cu", "sort": "sort.cu", "depth_sort": "sort.cu", "loss": "loss.cu",
            "preprocess_backward": "preprocess_backward.cu",
-           "backward_adam": "preprocess_backward.cu"}.get(dominant)
+           "backward_adam": "preprocess_backward.cu", "exchange_adam": "adam_reduce.cu"}.get(dominant)
     tr = NCU_TRAFFIC.get(dominant)
     rf["traffic"] = tr[0] if (tr and src and sha12(os.path.join(PKG_CSRC, src)) == tr[1]) else None
 
@@ -510,8 +515,11 @@ def main_ours(args):
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": WORKLOADS[args.config], "gaussians": scene.n,
                        "width": W, "height": H, "cameras": len(cams),
-                       "parallelism": ("data-parallel: one camera per rank, gradients reduce-scattered, "
-                                       "Adam sharded, parameters all-gathered" if args.parallel == "dp"
+                       "parallelism": (("data-parallel: one camera per rank; gradient exchange fused with "
+                                        "the sharded Adam over peer memory (gs_adam_step_reduce)"
+                                        if args.exchange == "p2p" else
+                                        "data-parallel: one camera per rank; NCCL reduce-scatter, "
+                                        "sharded Adam, NCCL all-gather") if args.parallel == "dp"
                                        else "replicas" if world > 1 else "single-gpu"),
                        "tile_rect": "3 sigma" if args.rect == "3sigma" else "opacity-aware",
                        "gradient_sums": "fixed-point (deterministic)" if args.deterministic else "float32 atomics",
@@ -530,6 +538,8 @@ def main_ours(args):
             "e2e": e2e, "gpu_launches": gpu_launches, "clocks": clk, "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
+    if hasattr(step, "close"):
+        step.close()
     if dist_on():
         import torch.distributed as dist
         dist.destroy_process_group()
@@ -750,6 +760,8 @@ def main():
     ap.add_argument("--parallel", choices=("replicas", "dp"), default="replicas",
                     help="N>1: independent replicas (default), or data-parallel training over cameras "
                          "(one camera per rank per iteration; value counts camera-iterations)")
+    ap.add_argument("--exchange", choices=("p2p", "nccl"), default="p2p",
+                    help="--parallel dp: the fused peer-memory exchange + Adam, or NCCL collectives")
     ap.add_argument("--op", choices=("step", "densify"), default="step",
                     help="the training step (default) or one densification pass")
     args = ap.parse_args()

@@ -688,6 +688,90 @@ gs_status gs_adam_step(float* param, float* grad, float* m, float* v, int64_t co
   return e == cudaSuccess ? GS_OK : GS_ERR_CUDA;
 }
 
+gs_status gs_adam_step_reduce(float* param, float* m, float* v, int64_t count, float* const* grads,
+                              int32_t n_grads, float* const* param_copies, int32_t n_copies,
+                              int32_t zero_grads, float grad_scale, float lr, float beta1, float beta2,
+                              float eps, int32_t step, void* stream) {
+  if (count < 0 || step < 1 || n_grads < 1 || n_grads > gs::kMaxRanks || n_copies < 0 ||
+      n_copies > gs::kMaxRanks || !grads || (n_copies > 0 && !param_copies))
+    return GS_ERR_INVALID_ARG;
+  if (!valid_betas(beta1, beta2, eps) || !std::isfinite(lr) || !std::isfinite(grad_scale))
+    return GS_ERR_INVALID_ARG;
+  gs::ReduceAdamArgs a{};
+  a.p = param;
+  a.m = m;
+  a.v = v;
+  a.count = count;
+  a.n_grads = n_grads;
+  a.n_copies = n_copies;
+  a.zero_grads = zero_grads != 0;
+  a.grad_scale = grad_scale;
+  a.s = gs::adam_scalars(lr, beta1, beta2, eps, step);
+  for (int r = 0; r < n_grads; ++r) a.grads[r] = grads[r];
+  for (int d = 0; d < n_copies; ++d) a.copies[d] = param_copies[d];
+  if (count > 0) {
+    if (!param || !m || !v || !aligned(param, 4) || !aligned(m, 4) || !aligned(v, 4)) return GS_ERR_INVALID_ARG;
+    for (int r = 0; r < n_grads; ++r)
+      if (!a.grads[r] || !aligned(a.grads[r], 4)) return GS_ERR_INVALID_ARG;
+    for (int d = 0; d < n_copies; ++d)
+      if (!a.copies[d] || !aligned(a.copies[d], 4)) return GS_ERR_INVALID_ARG;
+  }
+  const cudaError_t e = gs::launch_adam_reduce(a, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? GS_OK : GS_ERR_CUDA;
+}
+
+gs_status gs_shared_alloc(int64_t bytes, void** ptr, unsigned char* handle) {
+  if (bytes <= 0 || !ptr || !handle) return GS_ERR_INVALID_ARG;
+  *ptr = nullptr;
+  void* p = nullptr;
+  if (cudaMalloc(&p, static_cast<size_t>(bytes)) != cudaSuccess) {
+    cudaGetLastError();
+    return GS_ERR_CUDA;
+  }
+  cudaIpcMemHandle_t h;
+  if (cudaMemset(p, 0, static_cast<size_t>(bytes)) != cudaSuccess || cudaIpcGetMemHandle(&h, p) != cudaSuccess) {
+    cudaGetLastError();
+    cudaFree(p);
+    return GS_ERR_CUDA;
+  }
+  static_assert(sizeof(h) == GS_SHARED_HANDLE_BYTES, "IPC handle size");
+  std::memcpy(handle, &h, sizeof(h));
+  *ptr = p;
+  return GS_OK;
+}
+
+gs_status gs_shared_open(const unsigned char* handle, void** ptr) {
+  if (!handle || !ptr) return GS_ERR_INVALID_ARG;
+  *ptr = nullptr;
+  cudaIpcMemHandle_t h;
+  std::memcpy(&h, handle, sizeof(h));
+  void* p = nullptr;
+  if (cudaIpcOpenMemHandle(&p, h, cudaIpcMemLazyEnablePeerAccess) != cudaSuccess) {
+    cudaGetLastError();
+    return GS_ERR_CUDA;
+  }
+  *ptr = p;
+  return GS_OK;
+}
+
+gs_status gs_shared_close(void* ptr) {
+  if (!ptr) return GS_ERR_INVALID_ARG;
+  if (cudaIpcCloseMemHandle(ptr) != cudaSuccess) {
+    cudaGetLastError();
+    return GS_ERR_CUDA;
+  }
+  return GS_OK;
+}
+
+gs_status gs_shared_free(void* ptr) {
+  if (!ptr) return GS_ERR_INVALID_ARG;
+  if (cudaFree(ptr) != cudaSuccess) {
+    cudaGetLastError();
+    return GS_ERR_CUDA;
+  }
+  return GS_OK;
+}
+
 gs_status gs_profile_enable(gs_ctx* c, int32_t enabled) {
   if (!c) return GS_ERR_INVALID_ARG;
   auto& P = c->prof;

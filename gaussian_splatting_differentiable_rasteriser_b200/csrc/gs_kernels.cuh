@@ -235,4 +235,23 @@ cudaError_t launch_opacity_reset(float* logits, float* m, float* v, int64_t n, f
 cudaError_t launch_adam(float* p, float* g, float* m, float* v, int64_t count, float lr,
                         float beta1, float beta2, float eps, int step, cudaStream_t st);
 
+// ------------------------------------------- data-parallel exchange + Adam
+constexpr int kMaxRanks = 8;  // GPUs of one NVSwitch node
+
+struct ReduceAdamArgs {
+  float* p;  // this rank's shard: parameters and moments, updated in place
+  float* m;
+  float* v;
+  int64_t count;
+  float* grads[kMaxRanks];   // every rank's gradient at this shard (local or peer memory)
+  int n_grads;
+  float* copies[kMaxRanks];  // other ranks' parameter buffers at this shard (peer memory)
+  int n_copies;
+  int zero_grads;            // write zeros to every gradient source after reading it
+  float grad_scale;          // 1 / ranks: the mean gradient
+  AdamScalars s;
+};
+
+cudaError_t launch_adam_reduce(const ReduceAdamArgs& a, cudaStream_t st);
+
 }  // namespace gs

@@ -70,29 +70,89 @@ def exchange_and_update(grad_pad, param_pad, m_flat, v_flat, slices, total, worl
     grad_pad.zero_()
 
 
-class DataParallelTrainStep(TrainStep):
-    """TrainStep whose update is the data-parallel one: the backward writes this
-    rank's gradient (gs_render_backward), then exchange_and_update runs the
-    reduce-scatter, Adam on this rank's shard (gs_adam_step) and the all-gather.
-    The model's parameter and gradient buffers are moved into padded storage so
-    the collectives work in place. With torch.distributed initialised the
-    collectives run even for one rank; without it the step is the single-GPU one.
-    Densification reallocates the model's buffers: build a new step after it."""
+def p2p_pieces(slices, total, world, rank, param_ptrs, grad_ptrs):
+    """The gs_adam_step_reduce calls of one rank: for each parameter-group piece
+    of its shard, (group, start, stop, gradient source addresses in rank order,
+    addresses of the other ranks' parameter copies). Addresses are those of
+    each rank's padded float32 buffer."""
+    lo, hi = shard_bounds(total, world, rank)
+    out = []
+    for k, a, b in group_pieces(slices, lo, min(hi, total)):
+        out.append((k, a, b, [g + 4 * a for g in grad_ptrs],
+                    [p + 4 * a for r, p in enumerate(param_ptrs) if r != rank]))
+    return out
 
-    def __init__(self, model, max_entries, width, height, group=None, **kw):
+
+class DataParallelTrainStep(TrainStep):
+    """TrainStep whose update is the data-parallel one. The backward writes this
+    rank's gradient (gs_render_backward); then, with exchange="p2p" (default),
+    one gs_adam_step_reduce launch per parameter group in this rank's shard
+    reads every rank's gradient of the shard from peer memory, averages it in
+    rank order, runs Adam and writes the updated shard into every rank's
+    parameters; with exchange="nccl", exchange_and_update runs NCCL's
+    reduce-scatter, gs_adam_step on the shard and NCCL's all-gather.
+
+    The parameter and gradient buffers are padded so every rank's shard has
+    the same size and 16-byte-aligned bounds; for "p2p" they are shared
+    (gs_shared_alloc) and mapped by every other rank. With torch.distributed
+    initialised the exchange runs even for one rank; without it the step is the
+    single-GPU one. Densification reallocates the model's buffers: build a new
+    step after it. Call close() on every rank before the step is dropped."""
+
+    def __init__(self, model, max_entries, width, height, group=None, exchange="p2p", **kw):
+        if exchange not in ("p2p", "nccl"):
+            raise ValueError("exchange must be 'p2p' or 'nccl'")
         kw["fused_adam"] = False
         super().__init__(model, max_entries, width, height, **kw)
         self.group = group
+        self.exchange = exchange
         on = dist.is_available() and dist.is_initialized()
         self.world = dist.get_world_size(group) if on else 1
         self.rank = dist.get_rank(group) if on else 0
+        if self.world > native.MAX_RANKS:
+            raise ValueError(f"at most {native.MAX_RANKS} ranks (one node)")
         self.total = model.flat.numel()
         pad = padded_size(self.total, self.world)
         dev = model.flat.device
-        self.param_pad = torch.zeros(pad, dtype=torch.float32, device=dev)
-        self.grad_pad = torch.zeros(pad, dtype=torch.float32, device=dev)
+        self._peer_maps = []
+        if exchange == "p2p":
+            self._bufs = (native.SharedBuffer(pad), native.SharedBuffer(pad))
+            self.param_pad, self.grad_pad = self._bufs[0].tensor, self._bufs[1].tensor
+            mine = (self._bufs[0].ptr, self._bufs[1].ptr)
+            if self.world > 1:
+                handles = [None] * self.world
+                dist.all_gather_object(handles, (self._bufs[0].handle, self._bufs[1].handle), group=group)
+                ptrs = []
+                for r, (hp, hg) in enumerate(handles):
+                    if r == self.rank:
+                        ptrs.append(mine)
+                    else:
+                        pair = (native.shared_open(hp), native.shared_open(hg))
+                        self._peer_maps.extend(pair)
+                        ptrs.append(pair)
+            else:
+                ptrs = [mine]
+            self.param_ptrs = [p for p, _ in ptrs]
+            self.grad_ptrs = [g for _, g in ptrs]
+        else:
+            self.param_pad = torch.zeros(pad, dtype=torch.float32, device=dev)
+            self.grad_pad = torch.zeros(pad, dtype=torch.float32, device=dev)
         self.param_pad[: self.total].copy_(model.flat)
         model.attach_storage(self.param_pad[: self.total], self.grad_pad[: self.total])
+        self._flag = torch.zeros(1, dtype=torch.float32, device=dev)
+        self._nccl = on and dist.get_backend(group) == "nccl"
+
+    def _barrier(self):
+        """Every rank's work enqueued so far is complete before anything enqueued after
+        it runs: a one-float all-reduce on the stream (NCCL), or a device
+        synchronise plus a host barrier (other backends)."""
+        if self.world == 1:
+            return
+        if self._nccl:
+            dist.all_reduce(self._flag, group=self.group)
+        else:
+            torch.cuda.synchronize()
+            dist.barrier(group=self.group)
 
     @property
     def adam_launches(self):
@@ -100,12 +160,34 @@ class DataParallelTrainStep(TrainStep):
         return len(group_pieces(self.model.slices, lo, min(hi, self.total)))
 
     def update_from_grads(self):
-        """Reduce-scatter, Adam on this rank's shard, all-gather."""
+        """The exchange and the Adam step of this rank's shard."""
         m = self.model
         step = m.step_count
+        b1, b2 = self.betas
+        if self.exchange == "nccl":
+            def adam(p, g, mm, vv, k):
+                native.adam_step(p, g, mm, vv, self.lrs[k], step, b1, b2, self.eps)
 
-        def adam(p, g, mm, vv, k):
-            native.adam_step(p, g, mm, vv, self.lrs[k], step, self.betas[0], self.betas[1], self.eps)
+            exchange_and_update(self.grad_pad, self.param_pad, m.m_flat, m.v_flat, m.slices, self.total,
+                                self.world, self.rank, adam, self.group)
+            return
+        self._barrier()  # every rank's gradient is complete
+        one = self.world == 1
+        for k, a, b, gsrc, copies in p2p_pieces(m.slices, self.total, self.world, self.rank,
+                                                self.param_ptrs, self.grad_ptrs):
+            native.adam_step_reduce(self.param_pad[a:b], m.m_flat[a:b], m.v_flat[a:b], gsrc, copies,
+                                    self.lrs[k], step, grad_scale=1.0 / self.world, zero_grads=one,
+                                    beta1=b1, beta2=b2, eps=self.eps)
+        if not one:
+            self._barrier()  # every shard is read and every copy written
+            self.grad_pad.zero_()
 
-        exchange_and_update(self.grad_pad, self.param_pad, m.m_flat, m.v_flat, m.slices, self.total,
-                            self.world, self.rank, adam, self.group)
+    def close(self):
+        """Unmaps the other ranks' buffers; collective when there are several ranks
+        (no rank frees its buffers while another still maps them)."""
+        if self._peer_maps:
+            self._barrier()
+            for p in self._peer_maps:
+                native.shared_close(p)
+            self._peer_maps = []
+            self._barrier()

@@ -25,7 +25,11 @@ EXPORTED = ("gs_create", "gs_destroy", "gs_last_error", "gs_preprocess", "gs_ren
             "gs_profile_enable",
             "gs_profile_read", "gs_stage_name", "gs_debug_preprocess", "gs_debug_sorted",
             "gs_debug_screen_grads", "gs_set_option", "gs_loss_l1_dssim_noalloc",
-            "gs_set_densify_stats", "gs_densify", "gs_opacity_reset", "gs_loss_charbonnier")
+            "gs_set_densify_stats", "gs_densify", "gs_opacity_reset", "gs_loss_charbonnier",
+            "gs_adam_step_reduce", "gs_shared_alloc", "gs_shared_open", "gs_shared_close",
+            "gs_shared_free")
+GS_SHARED_HANDLE_BYTES = 64
+MAX_RANKS = 8
 GS_OPTION_OPACITY_RECT = 1
 GS_OPTION_DETERMINISTIC = 2
 STAGES = ("preprocess", "scan", "duplicate", "sort", "ranges", "blend_forward", "loss",
@@ -93,6 +97,12 @@ def load(path: str = LIB_PATH):
                              ctypes.POINTER(GsGrads), I64, ctypes.POINTER(I64), P]
     L.gs_opacity_reset.argtypes = [P, P, P, I64, F, P]
     L.gs_loss_charbonnier.argtypes = [P, P, P, I32, I32, ctypes.POINTER(F), ctypes.POINTER(F), F, P, P, P]
+    PP = ctypes.POINTER(P)
+    L.gs_adam_step_reduce.argtypes = [P, P, P, I64, PP, I32, PP, I32, I32, F, F, F, F, F, I32, P]
+    L.gs_shared_alloc.argtypes = [I64, PP, ctypes.c_char_p]
+    L.gs_shared_open.argtypes = [ctypes.c_char_p, PP]
+    L.gs_shared_close.argtypes = [P]
+    L.gs_shared_free.argtypes = [P]
     L.gs_set_option.argtypes = [P, I32, I32]
     L.gs_set_option.restype = ctypes.c_int
     L.gs_loss_l1_dssim_noalloc.argtypes = [P, P, I32, I32, F, P, P, P]
@@ -250,6 +260,72 @@ def adam_step(param, grad, m, v, lr, step, beta1=0.9, beta2=0.999, eps=1e-8, str
                         float(beta1), float(beta2), float(eps), int(step), _stream(stream))
     if st != GS_OK:
         raise GsError(st, "gs_adam_step rejected its arguments")
+
+
+def adam_step_reduce(param, m, v, grads, copies, lr, step, grad_scale=None, zero_grads=False, beta1=0.9,
+                     beta2=0.999, eps=1e-8, stream=None):
+    """gs_adam_step_reduce over the tensors param, m, v (this rank's piece of its
+    shard). grads / copies: device addresses (ints) of the same piece in every
+    rank's gradient buffer and in the other ranks' parameter buffers. grad_scale
+    defaults to 1 / len(grads)."""
+    L = load()
+    if not 1 <= len(grads) <= MAX_RANKS or len(copies) > MAX_RANKS:
+        raise ValueError(f"1..{MAX_RANKS} gradient sources and at most {MAX_RANKS} copies")
+    scale = 1.0 / len(grads) if grad_scale is None else float(grad_scale)
+    g = (ctypes.c_void_p * max(1, len(grads)))(*[ctypes.c_void_p(int(x)) for x in grads])
+    c = (ctypes.c_void_p * max(1, len(copies)))(*[ctypes.c_void_p(int(x)) for x in copies])
+    st = L.gs_adam_step_reduce(_ptr(param), _ptr(m), _ptr(v), param.numel(), g, len(grads), c, len(copies),
+                               int(bool(zero_grads)), scale, float(lr), float(beta1), float(beta2), float(eps),
+                               int(step), _stream(stream))
+    if st != GS_OK:
+        raise GsError(st, "gs_adam_step_reduce rejected its arguments")
+
+
+class SharedBuffer:
+    """float32 device memory that other processes can map (gs_shared_alloc), freed
+    with the object. `.tensor` is a torch view of it; `.handle` the bytes to send
+    to the other ranks; `.ptr` its device address."""
+
+    def __init__(self, numel):
+        L = load()
+        self.numel = int(numel)
+        p = ctypes.c_void_p()
+        h = ctypes.create_string_buffer(GS_SHARED_HANDLE_BYTES)
+        st = L.gs_shared_alloc(4 * self.numel, ctypes.byref(p), h)
+        if st != GS_OK:
+            raise GsError(st, "gs_shared_alloc failed")
+        self.ptr = int(p.value)
+        self.handle = bytes(h.raw)
+        import torch
+        self.tensor = torch.as_tensor(self, device=f"cuda:{torch.cuda.current_device()}")
+
+    @property
+    def __cuda_array_interface__(self):
+        return {"shape": (self.numel,), "typestr": "<f4", "data": (self.ptr, False), "version": 3,
+                "strides": None}
+
+    def __del__(self):
+        if getattr(self, "ptr", 0) and _lib is not None:
+            _lib.gs_shared_free(ctypes.c_void_p(self.ptr))
+            self.ptr = 0
+
+
+def shared_open(handle: bytes) -> int:
+    """Maps another process's SharedBuffer from its handle; returns the device address."""
+    L = load()
+    if len(handle) != GS_SHARED_HANDLE_BYTES:
+        raise ValueError("bad handle size")
+    p = ctypes.c_void_p()
+    st = L.gs_shared_open(handle, ctypes.byref(p))
+    if st != GS_OK:
+        raise GsError(st, "gs_shared_open failed")
+    return int(p.value)
+
+
+def shared_close(ptr: int):
+    st = load().gs_shared_close(ctypes.c_void_p(int(ptr)))
+    if st != GS_OK:
+        raise GsError(st, "gs_shared_close failed")
 
 
 def opacity_reset(logits, m, v, max_opacity=0.01, stream=None):

@@ -251,6 +251,52 @@ gs_status gs_render_backward_adam(gs_ctx *ctx, const gs_params *params, const gs
 gs_status gs_adam_step(float *param, float *grad, float *m, float *v, int64_t count, float lr,
                        float beta1, float beta2, float eps, int32_t step, void *stream);
 
+/* ------------------------------------------- data-parallel training ------
+ * Several GPUs of one node train one set of Gaussians, each rendering its own
+ * camera of the iteration ([GS] "Per step": one photo per step; with R
+ * ranks the batch gradient is the mean of the R per-rank gradients). Each
+ * rank owns a contiguous shard of the flat parameter buffer, the only part
+ * whose Adam moments it keeps.
+ *
+ * Step 5, data-parallel form - the gradient exchange fused with Adam over
+ * one rank's shard (one parameter group's part of it, so each group keeps its
+ * own lr): g = grad_scale * (grads[0][i] + ... + grads[n_grads-1][i]) summed
+ * in that order (bitwise the same on every run), then the gs_adam_step update
+ * of param[i], m[i], v[i] with g, then param[i] is also stored to every
+ * param_copies[d][i]. With zero_grads != 0 every gradient source is zeroed
+ * after it is read (so n_grads = 1, grad_scale = 1, zero_grads = 1 is
+ * gs_adam_step, bit for bit). grads and param_copies are HOST arrays of
+ * DEVICE pointers, each at the shard's first scalar: this GPU's own memory,
+ * or a peer GPU's memory opened with gs_shared_open (read and written with
+ * plain loads and stores over NVLink; no multicast). 1 <= n_grads <= 8,
+ * 0 <= n_copies <= 8. The caller orders the call after every rank's
+ * gradient is complete and every rank's next use of its parameters after
+ * every rank's call (stream-ordered barriers); the kernel itself waits on
+ * nothing. float4 accesses when every pointer is 16-byte aligned and count is
+ * a multiple of 4. Errors: GS_ERR_INVALID_ARG for NULL or misaligned
+ * (4-byte) pointers, counts out of range, count < 0, step < 1, bad betas or
+ * a non-finite lr or grad_scale; GS_ERR_CUDA if the launch fails. */
+gs_status gs_adam_step_reduce(float *param, float *m, float *v, int64_t count, float *const *grads,
+                              int32_t n_grads, float *const *param_copies, int32_t n_copies,
+                              int32_t zero_grads, float grad_scale, float lr, float beta1, float beta2,
+                              float eps, int32_t step, void *stream);
+
+/* Device memory that other processes on the node can map (CUDA IPC): the
+ * buffers whose shards gs_adam_step_reduce reads and writes on peers.
+ * gs_shared_alloc allocates `bytes` on the current device, zero-filled, and
+ * writes its GS_SHARED_HANDLE_BYTES-byte handle to the HOST array `handle`
+ * (to be sent to the other ranks); the caller frees it with gs_shared_free.
+ * gs_shared_open maps another process's allocation from its handle (peer
+ * access enabled lazily) and gs_shared_close unmaps it. Handles cannot be
+ * opened by the process that made them. Errors: GS_ERR_INVALID_ARG for NULL
+ * arguments or bytes <= 0; GS_ERR_CUDA if the CUDA call fails (nothing is
+ * leaked, *ptr is NULL). */
+#define GS_SHARED_HANDLE_BYTES 64
+gs_status gs_shared_alloc(int64_t bytes, void **ptr, unsigned char *handle);
+gs_status gs_shared_open(const unsigned char *handle, void **ptr);
+gs_status gs_shared_close(void *ptr);
+gs_status gs_shared_free(void *ptr);
+
 /* ------------------------------------------------------------ profiling --
  * When enabled, every kernel launch a context makes is bracketed by CUDA
  * events on the call's stream (a few microseconds of host time per launch;

@@ -92,3 +92,23 @@ def test_exchange_matches_adam_on_the_batch_mean_gradient(tmp_path):
     np.testing.assert_array_equal(p0, p1)
     # the shard's mean gradient is float32 (g0 + g1) / 2: within a few float32 ulps of lr-sized steps
     np.testing.assert_allclose(p0, ref, rtol=0, atol=1e-6)
+
+
+def test_p2p_pieces_address_every_rank_at_the_shard():
+    sys.path.insert(0, ROOT)
+    from gaussian_splatting_differentiable_rasteriser_b200 import data_parallel as dp
+    from gaussian_splatting_differentiable_rasteriser_b200.scenes import GROUP_NAMES
+    sizes = dict(zip(GROUP_NAMES, (300, 300, 400, 100, 4800)))
+    slices, total = _slices(sizes)
+    world = 4
+    pp = [1 << 40 | r << 32 for r in range(world)]
+    gp = [1 << 41 | r << 32 for r in range(world)]
+    covered = np.zeros(total, int)
+    for rank in range(world):
+        lo, hi = dp.shard_bounds(total, world, rank)
+        for k, a, b, gsrc, copies in dp.p2p_pieces(slices, total, world, rank, pp, gp):
+            assert lo <= a < b <= hi and slices[k].start <= a and b <= slices[k].stop
+            assert gsrc == [g + 4 * a for g in gp]
+            assert copies == [p + 4 * a for r, p in enumerate(pp) if r != rank]
+            covered[a:b] += 1
+    assert (covered == 1).all()

@@ -1,18 +1,33 @@
-"""The data-parallel step on the GPU with a one-rank NCCL group: the
-reduce-scatter, the sharded Adam and the all-gather run for real, and with the
-fixed-point (order-independent) gradient sums the result is bitwise the
-single-GPU step's (gs_render_backward, then gs_adam_step per group)."""
+"""The data-parallel step on the GPU.
+
+* gs_adam_step_reduce with every rank's buffers on this one GPU (one launch per
+  rank's shard, as each rank would issue it; the launches wait on nothing, so
+  this is the multi-rank data path run in order): every rank's parameters end
+  identical, equal bit for bit to Adam on the float32 rank-ordered mean
+  gradient, and within float32 rounding of the float64 oracle's Adam.
+* One source with zeroing is gs_adam_step, bit for bit.
+* The whole DataParallelTrainStep with a one-rank NCCL group, for both
+  exchanges, and with two processes on one GPU over gloo (the p2p exchange
+  reading and writing the other process's memory through CUDA IPC): with the
+  fixed-point (order-independent) gradient sums the parameters are bitwise
+  those of a single-GPU step on the mean gradient of the ranks' cameras.
+"""
+import datetime
 import os
 import socket
+import sys
 
 import numpy as np
 import pytest
 
+import oracle
 from gaussian_splatting_differentiable_rasteriser_b200 import scenes
 
 torch = pytest.importorskip("torch")
 
 pytestmark = pytest.mark.gpu
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 def free_port():
@@ -21,17 +36,110 @@ def free_port():
         return s.getsockname()[1]
 
 
-def test_one_rank_nccl_step_equals_the_single_gpu_step():
-    import datetime
-
-    import torch.distributed as dist
-
+@pytest.fixture(scope="module")
+def native():
     import __graft_entry__
     __graft_entry__.build()
-    from gaussian_splatting_differentiable_rasteriser_b200 import model, native
-    from gaussian_splatting_differentiable_rasteriser_b200.data_parallel import DataParallelTrainStep
+    from gaussian_splatting_differentiable_rasteriser_b200 import native as nat
     assert torch.cuda.is_available(), "GPU tests need a CUDA device"
-    native.load()
+    nat.load()
+    return nat
+
+
+def test_one_source_with_zeroing_is_adam_step(native):
+    g = torch.Generator().manual_seed(0)
+    for count, off in ((4096, 0), (1003, 0), (1000, 1)):
+        p, gr, m, v = (torch.randn(count + 8, generator=g).cuda() for _ in range(4))
+        v.abs_()
+        ref = [t.clone() for t in (p, gr, m, v)]
+        sl = slice(off, off + count)
+        native.adam_step(ref[0][sl], ref[1][sl], ref[2][sl], ref[3][sl], 1e-3, 3)
+        native.adam_step_reduce(p[sl], m[sl], v[sl], [gr[sl].data_ptr()], [], 1e-3, 3, zero_grads=True)
+        torch.cuda.synchronize()
+        for a, b in zip((p, gr, m, v), ref):
+            assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("world,count,aligned", [(2, 8192, True), (3, 3001, False), (4, 10_000, False),
+                                                 (8, 4 * 1237, True)])
+def test_emulated_ranks_reduce_adam_allgather(native, world, count, aligned):
+    from gaussian_splatting_differentiable_rasteriser_b200 import data_parallel as dp
+    from gaussian_splatting_differentiable_rasteriser_b200.scenes import GROUP_NAMES
+    rng = np.random.default_rng(world)
+    # five groups summing to count: ragged sizes (the scalar kernel), or multiples of
+    # 4 floats (16-byte-aligned pieces: the float4 kernel)
+    if aligned:
+        cuts = 4 * np.sort(rng.choice(np.arange(1, count // 4), 4, replace=False))
+    else:
+        cuts = np.sort(rng.choice(np.arange(1, count), 4, replace=False))
+    sizes = np.diff(np.concatenate([[0], cuts, [count]]))
+    slices, off = {}, 0
+    for k, n in zip(GROUP_NAMES, sizes):
+        slices[k] = slice(off, off + int(n))
+        off += int(n)
+    lrs = dict(zip(GROUP_NAMES, (1.6e-4, 5e-3, 1e-3, 5e-2, 2.5e-3)))
+    pad = dp.padded_size(count, world)
+    p0 = rng.normal(size=count).astype(np.float32)
+    m0 = rng.normal(0, 1e-2, count).astype(np.float32)
+    v0 = rng.uniform(0, 1e-4, count).astype(np.float32)
+    grads = [rng.normal(0, 1e-2, count).astype(np.float32) for _ in range(world)]
+    step = 4
+    params, gbufs, ms, vs = [], [], [], []
+    for r in range(world):
+        t = torch.zeros(pad, device="cuda")
+        t[:count] = torch.from_numpy(p0)
+        params.append(t)
+        t = torch.zeros(pad, device="cuda")
+        t[:count] = torch.from_numpy(grads[r])
+        gbufs.append(t)
+        ms.append(torch.zeros(pad, device="cuda"))
+        vs.append(torch.zeros(pad, device="cuda"))
+        ms[r][:count] = torch.from_numpy(m0)
+        vs[r][:count] = torch.from_numpy(v0)
+    pp = [t.data_ptr() for t in params]
+    gp = [t.data_ptr() for t in gbufs]
+    for r in range(world):
+        for k, a, b, gsrc, copies in dp.p2p_pieces(slices, count, world, r, pp, gp):
+            native.adam_step_reduce(params[r][a:b], ms[r][a:b], vs[r][a:b], gsrc, copies, lrs[k], step)
+    torch.cuda.synchronize()
+    out = [t[:count].cpu().numpy() for t in params]
+    for r in range(1, world):
+        np.testing.assert_array_equal(out[r], out[0])
+    for t in params:
+        assert not t[count:].any()
+    for r in range(world):  # sources are read, not zeroed
+        np.testing.assert_array_equal(gbufs[r][:count].cpu().numpy(), grads[r])
+    # bitwise: the float32 rank-ordered sum times 1/world, then gs_adam_step
+    gsum = torch.from_numpy(grads[0]).cuda()
+    for r in range(1, world):
+        gsum = gsum + torch.from_numpy(grads[r]).cuda()
+    gsum = gsum * np.float32(1.0 / world)
+    rp, rm, rv = (torch.from_numpy(x).cuda() for x in (p0, m0, v0))
+    for k in GROUP_NAMES:
+        s = slices[k]
+        native.adam_step(rp[s], gsum[s], rm[s], rv[s], lrs[k], step)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(out[0], rp.cpu().numpy())
+    m_all = np.zeros(count, np.float32)
+    for r in range(world):
+        lo, hi = dp.shard_bounds(count, world, r)
+        m_all[lo:min(hi, count)] = ms[r][lo:min(hi, count)].cpu().numpy()
+    np.testing.assert_array_equal(m_all, rm.cpu().numpy())
+    # the float64 oracle's Adam on the exact mean gradient
+    gmean = np.mean(np.stack(grads).astype(np.float64), axis=0)
+    for k in GROUP_NAMES:
+        s = slices[k]
+        op, _, om, ov = oracle.adam(p0[s], gmean[s], m0[s], v0[s], lrs[k], step)
+        np.testing.assert_allclose(out[0][s], op, rtol=0, atol=2e-6 + 1e-6 * lrs[k] / 1e-3)
+        np.testing.assert_allclose(m_all[s], om, rtol=1e-5, atol=1e-9)
+
+
+@pytest.mark.parametrize("exchange", ["p2p", "nccl"])
+def test_one_rank_nccl_step_equals_the_single_gpu_step(native, exchange):
+    import torch.distributed as dist
+
+    from gaussian_splatting_differentiable_rasteriser_b200 import model
+    from gaussian_splatting_differentiable_rasteriser_b200.data_parallel import DataParallelTrainStep
     scene = scenes.small()
     cam = scene.cameras[0]
     target = torch.from_numpy(scenes.uniform_image(cam.height, cam.width, seed=3)).cuda()
@@ -41,7 +149,7 @@ def test_one_rank_nccl_step_equals_the_single_gpu_step():
     try:
         ma, mb = model.GaussianModel(scene), model.GaussianModel(scene)
         cap = 1 << 20
-        a = DataParallelTrainStep(ma, cap, cam.width, cam.height, deterministic=True)
+        a = DataParallelTrainStep(ma, cap, cam.width, cam.height, deterministic=True, exchange=exchange)
         b = model.TrainStep(mb, cap, cam.width, cam.height, fused_adam=False, deterministic=True)
         assert a.world == 1 and a.adam_launches == len(scenes.GROUP_NAMES)
         for _ in range(3):
@@ -51,7 +159,73 @@ def test_one_rank_nccl_step_equals_the_single_gpu_step():
         assert torch.equal(ma.flat, mb.flat) and torch.equal(ma.m_flat, mb.m_flat)
         assert torch.equal(ma.v_flat, mb.v_flat)
         assert not a.grad_pad.any() and not a.param_pad[ma.flat.numel():].any()
-        # the parameters moved: the step is not a no-op
-        assert not torch.equal(ma.flat, model.GaussianModel(scene).flat)
+        assert not torch.equal(ma.flat, model.GaussianModel(scene).flat)  # the step moved them
+        a.close()
     finally:
         dist.destroy_process_group()
+
+
+def _rank(rank, world, port, out_dir, steps):
+    os.environ.update(RANK=str(rank), WORLD_SIZE=str(world), MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    import torch.distributed as dist
+
+    from gaussian_splatting_differentiable_rasteriser_b200 import model
+    from gaussian_splatting_differentiable_rasteriser_b200 import native as nat
+    from gaussian_splatting_differentiable_rasteriser_b200.data_parallel import DataParallelTrainStep
+    torch.cuda.set_device(0)
+    nat.load()
+    dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=120))
+    scene = scenes.small()
+    cams = [scenes.look_at((3.0 * np.sin(a), 0.3, -3.0 * np.cos(a)), (0.0, 0.0, 0.0), 256, 256, 256.0)
+            for a in (0.0, 0.4)]
+    targets = [torch.from_numpy(scenes.uniform_image(256, 256, seed=10 + r)).cuda() for r in range(world)]
+    m = model.GaussianModel(scene)
+    s = DataParallelTrainStep(m, 1 << 20, 256, 256, deterministic=True, exchange="p2p")
+    assert len(s._peer_maps) == 2 * (world - 1)
+    for _ in range(steps):
+        s(cams[rank], targets[rank])
+    torch.cuda.synchronize()
+    np.save(os.path.join(out_dir, f"p{rank}.npy"), m.flat.cpu().numpy())
+    np.save(os.path.join(out_dir, f"m{rank}.npy"), m.m_flat.cpu().numpy())
+    if rank == 0:
+        # the same iterations on one process: each camera's gradient on its own (from a
+        # zero buffer, as on its rank), summed in rank order, halved (exact), then Adam
+        # per group
+        r = model.GaussianModel(scene)
+        t = model.TrainStep(r, 1 << 20, 256, 256, fused_adam=False, deterministic=True)
+        for _ in range(steps):
+            r.step_count += 1
+            gsum = None
+            for c in range(world):
+                cs = nat.camera_struct(cams[c])
+                img, T, nc = t.forward(cs, 256, 256)
+                t.compute_loss(img, targets[c], t.dimage)
+                r.grad_flat.zero_()
+                t.ctx.render_backward(r.params_struct(), cs, T, nc, t.dimage, r.grads_struct())
+                gsum = r.grad_flat.clone() if gsum is None else gsum + r.grad_flat
+            r.grad_flat.copy_(gsum * 0.5)
+            t.update_from_grads()
+        torch.cuda.synchronize()
+        np.save(os.path.join(out_dir, "ref_p.npy"), r.flat.cpu().numpy())
+        np.save(os.path.join(out_dir, "ref_m.npy"), r.m_flat.cpu().numpy())
+    s.close()
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_two_processes_on_one_gpu_p2p_exchange(native, tmp_path):
+    import torch.multiprocessing as mp
+
+    from gaussian_splatting_differentiable_rasteriser_b200 import data_parallel as dp
+    world, steps = 2, 2
+    mp.start_processes(_rank, args=(world, free_port(), str(tmp_path), steps), nprocs=world, join=True,
+                       start_method="spawn")
+    p0, p1, ref = (np.load(tmp_path / f) for f in ("p0.npy", "p1.npy", "ref_p.npy"))
+    np.testing.assert_array_equal(p0, p1)
+    np.testing.assert_array_equal(p0, ref)
+    ref_m = np.load(tmp_path / "ref_m.npy")
+    total = ref_m.size
+    for r in range(world):
+        lo, hi = dp.shard_bounds(total, world, r)
+        np.testing.assert_array_equal(np.load(tmp_path / f"m{r}.npy")[lo:hi], ref_m[lo:hi])
