@@ -112,6 +112,8 @@ __device__ __forceinline__ uint32_t warp_lookback(const uint32_t* status, int64_
 // given j, the lanes' output runs are adjacent in memory.
 __global__ void __launch_bounds__(kDupThreads) duplicate_kernel(DuplicateArgs a) {
   __shared__ uint32_t s_warp[kDupThreads / 32];
+  __shared__ uint32_t s_pre[kDupThreads / 32][kDupPerThread][32];  // items' offsets in the warp's run
+  __shared__ uint32_t s_gid[kDupThreads / 32][kDupPerThread][32];  // items' Gaussians
   __shared__ uint32_t s_tile, s_excl;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (tid == 0) s_tile = atomicAdd(a.ticket, 1u);
@@ -124,6 +126,7 @@ __global__ void __launch_bounds__(kDupThreads) duplicate_kernel(DuplicateArgs a)
   for (int j = 0; j < kDupPerThread; ++j) {
     const int64_t idx = wbase + 32 * j + lane;
     gid[j] = idx < a.count ? __ldg(a.order + idx) : 0u;
+    s_gid[warp][j][lane] = gid[j];
   }
 #pragma unroll
   for (int j = 0; j < kDupPerThread; ++j) {
@@ -132,7 +135,6 @@ __global__ void __launch_bounds__(kDupThreads) duplicate_kernel(DuplicateArgs a)
     rc[j] = idx < a.count ? __ldg(a.rect + gid[j]) : make_uint2(1u, 1u);
   }
   // exclusive prefix of the tiles touched in (j, lane) order inside the warp
-  uint32_t pre[kDupPerThread];
   uint32_t run = 0;
 #pragma unroll
   for (int j = 0; j < kDupPerThread; ++j) {
@@ -145,7 +147,7 @@ __global__ void __launch_bounds__(kDupThreads) duplicate_kernel(DuplicateArgs a)
       const uint32_t n = __shfl_up_sync(0xffffffffu, v, o);
       if (lane >= o) v += n;
     }
-    pre[j] = run + v - c;
+    s_pre[warp][j][lane] = run + v - c;
     run += __shfl_sync(0xffffffffu, v, 31);
   }
   if (lane == 0) s_warp[warp] = run;
@@ -172,16 +174,66 @@ __global__ void __launch_bounds__(kDupThreads) duplicate_kernel(DuplicateArgs a)
     if (lane == 0 && run) record_error(a.err, kErrIndexRange);
     return;
   }
-#pragma unroll
+  // The warp writes each group j of 32 items' entries together. When every
+  // item of the group touches at most 2 tiles, each lane writes its own
+  // entries (adjacent to its neighbours'). Otherwise output o of the group
+  // goes to lane o mod 32, which finds the item that owns it by a binary
+  // search over the lanes' exclusive offsets: every store of the warp is then
+  // one run of 32 consecutive entries, however unevenly the tiles are spread
+  // over the items (a few large Gaussians touch hundreds of tiles).
+  // The items come back from shared memory (offsets, Gaussians) and the
+  // cache (rects, fetched one group ahead) rather than staying in registers,
+  // so this loop is not unrolled and the kernel keeps its occupancy.
+  const uint32_t tiles_x = static_cast<uint32_t>(a.tiles_x);
+  auto rect_of = [&](int j) {
+    return wbase + 32 * j + lane < a.count ? __ldg(a.rect + s_gid[warp][j][lane]) : make_uint2(1u, 1u);
+  };
+  uint2 r_next = rect_of(0);
+#pragma unroll 1
   for (int j = 0; j < kDupPerThread; ++j) {
-    const uint32_t x0 = rc[j].x & 0xffffu, x1 = rc[j].x >> 16, y0 = rc[j].y & 0xffffu, y1 = rc[j].y >> 16;
-    uint64_t off = off0 + pre[j];
-    for (uint32_t y = y0; y <= y1; ++y)
-      for (uint32_t x = x0; x <= x1; ++x) {
-        a.keys[off] = y * static_cast<uint32_t>(a.tiles_x) + x;
-        a.vals[off] = gid[j];
-        ++off;
+    const uint32_t g = s_gid[warp][j][lane];
+    const uint2 r = r_next;
+    if (j + 1 < kDupPerThread) r_next = rect_of(j + 1);
+    const uint32_t p = s_pre[warp][j][lane];
+    const uint32_t gstart = __shfl_sync(0xffffffffu, p, 0);
+    const uint32_t excl = p - gstart;  // this lane's first output in the group
+    const uint32_t x0 = r.x & 0xffffu, y0 = r.y & 0xffffu;
+    const uint32_t w = (r.x >> 16) + 1u - x0;
+    const uint32_t h = (r.y >> 16) + 1u - y0;  // padding items: w = h = 0
+    const uint32_t last_excl = __shfl_sync(0xffffffffu, excl, 31);
+    const uint32_t last_c = __shfl_sync(0xffffffffu, w * h, 31);
+    const uint32_t group_total = last_excl + last_c;
+    uint32_t* keys = a.keys + off0 + gstart;
+    uint32_t* vals = a.vals + off0 + gstart;
+    if (__all_sync(0xffffffffu, w * h <= 2u)) {
+      // every item touches at most 2 tiles: each lane writes its own (adjacent) entries
+      for (uint32_t k = 0; k < w * h; ++k) {
+        keys[excl + k] = w == 1u ? (y0 + k) * tiles_x + x0 : y0 * tiles_x + x0 + k;
+        vals[excl + k] = g;
       }
+      continue;
+    }
+    for (uint32_t ob = 0; ob < group_total; ob += 32) {
+      const uint32_t o = ob + static_cast<uint32_t>(lane);
+      // owner = the highest lane whose first output is <= o (it has a non-empty rect)
+      int owner = 0;
+#pragma unroll
+      for (int step = 16; step > 0; step >>= 1) {
+        const uint32_t e = __shfl_sync(0xffffffffu, excl, owner + step);
+        if (e <= o) owner += step;
+      }
+      const uint32_t oe = __shfl_sync(0xffffffffu, excl, owner);
+      const uint32_t ow = __shfl_sync(0xffffffffu, w, owner);
+      const uint32_t ox0 = __shfl_sync(0xffffffffu, x0, owner);
+      const uint32_t oy0 = __shfl_sync(0xffffffffu, y0, owner);
+      const uint32_t og = __shfl_sync(0xffffffffu, g, owner);
+      if (o < group_total) {
+        const uint32_t local = o - oe;
+        const uint32_t dy = local / ow;
+        keys[o] = (oy0 + dy) * tiles_x + ox0 + (local - dy * ow);
+        vals[o] = og;
+      }
+    }
   }
 }
 
@@ -407,14 +459,38 @@ __global__ void __launch_bounds__(kSortThreads) onesweep_kernel(OnesweepArgs a) 
 }
 
 // ------------------------------------------------------------------ ranges --
+// Each thread looks at kRangeItems consecutive sorted entries (two 16-byte
+// loads) and the one before them; every change of tile between neighbours
+// closes the previous tile's range and opens the next one's.
+constexpr int kRangeItems = 8;
+
 __global__ void __launch_bounds__(256) ranges_kernel(const uint32_t* keys, int64_t n, uint2* ranges,
                                                      int64_t num_tiles) {
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (i >= n) return;
-  const uint32_t tile = keys[i];
-  if (tile >= static_cast<uint64_t>(num_tiles)) return;
-  if (i == 0 || keys[i - 1] != tile) ranges[tile].x = static_cast<uint32_t>(i);
-  if (i == n - 1 || keys[i + 1] != tile) ranges[tile].y = static_cast<uint32_t>(i + 1);
+  const int64_t i0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) * kRangeItems;
+  if (i0 >= n) return;
+  uint32_t k[kRangeItems];
+  if (i0 + kRangeItems <= n) {
+    const uint4 a = __ldg(reinterpret_cast<const uint4*>(keys + i0));
+    const uint4 b = __ldg(reinterpret_cast<const uint4*>(keys + i0) + 1);
+    k[0] = a.x, k[1] = a.y, k[2] = a.z, k[3] = a.w, k[4] = b.x, k[5] = b.y, k[6] = b.z, k[7] = b.w;
+  } else {
+#pragma unroll
+    for (int j = 0; j < kRangeItems; ++j) k[j] = i0 + j < n ? __ldg(keys + i0 + j) : ~0u;
+  }
+  const uint64_t tiles = static_cast<uint64_t>(num_tiles);
+  uint32_t prev = i0 > 0 ? __ldg(keys + i0 - 1) : ~0u;
+#pragma unroll
+  for (int j = 0; j < kRangeItems; ++j) {
+    const int64_t i = i0 + j;
+    if (i >= n) break;
+    const uint32_t cur = k[j];
+    if (cur != prev) {
+      if (cur < tiles) ranges[cur].x = static_cast<uint32_t>(i);
+      if (prev < tiles) ranges[prev].y = static_cast<uint32_t>(i);
+    }
+    prev = cur;
+  }
+  if (i0 + kRangeItems >= n && prev < tiles) ranges[prev].y = static_cast<uint32_t>(n);
 }
 
 }  // namespace
@@ -477,7 +553,9 @@ cudaError_t launch_ranges(const uint32_t* keys, int64_t n, uint2* ranges, int64_
                           cudaStream_t st) {
   cudaError_t e = cudaMemsetAsync(ranges, 0, sizeof(uint2) * num_tiles, st);
   if (e != cudaSuccess || n == 0) return e;
-  ranges_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(keys, n, ranges, num_tiles);
+  const int64_t per_block = 256 * kRangeItems;
+  ranges_kernel<<<static_cast<unsigned>((n + per_block - 1) / per_block), 256, 0, st>>>(keys, n, ranges,
+                                                                                       num_tiles);
   return cudaGetLastError();
 }
 

@@ -1,6 +1,7 @@
 """Parity at full size: the Dense workload (3,000,000 Gaussians, SH degree 3,
-1920x1080) in the launch configuration the benchmark times (one TrainStep with
-its entry capacity), against the float64 oracle.
+1920x1080) and the Heavy-tail workload (6,000,000 Gaussians, 10% of them large,
+so long per-tile lists) in the launch configuration the benchmark times (one
+TrainStep with its entry capacity), against the float64 oracle.
 
 The oracle's preprocess and tile sort run on the whole scene, so those are
 compared in full (the sort bit-exact over every entry). The blend is compared
@@ -25,6 +26,7 @@ PIX_TOL = 1e-4
 LOSS_RTOL = 1e-5
 GRAD_RL2 = 1e-3
 BAND = 16
+MIN_UNAMBIGUOUS = {"dense": 0.99, "heavy_tail": 0.95}
 
 
 def dev(a, dtype=torch.float32):
@@ -41,14 +43,14 @@ def rel_l2(a, b):
     return np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-30)
 
 
-@pytest.fixture(scope="module")
-def dense():
+@pytest.fixture(scope="module", params=["dense", "heavy_tail"])
+def full(request):
     import __graft_entry__
     __graft_entry__.build()
     from gaussian_splatting_differentiable_rasteriser_b200 import model, native
     assert torch.cuda.is_available(), "GPU tests need a CUDA device"
     native.load()
-    scene = scenes.dense()
+    scene = scenes.CONFIGS[request.param]()
     cams = scene.cameras
     cam = cams[int(scenes.camera_schedule(len(cams), 1, seed=0)[0])]
     m = model.GaussianModel(scene)
@@ -63,8 +65,8 @@ def dense():
                 img=img, T=T, nc=nc, o=o)
 
 
-def test_dense_preprocess_and_sort_bit_exact(dense):
-    step, o, n = dense["step"], dense["o"], dense["scene"].n
+def test_full_preprocess_and_sort_bit_exact(full):
+    step, o, n = full["step"], full["o"], full["scene"].n
     out = dict(rect=torch.empty((n, 4), dtype=torch.int32, device="cuda"),
                touched=torch.empty(n, dtype=torch.int32, device="cuda"),
                depth=torch.empty(n, device="cuda"), mean2d=torch.empty((n, 2), device="cuda"))
@@ -82,7 +84,7 @@ def test_dense_preprocess_and_sort_bit_exact(dense):
     srt = o.sorted()
     K = step.last_entries
     assert K == srt["ids"].size
-    cam = dense["cam"]
+    cam = full["cam"]
     tx, ty = (cam.width + 15) // 16, (cam.height + 15) // 16
     ids = torch.empty(K, dtype=torch.int32, device="cuda")
     tiles = torch.empty(K, dtype=torch.int32, device="cuda")
@@ -106,13 +108,15 @@ def sample_pixels(cam, seed=5, n_random=4096):
     return np.concatenate(px), np.concatenate(py)
 
 
-def test_dense_forward_sampled_pixels(dense):
-    cam, o = dense["cam"], dense["o"]
+def test_full_forward_sampled_pixels(full):
+    cam, o = full["cam"], full["o"]
     px, py = sample_pixels(cam)
     r = o.render_pixels(px, py)
-    img, T, nc = host(dense["img"]), host(dense["T"]), host(dense["nc"])
+    img, T, nc = host(full["img"]), host(full["T"]), host(full["nc"])
     ok = ~r["ambiguous"].astype(bool)
-    assert ok.mean() > 0.99
+    # pixels with a threshold decision within 1e-6 relative of its cut are left out:
+    # the longer the lists (thousands per tile on Heavy-tail), the more of them
+    assert ok.mean() > MIN_UNAMBIGUOUS[full["scene"].name], ok.mean()
     got = img[:, py, px].T
     err = np.abs(got - r["rgb"])[ok]
     assert err.max() <= PIX_TOL, err.max()
@@ -124,13 +128,13 @@ def test_dense_forward_sampled_pixels(dense):
     assert np.all(nc >= 0)
 
 
-def band_gradient(dense):
+def band_gradient(full):
     """The loss gradient of the full image against a uniform target, kept on a
     16-row band through the image centre and zero elsewhere."""
-    cam = dense["cam"]
+    cam = full["cam"]
     H, W = cam.height, cam.width
     target = scenes.uniform_image(H, W, seed=21)
-    img32 = host(dense["img"])
+    img32 = host(full["img"])
     L, l1, ssim, d = oracle.loss(img32, target, 0.2)
     y0 = (H - BAND) // 2
     band = np.zeros((3, H, W), np.float32)
@@ -138,12 +142,12 @@ def band_gradient(dense):
     return target, (L, l1, ssim, d), band, y0
 
 
-def test_dense_loss_full_image(dense):
-    step = dense["step"]
-    target, (L, l1, ssim, dref), _, _ = band_gradient(dense)
+def test_full_loss_full_image(full):
+    step = full["step"]
+    target, (L, l1, ssim, dref), _, _ = band_gradient(full)
     out = torch.zeros(3, dtype=torch.float64, device="cuda")
-    d = torch.empty_like(dense["img"])
-    step.ctx.loss_l1_dssim(dense["img"], dev(target), 0.2, out, d)
+    d = torch.empty_like(full["img"])
+    step.ctx.loss_l1_dssim(full["img"], dev(target), 0.2, out, d)
     torch.cuda.synchronize()
     got = host(out)
     assert got[0] == pytest.approx(L, rel=LOSS_RTOL)
@@ -152,8 +156,8 @@ def test_dense_loss_full_image(dense):
     assert rel_l2(host(d), dref) < 1e-4
 
 
-def oracle_band_backward(dense, band, y0):
-    o, s = dense["o"], dense["scene"]
+def oracle_band_backward(full, band, y0):
+    o, s = full["o"], full["scene"]
     sg = np.zeros((s.n, 9))
     o.blend_backward_rows(y0, y0 + BAND, band.astype(np.float64), sg)
     out = dict(means=np.zeros((3, s.n_pad)), log_scales=np.zeros((3, s.n_pad)),
@@ -163,12 +167,12 @@ def oracle_band_backward(dense, band, y0):
     return sg, out
 
 
-def test_dense_backward_on_a_row_band(dense):
-    step, m, s = dense["step"], dense["m"], dense["scene"]
-    _, _, band, y0 = band_gradient(dense)
-    sg_ref, ref = oracle_band_backward(dense, band, y0)
+def test_full_backward_on_a_row_band(full):
+    step, m, s = full["step"], full["m"], full["scene"]
+    _, _, band, y0 = band_gradient(full)
+    sg_ref, ref = oracle_band_backward(full, band, y0)
     m.grad_flat.zero_()
-    step.ctx.render_backward(m.params_struct(), dense["cs"], dense["T"], dense["nc"], dev(band),
+    step.ctx.render_backward(m.params_struct(), full["cs"], full["T"], full["nc"], dev(band),
                              m.grads_struct())
     sg = torch.empty((s.n, 9), device="cuda")
     step.ctx.debug_screen_grads(sg)
@@ -176,7 +180,7 @@ def test_dense_backward_on_a_row_band(dense):
     sg = host(sg)
     assert np.any(sg_ref != 0, axis=1).sum() > 1000
     # a Gaussian none of whose tiles meets the band's tile rows gets exactly nothing
-    rect = dense["o"].preprocess()["rect"]  # x0, y0, x1, y1 in tiles
+    rect = full["o"].preprocess()["rect"]  # x0, y0, x1, y1 in tiles
     far = (rect[:, 3] < y0 // 16) | (rect[:, 1] > (y0 + BAND - 1) // 16)
     assert not sg[far].any(), "Gaussians away from the band got a screen gradient"
     assert rel_l2(sg, sg_ref) < GRAD_RL2
@@ -186,17 +190,17 @@ def test_dense_backward_on_a_row_band(dense):
     m.grad_flat.zero_()
 
 
-def test_dense_fused_backward_adam_on_a_row_band(dense):
-    step, m, s = dense["step"], dense["m"], dense["scene"]
-    _, _, band, y0 = band_gradient(dense)
-    _, ref = oracle_band_backward(dense, band, y0)
+def test_full_fused_backward_adam_on_a_row_band(full):
+    step, m, s = full["step"], full["m"], full["scene"]
+    _, _, band, y0 = band_gradient(full)
+    _, ref = oracle_band_backward(full, band, y0)
     m.load(s)
     m.m_flat.zero_()
     m.v_flat.zero_()
     m.grad_flat.zero_()
     em, ev = m.moments_structs()
     lr = 1e-3
-    step.ctx.render_backward_adam(m.params_struct(), dense["cs"], dense["T"], dense["nc"], dev(band),
+    step.ctx.render_backward_adam(m.params_struct(), full["cs"], full["T"], full["nc"], dev(band),
                                   None, em, ev, [lr] * 5, 1)
     torch.cuda.synchronize()
     assert not m.grad_flat.any().item()
