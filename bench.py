@@ -45,17 +45,17 @@ WORKLOADS = {
              "target = renders of a perturbed copy, seed 0",
 }
 
-# ncu DRAM traffic (read + write bytes per launch) of kernels on the dense workload,
-# with the sha256 (first 12 hex digits) of the source file each figure was taken from.
-# A figure whose source has changed since is reported as null. Both were captured
-# with ncu on the Mid workload (500k Gaussians, about 1.06M entries) and scaled to
-# Dense by the units a launch processes (n_pad 3,000,000 / 500,000 for the
-# per-Gaussian pass, entries 6.32M / 1.06M for the blend), in which traffic grows in
-# proportion. The fused pass's write counter undercounts: its last writes are still
-# in L2 when the kernel ends.
+# ncu DRAM traffic (read + write bytes) of kernels per unit of their work, with the
+# sha256 (first 12 hex digits) of the source file each figure was taken from. A
+# figure whose source has changed since is reported as null. Both were captured with
+# ncu on the Mid workload (500,000 Gaussians, 1,064,000 entries per step) and are
+# scaled to a launch of the benchmarked workload by the units it processes: the
+# Gaussians (n_pad) for the per-Gaussian pass, the (Gaussian, tile) entries for the
+# blend, in which traffic grows in proportion. The fused pass's write counter
+# undercounts: its last writes are still in L2 when the kernel ends.
 NCU_TRAFFIC = {
-    "backward_adam": ((408.091648e6 + 292.852480e6) * 6.0, "f1df474a7794"),
-    "blend_backward": ((85.319936e6 + 3.207936e6) * 6.32 / 1.064, "2dcc3feaade8"),
+    "backward_adam": ((408.091648e6 + 292.852480e6) / 500_000, "gaussians", "f1df474a7794"),
+    "blend_backward": ((85.319936e6 + 3.207936e6) / 1.064e6, "entries", "2dcc3feaade8"),
 }
 
 
@@ -489,7 +489,10 @@ def main_ours(args):
            "preprocess_backward": "preprocess_backward.cu",
            "backward_adam": "preprocess_backward.cu", "exchange_adam": "adam_reduce.cu"}.get(dominant)
     tr = NCU_TRAFFIC.get(dominant)
-    rf["traffic"] = tr[0] if (tr and src and sha12(os.path.join(PKG_CSRC, src)) == tr[1]) else None
+    rf["traffic"] = None
+    if tr and src and sha12(os.path.join(PKG_CSRC, src)) == tr[2]:
+        units = scene.n_pad if tr[1] == "gaussians" else (statistics.mean(ks) if ks else 0)
+        rf["traffic"] = tr[0] * units
 
     # launches of our kernels in the timed region: the profiler counts every kernel a
     # context launches (over the same steps), plus gs_adam_step per group when the
