@@ -64,6 +64,7 @@ def lib():
                                       ctypes.c_double, P, P, P, P, P]
         L.or_sh_basis.argtypes = [ctypes.c_int32, ctypes.c_int64, P, P]
         L.or_rotation_cov.argtypes = [P, P, P, P]
+        L.or_camera_backward.argtypes = [P, P, P]
         _lib = L
     return _lib
 
@@ -72,17 +73,21 @@ def _p(a):
     return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
 
 
-def camera(cam) -> OrCamera:
+def camera(cam, f64=False) -> OrCamera:
+    """The camera as the oracle reads it: the float32 values the CUDA path
+    receives, widened to float64; with f64 the camera's own values unrounded
+    (for derivative checks that move the pose by less than a float32 step)."""
+    rnd = (lambda v: float(v)) if f64 else (lambda v: float(np.float32(v)))
     c = OrCamera()
     c.width, c.height = int(cam.width), int(cam.height)
-    c.fx, c.fy, c.cx, c.cy = (float(np.float32(v)) for v in (cam.fx, cam.fy, cam.cx, cam.cy))
-    for i, v in enumerate(np.asarray(cam.R, np.float32).reshape(-1)):
-        c.R[i] = float(v)
+    c.fx, c.fy, c.cx, c.cy = (rnd(v) for v in (cam.fx, cam.fy, cam.cx, cam.cy))
+    for i, v in enumerate(np.asarray(cam.R, np.float64).reshape(-1)):
+        c.R[i] = rnd(v)
     for name in ("t", "campos", "bg"):
         arr = getattr(c, name)
-        for i, v in enumerate(np.asarray(getattr(cam, name), np.float32).reshape(-1)):
-            arr[i] = float(v)
-    c.near_z = float(np.float32(cam.near_z))
+        for i, v in enumerate(np.asarray(getattr(cam, name), np.float64).reshape(-1)):
+            arr[i] = rnd(v)
+    c.near_z = rnd(cam.near_z)
     return c
 
 
@@ -90,7 +95,7 @@ class Oracle:
     """One scene seen by one camera: preprocess and tile lists are built on
     construction; render/backward walk the lists per pixel."""
 
-    def __init__(self, scene, cam, active_degree=None, opacity_rect=False):
+    def __init__(self, scene, cam, active_degree=None, opacity_rect=False, camera_f64=False):
         self.L = lib()
         self.scene = scene
         self.cam = cam
@@ -103,7 +108,7 @@ class Oracle:
         arrs = [np.ascontiguousarray(a, dtype=dt) for a in
                 (scene.means, scene.log_scales, scene.quats, scene.opacity_logits, scene.sh)]
         self._keep = arrs
-        self._cam = camera(cam)
+        self._cam = camera(cam, camera_f64)
         fn = self.L.or_set_scene_f64 if f64 else self.L.or_set_scene
         rc = fn(self.h, scene.n, scene.n_pad, scene.sh_degree, self.active_degree,
                 *[_p(a) for a in arrs], ctypes.byref(self._cam))
@@ -200,6 +205,14 @@ class Oracle:
         self.L.or_project_backward(self.h, _p(screen_grad), int(i0), int(i1),
                                    *[_p(out[k]) for k in ("means", "log_scales", "quats",
                                                           "opacity_logits", "sh")])
+        return out
+
+    def camera_backward(self, screen_grad):
+        """dL/d(pose) = (dL/dw, dL/dt) for the pose update R <- exp([w]x) R,
+        t <- t + dt, from the screen gradient (n x 9) of this view."""
+        assert screen_grad.dtype == np.float64 and screen_grad.shape == (self.scene.n, 9)
+        out = np.zeros(6)
+        self.L.or_camera_backward(self.h, _p(np.ascontiguousarray(screen_grad)), _p(out))
         return out
 
 

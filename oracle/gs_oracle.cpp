@@ -272,8 +272,22 @@ struct Aux {
   double Y[16] = {0};
 };
 
-int tiles_x(const or_camera& cam) { return (cam.width + kTile - 1) / kTile; }
-int tiles_y(const or_camera& cam) { return (cam.height + kTile - 1) / kTile; }
+template <class Cam>
+int tiles_x(const Cam& cam) { return (cam.width + kTile - 1) / kTile; }
+template <class Cam>
+int tiles_y(const Cam& cam) { return (cam.height + kTile - 1) / kTile; }
+
+// A camera whose pose is a function of a perturbation (dual numbers): the
+// projection below is written once for both camera types.
+template <class S>
+struct PoseCamera {
+  int32_t width, height;
+  double fx, fy, cx, cy;
+  S R[9];
+  S t[3];
+  S campos[3];
+  double near_z;
+};
 
 // Rotation matrix of the normalised quaternion (w, x, y, z), row-major.
 template <class S>
@@ -319,12 +333,12 @@ void covariance3d(const S ls[3], const S q[4], S Sigma[9]) {
 // E = min(4.5, ln(max(o / alpha_min, 1.0001))) with alpha_min = 1/255 and no
 // compensation factor, and r = sqrt(2 E) sqrt(lambda_max). Beyond r along
 // the long axis o exp(-e) < 1/255, so the tiles it drops hold no contribution.
-template <class S>
-bool project(const or_camera& cam, const S p[3], const S ls[3], const S q[4], const S& logit,
+template <class S, class Cam>
+bool project(const Cam& cam, const S p[3], const S ls[3], const S q[4], const S& logit,
              const double* sh, int64_t sh_stride, int active_degree, Proj<S>& P, Aux& X,
              bool opacity_rect = false) {
   X = Aux();
-  const double* R = cam.R;
+  const auto* R = cam.R;
   // p_c = R p + t, each row summed left to right.
   S pc[3];
   for (int i = 0; i < 3; ++i)
@@ -818,6 +832,68 @@ void or_project_backward(void* h, const double* screen_grad, int64_t i0, int64_t
           g_sh[(static_cast<size_t>(ch) * K + k) * np + i] = gs[6 + ch] * X.Y[k];
       }
   }
+}
+
+// Gradient of the loss with respect to the camera pose ("How a computer
+// rebuilds a real place ... Gaussian Splats", section "Forgiving the camera
+// and the light": the render depends on the camera, so backprop gives it a
+// gradient too). The pose moves as R <- exp([w]x) R, t <- t + dt: a rotation
+// w of the camera frame and a shift dt of the translation, the
+// parametrisation of that section's code (rotation blame = cross(p_c - t,
+// dL/dp_c), translation blame = dL/dp_c). Here the derivative is the exact
+// one, by dual numbers through the whole projection: besides the position
+// path it includes the rotation of each Gaussian's camera-space covariance
+// and the move of the camera centre campos = -R^T t in the view direction of
+// the colour. out = {dL/dw (3), dL/dt (3)}, summed over the Gaussians from
+// their screen gradient (n x 9).
+void or_camera_backward(void* h, const double* screen_grad, double* out) {
+  const Ctx& c = *static_cast<Ctx*>(h);
+  using D = Dual<6>;
+  PoseCamera<D> pc;
+  pc.width = c.cam.width;
+  pc.height = c.cam.height;
+  pc.fx = c.cam.fx;
+  pc.fy = c.cam.fy;
+  pc.cx = c.cam.cx;
+  pc.cy = c.cam.cy;
+  pc.near_z = c.cam.near_z;
+  const D w[3] = {seed<6>(0.0, 0), seed<6>(0.0, 1), seed<6>(0.0, 2)};
+  // exp([w]x) = I + [w]x + O(w^2): the first-order part gives the exact derivative at w = 0
+  const D Wx[9] = {D(0.0), -w[2], w[1], w[2], D(0.0), -w[0], -w[1], w[0], D(0.0)};
+  for (int r = 0; r < 3; ++r)
+    for (int col = 0; col < 3; ++col) {
+      D acc(c.cam.R[3 * r + col]);
+      for (int k = 0; k < 3; ++k) acc = acc + Wx[3 * r + k] * c.cam.R[3 * k + col];
+      pc.R[3 * r + col] = acc;
+    }
+  for (int i = 0; i < 3; ++i) pc.t[i] = c.cam.t[i] + seed<6>(0.0, 3 + i);
+  // campos = -R^T t as a function of the pose; its value stays the camera's own
+  for (int i = 0; i < 3; ++i) {
+    D acc(0.0);
+    for (int k = 0; k < 3; ++k) acc = acc + pc.R[3 * k + i] * pc.t[k];
+    pc.campos[i] = -acc;
+    pc.campos[i].v = c.cam.campos[i];
+  }
+  const int64_t np = c.n_pad;
+  double g[6] = {0, 0, 0, 0, 0, 0};
+  for (int64_t i = 0; i < c.n; ++i) {
+    if (c.aux[i].touched == 0) continue;
+    const double* gs = &screen_grad[static_cast<size_t>(i) * kScreen];
+    bool any = false;
+    for (int o = 0; o < kScreen; ++o) any = any || gs[o] != 0.0;
+    if (!any) continue;
+    const D p[3] = {D(c.means[i]), D(c.means[np + i]), D(c.means[2 * np + i])};
+    const D ls[3] = {D(c.ls[i]), D(c.ls[np + i]), D(c.ls[2 * np + i])};
+    const D q[4] = {D(c.quats[i]), D(c.quats[np + i]), D(c.quats[2 * np + i]), D(c.quats[3 * np + i])};
+    const D logit(c.logits[i]);
+    Proj<D> P;
+    Aux X;
+    if (!project<D>(pc, p, ls, q, logit, &c.sh[i], np, c.active_degree, P, X, c.opacity_rect)) continue;
+    const D* outs[kScreen] = {&P.u, &P.v, &P.A, &P.B, &P.C, &P.o, &P.rgb[0], &P.rgb[1], &P.rgb[2]};
+    for (int o = 0; o < kScreen; ++o)
+      for (int j = 0; j < 6; ++j) g[j] += gs[o] * outs[o]->d[j];
+  }
+  for (int j = 0; j < 6; ++j) out[j] = g[j];
 }
 
 // Backward from dL/dimage [3][H][W] over the pixel rows [y0, y1) (other rows
