@@ -54,8 +54,8 @@ WORKLOADS = {
 # blend, in which traffic grows in proportion. The fused pass's write counter
 # undercounts: its last writes are still in L2 when the kernel ends.
 NCU_TRAFFIC = {
-    "backward_adam": ((408.091648e6 + 292.852480e6) / 500_000, "gaussians", "f1df474a7794"),
-    "blend_backward": ((85.319936e6 + 3.207936e6) / 1.064e6, "entries", "2dcc3feaade8"),
+    "backward_adam": ((409.251584e6 + 290.841600e6) / 500_000, "gaussians", "3df92fa0a447"),
+    "blend_backward": ((85.220352e6 + 2.926336e6) / 1.064e6, "entries", "2dcc3feaade8"),
 }
 
 
@@ -186,7 +186,7 @@ def max_over_ranks(x, world):
 
 # ------------------------------------------------------------------ workload
 def build_workload(config, device, opacity_rect=False, deterministic=False, loss="l1_dssim",
-                   data_parallel=False, exchange="p2p"):
+                   data_parallel=False, exchange="p2p", camera_grad=False):
     import numpy as np
     import torch
 
@@ -206,6 +206,10 @@ def build_workload(config, device, opacity_rect=False, deterministic=False, loss
     else:
         step = model.TrainStep(m, cap, W, H, device=device, opacity_rect=opacity_rect,
                                deterministic=deterministic, loss=loss)
+    if camera_grad:
+        # every backward also writes the view's pose gradient (6 float64)
+        step.camera_grad = torch.zeros(6, dtype=torch.float64, device=device)
+        step.ctx.set_camera_grad(step.camera_grad)
     # targets: renders of the perturbed copy (forward only, before any timing)
     targets = torch.empty((len(cams), 3, H, W), dtype=torch.float32, device=device)
     kmax = 0
@@ -310,6 +314,10 @@ def stage_models(scene, sh_k):
         # step): p, m, v read and written, 24 B per scalar of every group, plus the raw
         # screen-gradient sums, the screen record and two flags, per Gaussian
         "backward_adam": ("hbm", 24 * n_par + 48 + 48 + 5),
+        # camera-pose gradient, per Gaussian as a visible one reads it: 40 B of
+        # geometry parameters, the 48 B screen record, the 48 B raw sums, touched and
+        # clamp flags (5 B) and the 192 B of SH coefficients of three coloured channels
+        "camera_backward": ("hbm", 40 + 48 + 48 + 5 + 4 * 3 * sh_k),
         # FP32 instructions: 7 per pair the method's walk visits (2 subtractions + 5 for the
         # exponent's quadratic form), plus per blended pair 6 in the forward (weight, 3
         # colour FMAs, transmittance update) and 19 in the backward (T recovery 2,
@@ -460,7 +468,7 @@ def main_ours(args):
     device = f"cuda:{local}"
     scene, m, step, targets, kmax = build_workload(args.config, device, args.rect == "opacity",
                                                    args.deterministic, args.loss, args.parallel == "dp",
-                                                   args.exchange)
+                                                   args.exchange, args.camera_grad)
     cams = scene.cameras
     sched = scenes.camera_schedule(len(cams), args.warmup + args.steps, seed=rank)
     # clocks are sampled from the start of the warm-up to the end of the timed region
@@ -487,7 +495,8 @@ def main_ours(args):
     src = {"blend_forward": "blend.cu", "blend_backward": "blend.cu", "adam": "adam.cu",
            "preprocess": "preprocess.cu", "sort": "sort.cu", "depth_sort": "sort.cu", "loss": "loss.cu",
            "preprocess_backward": "preprocess_backward.cu",
-           "backward_adam": "preprocess_backward.cu", "exchange_adam": "adam_reduce.cu"}.get(dominant)
+           "backward_adam": "preprocess_backward.cu", "exchange_adam": "adam_reduce.cu",
+           "camera_backward": "camera_backward.cu"}.get(dominant)
     tr = NCU_TRAFFIC.get(dominant)
     rf["traffic"] = None
     if tr and src and sha12(os.path.join(PKG_CSRC, src)) == tr[2]:
@@ -527,6 +536,7 @@ def main_ours(args):
                        "tile_rect": "3 sigma" if args.rect == "3sigma" else "opacity-aware",
                        "gradient_sums": "fixed-point (deterministic)" if args.deterministic else "float32 atomics",
                        "loss": "L1 + D-SSIM (lambda 0.2)" if args.loss == "l1_dssim" else "Charbonnier + exposure",
+                       "camera_grad": bool(args.camera_grad),
                        "l2": "inputs larger than L2: 2.8 GB of parameter/gradient/moment state "
                              "streamed every step" if args.config == "dense" else "see workload",
                        "entries_per_step": int(statistics.mean(ks)) if ks else None},
@@ -765,6 +775,8 @@ def main():
                          "(one camera per rank per iteration; value counts camera-iterations)")
     ap.add_argument("--exchange", choices=("p2p", "nccl"), default="p2p",
                     help="--parallel dp: the fused peer-memory exchange + Adam, or NCCL collectives")
+    ap.add_argument("--camera-grad", action="store_true",
+                    help="each backward also computes the view's camera-pose gradient")
     ap.add_argument("--op", choices=("step", "densify"), default="step",
                     help="the training step (default) or one densification pass")
     args = ap.parse_args()

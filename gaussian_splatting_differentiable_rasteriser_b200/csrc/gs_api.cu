@@ -46,6 +46,10 @@ struct gs_ctx {
   uint32_t* loss_counter = nullptr;
   double* charb_partials = nullptr;  // [kCharbMaxBlocks][7]
   uint32_t* charb_counter = nullptr;
+  // camera-pose gradient: caller's output (NULL when off) and the kernel's scratch
+  double* cam_out = nullptr;
+  double* cam_partials = nullptr;  // [kCamBlocks][9]
+  uint32_t* cam_counter = nullptr;
   // readback record (device + pinned host); the device error word lives in it
   gs::ForwardInfo* info_dev = nullptr;
   gs::ForwardInfo* info_host = nullptr;
@@ -106,7 +110,7 @@ void free_all(gs_ctx* c) {
                   c->dvals[1], c->dup_status, c->keys[0], c->keys[1], c->vals[0], c->vals[1],
                   c->hist, c->offsets, c->status, c->counters, c->ranges, c->surv, c->surv_count,
                   c->sgrad_fixed, c->dens_counts, c->dens_prefix, c->dens_totals, c->charb_partials,
-                  c->charb_counter, c->loss_partials,
+                  c->charb_counter, c->cam_partials, c->cam_counter, c->loss_partials,
                   c->loss_counter, c->info_dev, c->pairs};
   for (void* b : bufs)
     if (b) cudaFree(b);
@@ -295,6 +299,8 @@ gs_status gs_create(gs_ctx** out, int64_t max_gaussians, int64_t max_entries, in
   GS_ALLOC(c->loss_counter, sizeof(uint32_t));
   GS_ALLOC(c->charb_partials, sizeof(double) * 7 * gs::kCharbMaxBlocks);
   GS_ALLOC(c->charb_counter, sizeof(uint32_t));
+  GS_ALLOC(c->cam_partials, sizeof(double) * 9 * gs::kCamBlocks);
+  GS_ALLOC(c->cam_counter, sizeof(uint32_t));
   GS_ALLOC(c->info_dev, sizeof(gs::ForwardInfo));
   GS_ALLOC(c->pairs, sizeof(unsigned long long) * 8);
 #undef GS_ALLOC
@@ -302,6 +308,7 @@ gs_status gs_create(gs_ctx** out, int64_t max_gaussians, int64_t max_entries, in
   if (e == cudaSuccess) e = cudaMallocHost(reinterpret_cast<void**>(&c->dens_host), sizeof(uint4));
   if (e == cudaSuccess) e = cudaMemset(c->loss_counter, 0, sizeof(uint32_t));
   if (e == cudaSuccess) e = cudaMemset(c->charb_counter, 0, sizeof(uint32_t));
+  if (e == cudaSuccess) e = cudaMemset(c->cam_counter, 0, sizeof(uint32_t));
   if (e == cudaSuccess) e = cudaMemset(c->info_dev, 0, sizeof(gs::ForwardInfo));
   if (e == cudaSuccess) e = cudaMemset(c->pairs, 0, sizeof(unsigned long long) * 8);
   if (e == cudaSuccess) e = cudaDeviceSynchronize();
@@ -606,6 +613,18 @@ gs_status backward_common(gs_ctx* c, const gs_params* p, const gs_camera* cam, c
   a.g_sh = g ? g->sh : nullptr;
   a.stat_accum = c->stat_accum;
   a.stat_count = c->stat_count;
+  if (c->cam_out) {
+    // camera-pose gradient of this view, from the raw sums and the parameters
+    // of the render (before any update)
+    prof_begin(c, st);
+    if (p->n > 0) {
+      gs::CameraGradArgs cg{c->cam_out, c->cam_partials, c->cam_counter};
+      GS_CUDA(c, gs::launch_camera_backward(a, cg, st));
+    } else {
+      GS_CUDA(c, cudaMemsetAsync(c->cam_out, 0, 6 * sizeof(double), st));
+    }
+    prof_end(c, GS_STAGE_CAMERA_BACKWARD, p->n, st, p->n > 0 ? 1 : 0);
+  }
   return GS_OK;
 }
 
@@ -811,7 +830,8 @@ gs_status gs_profile_read(gs_ctx* c, double* ms, int64_t* launches, int64_t* wor
 const char* gs_stage_name(int32_t stage) {
   static const char* names[GS_NUM_STAGES] = {"preprocess", "scan", "duplicate", "sort", "ranges",
                                              "blend_forward", "loss", "blend_backward",
-                                             "preprocess_backward", "backward_adam", "depth_sort"};
+                                             "preprocess_backward", "backward_adam", "depth_sort",
+                                             "camera_backward"};
   return (stage >= 0 && stage < GS_NUM_STAGES) ? names[stage] : "";
 }
 
@@ -853,6 +873,13 @@ gs_status gs_debug_screen_grads(gs_ctx* c, float* out, void* stream) {
   return GS_OK;
 }
 
+
+gs_status gs_set_camera_grad(gs_ctx* c, double* out) {
+  if (!c) return GS_ERR_INVALID_ARG;
+  if (out && !aligned(out, 8)) return fail(c, GS_ERR_INVALID_ARG, "camera gradient output must be 8-byte aligned");
+  c->cam_out = out;
+  return GS_OK;
+}
 
 gs_status gs_set_densify_stats(gs_ctx* c, float* grad_accum, uint32_t* view_count) {
   if (!c) return GS_ERR_INVALID_ARG;

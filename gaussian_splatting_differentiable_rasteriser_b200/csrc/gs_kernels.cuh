@@ -193,6 +193,16 @@ struct PreprocessBwdArgs {
 
 cudaError_t launch_preprocess_backward(const PreprocessBwdArgs& a, cudaStream_t st);
 
+// Camera-pose gradient of one view: out = {dL/dw (3), dL/dt (3)} in float64,
+// from the same per-Gaussian inputs as the projection backward.
+constexpr int kCamBlocks = 148 * 4;
+struct CameraGradArgs {
+  double* out;       // [6], device
+  double* partials;  // [kCamBlocks][9]
+  uint32_t* counter; // zero between calls (the last CTA resets it)
+};
+cudaError_t launch_camera_backward(const PreprocessBwdArgs& a, const CameraGradArgs& g, cudaStream_t st);
+
 // Parameters (written in place), accumulated gradients (zeroed), Adam moments
 // and per-group scalars, in group order means, log_scales, quats,
 // opacity_logits, sh.

@@ -27,13 +27,13 @@ EXPORTED = ("gs_create", "gs_destroy", "gs_last_error", "gs_preprocess", "gs_ren
             "gs_debug_screen_grads", "gs_set_option", "gs_loss_l1_dssim_noalloc",
             "gs_set_densify_stats", "gs_densify", "gs_opacity_reset", "gs_loss_charbonnier",
             "gs_adam_step_reduce", "gs_shared_alloc", "gs_shared_open", "gs_shared_close",
-            "gs_shared_free")
+            "gs_shared_free", "gs_set_camera_grad")
 GS_SHARED_HANDLE_BYTES = 64
 MAX_RANKS = 8
 GS_OPTION_OPACITY_RECT = 1
 GS_OPTION_DETERMINISTIC = 2
 STAGES = ("preprocess", "scan", "duplicate", "sort", "ranges", "blend_forward", "loss",
-          "blend_backward", "preprocess_backward", "backward_adam", "depth_sort")
+          "blend_backward", "preprocess_backward", "backward_adam", "depth_sort", "camera_backward")
 GROUPS = ("means", "log_scales", "quats", "opacity_logits", "sh")
 
 
@@ -103,6 +103,7 @@ def load(path: str = LIB_PATH):
     L.gs_shared_open.argtypes = [ctypes.c_char_p, PP]
     L.gs_shared_close.argtypes = [P]
     L.gs_shared_free.argtypes = [P]
+    L.gs_set_camera_grad.argtypes = [P, P]
     L.gs_set_option.argtypes = [P, I32, I32]
     L.gs_set_option.restype = ctypes.c_int
     L.gs_loss_l1_dssim_noalloc.argtypes = [P, P, I32, I32, F, P, P, P]
@@ -181,6 +182,12 @@ class Context:
         b = (ctypes.c_float * 3)(*[float(x) for x in bias])
         self._check(self.L.gs_loss_charbonnier(self.h, _ptr(image), _ptr(target), H, W, g, b, float(delta),
                                                _ptr(out), _ptr(dloss_dimage), _stream(stream)))
+
+    def set_camera_grad(self, out):
+        """Every later backward writes this view's pose gradient (dL/dw, dL/dt) to
+        `out` (6 float64 on the device); None turns it off."""
+        self._out_cam = out  # kept alive while the context points at it
+        self._check(self.L.gs_set_camera_grad(self.h, _ptr(out)))
 
     def set_densify_stats(self, grad_accum, view_count):
         self._check(self.L.gs_set_densify_stats(self.h, _ptr(grad_accum), _ptr(view_count)))

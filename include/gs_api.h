@@ -325,7 +325,8 @@ typedef enum {
   GS_STAGE_PREPROCESS_BACKWARD = 8,
   GS_STAGE_BACKWARD_ADAM = 9, /* the fused projection backward + Adam pass */
   GS_STAGE_DEPTH_SORT = 10,   /* compaction + depth sort of the visible Gaussians */
-  GS_NUM_STAGES = 11
+  GS_STAGE_CAMERA_BACKWARD = 11, /* camera-pose gradient (when gs_set_camera_grad is on) */
+  GS_NUM_STAGES = 12
 } gs_stage;
 
 gs_status gs_profile_enable(gs_ctx *ctx, int32_t enabled);
@@ -387,6 +388,24 @@ gs_status gs_loss_charbonnier(gs_ctx *ctx, const float *image_chw, const float *
  * both to stop accumulating. Errors: GS_ERR_INVALID_ARG if exactly one is
  * NULL. */
 gs_status gs_set_densify_stats(gs_ctx *ctx, float *grad_accum, uint32_t *view_count);
+
+/* Camera-pose gradient ([GS] "Forgiving the camera and the light": the render
+ * depends on the camera, so backprop gives it a gradient, which a trainer
+ * uses to refine imperfect poses). With out set (a DEVICE array of 6 doubles,
+ * 8-byte aligned), every later gs_render_backward / gs_render_backward_adam
+ * also writes to out the gradient of the loss with respect to this view's
+ * pose, for the update R <- exp([w]x) R, t <- t + dt of the camera given to
+ * the call: out = {dL/dw_x, dL/dw_y, dL/dw_z, dL/dt_x, dL/dt_y, dL/dt_z}
+ * (overwritten, not accumulated: each photo has its own pose). It is the
+ * exact derivative: the position path of that section's code, plus the
+ * rotation of each camera-space covariance and the move of the camera centre
+ * -R^T t in the colours' view directions. It is computed from the parameters
+ * passed to the call, before the fused call updates them. It is summed in
+ * float64 in a fixed order (deterministic for a given screen gradient, so
+ * bitwise reproducible with GS_OPTION_DETERMINISTIC). out = NULL turns it off
+ * (the default). The context keeps the pointer; the caller keeps the buffer
+ * alive. Errors: GS_ERR_INVALID_ARG for a NULL ctx or a misaligned out. */
+gs_status gs_set_camera_grad(gs_ctx *ctx, double *out);
 
 /* One densification pass from the set `in` (n Gaussians, planar with
  * in->n_pad) to the set `out` (planar with stride out_n_pad, written through

@@ -44,3 +44,10 @@ def test_create_rejects_bad_sizes_without_touching_the_device():
         native.GS_ERR_INVALID_ARG
     assert lib.gs_adam_step(None, None, None, None, 0, 1e-3, 0.9, 0.999, 1e-8, 0, None) == \
         native.GS_ERR_INVALID_ARG
+
+
+def test_stage_names_match_the_binding():
+    from gaussian_splatting_differentiable_rasteriser_b200 import native
+    L = native.load()
+    assert [L.gs_stage_name(k).decode() for k in range(len(native.STAGES))] == list(native.STAGES)
+    assert L.gs_stage_name(len(native.STAGES)).decode() == ""

@@ -172,8 +172,11 @@ def test_full_backward_on_a_row_band(full):
     _, _, band, y0 = band_gradient(full)
     sg_ref, ref = oracle_band_backward(full, band, y0)
     m.grad_flat.zero_()
+    cam_grad = torch.zeros(6, dtype=torch.float64, device="cuda")
+    step.ctx.set_camera_grad(cam_grad)
     step.ctx.render_backward(m.params_struct(), full["cs"], full["T"], full["nc"], dev(band),
                              m.grads_struct())
+    step.ctx.set_camera_grad(None)
     sg = torch.empty((s.n, 9), device="cuda")
     step.ctx.debug_screen_grads(sg)
     torch.cuda.synchronize()
@@ -187,6 +190,11 @@ def test_full_backward_on_a_row_band(full):
     for k in scenes.GROUP_NAMES:
         e = rel_l2(host(m.grads[k])[..., :s.n], ref[k][..., :s.n])
         assert e < GRAD_RL2, (k, e)
+    # the camera-pose gradient of the same band
+    cam_ref = full["o"].camera_backward(sg_ref)
+    got = host(cam_grad)
+    assert rel_l2(got[:3], cam_ref[:3]) < GRAD_RL2, (got, cam_ref)
+    assert rel_l2(got[3:], cam_ref[3:]) < GRAD_RL2, (got, cam_ref)
     m.grad_flat.zero_()
 
 
