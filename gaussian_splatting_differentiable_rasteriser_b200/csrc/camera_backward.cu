@@ -13,8 +13,10 @@
 //     with c = sum_i dL/dcampos_i = -sum_i (view-direction part of dL/dp_i),
 //     dL/dw += t x (R c) and dL/dt -= R c.
 //
-// B200 design: one pass over the Gaussians on a fixed grid of 148 x 4 CTAs
-// (grid-stride), reusing the projection backward's per-Gaussian algebra; each
+// B200 design: one pass over the Gaussians on a fixed grid of 148 x 3 CTAs,
+// one wave at 3 CTAs per SM (80 registers; the per-Gaussian chain of dependent
+// loads is latency-bound, so resident warps count), grid-stride, reusing the
+// projection backward's per-Gaussian algebra; each
 // thread sums its Gaussians' nine terms in float64, each CTA reduces them in a
 // fixed order, and the last CTA to finish adds the CTAs' partial sums in a
 // fixed order and forms the six outputs, so the result is deterministic for
@@ -32,7 +34,7 @@ namespace {
 constexpr int kCamThreads = 256;
 
 template <int kDeg>
-__global__ void __launch_bounds__(kCamThreads) camera_backward_kernel(PreprocessBwdArgs a, CameraGradArgs cg) {
+__global__ void __launch_bounds__(kCamThreads, 3) camera_backward_kernel(PreprocessBwdArgs a, CameraGradArgs cg) {
   __shared__ double s_red[9][kCamThreads / 32];
   __shared__ int s_last;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;

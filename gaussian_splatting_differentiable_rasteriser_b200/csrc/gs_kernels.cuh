@@ -195,7 +195,7 @@ cudaError_t launch_preprocess_backward(const PreprocessBwdArgs& a, cudaStream_t 
 
 // Camera-pose gradient of one view: out = {dL/dw (3), dL/dt (3)} in float64,
 // from the same per-Gaussian inputs as the projection backward.
-constexpr int kCamBlocks = 148 * 4;
+constexpr int kCamBlocks = 148 * 3;
 struct CameraGradArgs {
   double* out;       // [6], device
   double* partials;  // [kCamBlocks][9]
