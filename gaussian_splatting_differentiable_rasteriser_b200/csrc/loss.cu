@@ -176,9 +176,9 @@ __global__ void __launch_bounds__(kLossThreads, 4) loss_kernel(LossArgs a) {
 #pragma unroll
         for (int o = 0; o < 4; ++o) acc[c][o] = 0.f;
       if (q0 + 3 >= Y0 - kR) {  // rows above Y0 - 5 feed no output of this strip
+        int ring = ring_slot(q0 - kR - Y0 + 2 * kR);  // advanced one row at a time below
 #pragma unroll
         for (int rr = 0; rr < 14; ++rr) {
-          const int ring = ring_slot(q0 - kR + rr - Y0 + 2 * kR);
 #pragma unroll
           for (int c = 0; c < 5; ++c) {
             const float hv = s.h[c][ring][j];
@@ -188,6 +188,7 @@ __global__ void __launch_bounds__(kLossThreads, 4) loss_kernel(LossArgs a) {
               if (t >= 0 && t <= 2 * kR) acc[c][o] = __fmaf_rn(w[t], hv, acc[c][o]);
             }
           }
+          ring = ring + 1 == kRing ? 0 : ring + 1;
         }
       }
 #pragma unroll
@@ -248,9 +249,9 @@ __global__ void __launch_bounds__(kLossThreads, 4) loss_kernel(LossArgs a) {
       float acc[3][2];
 #pragma unroll
       for (int c = 0; c < 3; ++c) acc[c][0] = acc[c][1] = 0.f;
+      int ring = ring_slot(r0 - kR - Y0 + kR);  // advanced one row at a time below
 #pragma unroll
       for (int rr = 0; rr < 12; ++rr) {
-        const int ring = ring_slot(r0 - kR + rr - Y0 + kR);
 #pragma unroll
         for (int c = 0; c < 3; ++c) {
           const float av = s.a[c][ring][jj];
@@ -260,6 +261,7 @@ __global__ void __launch_bounds__(kLossThreads, 4) loss_kernel(LossArgs a) {
             if (t >= 0 && t <= 2 * kR) acc[c][o] = __fmaf_rn(w[t], av, acc[c][o]);
           }
         }
+        ring = ring + 1 == kRing ? 0 : ring + 1;
       }
       const int gx = x0 + jj;
 #pragma unroll
