@@ -112,3 +112,41 @@ def test_p2p_pieces_address_every_rank_at_the_shard():
             assert copies == [p + 4 * a for r, p in enumerate(pp) if r != rank]
             covered[a:b] += 1
     assert (covered == 1).all()
+
+
+def _rank_fails(rank, world, port, out_dir):
+    os.environ.update(RANK=str(rank), WORLD_SIZE=str(world), MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    from gaussian_splatting_differentiable_rasteriser_b200 import data_parallel as dp
+    from gaussian_splatting_differentiable_rasteriser_b200.scenes import GROUP_NAMES
+    dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=10))
+    slices, total = _slices(dict(zip(GROUP_NAMES, (8, 8, 8, 4, 36))))
+    pad = dp.padded_size(total, world)
+    status = "ok"
+    try:
+        if rank == 1:
+            raise RuntimeError("this rank's backward failed")  # leaves before the exchange
+        dp.exchange_and_update(torch.ones(pad), torch.zeros(pad), torch.zeros(total), torch.zeros(total),
+                               slices, total, world, rank, lambda *a: None)
+    except Exception as e:  # noqa: BLE001 - the test records what each rank saw
+        status = f"error: {type(e).__name__}"
+    open(os.path.join(out_dir, f"status{rank}.txt"), "w").write(status)
+    if rank == 1:
+        os._exit(0)  # leaves without a clean shutdown, as a crashed rank does
+    try:
+        dist.destroy_process_group()
+    except Exception:  # noqa: BLE001
+        pass
+
+
+def test_a_rank_that_fails_before_the_exchange_makes_the_others_fail_not_hang(tmp_path):
+    import torch.multiprocessing as mp
+    mp.start_processes(_rank_fails, args=(2, free_port(), str(tmp_path)), nprocs=2, join=True,
+                       start_method="spawn")
+    assert (tmp_path / "status1.txt").read_text().startswith("error")
+    assert (tmp_path / "status0.txt").read_text().startswith("error")
