@@ -110,13 +110,23 @@ class GaussianModel:
 DEFAULT_LR = {k: 1e-3 for k in GROUP_NAMES}
 
 
+def sh_degree_at(step: int, every: int, max_degree: int) -> int:
+    """SH bands unlocked before iteration `step` (0-based) when one more degree is
+    switched on every `every` iterations ("How a computer rebuilds a real place ...
+    Gaussian Splats", section "Spherical harmonics: color that changes with viewing
+    angle": degree 0 first, one degree about every 1000 steps)."""
+    return min(max_degree, step // every)
+
+
 class TrainStep:
     """Buffers and the call sequence of one iteration for images up to width x height."""
 
     def __init__(self, model: GaussianModel, max_entries: int, width: int, height: int, lrs=None,
                  lam=0.2, betas=(0.9, 0.999), eps=1e-8, device="cuda", fused_adam=True,
-                 opacity_rect=False, deterministic=False, loss="l1_dssim"):
+                 opacity_rect=False, deterministic=False, loss="l1_dssim", sh_ramp_every=None):
         self.model = model
+        # None: the model's active degree stays as set; otherwise it follows sh_degree_at
+        self.sh_ramp_every = sh_ramp_every
         self.fused_adam = fused_adam
         if loss not in ("l1_dssim", "charbonnier"):
             raise ValueError("loss must be 'l1_dssim' or 'charbonnier'")
@@ -151,6 +161,9 @@ class TrainStep:
 
     def __call__(self, cam, target):
         """One iteration against `target` ([3, H, W] float32 on the device)."""
+        if self.sh_ramp_every:
+            m = self.model
+            m.active_degree = sh_degree_at(m.step_count, self.sh_ramp_every, m.sh_degree)
         cs = native.camera_struct(cam)
         H, W = cam.height, cam.width
         img, T, nc = self.forward(cs, H, W)

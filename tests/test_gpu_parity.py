@@ -585,3 +585,29 @@ def test_training_step_with_the_charbonnier_loss(gs):
         upd = (host(m.params[k]).astype(np.float64) - p0)[..., : s.n]
         big = np.abs(ref[k][..., : s.n]) > 1e-3 * np.abs(ref[k][..., : s.n]).max()
         assert np.mean(np.abs(upd[big] - upd_ref[big]) <= 1e-6) > 0.99, k
+
+
+def test_sh_degree_ramp_leaves_inactive_bands_untouched(gs):
+    """TrainStep(sh_ramp_every=2): degree 0 for the first two iterations (the
+    higher SH bands neither colour nor move), then degree 1 (bands 1-3 move,
+    bands 4-15 still do not)."""
+    native, model = gs
+    s = scenes.small()
+    cam = s.cameras[0]
+    tgt = dev(scenes.uniform_image(cam.height, cam.width, seed=14))
+    m = model.GaussianModel(s)
+    st = model.TrainStep(m, 200_000, cam.width, cam.height, sh_ramp_every=2)
+    sh0 = host(m.params["sh"]).copy()
+    st(cam, tgt)
+    st(cam, tgt)
+    torch.cuda.synchronize()
+    assert m.active_degree == 0
+    sh1 = host(m.params["sh"]).copy()
+    np.testing.assert_array_equal(sh1[:, 1:], sh0[:, 1:])
+    assert not np.array_equal(sh1[:, 0], sh0[:, 0])
+    st(cam, tgt)
+    torch.cuda.synchronize()
+    assert m.active_degree == 1
+    sh2 = host(m.params["sh"])
+    np.testing.assert_array_equal(sh2[:, 4:], sh0[:, 4:])
+    assert not np.array_equal(sh2[:, 1:4], sh0[:, 1:4])
