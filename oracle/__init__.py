@@ -369,6 +369,52 @@ def densify(params, m, v, n, grad_accum, view_count, normals, grad_threshold, sc
     return out_p, out_m, out_v, n_out
 
 
+def relocate(params, m, v, n, normals, dead_opacity=0.02, donor_opacity=0.4, max_pairs=None):
+    """Recycling the dead ("How a computer rebuilds a real place ... Gaussian
+    Splats", section "Densification: cloning the busy blobs, recycling the
+    dead"), with the count fixed. Dead: opacity below dead_opacity; donors:
+    opacity above donor_opacity (both decided on the logit in float64). The
+    donors are taken largest first (largest log-scale, ties by index), the dead
+    in index order, and the j-th dead is paired with the j-th donor, for
+    j < min(dead, donors, max_pairs, len(normals)). For a pair (d, b): slot d
+    becomes a copy of b placed at mean_b + R_b S_b z_j (z_j = normals[j], the
+    donor's own Gaussian, as a split child is placed), both d and b take
+    log-scales log_scale_b - ln 1.6 ("both halves shrink"), and both restart
+    their Adam moments at zero. Every other slot is unchanged. Returns
+    (params, m, v, pairs) as float64 copies (pairs: list of (d, b))."""
+    groups = ("means", "log_scales", "quats", "opacity_logits", "sh")
+    P = {g: np.array(params[g], np.float64, copy=True) for g in groups}
+    M = {g: np.array(m[g], np.float64, copy=True) for g in groups}
+    V = {g: np.array(v[g], np.float64, copy=True) for g in groups}
+    dead_thr = math.log(dead_opacity / (1.0 - dead_opacity))
+    donor_thr = math.log(donor_opacity / (1.0 - donor_opacity))
+    logits = P["opacity_logits"][..., :n]
+    dead = [i for i in range(n) if logits[i] < dead_thr]
+    donors = [i for i in range(n) if logits[i] > donor_thr]
+    size = {i: float(np.max(np.float32(P["log_scales"][:, i]))) for i in donors}
+    donors.sort(key=lambda i: (-size[i], i))
+    count = min(len(dead), len(donors), len(normals))
+    if max_pairs is not None:
+        count = min(count, max_pairs)
+    pairs = []
+    for j in range(count):
+        d, b = dead[j], donors[j]
+        ls_b = P["log_scales"][:, b].copy()
+        R = _rotation(P["quats"][:, b])
+        child = P["means"][:, b] + R @ np.diag(np.exp(ls_b)) @ np.asarray(normals[j], np.float64)
+        for g in groups:
+            P[g][..., d] = P[g][..., b]
+        P["means"][:, d] = child
+        P["log_scales"][:, d] = ls_b - math.log(1.6)
+        P["log_scales"][:, b] = ls_b - math.log(1.6)
+        for g in groups:
+            for slot in (d, b):
+                M[g][..., slot] = 0.0
+                V[g][..., slot] = 0.0
+        pairs.append((d, b))
+    return P, M, V, pairs
+
+
 def opacity_reset(logits, m, v, max_opacity):
     """logit = min(logit, logit(max_opacity)); the moments of the logits set to zero."""
     cap = math.log(max_opacity / (1.0 - max_opacity))
