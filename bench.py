@@ -19,6 +19,7 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -755,6 +756,84 @@ def main_densify(args):
         dist.destroy_process_group()
 
 
+def main_relocate(args):
+    """Time of one recycling pass (gs_relocate) on the workload's Gaussians with
+    their own opacities (dead < 0.02, donors > 0.4), one normal draw per dead
+    Gaussian; the parameters are restored between passes, outside the timed
+    region. Roofline: HBM bytes of the classification, the donors' 4-pass sort and
+    the pair writes; the oracle timed on a 1/200 sample beside it."""
+    import numpy as np
+    import torch
+
+    import __graft_entry__
+
+    world, rank, local = dist_setup()
+    if rank == 0:
+        __graft_entry__.build()
+    barrier(world)
+    from gaussian_splatting_differentiable_rasteriser_b200 import model, native, scenes
+    from gaussian_splatting_differentiable_rasteriser_b200.scenes import GROUP_NAMES
+
+    native.load()
+    device = f"cuda:{local}"
+    scene = scenes.CONFIGS[args.config]()
+    m = model.GaussianModel(scene, device=device)
+    m.m_flat.normal_(0, 1e-3)
+    m.v_flat.uniform_(0, 1e-6)
+    backup = [t.clone() for t in (m.flat, m.m_flat, m.v_flat)]
+    logits = scene.opacity_logits[:scene.n].astype(np.float64)
+    dead = int((logits < math.log(0.02 / 0.98)).sum())
+    donors = int((logits > math.log(0.4 / 0.6)).sum())
+    normals = torch.from_numpy(np.random.default_rng(7).normal(size=(max(dead, 1), 3)).astype(np.float32)).to(device)
+    ctx = native.Context(scene.n_pad, 16, 16, 16)
+    total_ms, pairs = 0.0, 0
+    for it in range(args.warmup + args.steps):
+        for t, b in zip((m.flat, m.m_flat, m.v_flat), backup):
+            t.copy_(b)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        pairs = m.relocate(ctx, normals)
+        e1.record()
+        torch.cuda.synchronize()
+        if it >= args.warmup:
+            total_ms += e0.elapsed_time(e1)
+    ms = max_over_ranks(total_ms, world)
+    value = replica_throughput(world, args.steps, ms / 1e3)
+    n = scene.n
+    planes = 11 + 3 * scene.sh_k
+    algo_bytes = n * 16 + donors * (8 + 4 * 16) + dead * 4 + pairs * planes * 4 * 6
+    hbm_gbs, _, peak_kind = peaks()
+    achieved = algo_bytes * value / world / 1e9
+    cpu = None
+    if rank == 0 and not args.no_cpu_baseline:
+        import oracle
+        sl = slice(0, n, 200)
+        sub = {k: getattr(scene, k)[..., sl].astype(np.float64) for k in GROUP_NAMES}
+        zeros = {k: np.zeros_like(x) for k, x in sub.items()}
+        k_n = sub["opacity_logits"].shape[-1]
+        t0 = time.perf_counter()
+        oracle.relocate(sub, zeros, zeros, k_n, normals.cpu().numpy())
+        est = (time.perf_counter() - t0) * n / k_n
+        cpu = {"value": 1.0 / est, "unit": "passes/s", "cores": 1, "kind": "oracle",
+               "sample": f"float64 oracle relocate of every 200th of {n} Gaussians, scaled by 200; single-threaded"}
+    if rank == 0:
+        line = {"metric": "relocate passes/s (dead Gaussians recycled onto the largest donors)", "value": value,
+                "unit": "passes/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+                "config": {"workload": WORKLOADS[args.config], "gaussians": n, "dead": dead, "donors": donors,
+                           "pairs": int(pairs), "dead_opacity": 0.02, "donor_opacity": 0.4},
+                "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s",
+                             "frac": achieved / hbm_gbs, "traffic": None, "peak_source": peak_kind,
+                             "bytes_per_pass": algo_bytes},
+                "e2e": None, "gpu_launches": 10 * args.steps, "cpu_baseline": cpu}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -777,8 +856,8 @@ def main():
                     help="--parallel dp: the fused peer-memory exchange + Adam, or NCCL collectives")
     ap.add_argument("--camera-grad", action="store_true",
                     help="each backward also computes the view's camera-pose gradient")
-    ap.add_argument("--op", choices=("step", "densify"), default="step",
-                    help="the training step (default) or one densification pass")
+    ap.add_argument("--op", choices=("step", "densify", "relocate"), default="step",
+                    help="the training step (default), one densification pass or one recycling pass")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -786,6 +865,8 @@ def main():
         main_reference(args)
     elif args.op == "densify":
         main_densify(args)
+    elif args.op == "relocate":
+        main_relocate(args)
     else:
         main_ours(args)
 

@@ -195,6 +195,104 @@ __global__ void __launch_bounds__(kDensifyBlock) densify_write_kernel(DensifyArg
   }
 }
 
+// ------------------------------------------------------------- relocation
+// "How a computer rebuilds a real place ... Gaussian Splats", section
+// "Densification: cloning the busy blobs, recycling the dead": dead Gaussians
+// (opacity < ~0.02) are moved next to donors (opacity > ~0.4), the largest
+// donors first; both halves shrink by 1.6 and restart their Adam moments.
+// Classification, compaction (dead indices; donors with a descending-size key)
+// and, after a stable sort of the donors, one thread per pair.
+
+enum RelocClass : int { kRelocNone = 0, kRelocDead = 1, kRelocDonor = 2 };
+
+__device__ __forceinline__ int reloc_class(const RelocateArgs& a, int64_t i) {
+  const double logit = a.p[3][i];
+  if (logit < a.dead_logit) return kRelocDead;
+  if (logit > a.donor_logit) return kRelocDonor;
+  return kRelocNone;
+}
+
+// Largest log-scale as a key that sorts ascending for descending size (the
+// float's bits mapped to an order-preserving unsigned integer, then inverted).
+__device__ __forceinline__ uint32_t size_key(const RelocateArgs& a, int64_t i) {
+  const float* ls = a.p[1];
+  const float s = fmaxf(fmaxf(ls[i], ls[a.np + i]), ls[2 * a.np + i]);
+  const uint32_t u = __float_as_uint(s);
+  const uint32_t ord = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  return ~ord;
+}
+
+__global__ void __launch_bounds__(kDensifyBlock) relocate_count_kernel(RelocateArgs a) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * kDensifyBlock + threadIdx.x;
+  const int c = i < a.n ? reloc_class(a, i) : kRelocNone;
+  block_ranks(c == kRelocDead, c == kRelocDonor, false, a.block_counts + blockIdx.x);
+}
+
+__global__ void __launch_bounds__(kDensifyBlock) relocate_compact_kernel(RelocateArgs a) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * kDensifyBlock + threadIdx.x;
+  const int c = i < a.n ? reloc_class(a, i) : kRelocNone;
+  const Ranks r = block_ranks(c == kRelocDead, c == kRelocDonor, false, nullptr);
+  const uint4 P = a.block_prefix[blockIdx.x];
+  if (c == kRelocDead) {
+    const int64_t k = static_cast<int64_t>(P.x) + r.kept;
+    if (k < a.n) a.dead[k] = static_cast<uint32_t>(i);
+    else record_error(a.err, kErrIndexRange);
+  } else if (c == kRelocDonor) {
+    const int64_t k = static_cast<int64_t>(P.y) + r.clone;
+    if (k < a.n) {
+      a.donor_keys[k] = size_key(a, i);
+      a.donor_vals[k] = static_cast<uint32_t>(i);
+    } else {
+      record_error(a.err, kErrIndexRange);
+    }
+  }
+}
+
+__global__ void relocate_pair_kernel(RelocateArgs a) {
+  const int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (j >= a.pairs) return;
+  const int64_t d = a.dead[j], b = a.sorted_donors[j];
+  const int64_t np = a.np;
+  if (d >= a.n || b >= a.n) {
+    record_error(a.err, kErrIndexRange);
+    return;
+  }
+  // the donor's own Gaussian: mean + R(q/|q|) diag(exp(log-scales)) z_j
+  const float* q = a.p[2];
+  const double qw = q[b], qx = q[np + b], qy = q[2 * np + b], qz = q[3 * np + b];
+  const double qn = sqrt(qw * qw + qx * qx + qy * qy + qz * qz);
+  const double w = qw / qn, x = qx / qn, y = qy / qn, z = qz / qn;
+  const double R[9] = {1.0 - 2.0 * (y * y + z * z), 2.0 * (x * y - w * z), 2.0 * (x * z + w * y),
+                       2.0 * (x * y + w * z), 1.0 - 2.0 * (x * x + z * z), 2.0 * (y * z - w * x),
+                       2.0 * (x * z - w * y), 2.0 * (y * z + w * x), 1.0 - 2.0 * (x * x + y * y)};
+  const float* zj = a.normals + 3 * j;
+  double sz[3];
+  float ls_new[3], mean[3];
+  for (int c = 0; c < 3; ++c) {
+    const double ls = a.p[1][c * np + b];
+    sz[c] = exp(ls) * zj[c];
+    ls_new[c] = static_cast<float>(ls - log(1.6));
+  }
+  for (int c = 0; c < 3; ++c)
+    mean[c] = static_cast<float>(static_cast<double>(a.p[0][c * np + b]) + R[3 * c] * sz[0] + R[3 * c + 1] * sz[1] +
+                                 R[3 * c + 2] * sz[2]);
+  const int planes[5] = {3, 3, 4, 1, 3 * a.sh_k};
+  for (int g = 0; g < 5; ++g)
+    for (int c = 0; c < planes[g]; ++c) {
+      const int64_t o = c * np;
+      a.p[g][o + d] = a.p[g][o + b];
+      a.m[g][o + d] = 0.0f;
+      a.v[g][o + d] = 0.0f;
+      a.m[g][o + b] = 0.0f;
+      a.v[g][o + b] = 0.0f;
+    }
+  for (int c = 0; c < 3; ++c) {
+    a.p[0][c * np + d] = mean[c];
+    a.p[1][c * np + d] = ls_new[c];
+    a.p[1][c * np + b] = ls_new[c];
+  }
+}
+
 __global__ void opacity_reset_kernel(float* logits, float* m, float* v, int64_t n, float cap) {
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i >= n) return;
@@ -216,6 +314,20 @@ cudaError_t launch_densify_write(const DensifyArgs& a, uint4 totals, cudaStream_
   const int64_t nb = (a.n + kDensifyBlock - 1) / kDensifyBlock;
   if (nb == 0) return cudaSuccess;
   densify_write_kernel<<<static_cast<unsigned>(nb), kDensifyBlock, 0, st>>>(a, totals);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_relocate_classify(const RelocateArgs& a, cudaStream_t st) {
+  const int64_t nb = (a.n + kDensifyBlock - 1) / kDensifyBlock;
+  if (nb > 0) relocate_count_kernel<<<static_cast<unsigned>(nb), kDensifyBlock, 0, st>>>(a);
+  densify_scan_kernel<<<1, 1024, 0, st>>>(a.block_counts, nb, a.block_prefix, a.totals);
+  if (nb > 0) relocate_compact_kernel<<<static_cast<unsigned>(nb), kDensifyBlock, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_relocate_pairs(const RelocateArgs& a, cudaStream_t st) {
+  if (a.pairs == 0) return cudaSuccess;
+  relocate_pair_kernel<<<static_cast<unsigned>((a.pairs + 127) / 128), 128, 0, st>>>(a);
   return cudaGetLastError();
 }
 

@@ -48,6 +48,7 @@ struct gs_ctx {
   uint32_t* charb_counter = nullptr;
   // camera-pose gradient: caller's output (NULL when off) and the kernel's scratch
   double* cam_out = nullptr;
+  uint32_t* reloc_dead = nullptr;  // [max_g], allocated by the first gs_relocate
   double* cam_partials = nullptr;  // [kCamBlocks][9]
   uint32_t* cam_counter = nullptr;
   // readback record (device + pinned host); the device error word lives in it
@@ -110,7 +111,7 @@ void free_all(gs_ctx* c) {
                   c->dvals[1], c->dup_status, c->keys[0], c->keys[1], c->vals[0], c->vals[1],
                   c->hist, c->offsets, c->status, c->counters, c->ranges, c->surv, c->surv_count,
                   c->sgrad_fixed, c->dens_counts, c->dens_prefix, c->dens_totals, c->charb_partials,
-                  c->charb_counter, c->cam_partials, c->cam_counter, c->loss_partials,
+                  c->charb_counter, c->cam_partials, c->cam_counter, c->reloc_dead, c->loss_partials,
                   c->loss_counter, c->info_dev, c->pairs};
   for (void* b : bufs)
     if (b) cudaFree(b);
@@ -957,6 +958,84 @@ gs_status gs_densify(gs_ctx* c, const gs_params* in, const gs_grads* m_in, const
     return fail(c, GS_ERR_CAPACITY, "densification gives %lld Gaussians; the output holds %lld",
                 (long long)count, (long long)out_n_pad);
   GS_CUDA(c, gs::launch_densify_write(a, tot, st));
+  return GS_OK;
+}
+
+gs_status gs_relocate(gs_ctx* c, const gs_grads* params, const gs_grads* m, const gs_grads* v, int64_t n,
+                      int64_t n_pad, int32_t sh_degree, const float* normals, int64_t max_pairs,
+                      float dead_opacity, float donor_opacity, int64_t* n_pairs, void* stream) {
+  if (!c) return GS_ERR_INVALID_ARG;
+  if (!params || !m || !v || !n_pairs) return fail(c, GS_ERR_INVALID_ARG, "params, moments and n_pairs must be non-NULL");
+  *n_pairs = 0;
+  if (n < 0 || n_pad < n || n_pad % 4 != 0 || n > c->max_g)
+    return fail(c, GS_ERR_INVALID_ARG, "n must be in [0, max_gaussians], n_pad >= n and a multiple of 4");
+  if (sh_degree < 0 || sh_degree > 3) return fail(c, GS_ERR_INVALID_ARG, "sh_degree must be 0..3");
+  if (max_pairs < 0 || (max_pairs > 0 && (!normals || !aligned(normals, 4))))
+    return fail(c, GS_ERR_INVALID_ARG, "max_pairs must be >= 0 and normals non-NULL when it is > 0");
+  if (!(dead_opacity > 0.f && dead_opacity < donor_opacity && donor_opacity < 1.f))
+    return fail(c, GS_ERR_INVALID_ARG, "need 0 < dead_opacity < donor_opacity < 1");
+  const gs_grads* sets[3] = {params, m, v};
+  if (n > 0)
+    for (const gs_grads* g : sets) {
+      const float* q[5] = {g->means, g->log_scales, g->quats, g->opacity_logits, g->sh};
+      for (const float* x : q)
+        if (!x || !aligned(x, 4)) return fail(c, GS_ERR_INVALID_ARG, "a buffer pointer is NULL or misaligned");
+    }
+  if (n == 0 || max_pairs == 0) return GS_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (!c->reloc_dead) GS_CUDA(c, cudaMalloc(reinterpret_cast<void**>(&c->reloc_dead), sizeof(uint32_t) * c->max_g));
+  c->have_pre = c->have_fwd = false;  // the parameters change; so does the sort scratch
+  gs::RelocateArgs a{};
+  float* pp[5] = {params->means, params->log_scales, params->quats, params->opacity_logits, params->sh};
+  float* mm[5] = {m->means, m->log_scales, m->quats, m->opacity_logits, m->sh};
+  float* vv[5] = {v->means, v->log_scales, v->quats, v->opacity_logits, v->sh};
+  for (int k = 0; k < 5; ++k) {
+    a.p[k] = pp[k];
+    a.m[k] = mm[k];
+    a.v[k] = vv[k];
+  }
+  a.n = n;
+  a.np = n_pad;
+  a.sh_k = (sh_degree + 1) * (sh_degree + 1);
+  const double dd = dead_opacity, dn = donor_opacity;
+  a.dead_logit = std::log(dd / (1.0 - dd));
+  a.donor_logit = std::log(dn / (1.0 - dn));
+  a.block_counts = c->dens_counts;
+  a.block_prefix = c->dens_prefix;
+  a.totals = c->dens_totals;
+  a.dead = c->reloc_dead;
+  a.donor_keys = c->dkeys[0];
+  a.donor_vals = c->dvals[0];
+  a.err = &c->info_dev->device_error;
+  GS_CUDA(c, gs::launch_relocate_classify(a, st));
+  GS_CUDA(c, cudaMemcpyAsync(c->dens_host, c->dens_totals, sizeof(uint4), cudaMemcpyDeviceToHost, st));
+  GS_CUDA(c, cudaStreamSynchronize(st));
+  const int64_t dead = c->dens_host->x, donors = c->dens_host->y;
+  const int64_t pairs = std::min(std::min(dead, donors), max_pairs);
+  *n_pairs = pairs;
+  if (pairs == 0) return GS_OK;
+  // donors by descending size, stably (ties stay in index order)
+  gs::SortBuffers b;
+  b.keys[0] = c->dkeys[0];
+  b.keys[1] = c->dkeys[1];
+  b.vals[0] = c->dvals[0];
+  b.vals[1] = c->dvals[1];
+  b.hist = c->hist;
+  b.offsets = c->offsets;
+  b.status = c->status;
+  b.counters = c->counters;
+  b.err = &c->info_dev->device_error;
+  gs::SortPlan plan;
+  plan.n = donors;
+  plan.key_bits = 32;
+  plan.passes = 4;
+  plan.tiles = (donors + gs::kSortTileKeys - 1) / gs::kSortTileKeys;
+  int sorted = 0;
+  GS_CUDA(c, gs::launch_sort(plan, b, &sorted, st));
+  a.sorted_donors = c->dvals[sorted];
+  a.normals = normals;
+  a.pairs = pairs;
+  GS_CUDA(c, gs::launch_relocate_pairs(a, st));
   return GS_OK;
 }
 

@@ -241,6 +241,28 @@ cudaError_t launch_densify_count(const DensifyArgs& a, cudaStream_t st);
 cudaError_t launch_densify_write(const DensifyArgs& a, uint4 totals, cudaStream_t st);
 cudaError_t launch_opacity_reset(float* logits, float* m, float* v, int64_t n, float cap, cudaStream_t st);
 
+// Recycling dead Gaussians onto the largest donors, in place (count fixed).
+struct RelocateArgs {
+  float* p[5];  // means, log_scales, quats, opacity_logits, sh: planar with stride np, updated in place
+  float* m[5];  // Adam moments, same layout
+  float* v[5];
+  int64_t n, np;
+  int sh_k;
+  double dead_logit, donor_logit;  // logit < dead_logit: dead; logit > donor_logit: donor
+  uint4* block_counts;             // [blocks]: dead, donors
+  uint4* block_prefix;             // [blocks]: exclusive prefixes of the same
+  uint4* totals;                   // [1]
+  uint32_t* dead;                  // [n]: dead indices in index order
+  uint32_t* donor_keys;            // [n]: sort keys, largest log-scale first
+  uint32_t* donor_vals;            // [n]: donor indices in index order
+  const uint32_t* sorted_donors;   // the donor indices after the (stable) sort
+  const float* normals;            // [pairs][3] N(0, 1) draws
+  int64_t pairs;
+  uint32_t* err;
+};
+cudaError_t launch_relocate_classify(const RelocateArgs& a, cudaStream_t st);
+cudaError_t launch_relocate_pairs(const RelocateArgs& a, cudaStream_t st);
+
 // ---------------------------------------------------------------- Adam
 cudaError_t launch_adam(float* p, float* g, float* m, float* v, int64_t count, float lr,
                         float beta1, float beta2, float eps, int step, cudaStream_t st);

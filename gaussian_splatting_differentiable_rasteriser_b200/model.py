@@ -64,6 +64,14 @@ class GaussianModel:
             self.params[k] = self.flat[sl].view(shapes[k])
             self.grads[k] = self.grad_flat[sl].view(shapes[k])
 
+    def relocate(self, ctx, normals, dead_opacity=0.02, donor_opacity=0.4):
+        """Recycles dead Gaussians onto the largest donors in place (gs_relocate);
+        normals: [pairs, 3] float32 N(0, 1) draws on the device, one row per pair
+        at most. Returns the number of pairs made."""
+        em, ev = self.moments_structs()
+        return ctx.relocate(self._struct(self.params), em, ev, self.n, self.n_pad, self.sh_degree, normals,
+                            normals.shape[0], dead_opacity, donor_opacity)
+
     def densify(self, ctx, grad_accum, view_count, normals, grad_threshold, scale_threshold,
                 min_opacity, capacity=None):
         """One gs_densify pass into new buffers of `capacity` slots (default: room

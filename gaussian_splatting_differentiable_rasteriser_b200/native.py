@@ -27,7 +27,7 @@ EXPORTED = ("gs_create", "gs_destroy", "gs_last_error", "gs_preprocess", "gs_ren
             "gs_debug_screen_grads", "gs_set_option", "gs_loss_l1_dssim_noalloc",
             "gs_set_densify_stats", "gs_densify", "gs_opacity_reset", "gs_loss_charbonnier",
             "gs_adam_step_reduce", "gs_shared_alloc", "gs_shared_open", "gs_shared_close",
-            "gs_shared_free", "gs_set_camera_grad")
+            "gs_shared_free", "gs_set_camera_grad", "gs_relocate")
 GS_SHARED_HANDLE_BYTES = 64
 MAX_RANKS = 8
 GS_OPTION_OPACITY_RECT = 1
@@ -104,6 +104,8 @@ def load(path: str = LIB_PATH):
     L.gs_shared_close.argtypes = [P]
     L.gs_shared_free.argtypes = [P]
     L.gs_set_camera_grad.argtypes = [P, P]
+    L.gs_relocate.argtypes = [P, ctypes.POINTER(GsGrads), ctypes.POINTER(GsGrads), ctypes.POINTER(GsGrads),
+                              I64, I64, I32, P, I64, F, F, ctypes.POINTER(I64), P]
     L.gs_set_option.argtypes = [P, I32, I32]
     L.gs_set_option.restype = ctypes.c_int
     L.gs_loss_l1_dssim_noalloc.argtypes = [P, P, I32, I32, F, P, P, P]
@@ -188,6 +190,16 @@ class Context:
         `out` (6 float64 on the device); None turns it off."""
         self._out_cam = out  # kept alive while the context points at it
         self._check(self.L.gs_set_camera_grad(self.h, _ptr(out)))
+
+    def relocate(self, params: GsGrads, m: GsGrads, v: GsGrads, n, n_pad, sh_degree, normals, max_pairs,
+                 dead_opacity=0.02, donor_opacity=0.4, stream=None) -> int:
+        """gs_relocate in place; returns the number of pairs made."""
+        n_pairs = ctypes.c_int64(0)
+        self._check(self.L.gs_relocate(self.h, ctypes.byref(params), ctypes.byref(m), ctypes.byref(v), int(n),
+                                       int(n_pad), int(sh_degree), _ptr(normals), int(max_pairs),
+                                       float(dead_opacity), float(donor_opacity), ctypes.byref(n_pairs),
+                                       _stream(stream)))
+        return n_pairs.value
 
     def set_densify_stats(self, grad_accum, view_count):
         self._check(self.L.gs_set_densify_stats(self.h, _ptr(grad_accum), _ptr(view_count)))

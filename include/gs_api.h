@@ -441,6 +441,31 @@ gs_status gs_densify(gs_ctx *ctx, const gs_params *in, const gs_grads *m_in, con
  * heuristic": reset clamps opacity down to at most 0.01, the usual
  * max_opacity). All pointers DEVICE, [n] floats. Errors: GS_ERR_INVALID_ARG
  * for NULL pointers, n < 0 or max_opacity outside (0, 1). */
+/* Recycling dead Gaussians, in place ([GS] "Densification: cloning the busy
+ * blobs, recycling the dead", the variant with a fixed count). Among the first
+ * n Gaussians, dead ones (opacity < dead_opacity) and donors (opacity >
+ * donor_opacity) are found from the logits (decided in float64); the donors are
+ * ranked largest first (largest log-scale, ties by index) and the j-th dead
+ * Gaussian in index order is paired with the j-th donor, for j < min(dead,
+ * donors, max_pairs). For each pair (d, b): slot d becomes a copy of b placed
+ * at mean_b + R(q_b) diag(exp(log_scales_b)) z_j, with z_j = normals[3j..3j+2]
+ * (DEVICE, float32 N(0, 1) draws supplied by the caller); both d and b take
+ * log-scales log_scales_b - ln 1.6 ("both halves shrink"); both restart their
+ * Adam moments (m and v zeroed in every group). Every other slot is left as
+ * it was. params, m and v are the planar buffers of the parameters and of the
+ * two Adam moments (mutable, same layout as gs_params, n_pad columns), updated
+ * in place. The number of pairs made is written to the HOST int64 *n_pairs
+ * (the call waits on the stream once to read the counts). It uses the
+ * context's sort scratch, so the camera in flight is discarded (call
+ * gs_preprocess again). Errors: GS_ERR_INVALID_ARG for NULL or misaligned
+ * pointers, n > max_gaussians, n_pad < n or not a multiple of 4, sh_degree
+ * outside 0..3, max_pairs < 0 (or > 0 with NULL normals), or thresholds not
+ * satisfying 0 < dead_opacity < donor_opacity < 1; GS_ERR_CUDA if a launch or
+ * the scratch allocation fails. */
+gs_status gs_relocate(gs_ctx *ctx, const gs_grads *params, const gs_grads *m, const gs_grads *v, int64_t n,
+                      int64_t n_pad, int32_t sh_degree, const float *normals, int64_t max_pairs,
+                      float dead_opacity, float donor_opacity, int64_t *n_pairs, void *stream);
+
 gs_status gs_opacity_reset(float *opacity_logits, float *m_logits, float *v_logits, int64_t n,
                            float max_opacity, void *stream);
 

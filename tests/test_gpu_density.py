@@ -142,3 +142,38 @@ def test_opacity_reset_matches_oracle(gs):
     below = logits.astype(np.float64) <= ref
     np.testing.assert_array_equal(host(tl)[below], logits[below])
     assert not host(tm).any() and not host(tv).any()
+
+
+@pytest.mark.parametrize("rows", [40, 400])
+def test_relocation_matches_oracle(gs, rows):
+    """gs_relocate in place against the oracle's recycling: the same pairs (the
+    first `rows` pairs, or every dead Gaussian when there are fewer), the
+    recycled and shrunk Gaussians within float32 rounding, every other slot
+    bit for bit as before, and the reshaped Gaussians' moments at zero."""
+    native, model = gs
+    s = scenes.small()
+    m = model.GaussianModel(s)
+    ctx = native.Context(s.n_pad, 1 << 16, 64, 64)
+    gen = torch.Generator(device="cuda").manual_seed(1)
+    m.m_flat.normal_(0.0, 1e-3, generator=gen)
+    m.v_flat.uniform_(0.0, 1e-6, generator=gen)
+    groups = scenes.GROUP_NAMES
+    p0 = {k: host(m.params[k]).copy() for k in groups}
+    m0 = {k: host(m.m[k]).copy() for k in groups}
+    v0 = {k: host(m.v[k]).copy() for k in groups}
+    normals = np.random.default_rng(3).normal(size=(rows, 3)).astype(np.float32)
+    pairs = m.relocate(ctx, torch.from_numpy(normals).cuda())
+    torch.cuda.synchronize()
+    rp, rm, rv, ref_pairs = oracle.relocate(p0, m0, v0, s.n, normals)
+    assert pairs == len(ref_pairs) > 0
+    if rows == 40:
+        assert pairs == 40
+    touched = sorted({i for pr in ref_pairs for i in pr})
+    other = np.setdiff1d(np.arange(s.n_pad), touched)
+    for k in groups:
+        gp, gm, gv = host(m.params[k]), host(m.m[k]), host(m.v[k])
+        np.testing.assert_array_equal(gp[..., other], p0[k][..., other])
+        np.testing.assert_array_equal(gm[..., other], m0[k][..., other])
+        np.testing.assert_array_equal(gv[..., other], v0[k][..., other])
+        np.testing.assert_allclose(gp[..., touched], rp[k][..., touched], rtol=1e-6, atol=1e-6)
+        assert not gm[..., touched].any() and not gv[..., touched].any()
