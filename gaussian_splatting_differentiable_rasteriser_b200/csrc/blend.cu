@@ -158,6 +158,7 @@ __global__ void __launch_bounds__(256) blend_forward_kernel(BlendArgs a) {
     __syncwarp();
     const int cnt = __popc(mask);
     nsurv += cnt;
+    int last_k = -1;  // slot of this chunk's last blended survivor
     for (int k = 0; k < cnt; ++k) {
       const float2 xy = ws.xy[k];
       const float p = power2(ws.q[k], fx - xy.x, fy - xy.y);
@@ -170,10 +171,11 @@ __global__ void __launch_bounds__(256) blend_forward_kernel(BlendArgs a) {
         C1 = __fmaf_rn(w, c.y, C1);
         C2 = __fmaf_rn(w, c.z, C2);
         T = T * (1.0f - alpha);
-        last = ws.pos[k] + 1;
+        last_k = k;
         done = T < kTMin;
       }
     }
+    if (last_k >= 0) last = ws.pos[last_k] + 1;
     __syncwarp();  // the slots are rewritten by the next chunk
   }
   if (lane == 0) a.surv_count[tile * kWarps + warp] = static_cast<uint32_t>(nsurv);

@@ -201,7 +201,8 @@ __global__ void __launch_bounds__(kLossThreads, 4) loss_kernel(LossArgs a) {
           const float sxy = acc[4][o] - mux * muy;
           const float A1 = 2.f * mux * muy + C1, A2 = 2.f * sxy + C2;
           const float B1 = mux * mux + muy * muy + C1, B2 = sxx + syy + C2;
-          const float iB1 = 1.0f / B1, iB2 = 1.0f / B2;
+          // B1 >= C1 and B2 >= C2 > 0: the fast reciprocal is accurate to a few ulp here
+          const float iB1 = __fdividef(1.0f, B1), iB2 = __fdividef(1.0f, B2);
           const float iB = iB1 * iB2;
           const float S = A1 * A2 * iB;
           // partials with mu_y, E[y^2] fixed: sxx = E[x^2] - mux^2, sxy = E[xy] - mux muy
