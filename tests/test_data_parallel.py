@@ -1,13 +1,14 @@
 """The data-parallel exchange step on the host with the gloo backend, world
 size 2: the reduce-scatter / sharded Adam / all-gather leaves both ranks with
 the parameters of one Adam step on the batch-mean gradient, as the float64
-oracle computes it on the whole buffer; plus the sharding arithmetic."""
+oracle computes it on the whole buffer; the sharding arithmetic and the peer
+addresses of the fused exchange; and a rank that fails before the exchange
+makes its peer's collective fail instead of hang."""
 import os
 import socket
 import sys
 
 import numpy as np
-import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 

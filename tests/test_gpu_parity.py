@@ -5,8 +5,6 @@ absolute (pixels whose oracle walk came within a hair of a threshold are
 excluded and counted); loss within 1e-5 relative; per-group gradients within
 1e-3 relative L2; Adam within float32 rounding of the float64 update.
 """
-import math
-
 import numpy as np
 import pytest
 
