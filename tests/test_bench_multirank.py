@@ -2,7 +2,8 @@
 size 2: process-group set-up from the launcher's environment, the barrier,
 the max-over-ranks timing and the whole-job aggregate of independent replicas,
 and the reference arm under the launcher (rank 0 prints the one line, the
-other rank exits without work)."""
+other rank exits without work); plus the roofline arithmetic and the scaling
+of the ncu traffic figures."""
 import json
 import os
 import socket
@@ -63,3 +64,37 @@ def test_reference_arm_under_the_launcher_prints_once():
     assert line["impl"] == "reference" and line["n_gpus"] == 2
     assert line["value"] > 0 and line["e2e"]["value"] == line["value"]
     assert line["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_roofline_arithmetic():
+    """achieved = algorithmic bytes (or FP32 instructions) per launch / launch time;
+    frac = achieved / peak; the fused pass moves 59 x 24 + 101 B per Gaussian."""
+    sys.path.insert(0, ROOT)
+    import types
+
+    import bench
+    scene = types.SimpleNamespace(sh_k=16, n=3_000_000, n_pad=3_000_000)
+    prof = {"backward_adam": {"ms": 2.0, "launches": 2, "work": 6_000_000, "blended": 0},
+            "blend_forward": {"ms": 1.0, "launches": 2, "work": 4_000_000, "blended": 1_000_000},
+            "scan": {"ms": 0.1, "launches": 1, "work": 0, "blended": 0}}
+    per = bench.roofline(prof, scene, 6555.2, 1965.0)
+    assert "scan" not in per  # no model, no roofline entry
+    ba = per["backward_adam"]
+    assert ba["bound"] == "hbm" and ba["unit"] == "GB/s"
+    assert ba["achieved"] == pytest.approx(3_000_000 * (59 * 24 + 101) / 1e-3 / 1e9)
+    assert ba["frac"] == pytest.approx(ba["achieved"] / 6555.2)
+    bf = per["blend_forward"]
+    peak = 148 * 128 * 1965.0e6 / 1e12
+    assert bf["bound"] == "alu" and bf["peak"] == pytest.approx(peak)
+    assert bf["achieved"] == pytest.approx((2_000_000 * 7 + 500_000 * 6) / 0.5e-3 / 1e12)
+
+
+def test_traffic_figures_scale_per_unit_of_work():
+    sys.path.insert(0, ROOT)
+    import bench
+    per_g, unit, _ = bench.NCU_TRAFFIC["backward_adam"]
+    assert unit == "gaussians"
+    # at Mid (500,000 Gaussians) the figure is the captured launch's read + write bytes
+    assert per_g * 500_000 == pytest.approx(409.251584e6 + 290.841600e6)
+    per_e, unit, _ = bench.NCU_TRAFFIC["blend_backward"]
+    assert unit == "entries" and per_e * 1.064e6 == pytest.approx(85.220352e6 + 2.926336e6)
