@@ -1,7 +1,11 @@
 /*
  * gs_api.h - C ABI of the B200 (sm_100a) differentiable tile-based
  * Gaussian-splat rasteriser: preprocess, tile sort + forward blend, fused
- * L1 + D-SSIM loss, blend + projection backward, and a fused Adam step.
+ * L1 + D-SSIM loss, blend + projection backward, and a fused Adam step; plus
+ * the training loop's other steps on the same data: the Charbonnier +
+ * exposure loss, camera-pose gradients, adaptive density control and the
+ * recycling of dead Gaussians, and the data-parallel gradient exchange fused
+ * with Adam over peer memory.
  *
  * Conventions shared by every call
  *   - Every data pointer is a DEVICE pointer owned by the caller, unless the
