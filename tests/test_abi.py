@@ -1,5 +1,6 @@
 """The C ABI library loads on a machine without a GPU and exports every entry
-point the public header declares (no compute call is made)."""
+point the public header declares; argument checks that come before any CUDA
+call are exercised here too (no compute call is made)."""
 import ctypes
 import os
 import re
@@ -49,3 +50,35 @@ def test_stage_names_match_the_binding():
     L = native.load()
     assert [L.gs_stage_name(k).decode() for k in range(len(native.STAGES))] == list(native.STAGES)
     assert L.gs_stage_name(len(native.STAGES)).decode() == ""
+
+
+def test_new_entry_points_check_their_arguments_on_the_host():
+    """The data-parallel, shared-memory, camera-gradient and recycling entry
+    points reject bad arguments before any CUDA call (so this runs without a GPU)."""
+    from gaussian_splatting_differentiable_rasteriser_b200 import native
+    L = native.load()
+    bad = native.GS_ERR_INVALID_ARG
+    P = ctypes.c_void_p
+    grads = (P * 1)(P(16))
+    # gs_adam_step_reduce: no gradient source, too many, negative count, step 0, bad betas
+    for n_grads, count, step, b1 in ((0, 4, 1, 0.9), (9, 4, 1, 0.9), (1, -1, 1, 0.9), (1, 4, 0, 0.9),
+                                     (1, 4, 1, 1.0)):
+        assert L.gs_adam_step_reduce(None, None, None, count, grads, n_grads, None, 0, 0, 1.0, 1e-3, b1,
+                                     0.999, 1e-8, step, None) == bad
+    # copies requested with no array
+    assert L.gs_adam_step_reduce(None, None, None, 4, grads, 1, None, 1, 0, 1.0, 1e-3, 0.9, 0.999, 1e-8, 1,
+                                 None) == bad
+    # shared buffers: no size, no outputs, no handle, nothing to close or free
+    p = P()
+    h = ctypes.create_string_buffer(native.GS_SHARED_HANDLE_BYTES)
+    assert L.gs_shared_alloc(0, ctypes.byref(p), h) == bad
+    assert L.gs_shared_alloc(64, None, h) == bad
+    assert L.gs_shared_open(None, ctypes.byref(p)) == bad
+    assert L.gs_shared_close(None) == bad
+    assert L.gs_shared_free(None) == bad
+    # camera gradient and recycling need a context
+    assert L.gs_set_camera_grad(None, None) == bad
+    n_pairs = ctypes.c_int64(-1)
+    g = native.GsGrads()
+    assert L.gs_relocate(None, ctypes.byref(g), ctypes.byref(g), ctypes.byref(g), 0, 0, 0, None, 0, 0.02, 0.4,
+                         ctypes.byref(n_pairs), None) == bad
