@@ -94,6 +94,29 @@ class GaussianModel:
         for k in GROUP_NAMES:
             self.params[k].copy_(torch.from_numpy(getattr(scene, k)).to(torch.float32))
 
+    def state_dict(self) -> dict:
+        """Training state for torch.save: parameters and both Adam moments (flat,
+        planar group layout, copied to the host), sizes, degrees and the step count.
+        The gradient buffer is not saved: it is zero between iterations."""
+        return {"flat": self.flat.detach().cpu().clone(), "m_flat": self.m_flat.detach().cpu().clone(),
+                "v_flat": self.v_flat.detach().cpu().clone(), "n": self.n, "n_pad": self.n_pad,
+                "sh_degree": self.sh_degree, "active_degree": self.active_degree,
+                "step_count": self.step_count}
+
+    def load_state_dict(self, state: dict):
+        """Restores a state_dict (reallocating if the padded size differs)."""
+        if state["sh_degree"] != self.sh_degree:
+            raise ValueError("the state was saved with another SH degree")
+        if state["n_pad"] != self.n_pad:
+            self._alloc(state["n_pad"])
+        self.flat.copy_(state["flat"])
+        self.m_flat.copy_(state["m_flat"])
+        self.v_flat.copy_(state["v_flat"])
+        self.grad_flat.zero_()
+        self.n = state["n"]
+        self.active_degree = state["active_degree"]
+        self.step_count = state["step_count"]
+
     def params_struct(self) -> native.GsParams:
         p = native.GsParams()
         for k in GROUP_NAMES:
