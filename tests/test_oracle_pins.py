@@ -288,6 +288,98 @@ def test_adam_constant_gradient_closed_form():
         assert not g.any()
 
 
+def _adam_closed_form(p0, grads, lr, beta1, beta2, eps):
+    """Adam's trajectory from the sums the recursion unrolls to (no recursion):
+    m_t = (1 - b1) sum_k b1^(t-k) g_k and v_t = (1 - b2) sum_k b2^(t-k) g_k^2,
+    divided by the bias corrections 1 - b1^t and 1 - b2^t, then
+    p_t = p_(t-1) - lr m_hat_t / (sqrt(v_hat_t) + eps). Returns every p_t, m_t, v_t."""
+    p = np.array(p0, np.float64)
+    out = []
+    for t in range(1, len(grads) + 1):
+        m_t = (1 - beta1) * sum(beta1 ** (t - k) * grads[k - 1] for k in range(1, t + 1))
+        v_t = (1 - beta2) * sum(beta2 ** (t - k) * grads[k - 1] ** 2 for k in range(1, t + 1))
+        m_hat = m_t / (1 - beta1 ** t)
+        v_hat = v_t / (1 - beta2 ** t)
+        p = p - lr * m_hat / (np.sqrt(v_hat) + eps)
+        out.append((p.copy(), m_t, v_t))
+    return out
+
+
+def test_adam_varying_gradients_match_the_unrolled_sums():
+    """Three steps with different gradients (signs and sizes change from step to
+    step) and beta1 != beta2: the oracle's recursion must give the unrolled
+    moment sums, their bias corrections at the step's own power, and the
+    parameter trajectory. The constant-gradient test cannot tell beta1 from
+    beta2 (m_hat = g, v_hat = g^2 whichever decays which); this one can."""
+    rng = np.random.default_rng(15)
+    n = 64
+    p0 = rng.normal(0, 1, n)
+    grads = [rng.normal(0, 1, n) * s for s in (1.0, 3e-2, 5.0)]
+    grads[1][::3] *= -40.0  # some gradients flip sign and grow between steps
+    lr, b1, b2, eps = 1e-2, 0.9, 0.999, 1e-8
+    want = _adam_closed_form(p0, grads, lr, b1, b2, eps)
+    p, m, v = p0.copy(), np.zeros(n), np.zeros(n)
+    for t, g in enumerate(grads, start=1):
+        p, gz, m, v = oracle.adam(p, g, m, v, lr, t, beta1=b1, beta2=b2, eps=eps)
+        wp, wm, wv = want[t - 1]
+        np.testing.assert_allclose(m, wm, rtol=1e-13, atol=1e-300)
+        np.testing.assert_allclose(v, wv, rtol=1e-13, atol=1e-300)
+        np.testing.assert_allclose(p, wp, rtol=1e-13, atol=1e-15)
+        assert not gz.any()
+    # The same sums with the betas swapped, or with a bias correction one power
+    # off, land far outside that tolerance: the comparison above can see both.
+    swapped = _adam_closed_form(p0, grads, lr, b2, b1, eps)[-1][0]
+    assert np.abs(swapped - p).max() > 1e-4
+    off_by_one = p0.copy()
+    for t in range(1, 4):
+        m_t = (1 - b1) * sum(b1 ** (t - k) * grads[k - 1] for k in range(1, t + 1))
+        v_t = (1 - b2) * sum(b2 ** (t - k) * grads[k - 1] ** 2 for k in range(1, t + 1))
+        off_by_one = off_by_one - lr * (m_t / (1 - b1 ** (t + 1))) / (np.sqrt(v_t / (1 - b2 ** t)) + eps)
+    assert np.abs(off_by_one - p).max() > 1e-4
+
+
+def test_adam_scalar_worked_by_hand():
+    """Two steps on one scalar, every intermediate written out by hand:
+    g1 = 2:  m1 = 0.2,  v1 = 0.004,  m_hat = 2,  v_hat = 4,  p1 = 1 - 0.1 * 2 / (2 + eps)
+    g2 = -1: m2 = 0.9 * 0.2 - 0.1 = 0.08,  v2 = 0.999 * 0.004 + 0.001 = 0.004996,
+             m_hat = 0.08 / 0.19,  v_hat = 0.004996 / 0.001999,
+             p2 = p1 - 0.1 * m_hat / (sqrt(v_hat) + eps)."""
+    eps = 1e-8
+    p, _, m, v = oracle.adam([1.0], [2.0], [0.0], [0.0], 0.1, 1, eps=eps)
+    assert m[0] == pytest.approx(0.2, rel=1e-15)
+    assert v[0] == pytest.approx(0.004, rel=1e-14)
+    p1 = 1.0 - 0.1 * 2.0 / (2.0 + eps)
+    assert p[0] == pytest.approx(p1, rel=1e-15)
+    p, _, m, v = oracle.adam(p, [-1.0], m, v, 0.1, 2, eps=eps)
+    assert m[0] == pytest.approx(0.08, rel=1e-14)
+    assert v[0] == pytest.approx(0.004996, rel=1e-14)
+    m_hat = 0.08 / 0.19
+    v_hat = 0.004996 / 0.001999
+    assert p[0] == pytest.approx(p1 - 0.1 * m_hat / (math.sqrt(v_hat) + eps), rel=1e-14)
+
+
+def test_adam_matches_torch_float64():
+    """Library pin: torch.optim.Adam in float64 (its default betas and eps are the
+    oracle's) over four steps of changing gradients, per-group learning rates."""
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(16)
+    n = 40
+    p0 = rng.normal(0, 1, n)
+    grads = [rng.normal(0, 1, n) * (10.0 ** rng.uniform(-3, 1)) for _ in range(4)]
+    for lr in (1e-3, 0.05):
+        w = torch.tensor(p0.copy(), dtype=torch.float64, requires_grad=True)
+        opt = torch.optim.Adam([w], lr=lr, betas=(0.9, 0.999), eps=1e-8)
+        p, m, v = p0.copy(), np.zeros(n), np.zeros(n)
+        for t, g in enumerate(grads, start=1):
+            w.grad = torch.tensor(g, dtype=torch.float64)
+            opt.step()
+            p, _, m, v = oracle.adam(p, g, m, v, lr, t)
+            np.testing.assert_allclose(p, w.detach().numpy(), rtol=1e-12, atol=1e-15)
+            st = opt.state[w]
+            np.testing.assert_allclose(m, st["exp_avg"].numpy(), rtol=1e-13, atol=1e-300)
+            np.testing.assert_allclose(v, st["exp_avg_sq"].numpy(), rtol=1e-13, atol=1e-300)
+
+
 # ------------------------------------------------------------------------ SH
 def test_sh_printed_constants(gold):
     g = gold("sh_constants.txt")
