@@ -52,4 +52,19 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int ma
   return false;
 }
 
+// After a bounded wait has given up: keeps waiting for the phase with a
+// backoff (1 us sleeps, about `max_us` microseconds in all), so that the CTA
+// does not retire - and its shared memory is not handed to another CTA -
+// while copies into it may still be in flight. Returns true if the phase
+// completed. The copies only fail to land when the memory system has faulted;
+// if even this wait gives up, the CTA retires with the copies outstanding and
+// the recorded error makes the launch's results unusable.
+__device__ __forceinline__ bool mbar_drain(uint64_t* bar, uint32_t parity, int max_us) {
+  for (int k = 0; k < max_us; ++k) {
+    if (mbar_wait(bar, parity, 1)) return true;
+    __nanosleep(1000);
+  }
+  return false;
+}
+
 }  // namespace gs

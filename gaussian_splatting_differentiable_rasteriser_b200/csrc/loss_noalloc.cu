@@ -1,9 +1,10 @@
 // A variant of the fused loss entry point that allocates nothing.
 //
 // Some callers cannot call cudaMalloc at the point where they need the loss:
-// code being recorded into a CUDA graph (an allocation there is not allowed),
-// real-time loops whose memory is fixed after start-up, and hosts that give
-// the library device pointers for inputs and outputs but no allocator. For
+// a host application whose own allocator owns the GPU's memory and gives the
+// library device pointers for inputs and outputs but no allocator, and
+// real-time loops whose memory is fixed after start-up (cudaMalloc can
+// synchronise the device and stall such a loop). For
 // them, gs_loss_l1_dssim_noalloc runs the same loss kernel as
 // gs_loss_l1_dssim, with the kernel's scratch (one pair of float64 partial
 // sums per CTA and the completion counter) in file-scope __device__ arrays of
@@ -13,7 +14,9 @@
 // holds them (about 0.2 MB) until the process exits. In host code the array
 // names are host-side stand-ins, not device addresses, so the device address
 // is taken once per device with cudaGetSymbolAddress while that device is
-// current, and that address is what the kernel receives.
+// current, and that address is what the kernel receives. The first call on a
+// device does that lookup, so it should come before any stream capture. All
+// calls on a device share the arrays: calls that overlap on the GPU race.
 #include <cmath>
 #include <mutex>
 

@@ -70,8 +70,10 @@ __global__ void __launch_bounds__(kPreThreads, 3) preprocess_kernel(PreprocessAr
                       a.sh + (static_cast<int64_t>(ch) * a.sh_k + k) * np + i0, bytes, &sm.bar);
     bool ok = mbar_wait(&sm.bar, 0, 1 << 16);
     if (!ok) {
+      // Nothing computed from this slice is used (the error fails the
+      // launch), but the CTA must not retire before its copies have landed.
       record_error(a.err, kErrCopyTimeout);
-      mbar_wait(&sm.bar, 0, 1 << 16);  // let the copies land before the CTA can exit
+      mbar_drain(&sm.bar, 0, 2000000);
     }
     sm.ok = ok ? 1 : 0;
   }

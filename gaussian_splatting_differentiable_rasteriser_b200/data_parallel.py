@@ -70,6 +70,25 @@ def exchange_and_update(grad_pad, param_pad, m_flat, v_flat, slices, total, worl
     grad_pad.zero_()
 
 
+def gather_shards(flat, total, world, rank, group=None):
+    """The full buffer of `total` floats assembled from every rank's own shard of
+    `flat` (each rank's values outside its shard are ignored): the Adam moments
+    of a data-parallel model, where each rank updates only its shard. A copy on
+    the same device; `flat` itself is untouched."""
+    collective = dist.is_available() and dist.is_initialized() and world > 1
+    if not collective:
+        return flat[:total].clone()
+    pad = padded_size(total, world)
+    lo, hi = shard_bounds(total, world, rank)
+    mine = torch.zeros(hi - lo, dtype=flat.dtype, device=flat.device)
+    top = min(hi, total)
+    if lo < top:
+        mine[: top - lo].copy_(flat[lo:top])
+    out = torch.empty(pad, dtype=flat.dtype, device=flat.device)
+    dist.all_gather_into_tensor(out, mine, group=group)
+    return out[:total].clone()
+
+
 def p2p_pieces(slices, total, world, rank, param_ptrs, grad_ptrs):
     """The gs_adam_step_reduce calls of one rank: for each parameter-group piece
     of its shard, (group, start, stop, gradient source addresses in rank order,
@@ -138,7 +157,7 @@ class DataParallelTrainStep(TrainStep):
             self.param_pad = torch.zeros(pad, dtype=torch.float32, device=dev)
             self.grad_pad = torch.zeros(pad, dtype=torch.float32, device=dev)
         self.param_pad[: self.total].copy_(model.flat)
-        model.attach_storage(self.param_pad[: self.total], self.grad_pad[: self.total])
+        model.attach_storage(self.param_pad[: self.total], self.grad_pad[: self.total], owner=self)
         self._flag = torch.zeros(1, dtype=torch.float32, device=dev)
         self._nccl = on and dist.get_backend(group) == "nccl"
 
@@ -181,6 +200,23 @@ class DataParallelTrainStep(TrainStep):
         if not one:
             self._barrier()  # every shard is read and every copy written
             self.grad_pad.zero_()
+
+    def state_dict(self) -> dict:
+        """The model's training state with the Adam moments of every rank's shard
+        gathered (collective: every rank calls it; every rank gets the full state)."""
+        m = self.model
+        mf = gather_shards(m.m_flat, self.total, self.world, self.rank, self.group)
+        vf = gather_shards(m.v_flat, self.total, self.world, self.rank, self.group)
+        return m.state_dict(m_flat=mf, v_flat=vf)
+
+    def load_state_dict(self, state: dict):
+        """Restores a full state (as state_dict gives) on this rank: the parameters into
+        the shared buffers, the moments of every shard, the step count. The state must
+        have this step's sizes."""
+        m = self.model
+        if int(state["n_pad"]) != m.n_pad:
+            raise ValueError("the state has another size: build a new step for it")
+        m.load_state_dict(state)
 
     def close(self):
         """Unmaps the other ranks' buffers; collective when there are several ranks

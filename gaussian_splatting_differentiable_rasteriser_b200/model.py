@@ -27,6 +27,8 @@ class GaussianModel:
         self.n, self.sh_degree = scene.n, scene.sh_degree
         self.active_degree = scene.sh_degree if active_degree is None else active_degree
         self.device = device
+        # set while a data-parallel step owns the parameter and gradient storage
+        self.storage_owner = None
         self._alloc(scene.n_pad)
         self.load(scene)
         self.step_count = 0
@@ -53,10 +55,14 @@ class GaussianModel:
             self.v[k] = self.v_flat[sl].view(shapes[k])
             off += sizes[k]
 
-    def attach_storage(self, flat, grad_flat):
+    def attach_storage(self, flat, grad_flat, owner=None):
         """Moves the parameters and gradients into the given flat buffers (same size;
-        the current parameters must already be in `flat`) and rebuilds the group views."""
+        the current parameters must already be in `flat`) and rebuilds the group views.
+        `owner` (the data-parallel step that made the buffers) is recorded: while it is
+        set, state_dict() refuses (the owner's state_dict gathers the moments of every
+        rank) and load_state_dict() refuses a change of size."""
         assert flat.numel() == self.flat.numel() and grad_flat.numel() == self.grad_flat.numel()
+        self.storage_owner = owner
         self.flat, self.grad_flat = flat, grad_flat
         shapes = group_shapes(self.n_pad, self.sh_degree)
         for k in GROUP_NAMES:
@@ -94,21 +100,39 @@ class GaussianModel:
         for k in GROUP_NAMES:
             self.params[k].copy_(torch.from_numpy(getattr(scene, k)).to(torch.float32))
 
-    def state_dict(self) -> dict:
+    def state_dict(self, m_flat=None, v_flat=None) -> dict:
         """Training state for torch.save: parameters and both Adam moments (flat,
         planar group layout, copied to the host), sizes, degrees and the step count.
-        The gradient buffer is not saved: it is zero between iterations."""
-        return {"flat": self.flat.detach().cpu().clone(), "m_flat": self.m_flat.detach().cpu().clone(),
-                "v_flat": self.v_flat.detach().cpu().clone(), "n": self.n, "n_pad": self.n_pad,
+        The gradient buffer is not saved: it is zero between iterations. Refused while
+        a data-parallel step owns the storage, since each rank then holds the moments
+        of its own shard only: save through that step's state_dict(), which passes the
+        gathered moments here."""
+        if self.storage_owner is not None and m_flat is None:
+            raise RuntimeError("a data-parallel step owns this model's storage: save with its state_dict()")
+        m_flat = self.m_flat if m_flat is None else m_flat
+        v_flat = self.v_flat if v_flat is None else v_flat
+        return {"flat": self.flat.detach().cpu().clone(), "m_flat": m_flat.detach().cpu().clone(),
+                "v_flat": v_flat.detach().cpu().clone(), "n": self.n, "n_pad": self.n_pad,
                 "sh_degree": self.sh_degree, "active_degree": self.active_degree,
                 "step_count": self.step_count}
 
     def load_state_dict(self, state: dict):
-        """Restores a state_dict (reallocating if the padded size differs)."""
+        """Restores a state_dict (reallocating if the padded size differs; refused
+        while a data-parallel step owns the storage, whose buffers keep their size:
+        build a new step for another size)."""
         if state["sh_degree"] != self.sh_degree:
             raise ValueError("the state was saved with another SH degree")
-        if state["n_pad"] != self.n_pad:
-            self._alloc(state["n_pad"])
+        n, n_pad = int(state["n"]), int(state["n_pad"])
+        if not 0 <= n <= n_pad or n_pad % 4:
+            raise ValueError("the state's sizes are inconsistent (need 0 <= n <= n_pad, n_pad % 4 == 0)")
+        total = sum(int(torch.Size(s).numel()) for s in group_shapes(n_pad, self.sh_degree).values())
+        for k in ("flat", "m_flat", "v_flat"):
+            if state[k].numel() != total:
+                raise ValueError(f"the state's {k} holds {state[k].numel()} floats, its sizes need {total}")
+        if n_pad != self.n_pad:
+            if self.storage_owner is not None:
+                raise RuntimeError("a data-parallel step owns this model's storage: its size cannot change")
+            self._alloc(n_pad)
         self.flat.copy_(state["flat"])
         self.m_flat.copy_(state["m_flat"])
         self.v_flat.copy_(state["v_flat"])

@@ -202,10 +202,12 @@ gs_status gs_render_backward(gs_ctx *ctx, const gs_params *params, const gs_came
                              const float *dloss_dimage, gs_grads *grads, void *stream);
 
 /* Step 3 without allocation - the same fused loss as gs_loss_l1_dssim, for
- * callers that cannot allocate device memory where they need the loss (code
- * being captured into a CUDA graph, loops whose memory is fixed after
- * start-up, hosts that hand over only input and output pointers). The pages
- * describe no counterpart; this is an interface convenience of this library.
+ * callers that cannot allocate device memory where they need the loss: a
+ * host application whose own allocator owns the GPU's memory and hands the
+ * library only input and output pointers, and real-time loops whose memory is
+ * fixed after start-up (cudaMalloc can synchronise the device and stall the
+ * loop). The paper has no counterpart; this is an interface convenience of
+ * this library.
  * It needs no context: the kernel's scratch (per-CTA partial sums and a
  * completion counter, about 0.2 MB) is a file-scope __device__ array that
  * every GPU loading the library holds until the process exits. The first call

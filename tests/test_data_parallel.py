@@ -151,3 +151,89 @@ def test_a_rank_that_fails_before_the_exchange_makes_the_others_fail_not_hang(tm
                        start_method="spawn")
     assert (tmp_path / "status1.txt").read_text().startswith("error")
     assert (tmp_path / "status0.txt").read_text().startswith("error")
+
+
+def _rank_state(rank, world, port, out_dir):
+    os.environ.update(RANK=str(rank), WORLD_SIZE=str(world), MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    from gaussian_splatting_differentiable_rasteriser_b200 import data_parallel as dp
+    from gaussian_splatting_differentiable_rasteriser_b200 import model, scenes
+    dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+    m = model.GaussianModel(scenes.small(), device="cpu")
+    total = m.flat.numel()
+    g = torch.Generator().manual_seed(3)
+    M = torch.randn(total, generator=g)
+    V = torch.rand(total, generator=g)
+    # after data-parallel steps a rank's moments are right on its own shard only
+    lo, hi = dp.shard_bounds(total, world, rank)
+    m.m_flat.fill_(100.0 + rank)
+    m.v_flat.fill_(-1.0 - rank)
+    m.m_flat[lo:min(hi, total)] = M[lo:min(hi, total)]
+    m.v_flat[lo:min(hi, total)] = V[lo:min(hi, total)]
+    m.attach_storage(m.flat, m.grad_flat, owner=object())
+    refused = False
+    try:
+        m.state_dict()
+    except RuntimeError:
+        refused = True
+    assert refused, "a model whose storage a data-parallel step owns must not save its partial moments"
+    mf = dp.gather_shards(m.m_flat, total, world, rank)
+    vf = dp.gather_shards(m.v_flat, total, world, rank)
+    state = m.state_dict(m_flat=mf, v_flat=vf)
+    torch.save(state, os.path.join(out_dir, f"state{rank}.pt"))
+    dist.barrier()
+    if rank == 0:
+        torch.save({"M": M, "V": V}, os.path.join(out_dir, "truth.pt"))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_data_parallel_checkpoint_gathers_every_ranks_moments(tmp_path):
+    """Each rank updates the Adam moments of its own shard only; the checkpoint of a
+    data-parallel model must hold every shard's moments (gathered), on every rank,
+    and restore them into a fresh single-GPU model."""
+    import torch
+    import torch.multiprocessing as mp
+    sys.path.insert(0, ROOT)
+    from gaussian_splatting_differentiable_rasteriser_b200 import model, scenes
+    mp.start_processes(_rank_state, args=(2, free_port(), str(tmp_path)), nprocs=2, join=True,
+                       start_method="spawn")
+    truth = torch.load(tmp_path / "truth.pt")
+    s0, s1 = torch.load(tmp_path / "state0.pt"), torch.load(tmp_path / "state1.pt")
+    for s in (s0, s1):
+        assert torch.equal(s["m_flat"], truth["M"]) and torch.equal(s["v_flat"], truth["V"])
+    fresh = model.GaussianModel(scenes.small(seed=1), device="cpu")
+    fresh.load_state_dict(s0)
+    assert torch.equal(fresh.m_flat, truth["M"]) and torch.equal(fresh.v_flat, truth["V"])
+
+
+def test_an_owned_model_refuses_a_size_change_and_bad_states():
+    import pytest
+    import torch
+    sys.path.insert(0, ROOT)
+    from gaussian_splatting_differentiable_rasteriser_b200 import model, scenes
+    small = model.GaussianModel(scenes.small(), device="cpu")
+    sc = scenes.small()
+    sl = slice(0, 4096)
+    other = model.GaussianModel(scenes.make_scene("small/4096", sc.means[:, sl], sc.log_scales[:, sl],
+                                                  sc.quats[:, sl], sc.opacity_logits[sl], sc.sh_degree,
+                                                  sc.sh[:, :, sl], sc.cameras), device="cpu")
+    owned = model.GaussianModel(scenes.small(), device="cpu")
+    owned.attach_storage(owned.flat, owned.grad_flat, owner=object())
+    with pytest.raises(RuntimeError):
+        owned.load_state_dict(other.state_dict())
+    owned.load_state_dict(small.state_dict())  # same size: allowed
+    bad = small.state_dict()
+    bad["n"] = bad["n_pad"] + 1
+    with pytest.raises(ValueError):
+        small.load_state_dict(bad)
+    bad = small.state_dict()
+    bad["m_flat"] = bad["m_flat"][:-4]
+    with pytest.raises(ValueError):
+        small.load_state_dict(bad)
+    assert torch.equal(owned.flat, small.flat)

@@ -1,6 +1,8 @@
 """The allocation-free loss entry point (for callers that cannot call cudaMalloc
-where they need the loss, such as code being captured into a CUDA graph) must
-give the same loss and image gradient as the context-based entry point.
+where they need the loss: a host whose own allocator owns the GPU's memory, or a
+real-time loop whose memory is fixed after start-up) must give the same loss and
+image gradient as the context-based entry point. It runs the same kernel on the
+same inputs with a fixed-order reduction, so both must agree bit for bit.
 
 Called through the C ABI directly. Collected last (file name) so that a run that
 stops at the first failure has already run every other test; it passes both on
@@ -41,10 +43,8 @@ def test_noalloc_loss_matches_context_loss_twice(shape):
                                         stream)
         assert st == native.GS_OK
         torch.cuda.synchronize()
-        np.testing.assert_allclose(loss.cpu().numpy(), ref_loss.cpu().numpy(), rtol=1e-5)
-        a = d.cpu().numpy().astype(np.float64)
-        b = ref_d.cpu().numpy().astype(np.float64)
-        assert np.linalg.norm(a - b) <= 1e-4 * np.linalg.norm(b)
+        np.testing.assert_array_equal(loss.cpu().numpy(), ref_loss.cpu().numpy())
+        np.testing.assert_array_equal(d.cpu().numpy(), ref_d.cpu().numpy())
 
 
 def test_noalloc_loss_rejects_images_beyond_its_scratch():
