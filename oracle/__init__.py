@@ -95,13 +95,15 @@ class Oracle:
     """One scene seen by one camera: preprocess and tile lists are built on
     construction; render/backward walk the lists per pixel."""
 
-    def __init__(self, scene, cam, active_degree=None, opacity_rect=False, camera_f64=False):
+    def __init__(self, scene, cam, active_degree=None, opacity_rect=False, camera_f64=False, mip_comp=False):
         self.L = lib()
         self.scene = scene
         self.cam = cam
         self.h = self.L.or_create()
         if opacity_rect:
             self.L.or_set_option(self.h, 1, 1)
+        if mip_comp:  # opacity times the Mip-Splatting compensation factor
+            self.L.or_set_option(self.h, 2, 1)
         self.active_degree = scene.sh_degree if active_degree is None else active_degree
         f64 = np.asarray(scene.means).dtype == np.float64
         dt = np.float64 if f64 else np.float32

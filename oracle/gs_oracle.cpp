@@ -333,10 +333,21 @@ void covariance3d(const S ls[3], const S q[4], S Sigma[9]) {
 // E = min(4.5, ln(max(o / alpha_min, 1.0001))) with alpha_min = 1/255 and no
 // compensation factor, and r = sqrt(2 E) sqrt(lambda_max). Beyond r along
 // the long axis o exp(-e) < 1/255, so the tiles it drops hold no contribution.
+//
+// With mip_comp the opacity is multiplied by the compensation factor that
+// section "Flattening a 3D blob into a 2D oval (EWA projection)" attributes
+// to Mip-Splatting (its alpha is min(0.99, opacity * comp * exp(-e)), and the
+// opacity-aware radius uses opacity * comp). The pages print no formula; the
+// factor is the 2D Mip filter of Mip-Splatting (Yu et al., "Mip-Splatting:
+// Alias-free 3D Gaussian Splatting", CVPR 2024), comp = sqrt(det V /
+// det(V + s I)), with V the screen covariance before dilation and s the
+// pages' 0.3 px^2 dilation: the dilated splat then carries the integrated
+// weight of the undilated one, so a splat much smaller than a pixel does not
+// gain weight from the dilation. comp = 0 when det V <= 0.
 template <class S, class Cam>
 bool project(const Cam& cam, const S p[3], const S ls[3], const S q[4], const S& logit,
              const double* sh, int64_t sh_stride, int active_degree, Proj<S>& P, Aux& X,
-             bool opacity_rect = false) {
+             bool opacity_rect = false, bool mip_comp = false) {
   X = Aux();
   const auto* R = cam.R;
   // p_c = R p + t, each row summed left to right.
@@ -378,6 +389,11 @@ bool project(const Cam& cam, const S p[3], const S ls[3], const S q[4], const S&
   P.A = P.c / det;
   P.B = -P.b / det;
   P.C = P.a / det;
+  S comp(1.0);
+  if (mip_comp) {
+    S det0 = V[0] * V[3] - V[1] * V[1];
+    comp = val(det0) > 0.0 ? sqrt(det0 / det) : S(0.0);
+  }
 
   P.u = cam.fx * X_ / Z_ + cam.cx;
   P.v = cam.fy * Y_ / Z_ + cam.cy;
@@ -388,7 +404,7 @@ bool project(const Cam& cam, const S p[3], const S ls[3], const S q[4], const S&
   X.lmax = mid + std::sqrt(std::max(mid * mid - dt, 0.0));
   X.radius = kRadiusSigmas * std::sqrt(X.lmax);
   if (opacity_rect) {
-    const double o = 1.0 / (1.0 + std::exp(-val(logit)));
+    const double o = 1.0 / (1.0 + std::exp(-val(logit))) * val(comp);
     const double e_cut = std::min(4.5, std::log(std::max(o * 255.0, 1.0001)));
     X.radius = std::sqrt(2.0 * e_cut) * std::sqrt(X.lmax);
   }
@@ -409,7 +425,7 @@ bool project(const Cam& cam, const S p[3], const S ls[3], const S q[4], const S&
   if (tx0 > tx1 || ty0 > ty1) return false;
   X.touched = (tx1 - tx0 + 1) * (ty1 - ty0 + 1);
 
-  P.o = 1.0 / (1.0 + exp(-logit));
+  P.o = 1.0 / (1.0 + exp(-logit)) * comp;
 
   // View-dependent colour at the direction from the camera to the Gaussian.
   S d[3] = {p[0] - cam.campos[0], p[1] - cam.campos[1], p[2] - cam.campos[2]};
@@ -475,6 +491,7 @@ struct Ctx {
   std::vector<Entry> entries;            // sorted
   std::vector<int64_t> range_lo, range_hi;  // per tile, [lo, hi)
   bool opacity_rect = false;             // opacity-aware tile rect (see project)
+  bool mip_comp = false;                 // Mip-Splatting compensation factor (see project)
 };
 
 // Margins used to flag float32/float64 threshold ambiguity.
@@ -559,7 +576,7 @@ void run_preprocess_and_sort(Ctx& c) {
     Proj<double> P;
     Aux& X = c.aux[i];
     bool ok = project<double>(c.cam, p, ls, q, c.logits[i], &c.sh[i], np, c.active_degree, P, X,
-                              c.opacity_rect);
+                              c.opacity_rect, c.mip_comp);
     if (!ok) {
       X.touched = 0;
       continue;
@@ -613,12 +630,17 @@ extern "C" {
 void* or_create() { return new Ctx(); }
 void or_destroy(void* h) { delete static_cast<Ctx*>(h); }
 
-// Options, set before or_set_scene: 1 = opacity-aware tile rect (value 0/1).
+// Options, set before or_set_scene: 1 = opacity-aware tile rect, 2 = the
+// Mip-Splatting compensation factor in the opacity (values 0/1).
 // Returns 0, or 1 for an unknown option.
 int or_set_option(void* h, int32_t option, int32_t value) {
   Ctx& c = *static_cast<Ctx*>(h);
   if (option == 1) {
     c.opacity_rect = value != 0;
+    return 0;
+  }
+  if (option == 2) {
+    c.mip_comp = value != 0;
     return 0;
   }
   return 1;
@@ -812,7 +834,8 @@ void or_project_backward(void* h, const double* screen_grad, int64_t i0, int64_t
     D logit = seed<11>(c.logits[i], 10);
     Proj<D> P;
     Aux X;
-    project<D>(c.cam, p, ls, q, logit, &c.sh[i], np, c.active_degree, P, X, c.opacity_rect);
+    project<D>(c.cam, p, ls, q, logit, &c.sh[i], np, c.active_degree, P, X, c.opacity_rect,
+               c.mip_comp);
     const D* outs[kScreen] = {&P.u, &P.v, &P.A, &P.B, &P.C, &P.o, &P.rgb[0], &P.rgb[1], &P.rgb[2]};
     double gp[11] = {0};
     for (int o = 0; o < kScreen; ++o)
@@ -888,7 +911,9 @@ void or_camera_backward(void* h, const double* screen_grad, double* out) {
     const D logit(c.logits[i]);
     Proj<D> P;
     Aux X;
-    if (!project<D>(pc, p, ls, q, logit, &c.sh[i], np, c.active_degree, P, X, c.opacity_rect)) continue;
+    if (!project<D>(pc, p, ls, q, logit, &c.sh[i], np, c.active_degree, P, X, c.opacity_rect,
+                    c.mip_comp))
+      continue;
     const D* outs[kScreen] = {&P.u, &P.v, &P.A, &P.B, &P.C, &P.o, &P.rgb[0], &P.rgb[1], &P.rgb[2]};
     for (int o = 0; o < kScreen; ++o)
       for (int j = 0; j < 6; ++j) g[j] += gs[o] * outs[o]->d[j];
