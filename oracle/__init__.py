@@ -166,6 +166,21 @@ class Oracle:
                                 _p(out["n_contrib"]), _p(out["ambiguous"]))
         return out
 
+    def replay_pixels(self, px, py, flip) -> dict:
+        """The forward at pixels (px, py) with, per pixel, the near-threshold
+        decisions selected by bit mask `flip` taken the other way (bit k = the
+        k-th decision within the ambiguity margin, in walk order); n_amb = the
+        number of such decisions the walk met. flip = 0 is the plain walk."""
+        px = np.ascontiguousarray(px, np.int32)
+        py = np.ascontiguousarray(py, np.int32)
+        flip = np.ascontiguousarray(np.broadcast_to(np.asarray(flip, np.uint32), px.shape))
+        n = px.size
+        out = dict(rgb=np.zeros((n, 3)), T=np.zeros(n), n_contrib=np.zeros(n, np.int32),
+                   n_amb=np.zeros(n, np.int32))
+        self.L.or_render_pixels_replay(self.h, n, _p(px), _p(py), _p(flip), _p(out["rgb"]), _p(out["T"]),
+                                       _p(out["n_contrib"]), _p(out["n_amb"]))
+        return out
+
     def render_rows(self, y0, y1, out=None) -> dict:
         """Forward over the pixel rows [y0, y1) into full-size outputs (`out`, as
         returned by an earlier call, is reused when given)."""

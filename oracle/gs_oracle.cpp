@@ -498,7 +498,14 @@ struct Ctx {
 constexpr double kAlphaMargin = 1e-6;
 constexpr double kTMargin = 1e-3;  // relative
 
-void walk_pixel(const Ctx& c, int px, int py, PixelResult& out, std::vector<Contribution>* list) {
+// With flip != 0 the walk is replayed with some of its near-threshold
+// decisions taken the other way: the k-th such decision met (an alpha within
+// kAlphaMargin of 1/255, or a transmittance within kTMargin of 1e-4, counted
+// in walk order) is flipped when bit k of `flip` is set. A float32 renderer
+// may take any of those decisions either way; the replays are the results it
+// can then give. *n_amb receives the number of such decisions met.
+void walk_pixel(const Ctx& c, int px, int py, PixelResult& out, std::vector<Contribution>* list,
+                uint32_t flip = 0, int* n_amb = nullptr) {
   const or_camera& cam = c.cam;
   int tile = (py / kTile) * tiles_x(cam) + (px / kTile);
   double T = 1.0;
@@ -507,6 +514,7 @@ void walk_pixel(const Ctx& c, int px, int py, PixelResult& out, std::vector<Cont
   out.ambiguous = false;
   out.evaluated = 0;
   out.contributions = 0;
+  int amb = 0;
   if (list) list->clear();
   for (int64_t i = c.range_lo[tile]; i < c.range_hi[tile]; ++i) {
     int32_t g = c.entries[i].id;
@@ -517,8 +525,13 @@ void walk_pixel(const Ctx& c, int px, int py, PixelResult& out, std::vector<Cont
     double e = 0.5 * (s[2] * dx * dx + s[4] * dy * dy) + s[3] * dx * dy;
     double a = s[5] * std::exp(-e);
     double alpha = a > kAlphaMax ? kAlphaMax : a;
-    if (std::fabs(alpha - kAlphaMin) < kAlphaMargin) out.ambiguous = true;
-    if (alpha < kAlphaMin) continue;
+    bool skip = alpha < kAlphaMin;
+    if (std::fabs(alpha - kAlphaMin) < kAlphaMargin) {
+      out.ambiguous = true;
+      if (amb < 32 && ((flip >> amb) & 1u)) skip = !skip;
+      ++amb;
+    }
+    if (skip) continue;
     ++out.contributions;
     if (list) {
       // The same alpha as a function of (u, v, A, B, C, o), for the backward.
@@ -535,12 +548,18 @@ void walk_pixel(const Ctx& c, int px, int py, PixelResult& out, std::vector<Cont
     for (int ch = 0; ch < 3; ++ch) rgb[ch] += T * alpha * s[6 + ch];
     double Tn = T * (1.0 - alpha);
     out.n_contrib = static_cast<int32_t>(i - c.range_lo[tile]) + 1;
-    if (std::fabs(Tn - kTMin) < kTMargin * kTMin) out.ambiguous = true;
+    bool stop = Tn < kTMin;
+    if (std::fabs(Tn - kTMin) < kTMargin * kTMin) {
+      out.ambiguous = true;
+      if (amb < 32 && ((flip >> amb) & 1u)) stop = !stop;
+      ++amb;
+    }
     T = Tn;
-    if (T < kTMin) break;
+    if (stop) break;
   }
   for (int ch = 0; ch < 3; ++ch) out.rgb[ch] = rgb[ch] + T * cam.bg[ch];
   out.T = T;
+  if (n_amb) *n_amb = amb;
 }
 
 template <class In>
@@ -771,6 +790,25 @@ void or_render_pixels(void* h, int64_t npix, const int32_t* px, const int32_t* p
     if (T) T[i] = r.T;
     if (n_contrib) n_contrib[i] = r.n_contrib;
     if (ambiguous) ambiguous[i] = r.ambiguous ? 1 : 0;
+  }
+}
+
+// Replays of the forward at a list of pixels (test support for threshold
+// decisions a float32 renderer may take either way): pixel i is walked with
+// the near-threshold decisions in bit mask flip[i] flipped (see walk_pixel);
+// n_amb[i] = the number of near-threshold decisions that walk met.
+void or_render_pixels_replay(void* h, int64_t npix, const int32_t* px, const int32_t* py,
+                             const uint32_t* flip, double* rgb, double* T, int32_t* n_contrib,
+                             int32_t* n_amb) {
+  const Ctx& c = *static_cast<Ctx*>(h);
+  for (int64_t i = 0; i < npix; ++i) {
+    PixelResult r;
+    int amb = 0;
+    walk_pixel(c, px[i], py[i], r, nullptr, flip[i], &amb);
+    for (int ch = 0; ch < 3; ++ch) rgb[3 * i + ch] = r.rgb[ch];
+    T[i] = r.T;
+    n_contrib[i] = r.n_contrib;
+    n_amb[i] = amb;
   }
 }
 

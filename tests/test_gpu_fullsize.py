@@ -8,7 +8,9 @@ The oracle's preprocess and tile sort run on the whole scene, so those are
 compared in full (the sort bit-exact over every entry). The blend is compared
 on sampled pixels (random ones, plus every pixel of a corner tile, an interior
 tile and a tile of the ragged last tile row: 1080 = 67.5 tiles), which the
-oracle walks one by one. The loss is compared in full. The backward and the
+oracle walks one by one; a pixel whose walk meets a decision within float32
+reach of its threshold must equal one of the oracle's replays of the walk
+with such decisions taken either way. The loss is compared in full. The backward and the
 fused backward + Adam are compared for a loss gradient restricted to a band
 of 16 pixel rows: the oracle runs the blend backward of those rows and the
 projection backward of every Gaussian, and the property that rows outside the
@@ -28,6 +30,7 @@ LOSS_RTOL = 1e-5
 GRAD_RL2 = 1e-3
 BAND = 16
 MIN_UNAMBIGUOUS = {"mid": 0.99, "dense": 0.99, "heavy_tail": 0.95}
+REPLAY_BITS = 6  # ambiguous decisions per pixel whose 2^k replays are all tried
 
 
 def dev(a, dtype=torch.float32):
@@ -124,6 +127,21 @@ def test_full_forward_sampled_pixels(full):
     # T enters the pixel as T * background: compared at the pixel tolerance
     np.testing.assert_allclose(T[py, px][ok], r["T"][ok], rtol=0, atol=PIX_TOL)
     np.testing.assert_array_equal(nc[py, px][ok], r["n_contrib"][ok])
+    # Every ambiguous pixel must equal one of the oracle's replays of its walk with
+    # some of its near-threshold decisions taken the other way (a float32 renderer
+    # may take each of them either way): all pixels with up to REPLAY_BITS such
+    # decisions are checked; pixels with more must stay rare.
+    amb = np.nonzero(~ok)[0]
+    matched = np.zeros(amb.size, bool)
+    n_amb = o.replay_pixels(px[amb], py[amb], 0)["n_amb"]
+    bits = int(min(REPLAY_BITS, n_amb.max(initial=0)))
+    for mask in range(1 << bits):
+        rep = o.replay_pixels(px[amb], py[amb], mask)
+        matched |= ((np.abs(got[~ok] - rep["rgb"]).max(axis=1) <= PIX_TOL) &
+                    (np.abs(T[py, px][~ok] - rep["T"]) <= PIX_TOL) & (nc[py, px][~ok] == rep["n_contrib"]))
+    enumerable = n_amb <= REPLAY_BITS
+    assert matched[enumerable].all(), (np.nonzero(~matched[enumerable])[0][:10], n_amb[~matched][:10])
+    assert (~enumerable).sum() <= 0.005 * px.size, (~enumerable).sum()
     # properties that hold at every pixel
     assert np.all((T >= 0) & (T <= 1))
     assert np.all(nc >= 0)
@@ -231,3 +249,46 @@ def test_full_fused_backward_adam_on_a_row_band(full):
     m.load(s)
     m.m_flat.zero_()
     m.v_flat.zero_()
+
+
+def test_full_image_backward_at_mid(full):
+    """The blend and projection backward of the whole image's loss gradient (not a
+    band) at Mid, where the float64 oracle can walk every pixel: its row bands run
+    on the host's cores at once (its calls only read the shared scene state), each
+    band into a screen-gradient buffer of its own, summed in band order. Exercises
+    every tile and the atomics contention of a full-image gradient."""
+    if full["scene"].name != "mid":
+        pytest.skip("the oracle's full-image backward is timed for the Mid workload")
+    import concurrent.futures
+    import os
+    step, m, s, o = full["step"], full["m"], full["scene"], full["o"]
+    cam = full["cam"]
+    H = cam.height
+    _, (_, _, _, d), _, _ = band_gradient(full)
+    d64 = d.astype(np.float32).astype(np.float64)
+    nb = max(1, min(len(os.sched_getaffinity(0)), 32))
+    edges = np.linspace(0, H, nb + 1).astype(int)
+    bufs = [np.zeros((s.n, 9)) for _ in range(nb)]
+    with concurrent.futures.ThreadPoolExecutor(nb) as ex:
+        list(ex.map(lambda k: o.blend_backward_rows(edges[k], edges[k + 1], d64, bufs[k]), range(nb)))
+    sg_ref = np.sum(bufs, axis=0)
+    ref = dict(means=np.zeros((3, s.n_pad)), log_scales=np.zeros((3, s.n_pad)), quats=np.zeros((4, s.n_pad)),
+               opacity_logits=np.zeros(s.n_pad), sh=np.zeros((3, s.sh_k, s.n_pad)))
+    cuts = np.linspace(0, s.n, nb + 1).astype(int)
+    with concurrent.futures.ThreadPoolExecutor(nb) as ex:
+        list(ex.map(lambda k: o.project_backward(sg_ref, cuts[k], cuts[k + 1], ref), range(nb)))
+    m.grad_flat.zero_()
+    step.ctx.render_backward(m.params_struct(), full["cs"], full["T"], full["nc"], dev(d.astype(np.float32)),
+                             m.grads_struct())
+    sg = torch.empty((s.n, 9), device="cuda")
+    step.ctx.debug_screen_grads(sg)
+    torch.cuda.synchronize()
+    sg = host(sg)
+    touched = o.preprocess()["touched"] > 0
+    assert np.any(sg_ref[touched] != 0, axis=1).mean() > 0.5
+    assert not sg[~touched].any()
+    assert rel_l2(sg, sg_ref) < GRAD_RL2
+    for k in scenes.GROUP_NAMES:
+        e = rel_l2(host(m.grads[k])[..., :s.n], ref[k][..., :s.n])
+        assert e < GRAD_RL2, (k, e)
+    m.grad_flat.zero_()

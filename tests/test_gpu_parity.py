@@ -40,17 +40,20 @@ def host(t):
 class DeviceRun:
     """Preprocess + forward of one scene/camera through the C ABI."""
 
-    def __init__(self, native, model, scene, cam, max_entries=None, active_degree=None, opacity_rect=False):
+    def __init__(self, native, model, scene, cam, max_entries=None, active_degree=None, opacity_rect=False,
+                 mip_comp=False):
         self.native = native
         self.m = model.GaussianModel(scene, active_degree=active_degree)
         self.cam = cam
         self.cs = native.camera_struct(cam)
-        o = oracle.Oracle(scene, cam, active_degree, opacity_rect=opacity_rect)
+        o = oracle.Oracle(scene, cam, active_degree, opacity_rect=opacity_rect, mip_comp=mip_comp)
         self.oracle = o
         K_or = oracle.lib().or_num_entries(o.h)
         self.ctx = native.Context(scene.n_pad, max_entries or max(16, 2 * K_or + 16), cam.width, cam.height)
         if opacity_rect:
             self.ctx.set_option(native.GS_OPTION_OPACITY_RECT, 1)
+        if mip_comp:
+            self.ctx.set_option(native.GS_OPTION_MIP_COMPENSATION, 1)
         H, W = cam.height, cam.width
         self.image = torch.empty((3, H, W), device="cuda")
         self.T = torch.empty((H, W), device="cuda")
@@ -143,6 +146,18 @@ def check_pixels(run, o_render):
     # T enters the pixel as T * background: compared at the pixel tolerance
     np.testing.assert_allclose(T[ok], o_render["final_T"][ok], rtol=0, atol=PIX_TOL)
     np.testing.assert_array_equal(nc[ok], o_render["n_contrib"][ok])
+    # an ambiguous pixel (a decision within float32 reach of its threshold) must
+    # equal the oracle's walk with some of those decisions taken the other way
+    py, px = np.nonzero(amb)
+    if px.size:
+        n_amb = run.oracle.replay_pixels(px, py, 0)["n_amb"]
+        assert n_amb.max() <= 8, n_amb.max()
+        matched = np.zeros(px.size, bool)
+        for mask in range(1 << int(n_amb.max())):
+            rep = run.oracle.replay_pixels(px, py, mask)
+            matched |= ((np.abs(img[:, py, px].T - rep["rgb"]).max(axis=1) <= PIX_TOL) &
+                        (np.abs(T[py, px] - rep["T"]) <= PIX_TOL) & (nc[py, px] == rep["n_contrib"]))
+        assert matched.all(), np.nonzero(~matched)[0][:10]
     return amb.sum()
 
 
@@ -481,6 +496,69 @@ def test_opacity_aware_rect_path_matches_oracle(gs, name):
     for k in scenes.GROUP_NAMES:
         e = rel_l2(grads[k][..., :s.n], ref[k][..., :s.n])
         assert e < GRAD_RL2, (k, e)
+
+
+@pytest.mark.parametrize("name,rect", [("tiny", False), ("small", False), ("small", True)])
+def test_mip_compensation_path_matches_oracle(gs, name, rect):
+    """With the Mip-Splatting compensation factor: the screen opacities, the
+    pixels and every gradient against the oracle run with the factor; with the
+    opacity-aware rect (which uses opacity * comp) also the rects and the sort,
+    bit for bit. The factor changes the image by far more than the tolerance."""
+    native, model = gs
+    s, ci = SCENES[name]()
+    cam = s.cameras[ci]
+    run = DeviceRun(native, model, s, cam, opacity_rect=rect, mip_comp=True)
+    g = run.preprocess_out()
+    o = run.oracle.preprocess()
+    np.testing.assert_array_equal(g["touched"], o["touched"])
+    vis = o["touched"] > 0
+    np.testing.assert_array_equal(g["rect"][vis], o["rect"][vis])
+    np.testing.assert_allclose(g["opacity"][vis], o["screen"][vis, 5], rtol=3e-6, atol=1e-7)
+    ids, tiles, ranges = run.sorted_out()
+    srt = run.oracle.sorted()
+    np.testing.assert_array_equal(ids, srt["ids"])
+    np.testing.assert_array_equal(ranges.astype(np.int64), srt["ranges"])
+    r = run.oracle.render()
+    check_pixels(run, r)
+    plain = oracle.Oracle(s, cam, opacity_rect=rect).render()
+    assert np.abs(plain["image"] - r["image"]).max() > 1e-2
+    target = scenes.uniform_image(cam.height, cam.width, seed=7)
+    _, _, _, dimg = oracle.loss(r["image"].astype(np.float32), target, 0.2)
+    dimg32 = dimg.astype(np.float32)
+    ref = run.oracle.backward(dimg32.astype(np.float64))
+    grads, sg = run.backward(dimg32)
+    assert rel_l2(sg[vis], ref["screen"][vis]) < GRAD_RL2
+    for k in scenes.GROUP_NAMES:
+        e = rel_l2(grads[k][..., :s.n], ref[k][..., :s.n])
+        assert e < GRAD_RL2, (k, e)
+
+
+def test_mip_compensation_in_the_fused_training_step(gs):
+    """One fused backward + Adam step with the factor against the oracle's
+    backward and Adam on the same image gradient."""
+    native, model = gs
+    s = scenes.small()
+    cam = s.cameras[0]
+    run = DeviceRun(native, model, s, cam, mip_comp=True)
+    r = run.oracle.render()
+    target = scenes.uniform_image(cam.height, cam.width, seed=8)
+    _, _, _, dimg = oracle.loss(r["image"].astype(np.float32), target, 0.2)
+    dimg32 = dimg.astype(np.float32)
+    ref = run.oracle.backward(dimg32.astype(np.float64))
+    m = run.m
+    p0 = {k: host(m.params[k]).astype(np.float64) for k in scenes.GROUP_NAMES}
+    em, ev = m.moments_structs()
+    lr = 1e-3
+    run.ctx.render_backward_adam(m.params_struct(), run.cs, run.T, run.nc, torch.from_numpy(dimg32).cuda(),
+                                 None, em, ev, [lr] * 5, 1, 0.9, 0.999, 1e-8)
+    torch.cuda.synchronize()
+    for k in scenes.GROUP_NAMES:
+        want = oracle.adam(p0[k], ref[k], np.zeros_like(p0[k]), np.zeros_like(p0[k]), lr, 1)[0]
+        got = host(m.params[k]).astype(np.float64).reshape(-1)
+        # Adam's first step moves each scalar by lr sign(g) wherever |g| >> eps
+        sel = np.abs(ref[k].reshape(-1)) > 1e-5 * np.abs(ref[k]).max()
+        sel &= np.arange(got.size) % m.n_pad < s.n
+        assert np.mean(np.abs(got[sel] - want[sel]) <= 1e-6) > 0.995, k
 
 
 def test_set_option_rejects_unknown_options(gs):

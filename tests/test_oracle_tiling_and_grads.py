@@ -203,3 +203,30 @@ def test_opacity_aware_rect_drops_only_tiles_without_contribution():
     i3, ia = o3.render(), oa.render()
     np.testing.assert_allclose(ia["image"], i3["image"], rtol=0, atol=1e-12)
     np.testing.assert_allclose(ia["final_T"], i3["final_T"], rtol=0, atol=1e-12)
+
+
+def test_replay_without_flips_is_the_plain_walk_and_flips_change_only_ambiguous_pixels():
+    """The replay walk (test support for decisions a float32 renderer may take
+    either way) with no flip is the plain walk bit for bit; flipping changes
+    nothing at a pixel without near-threshold decisions, and at a pixel with
+    one it gives the walk with that decision taken the other way."""
+    s = scenes.small()
+    cam = s.cameras[0]
+    o = oracle.Oracle(s, cam)
+    ys, xs = np.mgrid[0:cam.height, 0:cam.width]
+    px, py = xs.ravel(), ys.ravel()
+    plain = o.render_pixels(px, py)
+    rep = o.replay_pixels(px, py, 0)
+    np.testing.assert_array_equal(rep["rgb"], plain["rgb"])
+    np.testing.assert_array_equal(rep["T"], plain["T"])
+    np.testing.assert_array_equal(rep["n_contrib"], plain["n_contrib"])
+    amb = plain["ambiguous"].astype(bool)
+    np.testing.assert_array_equal(rep["n_amb"] > 0, amb)
+    assert 0 < amb.sum() < 0.02 * amb.size
+    flipped = o.replay_pixels(px, py, 0xffffffff)
+    np.testing.assert_array_equal(flipped["rgb"][~amb], plain["rgb"][~amb])
+    changed = np.any(flipped["rgb"][amb] != plain["rgb"][amb], axis=1)
+    assert changed.mean() > 0.9
+    # a flipped alpha decision moves the pixel by about one contribution at the floor
+    d = np.abs(flipped["rgb"][amb] - plain["rgb"][amb]).max(axis=1)
+    assert np.median(d) < 1e-2
