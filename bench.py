@@ -233,7 +233,7 @@ def max_over_ranks(x, world):
 
 # ------------------------------------------------------------------ workload
 def build_workload(config, device, opacity_rect=False, deterministic=False, loss="l1_dssim",
-                   data_parallel=False, exchange="p2p", camera_grad=False):
+                   data_parallel=False, exchange="p2p", camera_grad=False, mip_comp=False):
     import numpy as np
     import torch
 
@@ -249,10 +249,11 @@ def build_workload(config, device, opacity_rect=False, deterministic=False, loss
     if data_parallel:
         from gaussian_splatting_differentiable_rasteriser_b200.data_parallel import DataParallelTrainStep
         step = DataParallelTrainStep(m, cap, W, H, device=device, opacity_rect=opacity_rect,
-                                     deterministic=deterministic, loss=loss, exchange=exchange)
+                                     deterministic=deterministic, loss=loss, exchange=exchange,
+                                     mip_comp=mip_comp)
     else:
         step = model.TrainStep(m, cap, W, H, device=device, opacity_rect=opacity_rect,
-                               deterministic=deterministic, loss=loss)
+                               deterministic=deterministic, loss=loss, mip_comp=mip_comp)
     if camera_grad:
         # every backward also writes the view's pose gradient (6 float64)
         step.camera_grad = torch.zeros(6, dtype=torch.float64, device=device)
@@ -580,7 +581,7 @@ def main_ours(args):
     device = f"cuda:{local}"
     scene, m, step, targets, kmax = build_workload(args.config, device, args.rect == "opacity",
                                                    args.deterministic, args.loss, args.parallel == "dp",
-                                                   args.exchange, args.camera_grad)
+                                                   args.exchange, args.camera_grad, args.mip)
     cams = scene.cameras
     sched = scenes.camera_schedule(len(cams), args.warmup + args.steps, seed=rank)
     # clocks are sampled from the start of the warm-up to the end of the timed region
@@ -650,6 +651,7 @@ def main_ours(args):
                        "gradient_sums": "fixed-point (deterministic)" if args.deterministic else "float32 atomics",
                        "loss": "L1 + D-SSIM (lambda 0.2)" if args.loss == "l1_dssim" else "Charbonnier + exposure",
                        "camera_grad": bool(args.camera_grad),
+                       "mip_compensation": bool(args.mip),
                        "l2": "inputs larger than L2: 2.1 GB of parameter and moment state (p, m, v) "
                              "streamed every step" if args.config == "dense" else "see workload",
                        "entries_per_step": int(statistics.mean(ks)) if ks else None},
@@ -983,6 +985,8 @@ def main():
                          "(one camera per rank per iteration; value counts camera-iterations)")
     ap.add_argument("--exchange", choices=("p2p", "nccl"), default="p2p",
                     help="--parallel dp: the fused peer-memory exchange + Adam, or NCCL collectives")
+    ap.add_argument("--mip", action="store_true",
+                    help="opacities times the Mip-Splatting compensation factor")
     ap.add_argument("--camera-grad", action="store_true",
                     help="each backward also computes the view's camera-pose gradient")
     ap.add_argument("--op", choices=("step", "densify", "relocate"), default="step",

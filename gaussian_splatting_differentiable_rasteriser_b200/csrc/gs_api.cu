@@ -62,6 +62,7 @@ struct gs_ctx {
   int sorted_buf = 0;
   // options (gs_set_option)
   int opacity_rect = 0;
+  int mip_comp = 0;
   unsigned long long* sgrad_fixed = nullptr;  // [max_g][9], allocated by GS_OPTION_DETERMINISTIC
   int deterministic = 0;
   // density control: caller-owned statistics buffers, and the pass's scratch
@@ -202,8 +203,8 @@ void prof_end(gs_ctx* c, int stage, int64_t work, cudaStream_t st, int kernels =
   P.work[stage] += work;
 }
 
-// Kernels one launch_sort enqueues: histogram + digit offsets + one per pass.
-int sort_kernels(const gs::SortPlan& p) { return (p.n > 1 && p.passes > 0) ? 2 + p.passes : 0; }
+// Kernels one launch_sort enqueues: upsweep, digit scan and downsweep per pass.
+int sort_kernels(const gs::SortPlan& p) { return (p.n > 1 && p.passes > 0) ? 3 * p.passes : 0; }
 
 __global__ void unpack_preprocess_kernel(const gs::Screen* screen, const float* depth,
                                          const uint2* rect, const uint32_t* touched,
@@ -341,6 +342,11 @@ gs_status gs_set_option(gs_ctx* c, int32_t option, int32_t value) {
       c->opacity_rect = value;
       c->have_pre = c->have_fwd = false;  // the tile lists depend on it
       return GS_OK;
+    case GS_OPTION_MIP_COMPENSATION:
+      if (value != 0 && value != 1) return fail(c, GS_ERR_INVALID_ARG, "option value must be 0 or 1");
+      c->mip_comp = value;
+      c->have_pre = c->have_fwd = false;  // the screen opacities depend on it
+      return GS_OK;
     case GS_OPTION_DETERMINISTIC:
       if (value != 0 && value != 1) return fail(c, GS_ERR_INVALID_ARG, "option value must be 0 or 1");
       if (value && !c->sgrad_fixed)
@@ -383,6 +389,7 @@ gs_status gs_preprocess(gs_ctx* c, const gs_params* p, const gs_camera* cam, voi
   a.depth_range = c->depth_range;
   a.err = &c->info_dev->device_error;
   a.opacity_rect = c->opacity_rect;
+  a.mip_comp = c->mip_comp;
   const int64_t nb = (p->n + 255) / 256;
   prof_begin(c, st);
   GS_CUDA(c, gs::launch_preprocess(a, nb, st));
@@ -468,12 +475,11 @@ gs_status gs_render_forward(gs_ctx* c, const gs_camera* cam, float* image, float
     d.max_entries = c->max_k;
     d.keys = c->keys[0];
     d.vals = c->vals[0];
-    d.status = c->dup_status;
-    d.ticket = c->counters + gs::kMaxPasses;
+    d.chunk_offsets = c->dup_status;
     d.err = &c->info_dev->device_error;
     prof_begin(c, st);
     GS_CUDA(c, gs::launch_duplicate(d, st));
-    prof_end(c, GS_STAGE_DUPLICATE, static_cast<int64_t>(K), st, V > 0 ? 1 : 0);
+    prof_end(c, GS_STAGE_DUPLICATE, static_cast<int64_t>(K), st, V > 0 ? 3 : 0);  // count, scan, write
     // 4. stable sort of the entries by tile
     gs::SortPlan plan;
     plan.n = static_cast<int64_t>(K);
@@ -614,6 +620,7 @@ gs_status backward_common(gs_ctx* c, const gs_params* p, const gs_camera* cam, c
   a.g_sh = g ? g->sh : nullptr;
   a.stat_accum = c->stat_accum;
   a.stat_count = c->stat_count;
+  a.mip_comp = c->mip_comp;
   if (c->cam_out) {
     // camera-pose gradient of this view, from the raw sums and the parameters
     // of the render (before any update)

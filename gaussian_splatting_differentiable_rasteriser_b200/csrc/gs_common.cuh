@@ -12,6 +12,7 @@ constexpr float kAlphaMax = 0.99f;      // alpha cap
 constexpr float kAlphaMin = 1.0f / 255.0f;  // contributions below are skipped
 constexpr float kTMin = 1e-4f;          // stop once T falls below this
 constexpr double kDilation = 0.3;       // px^2 added to the screen covariance diagonal
+constexpr float kDilationF = 0.3f;
 constexpr double kRadiusSigmas = 3.0;   // sqrt(2 * 4.5): the falloff cut E_CUT = 4.5
 constexpr float kLog2e = 1.4426950408889634f;
 

@@ -32,6 +32,7 @@ struct PreprocessArgs {
   uint32_t* depth_range;  // [min, max] of visible depth keys (atomics)
   uint32_t* err;          // device error word
   int opacity_rect;       // opacity-aware tile rect (GS_OPTION_OPACITY_RECT)
+  int mip_comp;           // opacity times the compensation factor (GS_OPTION_MIP_COMPENSATION)
 };
 
 cudaError_t launch_preprocess(const PreprocessArgs& a, int64_t num_blocks, cudaStream_t st);
@@ -70,8 +71,9 @@ struct CompactArgs {
 cudaError_t launch_compact(const CompactArgs& a, int64_t num_blocks, cudaStream_t st);
 
 // One (tile, index) entry per tile touched by each visible Gaussian, in the
-// depth order given by `order` (a single pass: each CTA's offset comes from a
-// decoupled look-back over the earlier CTAs' totals of tiles touched).
+// depth order given by `order`: the tiles touched by each chunk of kDupItems
+// Gaussians are counted, scanned, and each chunk's CTA writes its entries from
+// its offset (no wait between CTAs).
 struct DuplicateArgs {
   int64_t count;          // visible Gaussians
   const uint32_t* order;  // Gaussian indices sorted by depth
@@ -79,10 +81,9 @@ struct DuplicateArgs {
   const uint2* rect;
   int tiles_x;
   int64_t max_entries;
-  uint32_t* keys;    // tile
-  uint32_t* vals;    // Gaussian index
-  uint32_t* status;  // [ceil(count / kDupItems)] look-back words, zeroed
-  uint32_t* ticket;  // zeroed
+  uint32_t* keys;           // tile
+  uint32_t* vals;           // Gaussian index
+  uint32_t* chunk_offsets;  // [ceil(count / kDupItems)] scratch: tiles per chunk, then their prefix
   uint32_t* err;
 };
 constexpr int kDupThreads = 256;
@@ -189,6 +190,7 @@ struct PreprocessBwdArgs {
   // density-control statistics (both null when not accumulating)
   float* stat_accum;
   uint32_t* stat_count;
+  int mip_comp;  // the screen opacity includes the compensation factor (GS_OPTION_MIP_COMPENSATION)
 };
 
 cudaError_t launch_preprocess_backward(const PreprocessBwdArgs& a, cudaStream_t st);

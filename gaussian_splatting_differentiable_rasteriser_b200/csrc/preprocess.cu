@@ -33,8 +33,7 @@ constexpr int kGeomPlanes = 11;  // means 3, log-scales 3, quats 4, opacity logi
 template <int kDeg>
 struct PreprocessSmem {
   float plane[kGeomPlanes + 3 * (kDeg + 1) * (kDeg + 1)][kPreThreads];
-  uint64_t bar;
-  int ok;
+  uint64_t bar[2];  // geometry planes, SH planes
 };
 
 template <int kDeg>
@@ -50,38 +49,57 @@ __global__ void __launch_bounds__(kPreThreads, 3) preprocess_kernel(PreprocessAr
   // Stage the CTA's slice of every parameter plane in shared memory with bulk
   // asynchronous copies issued by one thread, so all of a Gaussian's loads
   // (about 240 B at degree 3) are in flight at once instead of behind the
-  // geometry's dependency chain. Planes start 16-byte aligned (n_pad % 4 == 0,
+  // geometry's dependency chain. The 11 geometry planes complete on one
+  // mbarrier and the SH planes on another: the float64 geometry runs while the
+  // SH planes are still arriving. Planes start 16-byte aligned (n_pad % 4 == 0,
   // 16-byte aligned parameter pointers) and a slice is a multiple of 4 floats.
   if (tid == 0) {
-    mbar_init(&sm.bar);
+    mbar_init(&sm.bar[0]);
+    mbar_init(&sm.bar[1]);
     const int cnt = static_cast<int>(np - i0 < kPreThreads ? np - i0 : kPreThreads);
     const uint32_t bytes = static_cast<uint32_t>(cnt) * 4u;
-    mbar_arrive_expect_tx(&sm.bar, bytes * kPlanes);
+    mbar_arrive_expect_tx(&sm.bar[0], bytes * kGeomPlanes);
 #pragma unroll
-    for (int c = 0; c < 3; ++c) bulk_copy_g2s(sm.plane[c], a.means + c * np + i0, bytes, &sm.bar);
+    for (int c = 0; c < 3; ++c) bulk_copy_g2s(sm.plane[c], a.means + c * np + i0, bytes, &sm.bar[0]);
 #pragma unroll
-    for (int c = 0; c < 3; ++c) bulk_copy_g2s(sm.plane[3 + c], a.log_scales + c * np + i0, bytes, &sm.bar);
+    for (int c = 0; c < 3; ++c) bulk_copy_g2s(sm.plane[3 + c], a.log_scales + c * np + i0, bytes, &sm.bar[0]);
 #pragma unroll
-    for (int c = 0; c < 4; ++c) bulk_copy_g2s(sm.plane[6 + c], a.quats + c * np + i0, bytes, &sm.bar);
-    bulk_copy_g2s(sm.plane[10], a.opacity_logits + i0, bytes, &sm.bar);
+    for (int c = 0; c < 4; ++c) bulk_copy_g2s(sm.plane[6 + c], a.quats + c * np + i0, bytes, &sm.bar[0]);
+    bulk_copy_g2s(sm.plane[10], a.opacity_logits + i0, bytes, &sm.bar[0]);
+    mbar_arrive_expect_tx(&sm.bar[1], bytes * (kPlanes - kGeomPlanes));
     for (int ch = 0; ch < 3; ++ch)
       for (int k = 0; k < nk; ++k)
         bulk_copy_g2s(sm.plane[kGeomPlanes + ch * nk + k],
-                      a.sh + (static_cast<int64_t>(ch) * a.sh_k + k) * np + i0, bytes, &sm.bar);
-    bool ok = mbar_wait(&sm.bar, 0, 1 << 16);
-    if (!ok) {
+                      a.sh + (static_cast<int64_t>(ch) * a.sh_k + k) * np + i0, bytes, &sm.bar[1]);
+  }
+  __syncthreads();  // the barriers are initialised before anyone waits on them
+  // Every thread waits for the geometry planes itself (bounded); thread 0
+  // records a timeout and, before the CTA can retire, waits for all copies.
+  bool ok = mbar_wait(&sm.bar[0], 0, 1 << 16);
+  if (!__syncthreads_and(ok)) {
+    if (tid == 0) {
       // Nothing computed from this slice is used (the error fails the
       // launch), but the CTA must not retire before its copies have landed.
       record_error(a.err, kErrCopyTimeout);
-      mbar_drain(&sm.bar, 0, 2000000);
+      mbar_drain(&sm.bar[0], 0, 2000000);
+      mbar_drain(&sm.bar[1], 0, 2000000);
     }
-    sm.ok = ok ? 1 : 0;
+    __syncthreads();
+    if (i < a.n) {  // parameters not staged: treat as culled
+      a.screen[i] = Screen{};
+      a.depth[i] = 0.0f;
+      a.rect[i] = make_uint2(1u, 1u);
+      a.touched[i] = 0u;
+      a.clamped[i] = 0u;
+    }
+    if (tid == 0) a.block_sums[blockIdx.x] = make_uint2(0u, 0u);
+    return;
   }
-  __syncthreads();
   uint32_t touched = 0;
   uint32_t dkey = 0;
   bool visible = false;
-  if (i < a.n && sm.ok) {
+  bool sh_ok = true;  // the SH planes arrived (waited for where colour is needed)
+  if (i < a.n) {
     const CamArgs& cam = a.cam;
     const double p[3] = {sm.plane[0][tid], sm.plane[1][tid], sm.plane[2][tid]};
     // p_c = R p + t, each row summed left to right without fused multiply-add:
@@ -141,6 +159,12 @@ __global__ void __launch_bounds__(kPreThreads, 3) preprocess_kernel(PreprocessAr
       const double cb = dot3(t0, u1);
       const double cc = dot3(t1, u1) + kDilation;
       const double det = ca * cc - cb * cb;
+      // Mip-Splatting compensation: sqrt(det V / det(V + 0.3 I)), V undilated
+      double comp = 1.0;
+      if (a.mip_comp) {
+        const double det0 = (ca - kDilation) * (cc - kDilation) - cb * cb;
+        comp = det0 > 0.0 ? sqrt(det0 / det) : 0.0;
+      }
       if (det > 0.0) {
         const double u = cam.fx * X * iz + cam.cx;
         const double v = cam.fy * Y * iz + cam.cy;
@@ -149,7 +173,7 @@ __global__ void __launch_bounds__(kPreThreads, 3) preprocess_kernel(PreprocessAr
         double rad = kRadiusSigmas * sqrt(lmax);
         if (a.opacity_rect) {
           // opacity-aware cut: beyond sqrt(2 E) sigma along the long axis alpha < 1/255
-          const double od = 1.0 / (1.0 + exp(-static_cast<double>(sm.plane[10][tid])));
+          const double od = 1.0 / (1.0 + exp(-static_cast<double>(sm.plane[10][tid]))) * comp;
           const double e_cut = fmin(4.5, log(fmax(od * 255.0, 1.0001)));
           rad = sqrt(2.0 * e_cut) * sqrt(lmax);
         }
@@ -165,8 +189,11 @@ __global__ void __launch_bounds__(kPreThreads, 3) preprocess_kernel(PreprocessAr
           touched = (x1 - x0 + 1) * (y1 - y0 + 1);
           visible = true;
           dkey = __float_as_uint(depth);
-          const float opacity = 1.0f / (1.0f + expf(-sm.plane[10][tid]));
-          // view-dependent colour at v = normalize(p - campos)
+          float opacity = 1.0f / (1.0f + expf(-sm.plane[10][tid]));
+          if (a.mip_comp) opacity = static_cast<float>(static_cast<double>(opacity) * comp);
+          // view-dependent colour at v = normalize(p - campos); its SH planes
+          // were still arriving while the geometry above ran
+          sh_ok = mbar_wait(&sm.bar[1], 0, 1 << 16);
           double d[3] = {p[0] - cam.campos[0], p[1] - cam.campos[1], p[2] - cam.campos[2]};
           const double dn = sqrt(dot3(d, d));
           const float dx = static_cast<float>(d[0] / dn), dy = static_cast<float>(d[1] / dn),
@@ -205,17 +232,25 @@ __global__ void __launch_bounds__(kPreThreads, 3) preprocess_kernel(PreprocessAr
         }
       }
     }
+    if (!sh_ok) {  // the SH copies did not land in time: treat as culled
+      s = Screen{};
+      rect = make_uint2(1u, 1u);
+      touched = 0u;
+      clamped = 0u;
+      visible = false;
+      record_error(a.err, kErrCopyTimeout);
+    }
     a.screen[i] = s;
     a.depth[i] = depth;
     a.rect[i] = rect;
     a.touched[i] = touched;
     a.clamped[i] = clamped;
-  } else if (i < a.n) {  // parameters not staged (the copy wait gave up): treat as culled
-    a.screen[i] = Screen{};
-    a.depth[i] = 0.0f;
-    a.rect[i] = make_uint2(1u, 1u);
-    a.touched[i] = 0u;
-    a.clamped[i] = 0u;
+  }
+  // Before the CTA can retire, its SH copies must have landed even where no
+  // thread needed them (every Gaussian of the slice culled).
+  if (tid == 0 && !mbar_wait(&sm.bar[1], 0, 1 << 16)) {
+    record_error(a.err, kErrCopyTimeout);
+    mbar_drain(&sm.bar[1], 0, 2000000);
   }
 
   // Block totals of tiles touched and of visible Gaussians (for the entry

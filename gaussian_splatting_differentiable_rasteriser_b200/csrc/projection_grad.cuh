@@ -56,11 +56,13 @@ __device__ __forceinline__ void geometry_grad(const PreprocessBwdArgs& a, int64_
   out.du = d_u;
   out.dv = d_v;
   const float dA = -0.5f * r0.w, dB = -r1.x, dC = -0.5f * r1.y;
-  const float d_o = r0.x / o;
+  const float d_o = o > 0.f ? r0.x / o : 0.f;  // dL/d(screen opacity)
   out.drgb[0] = (clamped & 1) ? 0.f : r1.z;
   out.drgb[1] = (clamped & 2) ? 0.f : r1.w;
   out.drgb[2] = (clamped & 4) ? 0.f : r2.x;
-  out.dlogit = d_o * o * (1.f - o);
+  // screen opacity o = sigmoid(logit) (times comp with the compensation factor)
+  const float sig = a.mip_comp ? 1.0f / (1.0f + expf(-a.opacity_logits[i])) : o;
+  out.dlogit = d_o * o * (1.f - sig);
 
   // Recompute the forward quantities.
   const float p[3] = {a.means[i], a.means[np + i], a.means[2 * np + i]};
@@ -103,9 +105,34 @@ __device__ __forceinline__ void geometry_grad(const PreprocessBwdArgs& a, int64_
   const float hb = 0.5f * dB;
   const float KG00 = A * dA + B * hb, KG01 = A * hb + B * dC;
   const float KG10 = B * dA + C * hb, KG11 = B * hb + C * dC;
-  const float GV00 = -(KG00 * A + KG01 * B);
-  const float GV01 = -(KG00 * B + KG01 * C);
-  const float GV11 = -(KG10 * B + KG11 * C);
+  float GV00 = -(KG00 * A + KG01 * B);
+  float GV01 = -(KG00 * B + KG01 * C);
+  float GV11 = -(KG10 * B + KG11 * C);
+  if (a.mip_comp && o > 0.f) {
+    // comp = sqrt(det V / det V'), V = T Sigma T^T, V' = V + 0.3 I (the pages'
+    // "comp" slot: dL/dcomp = dL/do * sigmoid(logit)); per symmetric entry
+    // d comp / dV00 = comp / 2 (V11 / det V - V'11 / det V'), and likewise.
+    float V[3] = {0.f, 0.f, 0.f};  // V00, V01, V11
+#pragma unroll
+    for (int r = 0; r < 3; ++r) {
+      const float s0 = Sig[3 * r] * T[0] + Sig[3 * r + 1] * T[1] + Sig[3 * r + 2] * T[2];
+      const float s1 = Sig[3 * r] * T[3] + Sig[3 * r + 1] * T[4] + Sig[3 * r + 2] * T[5];
+      V[0] += T[r] * s0;
+      V[1] += T[r] * s1;
+      V[2] += T[3 + r] * s1;
+    }
+    const float det0 = V[0] * V[2] - V[1] * V[1];
+    const float Vd0 = V[0] + kDilationF, Vd2 = V[2] + kDilationF;
+    const float det1 = Vd0 * Vd2 - V[1] * V[1];
+    if (det0 > 0.f && det1 > 0.f) {
+      const float comp = sqrtf(det0 / det1);
+      const float k = 0.5f * comp * d_o * sig;
+      const float i0 = 1.0f / det0, i1 = 1.0f / det1;
+      GV00 += k * (V[2] * i0 - Vd2 * i1);
+      GV11 += k * (V[0] * i0 - Vd0 * i1);
+      GV01 += k * (V[1] * i1 - V[1] * i0);
+    }
+  }
   const float GV[4] = {GV00, GV01, GV01, GV11};
 
   // V' = T Sigma T^T: dSigma = T^T G_V T; dT = 2 G_V T Sigma

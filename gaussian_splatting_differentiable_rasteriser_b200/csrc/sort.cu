@@ -22,11 +22,17 @@
 // (tile, depth) of entries emitted in index order, with about half the bytes
 // moved (16 B per item and pass instead of 24, 5 passes over fewer items).
 //
-// Each onesweep pass reads and writes every item once: a CTA ranks 4096 keys
-// in shared memory (per-warp digit counters, ballot ranking), publishes its
-// digit counts, obtains the exclusive prefix of all earlier CTAs by a
-// decoupled look-back whose every wait is bounded, and scatters through shared
-// memory so the global writes are runs of consecutive addresses.
+// Each radix pass is reduce-then-scan, three launches with no wait between
+// CTAs: an upsweep counts each 4096-key chunk's digits (and adds them to the
+// pass's digit totals), a scan turns the per-chunk counts of each digit into
+// global offsets, and a downsweep ranks its chunk's keys stably in shared
+// memory (per-warp digit counters, ballot ranking) and scatters them through
+// shared memory, so the global writes are runs of consecutive addresses. The
+// upsweep re-reads the keys (4 B of the pass's 20 B per item); at the sizes of
+// a training step they mostly come from L2. A single-pass decoupled look-back
+// avoids that read but serialises the CTAs of a wave: the prefix frontier
+// advances a few CTAs per L2 round trip, which bounded that design at these
+// sizes.
 #include <algorithm>
 
 #include "gs_kernels.cuh"
@@ -34,20 +40,6 @@
 namespace gs {
 
 namespace {
-
-constexpr uint32_t kFlagAggregate = 1u << 30;
-constexpr uint32_t kFlagPrefix = 2u << 30;
-constexpr uint32_t kValueMask = (1u << 30) - 1u;
-constexpr int kLookbackSpinLimit = 1 << 22;
-
-__device__ __forceinline__ uint32_t ld_relaxed(const uint32_t* p) {
-  uint32_t v;
-  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-__device__ __forceinline__ void st_relaxed(uint32_t* p, uint32_t v) {
-  asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
 
 // ---------------------------------------------------------------- compact --
 __global__ void __launch_bounds__(256) compact_kernel(CompactArgs a) {
@@ -72,39 +64,29 @@ __global__ void __launch_bounds__(256) compact_kernel(CompactArgs a) {
 }
 
 // -------------------------------------------------------------- duplicate --
-// Decoupled look-back over earlier CTAs' status words (flag | value) by one
-// warp, 32 predecessors per round; returns the sum of the values before
-// `tile`. Every wait is bounded; on giving up it records an error and returns
-// what it has.
-__device__ __forceinline__ uint32_t warp_lookback(const uint32_t* status, int64_t tile, int lane,
-                                                  uint32_t* err) {
-  uint32_t excl = 0;
-  int64_t t = tile - 1;
-  int spins = 0;
-  while (t >= 0) {
-    const uint32_t w = (t - lane >= 0) ? ld_relaxed(&status[t - lane]) : kFlagPrefix;
-    const uint32_t flag = w & ~kValueMask;
-    const unsigned not_ready = __ballot_sync(0xffffffffu, flag == 0u);
-    const unsigned is_prefix = __ballot_sync(0xffffffffu, flag == kFlagPrefix);
-    // lanes usable this round: up to (and including) the first prefix, before the first not-ready
-    const unsigned upto_prefix = is_prefix ? ((2u << (__ffs(is_prefix) - 1)) - 1u) : 0xffffffffu;
-    const unsigned before_wait = not_ready ? ((1u << (__ffs(not_ready) - 1)) - 1u) : 0xffffffffu;
-    const unsigned use = upto_prefix & before_wait;
-    uint32_t v = ((use >> lane) & 1u) ? (w & kValueMask) : 0u;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    excl += v;
-    if (is_prefix && (upto_prefix & ~before_wait) == 0u) break;  // reached a prefix
-    t -= __popc(use);
-    if (not_ready) {
-      if (++spins > kLookbackSpinLimit) {
-        record_error(err, kErrLookbackTimeout);
-        break;
-      }
-      __nanosleep(32);
-    }
+// Tiles touched by each chunk of kDupItems Gaussians in depth order (the
+// duplicate's CTA granularity): one CTA per chunk, one sum per chunk.
+__global__ void __launch_bounds__(kDupThreads) dup_count_kernel(const uint32_t* order, const uint32_t* touched,
+                                                                int64_t count, uint32_t* chunk_tiles) {
+  __shared__ uint32_t s_warp[kDupThreads / 32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t base = static_cast<int64_t>(blockIdx.x) * kDupItems;
+  uint32_t sum = 0;
+#pragma unroll 4
+  for (int j = 0; j < kDupPerThread; ++j) {
+    const int64_t idx = base + static_cast<int64_t>(j) * kDupThreads + tid;
+    if (idx < count) sum += __ldg(touched + __ldg(order + idx));
   }
-  return excl;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  if (lane == 0) s_warp[warp] = sum;
+  __syncthreads();
+  if (tid == 0) {
+    uint32_t t = 0;
+#pragma unroll
+    for (int k = 0; k < kDupThreads / 32; ++k) t += s_warp[k];
+    chunk_tiles[blockIdx.x] = t;
+  }
 }
 
 // Items are warp-striped: item j of lane l of warp w is the CTA's item
@@ -114,11 +96,8 @@ __global__ void __launch_bounds__(kDupThreads) duplicate_kernel(DuplicateArgs a)
   __shared__ uint32_t s_warp[kDupThreads / 32];
   __shared__ uint32_t s_pre[kDupThreads / 32][kDupPerThread][32];  // items' offsets in the warp's run
   __shared__ uint32_t s_gid[kDupThreads / 32][kDupPerThread][32];  // items' Gaussians
-  __shared__ uint32_t s_tile, s_excl;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  if (tid == 0) s_tile = atomicAdd(a.ticket, 1u);
-  __syncthreads();
-  const int64_t tile = s_tile;
+  const int64_t tile = blockIdx.x;
   const int64_t wbase = tile * kDupItems + static_cast<int64_t>(warp) * (32 * kDupPerThread);
   uint32_t gid[kDupPerThread];
   uint2 rc[kDupPerThread];
@@ -152,24 +131,11 @@ __global__ void __launch_bounds__(kDupThreads) duplicate_kernel(DuplicateArgs a)
   }
   if (lane == 0) s_warp[warp] = run;
   __syncthreads();
-  uint32_t before = 0, total = 0;
+  uint32_t before = 0;
 #pragma unroll
-  for (int k = 0; k < kDupThreads / 32; ++k) {
-    before += k < warp ? s_warp[k] : 0u;
-    total += s_warp[k];
-  }
-  uint32_t* st = a.status + tile;
-  if (warp == 0) {
-    if (lane == 0) st_relaxed(st, (tile == 0 ? kFlagPrefix : kFlagAggregate) | total);
-    uint32_t excl = 0;
-    if (tile > 0) {
-      excl = warp_lookback(a.status, tile, lane, a.err);
-      if (lane == 0) st_relaxed(st, kFlagPrefix | (excl + total));
-    }
-    if (lane == 0) s_excl = excl;
-  }
-  __syncthreads();
-  const uint64_t off0 = static_cast<uint64_t>(s_excl) + before;
+  for (int k = 0; k < kDupThreads / 32; ++k) before += k < warp ? s_warp[k] : 0u;
+  // this chunk's first entry: the exclusive prefix of the chunks' tile counts
+  const uint64_t off0 = static_cast<uint64_t>(__ldg(a.chunk_offsets + tile)) + before;
   if (off0 + run > static_cast<uint64_t>(a.max_entries)) {
     if (lane == 0 && run) record_error(a.err, kErrIndexRange);
     return;
@@ -237,86 +203,132 @@ __global__ void __launch_bounds__(kDupThreads) duplicate_kernel(DuplicateArgs a)
   }
 }
 
-// ------------------------------------------------------------- histogram --
-__global__ void __launch_bounds__(256) histogram_kernel(const uint32_t* keys, int64_t n,
-                                                        int passes, uint32_t* hist) {
-  __shared__ uint32_t s_hist[kMaxPasses][kRadix];
-  for (int k = threadIdx.x; k < kMaxPasses * kRadix; k += blockDim.x) (&s_hist[0][0])[k] = 0;
+// ---------------------------------------------------------------- upsweep --
+// Digit counts of one pass for the chunk of kSortTileKeys keys of this CTA,
+// digit-major (counts[d * chunks + chunk]), and the pass's digit totals
+// (hist[d], added with one atomic per digit and CTA).
+__global__ void __launch_bounds__(kSortThreads) upsweep_kernel(const uint32_t* keys, int64_t n, int shift,
+                                                               int64_t chunks, uint32_t* counts,
+                                                               uint32_t* hist) {
+  __shared__ uint32_t s_h[kSortThreads / 32][kRadix];
+  const int tid = threadIdx.x, warp = tid >> 5;
+  for (int k = tid; k < (kSortThreads / 32) * kRadix; k += kSortThreads) (&s_h[0][0])[k] = 0;
   __syncthreads();
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += stride) {
-    const uint32_t key = keys[i];
-    for (int p = 0; p < passes; ++p) atomicAdd(&s_hist[p][(key >> (8 * p)) & 0xffu], 1u);
-  }
-  __syncthreads();
-  for (int p = 0; p < passes; ++p) {
-    const uint32_t c = s_hist[p][threadIdx.x];
-    if (c) atomicAdd(&hist[p * kRadix + threadIdx.x], c);
-  }
-}
-
-// Exclusive scan of each pass's digit histogram: one CTA of 256 per pass.
-__global__ void __launch_bounds__(256) digit_offsets_kernel(const uint32_t* hist, uint32_t* offsets) {
-  __shared__ uint32_t s_warp[8];
-  const int p = blockIdx.x, d = threadIdx.x, lane = d & 31, warp = d >> 5;
-  const uint32_t c = hist[p * kRadix + d];
-  uint32_t v = c;
+  const int64_t base = static_cast<int64_t>(blockIdx.x) * kSortTileKeys;
+  // 16-byte loads: the chunk starts at a multiple of 4096 keys
 #pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    uint32_t n = __shfl_up_sync(0xffffffffu, v, o);
-    if (lane >= o) v += n;
+  for (int k = 0; k < kSortItems / 4; ++k) {
+    const int64_t idx = base + 4 * (static_cast<int64_t>(k) * kSortThreads + tid);
+    uint32_t v[4];
+    if (idx + 3 < n) {
+      const uint4 q = __ldg(reinterpret_cast<const uint4*>(keys + idx));
+      v[0] = q.x, v[1] = q.y, v[2] = q.z, v[3] = q.w;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) atomicAdd(&s_h[warp][(v[j] >> shift) & 0xffu], 1u);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (idx + j < n) atomicAdd(&s_h[warp][(__ldg(keys + idx + j) >> shift) & 0xffu], 1u);
+    }
   }
-  if (lane == 31) s_warp[warp] = v;
   __syncthreads();
-  uint32_t before = 0;
-  for (int k = 0; k < warp; ++k) before += s_warp[k];
-  offsets[p * kRadix + d] = before + v - c;
+  const int d = tid;  // kSortThreads == kRadix
+  uint32_t c = 0;
+#pragma unroll
+  for (int w = 0; w < kSortThreads / 32; ++w) c += s_h[w][d];
+  counts[static_cast<int64_t>(d) * chunks + blockIdx.x] = c;
+  if (c) atomicAdd(&hist[d], c);
 }
 
-// --------------------------------------------------------------- onesweep --
-struct OnesweepArgs {
+// ------------------------------------------------------------------- scan --
+// CTA d: the global offsets of digit d in every chunk, in place over its
+// counts: the keys of all smaller digits (the totals hist[0..d)) come first,
+// then digit d's keys of the chunks before.
+constexpr int kScanThreads = 1024;
+__global__ void __launch_bounds__(kScanThreads) scan_digits_kernel(uint32_t* counts, int64_t chunks,
+                                                                    const uint32_t* hist) {
+  __shared__ uint32_t s_warp[kScanThreads / 32];
+  __shared__ uint32_t s_carry;
+  const int d = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (warp == 0) {
+    uint32_t b = 0;
+    for (int k = lane; k < d; k += 32) b += hist[k];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) b += __shfl_xor_sync(0xffffffffu, b, o);
+    if (lane == 0) s_carry = b;
+  }
+  __syncthreads();
+  uint32_t* row = counts + static_cast<int64_t>(d) * chunks;
+  for (int64_t start = 0; start < chunks; start += 4 * kScanThreads) {
+    const int64_t i0 = start + 4 * static_cast<int64_t>(tid);
+    uint32_t v[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) v[j] = i0 + j < chunks ? row[i0 + j] : 0u;
+    const uint32_t t = v[0] + v[1] + v[2] + v[3];
+    uint32_t inc = t;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += y;
+    }
+    if (lane == 31) s_warp[warp] = inc;
+    __syncthreads();
+    uint32_t before = s_carry, total = 0;
+#pragma unroll 4
+    for (int w = 0; w < kScanThreads / 32; ++w) {
+      const uint32_t x = s_warp[w];
+      before += w < warp ? x : 0u;
+      total += x;
+    }
+    uint32_t run = before + inc - t;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (i0 + j < chunks) row[i0 + j] = run;
+      run += v[j];
+    }
+    __syncthreads();
+    if (tid == 0) s_carry += total;
+    __syncthreads();
+  }
+}
+
+// -------------------------------------------------------------- downsweep --
+struct DownsweepArgs {
   const uint32_t* keys_in;
   const uint32_t* vals_in;
   uint32_t* keys_out;
   uint32_t* vals_out;
   int64_t n;
   int shift;
-  int digit_bits;                 // significant bits of this pass's digit (1..8)
-  const uint32_t* digit_offsets;  // [256] for this pass
-  uint32_t* status;               // [tiles][256] for this pass, zeroed
-  uint32_t* ticket;               // zeroed
+  int digit_bits;          // significant bits of this pass's digit (1..8)
+  const uint32_t* offsets; // [256][chunks]: global first slot of each digit for each chunk
+  int64_t chunks;
   uint32_t* err;
 };
 
-// Shared memory of one onesweep CTA (dynamic: above the 48 KB static limit).
-struct OnesweepSmem {
+// Shared memory of one downsweep CTA (dynamic: above the 48 KB static limit).
+struct DownsweepSmem {
   uint32_t keys[kSortTileKeys];
   uint32_t vals[kSortTileKeys];
   uint32_t whist[kSortThreads / 32][kRadix];  // per-warp digit counts, then offsets
   uint32_t start[kRadix];  // first slot of each digit inside this CTA
   uint32_t base[kRadix];   // first global slot of each digit for this CTA
   uint32_t wsum[kSortThreads / 32];
-  uint32_t tile;
 };
 
-__global__ void __launch_bounds__(kSortThreads) onesweep_kernel(OnesweepArgs a) {
+__global__ void __launch_bounds__(kSortThreads) downsweep_kernel(DownsweepArgs a) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  OnesweepSmem& sm = *reinterpret_cast<OnesweepSmem*>(smem_raw);
-  uint32_t* s_keys = sm.keys;
-  uint32_t* s_vals = sm.vals;
+  DownsweepSmem& sm = *reinterpret_cast<DownsweepSmem*>(smem_raw);
   auto& s_whist = sm.whist;
-  uint32_t* s_start = sm.start;
-  uint32_t* s_base = sm.base;
-  uint32_t* s_wsum = sm.wsum;
-  uint32_t& s_tile = sm.tile;
-
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  if (tid == 0) s_tile = atomicAdd(a.ticket, 1u);
   for (int k = tid; k < (kSortThreads / 32) * kRadix; k += kSortThreads) (&s_whist[0][0])[k] = 0;
-  __syncthreads();
-  const uint32_t tile = s_tile;
-  const int64_t base = static_cast<int64_t>(tile) * kSortTileKeys;
+  const int64_t chunk = blockIdx.x;
+  const int64_t base = chunk * kSortTileKeys;
   const uint32_t lt_mask = (1u << lane) - 1u;
+  // The chunk's global slot of each digit (read early: its latency overlaps the ranking).
+  const uint32_t d_own = tid;  // kSortThreads == kRadix
+  const uint32_t gbase = d_own < (1u << a.digit_bits) ? __ldg(a.offsets + d_own * a.chunks + chunk) : 0u;
+  __syncthreads();
 
   // Load: warp w owns the 512 consecutive entries [base + 512 w, base + 512 (w + 1)),
   // item j of lane l is entry 32 j + l of that run (coalesced).
@@ -327,8 +339,8 @@ __global__ void __launch_bounds__(kSortThreads) onesweep_kernel(OnesweepArgs a) 
   for (int j = 0; j < kSortItems; ++j) {
     const int64_t idx = base + warp * (kSortItems * 32) + j * 32 + lane;
     if (idx < a.n) {
-      key[j] = a.keys_in[idx];
-      val[j] = a.vals_in[idx];
+      key[j] = __ldg(a.keys_in + idx);
+      val[j] = __ldg(a.vals_in + idx);
     } else {
       key[j] = ~0u;
       val[j] = 0u;
@@ -358,73 +370,26 @@ __global__ void __launch_bounds__(kSortThreads) onesweep_kernel(OnesweepArgs a) 
   __syncthreads();
 
   // Per digit: exclusive offsets of each warp, and the CTA total.
-  const uint32_t d = tid;  // kSortThreads == kRadix
   uint32_t count = 0;
 #pragma unroll
   for (int w = 0; w < kSortThreads / 32; ++w) {
-    const uint32_t c = s_whist[w][d];
-    s_whist[w][d] = count;
+    const uint32_t c = s_whist[w][d_own];
+    s_whist[w][d_own] = count;
     count += c;
   }
-  // Publish this CTA's count before anything else, so later CTAs can proceed.
-  uint32_t* st = a.status + static_cast<int64_t>(tile) * kRadix;
-  st_relaxed(&st[d], (tile == 0 ? kFlagPrefix : kFlagAggregate) | count);
-
   // CTA-wide exclusive scan of the digit counts.
   uint32_t v = count;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    uint32_t n = __shfl_up_sync(0xffffffffu, v, o);
-    if (lane >= o) v += n;
+    uint32_t y = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += y;
   }
-  if (lane == 31) s_wsum[warp] = v;
+  if (lane == 31) sm.wsum[warp] = v;
   __syncthreads();
   uint32_t before = 0;
-  for (int k = 0; k < warp; ++k) before += s_wsum[k];
-  s_start[d] = before + v - count;
-
-  // Decoupled look-back over earlier CTAs for this digit, kWindow predecessors
-  // per round: their status words are loaded together, so a run of
-  // aggregate-only predecessors costs one memory latency per kWindow CTAs.
-  // (When a whole wave of CTAs starts at once, none has its inclusive prefix
-  // yet and CTA k of the wave must sum back k aggregates.) Every wait is bounded.
-  constexpr int kWindow = 8;
-  uint32_t excl = 0;
-  if (tile > 0) {
-    int64_t t = static_cast<int64_t>(tile) - 1;
-    int spins = 0;
-    while (t >= 0) {
-      uint32_t w[kWindow];
-#pragma unroll
-      for (int k = 0; k < kWindow; ++k)
-        w[k] = (t - k >= 0) ? ld_relaxed(&a.status[(t - k) * kRadix + d]) : kFlagPrefix;
-      int used = 0;
-      bool stop = false, blocked = false;
-#pragma unroll
-      for (int k = 0; k < kWindow; ++k) {
-        if (stop || blocked) continue;
-        const uint32_t flag = w[k] & ~kValueMask;
-        if (flag == 0u) {
-          blocked = true;
-          continue;
-        }
-        excl += w[k] & kValueMask;
-        ++used;
-        if (flag == kFlagPrefix) stop = true;
-      }
-      if (stop) break;
-      t -= used;
-      if (blocked) {
-        if (++spins > kLookbackSpinLimit) {
-          record_error(a.err, kErrLookbackTimeout);
-          break;
-        }
-        __nanosleep(32);
-      }
-    }
-    st_relaxed(&st[d], kFlagPrefix | (excl + count));
-  }
-  s_base[d] = a.digit_offsets[d] + excl;
+  for (int k = 0; k < warp; ++k) before += sm.wsum[k];
+  sm.start[d_own] = before + v - count;
+  sm.base[d_own] = gbase;
   __syncthreads();
 
   // Scatter into shared memory in digit order, then out in runs.
@@ -433,28 +398,28 @@ __global__ void __launch_bounds__(kSortThreads) onesweep_kernel(OnesweepArgs a) 
     const int64_t idx = base + warp * (kSortItems * 32) + j * 32 + lane;
     if (idx < a.n) {
       const uint32_t dj = (key[j] >> a.shift) & 0xffu;
-      const uint32_t pos = s_start[dj] + s_whist[warp][dj] + rank[j];
+      const uint32_t pos = sm.start[dj] + s_whist[warp][dj] + rank[j];
       if (pos >= static_cast<uint32_t>(kSortTileKeys)) {
         record_error(a.err, kErrIndexRange);
         continue;
       }
-      s_keys[pos] = key[j];
-      s_vals[pos] = val[j];
+      sm.keys[pos] = key[j];
+      sm.vals[pos] = val[j];
     }
   }
   __syncthreads();
   const int64_t rem = a.n - base;
   const int tile_n = rem < kSortTileKeys ? static_cast<int>(rem) : kSortTileKeys;
   for (int k = tid; k < tile_n; k += kSortThreads) {
-    const uint32_t kk = s_keys[k];
+    const uint32_t kk = sm.keys[k];
     const uint32_t dk = (kk >> a.shift) & 0xffu;
-    const int64_t dst = static_cast<int64_t>(s_base[dk]) + (k - static_cast<int64_t>(s_start[dk]));
+    const int64_t dst = static_cast<int64_t>(sm.base[dk]) + (k - static_cast<int64_t>(sm.start[dk]));
     if (dst < 0 || dst >= a.n) {
       record_error(a.err, kErrIndexRange);
       continue;
     }
     a.keys_out[dst] = kk;
-    a.vals_out[dst] = s_vals[k];
+    a.vals_out[dst] = sm.vals[k];
   }
 }
 
@@ -503,11 +468,12 @@ cudaError_t launch_compact(const CompactArgs& a, int64_t num_blocks, cudaStream_
 
 cudaError_t launch_duplicate(const DuplicateArgs& a, cudaStream_t st) {
   if (a.count == 0) return cudaSuccess;
-  const int64_t tiles = (a.count + kDupItems - 1) / kDupItems;
-  cudaError_t e;
-  if ((e = cudaMemsetAsync(a.status, 0, sizeof(uint32_t) * tiles, st)) != cudaSuccess) return e;
-  if ((e = cudaMemsetAsync(a.ticket, 0, sizeof(uint32_t), st)) != cudaSuccess) return e;
-  duplicate_kernel<<<static_cast<unsigned>(tiles), kDupThreads, 0, st>>>(a);
+  const int64_t chunks = (a.count + kDupItems - 1) / kDupItems;
+  const unsigned grid = static_cast<unsigned>(chunks);
+  // per-chunk tile counts, their exclusive prefix in place (one scan row), then the entries
+  dup_count_kernel<<<grid, kDupThreads, 0, st>>>(a.order, a.touched, a.count, a.chunk_offsets);
+  scan_digits_kernel<<<1, kScanThreads, 0, st>>>(a.chunk_offsets, chunks, nullptr);
+  duplicate_kernel<<<grid, kDupThreads, 0, st>>>(a);
   return cudaGetLastError();
 }
 
@@ -516,32 +482,29 @@ cudaError_t launch_sort(const SortPlan& plan, const SortBuffers& b, int* out_buf
   if (plan.n <= 1 || plan.passes == 0) return cudaSuccess;
   cudaError_t e;
   if ((e = cudaMemsetAsync(b.hist, 0, sizeof(uint32_t) * kMaxPasses * kRadix, st)) != cudaSuccess) return e;
-  if ((e = cudaMemsetAsync(b.counters, 0, sizeof(uint32_t) * kMaxPasses, st)) != cudaSuccess) return e;
-  if ((e = cudaMemsetAsync(b.status, 0, sizeof(uint32_t) * kRadix * plan.tiles * plan.passes, st)) !=
-      cudaSuccess)
+  if ((e = cudaFuncSetAttribute(downsweep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(sizeof(DownsweepSmem)))) != cudaSuccess)
     return e;
-  if ((e = cudaFuncSetAttribute(onesweep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                static_cast<int>(sizeof(OnesweepSmem)))) != cudaSuccess)
-    return e;
-  int hist_blocks = static_cast<int>(std::min<int64_t>((plan.n + 4095) / 4096, 148 * 4));
-  histogram_kernel<<<hist_blocks, 256, 0, st>>>(b.keys[0], plan.n, plan.passes, b.hist);
-  digit_offsets_kernel<<<plan.passes, 256, 0, st>>>(b.hist, b.offsets);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const unsigned chunks = static_cast<unsigned>(plan.tiles);
   int cur = 0;
   for (int p = 0; p < plan.passes; ++p) {
-    OnesweepArgs o;
+    const int digit_bits = std::min(8, plan.key_bits - 8 * p);
+    uint32_t* counts = b.status + static_cast<int64_t>(p) * plan.tiles * kRadix;  // [256][chunks]
+    uint32_t* hist = b.hist + p * kRadix;
+    upsweep_kernel<<<chunks, kSortThreads, 0, st>>>(b.keys[cur], plan.n, 8 * p, plan.tiles, counts, hist);
+    scan_digits_kernel<<<1u << digit_bits, kScanThreads, 0, st>>>(counts, plan.tiles, hist);
+    DownsweepArgs o;
     o.keys_in = b.keys[cur];
     o.vals_in = b.vals[cur];
     o.keys_out = b.keys[cur ^ 1];
     o.vals_out = b.vals[cur ^ 1];
     o.n = plan.n;
     o.shift = 8 * p;
-    o.digit_bits = std::min(8, plan.key_bits - 8 * p);
-    o.digit_offsets = b.offsets + p * kRadix;
-    o.status = b.status + static_cast<int64_t>(p) * plan.tiles * kRadix;
-    o.ticket = b.counters + p;
+    o.digit_bits = digit_bits;
+    o.offsets = counts;
+    o.chunks = plan.tiles;
     o.err = b.err;
-    onesweep_kernel<<<static_cast<unsigned>(plan.tiles), kSortThreads, sizeof(OnesweepSmem), st>>>(o);
+    downsweep_kernel<<<chunks, kSortThreads, sizeof(DownsweepSmem), st>>>(o);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     cur ^= 1;
   }

@@ -178,7 +178,8 @@ class TrainStep:
 
     def __init__(self, model: GaussianModel, max_entries: int, width: int, height: int, lrs=None,
                  lam=0.2, betas=(0.9, 0.999), eps=1e-8, device="cuda", fused_adam=True,
-                 opacity_rect=False, deterministic=False, loss="l1_dssim", sh_ramp_every=None):
+                 opacity_rect=False, deterministic=False, loss="l1_dssim", sh_ramp_every=None,
+                 mip_comp=False):
         self.model = model
         # None: the model's active degree stays as set; otherwise it follows sh_degree_at
         self.sh_ramp_every = sh_ramp_every
@@ -193,6 +194,8 @@ class TrainStep:
             self.ctx.set_option(native.GS_OPTION_OPACITY_RECT, 1)
         if deterministic:
             self.ctx.set_option(native.GS_OPTION_DETERMINISTIC, 1)
+        if mip_comp:  # opacities times the Mip-Splatting compensation factor
+            self.ctx.set_option(native.GS_OPTION_MIP_COMPENSATION, 1)
         self.lrs = dict(DEFAULT_LR if lrs is None else lrs)
         self.lam, self.betas, self.eps = lam, betas, eps
         self.image = torch.empty((3, height, width), dtype=torch.float32, device=device)

@@ -32,6 +32,7 @@ GS_SHARED_HANDLE_BYTES = 64
 MAX_RANKS = 8
 GS_OPTION_OPACITY_RECT = 1
 GS_OPTION_DETERMINISTIC = 2
+GS_OPTION_MIP_COMPENSATION = 3
 STAGES = ("preprocess", "scan", "duplicate", "sort", "ranges", "blend_forward", "loss",
           "blend_backward", "preprocess_backward", "backward_adam", "depth_sort", "camera_backward")
 GROUPS = ("means", "log_scales", "quats", "opacity_logits", "sh")

@@ -109,10 +109,11 @@ typedef enum {
   /* Value 1: each Gaussian's tile rect uses the opacity-aware radius of [GS]
    * section "Why tiling, and the five stages" (the code after the list):
    * r = sqrt(2 E) sqrt(lambda_max) with E = min(4.5, ln(max(255 o, 1.0001))),
-   * alpha_min = 1/255 and no compensation factor, instead of 3 sqrt(lambda_max).
-   * Alpha stays below 1/255 in every tile it drops, so the image and
-   * gradients do not change; the (Gaussian, tile) lists get shorter. Value 0
-   * (the default): the 3-sigma rect. */
+   * alpha_min = 1/255, instead of 3 sqrt(lambda_max); o is the opacity times
+   * the compensation factor when GS_OPTION_MIP_COMPENSATION is set. Alpha
+   * stays below 1/255 in every tile it drops, so the image and gradients do
+   * not change; the (Gaussian, tile) lists get shorter. Value 0 (the
+   * default): the 3-sigma rect. */
   GS_OPTION_OPACITY_RECT = 1,
   /* Value 1: the backward accumulates each Gaussian's screen-space gradient
    * sums as 64-bit integers in 2^-40 fixed point instead of float32 atomics
@@ -124,7 +125,18 @@ typedef enum {
    * bitwise reproducible. Enabling it allocates 72 B per Gaussian of the
    * context (GS_ERR_CUDA if that fails). Value 0 (the default): float32
    * atomics. */
-  GS_OPTION_DETERMINISTIC = 2
+  GS_OPTION_DETERMINISTIC = 2,
+  /* Value 1: each Gaussian's opacity is multiplied by the Mip-Splatting
+   * compensation factor that [GS] section "Flattening a 3D blob into a 2D
+   * oval (EWA projection)" names (alpha = min(0.99, opacity * comp *
+   * exp(-e)) in "The painting itself", and opacity * comp in the
+   * opacity-aware radius), with the factor of Mip-Splatting's 2D filter,
+   * comp = sqrt(det V / det(V + 0.3 I)) for the screen covariance V before
+   * the 0.3 px^2 dilation (0 if det V <= 0): the dilated splat keeps the
+   * integrated weight of the undilated one. The backward carries its
+   * gradient into the covariance (the pages' "comp" slot). Value 0 (the
+   * default): no factor. */
+  GS_OPTION_MIP_COMPENSATION = 3
 } gs_option;
 
 /* Sets a context option; it applies from the next gs_preprocess (the state
