@@ -232,20 +232,32 @@ def max_over_ranks(x, world):
 
 
 # ------------------------------------------------------------------ workload
+def make_scene(config, gaussians=None):
+    """The workload's scene; `gaussians` draws a smaller (or larger) scene of the
+    same shape (Dense and Heavy-tail only), for captures that must stay small."""
+    from gaussian_splatting_differentiable_rasteriser_b200 import scenes
+    if gaussians is None:
+        return scenes.CONFIGS[config]()
+    if config not in ("dense", "heavy_tail"):
+        raise SystemExit("--gaussians applies to the dense and heavy_tail workloads")
+    return scenes.CONFIGS[config](n=int(gaussians))
+
+
 def build_workload(config, device, opacity_rect=False, deterministic=False, loss="l1_dssim",
-                   data_parallel=False, exchange="p2p", camera_grad=False, mip_comp=False):
+                   data_parallel=False, exchange="p2p", camera_grad=False, mip_comp=False,
+                   gaussians=None, capacity=None):
     import numpy as np
     import torch
 
     from gaussian_splatting_differentiable_rasteriser_b200 import model, native, scenes
 
-    scene = scenes.CONFIGS[config]()
+    scene = make_scene(config, gaussians)
     pert = scenes.perturbed(scene, 0.05, seed=1)
     cams = scene.cameras
     W = max(c.width for c in cams)
     H = max(c.height for c in cams)
     m = model.GaussianModel(pert, device=device)
-    cap = max(1 << 20, 8 * scene.n)
+    cap = capacity or max(1 << 20, 8 * scene.n)
     if data_parallel:
         from gaussian_splatting_differentiable_rasteriser_b200.data_parallel import DataParallelTrainStep
         step = DataParallelTrainStep(m, cap, W, H, device=device, opacity_rect=opacity_rect,
@@ -581,7 +593,8 @@ def main_ours(args):
     device = f"cuda:{local}"
     scene, m, step, targets, kmax = build_workload(args.config, device, args.rect == "opacity",
                                                    args.deterministic, args.loss, args.parallel == "dp",
-                                                   args.exchange, args.camera_grad, args.mip)
+                                                   args.exchange, args.camera_grad, args.mip,
+                                                   args.gaussians, args.capacity)
     cams = scene.cameras
     sched = scenes.camera_schedule(len(cams), args.warmup + args.steps, seed=rank)
     # clocks are sampled from the start of the warm-up to the end of the timed region
@@ -639,7 +652,9 @@ def main_ours(args):
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": WORKLOADS[args.config], "gaussians": scene.n,
+            "config": {"workload": WORKLOADS[args.config] + (f"; {scene.n} Gaussians drawn instead"
+                                                             if args.gaussians else ""),
+                       "gaussians": scene.n,
                        "width": W, "height": H, "cameras": len(cams),
                        "parallelism": (("data-parallel: one camera per rank; gradient exchange fused with "
                                         "the sharded Adam over peer memory (gs_adam_step_reduce)"
@@ -777,7 +792,9 @@ def main_reference(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 / value,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
-            "config": {"workload": WORKLOADS[args.config], "gaussians": scene.n, "width": W,
+            "config": {"workload": WORKLOADS[args.config] + (f"; {scene.n} Gaussians drawn instead"
+                                                             if args.gaussians else ""),
+                       "gaussians": scene.n, "width": W,
                        "height": H, "cameras": len(cams), "parallelism": "cpu"},
             "cpu_baseline": cpu,
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -985,6 +1002,10 @@ def main():
                          "(one camera per rank per iteration; value counts camera-iterations)")
     ap.add_argument("--exchange", choices=("p2p", "nccl"), default="p2p",
                     help="--parallel dp: the fused peer-memory exchange + Adam, or NCCL collectives")
+    ap.add_argument("--gaussians", type=int, default=None,
+                    help="draw this many Gaussians instead (dense, heavy_tail): a same-shaped smaller case")
+    ap.add_argument("--capacity", type=int, default=None,
+                    help="(Gaussian, tile) entry capacity of the context (default 8 per Gaussian)")
     ap.add_argument("--mip", action="store_true",
                     help="opacities times the Mip-Splatting compensation factor")
     ap.add_argument("--camera-grad", action="store_true",
