@@ -33,7 +33,7 @@ namespace {
 
 constexpr int kCamThreads = 256;
 
-template <int kDeg>
+template <int kDeg, bool kMip>
 __global__ void __launch_bounds__(kCamThreads, 3) camera_backward_kernel(PreprocessBwdArgs a, CameraGradArgs cg) {
   __shared__ double s_red[9][kCamThreads / 32];
   __shared__ int s_last;
@@ -46,7 +46,7 @@ __global__ void __launch_bounds__(kCamThreads, 3) camera_backward_kernel(Preproc
     if (a.touched[i] == 0) continue;
     GaussGrad g;
     CamTerms ct;
-    geometry_grad<true>(a, i, g, &ct);
+    geometry_grad<true, kMip>(a, i, g, &ct);
     // view-direction part of dL/dp: (dL/dv - v <v, dL/dv>) / |p - campos|
     float wsum[16];
 #pragma unroll
@@ -122,7 +122,10 @@ template <int kDeg>
 cudaError_t launch_cam_deg(const PreprocessBwdArgs& a, const CameraGradArgs& g, cudaStream_t st) {
   const int64_t want = (a.n + kCamThreads - 1) / kCamThreads;
   const unsigned grid = static_cast<unsigned>(want < kCamBlocks ? (want > 0 ? want : 1) : kCamBlocks);
-  camera_backward_kernel<kDeg><<<grid, kCamThreads, 0, st>>>(a, g);
+  if (a.mip_comp)
+    camera_backward_kernel<kDeg, true><<<grid, kCamThreads, 0, st>>>(a, g);
+  else
+    camera_backward_kernel<kDeg, false><<<grid, kCamThreads, 0, st>>>(a, g);
   return cudaGetLastError();
 }
 

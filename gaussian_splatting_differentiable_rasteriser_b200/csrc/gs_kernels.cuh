@@ -50,9 +50,23 @@ struct SortPlan {
   int64_t tiles;  // onesweep tiles of kSortTileKeys items
 };
 
-constexpr int kSortThreads = 256;
-constexpr int kSortItems = 16;
-constexpr int kSortTileKeys = kSortThreads * kSortItems;  // 4096
+// Radix-pass shape: threads per CTA (a multiple of 256), keys per thread and
+// the minimum CTAs per SM the downsweep is compiled for (build-time tunables;
+// 512 x 8 at two CTAs per SM measured fastest on B200: the pass is bound by
+// the latency of its ranking chain, so resident warps matter most).
+#ifndef GS_SORT_THREADS
+#define GS_SORT_THREADS 512
+#endif
+#ifndef GS_SORT_ITEMS
+#define GS_SORT_ITEMS 8
+#endif
+#ifndef GS_SORT_MINB
+#define GS_SORT_MINB 2
+#endif
+constexpr int kSortThreads = GS_SORT_THREADS;
+constexpr int kSortItems = GS_SORT_ITEMS;
+constexpr int kSortTileKeys = kSortThreads * kSortItems;
+static_assert(kSortThreads % 256 == 0 && kSortItems % 4 == 0, "radix-pass shape");
 constexpr int kRadix = 256;
 constexpr int kMaxPasses = 4;
 

@@ -39,7 +39,10 @@ struct CamTerms {
   float ax[3];
 };
 
-template <bool kCam = false>
+// kMip: the screen opacity includes the Mip-Splatting compensation factor
+// (GS_OPTION_MIP_COMPENSATION); a compile-time switch, so the default
+// instantiations carry none of its registers.
+template <bool kCam = false, bool kMip = false>
 __device__ __forceinline__ void geometry_grad(const PreprocessBwdArgs& a, int64_t i, GaussGrad& out,
                                               CamTerms* ct = nullptr) {
   const int64_t np = a.n_pad;
@@ -61,7 +64,7 @@ __device__ __forceinline__ void geometry_grad(const PreprocessBwdArgs& a, int64_
   out.drgb[1] = (clamped & 2) ? 0.f : r1.w;
   out.drgb[2] = (clamped & 4) ? 0.f : r2.x;
   // screen opacity o = sigmoid(logit) (times comp with the compensation factor)
-  const float sig = a.mip_comp ? 1.0f / (1.0f + expf(-a.opacity_logits[i])) : o;
+  const float sig = kMip ? 1.0f / (1.0f + expf(-a.opacity_logits[i])) : o;
   out.dlogit = d_o * o * (1.f - sig);
 
   // Recompute the forward quantities.
@@ -108,7 +111,7 @@ __device__ __forceinline__ void geometry_grad(const PreprocessBwdArgs& a, int64_
   float GV00 = -(KG00 * A + KG01 * B);
   float GV01 = -(KG00 * B + KG01 * C);
   float GV11 = -(KG10 * B + KG11 * C);
-  if (a.mip_comp && o > 0.f) {
+  if (kMip && o > 0.f) {
     // comp = sqrt(det V / det V'), V = T Sigma T^T, V' = V + 0.3 I (the pages'
     // "comp" slot: dL/dcomp = dL/do * sigmoid(logit)); per symmetric entry
     // d comp / dV00 = comp / 2 (V11 / det V - V'11 / det V'), and likewise.

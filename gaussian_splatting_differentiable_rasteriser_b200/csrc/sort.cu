@@ -232,12 +232,13 @@ __global__ void __launch_bounds__(kSortThreads) upsweep_kernel(const uint32_t* k
     }
   }
   __syncthreads();
-  const int d = tid;  // kSortThreads == kRadix
-  uint32_t c = 0;
+  for (int d = tid; d < kRadix; d += kSortThreads) {
+    uint32_t c = 0;
 #pragma unroll
-  for (int w = 0; w < kSortThreads / 32; ++w) c += s_h[w][d];
-  counts[static_cast<int64_t>(d) * chunks + blockIdx.x] = c;
-  if (c) atomicAdd(&hist[d], c);
+    for (int w = 0; w < kSortThreads / 32; ++w) c += s_h[w][d];
+    counts[static_cast<int64_t>(d) * chunks + blockIdx.x] = c;
+    if (c) atomicAdd(&hist[d], c);
+  }
 }
 
 // ------------------------------------------------------------------- scan --
@@ -310,95 +311,97 @@ struct DownsweepArgs {
 struct DownsweepSmem {
   uint32_t keys[kSortTileKeys];
   uint32_t vals[kSortTileKeys];
-  uint32_t whist[kSortThreads / 32][kRadix];  // per-warp digit counts, then offsets
-  uint32_t start[kRadix];  // first slot of each digit inside this CTA
-  uint32_t base[kRadix];   // first global slot of each digit for this CTA
-  uint32_t wsum[kSortThreads / 32];
+  uint32_t whist[kSortThreads / 32][kRadix];  // per-warp digit counts, then CTA slots
+  uint32_t out[kRadix];                       // global slot minus CTA slot of each digit
+  uint32_t wsum[kRadix / 32];
 };
 
-__global__ void __launch_bounds__(kSortThreads) downsweep_kernel(DownsweepArgs a) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  DownsweepSmem& sm = *reinterpret_cast<DownsweepSmem*>(smem_raw);
-  auto& s_whist = sm.whist;
+// kBits: significant bits of this pass's digit; kFull: the chunk holds
+// kSortTileKeys keys (every chunk but the last), so no key needs a bounds test.
+template <int kBits, bool kFull>
+__device__ __forceinline__ void downsweep_chunk(const DownsweepArgs& a, DownsweepSmem& sm, int64_t chunk) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  for (int k = tid; k < (kSortThreads / 32) * kRadix; k += kSortThreads) (&s_whist[0][0])[k] = 0;
-  const int64_t chunk = blockIdx.x;
   const int64_t base = chunk * kSortTileKeys;
+  const int valid_n = kFull ? kSortTileKeys : static_cast<int>(a.n - base);
   const uint32_t lt_mask = (1u << lane) - 1u;
-  // The chunk's global slot of each digit (read early: its latency overlaps the ranking).
-  const uint32_t d_own = tid;  // kSortThreads == kRadix
-  const uint32_t gbase = d_own < (1u << a.digit_bits) ? __ldg(a.offsets + d_own * a.chunks + chunk) : 0u;
-  __syncthreads();
+  auto& whist = sm.whist;
+  for (int k = tid; k < (kSortThreads / 32) * kRadix; k += kSortThreads) (&whist[0][0])[k] = 0;
+  // The chunk's global slot of each digit, read early: its latency overlaps the ranking.
+  const bool owns_digit = tid < kRadix;
+  const uint32_t gbase = owns_digit && tid < (1 << kBits) ? __ldg(a.offsets + tid * a.chunks + chunk) : 0u;
 
-  // Load: warp w owns the 512 consecutive entries [base + 512 w, base + 512 (w + 1)),
-  // item j of lane l is entry 32 j + l of that run (coalesced).
-  uint32_t key[kSortItems];
-  uint32_t val[kSortItems];
+  // Load: warp w owns the kSortItems * 32 consecutive keys from base + w kSortItems 32;
+  // item j of lane l is key 32 j + l of that run (coalesced, and in key order j-major).
+  const int wbase = warp * (kSortItems * 32);
+  uint32_t key[kSortItems], val[kSortItems], dig[kSortItems];
+#pragma unroll
+  for (int j = 0; j < kSortItems; ++j) {
+    const int e = wbase + 32 * j + lane;
+    if (kFull || e < valid_n) {
+      key[j] = __ldg(a.keys_in + base + e);
+      val[j] = __ldg(a.vals_in + base + e);
+    } else {
+      key[j] = 0u;
+      val[j] = 0u;
+    }
+    dig[j] = (key[j] >> a.shift) & ((1u << kBits) - 1u);
+  }
+  __syncthreads();  // counters zeroed
+
+  // Stable rank inside the warp: items in key order, lanes in lane order. The
+  // lanes holding the same digit come from one ballot per digit bit.
   uint32_t rank[kSortItems];
 #pragma unroll
   for (int j = 0; j < kSortItems; ++j) {
-    const int64_t idx = base + warp * (kSortItems * 32) + j * 32 + lane;
-    if (idx < a.n) {
-      key[j] = __ldg(a.keys_in + idx);
-      val[j] = __ldg(a.vals_in + idx);
-    } else {
-      key[j] = ~0u;
-      val[j] = 0u;
-    }
-  }
-  // Stable rank inside the warp: items in entry order, lanes in lane order.
-  // Lanes holding the same digit are found with one ballot per digit bit.
+    const bool valid = kFull || wbase + 32 * j + lane < valid_n;
+    uint32_t peers = kFull ? 0xffffffffu : __ballot_sync(0xffffffffu, valid);
 #pragma unroll
-  for (int j = 0; j < kSortItems; ++j) {
-    const int64_t idx = base + warp * (kSortItems * 32) + j * 32 + lane;
-    const bool valid = idx < a.n;
-    const uint32_t d = (key[j] >> a.shift) & 0xffu;
-    uint32_t peers = __ballot_sync(0xffffffffu, valid);
-#pragma unroll
-    for (int bit = 0; bit < 8; ++bit) {
-      if (bit >= a.digit_bits) break;
-      const bool on = (d >> bit) & 1u;
-      const uint32_t vote = __ballot_sync(0xffffffffu, on);
-      peers &= on ? vote : ~vote;
+    for (int bit = 0; bit < kBits; ++bit) {
+      const uint32_t on = 0u - ((dig[j] >> bit) & 1u);
+      const uint32_t vote = __ballot_sync(0xffffffffu, on != 0u);
+      peers &= ~(vote ^ on);
     }
-    const uint32_t b = valid ? s_whist[warp][d] : 0u;
+    const uint32_t b = valid ? whist[warp][dig[j]] : 0u;
     __syncwarp();
-    if (valid && lane == __ffs(peers) - 1) s_whist[warp][d] = b + __popc(peers);
+    if (valid && lane == __ffs(peers) - 1) whist[warp][dig[j]] = b + __popc(peers);
     __syncwarp();
     rank[j] = b + __popc(peers & lt_mask);
   }
   __syncthreads();
 
-  // Per digit: exclusive offsets of each warp, and the CTA total.
-  uint32_t count = 0;
+  // Per digit (thread d): the CTA-wide exclusive scan of the digit counts, then
+  // each warp's first CTA slot of the digit, and global slot minus CTA slot.
+  uint32_t count = 0, v = 0;
+  if (owns_digit) {
 #pragma unroll
-  for (int w = 0; w < kSortThreads / 32; ++w) {
-    const uint32_t c = s_whist[w][d_own];
-    s_whist[w][d_own] = count;
-    count += c;
-  }
-  // CTA-wide exclusive scan of the digit counts.
-  uint32_t v = count;
+    for (int w = 0; w < kSortThreads / 32; ++w) count += whist[w][tid];
+    v = count;
 #pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    uint32_t y = __shfl_up_sync(0xffffffffu, v, o);
-    if (lane >= o) v += y;
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, v, o);
+      if (lane >= o) v += y;
+    }
+    if (lane == 31) sm.wsum[warp] = v;
   }
-  if (lane == 31) sm.wsum[warp] = v;
   __syncthreads();
-  uint32_t before = 0;
-  for (int k = 0; k < warp; ++k) before += sm.wsum[k];
-  sm.start[d_own] = before + v - count;
-  sm.base[d_own] = gbase;
+  if (owns_digit) {
+    uint32_t start = v - count;
+    for (int k = 0; k < warp; ++k) start += sm.wsum[k];
+    sm.out[tid] = gbase - start;
+#pragma unroll
+    for (int w = 0; w < kSortThreads / 32; ++w) {
+      const uint32_t c = whist[w][tid];
+      whist[w][tid] = start;
+      start += c;
+    }
+  }
   __syncthreads();
 
-  // Scatter into shared memory in digit order, then out in runs.
+  // Scatter into shared memory in digit order, then out in runs of consecutive slots.
 #pragma unroll
   for (int j = 0; j < kSortItems; ++j) {
-    const int64_t idx = base + warp * (kSortItems * 32) + j * 32 + lane;
-    if (idx < a.n) {
-      const uint32_t dj = (key[j] >> a.shift) & 0xffu;
-      const uint32_t pos = sm.start[dj] + s_whist[warp][dj] + rank[j];
+    if (kFull || wbase + 32 * j + lane < valid_n) {
+      const uint32_t pos = whist[warp][dig[j]] + rank[j];
       if (pos >= static_cast<uint32_t>(kSortTileKeys)) {
         record_error(a.err, kErrIndexRange);
         continue;
@@ -408,18 +411,48 @@ __global__ void __launch_bounds__(kSortThreads) downsweep_kernel(DownsweepArgs a
     }
   }
   __syncthreads();
-  const int64_t rem = a.n - base;
-  const int tile_n = rem < kSortTileKeys ? static_cast<int>(rem) : kSortTileKeys;
-  for (int k = tid; k < tile_n; k += kSortThreads) {
+  for (int k = tid; k < valid_n; k += kSortThreads) {
     const uint32_t kk = sm.keys[k];
-    const uint32_t dk = (kk >> a.shift) & 0xffu;
-    const int64_t dst = static_cast<int64_t>(sm.base[dk]) + (k - static_cast<int64_t>(sm.start[dk]));
-    if (dst < 0 || dst >= a.n) {
+    const uint32_t dst = sm.out[(kk >> a.shift) & ((1u << kBits) - 1u)] + static_cast<uint32_t>(k);
+    if (static_cast<int64_t>(dst) >= a.n) {
       record_error(a.err, kErrIndexRange);
       continue;
     }
     a.keys_out[dst] = kk;
     a.vals_out[dst] = sm.vals[k];
+  }
+}
+
+template <int kBits>
+__global__ void __launch_bounds__(kSortThreads, GS_SORT_MINB) downsweep_kernel(DownsweepArgs a) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  DownsweepSmem& sm = *reinterpret_cast<DownsweepSmem*>(smem_raw);
+  const int64_t chunk = blockIdx.x;
+  if ((chunk + 1) * kSortTileKeys <= a.n)
+    downsweep_chunk<kBits, true>(a, sm, chunk);
+  else
+    downsweep_chunk<kBits, false>(a, sm, chunk);
+}
+
+template <int kBits>
+cudaError_t launch_downsweep(const DownsweepArgs& o, unsigned chunks, cudaStream_t st) {
+  cudaError_t e = cudaFuncSetAttribute(downsweep_kernel<kBits>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(sizeof(DownsweepSmem)));
+  if (e != cudaSuccess) return e;
+  downsweep_kernel<kBits><<<chunks, kSortThreads, sizeof(DownsweepSmem), st>>>(o);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_downsweep_bits(const DownsweepArgs& o, int bits, unsigned chunks, cudaStream_t st) {
+  switch (bits) {
+    case 1: return launch_downsweep<1>(o, chunks, st);
+    case 2: return launch_downsweep<2>(o, chunks, st);
+    case 3: return launch_downsweep<3>(o, chunks, st);
+    case 4: return launch_downsweep<4>(o, chunks, st);
+    case 5: return launch_downsweep<5>(o, chunks, st);
+    case 6: return launch_downsweep<6>(o, chunks, st);
+    case 7: return launch_downsweep<7>(o, chunks, st);
+    default: return launch_downsweep<8>(o, chunks, st);
   }
 }
 
@@ -482,9 +515,6 @@ cudaError_t launch_sort(const SortPlan& plan, const SortBuffers& b, int* out_buf
   if (plan.n <= 1 || plan.passes == 0) return cudaSuccess;
   cudaError_t e;
   if ((e = cudaMemsetAsync(b.hist, 0, sizeof(uint32_t) * kMaxPasses * kRadix, st)) != cudaSuccess) return e;
-  if ((e = cudaFuncSetAttribute(downsweep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                static_cast<int>(sizeof(DownsweepSmem)))) != cudaSuccess)
-    return e;
   const unsigned chunks = static_cast<unsigned>(plan.tiles);
   int cur = 0;
   for (int p = 0; p < plan.passes; ++p) {
@@ -504,8 +534,7 @@ cudaError_t launch_sort(const SortPlan& plan, const SortBuffers& b, int* out_buf
     o.offsets = counts;
     o.chunks = plan.tiles;
     o.err = b.err;
-    downsweep_kernel<<<chunks, kSortThreads, sizeof(DownsweepSmem), st>>>(o);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = launch_downsweep_bits(o, digit_bits, chunks, st)) != cudaSuccess) return e;
     cur ^= 1;
   }
   *out_buf = cur;
