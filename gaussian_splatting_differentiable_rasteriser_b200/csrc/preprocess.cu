@@ -26,6 +26,78 @@ __device__ __forceinline__ double dot3(const double* a, const double* b) {
 }
 
 constexpr int kPreThreads = 256;
+
+// Screen covariance of one Gaussian before the dilation, V = T Sigma T^T with
+// T = J W and Sigma = M M^T, M = R(q/|q|) diag(exp(ls)), computed in type S.
+// With w_k = t0 . M_k and v_k = t1 . M_k (M_k the columns of M, t0 and t1 the
+// rows of T): V = [[w.w, w.v], [w.v, v.v]] and det V = |w x v|^2 (Lagrange's
+// identity), so det V and det(V + 0.3 I) = det V + 0.3 (V00 + V11) + 0.09 are
+// sums of non-negative terms and carry no cancellation in float32.
+template <typename S>
+struct ScreenCov {
+  S a0, b0, c0, det0;
+};
+
+template <typename S>
+__device__ __forceinline__ ScreenCov<S> screen_cov(const float q4[4], const float ls3[3], double X, double Y,
+                                                   double Z, const CamArgs& cam) {
+  const S qw = q4[0], qx = q4[1], qy = q4[2], qz = q4[3];
+  const S qn = sqrt(qw * qw + qx * qx + qy * qy + qz * qz);
+  const S w = qw / qn, x = qx / qn, y = qy / qn, z = qz / qn;
+  const S one = 1, two = 2;
+  const S Rq[9] = {one - two * (y * y + z * z), two * (x * y - w * z), two * (x * z + w * y),
+                   two * (x * y + w * z), one - two * (x * x + z * z), two * (y * z - w * x),
+                   two * (x * z - w * y), two * (y * z + w * x), one - two * (x * x + y * y)};
+  const S sc[3] = {exp(static_cast<S>(ls3[0])), exp(static_cast<S>(ls3[1])), exp(static_cast<S>(ls3[2]))};
+  const S iz = one / static_cast<S>(Z);
+  const S fx = static_cast<S>(cam.fx), fy = static_cast<S>(cam.fy);
+  const S jx = fx * iz, jy = fy * iz;
+  const S jxz = -fx * static_cast<S>(X) * iz * iz, jyz = -fy * static_cast<S>(Y) * iz * iz;
+  S t0[3], t1[3];
+#pragma unroll
+  for (int c = 0; c < 3; ++c) {
+    t0[c] = jx * static_cast<S>(cam.R[c]) + jxz * static_cast<S>(cam.R[6 + c]);
+    t1[c] = jy * static_cast<S>(cam.R[3 + c]) + jyz * static_cast<S>(cam.R[6 + c]);
+  }
+  S wv[3], vv[3];
+#pragma unroll
+  for (int k = 0; k < 3; ++k) {
+    wv[k] = (t0[0] * Rq[k] + t0[1] * Rq[3 + k] + t0[2] * Rq[6 + k]) * sc[k];
+    vv[k] = (t1[0] * Rq[k] + t1[1] * Rq[3 + k] + t1[2] * Rq[6 + k]) * sc[k];
+  }
+  ScreenCov<S> r;
+  r.a0 = wv[0] * wv[0] + wv[1] * wv[1] + wv[2] * wv[2];
+  r.b0 = wv[0] * vv[0] + wv[1] * vv[1] + wv[2] * vv[2];
+  r.c0 = vv[0] * vv[0] + vv[1] * vv[1] + vv[2] * vv[2];
+  const S cx = wv[1] * vv[2] - wv[2] * vv[1], cy = wv[2] * vv[0] - wv[0] * vv[2], cz = wv[0] * vv[1] - wv[1] * vv[0];
+  r.det0 = cx * cx + cy * cy + cz * cz;
+  return r;
+}
+
+// Tile-rect radius from the dilated covariance (the largest eigenvalue, with
+// the cancellation-free discriminant) and, with the opacity-aware cut, the
+// opacity o (times the compensation factor).
+template <typename S>
+__device__ __forceinline__ S rect_radius(const ScreenCov<S>& v, bool opacity_rect, S o) {
+  const S a = v.a0 + static_cast<S>(kDilation), c = v.c0 + static_cast<S>(kDilation);
+  const S hd = static_cast<S>(0.5) * (a - c);
+  const S lmax = static_cast<S>(0.5) * (a + c) + sqrt(hd * hd + v.b0 * v.b0);
+  if (!opacity_rect) return static_cast<S>(kRadiusSigmas) * sqrt(lmax);
+  const S e_cut = fmin(static_cast<S>(4.5), log(fmax(o * static_cast<S>(255), static_cast<S>(1.0001))));
+  return sqrt(static_cast<S>(2) * e_cut) * sqrt(lmax);
+}
+
+// The compensation factor sqrt(det V / det(V + 0.3 I)) (1 when not enabled).
+template <typename S>
+__device__ __forceinline__ S compensation(const ScreenCov<S>& v, bool on) {
+  if (!on) return static_cast<S>(1);
+  const S det = v.det0 + static_cast<S>(kDilation) * (v.a0 + v.c0) + static_cast<S>(kDilation * kDilation);
+  return v.det0 > static_cast<S>(0) ? sqrt(v.det0 / det) : static_cast<S>(0);
+}
+
+// x is farther than m from every integer (the rounding of x by ceil or floor
+// cannot change within +-m).
+__device__ __forceinline__ bool clear_of_integers(double x, double m) { return fabs(x - rint(x)) > m; }
 constexpr int kGeomPlanes = 11;  // means 3, log-scales 3, quats 4, opacity logit 1
 
 // The parameters of a CTA's 256 Gaussians, one 1 KB row per plane: the
@@ -120,63 +192,41 @@ __global__ void __launch_bounds__(kPreThreads, 3) preprocess_kernel(PreprocessAr
     uint2 rect = make_uint2(1u, 1u);  // x0 = 1 > x1 = 0: empty
     uint8_t clamped = 0;
     if (Z > static_cast<double>(cam.near_z)) {
-      // Sigma = M M^T, M = R(q/|q|) diag(exp(ls))
-      const double qw = sm.plane[6][tid], qx = sm.plane[7][tid], qy = sm.plane[8][tid],
-                   qz = sm.plane[9][tid];
-      const double qn = sqrt(qw * qw + qx * qx + qy * qy + qz * qz);
-      const double w = qw / qn, x = qx / qn, y = qy / qn, z = qz / qn;
-      const double Rq[9] = {1.0 - 2.0 * (y * y + z * z), 2.0 * (x * y - w * z), 2.0 * (x * z + w * y),
-                            2.0 * (x * y + w * z), 1.0 - 2.0 * (x * x + z * z), 2.0 * (y * z - w * x),
-                            2.0 * (x * z - w * y), 2.0 * (y * z + w * x), 1.0 - 2.0 * (x * x + y * y)};
-      const double sc[3] = {exp(static_cast<double>(sm.plane[3][tid])),
-                            exp(static_cast<double>(sm.plane[4][tid])),
-                            exp(static_cast<double>(sm.plane[5][tid]))};
-      double M[9];
-#pragma unroll
-      for (int r = 0; r < 3; ++r)
-#pragma unroll
-        for (int c = 0; c < 3; ++c) M[3 * r + c] = Rq[3 * r + c] * sc[c];
-      const double S00 = dot3(M, M), S01 = dot3(M, M + 3), S02 = dot3(M, M + 6);
-      const double S11 = dot3(M + 3, M + 3), S12 = dot3(M + 3, M + 6), S22 = dot3(M + 6, M + 6);
-      // T = J W (rows t0, t1)
+      const float q4[4] = {sm.plane[6][tid], sm.plane[7][tid], sm.plane[8][tid], sm.plane[9][tid]};
+      const float ls3[3] = {sm.plane[3][tid], sm.plane[4][tid], sm.plane[5][tid]};
       const double iz = 1.0 / Z;
-      const double jx = cam.fx * iz, jy = cam.fy * iz;
-      const double jxz = -cam.fx * X * iz * iz, jyz = -cam.fy * Y * iz * iz;
-      double t0[3], t1[3];
-#pragma unroll
-      for (int c = 0; c < 3; ++c) {
-        t0[c] = jx * cam.R[c] + jxz * cam.R[6 + c];
-        t1[c] = jy * cam.R[3 + c] + jyz * cam.R[6 + c];
-      }
-      // Sigma' = T Sigma T^T + 0.3 I
-      const double u0[3] = {S00 * t0[0] + S01 * t0[1] + S02 * t0[2],
-                            S01 * t0[0] + S11 * t0[1] + S12 * t0[2],
-                            S02 * t0[0] + S12 * t0[1] + S22 * t0[2]};
-      const double u1[3] = {S00 * t1[0] + S01 * t1[1] + S02 * t1[2],
-                            S01 * t1[0] + S11 * t1[1] + S12 * t1[2],
-                            S02 * t1[0] + S12 * t1[1] + S22 * t1[2]};
-      const double ca = dot3(t0, u0) + kDilation;
-      const double cb = dot3(t0, u1);
-      const double cc = dot3(t1, u1) + kDilation;
-      const double det = ca * cc - cb * cb;
-      // Mip-Splatting compensation: sqrt(det V / det(V + 0.3 I)), V undilated
-      double comp = 1.0;
-      if (a.mip_comp) {
-        const double det0 = (ca - kDilation) * (cc - kDilation) - cb * cb;
-        comp = det0 > 0.0 ? sqrt(det0 / det) : 0.0;
-      }
-      if (det > 0.0) {
-        const double u = cam.fx * X * iz + cam.cx;
-        const double v = cam.fy * Y * iz + cam.cy;
-        const double mid = 0.5 * (ca + cc);
-        const double lmax = mid + sqrt(fmax(mid * mid - det, 0.0));
-        double rad = kRadiusSigmas * sqrt(lmax);
-        if (a.opacity_rect) {
-          // opacity-aware cut: beyond sqrt(2 E) sigma along the long axis alpha < 1/255
-          const double od = 1.0 / (1.0 + exp(-static_cast<double>(sm.plane[10][tid]))) * comp;
-          const double e_cut = fmin(4.5, log(fmax(od * 255.0, 1.0001)));
-          rad = sqrt(2.0 * e_cut) * sqrt(lmax);
+      const double u = cam.fx * X * iz + cam.cx;
+      const double v = cam.fy * Y * iz + cam.cy;
+      const float sig = 1.0f / (1.0f + expf(-sm.plane[10][tid]));
+      // The covariance chain in float32. The tile rect is an integer decision:
+      // where a rect bound lies within 1e-4 r + 1e-3 px of a tile boundary (far
+      // beyond the float32 error of r) the chain is redone in float64, the
+      // precision in which the rect is defined, so rects never depend on the
+      // float32 rounding.
+      const ScreenCov<float> vf = screen_cov<float>(q4, ls3, X, Y, Z, cam);
+      float comp = compensation<float>(vf, a.mip_comp != 0);
+      double rad = rect_radius<float>(vf, a.opacity_rect != 0, sig * comp);
+      float ca = vf.a0 + static_cast<float>(kDilation), cc = vf.c0 + static_cast<float>(kDilation), cb = vf.b0;
+      float det = vf.det0 + static_cast<float>(kDilation) * (vf.a0 + vf.c0) +
+                  static_cast<float>(kDilation * kDilation);
+      {
+        const double m = (1e-4 * rad + 1e-3) / kTile;
+        const bool sure = clear_of_integers((u - rad - (kTile - 1)) / kTile, m) &&
+                          clear_of_integers((u + rad) / kTile, m) &&
+                          clear_of_integers((v - rad - (kTile - 1)) / kTile, m) &&
+                          clear_of_integers((v + rad) / kTile, m) && rad == rad;
+        if (!sure) {
+          const ScreenCov<double> vd = screen_cov<double>(q4, ls3, X, Y, Z, cam);
+          const double compd = compensation<double>(vd, a.mip_comp != 0);
+          rad = rect_radius<double>(vd, a.opacity_rect != 0, static_cast<double>(sig) * compd);
+          comp = static_cast<float>(compd);
+          ca = static_cast<float>(vd.a0 + kDilation);
+          cc = static_cast<float>(vd.c0 + kDilation);
+          cb = static_cast<float>(vd.b0);
+          det = static_cast<float>(vd.det0 + kDilation * (vd.a0 + vd.c0) + kDilation * kDilation);
         }
+      }
+      if (det > 0.0f) {
         // tiles whose pixels [16 t, 16 t + 15] meet [u - r, u + r] (same for y)
         double fx0 = fmax(ceil((u - rad - (kTile - 1)) / kTile), 0.0);
         double fx1 = fmin(floor((u + rad) / kTile), static_cast<double>(cam.tiles_x - 1));
@@ -189,17 +239,15 @@ __global__ void __launch_bounds__(kPreThreads, 3) preprocess_kernel(PreprocessAr
           touched = (x1 - x0 + 1) * (y1 - y0 + 1);
           visible = true;
           dkey = __float_as_uint(depth);
-          float opacity = 1.0f / (1.0f + expf(-sm.plane[10][tid]));
-          if (a.mip_comp) opacity = static_cast<float>(static_cast<double>(opacity) * comp);
+          const float opacity = sig * comp;
           // view-dependent colour at v = normalize(p - campos); its SH planes
           // were still arriving while the geometry above ran
           sh_ok = mbar_wait(&sm.bar[1], 0, 1 << 16);
-          double d[3] = {p[0] - cam.campos[0], p[1] - cam.campos[1], p[2] - cam.campos[2]};
-          const double dn = sqrt(dot3(d, d));
-          const float dx = static_cast<float>(d[0] / dn), dy = static_cast<float>(d[1] / dn),
-                      dz = static_cast<float>(d[2] / dn);
+          const float d[3] = {static_cast<float>(p[0] - cam.campos[0]), static_cast<float>(p[1] - cam.campos[1]),
+                              static_cast<float>(p[2] - cam.campos[2])};
+          const float idn = rsqrtf(d[0] * d[0] + d[1] * d[1] + d[2] * d[2]);
           float Yk[16];
-          sh_basis(kDeg, dx, dy, dz, Yk);
+          sh_basis(kDeg, d[0] * idn, d[1] * idn, d[2] * idn, Yk);
           float rgb[3];
 #pragma unroll
           for (int ch = 0; ch < 3; ++ch) {
@@ -217,17 +265,15 @@ __global__ void __launch_bounds__(kPreThreads, 3) preprocess_kernel(PreprocessAr
           // ln(255 o), an ellipse with axis-aligned half-widths sqrt(2 E a),
           // sqrt(2 E c) (a, c the diagonal of Sigma'), widened by 0.1% + 0.02 px so
           // float32 rounding of the per-pixel alpha never passes the floor outside.
-          const double l2e = 1.4426950408889634;
-          const double E = log(255.0 * static_cast<double>(opacity));
+          const float E = logf(255.0f * opacity);
           float hx = -1.0f, hy = -1.0f;
-          if (E > 0.0) {
-            hx = static_cast<float>(sqrt(2.0 * E * ca) * 1.001 + 0.02);
-            hy = static_cast<float>(sqrt(2.0 * E * cc) * 1.001 + 0.02);
+          if (E > 0.0f) {
+            hx = sqrtf(2.0f * E * ca) * 1.001f + 0.02f;
+            hy = sqrtf(2.0f * E * cc) * 1.001f + 0.02f;
           }
-          s.a = make_float4(static_cast<float>(u), static_cast<float>(v),
-                            static_cast<float>(-0.5 * l2e * cc / det), static_cast<float>(l2e * cb / det));
-          s.b = make_float4(static_cast<float>(-0.5 * l2e * ca / det),
-                            static_cast<float>(log2(static_cast<double>(opacity))), rgb[0], rgb[1]);
+          const float idet = kLog2e / det;
+          s.a = make_float4(static_cast<float>(u), static_cast<float>(v), -0.5f * cc * idet, cb * idet);
+          s.b = make_float4(-0.5f * ca * idet, log2f(opacity), rgb[0], rgb[1]);
           s.c = make_float4(rgb[2], opacity, hx, hy);
         }
       }

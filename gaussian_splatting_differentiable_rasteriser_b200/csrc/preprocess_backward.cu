@@ -144,10 +144,13 @@ struct FusedSmem {
 // r % kStages, kStages rounds ahead of their use, so several planes' loads per
 // thread are in flight with no register held for them, and the first rounds
 // overlap the projection backward of phase 1. Measured on B200 (Dense, 3M
-// Gaussians): 2 planes x 2 stages at 5 CTAs per SM beat both 4 planes x 2
-// stages (3 CTAs per SM, 33% slower) and the register-staged stream (3% slower).
+// Gaussians; Heavy-tail, 6M): 1 plane x 2 stages at 7 CTAs per SM, 0.844 ms
+// (1.82 ms); 2 planes x 2 stages at 5 CTAs per SM 0.915 ms; 1 plane x 4
+// stages 0.933 ms; 2 planes x 3 stages 1.03 ms; 4 planes x 2 stages (3 CTAs
+// per SM) 1.23 ms; the register-staged stream 0.955 ms. Resident CTAs
+// matter more than the depth of each one's pipeline.
 #ifndef GS_FUSED_ROUND
-#define GS_FUSED_ROUND 2
+#define GS_FUSED_ROUND 1
 #endif
 #ifndef GS_FUSED_STAGES
 #define GS_FUSED_STAGES 2
