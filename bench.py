@@ -325,7 +325,7 @@ def profile_stages(step, cams, targets, sched, start, count):
         img, T, nc = step.forward(cs, cam.height, cam.width)
         ks.append(step.last_entries)
         step.compute_loss(img, targets[c], step.dimage)
-        if step.fused_adam:
+        if step.fused_adam or getattr(step, "exchange", None) == "views":
             step.backward_and_update(cs, T, nc, step.dimage)
             continue
         m.step_count += 1
@@ -382,6 +382,9 @@ def stage_models(scene, sh_k, loss="l1_dssim"):
         # source, zeroing it): the same 32 B per scalar; with several ranks the stage
         # also holds the two barriers and the NVLink transfers
         "exchange_adam": ("hbm", 32),
+        # the views update on one rank, per Gaussian of its range: p, m, v read and
+        # written (24 B per scalar), the view's screen record, raw sums and flags
+        "views_adam": ("hbm", 24 * n_par + 48 + 48 + 5),
         # fused projection backward + Adam with no accumulated gradient (one view per
         # step): p, m, v read and written, 24 B per scalar of every group, plus the raw
         # screen-gradient sums, the screen record and two flags, per Gaussian
@@ -623,6 +626,7 @@ def main_ours(args):
            "preprocess": "preprocess.cu", "sort": "sort.cu", "depth_sort": "sort.cu", "loss": "loss.cu",
            "preprocess_backward": "preprocess_backward.cu",
            "backward_adam": "preprocess_backward.cu", "exchange_adam": "adam_reduce.cu",
+           "views_adam": "views_adam.cu",
            "camera_backward": "camera_backward.cu"}.get(dominant)
     tr = NCU_TRAFFIC.get(dominant)
     rf["traffic"] = None
@@ -656,7 +660,10 @@ def main_ours(args):
                                                              if args.gaussians else ""),
                        "gaussians": scene.n,
                        "width": W, "height": H, "cameras": len(cams),
-                       "parallelism": (("data-parallel: one camera per rank; gradient exchange fused with "
+                       "parallelism": (("data-parallel: one camera per rank; each rank's screen-space view "
+                                        "read by the owner of each Gaussian, projection backward and Adam "
+                                        "fused (gs_adam_step_views)" if args.exchange == "views" else
+                                        "data-parallel: one camera per rank; gradient exchange fused with "
                                         "the sharded Adam over peer memory (gs_adam_step_reduce)"
                                         if args.exchange == "p2p" else
                                         "data-parallel: one camera per rank; NCCL reduce-scatter, "
@@ -1000,8 +1007,10 @@ def main():
     ap.add_argument("--parallel", choices=("replicas", "dp"), default="replicas",
                     help="N>1: independent replicas (default), or data-parallel training over cameras "
                          "(one camera per rank per iteration; value counts camera-iterations)")
-    ap.add_argument("--exchange", choices=("p2p", "nccl"), default="p2p",
-                    help="--parallel dp: the fused peer-memory exchange + Adam, or NCCL collectives")
+    ap.add_argument("--exchange", choices=("views", "p2p", "nccl"), default="views",
+                    help="--parallel dp: each rank's screen-space view read by the owner of each Gaussian "
+                         "(projection backward + Adam fused), the gradient exchange fused with Adam over peer "
+                         "memory, or NCCL collectives")
     ap.add_argument("--gaussians", type=int, default=None,
                     help="draw this many Gaussians instead (dense, heavy_tail): a same-shaped smaller case")
     ap.add_argument("--capacity", type=int, default=None,

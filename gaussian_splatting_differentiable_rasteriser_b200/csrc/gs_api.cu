@@ -19,6 +19,8 @@ struct gs_ctx {
   int32_t max_w = 0, max_h = 0;
   // per Gaussian
   gs::Screen* screen = nullptr;
+  gs::CamArgs* cam_dev = nullptr;  // the camera of the last blend backward (data-parallel views)
+  bool have_view = false;
   float* depth = nullptr;
   uint2* rect = nullptr;
   uint32_t* touched = nullptr;
@@ -113,7 +115,7 @@ void free_all(gs_ctx* c) {
                   c->hist, c->offsets, c->status, c->counters, c->ranges, c->surv, c->surv_count,
                   c->sgrad_fixed, c->dens_counts, c->dens_prefix, c->dens_totals, c->charb_partials,
                   c->charb_counter, c->cam_partials, c->cam_counter, c->reloc_dead, c->loss_partials,
-                  c->loss_counter, c->info_dev, c->pairs};
+                  c->loss_counter, c->info_dev, c->pairs, c->cam_dev};
   for (void* b : bufs)
     if (b) cudaFree(b);
   if (c->info_host) cudaFreeHost(c->info_host);
@@ -261,7 +263,7 @@ gs_status gs_create(gs_ctx** out, int64_t max_gaussians, int64_t max_entries, in
   c->max_w = max_width;
   c->max_h = max_height;
   c->max_tiles = static_cast<int64_t>((max_width + 15) / 16) * ((max_height + 15) / 16);
-  c->max_blocks = (max_gaussians + 255) / 256;
+  c->max_blocks = (max_gaussians + gs::kGaussBlock - 1) / gs::kGaussBlock;
   // the depth sort (visible Gaussians) and the tile sort (entries) share the look-back words
   c->max_sort_tiles = (std::max(max_entries, max_gaussians) + gs::kSortTileKeys - 1) / gs::kSortTileKeys;
   c->max_loss_blocks = gs::loss_num_blocks(max_height, max_width);
@@ -270,6 +272,7 @@ gs_status gs_create(gs_ctx** out, int64_t max_gaussians, int64_t max_entries, in
 #define GS_ALLOC(ptr, bytes) \
   if (e == cudaSuccess) e = cudaMalloc(reinterpret_cast<void**>(&(ptr)), (bytes))
   GS_ALLOC(c->screen, sizeof(gs::Screen) * G);
+  GS_ALLOC(c->cam_dev, sizeof(gs::CamArgs));
   GS_ALLOC(c->depth, sizeof(float) * G);
   GS_ALLOC(c->rect, sizeof(uint2) * G);
   GS_ALLOC(c->touched, sizeof(uint32_t) * G);
@@ -390,7 +393,7 @@ gs_status gs_preprocess(gs_ctx* c, const gs_params* p, const gs_camera* cam, voi
   a.err = &c->info_dev->device_error;
   a.opacity_rect = c->opacity_rect;
   a.mip_comp = c->mip_comp;
-  const int64_t nb = (p->n + 255) / 256;
+  const int64_t nb = (p->n + gs::kGaussBlock - 1) / gs::kGaussBlock;
   prof_begin(c, st);
   GS_CUDA(c, gs::launch_preprocess(a, nb, st));
   prof_end(c, GS_STAGE_PREPROCESS, p->n, st, p->n > 0 ? 1 : 0);
@@ -461,7 +464,7 @@ gs_status gs_render_forward(gs_ctx* c, const gs_camera* cam, float* image, float
     b.vals[1] = c->dvals[1];
     int dsorted = 0;
     prof_begin(c, st);
-    GS_CUDA(c, gs::launch_compact(ca2, (c->n + 255) / 256, st));
+    GS_CUDA(c, gs::launch_compact(ca2, (c->n + gs::kGaussBlock - 1) / gs::kGaussBlock, st));
     GS_CUDA(c, gs::launch_sort(dplan, b, &dsorted, st));
     prof_end(c, GS_STAGE_DEPTH_SORT, dplan.n > 1 ? dplan.n * dplan.passes : 0, st,
              (c->n > 0 ? 1 : 0) + sort_kernels(dplan));
@@ -669,10 +672,18 @@ gs_status gs_render_backward_adam(gs_ctx* c, const gs_params* p, const gs_camera
   for (int k = 0; k < 5; ++k)
     if (!std::isfinite(lr[k])) return fail(c, GS_ERR_INVALID_ARG, "learning rates must be finite");
   if (p && p->n_pad > 0) {
+    // the fused pass moves moments (and an accumulated gradient) as float4
     float* mp[] = {m->means, m->log_scales, m->quats, m->opacity_logits, m->sh,
                    v->means, v->log_scales, v->quats, v->opacity_logits, v->sh};
     for (float* q : mp)
-      if (!q || !aligned(q, 4)) return fail(c, GS_ERR_INVALID_ARG, "a moment pointer is NULL or misaligned");
+      if (!q || !aligned(q, 16))
+        return fail(c, GS_ERR_INVALID_ARG, "a moment pointer is NULL or not 16-byte aligned");
+    if (g) {
+      float* gp[] = {g->means, g->log_scales, g->quats, g->opacity_logits, g->sh};
+      for (float* q : gp)
+        if (!q || !aligned(q, 16))
+          return fail(c, GS_ERR_INVALID_ARG, "a gradient pointer is NULL or not 16-byte aligned");
+    }
   }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   gs::PreprocessBwdArgs a;
@@ -700,6 +711,112 @@ gs_status gs_render_backward_adam(gs_ctx* c, const gs_params* p, const gs_camera
   prof_begin(c, st);
   GS_CUDA(c, gs::launch_preprocess_backward_adam(a, f, st));
   prof_end(c, GS_STAGE_BACKWARD_ADAM, p->n_pad, st, p->n_pad > 0 ? 1 : 0);
+  return GS_OK;
+}
+
+gs_status gs_render_backward_screen(gs_ctx* c, const gs_params* p, const gs_camera* cam, const float* final_T,
+                                    const int32_t* n_contrib, const float* dloss_dimage, void* stream) {
+  if (!c) return GS_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  gs::PreprocessBwdArgs a;
+  gs_status s = backward_common(c, p, cam, final_T, n_contrib, dloss_dimage, nullptr, true, st, a);
+  if (s != GS_OK) return s;
+  // the camera of this view, for the ranks whose update kernels read it
+  GS_CUDA(c, cudaMemcpyAsync(c->cam_dev, &c->cam, sizeof(gs::CamArgs), cudaMemcpyHostToDevice, st));
+  c->have_view = true;
+  return GS_OK;
+}
+
+gs_status gs_get_view(const gs_ctx* c, gs_view* out) {
+  if (!c || !out) return GS_ERR_INVALID_ARG;
+  out->screen = c->screen;
+  out->sums = c->sgrad;
+  out->touched = c->touched;
+  out->clamped = c->clamped;
+  out->camera = c->cam_dev;
+  return GS_OK;
+}
+
+gs_status gs_shared_handle(const void* ptr, unsigned char* handle) {
+  if (!ptr || !handle) return GS_ERR_INVALID_ARG;
+  cudaIpcMemHandle_t h;
+  if (cudaIpcGetMemHandle(&h, const_cast<void*>(ptr)) != cudaSuccess) {
+    cudaGetLastError();
+    return GS_ERR_CUDA;
+  }
+  std::memcpy(handle, &h, sizeof(h));
+  return GS_OK;
+}
+
+gs_status gs_adam_step_views(gs_ctx* c, const gs_params* p, const gs_view* views, int32_t n_views, int64_t g_lo,
+                             int64_t g_hi, const gs_grads* copies, int32_t n_copies, gs_grads* m, gs_grads* v,
+                             const float* lr, float grad_scale, float beta1, float beta2, float eps, int32_t step,
+                             void* stream) {
+  if (!c) return GS_ERR_INVALID_ARG;
+  gs_status s = check_params(c, p);
+  if (s != GS_OK) return s;
+  if (!views || n_views < 1 || n_views > gs::kMaxRanks || n_copies < 0 || n_copies > gs::kMaxRanks ||
+      (n_copies > 0 && !copies))
+    return fail(c, GS_ERR_INVALID_ARG, "1..%d views and 0..%d copies required", gs::kMaxRanks, gs::kMaxRanks);
+  if (g_lo < 0 || g_hi < g_lo || g_hi > p->n_pad || g_lo % 4 != 0 || g_hi % 4 != 0)
+    return fail(c, GS_ERR_INVALID_ARG, "Gaussian range [%lld, %lld) must lie in [0, n_pad] on multiples of 4",
+                (long long)g_lo, (long long)g_hi);
+  if (!m || !v || !lr) return fail(c, GS_ERR_INVALID_ARG, "moments and learning rates must be non-NULL");
+  if (step < 1 || !valid_betas(beta1, beta2, eps) || !std::isfinite(grad_scale))
+    return fail(c, GS_ERR_INVALID_ARG, "step must be >= 1, betas in [0, 1), eps > 0, grad_scale finite");
+  for (int k = 0; k < 5; ++k)
+    if (!std::isfinite(lr[k])) return fail(c, GS_ERR_INVALID_ARG, "learning rates must be finite");
+  gs::ViewsAdamArgs a{};
+  a.base.means = p->means;
+  a.base.log_scales = p->log_scales;
+  a.base.quats = p->quats;
+  a.base.opacity_logits = p->opacity_logits;
+  a.base.sh = p->sh;
+  a.base.n = p->n;
+  a.base.n_pad = p->n_pad;
+  a.base.sh_k = (p->sh_degree + 1) * (p->sh_degree + 1);
+  a.base.active_degree = p->active_degree;
+  a.base.mip_comp = c->mip_comp;
+  a.n_views = n_views;
+  for (int r = 0; r < n_views; ++r) {
+    const gs_view& w = views[r];
+    if (!w.screen || !w.sums || !w.touched || !w.clamped || !w.camera || !aligned(w.screen, 16) ||
+        !aligned(w.sums, 16) || !aligned(w.touched, 4) || !aligned(w.camera, 4))
+      return fail(c, GS_ERR_INVALID_ARG, "view %d has a NULL or misaligned pointer", r);
+    a.views[r].screen = static_cast<const gs::Screen*>(w.screen);
+    a.views[r].sgrad = w.sums;
+    a.views[r].touched = w.touched;
+    a.views[r].clamped = w.clamped;
+    a.views[r].cam = static_cast<const gs::CamArgs*>(w.camera);
+  }
+  a.g_lo = g_lo;
+  a.g_hi = g_hi;
+  float* mm[5] = {m->means, m->log_scales, m->quats, m->opacity_logits, m->sh};
+  float* vv[5] = {v->means, v->log_scales, v->quats, v->opacity_logits, v->sh};
+  const float* pp[5] = {p->means, p->log_scales, p->quats, p->opacity_logits, p->sh};
+  for (int k = 0; k < 5; ++k) {
+    if (g_hi > g_lo && (!mm[k] || !vv[k] || !aligned(mm[k], 16) || !aligned(vv[k], 16)))
+      return fail(c, GS_ERR_INVALID_ARG, "a moment pointer is NULL or not 16-byte aligned");
+    a.f.p[k] = const_cast<float*>(pp[k]);  // documented: updated in place
+    a.f.g[k] = nullptr;
+    a.f.m[k] = mm[k];
+    a.f.v[k] = vv[k];
+    a.f.s[k] = gs::adam_scalars(lr[k], beta1, beta2, eps, step);
+  }
+  a.n_copies = n_copies;
+  for (int d = 0; d < n_copies; ++d) {
+    float* cp[5] = {copies[d].means, copies[d].log_scales, copies[d].quats, copies[d].opacity_logits, copies[d].sh};
+    for (int k = 0; k < 5; ++k) {
+      if (g_hi > g_lo && (!cp[k] || !aligned(cp[k], 16)))
+        return fail(c, GS_ERR_INVALID_ARG, "copy %d has a NULL or misaligned group pointer", d);
+      a.copies[d][k] = cp[k];
+    }
+  }
+  a.grad_scale = grad_scale;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  prof_begin(c, st);
+  GS_CUDA(c, gs::launch_views_adam(a, st));
+  prof_end(c, GS_STAGE_VIEWS_ADAM, g_hi - g_lo, st, g_hi > g_lo ? 1 : 0);
   return GS_OK;
 }
 
@@ -839,7 +956,7 @@ const char* gs_stage_name(int32_t stage) {
   static const char* names[GS_NUM_STAGES] = {"preprocess", "scan", "duplicate", "sort", "ranges",
                                              "blend_forward", "loss", "blend_backward",
                                              "preprocess_backward", "backward_adam", "depth_sort",
-                                             "camera_backward"};
+                                             "camera_backward", "views_adam"};
   return (stage >= 0 && stage < GS_NUM_STAGES) ? names[stage] : "";
 }
 

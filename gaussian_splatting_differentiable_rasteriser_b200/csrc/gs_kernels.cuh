@@ -17,6 +17,14 @@ struct ForwardInfo {
   uint32_t device_error;
 };
 
+// Gaussians per preprocess CTA, and the granularity of the per-block totals
+// (tiles touched, visible Gaussians) that the block scan and the compaction use.
+#ifndef GS_PRE_BLOCK
+#define GS_PRE_BLOCK 256
+#endif
+constexpr int kGaussBlock = GS_PRE_BLOCK;
+static_assert(kGaussBlock == 128 || kGaussBlock == 256, "preprocess block");
+
 struct PreprocessArgs {
   const float *means, *log_scales, *quats, *opacity_logits, *sh;
   int64_t n, n_pad;
@@ -100,8 +108,11 @@ struct DuplicateArgs {
   uint32_t* chunk_offsets;  // [ceil(count / kDupItems)] scratch: tiles per chunk, then their prefix
   uint32_t* err;
 };
+#ifndef GS_DUP_PER_THREAD
+#define GS_DUP_PER_THREAD 16
+#endif
 constexpr int kDupThreads = 256;
-constexpr int kDupPerThread = 16;
+constexpr int kDupPerThread = GS_DUP_PER_THREAD;  // visible Gaussians per thread of a duplicate CTA
 constexpr int kDupItems = kDupThreads * kDupPerThread;
 cudaError_t launch_duplicate(const DuplicateArgs& a, cudaStream_t st);
 
@@ -301,5 +312,29 @@ struct ReduceAdamArgs {
 };
 
 cudaError_t launch_adam_reduce(const ReduceAdamArgs& a, cudaStream_t st);
+
+// ------------------------------- data-parallel update from the views' sums
+// One rank's view of the Gaussians after its blend backward (device pointers,
+// local or peer memory): screen records, raw screen-gradient sums, touched and
+// clamp flags, and its camera record.
+struct ViewArgs {
+  const Screen* screen;
+  const float* sgrad;
+  const uint32_t* touched;
+  const uint8_t* clamped;
+  const CamArgs* cam;
+};
+
+struct ViewsAdamArgs {
+  PreprocessBwdArgs base;  // this rank's parameters, sizes and options (view fields unused)
+  ViewArgs views[kMaxRanks];
+  int n_views;
+  int64_t g_lo, g_hi;      // this rank's Gaussians [g_lo, g_hi), multiples of 4
+  FusedAdamArgs f;         // parameters (updated in place), moments, per-group scalars
+  float* copies[kMaxRanks][5];  // other ranks' parameter groups (peer memory)
+  int n_copies;
+  float grad_scale;        // 1 / ranks: the batch mean
+};
+cudaError_t launch_views_adam(const ViewsAdamArgs& a, cudaStream_t st);
 
 }  // namespace gs

@@ -25,7 +25,7 @@ __device__ __forceinline__ double dot3(const double* a, const double* b) {
   return a[0] * b[0] + a[1] * b[1] + a[2] * b[2];
 }
 
-constexpr int kPreThreads = 256;
+constexpr int kPreThreads = kGaussBlock;
 
 // Screen covariance of one Gaussian before the dilation, V = T Sigma T^T with
 // T = J W and Sigma = M M^T, M = R(q/|q|) diag(exp(ls)), computed in type S.
@@ -109,7 +109,7 @@ struct PreprocessSmem {
 };
 
 template <int kDeg>
-__global__ void __launch_bounds__(kPreThreads, 3) preprocess_kernel(PreprocessArgs a) {
+__global__ void __launch_bounds__(kPreThreads, kPreThreads == 256 ? 3 : 6) preprocess_kernel(PreprocessArgs a) {
   constexpr int nk = (kDeg + 1) * (kDeg + 1);
   constexpr int kPlanes = kGeomPlanes + 3 * nk;
   extern __shared__ __align__(128) unsigned char smem_raw[];
@@ -302,8 +302,8 @@ __global__ void __launch_bounds__(kPreThreads, 3) preprocess_kernel(PreprocessAr
   // Block totals of tiles touched and of visible Gaussians (for the entry
   // count and the compaction's prefix sum) and the depth-key range of visible
   // Gaussians (to size the depth sort's key).
-  __shared__ uint32_t s_sum[8];
-  __shared__ uint32_t s_vis[8];
+  __shared__ uint32_t s_sum[kPreThreads / 32];
+  __shared__ uint32_t s_vis[kPreThreads / 32];
   uint32_t t = touched;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);

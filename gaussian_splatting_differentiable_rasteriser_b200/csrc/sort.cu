@@ -42,8 +42,8 @@ namespace gs {
 namespace {
 
 // ---------------------------------------------------------------- compact --
-__global__ void __launch_bounds__(256) compact_kernel(CompactArgs a) {
-  __shared__ uint32_t s_warp[8];
+__global__ void __launch_bounds__(kGaussBlock) compact_kernel(CompactArgs a) {
+  __shared__ uint32_t s_warp[kGaussBlock / 32];
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const bool vis = i < a.n && a.touched[i] != 0u;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -495,7 +495,7 @@ __global__ void __launch_bounds__(256) ranges_kernel(const uint32_t* keys, int64
 
 cudaError_t launch_compact(const CompactArgs& a, int64_t num_blocks, cudaStream_t st) {
   if (num_blocks == 0) return cudaSuccess;
-  compact_kernel<<<static_cast<unsigned>(num_blocks), 256, 0, st>>>(a);
+  compact_kernel<<<static_cast<unsigned>(num_blocks), kGaussBlock, 0, st>>>(a);
   return cudaGetLastError();
 }
 

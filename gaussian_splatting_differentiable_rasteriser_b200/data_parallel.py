@@ -70,6 +70,30 @@ def exchange_and_update(grad_pad, param_pad, m_flat, v_flat, slices, total, worl
     grad_pad.zero_()
 
 
+def gaussian_bounds(n_pad: int, world: int, rank: int):
+    """[g_lo, g_hi) of the Gaussians rank owns in the "views" exchange: equal
+    ranges of whole float4 columns (multiples of 4 Gaussians), the last one
+    shorter when n_pad does not split evenly."""
+    per = (n_pad // 4 + world - 1) // world * 4
+    lo = min(n_pad, rank * per)
+    return lo, min(n_pad, lo + per)
+
+
+def gather_gaussian_shards(flat, n_pad, world, rank, group=None):
+    """The full planar buffer `flat` (every group's planes of n_pad Gaussians back
+    to back) assembled from every rank's own Gaussians [g_lo, g_hi) of each plane:
+    each rank zeroes the scalars it does not own and the buffers are summed
+    (every scalar has exactly one owner, so the sum is that owner's value)."""
+    collective = dist.is_available() and dist.is_initialized() and world > 1
+    if not collective:
+        return flat.clone()
+    lo, hi = gaussian_bounds(n_pad, world, rank)
+    col = torch.arange(flat.numel(), device=flat.device) % n_pad
+    mine = torch.where((col >= lo) & (col < hi), flat, torch.zeros_like(flat))
+    dist.all_reduce(mine, op=dist.ReduceOp.SUM, group=group)
+    return mine
+
+
 def gather_shards(flat, total, world, rank, group=None):
     """The full buffer of `total` floats assembled from every rank's own shard of
     `flat` (each rank's values outside its shard are ignored): the Adam moments
@@ -103,13 +127,20 @@ def p2p_pieces(slices, total, world, rank, param_ptrs, grad_ptrs):
 
 
 class DataParallelTrainStep(TrainStep):
-    """TrainStep whose update is the data-parallel one. The backward writes this
-    rank's gradient (gs_render_backward); then, with exchange="p2p" (default),
-    one gs_adam_step_reduce launch per parameter group in this rank's shard
-    reads every rank's gradient of the shard from peer memory, averages it in
-    rank order, runs Adam and writes the updated shard into every rank's
-    parameters; with exchange="nccl", exchange_and_update runs NCCL's
-    reduce-scatter, gs_adam_step on the shard and NCCL's all-gather.
+    """TrainStep whose update is the data-parallel one. With exchange="views"
+    (default) each rank runs only the blend backward of its camera
+    (gs_render_backward_screen); then one gs_adam_step_views launch on each rank
+    reads every rank's view of the Gaussians it owns (screen records, raw screen
+    sums, flags and camera, from peer memory), runs the projection backward of
+    every view, averages in rank order, applies Adam and writes the updated
+    parameters into every rank's buffer: no gradient buffer is written or
+    exchanged. With exchange="p2p" the backward writes this rank's gradient
+    (gs_render_backward), and one gs_adam_step_reduce launch per parameter
+    group in this rank's shard reads every rank's gradient of the shard from
+    peer memory, averages it in rank order, runs Adam and writes the updated
+    shard into every rank's parameters; with exchange="nccl",
+    exchange_and_update runs NCCL's reduce-scatter, gs_adam_step on the shard
+    and NCCL's all-gather. All three give the same bits.
 
     The parameter and gradient buffers are padded so every rank's shard has
     the same size and 16-byte-aligned bounds; for "p2p" they are shared
@@ -118,9 +149,9 @@ class DataParallelTrainStep(TrainStep):
     single-GPU one. Densification reallocates the model's buffers: build a new
     step after it. Call close() on every rank before the step is dropped."""
 
-    def __init__(self, model, max_entries, width, height, group=None, exchange="p2p", **kw):
-        if exchange not in ("p2p", "nccl"):
-            raise ValueError("exchange must be 'p2p' or 'nccl'")
+    def __init__(self, model, max_entries, width, height, group=None, exchange="views", **kw):
+        if exchange not in ("views", "p2p", "nccl"):
+            raise ValueError("exchange must be 'views', 'p2p' or 'nccl'")
         kw["fused_adam"] = False
         super().__init__(model, max_entries, width, height, **kw)
         self.group = group
@@ -134,6 +165,9 @@ class DataParallelTrainStep(TrainStep):
         pad = padded_size(self.total, self.world)
         dev = model.flat.device
         self._peer_maps = []
+        if exchange == "views":
+            self._init_views(model, on)
+            return
         if exchange == "p2p":
             self._bufs = (native.SharedBuffer(pad), native.SharedBuffer(pad))
             self.param_pad, self.grad_pad = self._bufs[0].tensor, self._bufs[1].tensor
@@ -161,6 +195,51 @@ class DataParallelTrainStep(TrainStep):
         self._flag = torch.zeros(1, dtype=torch.float32, device=dev)
         self._nccl = on and dist.get_backend(group) == "nccl"
 
+    def _init_views(self, model, on):
+        """Shared parameter buffer, this context's view buffers shared with the other
+        ranks, and the views / copies of every rank."""
+        self._bufs = (native.SharedBuffer(self.total),)
+        self.param_pad = self._bufs[0].tensor
+        self.param_pad.copy_(model.flat)
+        model.attach_storage(self.param_pad, model.grad_flat, owner=self)
+        self.g_lo, self.g_hi = gaussian_bounds(model.n_pad, self.world, self.rank)
+        my_view = self.ctx.view()
+        fields = native.GsView.FIELDS
+        views = [None] * self.world
+        views[self.rank] = my_view
+        self.copies = []
+        if self.world > 1:
+            mine = (self._bufs[0].handle, [native.shared_handle(getattr(my_view, f)) for f in fields])
+            handles = [None] * self.world
+            dist.all_gather_object(handles, mine, group=self.group)
+            for r, (hp, hv) in enumerate(handles):
+                if r == self.rank:
+                    continue
+                ptrs = [native.shared_open(h) for h in hv]
+                self._peer_maps.extend(ptrs)
+                views[r] = native.GsView(*ptrs)
+                base = native.shared_open(hp)
+                self._peer_maps.append(base)
+                self.copies.append(native.GsGrads(*[base + 4 * model.slices[k].start for k in GROUP_NAMES]))
+        self.views = views
+        self._flag = torch.zeros(1, dtype=torch.float32, device=model.flat.device)
+        self._nccl = on and dist.get_backend(self.group) == "nccl"
+
+    def backward_and_update(self, cs, T, nc, dimg):
+        """The "views" exchange: this rank's blend backward, then the update of its
+        Gaussians from every rank's view (the other exchanges: TrainStep's path)."""
+        if self.exchange != "views":
+            return super().backward_and_update(cs, T, nc, dimg)
+        m = self.model
+        m.step_count += 1
+        self.ctx.render_backward_screen(m.params_struct(), cs, T, nc, dimg)
+        self._barrier()  # every rank's view is complete
+        em, ev = m.moments_structs()
+        self.ctx.adam_step_views(m.params_struct(), self.views, self.g_lo, self.g_hi, self.copies, em, ev,
+                                 [self.lrs[k] for k in GROUP_NAMES], m.step_count, beta1=self.betas[0],
+                                 beta2=self.betas[1], eps=self.eps)
+        self._barrier()  # every rank's copies have landed
+
     def _barrier(self):
         """Every rank's work enqueued so far is complete before anything enqueued after
         it runs: a one-float all-reduce on the stream (NCCL), or a device
@@ -175,6 +254,8 @@ class DataParallelTrainStep(TrainStep):
 
     @property
     def adam_launches(self):
+        if self.exchange == "views":
+            return 1
         lo, hi = shard_bounds(self.total, self.world, self.rank)
         return len(group_pieces(self.model.slices, lo, min(hi, self.total)))
 
@@ -205,8 +286,12 @@ class DataParallelTrainStep(TrainStep):
         """The model's training state with the Adam moments of every rank's shard
         gathered (collective: every rank calls it; every rank gets the full state)."""
         m = self.model
-        mf = gather_shards(m.m_flat, self.total, self.world, self.rank, self.group)
-        vf = gather_shards(m.v_flat, self.total, self.world, self.rank, self.group)
+        if self.exchange == "views":
+            mf = gather_gaussian_shards(m.m_flat, m.n_pad, self.world, self.rank, self.group)
+            vf = gather_gaussian_shards(m.v_flat, m.n_pad, self.world, self.rank, self.group)
+        else:
+            mf = gather_shards(m.m_flat, self.total, self.world, self.rank, self.group)
+            vf = gather_shards(m.v_flat, self.total, self.world, self.rank, self.group)
         return m.state_dict(m_flat=mf, v_flat=vf)
 
     def load_state_dict(self, state: dict):

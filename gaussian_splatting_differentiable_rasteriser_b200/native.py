@@ -27,14 +27,16 @@ EXPORTED = ("gs_create", "gs_destroy", "gs_last_error", "gs_preprocess", "gs_ren
             "gs_debug_screen_grads", "gs_set_option", "gs_loss_l1_dssim_noalloc",
             "gs_set_densify_stats", "gs_densify", "gs_opacity_reset", "gs_loss_charbonnier",
             "gs_adam_step_reduce", "gs_shared_alloc", "gs_shared_open", "gs_shared_close",
-            "gs_shared_free", "gs_set_camera_grad", "gs_relocate")
+            "gs_shared_free", "gs_set_camera_grad", "gs_relocate", "gs_render_backward_screen",
+            "gs_get_view", "gs_shared_handle", "gs_adam_step_views")
 GS_SHARED_HANDLE_BYTES = 64
 MAX_RANKS = 8
 GS_OPTION_OPACITY_RECT = 1
 GS_OPTION_DETERMINISTIC = 2
 GS_OPTION_MIP_COMPENSATION = 3
 STAGES = ("preprocess", "scan", "duplicate", "sort", "ranges", "blend_forward", "loss",
-          "blend_backward", "preprocess_backward", "backward_adam", "depth_sort", "camera_backward")
+          "blend_backward", "preprocess_backward", "backward_adam", "depth_sort", "camera_backward",
+          "views_adam")
 GROUPS = ("means", "log_scales", "quats", "opacity_logits", "sh")
 
 
@@ -64,6 +66,14 @@ class GsGrads(ctypes.Structure):
     _fields_ = [("means", ctypes.c_void_p), ("log_scales", ctypes.c_void_p),
                 ("quats", ctypes.c_void_p), ("opacity_logits", ctypes.c_void_p),
                 ("sh", ctypes.c_void_p)]
+
+
+class GsView(ctypes.Structure):
+    """One rank's view (gs_view): device addresses of its screen records, raw
+    screen sums, touched counts, clamp flags and camera record."""
+    _fields_ = [("screen", ctypes.c_void_p), ("sums", ctypes.c_void_p), ("touched", ctypes.c_void_p),
+                ("clamped", ctypes.c_void_p), ("camera", ctypes.c_void_p)]
+    FIELDS = ("screen", "sums", "touched", "clamped", "camera")
 
 
 _lib = None
@@ -107,6 +117,12 @@ def load(path: str = LIB_PATH):
     L.gs_set_camera_grad.argtypes = [P, P]
     L.gs_relocate.argtypes = [P, ctypes.POINTER(GsGrads), ctypes.POINTER(GsGrads), ctypes.POINTER(GsGrads),
                               I64, I64, I32, P, I64, F, F, ctypes.POINTER(I64), P]
+    L.gs_render_backward_screen.argtypes = [P, ctypes.POINTER(GsParams), ctypes.POINTER(GsCamera), P, P, P, P]
+    L.gs_get_view.argtypes = [P, ctypes.POINTER(GsView)]
+    L.gs_shared_handle.argtypes = [P, ctypes.c_char_p]
+    L.gs_adam_step_views.argtypes = [P, ctypes.POINTER(GsParams), ctypes.POINTER(GsView), I32, I64, I64,
+                                     ctypes.POINTER(GsGrads), I32, ctypes.POINTER(GsGrads), ctypes.POINTER(GsGrads),
+                                     ctypes.POINTER(F), F, F, F, F, I32, P]
     L.gs_set_option.argtypes = [P, I32, I32]
     L.gs_set_option.restype = ctypes.c_int
     L.gs_loss_l1_dssim_noalloc.argtypes = [P, P, I32, I32, F, P, P, P]
@@ -185,6 +201,34 @@ class Context:
         b = (ctypes.c_float * 3)(*[float(x) for x in bias])
         self._check(self.L.gs_loss_charbonnier(self.h, _ptr(image), _ptr(target), H, W, g, b, float(delta),
                                                _ptr(out), _ptr(dloss_dimage), _stream(stream)))
+
+    def render_backward_screen(self, params: GsParams, cam: GsCamera, final_T, n_contrib, dloss_dimage,
+                               stream=None):
+        """The blend backward alone; the raw screen sums stay in the context as its view."""
+        self._check(self.L.gs_render_backward_screen(self.h, ctypes.byref(params), ctypes.byref(cam),
+                                                     _ptr(final_T), _ptr(n_contrib), _ptr(dloss_dimage),
+                                                     _stream(stream)))
+
+    def view(self) -> GsView:
+        """This context's view buffers (device addresses)."""
+        v = GsView()
+        self._check(self.L.gs_get_view(self.h, ctypes.byref(v)))
+        return v
+
+    def adam_step_views(self, params: GsParams, views, g_lo, g_hi, copies, exp_avg: GsGrads, exp_avg_sq: GsGrads,
+                        lrs, step, grad_scale=None, beta1=0.9, beta2=0.999, eps=1e-8, stream=None):
+        """gs_adam_step_views: views = [GsView] in rank order, copies = [GsGrads] of the
+        other ranks' parameter groups; grad_scale defaults to 1 / len(views)."""
+        if not 1 <= len(views) <= MAX_RANKS or len(copies) > MAX_RANKS:
+            raise ValueError(f"1..{MAX_RANKS} views and at most {MAX_RANKS} copies")
+        va = (GsView * len(views))(*views)
+        ca = (GsGrads * max(1, len(copies)))(*copies) if copies else None
+        lr = (ctypes.c_float * 5)(*[float(x) for x in lrs])
+        scale = 1.0 / len(views) if grad_scale is None else float(grad_scale)
+        self._check(self.L.gs_adam_step_views(self.h, ctypes.byref(params), va, len(views), int(g_lo), int(g_hi),
+                                              ca, len(copies), ctypes.byref(exp_avg), ctypes.byref(exp_avg_sq),
+                                              lr, scale, float(beta1), float(beta2), float(eps), int(step),
+                                              _stream(stream)))
 
     def set_camera_grad(self, out):
         """Every later backward writes this view's pose gradient (dL/dw, dL/dt) to
@@ -340,6 +384,16 @@ def shared_open(handle: bytes) -> int:
     if st != GS_OK:
         raise GsError(st, "gs_shared_open failed")
     return int(p.value)
+
+
+def shared_handle(ptr: int) -> bytes:
+    """The IPC handle of the device allocation starting at ptr (for shared_open on
+    another rank)."""
+    h = ctypes.create_string_buffer(GS_SHARED_HANDLE_BYTES)
+    st = load().gs_shared_handle(ctypes.c_void_p(int(ptr)), h)
+    if st != GS_OK:
+        raise GsError(st, "gs_shared_handle failed")
+    return bytes(h.raw)
 
 
 def shared_close(ptr: int):

@@ -299,6 +299,71 @@ gs_status gs_adam_step_reduce(float *param, float *m, float *v, int64_t count, f
                               int32_t zero_grads, float grad_scale, float lr, float beta1, float beta2,
                               float eps, int32_t step, void *stream);
 
+/* ------------------------------------- data-parallel update from views --
+ * The alternative to exchanging parameter gradients: each rank runs only the
+ * blend backward of its camera, and the rank that owns a range of Gaussians
+ * reads every rank's view of them (about 100 B per Gaussian and view instead
+ * of a 236 B gradient), runs the projection backward of every view, averages
+ * and applies Adam in one pass ([GS] section "Per step": one photo per step;
+ * with one photo per rank the batch gradient is the mean of the ranks'
+ * gradients). */
+
+/* One rank's view of the Gaussians after gs_render_backward_screen: DEVICE
+ * pointers (this GPU's, or a peer's opened with gs_shared_open) to its
+ * per-Gaussian screen records, raw screen-gradient sums, touched counts, clamp
+ * flags and its camera record. Each is the start of a device allocation of
+ * the context, so gs_shared_handle can make an IPC handle for it. */
+typedef struct {
+  const void *screen;
+  const float *sums;
+  const uint32_t *touched;
+  const uint8_t *clamped;
+  const void *camera;
+} gs_view;
+
+/* The blend backward of the last forward alone (step 4 up to the raw screen
+ * sums; [GS] "The clever bit: a single backward sweep through the blend"):
+ * the sums, the screen records, the flags and the camera stay in the context
+ * as its view, for gs_adam_step_views on this or other ranks. Arguments and
+ * errors as gs_render_backward. Density statistics are not accumulated. */
+gs_status gs_render_backward_screen(gs_ctx *ctx, const gs_params *params, const gs_camera *cam,
+                                    const float *final_T, const int32_t *n_contrib,
+                                    const float *dloss_dimage, void *stream);
+
+/* The context's view buffers (valid for the whole life of the context; their
+ * contents are those of the last gs_render_backward_screen). */
+gs_status gs_get_view(const gs_ctx *ctx, gs_view *out);
+
+/* The IPC handle (GS_SHARED_HANDLE_BYTES bytes, written to the HOST array
+ * `handle`) of a device allocation that starts at ptr, for gs_shared_open on
+ * another rank. GS_ERR_CUDA if ptr is not the start of a device allocation. */
+gs_status gs_shared_handle(const void *ptr, unsigned char *handle);
+
+/* Steps 4 (projection part) + 5 for the Gaussians [g_lo, g_hi) of this rank,
+ * over n_views ranks' views (1..8, in rank order): per Gaussian, the
+ * projection backward of every view that touched it, summed in rank order and
+ * multiplied by grad_scale (1 / ranks for the batch mean), then the Adam step
+ * of each scalar with its group's learning rate (lr: HOST array of 5, group
+ * order means, log_scales, quats, opacity_logits, sh). The parameters in
+ * *params are updated IN PLACE and also written into each of the n_copies
+ * (0..8) other ranks' parameter buffers (group pointers, usually peer memory;
+ * plain stores, no multicast). The result equals gs_render_backward on each
+ * view, gradients summed in rank order, then gs_adam_step_reduce with the same
+ * grad_scale, up to float32 rounding (the same operations in another kernel),
+ * and every rank's parameters end bit-identical. Only this rank's moments of
+ * [g_lo, g_hi) are read and written. g_lo and g_hi are multiples of 4 within
+ * [0, n_pad]; parameters, moments and copies 16-byte aligned; every view's
+ * parameters must equal these (the ranks hold replicas). The caller orders the
+ * call after every rank's gs_render_backward_screen and every rank's next
+ * forward after every rank's call (stream-ordered barriers); the kernel waits
+ * on nothing. Errors: GS_ERR_INVALID_ARG for NULL or misaligned pointers,
+ * counts or ranges out of bounds, step < 1, bad betas or non-finite lr /
+ * grad_scale; GS_ERR_CUDA if the launch fails. */
+gs_status gs_adam_step_views(gs_ctx *ctx, const gs_params *params, const gs_view *views, int32_t n_views,
+                             int64_t g_lo, int64_t g_hi, const gs_grads *copies, int32_t n_copies,
+                             gs_grads *exp_avg, gs_grads *exp_avg_sq, const float *lr, float grad_scale,
+                             float beta1, float beta2, float eps, int32_t step, void *stream);
+
 /* Device memory that other processes on the node can map (CUDA IPC): the
  * buffers whose shards gs_adam_step_reduce reads and writes on peers.
  * gs_shared_alloc allocates `bytes` on the current device, zero-filled, and
@@ -344,7 +409,8 @@ typedef enum {
   GS_STAGE_BACKWARD_ADAM = 9, /* the fused projection backward + Adam pass */
   GS_STAGE_DEPTH_SORT = 10,   /* compaction + depth sort of the visible Gaussians */
   GS_STAGE_CAMERA_BACKWARD = 11, /* camera-pose gradient (when gs_set_camera_grad is on) */
-  GS_NUM_STAGES = 12
+  GS_STAGE_VIEWS_ADAM = 12,      /* data-parallel update from the views' screen sums */
+  GS_NUM_STAGES = 13
 } gs_stage;
 
 gs_status gs_profile_enable(gs_ctx *ctx, int32_t enabled);

@@ -237,3 +237,49 @@ def test_an_owned_model_refuses_a_size_change_and_bad_states():
     with pytest.raises(ValueError):
         small.load_state_dict(bad)
     assert torch.equal(owned.flat, small.flat)
+
+
+def _rank_gaussian_gather(rank, world, port, out_dir):
+    os.environ.update(RANK=str(rank), WORLD_SIZE=str(world), MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    from gaussian_splatting_differentiable_rasteriser_b200 import data_parallel as dp
+    dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+    n_pad, planes = 1004, 7
+    truth = torch.randn(planes * n_pad, generator=torch.Generator().manual_seed(5))
+    lo, hi = dp.gaussian_bounds(n_pad, world, rank)
+    col = torch.arange(truth.numel()) % n_pad
+    mine = torch.where((col >= lo) & (col < hi), truth, torch.full_like(truth, 1e9 + rank))
+    full = dp.gather_gaussian_shards(mine, n_pad, world, rank)
+    torch.save(full, os.path.join(out_dir, f"g{rank}.pt"))
+    if rank == 0:
+        torch.save(truth, os.path.join(out_dir, "truth.pt"))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_gaussian_ranges_cover_every_gaussian_once_and_gather_exactly(tmp_path):
+    """The "views" exchange owns whole Gaussians: every rank's range is a multiple of
+    4 columns, the ranges tile [0, n_pad) once, and gathering each rank's own
+    columns of every plane gives back the full buffer bit for bit (gloo, 2 and 3
+    ranks)."""
+    import torch
+    import torch.multiprocessing as mp
+    sys.path.insert(0, ROOT)
+    from gaussian_splatting_differentiable_rasteriser_b200 import data_parallel as dp
+    for n_pad in (4, 1004, 3_000_000):
+        for world in (1, 2, 3, 8):
+            b = [dp.gaussian_bounds(n_pad, world, r) for r in range(world)]
+            assert b[0][0] == 0 and b[-1][1] == n_pad
+            assert all(b[r][1] == b[r + 1][0] for r in range(world - 1))
+            assert all(lo % 4 == 0 and hi % 4 == 0 and lo <= hi for lo, hi in b)
+    for world in (2, 3):
+        mp.start_processes(_rank_gaussian_gather, args=(world, free_port(), str(tmp_path)), nprocs=world,
+                           join=True, start_method="spawn")
+        truth = torch.load(tmp_path / "truth.pt")
+        for r in range(world):
+            assert torch.equal(torch.load(tmp_path / f"g{r}.pt"), truth)

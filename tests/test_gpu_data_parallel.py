@@ -6,11 +6,14 @@
   identical, equal bit for bit to Adam on the float32 rank-ordered mean
   gradient, and within float32 rounding of the float64 oracle's Adam.
 * One source with zeroing is gs_adam_step, bit for bit.
-* The whole DataParallelTrainStep with a one-rank NCCL group, for both
-  exchanges, and with two processes on one GPU over gloo (the p2p exchange
-  reading and writing the other process's memory through CUDA IPC): with the
-  fixed-point (order-independent) gradient sums the parameters are bitwise
-  those of a single-GPU step on the mean gradient of the ranks' cameras.
+* The whole DataParallelTrainStep with a one-rank NCCL group, for the three
+  exchanges, and with two processes on one GPU over gloo (the exchange reading
+  and writing the other process's memory through CUDA IPC): with the
+  fixed-point (order-independent) gradient sums the parameters are those of a
+  single-GPU step on the mean gradient of the ranks' cameras - bitwise for the
+  gradient exchanges, to float32 rounding for the views exchange (whose
+  replicas are bitwise equal among themselves).
+* The views exchange with 1-3 emulated ranks on one GPU.
 """
 import datetime
 import os
@@ -44,6 +47,18 @@ def native():
     assert torch.cuda.is_available(), "GPU tests need a CUDA device"
     nat.load()
     return nat
+
+
+def assert_close_params(a, b, frac=0.999):
+    """Two parameter (or moment) buffers from the same operations in different
+    kernels: nearly every scalar within float32 rounding; none off by more than
+    the size of a few Adam steps (an Adam step normalises the gradient, so a
+    gradient within rounding of zero may step either way)."""
+    a = a.detach().cpu().numpy().astype(np.float64)
+    b = b.detach().cpu().numpy().astype(np.float64)
+    close = np.abs(a - b) <= 1e-6 + 1e-6 * np.abs(b)
+    assert close.mean() >= frac, close.mean()
+    assert np.abs(a - b).max() <= 1e-2 + 1e-5 * np.abs(b).max()
 
 
 def test_one_source_with_zeroing_is_adam_step(native):
@@ -134,7 +149,7 @@ def test_emulated_ranks_reduce_adam_allgather(native, world, count, aligned):
         np.testing.assert_allclose(m_all[s], om, rtol=1e-5, atol=1e-9)
 
 
-@pytest.mark.parametrize("exchange", ["p2p", "nccl"])
+@pytest.mark.parametrize("exchange", ["views", "p2p", "nccl"])
 def test_one_rank_nccl_step_equals_the_single_gpu_step(native, exchange):
     import torch.distributed as dist
 
@@ -151,21 +166,28 @@ def test_one_rank_nccl_step_equals_the_single_gpu_step(native, exchange):
         cap = 1 << 20
         a = DataParallelTrainStep(ma, cap, cam.width, cam.height, deterministic=True, exchange=exchange)
         b = model.TrainStep(mb, cap, cam.width, cam.height, fused_adam=False, deterministic=True)
-        assert a.world == 1 and a.adam_launches == len(scenes.GROUP_NAMES)
+        assert a.world == 1 and a.adam_launches == (1 if exchange == "views" else len(scenes.GROUP_NAMES))
         for _ in range(3):
             la, lb = a(cam, target), b(cam, target)
         torch.cuda.synchronize()
-        np.testing.assert_array_equal(la.cpu().numpy(), lb.cpu().numpy())
-        assert torch.equal(ma.flat, mb.flat) and torch.equal(ma.m_flat, mb.m_flat)
-        assert torch.equal(ma.v_flat, mb.v_flat)
-        assert not a.grad_pad.any() and not a.param_pad[ma.flat.numel():].any()
+        if exchange == "views":
+            # the same operations in another kernel: equal up to float32 rounding
+            np.testing.assert_allclose(la.cpu().numpy(), lb.cpu().numpy(), rtol=1e-9, atol=1e-12)
+            assert_close_params(ma.flat, mb.flat)
+            assert_close_params(ma.m_flat, mb.m_flat)
+        else:
+            np.testing.assert_array_equal(la.cpu().numpy(), lb.cpu().numpy())
+            assert torch.equal(ma.flat, mb.flat) and torch.equal(ma.m_flat, mb.m_flat)
+            assert torch.equal(ma.v_flat, mb.v_flat)
+        if exchange != "views":
+            assert not a.grad_pad.any() and not a.param_pad[ma.flat.numel():].any()
         assert not torch.equal(ma.flat, model.GaussianModel(scene).flat)  # the step moved them
         a.close()
     finally:
         dist.destroy_process_group()
 
 
-def _rank(rank, world, port, out_dir, steps):
+def _rank(rank, world, port, out_dir, steps, exchange="p2p"):
     os.environ.update(RANK=str(rank), WORLD_SIZE=str(world), MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     sys.path.insert(0, ROOT)
     import torch.distributed as dist
@@ -181,8 +203,8 @@ def _rank(rank, world, port, out_dir, steps):
             for a in (0.0, 0.4)]
     targets = [torch.from_numpy(scenes.uniform_image(256, 256, seed=10 + r)).cuda() for r in range(world)]
     m = model.GaussianModel(scene)
-    s = DataParallelTrainStep(m, 1 << 20, 256, 256, deterministic=True, exchange="p2p")
-    assert len(s._peer_maps) == 2 * (world - 1)
+    s = DataParallelTrainStep(m, 1 << 20, 256, 256, deterministic=True, exchange=exchange)
+    assert len(s._peer_maps) == (2 if exchange == "p2p" else 6) * (world - 1)
     for _ in range(steps):
         s(cams[rank], targets[rank])
     torch.cuda.synchronize()
@@ -214,18 +236,118 @@ def _rank(rank, world, port, out_dir, steps):
     dist.destroy_process_group()
 
 
-def test_two_processes_on_one_gpu_p2p_exchange(native, tmp_path):
+@pytest.mark.parametrize("exchange", ["p2p", "views"])
+def test_two_processes_on_one_gpu_exchange(native, tmp_path, exchange):
+    """Two processes on one GPU over gloo, each mapping the other's buffers through
+    CUDA IPC: p2p reads the other's gradient and writes its parameters; views reads
+    the other's screen sums, flags and camera and writes its parameters."""
     import torch.multiprocessing as mp
 
     from gaussian_splatting_differentiable_rasteriser_b200 import data_parallel as dp
     world, steps = 2, 2
-    mp.start_processes(_rank, args=(world, free_port(), str(tmp_path), steps), nprocs=world, join=True,
+    mp.start_processes(_rank, args=(world, free_port(), str(tmp_path), steps, exchange), nprocs=world, join=True,
                        start_method="spawn")
     p0, p1, ref = (np.load(tmp_path / f) for f in ("p0.npy", "p1.npy", "ref_p.npy"))
-    np.testing.assert_array_equal(p0, p1)
-    np.testing.assert_array_equal(p0, ref)
+    np.testing.assert_array_equal(p0, p1)  # the replicas are the same bits
     ref_m = np.load(tmp_path / "ref_m.npy")
     total = ref_m.size
+    if exchange == "p2p":
+        np.testing.assert_array_equal(p0, ref)
+    else:
+        assert_close_params(torch.from_numpy(p0), torch.from_numpy(ref))
     for r in range(world):
-        lo, hi = dp.shard_bounds(total, world, r)
-        np.testing.assert_array_equal(np.load(tmp_path / f"m{r}.npy")[lo:hi], ref_m[lo:hi])
+        if exchange == "p2p":
+            lo, hi = dp.shard_bounds(total, world, r)
+            np.testing.assert_array_equal(np.load(tmp_path / f"m{r}.npy")[lo:hi], ref_m[lo:hi])
+        else:  # each rank holds the moments of its own Gaussians in every plane
+            n_pad = scenes.small().n_pad
+            lo, hi = dp.gaussian_bounds(n_pad, world, r)
+            col = np.arange(total) % n_pad
+            own = (col >= lo) & (col < hi)
+            assert_close_params(torch.from_numpy(np.load(tmp_path / f"m{r}.npy")[own]), torch.from_numpy(ref_m[own]))
+
+
+@pytest.mark.parametrize("world", [1, 2, 3])
+def test_views_exchange_emulated_ranks_equal_the_gradient_exchange(native, world):
+    """Each emulated rank (a context and a parameter replica on this GPU) renders its
+    own camera and runs only the blend backward; then every rank's
+    gs_adam_step_views updates its Gaussians from all the views and writes them
+    into every replica (the launches wait on nothing, so this is the multi-rank
+    data path run in order). With fixed-point (order-independent) screen sums the
+    replicas end with the same bits, equal up to float32 rounding to the gradient
+    exchange (each view's full gradient, summed in rank order, times 1 / ranks,
+    then Adam) and within float32 rounding of the float64 oracle's Adam on the
+    mean gradient."""
+    from gaussian_splatting_differentiable_rasteriser_b200 import data_parallel as dp
+    from gaussian_splatting_differentiable_rasteriser_b200 import model
+    scene = scenes.small()
+    cams = [scenes.look_at((3.0 * np.sin(a), 0.3 * a, -3.0 * np.cos(a)), (0.0, 0.0, 0.0), 256, 256, 256.0)
+            for a in (0.0, 0.5, -0.7)][:world]
+    targets = [scenes.uniform_image(256, 256, seed=30 + r) for r in range(world)]
+    lrs = [1.6e-4, 5e-3, 1e-3, 5e-2, 2.5e-3]
+    step = 3
+    g = torch.Generator().manual_seed(7)
+    reps, ctxs, dimgs = [], [], []
+    for r in range(world):
+        m = model.GaussianModel(scene)
+        if r == 0:
+            m0 = (torch.randn(m.m_flat.numel(), generator=g) * 1e-3).cuda()
+            v0 = (torch.rand(m.v_flat.numel(), generator=g) * 1e-6).cuda()
+        m.m_flat.copy_(m0)
+        m.v_flat.copy_(v0)
+        t = model.TrainStep(m, 1 << 20, 256, 256, fused_adam=False, deterministic=True)
+        cs = native.camera_struct(cams[r])
+        img, T, nc = t.forward(cs, 256, 256)
+        t.compute_loss(img, torch.from_numpy(targets[r]).cuda(), t.dimage)
+        reps.append((m, t, cs, T, nc))
+        dimgs.append(t.dimage.clone())
+    # the gradient exchange's result, on a separate replica
+    ref = model.GaussianModel(scene)
+    ref.m_flat.copy_(m0)
+    ref.v_flat.copy_(v0)
+    gsum = None
+    for r, (m, t, cs, T, nc) in enumerate(reps):
+        m.grad_flat.zero_()
+        t.ctx.render_backward(m.params_struct(), cs, T, nc, dimgs[r], m.grads_struct())
+        gsum = m.grad_flat.clone() if gsum is None else gsum + m.grad_flat
+        m.grad_flat.zero_()
+    ref.grad_flat.copy_(gsum * np.float32(1.0 / world))
+    for k, lr in zip(scenes.GROUP_NAMES, lrs):
+        native.adam_step(ref.params[k], ref.grads[k], ref.m[k], ref.v[k], lr, step)
+    # the views exchange
+    for r, (m, t, cs, T, nc) in enumerate(reps):
+        t.ctx.render_backward_screen(m.params_struct(), cs, T, nc, dimgs[r])
+    views = [t.ctx.view() for (_, t, _, _, _) in reps]
+    for r, (m, t, cs, T, nc) in enumerate(reps):
+        lo, hi = dp.gaussian_bounds(m.n_pad, world, r)
+        copies = [o[0]._struct(o[0].params) for q, o in enumerate(reps) if q != r]
+        em, ev = m.moments_structs()
+        t.ctx.adam_step_views(m.params_struct(), views, lo, hi, copies, em, ev, lrs, step)
+    torch.cuda.synchronize()
+    for m, *_ in reps:
+        assert torch.equal(m.flat, reps[0][0].flat)
+    assert_close_params(reps[0][0].flat, ref.flat)
+    n_pad = ref.n_pad
+    col = torch.arange(ref.m_flat.numel(), device="cuda") % n_pad
+    for r, (m, *_) in enumerate(reps):
+        lo, hi = dp.gaussian_bounds(n_pad, world, r)
+        own = (col >= lo) & (col < hi)
+        assert_close_params(m.m_flat[own], ref.m_flat[own])
+        assert_close_params(m.v_flat[own], ref.v_flat[own])
+    assert not torch.equal(ref.flat, model.GaussianModel(scene).flat)
+    # against the float64 oracle: Adam on the mean of the views' gradients
+    gm = {k: np.zeros(ref.params[k].shape) for k in scenes.GROUP_NAMES}
+    for r in range(world):
+        o = oracle.Oracle(scene, cams[r])
+        gr = o.backward(dimgs[r].cpu().numpy().astype(np.float64))
+        for k in scenes.GROUP_NAMES:
+            gm[k] += gr[k] / world
+    p0 = model.GaussianModel(scene)
+    for k, lr in zip(scenes.GROUP_NAMES, lrs):
+        sl = ref.slices[k]
+        want = oracle.adam(p0.params[k].cpu().numpy(), gm[k], m0[sl].cpu().numpy(), v0[sl].cpu().numpy(), lr,
+                           step)[0].reshape(ref.params[k].shape)
+        got = ref.params[k].cpu().numpy().astype(np.float64)
+        real = (np.arange(got.size) % n_pad < scene.n).reshape(got.shape)
+        assert np.mean(np.abs(got - want)[real] <= 2e-6 + 1e-3 * lr) > 0.999, k
+
