@@ -32,14 +32,13 @@ struct gs_ctx {
   // depth sort of the visible Gaussians
   uint32_t* dkeys[2] = {nullptr, nullptr};
   uint32_t* dvals[2] = {nullptr, nullptr};
-  uint32_t* dup_status = nullptr;
+  uint32_t* dup_offsets = nullptr;
   // tile sort of the entries
   uint32_t* keys[2] = {nullptr, nullptr};
   uint32_t* vals[2] = {nullptr, nullptr};
   uint32_t* hist = nullptr;
   uint32_t* offsets = nullptr;
-  uint32_t* status = nullptr;
-  uint32_t* counters = nullptr;
+  uint32_t* chunk_counts = nullptr;
   uint2* ranges = nullptr;
   uint2* surv = nullptr;           // [8][max_entries]: per-warp survivors of the blend's box test
   uint32_t* surv_count = nullptr;  // [max_tiles][8]
@@ -111,8 +110,8 @@ gs_status fail(gs_ctx* c, gs_status s, const char* fmt, ...) {
 void free_all(gs_ctx* c) {
   void* bufs[] = {c->screen, c->depth, c->rect, c->touched, c->clamped, c->sgrad, c->block_sums,
                   c->visible_prefix, c->depth_range, c->dkeys[0], c->dkeys[1], c->dvals[0],
-                  c->dvals[1], c->dup_status, c->keys[0], c->keys[1], c->vals[0], c->vals[1],
-                  c->hist, c->offsets, c->status, c->counters, c->ranges, c->surv, c->surv_count,
+                  c->dvals[1], c->dup_offsets, c->keys[0], c->keys[1], c->vals[0], c->vals[1],
+                  c->hist, c->offsets, c->chunk_counts, c->ranges, c->surv, c->surv_count,
                   c->sgrad_fixed, c->dens_counts, c->dens_prefix, c->dens_totals, c->charb_partials,
                   c->charb_counter, c->cam_partials, c->cam_counter, c->reloc_dead, c->loss_partials,
                   c->loss_counter, c->info_dev, c->pairs, c->cam_dev};
@@ -172,9 +171,7 @@ gs_status take_device_error(gs_ctx* c) {
   c->info_host->device_error = 0;
   cudaMemset(&c->info_dev->device_error, 0, sizeof(uint32_t));
   return fail(c, GS_ERR_DEVICE, "a kernel recorded a device fault (code 0x%x: %s)", e,
-              (e & gs::kErrLookbackTimeout) ? "sort look-back wait gave up"
-              : (e & gs::kErrCopyTimeout)   ? "parameter copy wait gave up"
-                                            : "index out of range");
+              (e & gs::kErrCopyTimeout) ? "parameter copy wait gave up" : "index out of range");
 }
 
 void prof_harvest(gs_ctx* c) {
@@ -264,7 +261,7 @@ gs_status gs_create(gs_ctx** out, int64_t max_gaussians, int64_t max_entries, in
   c->max_h = max_height;
   c->max_tiles = static_cast<int64_t>((max_width + 15) / 16) * ((max_height + 15) / 16);
   c->max_blocks = (max_gaussians + gs::kGaussBlock - 1) / gs::kGaussBlock;
-  // the depth sort (visible Gaussians) and the tile sort (entries) share the look-back words
+  // the depth sort (visible Gaussians) and the tile sort (entries) share the per-chunk digit counts
   c->max_sort_tiles = (std::max(max_entries, max_gaussians) + gs::kSortTileKeys - 1) / gs::kSortTileKeys;
   c->max_loss_blocks = gs::loss_num_blocks(max_height, max_width);
   const int64_t G = max_gaussians, K = max_entries;
@@ -285,15 +282,14 @@ gs_status gs_create(gs_ctx** out, int64_t max_gaussians, int64_t max_entries, in
   GS_ALLOC(c->dkeys[1], sizeof(uint32_t) * G);
   GS_ALLOC(c->dvals[0], sizeof(uint32_t) * G);
   GS_ALLOC(c->dvals[1], sizeof(uint32_t) * G);
-  GS_ALLOC(c->dup_status, sizeof(uint32_t) * ((G + gs::kDupItems - 1) / gs::kDupItems));
+  GS_ALLOC(c->dup_offsets, sizeof(uint32_t) * ((G + gs::kDupItems - 1) / gs::kDupItems));
   GS_ALLOC(c->keys[0], sizeof(uint32_t) * K);
   GS_ALLOC(c->keys[1], sizeof(uint32_t) * K);
   GS_ALLOC(c->vals[0], sizeof(uint32_t) * K);
   GS_ALLOC(c->vals[1], sizeof(uint32_t) * K);
   GS_ALLOC(c->hist, sizeof(uint32_t) * gs::kMaxPasses * gs::kRadix);
   GS_ALLOC(c->offsets, sizeof(uint32_t) * gs::kMaxPasses * gs::kRadix);
-  GS_ALLOC(c->status, sizeof(uint32_t) * gs::kMaxPasses * gs::kRadix * c->max_sort_tiles);
-  GS_ALLOC(c->counters, sizeof(uint32_t) * (gs::kMaxPasses + 1));  // + the duplicate's ticket
+  GS_ALLOC(c->chunk_counts, sizeof(uint32_t) * gs::kMaxPasses * gs::kRadix * c->max_sort_tiles);
   GS_ALLOC(c->ranges, sizeof(uint2) * c->max_tiles);
   GS_ALLOC(c->surv, sizeof(uint2) * 8 * K);
   GS_ALLOC(c->surv_count, sizeof(uint32_t) * 8 * c->max_tiles);
@@ -438,8 +434,7 @@ gs_status gs_render_forward(gs_ctx* c, const gs_camera* cam, float* image, float
     gs::SortBuffers b;
     b.hist = c->hist;
     b.offsets = c->offsets;
-    b.status = c->status;
-    b.counters = c->counters;
+    b.chunk_counts = c->chunk_counts;
     b.err = &c->info_dev->device_error;
     // 1 + 2. visible Gaussians in index order, sorted by depth key
     const uint32_t dmin = c->info_host->depth_min;
@@ -478,7 +473,7 @@ gs_status gs_render_forward(gs_ctx* c, const gs_camera* cam, float* image, float
     d.max_entries = c->max_k;
     d.keys = c->keys[0];
     d.vals = c->vals[0];
-    d.chunk_offsets = c->dup_status;
+    d.chunk_offsets = c->dup_offsets;
     d.err = &c->info_dev->device_error;
     prof_begin(c, st);
     GS_CUDA(c, gs::launch_duplicate(d, st));
@@ -1146,8 +1141,7 @@ gs_status gs_relocate(gs_ctx* c, const gs_grads* params, const gs_grads* m, cons
   b.vals[1] = c->dvals[1];
   b.hist = c->hist;
   b.offsets = c->offsets;
-  b.status = c->status;
-  b.counters = c->counters;
+  b.chunk_counts = c->chunk_counts;
   b.err = &c->info_dev->device_error;
   gs::SortPlan plan;
   plan.n = donors;

@@ -66,7 +66,6 @@ struct CamArgs {
 // Device-side error word: kernels that give up on a bounded wait or detect an
 // out-of-range index OR a code into it and skip the access.
 enum DeviceError : uint32_t {
-  kErrLookbackTimeout = 1u,
   kErrIndexRange = 2u,
   kErrCopyTimeout = 4u,
 };

@@ -55,7 +55,7 @@ struct SortPlan {
   int64_t n;      // items
   int key_bits;   // significant low bits of the keys
   int passes;     // ceil(key_bits / 8)
-  int64_t tiles;  // onesweep tiles of kSortTileKeys items
+  int64_t tiles;  // chunks of kSortTileKeys keys (one CTA each)
 };
 
 // Radix-pass shape: threads per CTA (a multiple of 256), keys per thread and
@@ -109,7 +109,7 @@ struct DuplicateArgs {
   uint32_t* err;
 };
 #ifndef GS_DUP_PER_THREAD
-#define GS_DUP_PER_THREAD 16
+#define GS_DUP_PER_THREAD 2
 #endif
 constexpr int kDupThreads = 256;
 constexpr int kDupPerThread = GS_DUP_PER_THREAD;  // visible Gaussians per thread of a duplicate CTA
@@ -121,8 +121,7 @@ struct SortBuffers {
   uint32_t* vals[2];
   uint32_t* hist;      // [kMaxPasses][256] digit counts
   uint32_t* offsets;   // [kMaxPasses][256] exclusive digit offsets
-  uint32_t* status;    // [kMaxPasses][tiles][256] look-back words
-  uint32_t* counters;  // [kMaxPasses] tile tickets
+  uint32_t* chunk_counts;  // [kMaxPasses][256][tiles] per-chunk digit counts, then their offsets
   uint32_t* err;
 };
 

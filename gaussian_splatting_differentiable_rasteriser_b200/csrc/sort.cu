@@ -15,7 +15,8 @@
 //   2. sort them by that key (ceil(depth_bits / 8) passes, typically 3, over
 //      the visible Gaussians only - about 2.2x fewer items than entries);
 //   3. duplicate in that depth order: one (tile, index) entry per touched
-//      tile, each CTA's output offset found by a decoupled look-back;
+//      tile; a count kernel sums the tiles of each chunk of Gaussians and a
+//      scan turns the sums into each chunk's output offset;
 //   4. sort the entries by tile (ceil(tile_bits / 8) passes, 2 at 1080p).
 // Every step is stable, so equal depth keys stay in index order and each
 // tile's entries stay in (depth, index) order: the same order as one sort by
@@ -519,7 +520,7 @@ cudaError_t launch_sort(const SortPlan& plan, const SortBuffers& b, int* out_buf
   int cur = 0;
   for (int p = 0; p < plan.passes; ++p) {
     const int digit_bits = std::min(8, plan.key_bits - 8 * p);
-    uint32_t* counts = b.status + static_cast<int64_t>(p) * plan.tiles * kRadix;  // [256][chunks]
+    uint32_t* counts = b.chunk_counts + static_cast<int64_t>(p) * plan.tiles * kRadix;  // [256][chunks]
     uint32_t* hist = b.hist + p * kRadix;
     upsweep_kernel<<<chunks, kSortThreads, 0, st>>>(b.keys[cur], plan.n, 8 * p, plan.tiles, counts, hist);
     scan_digits_kernel<<<1u << digit_bits, kScanThreads, 0, st>>>(counts, plan.tiles, hist);

@@ -171,8 +171,10 @@ def test_one_rank_nccl_step_equals_the_single_gpu_step(native, exchange):
             la, lb = a(cam, target), b(cam, target)
         torch.cuda.synchronize()
         if exchange == "views":
-            # the same operations in another kernel: equal up to float32 rounding
-            np.testing.assert_allclose(la.cpu().numpy(), lb.cpu().numpy(), rtol=1e-9, atol=1e-12)
+            # the same operations in another kernel: the parameters agree up to
+            # float32 rounding after each step, so the losses of the later steps
+            # agree to about that relative precision
+            np.testing.assert_allclose(la.cpu().numpy(), lb.cpu().numpy(), rtol=1e-7, atol=1e-12)
             assert_close_params(ma.flat, mb.flat)
             assert_close_params(ma.m_flat, mb.m_flat)
         else:
