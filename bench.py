@@ -48,15 +48,16 @@ WORKLOADS = {
 
 # ncu DRAM traffic (read + write bytes) of kernels per unit of their work, with the
 # sha256 (first 12 hex digits) of the source file each figure was taken from. A
-# figure whose source has changed since is reported as null. Both were captured with
-# ncu on the Mid workload (500,000 Gaussians, 1,064,000 entries per step) and are
-# scaled to a launch of the benchmarked workload by the units it processes: the
-# Gaussians (n_pad) for the per-Gaussian pass, the (Gaussian, tile) entries for the
-# blend, in which traffic grows in proportion. The fused pass's write counter
-# undercounts: its last writes are still in L2 when the kernel ends.
+# figure whose source has changed since is reported as null. Each was captured with
+# ncu on one launch of a smaller case of the same shape and is scaled to a launch
+# of the benchmarked workload by the units it processes: the Gaussians (n_pad) for
+# the per-Gaussian pass, the (Gaussian, tile) entries for the blend, in which
+# traffic grows in proportion.
 NCU_TRAFFIC = {
-    "backward_adam": ((409.251584e6 + 290.841600e6) / 500_000, "gaussians", "3df92fa0a447"),
-    "blend_backward": ((85.220352e6 + 2.926336e6) / 1.064e6, "entries", "2dcc3feaade8"),
+    # Dense-shaped scene of 1.5M Gaussians, one launch (ncu full set)
+    "backward_adam": ((1.272110e9 + 1.007214e9) / 1_500_000, "gaussians", "54499bdf7842"),
+    # Dense-shaped scene of 1.5M Gaussians (3,185,918 entries), one launch
+    "blend_backward": ((335.123712e6 + 57.220608e6) / 3_185_918, "entries", "5abe19b2dac3"),
 }
 
 
