@@ -39,18 +39,23 @@ namespace {
 
 constexpr int kWarps = 8;
 
-// Warp-private slots of the surviving Gaussians of the current chunk.
+// Warp-private slots of the surviving Gaussians of the current chunk. The
+// centre, the list position and the Gaussian share one 16-byte slot, so a
+// survivor's bookkeeping comes with the load of its centre.
 struct WarpSlots {
-  float2 xy[32];
+  float4 xyp[32];  // u, v, list position relative to the tile start (int bits), Gaussian (uint bits)
   float4 q[32];    // A', B', C', log2(o)
   float4 col[32];  // r, g, b, o
-  int pos[32];     // list position relative to the tile start
-  uint32_t id[32];
 };
 
-// One gathered list entry: the screen record of its Gaussian.
+__device__ __forceinline__ int slot_pos(const float4& xyp) { return __float_as_int(xyp.z); }
+__device__ __forceinline__ uint32_t slot_id(const float4& xyp) { return __float_as_uint(xyp.w); }
+
+// One gathered list entry: its Gaussian and that Gaussian's screen record.
 struct Entry {
-  Screen s;
+  float4 box;  // u, v, hx, hy
+  float4 q;    // A', B', C', log2(o)
+  float4 col;  // r, g, b, o
   uint32_t gid;
   bool valid;
 };
@@ -65,29 +70,27 @@ __device__ __forceinline__ Entry load_entry(const Screen* screen, uint32_t gid, 
   e.gid = gid;
   if (valid) {
     const float4* r = reinterpret_cast<const float4*>(screen + gid);
-    e.s.a = __ldg(r);
-    e.s.b = __ldg(r + 1);
-    e.s.c = __ldg(r + 2);
+    e.box = __ldg(r);
+    e.q = __ldg(r + 1);
+    e.col = __ldg(r + 2);
   } else {
-    e.s.a = e.s.b = e.s.c = make_float4(0.f, 0.f, 0.f, 0.f);
+    e.box = e.q = e.col = make_float4(0.f, 0.f, 0.f, 0.f);
   }
   return e;
 }
 
 // The entry's alpha >= 1/255 box meets the pixel block [bx0, bx0+7] x [by0, by0+3].
 __device__ __forceinline__ bool hits_block(const Entry& e, float bx0, float by0) {
-  const float u = e.s.a.x, v = e.s.a.y, hx = e.s.c.z, hy = e.s.c.w;
+  const float u = e.box.x, v = e.box.y, hx = e.box.z, hy = e.box.w;
   const float cx = fminf(fmaxf(u, bx0), bx0 + 7.0f);
   const float cy = fminf(fmaxf(v, by0), by0 + 3.0f);
   return e.valid && fabsf(u - cx) <= hx && fabsf(v - cy) <= hy;
 }
 
 __device__ __forceinline__ void put_slot(WarpSlots& w, int slot, const Entry& e, int pos) {
-  w.xy[slot] = make_float2(e.s.a.x, e.s.a.y);
-  w.q[slot] = make_float4(e.s.a.z, e.s.a.w, e.s.b.x, e.s.b.y);
-  w.col[slot] = make_float4(e.s.b.z, e.s.b.w, e.s.c.x, e.s.c.y);
-  w.pos[slot] = pos;
-  w.id[slot] = e.gid;
+  w.xyp[slot] = make_float4(e.box.x, e.box.y, __int_as_float(pos), __uint_as_float(e.gid));
+  w.q[slot] = e.q;
+  w.col[slot] = e.col;
 }
 
 // 2^x in one MUFU instruction (flushes results below 2^-126 to 0, far under
@@ -135,7 +138,8 @@ __global__ void __launch_bounds__(256) blend_forward_kernel(BlendArgs a) {
   int last = 0;
   bool done = !inside;
   unsigned blended = 0;
-  // this warp's survivors of the box test, in list order, for the backward
+  // this warp's survivors of the box test that blend at one of its pixels, in
+  // list order, for the backward
   uint2* surv = a.surv + 8LL * beg + static_cast<int64_t>(warp) * (end - beg);
   int nsurv = 0;
 
@@ -150,17 +154,13 @@ __global__ void __launch_bounds__(256) blend_forward_kernel(BlendArgs a) {
     gid_next = load_gid(a.order, base + 64 + lane, beg, end);
     const bool keep = hits_block(cur, bx0, by0);
     const unsigned mask = __ballot_sync(0xffffffffu, keep);
-    if (keep) {
-      const int slot = __popc(mask & lt);
-      put_slot(ws, slot, cur, base + lane - beg);
-      surv[nsurv + slot] = make_uint2(static_cast<uint32_t>(base + lane - beg), cur.gid);
-    }
+    const int slot = __popc(mask & lt);
+    if (keep) put_slot(ws, slot, cur, base + lane - beg);
     __syncwarp();
     const int cnt = __popc(mask);
-    nsurv += cnt;
-    int last_k = -1;  // slot of this chunk's last blended survivor
+    unsigned blent = 0u;  // slots that blended at this pixel
     for (int k = 0; k < cnt; ++k) {
-      const float2 xy = ws.xy[k];
+      const float4 xy = ws.xyp[k];
       const float p = power2(ws.q[k], fx - xy.x, fy - xy.y);
       const float alpha = fminf(kAlphaMax, fast_exp2(p));
       if (!done && alpha >= kAlphaMin) {
@@ -171,11 +171,19 @@ __global__ void __launch_bounds__(256) blend_forward_kernel(BlendArgs a) {
         C1 = __fmaf_rn(w, c.y, C1);
         C2 = __fmaf_rn(w, c.z, C2);
         T = T * (1.0f - alpha);
-        last_k = k;
+        blent |= 1u << k;
         done = T < kTMin;
       }
     }
-    if (last_k >= 0) last = ws.pos[last_k] + 1;
+    // The backward needs only the survivors that blended at some pixel of the
+    // warp (about a fifth of the box survivors blend at none on dense scenes).
+    const unsigned used = __reduce_or_sync(0xffffffffu, blent);
+    const bool put = keep && ((used >> slot) & 1u);
+    const unsigned pm = __ballot_sync(0xffffffffu, put);
+    if (put) surv[nsurv + __popc(pm & lt)] = make_uint2(static_cast<uint32_t>(base + lane - beg), cur.gid);
+    nsurv += __popc(pm);
+    // the last contributor so far: this chunk's last blended slot, if any
+    if (blent) last = slot_pos(ws.xyp[31 - __clz(blent)]) + 1;
     __syncwarp();  // the slots are rewritten by the next chunk
   }
   if (lane == 0) a.surv_count[tile * kWarps + warp] = static_cast<uint32_t>(nsurv);
@@ -199,14 +207,13 @@ __global__ void __launch_bounds__(256) blend_forward_kernel(BlendArgs a) {
 
 // Per-warp batch of Gaussians that had a contributing pixel in the backward:
 // per (Gaussian, pixel) the two per-pixel factors the nine raw sums are built
-// from, w = dL/dalpha * o exp(-e) and alpha T, plus each Gaussian's id and
-// centre. Rows are padded to 33 so that a lane per Gaussian reads without bank
-// conflicts.
+// from, w = dL/dalpha * o exp(-e) and alpha T, plus each Gaussian's slot
+// (centre and id). Rows are padded to 33 so that a lane per Gaussian reads
+// without bank conflicts.
 constexpr int kBatch = 16;
 struct WarpBatch {
   float2 wa[kBatch][33];  // (w, alpha T) of Gaussian j at pixel p (lane p)
-  float2 uv[kBatch];      // centre (u, v)
-  uint32_t id[kBatch];
+  float4 xyp[kBatch];     // the Gaussian's slot: centre (u, v), position, id
   float4 g[32];           // dL/d(pixel colour) of the warp's pixels
 };
 
@@ -275,10 +282,10 @@ __device__ __forceinline__ void flush_batch(const WarpBatch& b, int cnt, int lan
   c1 += __shfl_xor_sync(full, c1, 16);
   c2 += __shfl_xor_sync(full, c2, 16);
   if (j < cnt) {
-    const float2 uv = b.uv[j];
+    const float4 uv = b.xyp[j];
     const float a = uv.x - cxb, bb = uv.y - cyb;
-    float* dst = sgrad + static_cast<int64_t>(b.id[j]) * kGradStride;
-    unsigned long long* fdst = kFixed ? sgrad_fixed + static_cast<int64_t>(b.id[j]) * kFixedStride : nullptr;
+    float* dst = sgrad + static_cast<int64_t>(slot_id(uv)) * kGradStride;
+    unsigned long long* fdst = kFixed ? sgrad_fixed + static_cast<int64_t>(slot_id(uv)) * kFixedStride : nullptr;
     if (h == 0) {
       const float sy = __fmaf_rn(-bb, m0, my);
       add_sum<kFixed>(dst, fdst, 0, m0);
@@ -344,10 +351,11 @@ __global__ void __launch_bounds__(256) blend_backward_kernel(BlendArgs a) {
   unsigned blended = 0;
   int bcnt = 0;  // Gaussians in the warp's batch (warp-uniform)
 
-  // The forward stored this warp's survivors of the box test (list position,
-  // Gaussian) in list order; walk them from the last one down. Lane l takes
-  // survivor hi - 1 - l, so ballot order (lane order) is descending list order;
-  // survivors at or past the warp's last contributor are dropped.
+  // The forward stored this warp's survivors of the box test that blend at one
+  // of its pixels (list position, Gaussian) in list order; walk them from the
+  // last one down. Lane l takes survivor hi - 1 - l, so ballot order (lane
+  // order) is descending list order; survivors at or past the warp's last
+  // contributor are dropped.
   const int end = static_cast<int>(range.y);
   const uint2* surv = a.surv + 8LL * beg + static_cast<int64_t>(warp) * (end - beg);
   const int nsurv = min(static_cast<int>(a.surv_count[tile * kWarps + warp]), end - beg);
@@ -369,8 +377,8 @@ __global__ void __launch_bounds__(256) blend_backward_kernel(BlendArgs a) {
     __syncwarp();
     const int cnt = __popc(mask);
     for (int k = 0; k < cnt; ++k) {
-      const int pos = ws.pos[k];
-      const float2 xy = ws.xy[k];
+      const float4 xy = ws.xyp[k];
+      const int pos = slot_pos(xy);
       const float dx = fx - xy.x, dy = fy - xy.y;
       const float raw = fast_exp2(power2(ws.q[k], dx, dy));
       const float alpha = fminf(kAlphaMax, raw);
@@ -389,10 +397,7 @@ __global__ void __launch_bounds__(256) blend_backward_kernel(BlendArgs a) {
         w = raw <= kAlphaMax ? dalpha * raw : 0.0f;  // zero through the cap
       }
       wb.wa[bcnt][lane] = make_float2(w, aT);
-      if (lane == 0) {
-        wb.id[bcnt] = ws.id[k];
-        wb.uv[bcnt] = xy;
-      }
+      if (lane == 0) wb.xyp[bcnt] = xy;
       if (++bcnt == kBatch) {
         __syncwarp();
         flush_batch<kFixed>(wb, kBatch, lane, bx0 + 3.5f, by0 + 1.5f, a.sgrad, a.sgrad_fixed);

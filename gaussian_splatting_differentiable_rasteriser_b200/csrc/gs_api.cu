@@ -224,9 +224,9 @@ __global__ void unpack_preprocess_kernel(const gs::Screen* screen, const float* 
   }
   if (opacity) opacity[i] = gs::screen_opacity(s);
   if (rgb) {
-    rgb[3 * i] = s.b.z;
-    rgb[3 * i + 1] = s.b.w;
-    rgb[3 * i + 2] = s.c.x;
+    rgb[3 * i] = s.c.x;
+    rgb[3 * i + 1] = s.c.y;
+    rgb[3 * i + 2] = s.c.z;
   }
   if (dep) dep[i] = depth[i];
   if (rc) {

@@ -22,10 +22,12 @@ constexpr float kLog2e = 1.4426950408889634f;
 //   p = A' dx^2 + B' dx dy + C' dy^2 + log2(o),
 //   A' = -A log2(e) / 2, B' = -B log2(e), C' = -C log2(e) / 2
 // for the conic (A, B, C) (e = A dx^2 / 2 + B dx dy + C dy^2 / 2).
-//   a = (u, v, A', B')
-//   b = (C', log2(o), r, g)
-//   c = (blue, o, hx, hy)   hx, hy: conservative half-widths of the box holding
-//                           every pixel where o exp(-e) >= 1/255 (negative if none)
+//   a = (u, v, hx, hy)   hx, hy: conservative half-widths of the box holding
+//                        every pixel where o exp(-e) >= 1/255 (negative if none)
+//   b = (A', B', C', log2(o))
+//   c = (r, g, b, o)
+// The box test of the blend needs only a; b and c are gathered for the
+// entries that pass it.
 struct alignas(16) Screen {
   float4 a, b, c;
 };
@@ -33,10 +35,10 @@ struct alignas(16) Screen {
 // Scale between the natural conic entries and the stored exponent form.
 constexpr float kConicToExpAC = -0.5f * 1.4426950408889634f;  // A' = A * this (also C)
 constexpr float kConicToExpB = -1.4426950408889634f;          // B' = B * this
-__device__ __forceinline__ float conic_A(const Screen& s) { return s.a.z / kConicToExpAC; }
-__device__ __forceinline__ float conic_B(const Screen& s) { return s.a.w / kConicToExpB; }
-__device__ __forceinline__ float conic_C(const Screen& s) { return s.b.x / kConicToExpAC; }
-__device__ __forceinline__ float screen_opacity(const Screen& s) { return s.c.y; }
+__device__ __forceinline__ float conic_A(const Screen& s) { return s.b.x / kConicToExpAC; }
+__device__ __forceinline__ float conic_B(const Screen& s) { return s.b.y / kConicToExpB; }
+__device__ __forceinline__ float conic_C(const Screen& s) { return s.b.z / kConicToExpAC; }
+__device__ __forceinline__ float screen_opacity(const Screen& s) { return s.c.w; }
 
 // Raw per-Gaussian screen-gradient sums accumulated by the blend backward
 // (12 floats, 9 used). With w = dL/dalpha * o exp(-e) summed over pixels:

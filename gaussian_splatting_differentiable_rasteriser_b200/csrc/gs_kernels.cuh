@@ -148,9 +148,10 @@ struct BlendArgs {
   // when not null: pairs[0] += (pixel, Gaussian) pairs the method's walk visits,
   // pairs[2] += pairs that blend (alpha >= 1/255 before the walk stops)
   unsigned long long* pairs;
-  // per warp (8 per tile) the entries that pass its box test, written by the
-  // forward and walked by the backward: (list position, Gaussian) in list
-  // order, warp w of a tile with list [beg, end) at surv[8 beg + w (end - beg)]
+  // per warp (8 per tile) the entries that pass its box test and blend at one
+  // of its pixels, written by the forward and walked by the backward: (list
+  // position, Gaussian) in list order, warp w of a tile with list [beg, end) at
+  // surv[8 beg + w (end - beg)]
   uint2* surv;
   uint32_t* surv_count;  // [tiles][8]
   // backward in deterministic mode: the raw sums in fixed point ([n][9], zeroed)

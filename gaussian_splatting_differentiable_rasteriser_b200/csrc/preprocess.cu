@@ -272,9 +272,9 @@ __global__ void __launch_bounds__(kPreThreads, kPreThreads == 256 ? 3 : 6) prepr
             hy = sqrtf(2.0f * E * cc) * 1.001f + 0.02f;
           }
           const float idet = kLog2e / det;
-          s.a = make_float4(static_cast<float>(u), static_cast<float>(v), -0.5f * cc * idet, cb * idet);
-          s.b = make_float4(-0.5f * ca * idet, log2f(opacity), rgb[0], rgb[1]);
-          s.c = make_float4(rgb[2], opacity, hx, hy);
+          s.a = make_float4(static_cast<float>(u), static_cast<float>(v), hx, hy);
+          s.b = make_float4(-0.5f * cc * idet, cb * idet, -0.5f * ca * idet, log2f(opacity));
+          s.c = make_float4(rgb[0], rgb[1], rgb[2], opacity);
         }
       }
     }
@@ -346,12 +346,20 @@ __global__ void __launch_bounds__(1024) scan_blocks_kernel(const uint2* block_su
   const int tid = threadIdx.x;
   const int64_t per = (nb + blockDim.x - 1) / blockDim.x;
   const int64_t lo = tid * per, hi = min(nb, lo + per);
+  // each thread's run is read kRun sums at a time, all loads of a group in
+  // flight together (a thread has about a dozen sums at 3M Gaussians)
+  constexpr int kRun = 8;
   uint64_t entries = 0;
   uint32_t local = 0;
-  for (int64_t k = lo; k < hi; ++k) {
-    const uint2 b = block_sums[k];
-    entries += b.x;
-    local += b.y;
+  for (int64_t k0 = lo; k0 < hi; k0 += kRun) {
+    uint2 b[kRun];
+#pragma unroll
+    for (int u = 0; u < kRun; ++u) b[u] = k0 + u < hi ? block_sums[k0 + u] : make_uint2(0u, 0u);
+#pragma unroll
+    for (int u = 0; u < kRun; ++u) {
+      entries += b[u].x;
+      local += b[u].y;
+    }
   }
   const int lane = tid & 31, warp = tid >> 5;
 #pragma unroll
@@ -383,9 +391,15 @@ __global__ void __launch_bounds__(1024) scan_blocks_kernel(const uint2* block_su
   }
   __syncthreads();
   uint32_t run = v - local + (warp > 0 ? s_vwarp[warp - 1] : 0u);
-  for (int64_t k = lo; k < hi; ++k) {
-    visible_prefix[k] = run;
-    run += block_sums[k].y;
+  for (int64_t k0 = lo; k0 < hi; k0 += kRun) {
+    uint32_t c[kRun];
+#pragma unroll
+    for (int u = 0; u < kRun; ++u) c[u] = k0 + u < hi ? block_sums[k0 + u].y : 0u;
+#pragma unroll
+    for (int u = 0; u < kRun; ++u) {
+      if (k0 + u < hi) visible_prefix[k0 + u] = run;
+      run += c[u];
+    }
   }
   if (tid == 0) {
     info->num_entries = s_warp[0];

@@ -43,25 +43,42 @@ namespace gs {
 namespace {
 
 // ---------------------------------------------------------------- compact --
+// Each CTA compacts kCompactBlocks consecutive preprocess blocks (one Gaussian
+// of each per thread), with all their loads in flight together.
+constexpr int kCompactBlocks = 4;
+
 __global__ void __launch_bounds__(kGaussBlock) compact_kernel(CompactArgs a) {
-  __shared__ uint32_t s_warp[kGaussBlock / 32];
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const bool vis = i < a.n && a.touched[i] != 0u;
+  __shared__ uint32_t s_warp[kCompactBlocks][kGaussBlock / 32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const uint32_t m = __ballot_sync(0xffffffffu, vis);
-  if (lane == 0) s_warp[warp] = __popc(m);
-  __syncthreads();
-  if (!vis) return;
-  uint32_t before = 0;
-  for (int k = 0; k < warp; ++k) before += s_warp[k];
-  const int64_t off = static_cast<int64_t>(a.visible_prefix[blockIdx.x]) + before +
-                      __popc(m & ((1u << lane) - 1u));
-  if (off >= a.max_out) {
-    record_error(a.err, kErrIndexRange);
-    return;
+  const int64_t b0 = static_cast<int64_t>(blockIdx.x) * kCompactBlocks;
+  bool vis[kCompactBlocks];
+  uint32_t key[kCompactBlocks], pre[kCompactBlocks], m[kCompactBlocks];
+#pragma unroll
+  for (int u = 0; u < kCompactBlocks; ++u) {
+    const int64_t i = (b0 + u) * kGaussBlock + threadIdx.x;
+    vis[u] = i < a.n && a.touched[i] != 0u;
+    key[u] = i < a.n ? __float_as_uint(a.depth[i]) - a.depth_min : 0u;
+    pre[u] = (b0 + u) * kGaussBlock < a.n ? a.visible_prefix[b0 + u] : 0u;
   }
-  a.keys[off] = __float_as_uint(a.depth[i]) - a.depth_min;
-  a.vals[off] = static_cast<uint32_t>(i);
+#pragma unroll
+  for (int u = 0; u < kCompactBlocks; ++u) {
+    m[u] = __ballot_sync(0xffffffffu, vis[u]);
+    if (lane == 0) s_warp[u][warp] = __popc(m[u]);
+  }
+  __syncthreads();
+#pragma unroll
+  for (int u = 0; u < kCompactBlocks; ++u) {
+    if (!vis[u]) continue;
+    uint32_t before = 0;
+    for (int k = 0; k < warp; ++k) before += s_warp[u][k];
+    const int64_t off = static_cast<int64_t>(pre[u]) + before + __popc(m[u] & ((1u << lane) - 1u));
+    if (off >= a.max_out) {
+      record_error(a.err, kErrIndexRange);
+      continue;
+    }
+    a.keys[off] = key[u];
+    a.vals[off] = static_cast<uint32_t>((b0 + u) * kGaussBlock + threadIdx.x);
+  }
 }
 
 // -------------------------------------------------------------- duplicate --
@@ -213,20 +230,31 @@ __global__ void __launch_bounds__(kSortThreads) upsweep_kernel(const uint32_t* k
                                                                uint32_t* hist) {
   __shared__ uint32_t s_h[kSortThreads / 32][kRadix];
   const int tid = threadIdx.x, warp = tid >> 5;
+  const int64_t base = static_cast<int64_t>(blockIdx.x) * kSortTileKeys;
+  const bool full = base + kSortTileKeys <= n;
+  // A full chunk's keys are loaded (16 bytes at a time: the chunk starts at a
+  // multiple of kSortTileKeys keys) before the counters are cleared, so the
+  // loads are in flight meanwhile.
+  uint4 q[kSortItems / 4];
+  if (full) {
+#pragma unroll
+    for (int k = 0; k < kSortItems / 4; ++k)
+      q[k] = __ldg(reinterpret_cast<const uint4*>(keys + base + 4 * (static_cast<int64_t>(k) * kSortThreads + tid)));
+  }
   for (int k = tid; k < (kSortThreads / 32) * kRadix; k += kSortThreads) (&s_h[0][0])[k] = 0;
   __syncthreads();
-  const int64_t base = static_cast<int64_t>(blockIdx.x) * kSortTileKeys;
-  // 16-byte loads: the chunk starts at a multiple of 4096 keys
+  if (full) {
 #pragma unroll
-  for (int k = 0; k < kSortItems / 4; ++k) {
-    const int64_t idx = base + 4 * (static_cast<int64_t>(k) * kSortThreads + tid);
-    uint32_t v[4];
-    if (idx + 3 < n) {
-      const uint4 q = __ldg(reinterpret_cast<const uint4*>(keys + idx));
-      v[0] = q.x, v[1] = q.y, v[2] = q.z, v[3] = q.w;
+    for (int k = 0; k < kSortItems / 4; ++k) {
+      atomicAdd(&s_h[warp][(q[k].x >> shift) & 0xffu], 1u);
+      atomicAdd(&s_h[warp][(q[k].y >> shift) & 0xffu], 1u);
+      atomicAdd(&s_h[warp][(q[k].z >> shift) & 0xffu], 1u);
+      atomicAdd(&s_h[warp][(q[k].w >> shift) & 0xffu], 1u);
+    }
+  } else {
 #pragma unroll
-      for (int j = 0; j < 4; ++j) atomicAdd(&s_h[warp][(v[j] >> shift) & 0xffu], 1u);
-    } else {
+    for (int k = 0; k < kSortItems / 4; ++k) {
+      const int64_t idx = base + 4 * (static_cast<int64_t>(k) * kSortThreads + tid);
 #pragma unroll
       for (int j = 0; j < 4; ++j)
         if (idx + j < n) atomicAdd(&s_h[warp][(__ldg(keys + idx + j) >> shift) & 0xffu], 1u);
@@ -254,7 +282,11 @@ __global__ void __launch_bounds__(kScanThreads) scan_digits_kernel(uint32_t* cou
   const int d = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (warp == 0) {
     uint32_t b = 0;
-    for (int k = lane; k < d; k += 32) b += hist[k];
+#pragma unroll
+    for (int u = 0; u < kRadix / 32; ++u) {  // d < kRadix: all loads in flight at once
+      const int k = lane + 32 * u;
+      b += k < d ? hist[k] : 0u;
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) b += __shfl_xor_sync(0xffffffffu, b, o);
     if (lane == 0) s_carry = b;
@@ -496,7 +528,7 @@ __global__ void __launch_bounds__(256) ranges_kernel(const uint32_t* keys, int64
 
 cudaError_t launch_compact(const CompactArgs& a, int64_t num_blocks, cudaStream_t st) {
   if (num_blocks == 0) return cudaSuccess;
-  compact_kernel<<<static_cast<unsigned>(num_blocks), kGaussBlock, 0, st>>>(a);
+  compact_kernel<<<static_cast<unsigned>((num_blocks + kCompactBlocks - 1) / kCompactBlocks), kGaussBlock, 0, st>>>(a);
   return cudaGetLastError();
 }
 

@@ -92,7 +92,7 @@ typedef struct gs_ctx gs_ctx;
 /* Allocates a context for up to max_gaussians Gaussians, max_entries
  * (Gaussian, tile) entries and images up to max_width x max_height. Device
  * memory: about 150 B per Gaussian plus 80 B per entry (sort buffers and the
- * blend's per-warp lists of the entries that reach each 8x4 pixel block).
+ * blend's per-warp lists of the entries that blend in each 8x4 pixel block).
  * The entry budget mirrors the global (blob, tile) budget of [GS] section
  * "Why tiling, and the five stages". The caller owns *ctx and frees it with
  * gs_destroy. Returns GS_ERR_INVALID_ARG for non-positive sizes and
