@@ -307,8 +307,10 @@ struct BackwardSmem {
   WarpBatch batches[kWarps];
 };
 
+// Four CTAs per SM (64 registers) where that needs no spills; the
+// fixed-point variant keeps three.
 template <bool kCount, bool kFixed>
-__global__ void __launch_bounds__(256) blend_backward_kernel(BlendArgs a) {
+__global__ void __launch_bounds__(256, kFixed ? 3 : 4) blend_backward_kernel(BlendArgs a) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   BackwardSmem& sm = *reinterpret_cast<BackwardSmem*>(smem_raw);
   WarpSlots* slots = sm.slots;

@@ -10,9 +10,11 @@
 // B200 notes: the kernel is HBM-bound (236 B of parameters in, 48 + 17 B out
 // per Gaussian at SH degree 3). Each CTA stages its Gaussians' parameter
 // planes in shared memory with bulk asynchronous copies (the untiled TMA
-// path) completed on an mbarrier, then computes from shared memory. The geometry runs in float64 - free next to the memory time - so that
-// the integer decisions taken from it (culling, tile rect, depth key) are
-// stable to ~1e-15 and do not depend on float32 rounding order.
+// path) completed on mbarriers, then computes from shared memory. The
+// camera-space position and depth key are computed in float64 and the
+// covariance chain in float32, redone in float64 where a tile bound lies near
+// a tile boundary, so that the integer decisions taken from them (culling,
+// tile rect, depth key) do not depend on float32 rounding.
 #include "bulk_copy.cuh"
 #include "gs_kernels.cuh"
 #include "sh.cuh"
@@ -20,10 +22,6 @@
 namespace gs {
 
 namespace {
-
-__device__ __forceinline__ double dot3(const double* a, const double* b) {
-  return a[0] * b[0] + a[1] * b[1] + a[2] * b[2];
-}
 
 constexpr int kPreThreads = kGaussBlock;
 
