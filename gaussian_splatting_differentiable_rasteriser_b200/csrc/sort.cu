@@ -82,6 +82,17 @@ __global__ void __launch_bounds__(kGaussBlock) compact_kernel(CompactArgs a) {
 }
 
 // -------------------------------------------------------------- duplicate --
+// floor(n / d) for n < 2^22 and 0 < d: n and d are exact in float32, the
+// fast quotient is within 2 ulp, i.e. within 1 of n / d below 2^22, so the
+// truncated quotient is off by at most one, which one correction step fixes.
+__device__ __forceinline__ uint32_t div_small(uint32_t n, uint32_t d) {
+  uint32_t q = static_cast<uint32_t>(__fdividef(static_cast<float>(n), static_cast<float>(d)));
+  const int32_t r = static_cast<int32_t>(n - q * d);
+  if (r < 0) --q;
+  else if (static_cast<uint32_t>(r) >= d) ++q;
+  return q;
+}
+
 // Tiles touched by each chunk of kDupItems Gaussians in depth order (the
 // duplicate's CTA granularity): one CTA per chunk, one sum per chunk.
 __global__ void __launch_bounds__(kDupThreads) dup_count_kernel(const uint32_t* order, const uint32_t* touched,
@@ -213,7 +224,7 @@ __global__ void __launch_bounds__(kDupThreads) duplicate_kernel(DuplicateArgs a)
       const uint32_t og = __shfl_sync(0xffffffffu, g, owner);
       if (o < group_total) {
         const uint32_t local = o - oe;
-        const uint32_t dy = local / ow;
+        const uint32_t dy = group_total < (1u << 22) ? div_small(local, ow) : local / ow;
         keys[o] = (oy0 + dy) * tiles_x + ox0 + (local - dy * ow);
         vals[o] = og;
       }
