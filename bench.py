@@ -307,7 +307,14 @@ def profile_stages(step, cams, targets, sched, start, count):
     """Per-stage kernel times (library events) plus Adam (torch events: the
     Adam launches are the only work between them on the current stream). For the
     data-parallel step that stage is "exchange_adam": reduce-scatter, Adam on the
-    shard, all-gather."""
+    shard, all-gather.
+
+    The stages are read back after every group of (up to) 5 steps and each
+    stage's time is the median over the groups: a stage's events also span any
+    time the device waits for the host inside it, and a rare host delay (the
+    process descheduled in the middle of a call) would otherwise inflate the
+    mean of one stage. Reading back synchronises, so groups keep that to one
+    step in five."""
     import torch
 
     from gaussian_splatting_differentiable_rasteriser_b200 import native
@@ -315,10 +322,11 @@ def profile_stages(step, cams, targets, sched, start, count):
     ctx = step.ctx
     ctx.profile_enable(True)
     ctx.profile_read()
-    adam_ms = 0.0
-    adam_launches = 0
     m = step.model
     ks = []
+    group = max(1, min(5, count // 5))
+    groups = []
+    adam = []
     # one untimed profiled step first: the counting variants of the blend kernels
     # are launched for the first time there, and a first launch can include the
     # loading of the kernel's code between the stage's events
@@ -341,16 +349,24 @@ def profile_stages(step, cams, targets, sched, start, count):
             e0.record()
             step.update_from_grads()
             e1.record()
-            torch.cuda.synchronize()
             if timed:
-                adam_ms += e0.elapsed_time(e1)
-                adam_launches += step.adam_launches
-        if not timed:
+                adam.append((e0, e1))
+        j = i - start + 1  # timed steps so far
+        if not timed or j % group == 0 or j == count:
             torch.cuda.synchronize()
-            ctx.profile_read()
-    prof = ctx.profile_read()
+            stages = ctx.profile_read()
+            if timed:
+                groups.append((stages, j - sum(n for _, n in groups)))
     ctx.profile_enable(False)
+    prof = {}
+    for name in groups[0][0] if groups else ():
+        d = {k: sum(g[name][k] for g, _ in groups) for k in ("launches", "work", "blended")}
+        # median over the groups of the stage's time per step, times the steps
+        d["ms"] = statistics.median(g[name]["ms"] / n for g, n in groups) * count
+        prof[name] = d
     name = "exchange_adam" if hasattr(step, "param_pad") else "adam"
+    adam_ms = statistics.median(e0.elapsed_time(e1) for e0, e1 in adam) * len(adam) if adam else 0.0
+    adam_launches = len(adam) * step.adam_launches
     prof[name] = {"ms": adam_ms, "launches": adam_launches, "work": adam_launches and count * m.flat.numel()}
     return prof, ks
 

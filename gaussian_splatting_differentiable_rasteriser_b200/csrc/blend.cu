@@ -119,7 +119,7 @@ __device__ __forceinline__ void count_pairs(unsigned long long* pairs, unsigned 
 template <bool kCount>
 __global__ void __launch_bounds__(256) blend_forward_kernel(BlendArgs a) {
   __shared__ WarpSlots slots[kWarps];
-  const int tile = blockIdx.x;
+  const int tile = static_cast<int>(a.tile_order[blockIdx.x]);
   const int tx = tile % a.cam.tiles_x, ty = tile / a.cam.tiles_x;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   WarpSlots& ws = slots[warp];
@@ -315,7 +315,7 @@ __global__ void __launch_bounds__(256, kFixed ? 3 : 4) blend_backward_kernel(Ble
   BackwardSmem& sm = *reinterpret_cast<BackwardSmem*>(smem_raw);
   WarpSlots* slots = sm.slots;
   WarpBatch* batches = sm.batches;
-  const int tile = blockIdx.x;
+  const int tile = static_cast<int>(a.tile_order[blockIdx.x]);
   const int tx = tile % a.cam.tiles_x, ty = tile / a.cam.tiles_x;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   WarpSlots& ws = slots[warp];

@@ -40,6 +40,7 @@ struct gs_ctx {
   uint32_t* offsets = nullptr;
   uint32_t* chunk_counts = nullptr;
   uint2* ranges = nullptr;
+  uint32_t* tile_order = nullptr;  // [max_tiles] tiles by descending list length
   uint2* surv = nullptr;           // [8][max_entries]: per-warp survivors of the blend's box test
   uint32_t* surv_count = nullptr;  // [max_tiles][8]
   // loss
@@ -111,7 +112,7 @@ void free_all(gs_ctx* c) {
   void* bufs[] = {c->screen, c->depth, c->rect, c->touched, c->clamped, c->sgrad, c->block_sums,
                   c->visible_prefix, c->depth_range, c->dkeys[0], c->dkeys[1], c->dvals[0],
                   c->dvals[1], c->dup_offsets, c->keys[0], c->keys[1], c->vals[0], c->vals[1],
-                  c->hist, c->offsets, c->chunk_counts, c->ranges, c->surv, c->surv_count,
+                  c->hist, c->offsets, c->chunk_counts, c->ranges, c->tile_order, c->surv, c->surv_count,
                   c->sgrad_fixed, c->dens_counts, c->dens_prefix, c->dens_totals, c->charb_partials,
                   c->charb_counter, c->cam_partials, c->cam_counter, c->reloc_dead, c->loss_partials,
                   c->loss_counter, c->info_dev, c->pairs, c->cam_dev};
@@ -291,6 +292,7 @@ gs_status gs_create(gs_ctx** out, int64_t max_gaussians, int64_t max_entries, in
   GS_ALLOC(c->offsets, sizeof(uint32_t) * gs::kMaxPasses * gs::kRadix);
   GS_ALLOC(c->chunk_counts, sizeof(uint32_t) * gs::kMaxPasses * gs::kRadix * c->max_sort_tiles);
   GS_ALLOC(c->ranges, sizeof(uint2) * c->max_tiles);
+  GS_ALLOC(c->tile_order, sizeof(uint32_t) * c->max_tiles);
   GS_ALLOC(c->surv, sizeof(uint2) * 8 * K);
   GS_ALLOC(c->surv_count, sizeof(uint32_t) * 8 * c->max_tiles);
   GS_ALLOC(c->dens_counts, sizeof(uint4) * ((G + gs::kDensifyBlock - 1) / gs::kDensifyBlock));
@@ -494,9 +496,11 @@ gs_status gs_render_forward(gs_ctx* c, const gs_camera* cam, float* image, float
   }
   prof_begin(c, st);
   GS_CUDA(c, gs::launch_ranges(c->keys[sorted], static_cast<int64_t>(K), c->ranges, tiles, st));
-  prof_end(c, GS_STAGE_RANGES, static_cast<int64_t>(K), st, K > 0 ? 1 : 0);
+  GS_CUDA(c, gs::launch_tile_order(c->ranges, tiles, c->tile_order, st));
+  prof_end(c, GS_STAGE_RANGES, static_cast<int64_t>(K), st, (K > 0 ? 1 : 0) + 1);
   gs::BlendArgs ba{};
   ba.ranges = c->ranges;
+  ba.tile_order = c->tile_order;
   ba.order = c->vals[sorted];
   ba.screen = c->screen;
   ba.cam = c->cam;
@@ -582,6 +586,7 @@ gs_status backward_common(gs_ctx* c, const gs_params* p, const gs_camera* cam, c
   }
   gs::BlendArgs ba{};
   ba.ranges = c->ranges;
+  ba.tile_order = c->tile_order;
   ba.order = c->vals[c->sorted_buf];
   ba.screen = c->screen;
   ba.cam = c->cam;

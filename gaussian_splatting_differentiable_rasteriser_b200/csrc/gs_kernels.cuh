@@ -131,10 +131,14 @@ cudaError_t launch_sort(const SortPlan& plan, const SortBuffers& b, int* out_buf
 // Per-tile [first, last) of the tile-sorted entries (keys = tile indices).
 cudaError_t launch_ranges(const uint32_t* keys, int64_t n, uint2* ranges, int64_t num_tiles,
                           cudaStream_t st);
+// The tiles in descending order of list length (by powers of two), the order
+// in which the blend kernels take them.
+cudaError_t launch_tile_order(const uint2* ranges, int64_t num_tiles, uint32_t* order, cudaStream_t st);
 
 // ---------------------------------------------------------------- blending
 struct BlendArgs {
   const uint2* ranges;
+  const uint32_t* tile_order;  // CTA b blends tile tile_order[b]
   const uint32_t* order;  // sorted Gaussian index per entry
   const Screen* screen;
   CamArgs cam;

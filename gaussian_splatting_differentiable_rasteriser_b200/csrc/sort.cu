@@ -535,7 +535,72 @@ __global__ void __launch_bounds__(256) ranges_kernel(const uint32_t* keys, int64
   if (i0 + kRangeItems >= n && prev < tiles) ranges[prev].y = static_cast<uint32_t>(n);
 }
 
+// The tiles by descending list length, in buckets of equal bit length (the
+// order inside a bucket is the atomics' order; a tile's result does not
+// depend on when it runs). Taking the longest tiles first keeps a kernel over
+// the tiles from ending on a long tile that started late.
+constexpr int kOrderThreads = 1024;
+__global__ void __launch_bounds__(kOrderThreads) tile_order_kernel(const uint2* ranges, int64_t num_tiles,
+                                                                   uint32_t* order) {
+  __shared__ uint32_t cnt[33];  // by __clz(length): 0 for the longest, 32 for empty tiles
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const unsigned lt = (1u << lane) - 1u;
+  constexpr int kPer = 8;  // tiles per thread and round, loaded together
+  constexpr int kRound = kPer * kOrderThreads;
+  if (tid < 33) cnt[tid] = 0u;
+  // bucket of tile t (33 past the end)
+  auto bucket_of = [&](int64_t t) -> uint32_t {
+    if (t >= num_tiles) return 33u;
+    const uint2 r = ranges[t];
+    return __clz(r.y - r.x);
+  };
+  __syncthreads();
+  // Warp w's tiles of a round are [r + 32 (kPer w + j), + 32), j < kPer: the
+  // lanes of a warp with the same bucket add to it once.
+  for (int64_t r0 = 0; r0 < num_tiles; r0 += kRound) {
+    uint32_t b[kPer];
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) b[j] = bucket_of(r0 + 32 * (kPer * warp + j) + lane);
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const unsigned same = __match_any_sync(0xffffffffu, b[j]);
+      if (b[j] < 33u && (same & lt) == 0u) atomicAdd(&cnt[b[j]], __popc(same));
+    }
+  }
+  __syncthreads();
+  if (tid == 0) {
+    uint32_t run = 0u;
+    for (int k = 0; k < 33; ++k) {
+      const uint32_t c = cnt[k];
+      cnt[k] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
+  for (int64_t r0 = 0; r0 < num_tiles; r0 += kRound) {
+    uint32_t b[kPer];
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) b[j] = bucket_of(r0 + 32 * (kPer * warp + j) + lane);
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const int64_t t = r0 + 32 * (kPer * warp + j) + lane;
+      const unsigned same = __match_any_sync(0xffffffffu, b[j]);
+      const int leader = __ffs(same) - 1;
+      uint32_t base = 0u;
+      if (b[j] < 33u && lane == leader) base = atomicAdd(&cnt[b[j]], __popc(same));
+      base = __shfl_sync(0xffffffffu, base, leader);
+      if (b[j] < 33u) order[base + __popc(same & lt)] = static_cast<uint32_t>(t);
+    }
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_tile_order(const uint2* ranges, int64_t num_tiles, uint32_t* order, cudaStream_t st) {
+  if (num_tiles <= 0) return cudaSuccess;
+  tile_order_kernel<<<1, kOrderThreads, 0, st>>>(ranges, num_tiles, order);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_compact(const CompactArgs& a, int64_t num_blocks, cudaStream_t st) {
   if (num_blocks == 0) return cudaSuccess;
