@@ -8,29 +8,29 @@
 // training" study notes (bailiping.com), slide on alpha (cap 0.99, skip below
 // 1/255, stop when nearly opaque) and slide "r is the RGB loss gradient".
 //
-// B200 design. One CTA of 256 threads per 16x16 tile, one pixel per thread;
-// each warp owns an 8x4 pixel block and walks the tile's list on its own (no
-// CTA-wide barrier: a warp whose pixels are saturated stops while its
-// neighbours go on). The list is consumed 32 entries at a time: lane l gathers
-// entry base + l (its 48-byte screen record, prefetched one chunk ahead into
-// registers), tests the record's alpha >= 1/255 box against the warp's block,
-// and a ballot compacts the survivors into the warp's slice of shared memory.
-// The pixel loop then visits only survivors, so a Gaussian that cannot reach
-// the block costs 1/32 of a warp instruction slot instead of a full
-// evaluation; the box is conservative, so results do not change.
+// B200 design. One CTA of 256 threads per 16x16 tile, one pixel per thread,
+// the tiles taken longest list first; each warp owns an 8x4 pixel block and
+// walks the tile's list on its own (no CTA-wide barrier: a warp whose pixels
+// are saturated stops while its neighbours go on). The list is consumed 32
+// entries at a time: lane l gathers entry base + l (its 48-byte screen record,
+// prefetched one chunk ahead into registers), tests the record's
+// alpha >= 1/255 box against the warp's block, and a ballot compacts the
+// survivors into the warp's slots in shared memory. The pixel loop then
+// visits only survivors, so a Gaussian that cannot reach the block costs 1/32
+// of a warp instruction slot instead of a full evaluation; the box is
+// conservative, so results do not change.
 // Per evaluated pair: alpha = min(0.99, 2^p) with the exponent-ready conic of
 // the screen record (7 FP32 ops and one MUFU.EX2).
-// The forward stores only the final T and n_contrib per pixel; the backward
-// re-walks back to front from each pixel's last contributor, recovers T by
+// The forward stores only the final T and n_contrib per pixel, and for each
+// warp the survivors that blended at one of its pixels. The backward walks
+// those back to front from each pixel's last contributor, recovers T by
 // dividing by (1 - alpha), and keeps one running scalar g . S (S = colour
-// already composited behind) instead of three channels. Per pair it forms 9
-// raw sums (w, w dx, w dy, w dx^2, w dx dy, w dy^2, dL/dc) with
-// w = dL/dalpha * o exp(-e); a warp reduce-scatter (12 shuffles instead of 45)
-// leaves the 9 warp totals in 9 lanes, which issue one coalesced group of 9
-// float32 atomics. When only a few lanes contribute (a quarter of the cases on
-// dense scenes) they add their values directly instead. The conic/opacity/
-// mean2d chain of those sums is applied once per Gaussian in the projection
-// backward.
+// already composited behind) instead of three channels. Per (Gaussian, pixel)
+// it keeps two factors, w = dL/dalpha * o exp(-e) and alpha T, in a per-warp
+// batch in shared memory; every 16 Gaussians two lanes per Gaussian reduce
+// its row into its 9 raw sums (w, w dx, w dy, w dx^2, w dx dy, w dy^2, dL/dc)
+// and add them with float32 atomics. The conic/opacity/mean2d chain
+// of those sums is applied once per Gaussian in the projection backward.
 #include "gs_kernels.cuh"
 
 namespace gs {
