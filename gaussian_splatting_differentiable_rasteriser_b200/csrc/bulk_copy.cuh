@@ -37,6 +37,12 @@ __device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32
       : "memory");
 }
 
+// Starts bringing `bytes` at `src` into L2 (same alignment rules as a copy;
+// nothing to wait for: a later copy of the same bytes finds them in L2).
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // Waits for phase `parity` of `bar` to complete, polling at most `max_polls`
 // times; returns false if it gave up.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int max_polls) {

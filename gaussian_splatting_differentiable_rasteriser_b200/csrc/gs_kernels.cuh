@@ -41,6 +41,7 @@ struct PreprocessArgs {
   uint32_t* err;          // device error word
   int opacity_rect;       // opacity-aware tile rect (GS_OPTION_OPACITY_RECT)
   int mip_comp;           // opacity times the compensation factor (GS_OPTION_MIP_COMPENSATION)
+  int64_t prefetch_ahead; // set by the launcher: CTA b prefetches slice b + this into L2
 };
 
 cudaError_t launch_preprocess(const PreprocessArgs& a, int64_t num_blocks, cudaStream_t st);

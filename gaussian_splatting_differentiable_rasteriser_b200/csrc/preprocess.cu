@@ -141,6 +141,24 @@ __global__ void __launch_bounds__(kPreThreads, kPreThreads == 256 ? 3 : 6) prepr
       for (int k = 0; k < nk; ++k)
         bulk_copy_g2s(sm.plane[kGeomPlanes + ch * nk + k],
                       a.sh + (static_cast<int64_t>(ch) * a.sh_k + k) * np + i0, bytes, &sm.bar[1]);
+    // The CTA that will start about when this one ends (one grid of resident
+    // CTAs later) finds its planes in L2: its copies then wait on L2, not on
+    // DRAM, and this CTA's copies overlap the DRAM reads of the next slices.
+    const int64_t nb = static_cast<int64_t>(blockIdx.x) + a.prefetch_ahead;
+    if (a.prefetch_ahead > 0 && nb < static_cast<int64_t>(gridDim.x)) {
+      const int64_t j0 = nb * kPreThreads;
+      const uint32_t pbytes = static_cast<uint32_t>(np - j0 < kPreThreads ? np - j0 : kPreThreads) * 4u;
+#pragma unroll
+      for (int c = 0; c < 3; ++c) bulk_prefetch_l2(a.means + c * np + j0, pbytes);
+#pragma unroll
+      for (int c = 0; c < 3; ++c) bulk_prefetch_l2(a.log_scales + c * np + j0, pbytes);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) bulk_prefetch_l2(a.quats + c * np + j0, pbytes);
+      bulk_prefetch_l2(a.opacity_logits + j0, pbytes);
+      for (int ch = 0; ch < 3; ++ch)
+        for (int k = 0; k < nk; ++k)
+          bulk_prefetch_l2(a.sh + (static_cast<int64_t>(ch) * a.sh_k + k) * np + j0, pbytes);
+    }
   }
   __syncthreads();  // the barriers are initialised before anyone waits on them
   // Every thread waits for the geometry planes itself (bounded); thread 0
@@ -408,10 +426,18 @@ __global__ void __launch_bounds__(1024) scan_blocks_kernel(const uint2* block_su
 }
 
 template <int kDeg>
-cudaError_t launch_preprocess_deg(const PreprocessArgs& a, unsigned grid, cudaStream_t st) {
+cudaError_t launch_preprocess_deg(const PreprocessArgs& args, unsigned grid, cudaStream_t st) {
   const int smem = static_cast<int>(sizeof(PreprocessSmem<kDeg>));
   cudaError_t e = cudaFuncSetAttribute(preprocess_kernel<kDeg>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
+  // resident CTAs: SMs x CTAs per SM
+  int dev = 0, sms = 0, per_sm = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, preprocess_kernel<kDeg>, kPreThreads, smem);
+  if (e != cudaSuccess) return e;
+  PreprocessArgs a = args;
+  a.prefetch_ahead = static_cast<int64_t>(sms) * per_sm;
   preprocess_kernel<kDeg><<<grid, kPreThreads, smem, st>>>(a);
   return cudaGetLastError();
 }
