@@ -181,9 +181,13 @@ struct LossArgs {
 };
 
 // The loss runs one CTA per channel and strip of kLossCols columns x
-// kLossStrip rows.
+// kLossStrip rows (kLossStrip a multiple of 16; a build-time tunable).
+#ifndef GS_LOSS_STRIP
+#define GS_LOSS_STRIP 128
+#endif
 constexpr int kLossCols = 32;
-constexpr int kLossStrip = 128;
+constexpr int kLossStrip = GS_LOSS_STRIP;
+static_assert(kLossStrip % 16 == 0, "loss strip");
 constexpr int64_t loss_blocks(int height, int width) {
   return 3 * static_cast<int64_t>((width + kLossCols - 1) / kLossCols) *
          ((height + kLossStrip - 1) / kLossStrip);
