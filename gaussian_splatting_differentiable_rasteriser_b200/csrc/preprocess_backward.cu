@@ -101,7 +101,6 @@ struct FusedSmem {
   float geom[kGeomPlanes][kFusedBlock];  // view gradient of the geometric scalars
   float drgb[3][kFusedBlock];            // masked dL/dcolour (0 when invisible)
   float Y[16][kFusedBlock];              // SH basis at the view direction
-  PlaneInfo plane[kStreamMaxPlanes];
 };
 
 // kAccum: the caller's gradient buffer holds an accumulated gradient, which is
@@ -160,7 +159,6 @@ __global__ void __launch_bounds__(kFusedBlock) preprocess_backward_adam_kernel(P
       for (int k = 0; k < 16; ++k) sm.Y[k][t] = 0.f;
     }
   }
-  if (t < planes) sm.plane[t] = plane_info(t, a.sh_k, nk);
   __syncthreads();
 
   // Phase 2: Adam over the CTA's planes; the view gradient adds to the
@@ -173,7 +171,7 @@ __global__ void __launch_bounds__(kFusedBlock) preprocess_backward_adam_kernel(P
     }
     return g;
   };
-  adam_stream<kAccum>(sm.plane, f, np, i0, cols, planes, a.sh_k, nk, stage, grad);
+  adam_stream<kAccum>(f, np, i0, cols, planes, a.sh_k, nk, stage, grad);
 }
 
 // Natural screen-space gradient from the raw sums (for stage checks).

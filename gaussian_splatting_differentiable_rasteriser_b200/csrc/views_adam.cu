@@ -23,7 +23,7 @@
 // the same bits: each Gaussian is updated by one kernel and copied. Plain loads
 // and stores only (no multicast); the kernel waits on nothing: the caller
 // orders it after every rank's blend backward and before any rank's next
-// forward. Five CTAs of 128 per SM (96 registers, 44 KB of shared memory).
+// forward. Five CTAs of 128 per SM (96 registers, 43 KB of shared memory).
 #include "adam_math.cuh"
 #include "adam_stream.cuh"
 #include "gs_kernels.cuh"
@@ -41,7 +41,6 @@ struct ViewsSmem {
   float geom[kViewsGeom][kViewsBlock];  // summed, scaled gradient of the geometric scalars
   float shg[48][kViewsBlock];           // summed, scaled gradient of the active SH coefficients
   CamArgs cam[kMaxRanks];
-  PlaneInfo plane[kStreamMaxPlanes];
 };
 
 template <int kDeg, bool kMip>
@@ -65,7 +64,6 @@ __global__ void __launch_bounds__(kViewsBlock, 5) views_backward_adam_kernel(Vie
         reinterpret_cast<const uint32_t*>(a.views[k / kCamWords].cam)[k % kCamWords];
 #pragma unroll
   for (int c = 0; c < 3 * nk; ++c) sm.shg[c][t] = 0.f;
-  if (t < planes) sm.plane[t] = plane_info(t, a.base.sh_k, nk);
   __syncthreads();
 
   // Phase 1: this Gaussian's gradient, view by view in rank order.
@@ -119,7 +117,7 @@ __global__ void __launch_bounds__(kViewsBlock, 5) views_backward_adam_kernel(Vie
     if (pl < kViewsGeom) return sm.geom[pl][j];
     return info.k >= 0 ? sm.shg[info.ch * nk + info.k][j] : 0.f;
   };
-  adam_stream<false>(sm.plane, a.f, np, i0, cols, planes, a.base.sh_k, nk, stage, grad, a.copies, a.n_copies);
+  adam_stream<false>(a.f, np, i0, cols, planes, a.base.sh_k, nk, stage, grad, a.copies, a.n_copies);
 }
 
 template <int kDeg, bool kMip>
