@@ -54,10 +54,9 @@ WORKLOADS = {
 # the per-Gaussian pass, the (Gaussian, tile) entries for the blend, in which
 # traffic grows in proportion.
 NCU_TRAFFIC = {
-    # Dense-shaped scene of 1.5M Gaussians, one launch (ncu full set)
-    "backward_adam": ((1.272110e9 + 1.007214e9) / 1_500_000, "gaussians", "54499bdf7842"),
-    # Dense-shaped scene of 1.5M Gaussians (3,185,918 entries), one launch
-    "blend_backward": ((335.123712e6 + 57.220608e6) / 3_185_918, "entries", "5abe19b2dac3"),
+    # Dense-shaped scene of 1.5M Gaussians (3,185,918 entries), one launch of each
+    "backward_adam": ((1287.454464e6 + 998.974720e6) / 1_500_000, "gaussians", "fbd93582c070"),
+    "blend_backward": ((350.716672e6 + 69.543680e6) / 3_185_918, "entries", "9f44c98dd94b"),
 }
 
 

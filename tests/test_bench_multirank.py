@@ -96,8 +96,8 @@ def test_traffic_figures_scale_per_unit_of_work():
     assert unit == "gaussians"
     # on the captured case (a Dense-shaped scene of 1.5M Gaussians, 3,185,918 entries)
     # each figure gives back the launch's read + write bytes
-    assert per_g * 1_500_000 == pytest.approx(1.272110e9 + 1.007214e9)
+    assert per_g * 1_500_000 == pytest.approx(1287.454464e6 + 998.974720e6)
     # and it is close to the fused pass's algorithmic bytes per Gaussian (24 B per scalar + 101 B)
     assert per_g == pytest.approx(24 * 59 + 101, rel=0.01)
     per_e, unit, _ = bench.NCU_TRAFFIC["blend_backward"]
-    assert unit == "entries" and per_e * 3_185_918 == pytest.approx(335.123712e6 + 57.220608e6)
+    assert unit == "entries" and per_e * 3_185_918 == pytest.approx(350.716672e6 + 69.543680e6)
