@@ -386,7 +386,10 @@ __global__ void __launch_bounds__(256, kFixed ? 3 : 4) blend_backward_kernel(Ble
       const float alpha = fminf(kAlphaMax, raw);
       const bool contrib = pos < last && alpha >= kAlphaMin;
       if (kCount && contrib) ++blended;
-      if (!__any_sync(0xffffffffu, contrib)) continue;
+      // Every stored survivor blended at some pixel of the warp in the forward,
+      // with the same alpha and before that pixel's last contributor, so some
+      // lane contributes here: no vote is needed to skip it (and a survivor
+      // with none would only add zeros).
       float w = 0.0f, aT = 0.0f;
       if (contrib) {
         const float rcp = __fdividef(1.0f, 1.0f - alpha);
