@@ -166,7 +166,7 @@ gs_status gs_preprocess(gs_ctx *ctx, const gs_params *params, const gs_camera *c
  * [DR] section "The trick: recompute the blend state instead of storing it";
  * [SN] slide on alpha and the background term).
  * Orders the (Gaussian, tile) entries by (tile, depth, index): the visible
- * Gaussians are sorted by depth with a stable LSD onesweep radix sort, one
+ * Gaussians are sorted by depth with a stable LSD radix sort, one
  * entry per touched tile is emitted in that order (prefix sum over
  * tiles_touched), and the entries are sorted stably by tile; then per-tile
  * ranges are extracted and each 16x16 tile is blended front to back:
