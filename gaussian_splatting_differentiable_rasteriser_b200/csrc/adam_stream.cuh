@@ -119,8 +119,9 @@ __device__ __forceinline__ void adam_stream_prologue(const FusedAdamArgs& f, int
   for (int r = 0; r < kStages; ++r) adam_issue_round<kAccum>(f, np, i0, cols, planes, sh_k, nk, r, stage);
 }
 
-// The stream proper. grad(pl, info, j, g) returns the gradient of plane pl at
-// the slice's Gaussian j, given g (the accumulated gradient, 0 without one);
+// The stream proper. grad(pl, info, col, g) returns the gradients of plane pl
+// at the slice's Gaussians 4 col .. 4 col + 3, given g (the accumulated
+// gradients, 0 without them);
 // the updated parameters also go to each of the n_copies parameter buffers.
 // Each round's plane_info is computed from the plane index (a few compares)
 // rather than read from a table in shared memory: the stores' addresses then
@@ -159,11 +160,9 @@ __device__ __forceinline__ void adam_stream(const FusedAdamArgs& f, int64_t np,
       float* m4 = &M[sidx].x;
       float* v4 = &V[sidx].x;
       const AdamScalars sc = f.s[info[sidx].grp];
+      G[sidx] = grad(pl, info[sidx], col, G[sidx]);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        g4[e] = grad(pl, info[sidx], 4 * col + e, g4[e]);
-        adam_one(p4[e], g4[e], m4[e], v4[e], sc);
-      }
+      for (int e = 0; e < 4; ++e) adam_one(p4[e], g4[e], m4[e], v4[e], sc);
       const int64_t off = static_cast<int64_t>(info[sidx].c) * np + i0 + 4 * col;
       *reinterpret_cast<float4*>(f.p[info[sidx].grp] + off) = P[sidx];
       if (kAccum) *reinterpret_cast<float4*>(f.g[info[sidx].grp] + off) = G[sidx];

@@ -163,11 +163,16 @@ __global__ void __launch_bounds__(kFusedBlock) preprocess_backward_adam_kernel(P
 
   // Phase 2: Adam over the CTA's planes; the view gradient adds to the
   // accumulated one (zero without a gradient buffer).
-  auto grad = [&](int pl, const PlaneInfo& info, int j, float g) {
-    if (pl < kGeomPlanes) return __fadd_rn(g, sm.geom[pl][j]);
+  auto grad = [&](int pl, const PlaneInfo& info, int col, float4 g) {
+    if (pl < kGeomPlanes) {
+      const float4 d = reinterpret_cast<const float4*>(sm.geom[pl])[col];
+      return make_float4(__fadd_rn(g.x, d.x), __fadd_rn(g.y, d.y), __fadd_rn(g.z, d.z), __fadd_rn(g.w, d.w));
+    }
     if (info.k >= 0) {
-      const float dc = sm.drgb[info.ch][j];
-      if (dc != 0.f) return __fmaf_rn(dc, sm.Y[info.k][j], g);
+      const float4 dc = reinterpret_cast<const float4*>(sm.drgb[info.ch])[col];
+      const float4 y = reinterpret_cast<const float4*>(sm.Y[info.k])[col];
+      return make_float4(dc.x != 0.f ? __fmaf_rn(dc.x, y.x, g.x) : g.x, dc.y != 0.f ? __fmaf_rn(dc.y, y.y, g.y) : g.y,
+                         dc.z != 0.f ? __fmaf_rn(dc.z, y.z, g.z) : g.z, dc.w != 0.f ? __fmaf_rn(dc.w, y.w, g.w) : g.w);
     }
     return g;
   };

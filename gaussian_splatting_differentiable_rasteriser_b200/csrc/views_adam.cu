@@ -113,9 +113,10 @@ __global__ void __launch_bounds__(kViewsBlock, 5) views_backward_adam_kernel(Vie
 
   // Phase 2: Adam over the CTA's planes; the updated parameters also go to
   // every other rank's buffer.
-  auto grad = [&](int pl, const PlaneInfo& info, int j, float) {
-    if (pl < kViewsGeom) return sm.geom[pl][j];
-    return info.k >= 0 ? sm.shg[info.ch * nk + info.k][j] : 0.f;
+  auto grad = [&](int pl, const PlaneInfo& info, int col, float4) {
+    if (pl < kViewsGeom) return reinterpret_cast<const float4*>(sm.geom[pl])[col];
+    return info.k >= 0 ? reinterpret_cast<const float4*>(sm.shg[info.ch * nk + info.k])[col]
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
   };
   adam_stream<false>(a.f, np, i0, cols, planes, a.base.sh_k, nk, stage, grad, a.copies, a.n_copies);
 }
