@@ -55,7 +55,7 @@ WORKLOADS = {
 # traffic grows in proportion.
 NCU_TRAFFIC = {
     # Dense-shaped scene of 1.5M Gaussians (3,185,918 entries), one launch of each
-    "backward_adam": ((1287.454464e6 + 998.974720e6) / 1_500_000, "gaussians", "fbd93582c070"),
+    "backward_adam": ((1287.691520e6 + 998.944768e6) / 1_500_000, "gaussians", "46b643ddc7b2"),
     "blend_backward": ((350.716672e6 + 69.543680e6) / 3_185_918, "entries", "9f44c98dd94b"),
 }
 

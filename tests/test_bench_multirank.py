@@ -96,7 +96,7 @@ def test_traffic_figures_scale_per_unit_of_work():
     assert unit == "gaussians"
     # on the captured case (a Dense-shaped scene of 1.5M Gaussians, 3,185,918 entries)
     # each figure gives back the launch's read + write bytes
-    assert per_g * 1_500_000 == pytest.approx(1287.454464e6 + 998.974720e6)
+    assert per_g * 1_500_000 == pytest.approx(1287.691520e6 + 998.944768e6)
     # and it is close to the fused pass's algorithmic bytes per Gaussian (24 B per scalar + 101 B)
     assert per_g == pytest.approx(24 * 59 + 101, rel=0.01)
     per_e, unit, _ = bench.NCU_TRAFFIC["blend_backward"]
