@@ -378,6 +378,7 @@ __global__ void __launch_bounds__(256, kFixed ? 3 : 4) blend_backward_kernel(Ble
     if (keep) put_slot(ws, __popc(mask & lt), cur, pos_cur);
     __syncwarp();
     const int cnt = __popc(mask);
+#pragma unroll 2
     for (int k = 0; k < cnt; ++k) {
       const float4 xy = ws.xyp[k];
       const int pos = slot_pos(xy);
@@ -390,17 +391,20 @@ __global__ void __launch_bounds__(256, kFixed ? 3 : 4) blend_backward_kernel(Ble
       // with the same alpha and before that pixel's last contributor, so some
       // lane contributes here: no vote is needed to skip it (and a survivor
       // with none would only add zeros).
-      float w = 0.0f, aT = 0.0f;
-      if (contrib) {
-        const float rcp = __fdividef(1.0f, 1.0f - alpha);
-        T = T * rcp;  // transmittance in front of this Gaussian
-        const float4 c = ws.col[k];
-        const float gc = __fmaf_rn(g2, c.z, __fmaf_rn(g1, c.y, g0 * c.x));
-        const float dalpha = __fmaf_rn(T, gc, -gS * rcp);  // dI/dalpha = T c - S / (1 - alpha)
-        aT = alpha * T;
-        gS = __fmaf_rn(gc, aT, gS);
-        w = raw <= kAlphaMax ? dalpha * raw : 0.0f;  // zero through the cap
-      }
+      // Every lane computes the update (the warp runs it anyway, as some lane
+      // contributes) and keeps it only where its pixel contributes: with no
+      // branch, the two survivors of an unrolled pair overlap their loads and
+      // exponentials.
+      const float rcp = __fdividef(1.0f, 1.0f - alpha);
+      const float Tf = T * rcp;  // transmittance in front of this Gaussian
+      const float4 c = ws.col[k];
+      const float gc = __fmaf_rn(g2, c.z, __fmaf_rn(g1, c.y, g0 * c.x));
+      const float dalpha = __fmaf_rn(Tf, gc, -gS * rcp);  // dI/dalpha = T c - S / (1 - alpha)
+      const float aTf = alpha * Tf;
+      const float aT = contrib ? aTf : 0.0f;
+      const float w = (contrib && raw <= kAlphaMax) ? dalpha * raw : 0.0f;  // zero through the cap
+      T = contrib ? Tf : T;
+      gS = __fmaf_rn(gc, aT, gS);
       wb.wa[bcnt][lane] = make_float2(w, aT);
       if (lane == 0) wb.xyp[bcnt] = xy;
       if (++bcnt == kBatch) {
