@@ -207,13 +207,13 @@ __global__ void __launch_bounds__(256) blend_forward_kernel(BlendArgs a) {
 
 // Per-warp batch of Gaussians that had a contributing pixel in the backward:
 // per (Gaussian, pixel) the two per-pixel factors the nine raw sums are built
-// from, w = dL/dalpha * o exp(-e) and alpha T, plus each Gaussian's slot
-// (centre and id). Rows are padded to 33 so that a lane per Gaussian reads
-// without bank conflicts.
+// from, w = dL/dalpha * o exp(-e) and alpha T. Rows are padded to 33 so that a
+// lane per Gaussian reads without bank conflicts. Each Gaussian's centre and
+// id stay in the registers of the two lanes that reduce it (shared memory
+// bandwidth, not issue, is the backward's tightest limit).
 constexpr int kBatch = 16;
 struct WarpBatch {
   float2 wa[kBatch][33];  // (w, alpha T) of Gaussian j at pixel p (lane p)
-  float4 xyp[kBatch];     // the Gaussian's slot: centre (u, v), position, id
   float4 g[32];           // dL/d(pixel colour) of the warp's pixels
 };
 
@@ -242,7 +242,7 @@ __device__ __forceinline__ void add_sum(float* dst, unsigned long long* fdst, in
 
 template <bool kFixed>
 __device__ __forceinline__ void flush_batch(const WarpBatch& b, int cnt, int lane, float cxb, float cyb,
-                                            float* sgrad, unsigned long long* sgrad_fixed) {
+                                            float2 uv, uint32_t gid, float* sgrad, unsigned long long* sgrad_fixed) {
   const int j = lane & 15, h = lane >> 4;
   float m0 = 0.f, mx = 0.f, my = 0.f, mxx = 0.f, mxy = 0.f, myy = 0.f;
   float c0 = 0.f, c1 = 0.f, c2 = 0.f;
@@ -282,10 +282,9 @@ __device__ __forceinline__ void flush_batch(const WarpBatch& b, int cnt, int lan
   c1 += __shfl_xor_sync(full, c1, 16);
   c2 += __shfl_xor_sync(full, c2, 16);
   if (j < cnt) {
-    const float4 uv = b.xyp[j];
     const float a = uv.x - cxb, bb = uv.y - cyb;
-    float* dst = sgrad + static_cast<int64_t>(slot_id(uv)) * kGradStride;
-    unsigned long long* fdst = kFixed ? sgrad_fixed + static_cast<int64_t>(slot_id(uv)) * kFixedStride : nullptr;
+    float* dst = sgrad + static_cast<int64_t>(gid) * kGradStride;
+    unsigned long long* fdst = kFixed ? sgrad_fixed + static_cast<int64_t>(gid) * kFixedStride : nullptr;
     if (h == 0) {
       const float sy = __fmaf_rn(-bb, m0, my);
       add_sum<kFixed>(dst, fdst, 0, m0);
@@ -352,6 +351,8 @@ __global__ void __launch_bounds__(256, kFixed ? 3 : 4) blend_backward_kernel(Ble
   const int top = beg + max(0, min(wlast, static_cast<int>(range.y - range.x)));  // exclusive
   unsigned blended = 0;
   int bcnt = 0;  // Gaussians in the warp's batch (warp-uniform)
+  float2 buv = make_float2(0.f, 0.f);  // centre and Gaussian of batch entry lane % 16
+  uint32_t bid = 0u;
 
   // The forward stored this warp's survivors of the box test that blend at one
   // of its pixels (list position, Gaussian) in list order; walk them from the
@@ -406,17 +407,20 @@ __global__ void __launch_bounds__(256, kFixed ? 3 : 4) blend_backward_kernel(Ble
       T = contrib ? Tf : T;
       gS = __fmaf_rn(gc, aT, gS);
       wb.wa[bcnt][lane] = make_float2(w, aT);
-      if (lane == 0) wb.xyp[bcnt] = xy;
+      if ((lane & 15) == bcnt) {  // lanes j and j + 16 keep batch entry j's centre and Gaussian
+        buv = make_float2(xy.x, xy.y);
+        bid = slot_id(xy);
+      }
       if (++bcnt == kBatch) {
         __syncwarp();
-        flush_batch<kFixed>(wb, kBatch, lane, bx0 + 3.5f, by0 + 1.5f, a.sgrad, a.sgrad_fixed);
+        flush_batch<kFixed>(wb, kBatch, lane, bx0 + 3.5f, by0 + 1.5f, buv, bid, a.sgrad, a.sgrad_fixed);
         bcnt = 0;
         __syncwarp();
       }
     }
     __syncwarp();  // the slots are rewritten by the next chunk
   }
-  if (bcnt > 0) flush_batch<kFixed>(wb, bcnt, lane, bx0 + 3.5f, by0 + 1.5f, a.sgrad, a.sgrad_fixed);
+  if (bcnt > 0) flush_batch<kFixed>(wb, bcnt, lane, bx0 + 3.5f, by0 + 1.5f, buv, bid, a.sgrad, a.sgrad_fixed);
   if (kCount) {
     // the method's backward walk visits every entry before the pixel's last contributor
     count_pairs(a.pairs, static_cast<unsigned>(min(last, static_cast<int>(range.y - range.x))));
