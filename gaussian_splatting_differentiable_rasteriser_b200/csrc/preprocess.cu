@@ -113,7 +113,11 @@ __global__ void __launch_bounds__(kPreThreads, kPreThreads == 256 ? 3 : 6) prepr
   extern __shared__ __align__(128) unsigned char smem_raw[];
   PreprocessSmem<kDeg>& sm = *reinterpret_cast<PreprocessSmem<kDeg>*>(smem_raw);
   const int tid = threadIdx.x;
-  const int64_t i0 = static_cast<int64_t>(blockIdx.x) * kPreThreads;
+  // Slices are taken from the last to the first: the fused backward + Adam pass
+  // of the previous step walks the parameters upwards, so the last slices'
+  // parameters are still in L2 when this kernel starts.
+  const int64_t blk = static_cast<int64_t>(gridDim.x) - 1 - static_cast<int64_t>(blockIdx.x);
+  const int64_t i0 = blk * kPreThreads;
   const int64_t i = i0 + tid;
   const int64_t np = a.n_pad;
   // Stage the CTA's slice of every parameter plane in shared memory with bulk
@@ -144,8 +148,8 @@ __global__ void __launch_bounds__(kPreThreads, kPreThreads == 256 ? 3 : 6) prepr
     // The CTA that will start about when this one ends (one grid of resident
     // CTAs later) finds its planes in L2: its copies then wait on L2, not on
     // DRAM, and this CTA's copies overlap the DRAM reads of the next slices.
-    const int64_t nb = static_cast<int64_t>(blockIdx.x) + a.prefetch_ahead;
-    if (a.prefetch_ahead > 0 && nb < static_cast<int64_t>(gridDim.x)) {
+    const int64_t nb = blk - a.prefetch_ahead;
+    if (a.prefetch_ahead > 0 && nb >= 0) {
       const int64_t j0 = nb * kPreThreads;
       const uint32_t pbytes = static_cast<uint32_t>(np - j0 < kPreThreads ? np - j0 : kPreThreads) * 4u;
 #pragma unroll
@@ -180,7 +184,7 @@ __global__ void __launch_bounds__(kPreThreads, kPreThreads == 256 ? 3 : 6) prepr
       a.touched[i] = 0u;
       a.clamped[i] = 0u;
     }
-    if (tid == 0) a.block_sums[blockIdx.x] = make_uint2(0u, 0u);
+    if (tid == 0) a.block_sums[blk] = make_uint2(0u, 0u);
     return;
   }
   uint32_t touched = 0;
@@ -346,7 +350,7 @@ __global__ void __launch_bounds__(kPreThreads, kPreThreads == 256 ? 3 : 6) prepr
       b += s_sum[k];
       v += s_vis[k];
     }
-    a.block_sums[blockIdx.x] = make_uint2(b, v);
+    a.block_sums[blk] = make_uint2(b, v);
   }
 }
 
