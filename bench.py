@@ -302,6 +302,9 @@ def time_device(step, cams, targets, sched, start, count, world):
     return ev0.elapsed_time(ev1)
 
 
+BLEND_STAGES = ("blend_forward", "blend_backward")
+
+
 def profile_stages(step, cams, targets, sched, start, count):
     """Per-stage kernel times (library events) plus Adam (torch events: the
     Adam launches are the only work between them on the current stream). For the
@@ -326,9 +329,8 @@ def profile_stages(step, cams, targets, sched, start, count):
     group = max(1, min(5, count // 5))
     groups = []
     adam = []
-    # one untimed profiled step first: the counting variants of the blend kernels
-    # are launched for the first time there, and a first launch can include the
-    # loading of the kernel's code between the stage's events
+    # one untimed profiled step first, so that no stage's events span a first
+    # launch (which can include the loading of the kernel's code)
     for i in range(start - 1, start + count):
         timed = i >= start
         c = int(sched[i % len(sched)])
@@ -356,10 +358,31 @@ def profile_stages(step, cams, targets, sched, start, count):
             stages = ctx.profile_read()
             if timed:
                 groups.append((stages, j - sum(n for _, n in groups)))
+    # The (pixel, Gaussian) pairs of the two blends, for their instruction
+    # model, from a second pass over the same cameras with the counting variants
+    # of the blend kernels (whose times are not used: the pass above timed the
+    # kernels a training run launches).
+    ctx.profile_enable(True, count_pairs=True)
+    for i in range(start, start + count):
+        c = int(sched[i % len(sched)])
+        cam = cams[c]
+        cs = native.camera_struct(cam)
+        img, T, nc = step.forward(cs, cam.height, cam.width)
+        step.compute_loss(img, targets[c], step.dimage)
+        if step.fused_adam or getattr(step, "exchange", None) == "views":
+            step.backward_and_update(cs, T, nc, step.dimage)
+        else:
+            m.step_count += 1
+            ctx.render_backward(m.params_struct(), cs, T, nc, step.dimage, m.grads_struct())
+            step.update_from_grads()
+    torch.cuda.synchronize()
+    counted = ctx.profile_read()
     ctx.profile_enable(False)
     prof = {}
     for name in groups[0][0] if groups else ():
         d = {k: sum(g[name][k] for g, _ in groups) for k in ("launches", "work", "blended")}
+        if name in BLEND_STAGES:
+            d["work"], d["blended"] = counted[name]["work"], counted[name]["blended"]
         # median over the groups of the stage's time per step, times the steps
         d["ms"] = statistics.median(g[name]["ms"] / n for g, n in groups) * count
         prof[name] = d

@@ -77,7 +77,7 @@ struct gs_ctx {
   // profiling (off by default)
   struct Profiler {
     static constexpr int kMaxRec = 128;
-    bool on = false, created = false;
+    bool on = false, count = false, created = false;
     cudaEvent_t ev[2 * kMaxRec];
     int stage[kMaxRec];
     int nrec = 0;
@@ -508,7 +508,7 @@ gs_status gs_render_forward(gs_ctx* c, const gs_camera* cam, float* image, float
   ba.image = image;
   ba.final_T = final_T;
   ba.n_contrib = n_contrib;
-  ba.pairs = c->prof.on ? c->pairs : nullptr;
+  ba.pairs = c->prof.count ? c->pairs : nullptr;
   ba.surv = c->surv;
   ba.surv_count = c->surv_count;
   prof_begin(c, st);
@@ -594,7 +594,7 @@ gs_status backward_common(gs_ctx* c, const gs_params* p, const gs_camera* cam, c
   ba.n_contrib = const_cast<int32_t*>(n_contrib);
   ba.dimage = dloss_dimage;
   ba.sgrad = c->sgrad;
-  ba.pairs = c->prof.on ? c->pairs + 4 : nullptr;
+  ba.pairs = c->prof.count ? c->pairs + 4 : nullptr;
   ba.surv = c->surv;
   ba.surv_count = c->surv_count;
   ba.sgrad_fixed = c->deterministic ? c->sgrad_fixed : nullptr;
@@ -923,8 +923,11 @@ gs_status gs_profile_enable(gs_ctx* c, int32_t enabled) {
     for (auto& e : P.ev) GS_CUDA(c, cudaEventCreate(&e));
     P.created = true;
   }
-  if (P.on && !enabled) prof_harvest(c);
-  P.on = enabled != 0;
+  if (enabled & ~(GS_PROFILE_TIME | GS_PROFILE_COUNT))
+    return fail(c, GS_ERR_INVALID_ARG, "unknown profiling flags 0x%x", static_cast<unsigned>(enabled));
+  if (P.on && !(enabled & GS_PROFILE_TIME)) prof_harvest(c);
+  P.on = (enabled & GS_PROFILE_TIME) != 0;
+  P.count = (enabled & GS_PROFILE_COUNT) != 0;
   return GS_OK;
 }
 

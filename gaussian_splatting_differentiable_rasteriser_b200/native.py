@@ -34,6 +34,8 @@ MAX_RANKS = 8
 GS_OPTION_OPACITY_RECT = 1
 GS_OPTION_DETERMINISTIC = 2
 GS_OPTION_MIP_COMPENSATION = 3
+PROFILE_TIME = 1   # GS_PROFILE_TIME
+PROFILE_COUNT = 2  # GS_PROFILE_COUNT
 STAGES = ("preprocess", "scan", "duplicate", "sort", "ranges", "blend_forward", "loss",
           "blend_backward", "preprocess_backward", "backward_adam", "depth_sort", "camera_backward",
           "views_adam")
@@ -292,8 +294,12 @@ class Context:
             _ptr(dloss_dimage), g, ctypes.byref(exp_avg), ctypes.byref(exp_avg_sq),
             lr, float(beta1), float(beta2), float(eps), int(step), _stream(stream)))
 
-    def profile_enable(self, on=True):
-        self._check(self.L.gs_profile_enable(self.h, 1 if on else 0))
+    def profile_enable(self, on=True, count_pairs=False):
+        """Stage timing of the production kernels (on); count_pairs also makes
+        the two blends count their (pixel, Gaussian) pairs, through counting
+        variants whose times then replace the production kernels'."""
+        self._check(self.L.gs_profile_enable(self.h, (PROFILE_TIME if on else 0) |
+                                             (PROFILE_COUNT if count_pairs else 0)))
 
     def profile_read(self) -> dict:
         n = len(STAGES)

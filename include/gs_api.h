@@ -381,21 +381,30 @@ gs_status gs_shared_close(void *ptr);
 gs_status gs_shared_free(void *ptr);
 
 /* ------------------------------------------------------------ profiling --
- * When enabled, every kernel launch a context makes is bracketed by CUDA
- * events on the call's stream (a few microseconds of host time per launch;
- * leave it off for throughput runs). gs_profile_read waits for the recorded
- * events, returns per-stage totals accumulated since the previous read and
- * resets them. Each output is a HOST array of GS_NUM_STAGES entries (any may
- * be NULL): ms = summed kernel time, launches = kernel launches, work = the units
- * processed (Gaussians for the per-Gaussian stages - n_pad for the fused
- * backward + Adam pass -, visible Gaussians x passes for the depth sort,
- * entries x passes for the tile sort, entries for the duplication and
- * ranges, pixels for the loss; for the two blends the
- * (pixel, Gaussian) pairs the method's walk visits: every list entry up to
- * the pixel's stopping point in the forward, every entry before its last
- * contributor in the backward), blended = for the two blends the pairs that
- * actually blend (alpha >= 1/255 before the walk stops), 0 elsewhere. gs_adam_step takes no context and is not profiled
- * here. */
+ * gs_profile_enable takes a set of flags (0 turns profiling off):
+ *   GS_PROFILE_TIME  - every kernel launch a context makes is bracketed by
+ *                      CUDA events on the call's stream (a few microseconds
+ *                      of host time per launch; leave it off for throughput
+ *                      runs). The kernels timed are the ones a run without
+ *                      profiling launches.
+ *   GS_PROFILE_COUNT - the two blends count (pixel, Gaussian) pairs: their
+ *                      counting variants run instead (slower, so stage times
+ *                      taken together with this flag are those variants').
+ * gs_profile_read waits for the recorded events, returns per-stage totals
+ * accumulated since the previous read and resets them. Each output is a HOST
+ * array of GS_NUM_STAGES entries (any may be NULL): ms = summed kernel time,
+ * launches = kernel launches, work = the units processed (Gaussians for the
+ * per-Gaussian stages - n_pad for the fused backward + Adam pass -, visible
+ * Gaussians x passes for the depth sort, entries x passes for the tile sort,
+ * entries for the duplication and ranges, pixels for the loss; for the two
+ * blends, when counting, the (pixel, Gaussian) pairs the method's walk
+ * visits: every list entry up to the pixel's stopping point in the forward,
+ * every entry before its last contributor in the backward, and 0 when not
+ * counting), blended = for the two blends the pairs that actually blend
+ * (alpha >= 1/255 before the walk stops) when counting, 0 elsewhere.
+ * Unknown flags give GS_ERR_INVALID_ARG. gs_adam_step takes no context and is
+ * not profiled here. */
+typedef enum { GS_PROFILE_TIME = 1, GS_PROFILE_COUNT = 2 } gs_profile_flag;
 typedef enum {
   GS_STAGE_PREPROCESS = 0,
   GS_STAGE_SCAN = 1,

@@ -52,6 +52,19 @@ def test_stage_names_match_the_binding():
     assert L.gs_stage_name(len(native.STAGES)).decode() == ""
 
 
+def test_header_constants_match_the_binding():
+    """The option and profiling flag values the binding passes are the header's."""
+    from gaussian_splatting_differentiable_rasteriser_b200 import native
+    text = open(HEADER).read()
+    defines = {m.group(1): int(m.group(2)) for m in re.finditer(r"\b(GS_[A-Z_]+) = (\d+)", text)}
+    assert defines["GS_PROFILE_TIME"] == native.PROFILE_TIME
+    assert defines["GS_PROFILE_COUNT"] == native.PROFILE_COUNT
+    for name in ("GS_OPTION_OPACITY_RECT", "GS_OPTION_DETERMINISTIC", "GS_OPTION_MIP_COMPENSATION"):
+        assert defines[name] == getattr(native, name), name
+    L = native.load()
+    assert L.gs_profile_enable(None, native.PROFILE_TIME) == native.GS_ERR_INVALID_ARG
+
+
 def test_new_entry_points_check_their_arguments_on_the_host():
     """The data-parallel, shared-memory, camera-gradient and recycling entry
     points reject bad arguments before any CUDA call (so this runs without a GPU)."""
