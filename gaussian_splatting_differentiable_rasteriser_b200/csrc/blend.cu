@@ -208,9 +208,10 @@ __global__ void __launch_bounds__(256) blend_forward_kernel(BlendArgs a) {
 // Per-warp batch of Gaussians that had a contributing pixel in the backward:
 // per (Gaussian, pixel) the two per-pixel factors the nine raw sums are built
 // from, w = dL/dalpha * o exp(-e) and alpha T. Rows are padded to 33 so that a
-// lane per Gaussian reads without bank conflicts. Each Gaussian's centre and
-// id stay in the registers of the two lanes that reduce it (shared memory
-// bandwidth, not issue, is the backward's tightest limit).
+// lane per Gaussian reads without bank conflicts. A batch is one half of a
+// chunk's slots, so the reduction reads each Gaussian's centre and id from its
+// slot (shared-memory bandwidth, not issue, is the backward's tightest limit:
+// nothing per survivor is copied into the batch but its two factors).
 constexpr int kBatch = 16;
 struct WarpBatch {
   float2 wa[kBatch][33];  // (w, alpha T) of Gaussian j at pixel p (lane p)
@@ -350,9 +351,6 @@ __global__ void __launch_bounds__(256, kFixed ? 3 : 4) blend_backward_kernel(Ble
   for (int o = 16; o > 0; o >>= 1) wlast = max(wlast, __shfl_xor_sync(0xffffffffu, wlast, o));
   const int top = beg + max(0, min(wlast, static_cast<int>(range.y - range.x)));  // exclusive
   unsigned blended = 0;
-  int bcnt = 0;  // Gaussians in the warp's batch (warp-uniform)
-  float2 buv = make_float2(0.f, 0.f);  // centre and Gaussian of batch entry lane % 16
-  uint32_t bid = 0u;
 
   // The forward stored this warp's survivors of the box test that blend at one
   // of its pixels (list position, Gaussian) in list order; walk them from the
@@ -379,7 +377,6 @@ __global__ void __launch_bounds__(256, kFixed ? 3 : 4) blend_backward_kernel(Ble
     if (keep) put_slot(ws, __popc(mask & lt), cur, pos_cur);
     __syncwarp();
     const int cnt = __popc(mask);
-#pragma unroll 2
     for (int k = 0; k < cnt; ++k) {
       const float4 xy = ws.xyp[k];
       const int pos = slot_pos(xy);
@@ -393,9 +390,8 @@ __global__ void __launch_bounds__(256, kFixed ? 3 : 4) blend_backward_kernel(Ble
       // lane contributes here: no vote is needed to skip it (and a survivor
       // with none would only add zeros).
       // Every lane computes the update (the warp runs it anyway, as some lane
-      // contributes) and keeps it only where its pixel contributes: with no
-      // branch, the two survivors of an unrolled pair overlap their loads and
-      // exponentials.
+      // contributes) and keeps it only where its pixel contributes: no branch,
+      // so the next survivor's loads and exponential can start early.
       const float rcp = __fdividef(1.0f, 1.0f - alpha);
       const float Tf = T * rcp;  // transmittance in front of this Gaussian
       const float4 c = ws.col[k];
@@ -406,21 +402,21 @@ __global__ void __launch_bounds__(256, kFixed ? 3 : 4) blend_backward_kernel(Ble
       const float w = (contrib && raw <= kAlphaMax) ? dalpha * raw : 0.0f;  // zero through the cap
       T = contrib ? Tf : T;
       gS = __fmaf_rn(gc, aT, gS);
-      wb.wa[bcnt][lane] = make_float2(w, aT);
-      if ((lane & 15) == bcnt) {  // lanes j and j + 16 keep batch entry j's centre and Gaussian
-        buv = make_float2(xy.x, xy.y);
-        bid = slot_id(xy);
-      }
-      if (++bcnt == kBatch) {
+      // A batch is slots 16 h .. 16 h + 15 of the chunk (fewer in its last
+      // one), so its Gaussians' centres and ids are still in the slots when it
+      // is reduced.
+      const int row = k & (kBatch - 1);
+      wb.wa[row][lane] = make_float2(w, aT);
+      if (row == kBatch - 1 || k == cnt - 1) {
         __syncwarp();
-        flush_batch<kFixed>(wb, kBatch, lane, bx0 + 3.5f, by0 + 1.5f, buv, bid, a.sgrad, a.sgrad_fixed);
-        bcnt = 0;
+        const float4 bxy = ws.xyp[k - row + (lane & (kBatch - 1))];
+        flush_batch<kFixed>(wb, row + 1, lane, bx0 + 3.5f, by0 + 1.5f, make_float2(bxy.x, bxy.y), slot_id(bxy),
+                            a.sgrad, a.sgrad_fixed);
         __syncwarp();
       }
     }
     __syncwarp();  // the slots are rewritten by the next chunk
   }
-  if (bcnt > 0) flush_batch<kFixed>(wb, bcnt, lane, bx0 + 3.5f, by0 + 1.5f, buv, bid, a.sgrad, a.sgrad_fixed);
   if (kCount) {
     // the method's backward walk visits every entry before the pixel's last contributor
     count_pairs(a.pairs, static_cast<unsigned>(min(last, static_cast<int>(range.y - range.x))));
