@@ -181,9 +181,12 @@ struct LossArgs {
 };
 
 // The loss runs one CTA per channel and strip of kLossCols columns x
-// kLossStrip rows (kLossStrip a multiple of 16; a build-time tunable).
+// kLossStrip rows (kLossStrip a multiple of 16; a build-time tunable). At
+// 1920x1080, 192 rows give 1,080 CTAs, just under two waves of 4 per SM on
+// 148 SMs, with a 20-row pipeline fill per strip (measured: 0.175 ms against
+// 0.186 ms for 128 rows, 0.187 for 176 and 0.183 for 368).
 #ifndef GS_LOSS_STRIP
-#define GS_LOSS_STRIP 128
+#define GS_LOSS_STRIP 192
 #endif
 constexpr int kLossCols = 32;
 constexpr int kLossStrip = GS_LOSS_STRIP;
