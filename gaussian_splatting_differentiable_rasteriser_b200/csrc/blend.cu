@@ -118,6 +118,8 @@ __device__ __forceinline__ void count_pairs(unsigned long long* pairs, unsigned 
 
 template <bool kCount>
 __global__ void __launch_bounds__(256) blend_forward_kernel(BlendArgs a) {
+  chain_wait();
+  chain_release();
   __shared__ WarpSlots slots[kWarps];
   const int tile = static_cast<int>(a.tile_order[blockIdx.x]);
   const int tx = tile % a.cam.tiles_x, ty = tile / a.cam.tiles_x;
@@ -311,6 +313,8 @@ struct BackwardSmem {
 // fixed-point variant keeps three.
 template <bool kCount, bool kFixed>
 __global__ void __launch_bounds__(256, kFixed ? 3 : 4) blend_backward_kernel(BlendArgs a) {
+  chain_wait();
+  chain_release();
   extern __shared__ __align__(16) unsigned char smem_raw[];
   BackwardSmem& sm = *reinterpret_cast<BackwardSmem*>(smem_raw);
   WarpSlots* slots = sm.slots;
@@ -448,11 +452,8 @@ cudaError_t launch_decode_fixed(const unsigned long long* fixed, int64_t n, floa
 cudaError_t launch_blend_forward(const BlendArgs& a, cudaStream_t st) {
   const int tiles = a.cam.tiles_x * a.cam.tiles_y;
   if (tiles == 0) return cudaSuccess;
-  if (a.pairs)
-    blend_forward_kernel<true><<<tiles, 256, 0, st>>>(a);
-  else
-    blend_forward_kernel<false><<<tiles, 256, 0, st>>>(a);
-  return cudaGetLastError();
+  return a.pairs ? launch_chained(blend_forward_kernel<true>, dim3(tiles), dim3(256), 0, st, a)
+                 : launch_chained(blend_forward_kernel<false>, dim3(tiles), dim3(256), 0, st, a);
 }
 
 template <bool kCount, bool kFixed>
@@ -461,8 +462,7 @@ cudaError_t launch_backward_variant(const BlendArgs& a, int tiles, cudaStream_t 
   cudaError_t e = cudaFuncSetAttribute(blend_backward_kernel<kCount, kFixed>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  blend_backward_kernel<kCount, kFixed><<<tiles, 256, smem, st>>>(a);
-  return cudaGetLastError();
+  return launch_chained(blend_backward_kernel<kCount, kFixed>, dim3(tiles), dim3(256), smem, st, a);
 }
 
 cudaError_t launch_blend_backward(const BlendArgs& a, cudaStream_t st) {

@@ -7,6 +7,33 @@
 
 namespace gs {
 
+// Programmatic dependent launch. The kernels of a training step are launched
+// with launch_chained: a kernel's CTAs may then be scheduled while the kernel
+// before it on the stream is still finishing, so that the launch of each stage
+// overlaps the tail of the previous one. Every such kernel calls chain_wait()
+// first, before it reads or writes anything (it returns once the previous
+// kernel has completed and its writes are visible; a no-op for a kernel
+// launched the ordinary way), and then chain_release(), which lets the next
+// kernel be scheduled once all of this kernel's CTAs have started.
+__device__ __forceinline__ void chain_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void chain_release() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... P, typename... A>
+inline cudaError_t launch_chained(void (*kernel)(P...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                                  A&&... args) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<A&&>(args)...);
+}
+
 // Written by the preprocess + block scan and read back by the host before the
 // sort: the entry count, the number of visible Gaussians and the range of
 // depth keys of visible Gaussians.

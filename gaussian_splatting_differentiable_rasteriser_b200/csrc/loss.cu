@@ -87,6 +87,8 @@ __device__ __forceinline__ void load_rows(const LossArgs& a, const float* X, con
 }
 
 __global__ void __launch_bounds__(kLossThreads, 4) loss_kernel(LossArgs a) {
+  chain_wait();
+  chain_release();
   extern __shared__ __align__(16) unsigned char smem_raw[];
   LossSmem& s = *reinterpret_cast<LossSmem*>(smem_raw);
   const int tid = threadIdx.x;
@@ -352,8 +354,7 @@ cudaError_t launch_loss(const LossArgs& a, cudaStream_t st) {
                                        static_cast<int>(sizeof(LossSmem)));
   if (e != cudaSuccess) return e;
   dim3 grid((a.width + kCols - 1) / kCols, (a.height + kStrip - 1) / kStrip, 3);
-  loss_kernel<<<grid, kLossThreads, sizeof(LossSmem), st>>>(a);
-  return cudaGetLastError();
+  return launch_chained(loss_kernel, grid, dim3(kLossThreads), sizeof(LossSmem), st, a);
 }
 
 int64_t loss_num_blocks(int height, int width) { return loss_blocks(height, width); }

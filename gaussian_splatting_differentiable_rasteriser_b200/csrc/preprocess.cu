@@ -108,6 +108,8 @@ struct PreprocessSmem {
 
 template <int kDeg>
 __global__ void __launch_bounds__(kPreThreads, kPreThreads == 256 ? 3 : 6) preprocess_kernel(PreprocessArgs a) {
+  chain_wait();
+  chain_release();
   constexpr int nk = (kDeg + 1) * (kDeg + 1);
   constexpr int kPlanes = kGeomPlanes + 3 * nk;
   extern __shared__ __align__(128) unsigned char smem_raw[];
@@ -361,6 +363,8 @@ __global__ void __launch_bounds__(1024) scan_blocks_kernel(const uint2* block_su
                                                            uint32_t* visible_prefix,
                                                            const uint32_t* depth_range,
                                                            ForwardInfo* info) {
+  chain_wait();
+  chain_release();
   __shared__ uint64_t s_warp[32];
   __shared__ uint32_t s_vwarp[32];
   const int tid = threadIdx.x;
@@ -442,8 +446,7 @@ cudaError_t launch_preprocess_deg(const PreprocessArgs& args, unsigned grid, cud
   if (e != cudaSuccess) return e;
   PreprocessArgs a = args;
   a.prefetch_ahead = static_cast<int64_t>(sms) * per_sm;
-  preprocess_kernel<kDeg><<<grid, kPreThreads, smem, st>>>(a);
-  return cudaGetLastError();
+  return launch_chained(preprocess_kernel<kDeg>, dim3(grid), dim3(kPreThreads), smem, st, a);
 }
 
 }  // namespace
@@ -461,8 +464,8 @@ cudaError_t launch_preprocess(const PreprocessArgs& a, int64_t num_blocks, cudaS
 
 cudaError_t launch_scan_blocks(const uint2* block_sums, int64_t num_blocks, uint32_t* visible_prefix,
                                const uint32_t* depth_range, ForwardInfo* info, cudaStream_t st) {
-  scan_blocks_kernel<<<1, 1024, 0, st>>>(block_sums, num_blocks, visible_prefix, depth_range, info);
-  return cudaGetLastError();
+  return launch_chained(scan_blocks_kernel, dim3(1), dim3(1024), 0, st, block_sums, num_blocks, visible_prefix,
+                        depth_range, info);
 }
 
 }  // namespace gs

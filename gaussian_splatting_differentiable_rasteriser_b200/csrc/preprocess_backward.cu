@@ -109,6 +109,8 @@ struct FusedSmem {
 template <int kDeg, bool kAccum, bool kStats, bool kMip>
 __global__ void __launch_bounds__(kFusedBlock) preprocess_backward_adam_kernel(PreprocessBwdArgs a,
                                                                               FusedAdamArgs f) {
+  chain_wait();
+  chain_release();
   __shared__ __align__(16) FusedSmem sm;
   const int t = threadIdx.x;
   const int64_t i0 = static_cast<int64_t>(blockIdx.x) * kFusedBlock;
@@ -223,8 +225,8 @@ cudaError_t launch_fused_mip(const PreprocessBwdArgs& a, const FusedAdamArgs& f,
   cudaError_t e = cudaFuncSetAttribute(preprocess_backward_adam_kernel<kDeg, kAccum, kStats, kMip>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  preprocess_backward_adam_kernel<kDeg, kAccum, kStats, kMip><<<grid, kFusedBlock, smem, st>>>(a, f);
-  return cudaGetLastError();
+  return launch_chained(preprocess_backward_adam_kernel<kDeg, kAccum, kStats, kMip>, dim3(grid), dim3(kFusedBlock),
+                        smem, st, a, f);
 }
 
 template <int kDeg, bool kAccum, bool kStats>

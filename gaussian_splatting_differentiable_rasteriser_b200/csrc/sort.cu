@@ -48,6 +48,8 @@ namespace {
 constexpr int kCompactBlocks = 4;
 
 __global__ void __launch_bounds__(kGaussBlock) compact_kernel(CompactArgs a) {
+  chain_wait();
+  chain_release();
   __shared__ uint32_t s_warp[kCompactBlocks][kGaussBlock / 32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t b0 = static_cast<int64_t>(blockIdx.x) * kCompactBlocks;
@@ -97,6 +99,8 @@ __device__ __forceinline__ uint32_t div_small(uint32_t n, uint32_t d) {
 // duplicate's CTA granularity): one CTA per chunk, one sum per chunk.
 __global__ void __launch_bounds__(kDupThreads) dup_count_kernel(const uint32_t* order, const uint32_t* touched,
                                                                 int64_t count, uint32_t* chunk_tiles) {
+  chain_wait();
+  chain_release();
   __shared__ uint32_t s_warp[kDupThreads / 32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t base = static_cast<int64_t>(blockIdx.x) * kDupItems;
@@ -122,6 +126,8 @@ __global__ void __launch_bounds__(kDupThreads) dup_count_kernel(const uint32_t* 
 // 32 (kDupPerThread w + j) + l, so the order reads are coalesced and, for a
 // given j, the lanes' output runs are adjacent in memory.
 __global__ void __launch_bounds__(kDupThreads) duplicate_kernel(DuplicateArgs a) {
+  chain_wait();
+  chain_release();
   __shared__ uint32_t s_warp[kDupThreads / 32];
   __shared__ uint32_t s_pre[kDupThreads / 32][kDupPerThread][32];  // items' offsets in the warp's run
   __shared__ uint32_t s_gid[kDupThreads / 32][kDupPerThread][32];  // items' Gaussians
@@ -239,6 +245,8 @@ __global__ void __launch_bounds__(kDupThreads) duplicate_kernel(DuplicateArgs a)
 __global__ void __launch_bounds__(kSortThreads) upsweep_kernel(const uint32_t* keys, int64_t n, int shift,
                                                                int64_t chunks, uint32_t* counts,
                                                                uint32_t* hist) {
+  chain_wait();
+  chain_release();
   __shared__ uint32_t s_h[kSortThreads / 32][kRadix];
   const int tid = threadIdx.x, warp = tid >> 5;
   const int64_t base = static_cast<int64_t>(blockIdx.x) * kSortTileKeys;
@@ -288,6 +296,8 @@ __global__ void __launch_bounds__(kSortThreads) upsweep_kernel(const uint32_t* k
 constexpr int kScanThreads = 1024;
 __global__ void __launch_bounds__(kScanThreads) scan_digits_kernel(uint32_t* counts, int64_t chunks,
                                                                     const uint32_t* hist) {
+  chain_wait();
+  chain_release();
   __shared__ uint32_t s_warp[kScanThreads / 32];
   __shared__ uint32_t s_carry;
   const int d = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -469,6 +479,8 @@ __device__ __forceinline__ void downsweep_chunk(const DownsweepArgs& a, Downswee
 
 template <int kBits>
 __global__ void __launch_bounds__(kSortThreads, GS_SORT_MINB) downsweep_kernel(DownsweepArgs a) {
+  chain_wait();
+  chain_release();
   extern __shared__ __align__(16) unsigned char smem_raw[];
   DownsweepSmem& sm = *reinterpret_cast<DownsweepSmem*>(smem_raw);
   const int64_t chunk = blockIdx.x;
@@ -483,8 +495,7 @@ cudaError_t launch_downsweep(const DownsweepArgs& o, unsigned chunks, cudaStream
   cudaError_t e = cudaFuncSetAttribute(downsweep_kernel<kBits>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(sizeof(DownsweepSmem)));
   if (e != cudaSuccess) return e;
-  downsweep_kernel<kBits><<<chunks, kSortThreads, sizeof(DownsweepSmem), st>>>(o);
-  return cudaGetLastError();
+  return launch_chained(downsweep_kernel<kBits>, dim3(chunks), dim3(kSortThreads), sizeof(DownsweepSmem), st, o);
 }
 
 cudaError_t launch_downsweep_bits(const DownsweepArgs& o, int bits, unsigned chunks, cudaStream_t st) {
@@ -508,6 +519,8 @@ constexpr int kRangeItems = 8;
 
 __global__ void __launch_bounds__(256) ranges_kernel(const uint32_t* keys, int64_t n, uint2* ranges,
                                                      int64_t num_tiles) {
+  chain_wait();
+  chain_release();
   const int64_t i0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) * kRangeItems;
   if (i0 >= n) return;
   uint32_t k[kRangeItems];
@@ -542,6 +555,8 @@ __global__ void __launch_bounds__(256) ranges_kernel(const uint32_t* keys, int64
 constexpr int kOrderThreads = 1024;
 __global__ void __launch_bounds__(kOrderThreads) tile_order_kernel(const uint2* ranges, int64_t num_tiles,
                                                                    uint32_t* order) {
+  chain_wait();
+  chain_release();
   __shared__ uint32_t cnt[33];  // by __clz(length): 0 for the longest, 32 for empty tiles
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const unsigned lt = (1u << lane) - 1u;
@@ -598,14 +613,13 @@ __global__ void __launch_bounds__(kOrderThreads) tile_order_kernel(const uint2* 
 
 cudaError_t launch_tile_order(const uint2* ranges, int64_t num_tiles, uint32_t* order, cudaStream_t st) {
   if (num_tiles <= 0) return cudaSuccess;
-  tile_order_kernel<<<1, kOrderThreads, 0, st>>>(ranges, num_tiles, order);
-  return cudaGetLastError();
+  return launch_chained(tile_order_kernel, dim3(1), dim3(kOrderThreads), 0, st, ranges, num_tiles, order);
 }
 
 cudaError_t launch_compact(const CompactArgs& a, int64_t num_blocks, cudaStream_t st) {
   if (num_blocks == 0) return cudaSuccess;
-  compact_kernel<<<static_cast<unsigned>((num_blocks + kCompactBlocks - 1) / kCompactBlocks), kGaussBlock, 0, st>>>(a);
-  return cudaGetLastError();
+  return launch_chained(compact_kernel, dim3(static_cast<unsigned>((num_blocks + kCompactBlocks - 1) / kCompactBlocks)),
+                        dim3(kGaussBlock), 0, st, a);
 }
 
 cudaError_t launch_duplicate(const DuplicateArgs& a, cudaStream_t st) {
@@ -613,10 +627,12 @@ cudaError_t launch_duplicate(const DuplicateArgs& a, cudaStream_t st) {
   const int64_t chunks = (a.count + kDupItems - 1) / kDupItems;
   const unsigned grid = static_cast<unsigned>(chunks);
   // per-chunk tile counts, their exclusive prefix in place (one scan row), then the entries
-  dup_count_kernel<<<grid, kDupThreads, 0, st>>>(a.order, a.touched, a.count, a.chunk_offsets);
-  scan_digits_kernel<<<1, kScanThreads, 0, st>>>(a.chunk_offsets, chunks, nullptr);
-  duplicate_kernel<<<grid, kDupThreads, 0, st>>>(a);
-  return cudaGetLastError();
+  cudaError_t e = launch_chained(dup_count_kernel, dim3(grid), dim3(kDupThreads), 0, st, a.order, a.touched, a.count,
+                                 a.chunk_offsets);
+  if (e == cudaSuccess)
+    e = launch_chained(scan_digits_kernel, dim3(1), dim3(kScanThreads), 0, st, a.chunk_offsets, chunks, nullptr);
+  if (e == cudaSuccess) e = launch_chained(duplicate_kernel, dim3(grid), dim3(kDupThreads), 0, st, a);
+  return e;
 }
 
 cudaError_t launch_sort(const SortPlan& plan, const SortBuffers& b, int* out_buf, cudaStream_t st) {
@@ -630,8 +646,12 @@ cudaError_t launch_sort(const SortPlan& plan, const SortBuffers& b, int* out_buf
     const int digit_bits = std::min(8, plan.key_bits - 8 * p);
     uint32_t* counts = b.chunk_counts + static_cast<int64_t>(p) * plan.tiles * kRadix;  // [256][chunks]
     uint32_t* hist = b.hist + p * kRadix;
-    upsweep_kernel<<<chunks, kSortThreads, 0, st>>>(b.keys[cur], plan.n, 8 * p, plan.tiles, counts, hist);
-    scan_digits_kernel<<<1u << digit_bits, kScanThreads, 0, st>>>(counts, plan.tiles, hist);
+    if ((e = launch_chained(upsweep_kernel, dim3(chunks), dim3(kSortThreads), 0, st, b.keys[cur], plan.n, 8 * p,
+                            plan.tiles, counts, hist)) != cudaSuccess)
+      return e;
+    if ((e = launch_chained(scan_digits_kernel, dim3(1u << digit_bits), dim3(kScanThreads), 0, st, counts, plan.tiles,
+                            hist)) != cudaSuccess)
+      return e;
     DownsweepArgs o;
     o.keys_in = b.keys[cur];
     o.vals_in = b.vals[cur];
@@ -655,9 +675,8 @@ cudaError_t launch_ranges(const uint32_t* keys, int64_t n, uint2* ranges, int64_
   cudaError_t e = cudaMemsetAsync(ranges, 0, sizeof(uint2) * num_tiles, st);
   if (e != cudaSuccess || n == 0) return e;
   const int64_t per_block = 256 * kRangeItems;
-  ranges_kernel<<<static_cast<unsigned>((n + per_block - 1) / per_block), 256, 0, st>>>(keys, n, ranges,
-                                                                                       num_tiles);
-  return cudaGetLastError();
+  return launch_chained(ranges_kernel, dim3(static_cast<unsigned>((n + per_block - 1) / per_block)), dim3(256), 0, st,
+                        keys, n, ranges, num_tiles);
 }
 
 }  // namespace gs

@@ -45,6 +45,8 @@ struct ViewsSmem {
 
 template <int kDeg, bool kMip>
 __global__ void __launch_bounds__(kViewsBlock, 5) views_backward_adam_kernel(ViewsAdamArgs a) {
+  chain_wait();
+  chain_release();
   __shared__ __align__(16) ViewsSmem sm;
   extern __shared__ __align__(16) float4 stage[];
   constexpr int nk = (kDeg + 1) * (kDeg + 1);
@@ -127,8 +129,7 @@ cudaError_t launch_views_mip(const ViewsAdamArgs& a, unsigned grid, cudaStream_t
   cudaError_t e = cudaFuncSetAttribute(views_backward_adam_kernel<kDeg, kMip>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  views_backward_adam_kernel<kDeg, kMip><<<grid, kViewsBlock, smem, st>>>(a);
-  return cudaGetLastError();
+  return launch_chained(views_backward_adam_kernel<kDeg, kMip>, dim3(grid), dim3(kViewsBlock), smem, st, a);
 }
 
 template <int kDeg>
