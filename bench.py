@@ -55,8 +55,8 @@ WORKLOADS = {
 # traffic grows in proportion.
 NCU_TRAFFIC = {
     # Dense-shaped scene of 1.5M Gaussians (3,185,918 entries), one launch of each
-    "backward_adam": ((1287.691520e6 + 998.944768e6) / 1_500_000, "gaussians", "46b643ddc7b2"),
-    "blend_backward": ((350.716672e6 + 69.543680e6) / 3_185_918, "entries", "9f44c98dd94b"),
+    "backward_adam": ((1288.303360e6 + 999.343872e6) / 1_500_000, "gaussians", "9d3c5f2752f4"),
+    "blend_backward": ((349.820160e6 + 69.461760e6) / 3_185_918, "entries", "a191b2bc2f52"),
 }
 
 
