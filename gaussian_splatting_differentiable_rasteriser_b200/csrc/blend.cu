@@ -27,7 +27,8 @@
 // dividing by (1 - alpha), and keeps one running scalar g . S (S = colour
 // already composited behind) instead of three channels. Per (Gaussian, pixel)
 // it keeps two factors, w = dL/dalpha * o exp(-e) and alpha T, in a per-warp
-// batch in shared memory; every 16 Gaussians two lanes per Gaussian reduce
+// batch in shared memory; at the end of each half of a chunk of survivor
+// slots (16 Gaussians, fewer at a walk's start) two lanes per Gaussian reduce
 // its row into its 9 raw sums (w, w dx, w dy, w dx^2, w dx dy, w dy^2, dL/dc)
 // and add them with float32 atomics. The conic/opacity/mean2d chain
 // of those sums is applied once per Gaussian in the projection backward.
@@ -212,7 +213,7 @@ __global__ void __launch_bounds__(256) blend_forward_kernel(BlendArgs a) {
 // from, w = dL/dalpha * o exp(-e) and alpha T. Rows are padded to 33 so that a
 // lane per Gaussian reads without bank conflicts. A batch is one half of a
 // chunk's slots, so the reduction reads each Gaussian's centre and id from its
-// slot (shared-memory bandwidth, not issue, is the backward's tightest limit:
+// slot (shared-memory bandwidth limits the backward as much as issue does:
 // nothing per survivor is copied into the batch but its two factors).
 constexpr int kBatch = 16;
 struct WarpBatch {
