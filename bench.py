@@ -56,7 +56,7 @@ WORKLOADS = {
 NCU_TRAFFIC = {
     # Dense-shaped scene of 1.5M Gaussians (3,185,918 entries), one launch of each
     "backward_adam": ((1288.303360e6 + 999.343872e6) / 1_500_000, "gaussians", "9d3c5f2752f4"),
-    "blend_backward": ((349.820160e6 + 69.461760e6) / 3_185_918, "entries", "a191b2bc2f52"),
+    "blend_backward": ((349.820160e6 + 69.461760e6) / 3_185_918, "entries", "910f1addacf9"),
 }
 
 
