@@ -14,6 +14,10 @@
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
  *     Work is enqueued asynchronously on it. gs_render_forward is the one call
  *     that waits on the stream (it reads the entry count back to the host).
+ *     The training step's kernels are launched with programmatic dependent
+ *     launch: a kernel may be scheduled while the work ahead of it on the
+ *     stream drains, but it touches no memory before that work has completed,
+ *     so stream order holds as for ordinary launches.
  *   - Parameters are structure-of-arrays, planar float32, with n <= n_pad,
  *     n_pad a multiple of 4 and 16-byte aligned base pointers, so every plane
  *     starts 16-byte aligned:
