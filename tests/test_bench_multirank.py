@@ -2,8 +2,10 @@
 size 2: process-group set-up from the launcher's environment, the barrier,
 the max-over-ranks timing and the whole-job aggregate of independent replicas,
 and the reference arm under the launcher (rank 0 prints the one line, the
-other rank exits without work); plus the roofline arithmetic and the scaling
-of the ncu traffic figures."""
+other rank exits without work); plus the roofline arithmetic, the scaling
+of the ncu traffic figures, and the profiled pass taking its stage times from
+the production kernels and the blends' pair counts from a separate counting
+pass (a fake context, no GPU)."""
 import json
 import os
 import socket
@@ -101,3 +103,71 @@ def test_traffic_figures_scale_per_unit_of_work():
     assert per_g == pytest.approx(24 * 59 + 101, rel=0.01)
     per_e, unit, _ = bench.NCU_TRAFFIC["blend_backward"]
     assert unit == "entries" and per_e * 3_185_918 == pytest.approx(349.820160e6 + 69.461760e6)
+
+
+class _FakeCtx:
+    """Stands in for a library context: times (fixed per-stage figures) when
+    profiling is on, counts the blends' pairs only when asked to."""
+
+    def __init__(self):
+        self.modes = []
+        self.steps = 0
+
+    def profile_enable(self, on=True, count_pairs=False):
+        self.modes.append((on, count_pairs))
+        self.steps = 0
+
+    def profile_read(self):
+        on, count = self.modes[-1] if self.modes else (False, False)
+        n, self.steps = self.steps, 0
+        out = {}
+        for name, ms in (("blend_forward", 0.5), ("blend_backward", 0.7), ("backward_adam", 0.9)):
+            blend = name.startswith("blend")
+            # the counting variants are slower: their times must not be used
+            t = ms * (3.0 if count and blend else 1.0)
+            out[name] = {"ms": t * n, "launches": n, "work": (1000 * n if count and blend else 7 * n),
+                         "blended": (200 * n if count and blend else 0)}
+        return out
+
+
+class _FakeStep:
+    fused_adam = True
+    adam_launches = 0
+
+    def __init__(self):
+        self.ctx = _FakeCtx()
+        self.model = type("M", (), {"step_count": 0})()
+        self.dimage = None
+        self.last_entries = 123
+
+    def forward(self, cs, h, w):
+        self.ctx.steps += 1
+        return None, None, None
+
+    def compute_loss(self, img, target, dimage):
+        pass
+
+    def backward_and_update(self, cs, T, nc, dimage):
+        pass
+
+
+def test_profiled_stage_times_come_from_the_timing_pass_and_pair_counts_from_the_counting_pass(monkeypatch):
+    sys.path.insert(0, ROOT)
+    import torch
+
+    import bench
+    from gaussian_splatting_differentiable_rasteriser_b200 import native
+    monkeypatch.setattr(torch.cuda, "synchronize", lambda *a, **k: None)
+    monkeypatch.setattr(native, "camera_struct", lambda cam: cam)
+    step = _FakeStep()
+    cam = type("C", (), {"height": 4, "width": 4})()
+    prof, ks = bench.profile_stages(step, [cam], [None], [0], start=1, count=10)
+    # timing pass first (production kernels), then the counting pass, then off
+    assert step.ctx.modes == [(True, False), (True, True), (False, False)]
+    assert prof["blend_forward"]["ms"] == pytest.approx(0.5 * 10)
+    assert prof["blend_backward"]["ms"] == pytest.approx(0.7 * 10)
+    assert prof["blend_backward"]["work"] == 1000 * 10 and prof["blend_backward"]["blended"] == 200 * 10
+    # stages without a counting variant keep the timing pass's work units
+    assert prof["backward_adam"]["work"] == 7 * 10 and prof["backward_adam"]["ms"] == pytest.approx(9.0)
+    assert ks == [123] * 10
+    assert prof["adam"]["launches"] == 0  # the fused pass: no separate Adam launches
