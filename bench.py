@@ -746,7 +746,8 @@ def main_ours(args):
 def e2e_run(step, cams, targets, sched, args, world):
     """Same steps through the public API with the target of every step copied
     from pinned host memory (double-buffered on a copy stream, overlapped with the
-    previous step's work) and each step's loss read back to the host."""
+    previous step's work) and each step's loss read back to the host (on the copy
+    stream, as soon as the loss kernel has run)."""
     import torch
 
     from gaussian_splatting_differentiable_rasteriser_b200 import native
@@ -755,6 +756,8 @@ def e2e_run(step, cams, targets, sched, args, world):
     dev_t = [torch.empty_like(targets[0]) for _ in range(2)]
     copy_stream = torch.cuda.Stream()
     copied = [torch.cuda.Event() for _ in range(2)]
+    loss_ready = [torch.cuda.Event() for _ in range(2)]
+    loss_read = [torch.cuda.Event() for _ in range(2)]
     loss_host = torch.empty((2, 3), dtype=torch.float64).pin_memory()
     m = step.model
     n = args.steps
@@ -767,23 +770,36 @@ def e2e_run(step, cams, targets, sched, args, world):
     with torch.cuda.stream(copy_stream):
         dev_t[0].copy_(host_t[c0], non_blocking=True)
         copied[0].record(copy_stream)
+    compute = torch.cuda.current_stream()
     for j in range(n):
         i = start + j
         c = int(sched[i % len(sched)])
         cam = cams[c]
         cs = native.camera_struct(cam)
+        # Cross-stream waits sit at the step boundary, where the step's chain
+        # of kernels starts anyway: this step's target has landed (it was copied
+        # during the previous step), and the previous loss has been read out of
+        # the loss buffer before this step's loss kernel rewrites it.
+        compute.wait_event(copied[j % 2])
+        if j > 0:
+            compute.wait_event(loss_read[(j - 1) % 2])
         img, T, nc = step.forward(cs, cam.height, cam.width)  # waits for all earlier work
         if j > 0:
+            loss_read[(j - 1) % 2].synchronize()
             losses.append(float(loss_host[(j - 1) % 2, 0]))
         if j + 1 < n:
             cn = int(sched[(i + 1) % len(sched)])
             with torch.cuda.stream(copy_stream):
                 dev_t[(j + 1) % 2].copy_(host_t[cn], non_blocking=True)
                 copied[(j + 1) % 2].record(copy_stream)
-        torch.cuda.current_stream().wait_event(copied[j % 2])
         step.compute_loss(img, dev_t[j % 2], step.dimage)
+        # the loss goes to the host on the copy stream, off the compute stream
+        loss_ready[j % 2].record(compute)
+        with torch.cuda.stream(copy_stream):
+            copy_stream.wait_event(loss_ready[j % 2])
+            loss_host[j % 2].copy_(step.loss[:3], non_blocking=True)
+            loss_read[j % 2].record(copy_stream)
         step.backward_and_update(cs, T, nc, step.dimage)
-        loss_host[j % 2].copy_(step.loss[:3], non_blocking=True)
     torch.cuda.synchronize()
     losses.append(float(loss_host[(n - 1) % 2, 0]))
     dt = time.perf_counter() - t0
