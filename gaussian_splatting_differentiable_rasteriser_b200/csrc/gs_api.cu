@@ -58,6 +58,11 @@ struct gs_ctx {
   gs::ForwardInfo* info_host = nullptr;
   // state of the camera in flight
   bool have_pre = false, have_fwd = false;
+  // The screen-gradient sums (float32, or fixed point in deterministic mode)
+  // are zeroed by gs_render_forward while the host waits for the entry count;
+  // the backward zeroes them itself when these are false.
+  bool sgrad_zeroed = false, sgrad_fixed_zeroed = false;
+  cudaEvent_t info_ev = nullptr;  // the entry count has reached the host
   int64_t n = 0, n_pad = 0;
   gs::CamArgs cam{};
   int64_t K = 0;
@@ -122,6 +127,7 @@ void free_all(gs_ctx* c) {
   if (c->dens_host) cudaFreeHost(c->dens_host);
   if (c->prof.created)
     for (auto& e : c->prof.ev) cudaEventDestroy(e);
+  if (c->info_ev) cudaEventDestroy(c->info_ev);
 }
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
@@ -307,6 +313,7 @@ gs_status gs_create(gs_ctx** out, int64_t max_gaussians, int64_t max_entries, in
   GS_ALLOC(c->info_dev, sizeof(gs::ForwardInfo));
   GS_ALLOC(c->pairs, sizeof(unsigned long long) * 8);
 #undef GS_ALLOC
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&c->info_ev, cudaEventDisableTiming);
   if (e == cudaSuccess) e = cudaMallocHost(reinterpret_cast<void**>(&c->info_host), sizeof(gs::ForwardInfo));
   if (e == cudaSuccess) e = cudaMallocHost(reinterpret_cast<void**>(&c->dens_host), sizeof(uint4));
   if (e == cudaSuccess) e = cudaMemset(c->loss_counter, 0, sizeof(uint32_t));
@@ -422,7 +429,19 @@ gs_status gs_render_forward(gs_ctx* c, const gs_camera* cam, float* image, float
   // The one host/device crossing of the step: entry count and depth-key range.
   GS_CUDA(c, cudaMemcpyAsync(c->info_host, c->info_dev, sizeof(gs::ForwardInfo),
                              cudaMemcpyDeviceToHost, st));
-  GS_CUDA(c, cudaStreamSynchronize(st));
+  GS_CUDA(c, cudaEventRecord(c->info_ev, st));
+  // The backward's screen-gradient sums are cleared now: the device does it
+  // while the host waits for the counts, and the backward then needs no
+  // memset between the loss and the blend backward.
+  c->sgrad_zeroed = c->sgrad_fixed_zeroed = false;
+  if (c->n > 0) {
+    if (c->deterministic)
+      GS_CUDA(c, cudaMemsetAsync(c->sgrad_fixed, 0, sizeof(unsigned long long) * gs::kFixedStride * c->n, st));
+    else
+      GS_CUDA(c, cudaMemsetAsync(c->sgrad, 0, sizeof(float) * gs::kGradStride * c->n, st));
+    (c->deterministic ? c->sgrad_fixed_zeroed : c->sgrad_zeroed) = true;
+  }
+  GS_CUDA(c, cudaEventSynchronize(c->info_ev));
   if ((s = take_device_error(c)) != GS_OK) return s;
   const uint64_t K = c->info_host->num_entries;
   if (num_entries_out) *num_entries_out = static_cast<int64_t>(K);
@@ -579,11 +598,12 @@ gs_status backward_common(gs_ctx* c, const gs_params* p, const gs_camera* cam, c
       if (!q || !aligned(q, 4)) return fail(c, GS_ERR_INVALID_ARG, "a gradient pointer is NULL or misaligned");
   }
   if (p->n > 0) {
-    if (c->deterministic)
+    if (c->deterministic && !c->sgrad_fixed_zeroed)
       GS_CUDA(c, cudaMemsetAsync(c->sgrad_fixed, 0, sizeof(unsigned long long) * gs::kFixedStride * p->n, st));
-    else
+    else if (!c->deterministic && !c->sgrad_zeroed)
       GS_CUDA(c, cudaMemsetAsync(c->sgrad, 0, sizeof(float) * gs::kGradStride * p->n, st));
   }
+  c->sgrad_zeroed = c->sgrad_fixed_zeroed = false;  // the blend backward adds into them
   gs::BlendArgs ba{};
   ba.ranges = c->ranges;
   ba.tile_order = c->tile_order;
