@@ -465,6 +465,30 @@ def test_fused_backward_adam_adds_an_accumulated_gradient(gs):
         assert np.mean(dp <= 1e-6) > 0.999, k
 
 
+def test_a_second_backward_after_one_forward_starts_from_cleared_sums(gs):
+    """The forward clears the screen-gradient sums for the backward; a second
+    backward of the same forward must clear them itself, so both give the same
+    gradient (up to the float32 atomics' summation order) instead of the second
+    adding onto the first."""
+    native, model = gs
+    s = scenes.small()
+    cam = s.cameras[0]
+    cs = native.camera_struct(cam)
+    H, W = cam.height, cam.width
+    d = dev(np.random.default_rng(23).normal(0, 1e-5, (3, H, W)))
+    m = model.GaussianModel(s)
+    st = model.TrainStep(m, 200_000, W, H, fused_adam=False)
+    _, T, nc = st.forward(cs, H, W)
+    grads = []
+    for _ in range(2):
+        m.grad_flat.zero_()
+        st.ctx.render_backward(m.params_struct(), cs, T, nc, d, m.grads_struct())
+        torch.cuda.synchronize()
+        grads.append(host(m.grad_flat).astype(np.float64))
+    assert np.abs(grads[0]).max() > 0
+    assert rel_l2(grads[1], grads[0]) < 1e-4
+
+
 @pytest.mark.parametrize("name", ["tiny", "small"])
 def test_opacity_aware_rect_path_matches_oracle(gs, name):
     """With the opacity-aware tile rect: rects and the sort bit-exact, pixels
